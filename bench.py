@@ -1,0 +1,366 @@
+"""Benchmark of the two-level sparse decode step (AsyncTLS hot path) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config c2] [--impl tls|reference]
+
+A step is one pass of the per-step path over one batch: level-1 block
+selection, level-2 token selection and sparse attention (three kernel
+launches).  Inputs are seeded synthetic caches of the workload's shape,
+resident in HBM before timing.  Between timed steps a 256 MB buffer is written
+(untimed) so every step starts with a cold L2; each step is timed with CUDA
+events on the launching stream.  Multi-GPU runs are weak scaling: every rank
+owns an independent batch (no collective on the data path); the reported
+time is the max over ranks.
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle on
+the host cores instead (the only reference arm this method has).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse decode-attn µs/step, achieved HBM GB/s vs peak; decode tokens/s"
+FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--config", default="c2")
+    ap.add_argument("--impl", default="tls", choices=["tls", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=300)
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- workload
+
+def workload(cfg, rank):
+    import synth
+    c = cfg.scaled(seed=cfg.seed + 1000 * rank) if rank else cfg
+    q = synth.gen_queries(c)
+    K, V, _ = synth.gen_kv(c, q)
+    lab = synth.gen_label_channels(c)
+    return c, q, K, V, lab
+
+
+def algorithmic_bytes(cfg):
+    """Bytes the step must move: metadata, candidate label codes+scales,
+    gathered K/V rows, queries, index lists and the fp32 output."""
+    rows = cfg.rows
+    meta = rows * cfg.n_blocks * 2 * cfg.qk_dim * 2
+    n_cand = cfg.K_b * cfg.block_size
+    label = rows * n_cand * (cfg.n_label // 2 + 4)
+    row_bytes = (cfg.qk_dim + (cfg.v_dim if cfg.separate_v else 0)) * 2
+    gather = rows * cfg.k * row_bytes
+    q = cfg.batch * cfg.n_q_heads * cfg.qk_dim * 2
+    out = cfg.batch * cfg.n_q_heads * cfg.v_dim * 4
+    idx = rows * (cfg.K_b + cfg.k) * 4 * 2
+    attn = gather + q + out + rows * cfg.k * 4
+    return dict(meta=meta, label=label, gather=gather, q=q, out=out, idx=idx,
+                step=meta + label + gather + q + out + idx, attn=attn)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_hash(name):
+    p = os.path.join(ROOT, "two_level_sparse_block_b200", "csrc", name)
+    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel_file, workload_name):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current source of the kernel; otherwise None."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    e = d.get(kernel_file, {}).get(workload_name)
+    if not e or e.get("source_sha256_16") != kernel_source_hash(kernel_file):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 10:
+                continue
+            if self.uuid and self.uuid not in f[1]:
+                continue
+            try:
+                rows.append((float(f[2]), float(f[3]), f[6:10]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, fl in rows for i, v in enumerate(fl) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle arm
+
+def time_oracle(cfg, q, K, V, lab, seconds, rows_sample=8):
+    """Times the float64 oracle's per-step path (levels 1, 2 and attention;
+    the index build is prepared outside the timed region, as on the GPU)."""
+    import oracle
+    try:
+        import threadpoolctl
+        limiter = threadpoolctl.threadpool_limits(1)
+    except Exception:
+        limiter = None
+    rng = np.random.default_rng(0)
+    all_rows = [(b, h) for b in range(cfg.batch) for h in range(cfg.n_kv_heads)]
+    pick = [all_rows[i] for i in sorted(rng.choice(len(all_rows), min(rows_sample, len(all_rows)), replace=False))]
+    g = cfg.group
+    prepared = []
+    for b, h in pick:
+        kb = K[b, h]
+        prepared.append((b, h, oracle.block_meta(kb, cfg.block_size), oracle.quant_label(kb, lab[h])))
+    done = 0
+    t0 = time.perf_counter()
+    while True:
+        b, h, meta, label = prepared[done % len(prepared)]
+        oracle.decode_row(q[b, h * g:(h + 1) * g], K[b, h], None if V is None else V[b, h], lab[h], cfg.block_size,
+                          cfg.K_b, cfg.k, cfg.softmax_scale, v_offset=cfg.v_offset, v_dim=cfg.v_dim, meta=meta,
+                          label=label)
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= seconds and done >= len(prepared):
+            break
+    if limiter is not None:
+        limiter.unregister()
+    per_row = el / done
+    step_s = per_row * cfg.rows
+    return {"value": cfg.batch / step_s, "unit": "decode tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{done} (batch row, KV head) decode_row calls over {len(pick)} seeded rows of "
+                      f"{cfg.name} in {el:.1f} s; scaled to all {cfg.rows} rows of one step",
+            "s_per_step": step_s}
+
+
+def run_reference(args, cfg):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    cfg, q, K, V, lab = workload(cfg, 0)
+    per_step = max(0.5, args.cpu_seconds / max(1, args.steps))
+    for _ in range(args.warmup):
+        time_oracle(cfg, q, K, V, lab, 0.0, rows_sample=1)
+    t = []
+    res = None
+    for _ in range(args.steps):
+        res = time_oracle(cfg, q, K, V, lab, per_step, rows_sample=2)
+        t.append(res["s_per_step"])
+    step_s = statistics.mean(t)
+    value = cfg.batch / step_s
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "decode tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg.name, "batch": cfg.batch, "ctx_len": cfg.ctx_len, "K_b": cfg.K_b, "k": cfg.k},
+            "cpu_baseline": {"value": value, "unit": "decode tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": f"each step: {res['sample']}"},
+            "e2e": {"value": value, "unit": "decode tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def main():
+    args = parse()
+    import synth
+    cfg = synth.get_config(args.config)
+    if args.impl == "reference":
+        run_reference(args, cfg)
+        return
+
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    from two_level_sparse_block_b200 import build, runtime, tls
+    build.build()
+
+    c, q, K, V, lab = workload(cfg, rank)
+    st = runtime.state_for_config(c, q, K, V, lab, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    torch.cuda.synchronize(dev)
+
+    def step_events(n):
+        return [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n)]
+
+    def timed_steps(n, evs):
+        for i in range(n):
+            flush.fill_(float(i))
+            e = evs[i]
+            e[0].record(stream)
+            st.select_blocks(stream=stream)
+            e[1].record(stream)
+            st.select_tokens(stream=stream)
+            e[2].record(stream)
+            st.attend(stream=stream)
+            e[3].record(stream)
+
+    warm = step_events(args.warmup)
+    timed_steps(args.warmup, warm)
+    torch.cuda.synchronize(dev)
+    if st.check_device_error() != 0:
+        raise RuntimeError("device error during warm-up")
+
+    evs = step_events(args.steps)
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.3)
+    wall0 = time.perf_counter()
+    timed_steps(args.steps, evs)
+    torch.cuda.synchronize(dev)
+    wall = time.perf_counter() - wall0
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    err = st.check_device_error()
+    if err != 0:
+        raise RuntimeError(f"device error {err} during the timed steps")
+
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    blk_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    tok_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    att_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    total_ms = sum(step_ms)
+    t = torch.tensor([total_ms, sum(att_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, att_total = float(t[0]), float(t[1])
+    ms_per_step = total_ms / args.steps
+    value = world * c.batch / (ms_per_step / 1e3)
+
+    # end to end through the public API: pinned host q in, host out back, every step
+    q_host = torch.empty(st.q.shape, dtype=torch.bfloat16).pin_memory()
+    q_host.copy_(st.q.cpu())
+    out_host = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
+    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.e2e_steps)]
+    q_dev = torch.empty_like(st.q)
+    for i in range(args.e2e_steps):
+        flush.fill_(float(i))
+        e2e_ev[i][0].record(stream)
+        q_dev.copy_(q_host, non_blocking=True)
+        st.step(q=q_dev, stream=stream)
+        out_host.copy_(st.out, non_blocking=True)
+        e2e_ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = sum(e[0].elapsed_time(e[1]) for e in e2e_ev) / args.e2e_steps
+    t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_ms = float(t[0])
+
+    ab = algorithmic_bytes(c)
+    peak, peak_kind = load_peaks()
+    att_avg_s = att_total / args.steps / 1e3
+    achieved = ab["attn"] / att_avg_s / 1e9
+    step_gbs = ab["step"] / (ms_per_step / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "decode tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "us_per_step": ms_per_step * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, fp32 accumulate",
+        "data": "synthetic (seeded; shapes of the workload, random K/V with outlier channels and planted tokens)",
+        "config": {"workload": c.name, "batch_per_gpu": c.batch, "q_heads": c.n_q_heads, "kv_heads": c.n_kv_heads,
+                   "head_dim": c.qk_dim, "ctx_len": c.ctx_len, "block_size": c.block_size, "K_b": c.K_b,
+                   "k": c.k, "label_channels": c.n_label, "parallelism": f"weak x{world} (independent batches)",
+                   "l2": "256 MB buffer written between timed steps (cold L2)"},
+        "stage_us": {"select_blocks": 1e3 * statistics.mean(blk_ms), "select_tokens": 1e3 * statistics.mean(tok_ms),
+                     "sparse_decode_attn": 1e3 * statistics.mean(att_ms)},
+        "step_hbm": {"algorithmic_bytes": ab["step"], "achieved_gbs": step_gbs, "frac_of_peak": step_gbs / peak},
+        "roofline": {"kernel": "sparse_attn_kernel (decode_attn.cu)", "bound": "hbm", "achieved": achieved,
+                     "peak": peak, "peak_source": f"hbm_gbs {peak_kind}", "unit": "GB/s", "frac": achieved / peak,
+                     "algorithmic_bytes_per_launch": ab["attn"],
+                     "traffic": recorded_traffic("decode_attn.cu", c.name)},
+        "gpu_launches": 3 * args.steps,
+        "e2e": {"value": world * c.batch / (e2e_ms / 1e3), "unit": "decode tokens/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": int(st.q.numel() * 2), "d2h_bytes_per_step": int(st.out.numel() * st.out.element_size()),
+                "path": "tls_decode_step via the Python binding, q from pinned host, out to pinned host"},
+        "clocks": clocks,
+        "wall_s_timed": wall,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = time_oracle(c, q, K, V, lab, args.cpu_seconds)
+        line["cpu_baseline"].pop("s_per_step", None)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,265 @@
+/*
+ * tls.h -- C ABI of libtls, the two-level sparse decode step of AsyncTLS on
+ * NVIDIA B200 (sm_100a).
+ *
+ * Source of the method: "AsyncTLS: Efficient Generative LLM Inference with
+ * Asynchronous Two-level Sparse Attention" (gist.science technical summaries
+ * in English, Italian and Japanese).  Section names below refer to the
+ * English summary unless another page is named:
+ *   2.A Stage 1  coarse block filtering: blocks, a block-level index, the
+ *                Quest score recast as a GEMM, top-K_b blocks;
+ *                (Italian 2.A.1: the block index is the max/min of the keys)
+ *   2.A Stage 2  fine token selection inside the chosen blocks (Double
+ *                Sparsity): selected channels, INT4 keys, top-K_t tokens;
+ *                (Italian 2.A.2: attention runs on the chosen tokens only)
+ *   2.B          asynchronous offloading engine: temporal locality, staggered
+ *                execution, incremental transfer T_t = M_t \ C_t.
+ *
+ * Conventions for every call
+ *   - Pointers named "device" point to GPU memory (cudaMalloc / torch CUDA
+ *     tensors); "host" pointers point to CPU memory.  The caller owns every
+ *     buffer; the library keeps no pointer after a call returns, except the
+ *     handles of tls_block_cache_create / tls_engine_create, which keep the
+ *     pointers given to them until destroyed.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Kernel calls are asynchronous on that stream.
+ *   - bf16 is IEEE bfloat16 stored as 16-bit words; all tensors are dense,
+ *     row-major and C-contiguous unless a row stride is given (in elements).
+ *   - Arguments are validated before anything is launched.  A rejected call
+ *     returns TLS_ERR_INVALID_ARG or TLS_ERR_UNSUPPORTED, launches nothing,
+ *     and tls_last_error() describes why.  A failed launch returns
+ *     TLS_ERR_CUDA.  Errors inside kernels that use bounded waits are
+ *     reported through the workspace error word (tls_workspace_error).
+ *   - Shapes: B batch, Hq query heads, Hkv KV heads (Hq % Hkv == 0,
+ *     G = Hq / Hkv heads share one KV head), Dqk key dim, Dv value dim,
+ *     N context length, bs block size, NB = N / bs, R label channels,
+ *     "row" = one (batch, KV head) pair, rows = B * Hkv.
+ */
+#ifndef TLS_H
+#define TLS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TLS_API __attribute__((visibility("default")))
+#else
+#define TLS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum tls_status {
+  TLS_OK = 0,
+  TLS_ERR_INVALID_ARG = 1,  /* bad shape, pointer, alignment or size */
+  TLS_ERR_UNSUPPORTED = 2,  /* valid but not built (e.g. a head dim with no kernel) */
+  TLS_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+  TLS_ERR_TIMEOUT = 4,      /* a bounded wait ran out (device word or host deadline) */
+  TLS_ERR_CAPACITY = 5,     /* block cache has too few free slots */
+  TLS_ERR_COPY = 6          /* a host->device block copy failed (or was failed on purpose) */
+} tls_status;
+
+typedef struct tls_shape {
+  int32_t batch;        /* B >= 1 */
+  int32_t n_q_heads;    /* Hq, a multiple of n_kv_heads */
+  int32_t n_kv_heads;   /* Hkv >= 1 */
+  int32_t qk_dim;       /* Dqk: multiple of 32, <= 640 */
+  int32_t v_dim;        /* Dv: multiple of 8, <= 512 */
+  int32_t v_offset;     /* -1: V is its own tensor; >= 0: V of a token is its K row
+                           slice [v_offset, v_offset + v_dim) (MLA shared latent) */
+  int32_t block_size;   /* bs: tokens per block, multiple of 8, <= 256 */
+  int32_t n_label;      /* R: label channels, even, 2..64, <= qk_dim */
+  int64_t ctx_len;      /* N: multiple of block_size */
+  float softmax_scale;  /* logits are softmax_scale * q.k (e.g. 1/sqrt(Dqk)) */
+} tls_shape;
+
+/* Output element type of tls_sparse_decode_attn. */
+enum { TLS_OUT_F32 = 0, TLS_OUT_BF16 = 1 };
+
+/* Where the attention kernel finds K/V rows. */
+typedef struct tls_kv_view {
+  const void* k;           /* device bf16 K rows */
+  const void* v;           /* device bf16 V rows; unused when v_offset >= 0 */
+  int64_t k_row_stride;    /* elements between consecutive K rows (>= Dqk, multiple of 8) */
+  int64_t v_row_stride;    /* elements between consecutive V rows (>= Dv, multiple of 8) */
+  const int32_t* slot_of_block; /* NULL: dense cache, row r = b*Hkv + h, token t at
+                                   k + (r*N + t) * k_row_stride.
+                                   Else device int32 [B, Hkv, NB]: block -> slot in a
+                                   shared pool; token t of block j at
+                                   k + (slot*bs + t % bs) * k_row_stride. */
+  int32_t n_slots;         /* pool size when slot_of_block != NULL */
+} tls_kv_view;
+
+/* Thread-local description of the last rejected or failed call ("" if none). */
+TLS_API const char* tls_last_error(void);
+
+/* Library version, major*10000 + minor*100 + patch. */
+TLS_API int32_t tls_version(void);
+
+/*
+ * Bytes of device workspace needed by tls_select_blocks, tls_select_tokens,
+ * tls_sparse_decode_attn and tls_decode_step for this shape, K_b and k.
+ * The workspace must be zero-filled once after allocation; every call that
+ * completes leaves its counters at zero again, so it can be reused without
+ * clearing.  Calls that run concurrently on different streams may share one
+ * workspace only if they are different entry points (each uses its own
+ * region); two concurrent calls of the same entry point need two workspaces.
+ * Returns 0 if the shape is invalid.
+ */
+TLS_API size_t tls_workspace_bytes(const tls_shape* shape, int32_t K_b, int32_t k);
+
+/*
+ * Reads (and, if clear != 0, zeroes) the workspace error word on `stream`,
+ * synchronising that stream.  *code = 0 when no kernel reported an error;
+ * otherwise a TLS_ERR_* value set by a kernel whose bounded wait ran out.
+ */
+TLS_API tls_status tls_workspace_error(const void* ws, int32_t clear, int32_t* code, void* stream);
+
+/*
+ * Index build, part 1 (Stage 1 block-level index; Italian 2.A.1 max/min of
+ * the keys).  For every row and every block j with t0 <= j*bs < t1:
+ *   meta[row, j, c]       = max over the block's tokens of K[row, t, c]
+ *   meta[row, j, Dqk + c] = min over the block's tokens of K[row, t, c]
+ * k: device bf16, row r's token t at k + (r*N + t) * k_row_stride.
+ * meta: device bf16 [B, Hkv, NB, 2*Dqk].  t0, t1 multiples of bs,
+ * 0 <= t0 < t1 <= N.  The values are exact (max/min picks an input).
+ */
+TLS_API tls_status tls_build_block_meta(const tls_shape* shape, const void* k, int64_t k_row_stride,
+                                int64_t t0, int64_t t1, void* meta, void* stream);
+
+/*
+ * Index build, part 2 (Stage 2: channel selection + INT4 keys).  For every
+ * row and token t0 <= t < t1, with x_r = K[row, t, label_ch[h, r]]:
+ *   s = max_r |x_r| / 7                  (float32, IEEE division)
+ *   code_r = rint(x_r / s) in [-7, 7]    (float32, ties to even; s = 0 -> 0)
+ * codes: device uint8 [B, Hkv, N, R/2]; byte j holds code 2j in its low
+ * nibble and code 2j+1 in its high nibble, two's complement.
+ * scales: device float32 [B, Hkv, N].  label_ch: device int32 [Hkv, R],
+ * each in [0, Dqk).  Codes and scales are bit-exact by this definition.
+ */
+TLS_API tls_status tls_quant_label_cache(const tls_shape* shape, const void* k, int64_t k_row_stride,
+                                 const int32_t* label_ch, int64_t t0, int64_t t1,
+                                 uint8_t* codes, float* scales, void* stream);
+
+/*
+ * Level 1 (Stage 1): block scores as one GEMM per row on tcgen05 tensor cores,
+ *   S[h, j] = [relu(q_h), min(q_h, 0)] . [kmax_j ; kmin_j]   (fp32 accumulate)
+ * which equals Quest's sum_c max(q_hc*kmax_jc, q_hc*kmin_jc); the G heads of
+ * a row combine by max: agg[row, j] = max_h S[h, j].  Then the K_b blocks
+ * with the largest agg (ties: lower block index) are written ascending.
+ * q: device bf16 [B, Hq, Dqk] (16-byte aligned); meta as built above
+ * (16-byte aligned).  block_idx: device int32 [B, Hkv, K_b].
+ * block_score: optional device float32 [B, Hkv, NB] receiving agg.
+ * 1 <= K_b <= NB, NB <= 16384.
+ */
+TLS_API tls_status tls_select_blocks(const tls_shape* shape, const void* q, const void* meta, int32_t K_b,
+                             int32_t* block_idx, float* block_score,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Level 2 (Stage 2): for each candidate token t of the row's K_b chosen
+ * blocks (candidates in ascending token order),
+ *   score(t) = max_h  s_t * sum_r q_h[label_ch[h_kv, r]] * code_{t, r}
+ * then the k best candidates (ties: lower token index) are written
+ * ascending as absolute token positions.
+ * block_idx: device int32 [B, Hkv, K_b], ascending per row (as written by
+ * tls_select_blocks).  token_idx: device int32 [B, Hkv, k].
+ * token_score: optional device float32 [B, Hkv, K_b*bs] receiving the
+ * candidate scores.  1 <= k <= K_b*bs <= 16384.
+ */
+TLS_API tls_status tls_select_tokens(const tls_shape* shape, const void* q, const int32_t* label_ch,
+                             const uint8_t* codes, const float* scales, const int32_t* block_idx,
+                             int32_t K_b, int32_t k, int32_t* token_idx, float* token_score,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Attention over the chosen tokens only (Italian 2.A.2).  For each query
+ * head h of row (b, kv) with its row's token list T (token_idx, k entries):
+ *   p = softmax(softmax_scale * q_h . K[T]^T),  out[b, h] = p . V[T]
+ *   lse[b, h] = log(sum_t exp(softmax_scale * q_h . K_t))   (natural log)
+ * bf16 inputs, fp32 products, fp32 softmax and accumulation; split-K over
+ * the token list with a log-sum-exp merge inside the same launch.
+ * out: device [B, Hq, Dv], float32 (out_dtype TLS_OUT_F32) or bf16
+ * (TLS_OUT_BF16, round to nearest even).  lse: optional device float32 [B, Hq].
+ * Token indices must lie in [0, N); with a slot table, every block they fall
+ * in must map to a slot in [0, n_slots) (not checked on the device).
+ */
+TLS_API tls_status tls_sparse_decode_attn(const tls_shape* shape, const void* q, const tls_kv_view* kv,
+                                  const int32_t* token_idx, int32_t k, int32_t out_dtype,
+                                  void* out, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * One synchronous decode step: tls_select_blocks, tls_select_tokens and
+ * tls_sparse_decode_attn in order on `stream` (three kernel launches),
+ * sharing one workspace.  block_idx / token_idx are outputs as above.
+ */
+TLS_API tls_status tls_decode_step(const tls_shape* shape, const void* q, const void* meta,
+                           const int32_t* label_ch, const uint8_t* codes, const float* scales,
+                           const tls_kv_view* kv, int32_t K_b, int32_t k,
+                           int32_t* block_idx, int32_t* token_idx, int32_t out_dtype,
+                           void* out, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Offloaded KV: HBM block cache with incremental transfer (section 2.B).
+ * ------------------------------------------------------------------------ */
+typedef struct tls_block_cache tls_block_cache;
+
+/*
+ * Creates the host-side state of a block cache.  Full K/V live in host
+ * memory (pinned, for asynchronous copies): row r's token t at
+ * host_k + (r*N + t) * host_k_row_stride (likewise V; host_v may be NULL when
+ * v_offset >= 0).  The device pool holds n_slots blocks:
+ * slot_k [n_slots, bs, host_k_row_stride] and slot_v [n_slots, bs,
+ * host_v_row_stride] (bf16).  slot_table_dev: device int32 [B, Hkv, NB],
+ * written by the library (-1 = not resident); the attention kernel reads it
+ * through tls_kv_view.slot_of_block.  The handle allocates two small pinned
+ * staging tables (B*Hkv*NB int32 each) and nothing on the device.
+ * Any pointer may be NULL only for host-only use of tls_block_cache_plan.
+ */
+TLS_API tls_status tls_block_cache_create(const tls_shape* shape, const void* host_k, const void* host_v,
+                                  int64_t host_k_row_stride, int64_t host_v_row_stride,
+                                  int32_t n_slots, void* slot_k, void* slot_v,
+                                  int32_t* slot_table_dev, tls_block_cache** out);
+TLS_API void tls_block_cache_destroy(tls_block_cache* cache);
+
+/*
+ * Host-only planning of one incremental transfer (section 2.B): for every
+ * row, T_t = M_t \ C_t where M_t = new_block_idx[row] and C_t is the set of
+ * resident blocks.  Each block of T_t gets a victim slot that holds no block
+ * of in_use_block_idx[row] (the blocks the running attention reads, M_{t-1})
+ * nor of M_t, preferring free slots, then the least recently used, then the
+ * lower slot.  The plan is committed to the cache's host mirror.
+ * new_block_idx, in_use_block_idx: host int32 [B, Hkv, K_b] (in_use may be
+ * NULL for none).  copy_row/copy_block/copy_slot: host int32 arrays of
+ * capacity B*Hkv*K_b receiving the plan (may be NULL); *n_copy = |T_t| summed
+ * over rows.  Returns TLS_ERR_CAPACITY (and commits nothing) if victims run out.
+ */
+TLS_API tls_status tls_block_cache_plan(tls_block_cache* cache, const int32_t* new_block_idx,
+                                const int32_t* in_use_block_idx, int32_t K_b,
+                                int32_t* copy_row, int32_t* copy_block, int32_t* copy_slot,
+                                int32_t* n_copy);
+
+/*
+ * Incremental prefetch (section 2.B): plans as tls_block_cache_plan, then
+ * issues one cudaMemcpyAsync per copied run of blocks (K and V) from host
+ * memory into the chosen slots on copy_stream and one copy of the updated
+ * slot table.  The caller must order copy_stream after every kernel still
+ * reading a slot that may be evicted (the previous step's attention).
+ * *n_copied = blocks copied.  Setting the environment variable
+ * TLS_FAULT_INJECT=copy makes the copy step fail with TLS_ERR_COPY before
+ * anything is issued (host-side fault injection for tests).
+ */
+TLS_API tls_status tls_prefetch_diff(tls_block_cache* cache, const int32_t* new_block_idx_host,
+                             const int32_t* in_use_block_idx_host, int32_t K_b,
+                             void* copy_stream, int32_t* n_copied);
+
+/* Copies the host mirror of the slot table (int32 [B, Hkv, NB]) into `table`. */
+TLS_API tls_status tls_block_cache_table(const tls_block_cache* cache, int32_t* table);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TLS_H */

@@ -25,8 +25,10 @@ reading of the workload descriptions):
 
 from __future__ import annotations
 
+import concurrent.futures
 import dataclasses
 import math
+import os
 
 import numpy as np
 
@@ -167,13 +169,18 @@ def gen_kv(cfg: WorkloadConfig, q_bits: np.ndarray, layer: int = 0, rows=None):
     if cfg.separate_v:
         vv = np.empty((cfg.batch, cfg.n_kv_heads, cfg.ctx_len, cfg.v_dim), dtype=np.uint16)
     planted = {}
-    for b in range(cfg.batch):
-        for h in range(cfg.n_kv_heads):
-            if rows is not None and (b, h) not in rows:
-                continue
-            r = gen_row(cfg, b, h, q_bits, layer)
-            kk[b, h] = r.k
-            if vv is not None:
-                vv[b, h] = r.v
-            planted[(b, h)] = (r.planted_pos, r.planted_head)
+    todo = [(b, h) for b in range(cfg.batch) for h in range(cfg.n_kv_heads) if rows is None or (b, h) in rows]
+
+    def one(bh):
+        b, h = bh
+        r = gen_row(cfg, b, h, q_bits, layer)
+        kk[b, h] = r.k
+        if vv is not None:
+            vv[b, h] = r.v
+        return bh, (r.planted_pos, r.planted_head)
+
+    # rows draw from independent streams, so threads change no value
+    with concurrent.futures.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
+        for bh, pl in ex.map(one, todo):
+            planted[bh] = pl
     return kk, vv, planted

@@ -1,0 +1,157 @@
+"""The C ABI without a GPU: the library loads, exports every declared entry
+point, validates arguments, and its host-only block-cache planner follows the
+incremental-transfer rule T_t = M_t \\ C_t (AsyncTLS English summary 2.B)."""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def tls():
+    from two_level_sparse_block_b200 import build
+    build.build()
+    from two_level_sparse_block_b200 import tls as t
+    return t
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "tls.h")).read()
+    return re.findall(r"^TLS_API\s+[\w\s\*]+?\b(tls_\w+)\s*\(", text, flags=re.M)
+
+
+def test_library_exports_every_declared_symbol(tls):
+    names = declared_functions()
+    assert len(names) >= 15
+    lib = ctypes.CDLL(tls.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/tls.h but not exported"
+    # and the binding wraps each of them under the same name
+    for n in names:
+        assert hasattr(tls, n), f"binding lacks {n}"
+
+
+def test_version_and_error_string(tls):
+    assert tls.tls_version() >= 100
+    assert isinstance(tls.tls_last_error(), str)
+
+
+def c2_shape(tls, **kw):
+    f = dict(batch=8, n_q_heads=32, n_kv_heads=8, qk_dim=128, v_dim=128, v_offset=-1, block_size=64, n_label=16,
+             ctx_len=32768, softmax_scale=128 ** -0.5)
+    f.update(kw)
+    return tls.make_shape(**f)
+
+
+def test_workspace_validation(tls):
+    s = c2_shape(tls)
+    a = tls.tls_workspace_bytes(s, 64, 2048)
+    assert a > 0 and a % 256 == 0
+    assert tls.tls_workspace_bytes(s, 64, 4096) > 0
+    assert tls.tls_workspace_bytes(s, 64, 4097) == 0   # k > K_b * bs
+    assert tls.tls_workspace_bytes(s, 513, 64) == 0    # K_b > NB
+    assert tls.tls_workspace_bytes(s, 0, 1) == 0
+    for bad in (dict(qk_dim=100), dict(n_q_heads=30), dict(block_size=12), dict(n_label=15),
+                dict(ctx_len=32760), dict(v_offset=4), dict(softmax_scale=0.0), dict(v_dim=520)):
+        assert tls.tls_workspace_bytes(c2_shape(tls, **bad), 64, 2048) == 0, bad
+    mla = c2_shape(tls, batch=4, n_q_heads=128, n_kv_heads=1, qk_dim=576, v_dim=512, v_offset=0,
+                   ctx_len=65536, n_label=32)
+    assert tls.tls_workspace_bytes(mla, 128, 4096) > 0
+
+
+def test_entry_points_reject_null_arguments_without_a_gpu(tls):
+    s = c2_shape(tls)
+    with pytest.raises(tls.TlsError) as e:
+        tls.tls_select_blocks(s, None, None, 64, None, None, None, 0, stream=0)
+    assert e.value.status == tls.TLS_ERR_INVALID_ARG
+    with pytest.raises(tls.TlsError) as e:
+        tls.tls_build_block_meta(s, None, 128, 0, 64, None, stream=0)
+    assert e.value.status == tls.TLS_ERR_INVALID_ARG
+
+
+def _trajectory(nb, K_b, steps, seed):
+    """Block sets with temporal locality: each step swaps a few blocks."""
+    rng = np.random.default_rng(seed)
+    cur = np.sort(rng.choice(nb, K_b, replace=False))
+    out = [cur]
+    for _ in range(steps - 1):
+        n_swap = int(rng.integers(0, max(2, K_b // 4)))
+        keep = rng.choice(cur, K_b - n_swap, replace=False)
+        rest = np.setdiff1d(np.arange(nb), keep)
+        cur = np.sort(np.concatenate([keep, rng.choice(rest, n_swap, replace=False)]))
+        out.append(cur)
+    return out
+
+
+@pytest.mark.parametrize("rows,n_slots_factor", [(1, 2), (3, 2), (2, 3)])
+def test_block_cache_plan_follows_incremental_transfer(tls, rows, n_slots_factor):
+    nb, K_b, bs = 64, 8, 16
+    s = c2_shape(tls, batch=rows, n_q_heads=4, n_kv_heads=1, ctx_len=nb * bs, block_size=bs)
+    n_slots = n_slots_factor * K_b * rows
+    h = tls.tls_block_cache_create(s, None, None, 128, 128, n_slots, None, None, None)
+    try:
+        trajs = [_trajectory(nb, K_b, 40, seed=r) for r in range(rows)]
+        resident = [set() for _ in range(rows)]
+        prev = None
+        for t in range(40):
+            new = np.stack([trajs[r][t] for r in range(rows)]).astype(np.int32)
+            cap = rows * K_b
+            cr, cb, cs = (np.zeros(cap, np.int32) for _ in range(3))
+            before = tls_table(tls, h, rows, nb)
+            n = tls.tls_block_cache_plan(h, new, prev, K_b, cr, cb, cs)
+            after = tls_table(tls, h, rows, nb)
+            copied = {(int(cr[i]), int(cb[i])) for i in range(n)}
+            for r in range(rows):
+                want = oracle.plan_transfer(new[r], sorted(resident[r]))
+                assert sorted(b for rr, b in copied if rr == r) == want.tolist()
+                resident[r] = {b for b in range(nb) if after[r, b] >= 0}
+                assert set(new[r].tolist()) <= resident[r]
+            # a victim slot never held a block the running step still reads (M_{t-1}) or keeps (M_t)
+            for i in range(n):
+                slot = int(cs[i])
+                for r in range(rows):
+                    for blk in np.where(before[r] == slot)[0]:
+                        assert blk not in new[r]
+                        if prev is not None:
+                            assert blk not in prev[r]
+            # the slot table is a partial injection
+            used = after[after >= 0]
+            assert used.size == np.unique(used).size and used.max() < n_slots
+            prev = new
+    finally:
+        tls.tls_block_cache_destroy(h)
+
+
+def tls_table(tls, h, rows, nb):
+    t = np.zeros((rows, nb), dtype=np.int32)
+    tls.tls_block_cache_table(h, t)
+    return t
+
+
+def test_block_cache_plan_capacity_error_commits_nothing(tls):
+    nb, K_b, bs = 32, 8, 16
+    s = c2_shape(tls, batch=1, n_q_heads=4, n_kv_heads=1, ctx_len=nb * bs, block_size=bs)
+    h = tls.tls_block_cache_create(s, None, None, 128, 128, 12, None, None, None)
+    try:
+        a = np.arange(8, dtype=np.int32)[None]
+        assert tls.tls_block_cache_plan(h, a, None, K_b) == 8
+        b = np.arange(8, 16, dtype=np.int32)[None]
+        before = tls_table(tls, h, 1, nb)
+        with pytest.raises(tls.TlsError) as e:
+            tls.tls_block_cache_plan(h, b, a, K_b)  # needs 8 free slots, only 4 are not in use
+        assert e.value.status == tls.TLS_ERR_CAPACITY
+        assert np.array_equal(before, tls_table(tls, h, 1, nb))
+        with pytest.raises(tls.TlsError) as e:
+            tls.tls_block_cache_plan(h, np.array([[0, 0, 1, 2, 3, 4, 5, 6]], np.int32), None, K_b)
+        assert e.value.status == tls.TLS_ERR_INVALID_ARG
+    finally:
+        tls.tls_block_cache_destroy(h)

@@ -1,0 +1,259 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Index build: bit-exact.  Selections: bit-exact up to float32 ties at the k-th
+boundary (tests/parity.py).  Outputs: <= 2e-3 max row-relative error.
+Workloads are the five configured shapes (full size; the oracle checks a
+sample of rows) and small ragged shapes that span several tiles.
+"""
+
+from __future__ import annotations
+
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from synth import f32_from_bf16_bits, get_config
+from tests.parity import check_output, check_selection
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="session", autouse=True)
+def _built():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from two_level_sparse_block_b200 import build
+    build.build()
+
+
+def _rt():
+    from two_level_sparse_block_b200 import runtime, tls
+    return runtime, tls
+
+
+@functools.lru_cache(maxsize=4)
+def gen_case(cfg):
+    q = synth.gen_queries(cfg)
+    K, V, planted = synth.gen_kv(cfg, q)
+    lab = synth.gen_label_channels(cfg)
+    return q, K, V, lab
+
+
+def small(name, **kw):
+    base = dict(name=name, description="small parity shape", batch=2, n_q_heads=8, n_kv_heads=2, qk_dim=128,
+                v_dim=128, v_offset=-1, ctx_len=2048, block_size=16, K_b=12, k=100, n_label=16, seed=11,
+                n_outlier=3, planted_per_row=16, planted_blocks=4, label_from_outliers=True)
+    base.update(kw)
+    return synth.WorkloadConfig(**base)
+
+
+SMALL = [
+    small("s_gqa4"),
+    small("s_g3_ragged", n_q_heads=6, n_kv_heads=2, ctx_len=200 * 16, K_b=37, k=333, seed=12),
+    small("s_g1", n_q_heads=3, n_kv_heads=3, K_b=5, k=80, seed=13),
+    small("s_g6_d64", n_q_heads=12, n_kv_heads=2, qk_dim=64, v_dim=64, K_b=9, k=144, n_label=8, seed=14),
+    small("s_g16_bs32", n_q_heads=16, n_kv_heads=1, block_size=32, ctx_len=4096, K_b=20, k=640, seed=15),
+    small("s_mla", batch=2, n_q_heads=16, n_kv_heads=1, qk_dim=576, v_dim=512, v_offset=0, ctx_len=1024,
+          block_size=64, K_b=6, k=200, n_label=32, n_outlier=0, label_from_outliers=False, kv_std=0.7071, seed=16),
+    small("s_k_eq_1", K_b=1, k=1, seed=17),
+    small("s_all", ctx_len=512, K_b=32, k=512, seed=18),
+]
+FULL = [get_config(c) for c in ("c1", "c2", "c3", "c4")]
+
+
+def make_state(cfg, **kw):
+    runtime, tls = _rt()
+    q, K, V, lab = gen_case(cfg)
+    st = runtime.state_for_config(cfg, q, K, V, lab, **kw)
+    torch.cuda.synchronize()
+    return st, (q, K, V, lab)
+
+
+def sample_rows(cfg, n=3):
+    rows = [(b, h) for b in range(cfg.batch) for h in range(cfg.n_kv_heads)]
+    if len(rows) <= n:
+        return rows
+    rng = np.random.default_rng(cfg.seed + 99)
+    pick = [rows[0], rows[-1]] + [rows[i] for i in rng.choice(np.arange(1, len(rows) - 1), n - 2, replace=False)]
+    return pick
+
+
+def oracle_row(cfg, data, b, h, **kw):
+    q, K, V, lab = data
+    g = cfg.group
+    vb = None if V is None else V[b, h]
+    return oracle.decode_row(q[b, h * g:(h + 1) * g], K[b, h], vb, lab[h], cfg.block_size, cfg.K_b, cfg.k,
+                             cfg.softmax_scale, v_offset=cfg.v_offset, v_dim=cfg.v_dim, **kw)
+
+
+def run_stages(st):
+    st.select_blocks(keep_scores=True)
+    st.select_tokens(keep_scores=True)
+    st.attend()
+    torch.cuda.synchronize()
+    assert st.check_device_error() == 0
+    return dict(block_idx=st.block_idx.cpu().numpy(), token_idx=st.token_idx.cpu().numpy(),
+                block_score=st.block_score.cpu().numpy(), token_score=st.token_score.cpu().numpy(),
+                out=st.out.float().cpu().numpy(), lse=st.lse.cpu().numpy())
+
+
+def check_row(cfg, data, got, st, b, h):
+    q, K, V, lab = data
+    g = cfg.group
+    kb = K[b, h]
+    meta = oracle.block_meta(kb, cfg.block_size)
+    label = oracle.quant_label(kb, lab[h])
+    where = f"{cfg.name} row ({b},{h})"
+
+    # index: bit-exact
+    gm = st.meta[b, h].float().cpu().numpy().astype(np.float64)
+    assert np.array_equal(gm[:, :cfg.qk_dim], meta[0]), f"{where}: kmax differs"
+    assert np.array_equal(gm[:, cfg.qk_dim:], meta[1]), f"{where}: kmin differs"
+    assert np.array_equal(st.codes[b, h].cpu().numpy(), oracle.pack_codes(label[0])), f"{where}: INT4 codes differ"
+    assert np.array_equal(st.scales[b, h].cpu().numpy().view(np.uint32), label[1].view(np.uint32)), \
+        f"{where}: scales differ"
+
+    # level 1
+    r1 = oracle_row(cfg, data, b, h, meta=meta, label=label)
+    agg = r1["agg"]
+    scale = np.max(np.abs(agg))
+    assert np.max(np.abs(got["block_score"][b, h] - agg)) <= 1e-5 * scale, f"{where}: block scores"
+    swaps_b = check_selection(got["block_idx"][b, h], agg, cfg.K_b, where + " blocks")
+
+    # Quest bound on the GPU scores (float32, 1e-5 relative slack), on sampled tokens
+    qf = f32_from_bf16_bits(q[b, h * g:(h + 1) * g]).astype(np.float64)
+    rng = np.random.default_rng(b * 131 + h)
+    toks = rng.choice(cfg.ctx_len, size=min(2048, cfg.ctx_len), replace=False)
+    dots = (qf @ f32_from_bf16_bits(kb[toks]).astype(np.float64).T).max(axis=0)
+    bound = got["block_score"][b, h][toks // cfg.block_size]
+    assert np.all(bound >= dots - 1e-5 * scale), f"{where}: Quest bound violated on the GPU"
+
+    # level 2 on the GPU's block set
+    gb = got["block_idx"][b, h]
+    r2 = oracle_row(cfg, data, b, h, meta=meta, label=label, block_idx=gb)
+    ts = r2["token_score"]
+    tscale = np.max(np.abs(ts))
+    assert np.max(np.abs(got["token_score"][b, h] - ts)) <= 1e-5 * tscale, f"{where}: token scores"
+    cand = r2["cand"]
+    pos = np.searchsorted(cand, got["token_idx"][b, h])
+    assert np.array_equal(cand[pos], got["token_idx"][b, h]), f"{where}: token outside the chosen blocks"
+    swaps_t = check_selection(pos, ts, cfg.k, where + " tokens")
+
+    # attention on the GPU's token set
+    r3 = oracle_row(cfg, data, b, h, meta=meta, label=label, block_idx=gb, token_idx=got["token_idx"][b, h])
+    err = check_output(got["out"][b, h * g:(h + 1) * g], r3["out"], where + " out")
+    assert np.max(np.abs(got["lse"][b, h * g:(h + 1) * g] - r3["lse"])) <= 1e-4 * max(1.0, np.max(np.abs(r3["lse"]))), \
+        f"{where}: lse"
+    return swaps_b, swaps_t, err
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
+def test_small_shapes_all_rows(cfg):
+    st, data = make_state(cfg)
+    got = run_stages(st)
+    for b in range(cfg.batch):
+        for h in range(cfg.n_kv_heads):
+            check_row(cfg, data, got, st, b, h)
+
+
+@pytest.mark.parametrize("cfg", FULL, ids=lambda c: c.name)
+def test_full_size_sampled_rows(cfg):
+    st, data = make_state(cfg)
+    got = run_stages(st)
+    for b, h in sample_rows(cfg):
+        check_row(cfg, data, got, st, b, h)
+    # the fused step gives the same lists and outputs as the three calls
+    st.step()
+    torch.cuda.synchronize()
+    assert np.array_equal(st.block_idx.cpu().numpy(), got["block_idx"])
+    assert np.array_equal(st.token_idx.cpu().numpy(), got["token_idx"])
+    assert np.array_equal(st.out.float().cpu().numpy(), got["out"])
+
+
+def test_select_everything_equals_dense_attention():
+    cfg = small("s_dense", ctx_len=1024, block_size=32, K_b=32, k=1024, seed=21)
+    st, data = make_state(cfg)
+    got = run_stages(st)
+    q, K, V, lab = data
+    g = cfg.group
+    for b in range(cfg.batch):
+        for h in range(cfg.n_kv_heads):
+            assert got["block_idx"][b, h].tolist() == list(range(cfg.n_blocks))
+            assert got["token_idx"][b, h].tolist() == list(range(cfg.ctx_len))
+            qq = torch.from_numpy(f32_from_bf16_bits(q[b, h * g:(h + 1) * g]).astype(np.float64))
+            kk = torch.from_numpy(f32_from_bf16_bits(K[b, h]).astype(np.float64))
+            vv = torch.from_numpy(f32_from_bf16_bits(V[b, h]).astype(np.float64))
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                qq[:, None, :], kk[None].expand(g, -1, -1), vv[None].expand(g, -1, -1),
+                scale=cfg.softmax_scale)[:, 0, :].numpy()
+            check_output(got["out"][b, h * g:(h + 1) * g], ref, "dense")
+
+
+def test_equal_scores_pick_lowest_indices():
+    runtime, tls = _rt()
+    cfg = small("s_ties", batch=1, n_kv_heads=1, n_q_heads=4, ctx_len=1024, block_size=16, K_b=7, k=50)
+    q = synth.gen_queries(cfg)
+    K = np.full((1, 1, cfg.ctx_len, cfg.qk_dim), 0x3F80, dtype=np.uint16)  # every key = 1.0
+    V = synth.gen_kv(cfg, q)[1]
+    lab = synth.gen_label_channels(cfg)
+    st = runtime.state_for_config(cfg, q, K, V, lab)
+    got = run_stages(st)
+    assert got["block_idx"][0, 0].tolist() == list(range(7))
+    assert got["token_idx"][0, 0].tolist() == list(range(50))
+
+
+def test_bf16_output_and_repeat_calls():
+    runtime, tls = _rt()
+    cfg = SMALL[1]
+    st32, data = make_state(cfg)
+    st16, _ = make_state(cfg, out_dtype=tls.TLS_OUT_BF16)
+    a = run_stages(st32)
+    for _ in range(3):  # counters in the workspace must reset after every call
+        b = run_stages(st16)
+    assert np.array_equal(a["token_idx"], b["token_idx"])
+    ref = torch.from_numpy(a["out"]).to(torch.bfloat16).float().numpy()
+    assert np.array_equal(b["out"], ref)
+
+
+def test_slot_table_view_matches_dense():
+    runtime, tls = _rt()
+    cfg = SMALL[0]
+    st, data = make_state(cfg)
+    run_stages(st)
+    dense = st.out.clone()
+    # scatter every block into a shuffled slot pool and read through the table
+    rows, nb, bs = cfg.rows, cfg.n_blocks, cfg.block_size
+    perm = torch.randperm(rows * nb, generator=torch.Generator().manual_seed(5)).to(torch.int32)
+    pool_k = torch.empty((rows * nb, bs, cfg.qk_dim), dtype=torch.bfloat16, device="cuda")
+    pool_v = torch.empty((rows * nb, bs, cfg.v_dim), dtype=torch.bfloat16, device="cuda")
+    pool_k[perm.long().cuda()] = st.kc.reshape(rows * nb, bs, cfg.qk_dim)
+    pool_v[perm.long().cuda()] = st.vc.reshape(rows * nb, bs, cfg.v_dim)
+    table = perm.reshape(cfg.batch, cfg.n_kv_heads, nb).cuda()
+    kv = tls.make_kv_view(pool_k, pool_v, cfg.qk_dim, cfg.v_dim, table, rows * nb)
+    st.attend(kv=kv)
+    torch.cuda.synchronize()
+    assert torch.equal(st.out, dense)
+
+
+def test_invalid_arguments_launch_nothing():
+    runtime, tls = _rt()
+    cfg = SMALL[0]
+    st, data = make_state(cfg)
+    bad = tls.make_shape(cfg.batch, cfg.n_q_heads, cfg.n_kv_heads, cfg.qk_dim, cfg.v_dim, -1, cfg.block_size,
+                         cfg.n_label, cfg.ctx_len, cfg.softmax_scale)
+    with pytest.raises(tls.TlsError) as e:
+        tls.tls_select_blocks(bad, st.q, st.meta, cfg.n_blocks + 1, st.block_idx, None, st.ws, st.ws_bytes)
+    assert e.value.status == tls.TLS_ERR_INVALID_ARG
+    with pytest.raises(tls.TlsError):
+        tls.tls_select_tokens(bad, st.q, st.label_ch, st.codes, st.scales, st.block_idx, cfg.K_b,
+                              cfg.K_b * cfg.block_size + 1, st.token_idx, None, st.ws, st.ws_bytes)
+    with pytest.raises(tls.TlsError):
+        tls.tls_sparse_decode_attn(bad, st.q, st.kv, st.token_idx, cfg.k, 7, st.out, None, st.ws, st.ws_bytes)
+    with pytest.raises(tls.TlsError):
+        tls.tls_select_blocks(bad, st.q, st.meta, cfg.K_b, st.block_idx, None, st.ws, 16)
+    torch.cuda.synchronize()
+    assert st.check_device_error() == 0

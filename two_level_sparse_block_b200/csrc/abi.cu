@@ -1,0 +1,230 @@
+// C-ABI entry points of libtls for the per-step path, argument validation and
+// the workspace plan.  Kernels live in block_select.cu, token_select.cu and
+// decode_attn.cu; the index build in index_build.cu; the block cache and
+// incremental prefetch in block_cache.cu.
+
+#include <cstring>
+
+#include "host_common.h"
+
+namespace tls {
+
+tls_status select_blocks_impl(const tls_shape& s, const void* q, const void* meta, int K_b, int32_t* block_idx,
+                              float* block_score, uint8_t* ws, const WsLayout& L, cudaStream_t stream);
+tls_status select_tokens_impl(const tls_shape& s, const void* q, const int32_t* label_ch, const uint8_t* codes,
+                              const float* scales, const int32_t* block_idx, int K_b, int k, int32_t* token_idx,
+                              float* token_score, uint8_t* ws, const WsLayout& L, cudaStream_t stream);
+tls_status sparse_attn_impl(const tls_shape& s, const void* q, const tls_kv_view& kv, const int32_t* token_idx,
+                            int k, int out_dtype, void* out, float* lse, uint8_t* ws, const WsLayout& L,
+                            cudaStream_t stream);
+int attn_heads_per_cta(const tls_shape& s);
+
+namespace {
+thread_local char g_err[512] = {0};
+}
+
+tls_status fail(tls_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+void clear_error() { g_err[0] = 0; }
+
+tls_status check_shape(const tls_shape* p) {
+  if (p == nullptr) return fail(TLS_ERR_INVALID_ARG, "shape is NULL");
+  const tls_shape& s = *p;
+  if (s.batch < 1 || s.n_kv_heads < 1 || s.n_q_heads < 1 || s.n_q_heads % s.n_kv_heads != 0)
+    return fail(TLS_ERR_INVALID_ARG, "bad heads/batch: B=%d Hq=%d Hkv=%d", s.batch, s.n_q_heads, s.n_kv_heads);
+  if (s.qk_dim < 32 || s.qk_dim % 32 != 0 || s.qk_dim > 640)
+    return fail(TLS_ERR_INVALID_ARG, "qk_dim %d must be a multiple of 32 in [32, 640]", s.qk_dim);
+  if (s.v_dim < 8 || s.v_dim % 8 != 0 || s.v_dim > 512)
+    return fail(TLS_ERR_INVALID_ARG, "v_dim %d must be a multiple of 8 in [8, 512]", s.v_dim);
+  if (s.v_offset >= 0 && (s.v_offset % 8 != 0 || s.v_offset + s.v_dim > s.qk_dim))
+    return fail(TLS_ERR_INVALID_ARG, "v_offset %d: V slice must be 8-aligned and inside the K row", s.v_offset);
+  if (s.v_offset < -1) return fail(TLS_ERR_INVALID_ARG, "v_offset must be -1 or >= 0");
+  if (s.block_size < 8 || s.block_size > 256 || s.block_size % 8 != 0)
+    return fail(TLS_ERR_INVALID_ARG, "block_size %d must be a multiple of 8 in [8, 256]", s.block_size);
+  if (s.n_label < 2 || s.n_label > 64 || s.n_label % 2 != 0 || s.n_label > s.qk_dim)
+    return fail(TLS_ERR_INVALID_ARG, "n_label %d must be even, in [2, 64] and <= qk_dim", s.n_label);
+  if (s.ctx_len < s.block_size || s.ctx_len % s.block_size != 0)
+    return fail(TLS_ERR_INVALID_ARG, "ctx_len %lld must be a positive multiple of block_size",
+                (long long)s.ctx_len);
+  if (s.ctx_len > (int64_t)1 << 31) return fail(TLS_ERR_INVALID_ARG, "ctx_len above 2^31");
+  if (!(s.softmax_scale > 0.0f)) return fail(TLS_ERR_INVALID_ARG, "softmax_scale must be > 0");
+  return TLS_OK;
+}
+
+tls_status plan_workspace(const tls_shape& s, int K_b, int k, WsLayout* out) {
+  const int rows = rows_of(s);
+  const int64_t nb = n_blocks(s);
+  const int g = group_of(s);
+  if (K_b < 1 || K_b > nb) return fail(TLS_ERR_INVALID_ARG, "K_b %d must be in [1, NB=%lld]", K_b, (long long)nb);
+  if (nb > 16384) return fail(TLS_ERR_UNSUPPORTED, "NB %lld above 16384", (long long)nb);
+  const int64_t n_cand = (int64_t)K_b * s.block_size;
+  if (n_cand > 16384) return fail(TLS_ERR_UNSUPPORTED, "K_b*block_size %lld above 16384", (long long)n_cand);
+  if (k < 1 || k > n_cand) return fail(TLS_ERR_INVALID_ARG, "k %d must be in [1, K_b*bs=%lld]", k, (long long)n_cand);
+  WsLayout L;
+  L.heads_per_cta = attn_heads_per_cta(s);
+  L.head_groups = (g + L.heads_per_cta - 1) / L.heads_per_cta;
+  const int target = 4 * kNumSMs;
+  int splits = (target + rows * L.head_groups - 1) / (rows * L.head_groups);
+  const int max_splits = (k + 15) / 16;
+  if (splits > max_splits) splits = max_splits;
+  if (splits < 1) splits = 1;
+  int tps = (k + splits - 1) / splits;
+  tps = (int)align_up((size_t)tps, 8);
+  L.tokens_per_split = tps;
+  L.splits = (k + tps - 1) / tps;
+  size_t off = 0;
+  L.err = off;
+  off += 256;
+  L.blk_counter = off;
+  off = align_up(off + (size_t)rows * 4, 256);
+  L.tok_counter = off;
+  off = align_up(off + (size_t)rows * 4, 256);
+  L.att_counter = off;
+  off = align_up(off + (size_t)rows * L.head_groups * 4, 256);
+  // regions that depend on fewer arguments come first, so that the offsets
+  // a call uses do not depend on arguments it is not given
+  L.agg = off;
+  off = align_up(off + (size_t)rows * nb * 4, 256);
+  L.partial = off;
+  off = align_up(off + (size_t)rows * g * L.splits * (s.v_dim + 2) * 4, 256);
+  L.tscore = off;
+  off = align_up(off + (size_t)rows * n_cand * 4, 256);
+  L.total = off;
+  *out = L;
+  return TLS_OK;
+}
+
+static tls_status check_ws(const tls_shape& s, int K_b, int k, void* ws, size_t ws_bytes, WsLayout* L) {
+  tls_status st = plan_workspace(s, K_b, k, L);
+  if (st != TLS_OK) return st;
+  if (ws == nullptr || !aligned16(ws)) return fail(TLS_ERR_INVALID_ARG, "workspace NULL or not 16-byte aligned");
+  if (ws_bytes < L->total)
+    return fail(TLS_ERR_INVALID_ARG, "workspace %zu bytes < required %zu", ws_bytes, L->total);
+  return TLS_OK;
+}
+
+static tls_status check_kv(const tls_shape& s, const tls_kv_view* kv) {
+  if (kv == nullptr || kv->k == nullptr) return fail(TLS_ERR_INVALID_ARG, "kv view or kv.k is NULL");
+  if (!aligned16(kv->k)) return fail(TLS_ERR_INVALID_ARG, "kv.k must be 16-byte aligned");
+  if (kv->k_row_stride < s.qk_dim || kv->k_row_stride % 8 != 0)
+    return fail(TLS_ERR_INVALID_ARG, "kv.k_row_stride must be >= qk_dim and a multiple of 8");
+  if (s.v_offset < 0) {
+    if (kv->v == nullptr || !aligned16(kv->v)) return fail(TLS_ERR_INVALID_ARG, "kv.v NULL or not 16-byte aligned");
+    if (kv->v_row_stride < s.v_dim || kv->v_row_stride % 8 != 0)
+      return fail(TLS_ERR_INVALID_ARG, "kv.v_row_stride must be >= v_dim and a multiple of 8");
+  }
+  if (kv->slot_of_block != nullptr && kv->n_slots < 1)
+    return fail(TLS_ERR_INVALID_ARG, "kv.n_slots must be >= 1 with a slot table");
+  return TLS_OK;
+}
+
+}  // namespace tls
+
+using namespace tls;
+
+extern "C" const char* tls_last_error(void) { return g_err; }
+
+extern "C" int32_t tls_version(void) { return 100; }
+
+extern "C" size_t tls_workspace_bytes(const tls_shape* shape, int32_t K_b, int32_t k) {
+  if (check_shape(shape) != TLS_OK) return 0;
+  WsLayout L;
+  if (plan_workspace(*shape, K_b, k, &L) != TLS_OK) return 0;
+  return L.total;
+}
+
+extern "C" tls_status tls_workspace_error(const void* ws, int32_t clear, int32_t* code, void* stream) {
+  clear_error();
+  if (ws == nullptr || code == nullptr) return fail(TLS_ERR_INVALID_ARG, "workspace_error: NULL argument");
+  int32_t words[2] = {0, 0};
+  cudaStream_t cs = (cudaStream_t)stream;
+  tls_status st = cuda_check(cudaMemcpyAsync(words, ws, sizeof(words), cudaMemcpyDeviceToHost, cs),
+                             "workspace_error: copy");
+  if (st != TLS_OK) return st;
+  if (clear) {
+    st = cuda_check(cudaMemsetAsync(const_cast<void*>(ws), 0, sizeof(words), cs), "workspace_error: clear");
+    if (st != TLS_OK) return st;
+  }
+  st = cuda_check(cudaStreamSynchronize(cs), "workspace_error: sync");
+  if (st != TLS_OK) return st;
+  *code = words[0];
+  if (words[0] != 0) fail((tls_status)words[0], "kernel error %d at site %d", words[0], words[1]);
+  return TLS_OK;
+}
+
+extern "C" tls_status tls_select_blocks(const tls_shape* shape, const void* q, const void* meta, int32_t K_b,
+                                        int32_t* block_idx, float* block_score, void* ws, size_t ws_bytes,
+                                        void* stream) {
+  clear_error();
+  tls_status st = check_shape(shape);
+  if (st != TLS_OK) return st;
+  if (q == nullptr || meta == nullptr || block_idx == nullptr)
+    return fail(TLS_ERR_INVALID_ARG, "select_blocks: null pointer");
+  if (!aligned16(q) || !aligned16(meta)) return fail(TLS_ERR_INVALID_ARG, "select_blocks: q/meta not 16-byte aligned");
+  WsLayout L;
+  st = check_ws(*shape, K_b, 1, ws, ws_bytes, &L);
+  if (st != TLS_OK) return st;
+  return select_blocks_impl(*shape, q, meta, K_b, block_idx, block_score, (uint8_t*)ws, L, (cudaStream_t)stream);
+}
+
+extern "C" tls_status tls_select_tokens(const tls_shape* shape, const void* q, const int32_t* label_ch,
+                                        const uint8_t* codes, const float* scales, const int32_t* block_idx,
+                                        int32_t K_b, int32_t k, int32_t* token_idx, float* token_score, void* ws,
+                                        size_t ws_bytes, void* stream) {
+  clear_error();
+  tls_status st = check_shape(shape);
+  if (st != TLS_OK) return st;
+  if (q == nullptr || label_ch == nullptr || codes == nullptr || scales == nullptr || block_idx == nullptr ||
+      token_idx == nullptr)
+    return fail(TLS_ERR_INVALID_ARG, "select_tokens: null pointer");
+  if (!aligned16(q) || !aligned16(codes)) return fail(TLS_ERR_INVALID_ARG, "select_tokens: q/codes not 16-byte aligned");
+  WsLayout L;
+  st = check_ws(*shape, K_b, k, ws, ws_bytes, &L);
+  if (st != TLS_OK) return st;
+  return select_tokens_impl(*shape, q, label_ch, codes, scales, block_idx, K_b, k, token_idx, token_score,
+                            (uint8_t*)ws, L, (cudaStream_t)stream);
+}
+
+extern "C" tls_status tls_sparse_decode_attn(const tls_shape* shape, const void* q, const tls_kv_view* kv,
+                                             const int32_t* token_idx, int32_t k, int32_t out_dtype, void* out,
+                                             float* lse, void* ws, size_t ws_bytes, void* stream) {
+  clear_error();
+  tls_status st = check_shape(shape);
+  if (st != TLS_OK) return st;
+  st = check_kv(*shape, kv);
+  if (st != TLS_OK) return st;
+  if (q == nullptr || token_idx == nullptr || out == nullptr)
+    return fail(TLS_ERR_INVALID_ARG, "sparse_decode_attn: null pointer");
+  if (!aligned16(q)) return fail(TLS_ERR_INVALID_ARG, "sparse_decode_attn: q not 16-byte aligned");
+  if (out_dtype != TLS_OUT_F32 && out_dtype != TLS_OUT_BF16)
+    return fail(TLS_ERR_INVALID_ARG, "sparse_decode_attn: out_dtype must be TLS_OUT_F32 or TLS_OUT_BF16");
+  if (k < 1 || k > shape->ctx_len) return fail(TLS_ERR_INVALID_ARG, "sparse_decode_attn: k %d out of range", k);
+  // the attention plan depends on k only; take K_b as large as the context allows
+  const int64_t nb = n_blocks(*shape);
+  int K_b = (int)((k + shape->block_size - 1) / shape->block_size);
+  if (K_b > nb) K_b = (int)nb;
+  WsLayout L;
+  st = check_ws(*shape, K_b, k, ws, ws_bytes, &L);
+  if (st != TLS_OK) return st;
+  return sparse_attn_impl(*shape, q, *kv, token_idx, k, out_dtype, out, lse, (uint8_t*)ws, L,
+                          (cudaStream_t)stream);
+}
+
+extern "C" tls_status tls_decode_step(const tls_shape* shape, const void* q, const void* meta,
+                                      const int32_t* label_ch, const uint8_t* codes, const float* scales,
+                                      const tls_kv_view* kv, int32_t K_b, int32_t k, int32_t* block_idx,
+                                      int32_t* token_idx, int32_t out_dtype, void* out, float* lse, void* ws,
+                                      size_t ws_bytes, void* stream) {
+  tls_status st = tls_select_blocks(shape, q, meta, K_b, block_idx, nullptr, ws, ws_bytes, stream);
+  if (st != TLS_OK) return st;
+  st = tls_select_tokens(shape, q, label_ch, codes, scales, block_idx, K_b, k, token_idx, nullptr, ws, ws_bytes,
+                         stream);
+  if (st != TLS_OK) return st;
+  return tls_sparse_decode_attn(shape, q, kv, token_idx, k, out_dtype, out, lse, ws, ws_bytes, stream);
+}

@@ -1,0 +1,248 @@
+// HBM block cache with incremental transfer (AsyncTLS, English summary 2.B:
+// only the blocks of the new candidate set that are not resident,
+// T_t = M_t \ C_t, cross PCIe; the copies overlap the running attention).
+//
+// Host state: a mirror of the device slot table (block -> slot), the owner
+// of every slot and its last use.  Planning is pure host code; the prefetch
+// issues one cudaMemcpyAsync per run of blocks that are adjacent both in host
+// memory and in the slot pool, then one copy of the slot table.
+
+#include <algorithm>
+#include <cstdlib>
+#include <cstring>
+#include <vector>
+
+#include "host_common.h"
+
+struct tls_block_cache {
+  tls_shape shape;
+  int rows = 0;
+  int nb = 0;
+  const uint8_t* host_k = nullptr;
+  const uint8_t* host_v = nullptr;
+  int64_t hk_stride = 0, hv_stride = 0;
+  int n_slots = 0;
+  uint8_t* slot_k = nullptr;
+  uint8_t* slot_v = nullptr;
+  int32_t* table_dev = nullptr;
+  std::vector<int32_t> table;       // [rows * nb] -> slot or -1
+  std::vector<int64_t> owner;       // [n_slots] -> row * nb + block, or -1
+  std::vector<int64_t> last_use;    // [n_slots] planning step of the last use
+  int64_t step = 0;
+  int32_t* staging[2] = {nullptr, nullptr};  // pinned copies of the table
+  cudaEvent_t staged[2] = {nullptr, nullptr};
+  int cur = 0;
+};
+
+namespace tls {
+namespace {
+
+struct Copy {
+  int32_t row, block, slot;
+};
+
+bool fault_injected_copy() {
+  const char* e = std::getenv("TLS_FAULT_INJECT");
+  return e != nullptr && std::strcmp(e, "copy") == 0;
+}
+
+// Plans T_t and its victim slots without changing the cache.
+tls_status plan(const tls_block_cache& c, const int32_t* new_idx, const int32_t* in_use, int K_b,
+                std::vector<Copy>* copies, std::vector<int32_t>* victims) {
+  const int64_t total = (int64_t)c.rows * c.nb;
+  std::vector<char> keep(c.n_slots, 0);
+  std::vector<char> seen(total, 0);
+  copies->clear();
+  for (int r = 0; r < c.rows; ++r) {
+    for (int i = 0; i < K_b; ++i) {
+      const int32_t blk = new_idx[(int64_t)r * K_b + i];
+      if (blk < 0 || blk >= c.nb) return fail(TLS_ERR_INVALID_ARG, "plan: block %d out of range in row %d", blk, r);
+      const int64_t key = (int64_t)r * c.nb + blk;
+      if (seen[key]) return fail(TLS_ERR_INVALID_ARG, "plan: block %d repeated in row %d", blk, r);
+      seen[key] = 1;
+      const int32_t s = c.table[key];
+      if (s >= 0) keep[s] = 1;
+      else copies->push_back({r, blk, -1});
+    }
+    if (in_use != nullptr) {
+      for (int i = 0; i < K_b; ++i) {
+        const int32_t blk = in_use[(int64_t)r * K_b + i];
+        if (blk < 0 || blk >= c.nb) continue;
+        const int32_t s = c.table[(int64_t)r * c.nb + blk];
+        if (s >= 0) keep[s] = 1;
+      }
+    }
+  }
+  // free slots first (ascending), then least recently used, then lower slot
+  std::vector<int32_t> cand;
+  for (int s = 0; s < c.n_slots; ++s)
+    if (!keep[s] && c.owner[s] < 0) cand.push_back(s);
+  std::vector<int32_t> used;
+  for (int s = 0; s < c.n_slots; ++s)
+    if (!keep[s] && c.owner[s] >= 0) used.push_back(s);
+  std::stable_sort(used.begin(), used.end(), [&](int32_t a, int32_t b) {
+    if (c.last_use[a] != c.last_use[b]) return c.last_use[a] < c.last_use[b];
+    return a < b;
+  });
+  cand.insert(cand.end(), used.begin(), used.end());
+  if (cand.size() < copies->size())
+    return fail(TLS_ERR_CAPACITY, "plan: %zu blocks to copy but only %zu evictable slots", copies->size(),
+                cand.size());
+  victims->assign(cand.begin(), cand.begin() + copies->size());
+  return TLS_OK;
+}
+
+void commit(tls_block_cache& c, const int32_t* new_idx, int K_b, std::vector<Copy>& copies,
+            const std::vector<int32_t>& victims) {
+  c.step += 1;
+  for (size_t i = 0; i < copies.size(); ++i) {
+    const int32_t s = victims[i];
+    if (c.owner[s] >= 0) c.table[c.owner[s]] = -1;
+    const int64_t key = (int64_t)copies[i].row * c.nb + copies[i].block;
+    c.owner[s] = key;
+    c.table[key] = s;
+    copies[i].slot = s;
+  }
+  for (int r = 0; r < c.rows; ++r)
+    for (int i = 0; i < K_b; ++i) {
+      const int32_t s = c.table[(int64_t)r * c.nb + new_idx[(int64_t)r * K_b + i]];
+      c.last_use[s] = c.step;
+    }
+}
+
+}  // namespace
+}  // namespace tls
+
+using namespace tls;
+
+extern "C" tls_status tls_block_cache_create(const tls_shape* shape, const void* host_k, const void* host_v,
+                                             int64_t host_k_row_stride, int64_t host_v_row_stride, int32_t n_slots,
+                                             void* slot_k, void* slot_v, int32_t* slot_table_dev,
+                                             tls_block_cache** out) {
+  clear_error();
+  tls_status st = check_shape(shape);
+  if (st != TLS_OK) return st;
+  if (out == nullptr) return fail(TLS_ERR_INVALID_ARG, "block_cache_create: out is NULL");
+  if (n_slots < 1) return fail(TLS_ERR_INVALID_ARG, "block_cache_create: n_slots must be >= 1");
+  if (host_k_row_stride < shape->qk_dim)
+    return fail(TLS_ERR_INVALID_ARG, "block_cache_create: host_k_row_stride must be >= qk_dim");
+  if (shape->v_offset < 0 && host_v != nullptr && host_v_row_stride < shape->v_dim)
+    return fail(TLS_ERR_INVALID_ARG, "block_cache_create: host_v_row_stride must be >= v_dim");
+  auto* c = new tls_block_cache();
+  c->shape = *shape;
+  c->rows = rows_of(*shape);
+  c->nb = (int)n_blocks(*shape);
+  c->host_k = (const uint8_t*)host_k;
+  c->host_v = shape->v_offset < 0 ? (const uint8_t*)host_v : nullptr;
+  c->hk_stride = host_k_row_stride;
+  c->hv_stride = host_v_row_stride;
+  c->n_slots = n_slots;
+  c->slot_k = (uint8_t*)slot_k;
+  c->slot_v = (uint8_t*)slot_v;
+  c->table_dev = slot_table_dev;
+  c->table.assign((size_t)c->rows * c->nb, -1);
+  c->owner.assign(n_slots, -1);
+  c->last_use.assign(n_slots, 0);
+  if (slot_table_dev != nullptr) {
+    for (int i = 0; i < 2; ++i) {
+      cudaError_t e = cudaHostAlloc((void**)&c->staging[i], c->table.size() * sizeof(int32_t), cudaHostAllocDefault);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->staged[i], cudaEventDisableTiming);
+      if (e != cudaSuccess) {
+        tls_block_cache_destroy(c);
+        return cuda_check(e, "block_cache_create: pinned staging");
+      }
+    }
+  }
+  *out = c;
+  return TLS_OK;
+}
+
+extern "C" void tls_block_cache_destroy(tls_block_cache* c) {
+  if (c == nullptr) return;
+  for (int i = 0; i < 2; ++i) {
+    if (c->staged[i] != nullptr) {
+      cudaEventSynchronize(c->staged[i]);
+      cudaEventDestroy(c->staged[i]);
+    }
+    if (c->staging[i] != nullptr) cudaFreeHost(c->staging[i]);
+  }
+  delete c;
+}
+
+extern "C" tls_status tls_block_cache_plan(tls_block_cache* c, const int32_t* new_block_idx,
+                                           const int32_t* in_use_block_idx, int32_t K_b, int32_t* copy_row,
+                                           int32_t* copy_block, int32_t* copy_slot, int32_t* n_copy) {
+  clear_error();
+  if (c == nullptr || new_block_idx == nullptr || n_copy == nullptr)
+    return fail(TLS_ERR_INVALID_ARG, "block_cache_plan: NULL argument");
+  if (K_b < 1 || K_b > c->nb) return fail(TLS_ERR_INVALID_ARG, "block_cache_plan: K_b out of range");
+  std::vector<Copy> copies;
+  std::vector<int32_t> victims;
+  tls_status st = plan(*c, new_block_idx, in_use_block_idx, K_b, &copies, &victims);
+  if (st != TLS_OK) return st;
+  commit(*c, new_block_idx, K_b, copies, victims);
+  for (size_t i = 0; i < copies.size(); ++i) {
+    if (copy_row) copy_row[i] = copies[i].row;
+    if (copy_block) copy_block[i] = copies[i].block;
+    if (copy_slot) copy_slot[i] = copies[i].slot;
+  }
+  *n_copy = (int32_t)copies.size();
+  return TLS_OK;
+}
+
+extern "C" tls_status tls_prefetch_diff(tls_block_cache* c, const int32_t* new_block_idx_host,
+                                        const int32_t* in_use_block_idx_host, int32_t K_b, void* copy_stream,
+                                        int32_t* n_copied) {
+  clear_error();
+  if (c == nullptr || new_block_idx_host == nullptr || n_copied == nullptr)
+    return fail(TLS_ERR_INVALID_ARG, "prefetch_diff: NULL argument");
+  if (c->host_k == nullptr || c->slot_k == nullptr || c->table_dev == nullptr)
+    return fail(TLS_ERR_INVALID_ARG, "prefetch_diff: cache was created without device buffers");
+  if (K_b < 1 || K_b > c->nb) return fail(TLS_ERR_INVALID_ARG, "prefetch_diff: K_b out of range");
+  if (fault_injected_copy()) return fail(TLS_ERR_COPY, "prefetch_diff: copy failure injected (TLS_FAULT_INJECT=copy)");
+  std::vector<Copy> copies;
+  std::vector<int32_t> victims;
+  tls_status st = plan(*c, new_block_idx_host, in_use_block_idx_host, K_b, &copies, &victims);
+  if (st != TLS_OK) return st;
+  commit(*c, new_block_idx_host, K_b, copies, victims);
+
+  cudaStream_t cs = (cudaStream_t)copy_stream;
+  const int bs = c->shape.block_size;
+  const int64_t n = c->shape.ctx_len;
+  const size_t kblk = (size_t)bs * c->hk_stride * 2, vblk = (size_t)bs * c->hv_stride * 2;
+  size_t i = 0;
+  while (i < copies.size()) {
+    size_t j = i + 1;
+    while (j < copies.size() && copies[j].row == copies[i].row &&
+           copies[j].block == copies[j - 1].block + 1 && copies[j].slot == copies[j - 1].slot + 1)
+      ++j;
+    const size_t len = j - i;
+    const int64_t tok0 = (int64_t)copies[i].row * n + (int64_t)copies[i].block * bs;
+    cudaError_t e = cudaMemcpyAsync(c->slot_k + (size_t)copies[i].slot * kblk,
+                                    c->host_k + (size_t)tok0 * c->hk_stride * 2, len * kblk,
+                                    cudaMemcpyHostToDevice, cs);
+    if (e == cudaSuccess && c->host_v != nullptr && c->slot_v != nullptr)
+      e = cudaMemcpyAsync(c->slot_v + (size_t)copies[i].slot * vblk, c->host_v + (size_t)tok0 * c->hv_stride * 2,
+                          len * vblk, cudaMemcpyHostToDevice, cs);
+    if (e != cudaSuccess) return fail(TLS_ERR_COPY, "prefetch_diff: block copy failed: %s", cudaGetErrorString(e));
+    i = j;
+  }
+  // publish the new slot table through a pinned staging copy
+  const int b = c->cur;
+  cudaError_t e = cudaEventSynchronize(c->staged[b]);
+  if (e != cudaSuccess) return cuda_check(e, "prefetch_diff: staging wait");
+  std::memcpy(c->staging[b], c->table.data(), c->table.size() * sizeof(int32_t));
+  e = cudaMemcpyAsync(c->table_dev, c->staging[b], c->table.size() * sizeof(int32_t), cudaMemcpyHostToDevice, cs);
+  if (e == cudaSuccess) e = cudaEventRecord(c->staged[b], cs);
+  if (e != cudaSuccess) return fail(TLS_ERR_COPY, "prefetch_diff: slot table copy failed: %s", cudaGetErrorString(e));
+  c->cur ^= 1;
+  *n_copied = (int32_t)copies.size();
+  return TLS_OK;
+}
+
+extern "C" tls_status tls_block_cache_table(const tls_block_cache* c, int32_t* table) {
+  clear_error();
+  if (c == nullptr || table == nullptr) return fail(TLS_ERR_INVALID_ARG, "block_cache_table: NULL argument");
+  std::memcpy(table, c->table.data(), c->table.size() * sizeof(int32_t));
+  return TLS_OK;
+}

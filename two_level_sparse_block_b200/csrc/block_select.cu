@@ -1,0 +1,361 @@
+// Level 1 of the two-level selection (AsyncTLS, English summary 2.A Stage 1:
+// the Quest block score recast as a GEMM so the heads sharing a KV head use
+// the tensor cores, then the top-K_b blocks; Italian summary 2.A.1: the block
+// index is the max/min of the keys).
+//
+// Per row (batch, KV head) the scores form one GEMM
+//     S[j, h] = sum_k  meta[j, k] * Q'[h, k],   Q' = [relu(q_h), min(q_h, 0)]
+// with meta[j] = [kmax_j ; kmin_j] (K = 2*Dqk).  The blocks are the MMA's M
+// dimension (128 per CTA) and the G heads its N dimension (padded to a
+// multiple of 16), so even G = 4 fills an M = 128 tcgen05 tile.
+//
+// CTA roles (128 threads):
+//   warp 0 lane 0   TMA producer: 128 x 64 bf16 metadata tiles, 128B swizzle
+//   warp 1 lane 0   MMA issuer: tcgen05.mma kind::f16, fp32 accumulator in TMEM
+//   warps 2-3       build the Q' tile of each stage in the same swizzled layout
+//   all warps       epilogue: tcgen05.ld one accumulator row per thread,
+//                   max over the G real heads -> agg[row, j]
+// The last CTA of a row to finish (atomic ticket in the workspace) runs the
+// deterministic top-K_b over the row's NB scores, read back from L2.
+//
+// Every mbarrier wait is bounded (2 s); on expiry the workspace error word
+// is set and the CTA skips the rest of its work, frees its TMEM and returns.
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "device_common.cuh"
+#include "host_common.h"
+
+namespace tls {
+
+constexpr int kBsTile = 128;     // blocks per CTA (MMA M)
+constexpr int kBsChunk = 64;     // K elements per pipeline stage (128 B of bf16)
+constexpr int kBsStages = 4;
+constexpr uint64_t kWaitNs = 2000000000ull;
+
+struct BlockScoreParams {
+  const uint16_t* q;
+  int n_q_heads, n_kv_heads, group, dqk;
+  int nb, K_b;
+  float* agg;          // workspace [rows, nb]
+  float* block_score;  // optional copy of agg
+  unsigned* counters;  // workspace [rows]
+  int32_t* block_idx;  // [rows, K_b]
+  int* err;            // workspace error word
+};
+
+__device__ __forceinline__ uint32_t relu_bf16x2(uint32_t w) {
+  uint32_t neg = (w & 0x80008000u) >> 15;  // 1 in each negative half
+  return w & ~(neg * 0xFFFFu);
+}
+__device__ __forceinline__ uint32_t min0_bf16x2(uint32_t w) {
+  uint32_t neg = (w & 0x80008000u) >> 15;
+  return w & (neg * 0xFFFFu);
+}
+
+template <int NPAD>
+struct BsSmem {
+  static constexpr int A_BYTES = kBsTile * 128;
+  static constexpr int B_BYTES = NPAD * 128;
+  static constexpr int STAGE_BYTES = kBsStages * (A_BYTES + B_BYTES);
+};
+
+template <int NPAD>
+__global__ void __launch_bounds__(128, 1)
+    block_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, BlockScoreParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  using L = BsSmem<NPAD>;
+  const int sel_bytes = p.nb * 4 + (int)sizeof(TopkScratch);
+  const int body = L::STAGE_BYTES > sel_bytes ? L::STAGE_BYTES : sel_bytes;
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kBsStages * L::A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + ((body + 7) & ~7));
+  uint64_t* empty = full + kBsStages;
+  uint64_t* done = empty + kBsStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* flags = reinterpret_cast<volatile int*>(tmem_slot + 1);  // [0] last CTA, [1] failed
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int row = blockIdx.y, mt = blockIdx.x;
+  const int nk = (2 * p.dqk) / kBsChunk;
+  constexpr uint32_t kCols = NPAD < 32 ? 32u : (uint32_t)NPAD;
+
+  if (tid == 0) {
+    for (int s = 0; s < kBsStages; ++s) {
+      mbar_init(&full[s], 1 + 64);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(done, 1);
+    flags[0] = 0;
+    flags[1] = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) tmem_alloc(tmem_slot, kCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int kc = 0; kc < nk; ++kc) {
+        const int s = kc % kBsStages, r = kc / kBsStages;
+        if (r > 0 && !mbar_wait_bounded(&empty[s], (r - 1) & 1, kWaitNs)) {
+          report_error(p.err, kErrTimeout, 101);
+          flags[1] = 1;
+          break;
+        }
+        mbar_arrive_expect_tx(&full[s], L::A_BYTES);
+        tma_load_2d(sA + s * L::A_BYTES, &tmap, &full[s], kc * kBsChunk, row * p.nb + mt * kBsTile);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(kBsTile, NPAD);
+      bool ok = true;
+      for (int kc = 0; kc < nk; ++kc) {
+        const int s = kc % kBsStages, r = kc / kBsStages;
+        if (!mbar_wait_bounded(&full[s], r & 1, kWaitNs)) {
+          report_error(p.err, kErrTimeout, 102);
+          flags[1] = 1;
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(sA + s * L::A_BYTES);
+        const uint32_t b0 = smem_u32(sB + s * L::B_BYTES);
+#pragma unroll
+        for (int k16 = 0; k16 < kBsChunk / 16; ++k16)
+          tc_mma_bf16(tmem, sw128_kmajor_desc(a0 + k16 * 32), sw128_kmajor_desc(b0 + k16 * 32), idesc,
+                      (kc | k16) != 0);
+        tc_commit(&empty[s]);
+      }
+      if (ok) tc_commit(done);
+    }
+  } else {
+    // Q' producers: row h of a stage holds Q'[h, kc*64 .. kc*64+63] as eight
+    // 16-byte chunks, chunk c stored at position c ^ (h % 8) (128B swizzle).
+    const int t = tid - 64;
+    const int g = p.group;
+    const int b = row / p.n_kv_heads, kvh = row % p.n_kv_heads;
+    const uint16_t* qg = p.q + ((int64_t)b * p.n_q_heads + (int64_t)kvh * g) * p.dqk;
+    for (int kc = 0; kc < nk; ++kc) {
+      const int s = kc % kBsStages, r = kc / kBsStages;
+      if (r > 0 && !mbar_wait_bounded(&empty[s], (r - 1) & 1, kWaitNs)) {
+        report_error(p.err, kErrTimeout, 103);
+        flags[1] = 1;
+        break;
+      }
+      uint8_t* dst = sB + s * L::B_BYTES;
+      for (int v = t; v < NPAD * 8; v += 64) {
+        const int h = v >> 3, c = v & 7;
+        const int e0 = kc * kBsChunk + c * 8;
+        uint4 w = make_uint4(0u, 0u, 0u, 0u);
+        if (h < g) {
+          const bool lo_half = e0 < p.dqk;
+          const uint4 x = *reinterpret_cast<const uint4*>(qg + (int64_t)h * p.dqk + (lo_half ? e0 : e0 - p.dqk));
+          if (lo_half) w = make_uint4(relu_bf16x2(x.x), relu_bf16x2(x.y), relu_bf16x2(x.z), relu_bf16x2(x.w));
+          else w = make_uint4(min0_bf16x2(x.x), min0_bf16x2(x.y), min0_bf16x2(x.z), min0_bf16x2(x.w));
+        }
+        *reinterpret_cast<uint4*>(dst + h * 128 + ((c ^ (h & 7)) << 4)) = w;
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&full[s]);
+    }
+  }
+  __syncwarp();
+
+  // Epilogue: thread (warp w, lane l) owns accumulator row m = 32w + l.
+  bool ok = mbar_wait_bounded(done, 0, kWaitNs) && flags[1] == 0;
+  ok = __all_sync(0xffffffffu, ok);
+  tc_fence_after();
+  if (ok) {
+    const int j = mt * kBsTile + warp * 32 + lane;
+    float best = -INFINITY;
+#pragma unroll
+    for (int c0 = 0; c0 < NPAD; c0 += 16) {
+      float v[16];
+      tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if (c0 + i < p.group) best = fmaxf(best, v[i]);
+    }
+    if (j < p.nb) {
+      p.agg[(int64_t)row * p.nb + j] = best;
+      if (p.block_score != nullptr) p.block_score[(int64_t)row * p.nb + j] = best;
+    }
+  } else if (lane == 0) {
+    report_error(p.err, kErrTimeout, 104);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kCols);
+  }
+
+  // Last CTA of this row selects the top-K_b blocks.
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    unsigned prev = atomicInc(&p.counters[row], gridDim.x - 1);
+    flags[0] = (prev == gridDim.x - 1) ? 1 : 0;
+  }
+  __syncthreads();
+  if (flags[0] == 0) return;
+  __threadfence();
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem);
+  TopkScratch* ts = reinterpret_cast<TopkScratch*>(keys + p.nb);
+  const float* arow = p.agg + (int64_t)row * p.nb;
+  for (int i = tid; i < p.nb; i += 128) keys[i] = float_key(__ldcg(arow + i));
+  __syncthreads();
+  cta_topk_ascending<128>(keys, p.nb, p.K_b, p.block_idx + (int64_t)row * p.K_b, *ts, [](int i) { return i; });
+}
+
+// CUDA-core variant of the same scores (diagnostic; selected with
+// TLS_BLOCK_SCORE_KERNEL=simt).  One thread per block, Q' in shared memory.
+__global__ void __launch_bounds__(128) block_score_simt_kernel(const uint16_t* __restrict__ meta, BlockScoreParams p) {
+  extern __shared__ float qs[];  // [G][2*dqk] as float, then select scratch
+  const int tid = threadIdx.x;
+  const int row = blockIdx.y;
+  const int g = p.group, k2 = 2 * p.dqk;
+  const int b = row / p.n_kv_heads, kvh = row % p.n_kv_heads;
+  const uint16_t* qg = p.q + ((int64_t)b * p.n_q_heads + (int64_t)kvh * g) * p.dqk;
+  for (int i = tid; i < g * k2; i += 128) {
+    const int h = i / k2, e = i % k2;
+    const float x = __uint_as_float((uint32_t)qg[(int64_t)h * p.dqk + (e < p.dqk ? e : e - p.dqk)] << 16);
+    qs[i] = e < p.dqk ? fmaxf(x, 0.0f) : fminf(x, 0.0f);
+  }
+  __syncthreads();
+  const int j = blockIdx.x * 128 + tid;
+  if (j < p.nb) {
+    const uint16_t* m = meta + ((int64_t)row * p.nb + j) * k2;
+    float best = -INFINITY;
+    for (int h = 0; h < g; ++h) {
+      float acc = 0.0f;
+      for (int e = 0; e < k2; e += 8) {
+        float f[8];
+        unpack8(*reinterpret_cast<const uint4*>(m + e), f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc = fmaf(qs[h * k2 + e + i], f[i], acc);
+      }
+      best = fmaxf(best, acc);
+    }
+    p.agg[(int64_t)row * p.nb + j] = best;
+    if (p.block_score != nullptr) p.block_score[(int64_t)row * p.nb + j] = best;
+  }
+  __threadfence();
+  __syncthreads();
+  __shared__ int last;
+  if (tid == 0) last = atomicInc(&p.counters[row], gridDim.x - 1) == gridDim.x - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  uint32_t* keys = reinterpret_cast<uint32_t*>(qs + (size_t)g * k2);
+  TopkScratch* ts = reinterpret_cast<TopkScratch*>(keys + p.nb);
+  const float* arow = p.agg + (int64_t)row * p.nb;
+  for (int i = tid; i < p.nb; i += 128) keys[i] = float_key(__ldcg(arow + i));
+  __syncthreads();
+  cta_topk_ascending<128>(keys, p.nb, p.K_b, p.block_idx + (int64_t)row * p.K_b, *ts, [](int i) { return i; });
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+tls_status get_encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (g_encode == nullptr) return fail(TLS_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  return TLS_OK;
+}
+
+bool use_simt() {
+  static const bool v = [] {
+    const char* e = std::getenv("TLS_BLOCK_SCORE_KERNEL");
+    return e != nullptr && std::strcmp(e, "simt") == 0;
+  }();
+  return v;
+}
+
+template <int NPAD>
+tls_status launch_tc(const CUtensorMap& tmap, const BlockScoreParams& p, int rows, cudaStream_t stream) {
+  using L = BsSmem<NPAD>;
+  const int sel_bytes = p.nb * 4 + (int)sizeof(TopkScratch);
+  const int body = L::STAGE_BYTES > sel_bytes ? L::STAGE_BYTES : sel_bytes;
+  const size_t smem = 1024 + (size_t)((body + 7) & ~7) + (2 * kBsStages + 1) * 8 + 16;
+  cudaError_t e = cudaFuncSetAttribute(block_score_tc_kernel<NPAD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return cuda_check(e, "select_blocks: set smem attribute");
+  dim3 grid((unsigned)((p.nb + kBsTile - 1) / kBsTile), (unsigned)rows);
+  block_score_tc_kernel<NPAD><<<grid, 128, smem, stream>>>(tmap, p);
+  return launch_check("select_blocks: block_score_tc launch");
+}
+
+}  // namespace
+
+tls_status select_blocks_impl(const tls_shape& s, const void* q, const void* meta, int K_b, int32_t* block_idx,
+                              float* block_score, uint8_t* ws, const WsLayout& L, cudaStream_t stream) {
+  const int rows = rows_of(s);
+  const int nb = (int)n_blocks(s);
+  BlockScoreParams p;
+  p.q = (const uint16_t*)q;
+  p.n_q_heads = s.n_q_heads;
+  p.n_kv_heads = s.n_kv_heads;
+  p.group = group_of(s);
+  p.dqk = s.qk_dim;
+  p.nb = nb;
+  p.K_b = K_b;
+  p.agg = reinterpret_cast<float*>(ws + L.agg);
+  p.block_score = block_score;
+  p.counters = reinterpret_cast<unsigned*>(ws + L.blk_counter);
+  p.block_idx = block_idx;
+  p.err = reinterpret_cast<int*>(ws + L.err);
+
+  if (use_simt()) {
+    const size_t smem = (size_t)p.group * 2 * s.qk_dim * 4 + (size_t)nb * 4 + sizeof(TopkScratch) + 16;
+    cudaError_t e = cudaFuncSetAttribute(block_score_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return cuda_check(e, "select_blocks: set smem attribute");
+    dim3 grid((unsigned)((nb + 127) / 128), (unsigned)rows);
+    block_score_simt_kernel<<<grid, 128, smem, stream>>>((const uint16_t*)meta, p);
+    return launch_check("select_blocks: block_score_simt launch");
+  }
+
+  tls_status st = get_encoder();
+  if (st != TLS_OK) return st;
+  CUtensorMap tmap;
+  const cuuint64_t dims[2] = {(cuuint64_t)(2 * s.qk_dim), (cuuint64_t)rows * (cuuint64_t)nb};
+  const cuuint64_t strides[1] = {(cuuint64_t)(2 * s.qk_dim) * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)kBsChunk, (cuuint32_t)kBsTile};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(meta), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(TLS_ERR_CUDA, "select_blocks: cuTensorMapEncodeTiled failed (%d)", (int)r);
+
+  const int g = p.group;
+  if (g <= 16) return launch_tc<16>(tmap, p, rows, stream);
+  if (g <= 32) return launch_tc<32>(tmap, p, rows, stream);
+  if (g <= 64) return launch_tc<64>(tmap, p, rows, stream);
+  if (g <= 128) return launch_tc<128>(tmap, p, rows, stream);
+  if (g <= 256) return launch_tc<256>(tmap, p, rows, stream);
+  return fail(TLS_ERR_UNSUPPORTED, "select_blocks: group size %d > 256", g);
+}
+
+}  // namespace tls

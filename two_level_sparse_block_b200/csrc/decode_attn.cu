@@ -1,0 +1,318 @@
+// Attention over the chosen tokens only (AsyncTLS, Italian summary 2.A.2; the
+// token list comes from level 2, English summary 2.A Stage 2).
+//
+// Split-K flash decoding.  Grid (splits, head groups, rows); a CTA takes a
+// contiguous slice of the row's token list and HG heads of the group.  Each
+// half-warp handles one token at a time: its 16 lanes load the token's K row
+// (and V row) with 16-byte loads, reduce the per-head dot products with
+// shuffles, and keep an online softmax (base-2 exponentials, fp32) plus an
+// fp32 accumulator.  The CTA folds its 8 half-warps, writes (m, l, acc) to
+// the workspace, and the last CTA of each (row, head group) merges the splits
+// by log-sum-exp and writes the output (fp32 or bf16) and the natural-log lse.
+
+#include "device_common.cuh"
+#include "host_common.h"
+
+namespace tls {
+
+struct AttnParams {
+  const uint16_t* q;
+  const uint16_t* k;
+  const uint16_t* v;
+  int64_t k_stride, v_stride;
+  const int32_t* slot_of_block;
+  int bs, nb, n_slots;
+  int64_t ctx_len;
+  const int32_t* token_idx;
+  int k_sel;
+  int n_q_heads, n_kv_heads, group, dqk, dv;
+  float scale_log2;
+  int tokens_per_split, splits, head_groups;
+  float* partial;      // workspace [rows][G][splits][dv + 2]
+  unsigned* counters;  // workspace [rows * head_groups]
+  void* out;
+  int out_bf16;
+  float* lse;
+};
+
+template <int PK, int PV, int HG, int U>
+__global__ void __launch_bounds__(128) sparse_attn_kernel(AttnParams p) {
+  extern __shared__ float red[];  // [8][HG] m, [8][HG] l, [8][HG][dv] acc
+  __shared__ int last;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int l16 = lane & 15, half = lane >> 4;
+  const int hw = warp * 2 + half;  // half-warp id 0..7
+  const int split = blockIdx.x, hg = blockIdx.y, row = blockIdx.z;
+  const int g = p.group;
+  const int b = row / p.n_kv_heads, kvh = row % p.n_kv_heads;
+  const int h0 = hg * HG;
+
+  // q slice of this lane: element e = pass*128 + l16*8 + i
+  float qf[HG][PK][8];
+#pragma unroll
+  for (int hh = 0; hh < HG; ++hh) {
+    const int h = h0 + hh;
+#pragma unroll
+    for (int ps = 0; ps < PK; ++ps) {
+      const int e = ps * 128 + l16 * 8;
+      if (h < g && e < p.dqk) {
+        const uint4 w = *reinterpret_cast<const uint4*>(p.q + ((int64_t)b * p.n_q_heads + kvh * g + h) * p.dqk + e);
+        unpack8(w, qf[hh][ps]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) qf[hh][ps][i] = 0.0f;
+      }
+    }
+  }
+
+  float m[HG], l[HG], acc[HG][PV][8];
+#pragma unroll
+  for (int hh = 0; hh < HG; ++hh) {
+    m[hh] = -INFINITY;
+    l[hh] = 0.0f;
+#pragma unroll
+    for (int ps = 0; ps < PV; ++ps)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[hh][ps][i] = 0.0f;
+  }
+
+  const int t_begin = split * p.tokens_per_split;
+  const int t_end = min(p.k_sel, t_begin + p.tokens_per_split);
+  const int32_t* tix = p.token_idx + (int64_t)row * p.k_sel;
+
+  for (int base = t_begin; base < t_end; base += 8 * U) {
+    uint4 kw[U][PK], vw[U][PV];
+    bool valid[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int t = base + u * 8 + hw;
+      valid[u] = t < t_end;
+      int64_t krow = 0, vrow = 0;
+      if (valid[u]) {
+        // indices are clamped so a bad list can never address outside the cache
+        const int64_t tok = min(max((int64_t)tix[t], (int64_t)0), p.ctx_len - 1);
+        int64_t r;
+        if (p.slot_of_block != nullptr) {
+          const int64_t slot = min(max(p.slot_of_block[(int64_t)row * p.nb + tok / p.bs], 0), p.n_slots - 1);
+          r = slot * p.bs + tok % p.bs;
+        } else {
+          r = (int64_t)row * p.ctx_len + tok;
+        }
+        krow = r * p.k_stride;
+        vrow = r * p.v_stride;
+      }
+#pragma unroll
+      for (int ps = 0; ps < PK; ++ps) {
+        const int e = ps * 128 + l16 * 8;
+        kw[u][ps] = (valid[u] && e < p.dqk) ? __ldg(reinterpret_cast<const uint4*>(p.k + krow + e))
+                                            : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int ps = 0; ps < PV; ++ps) {
+        const int e = ps * 128 + l16 * 8;
+        vw[u][ps] = (valid[u] && e < p.dv) ? __ldg(reinterpret_cast<const uint4*>(p.v + vrow + e))
+                                           : make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+
+    float sc[U][HG];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      float part[HG];
+#pragma unroll
+      for (int hh = 0; hh < HG; ++hh) part[hh] = 0.0f;
+#pragma unroll
+      for (int ps = 0; ps < PK; ++ps) {
+        float kf[8];
+        unpack8(kw[u][ps], kf);
+#pragma unroll
+        for (int hh = 0; hh < HG; ++hh)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) part[hh] = fmaf(qf[hh][ps][i], kf[i], part[hh]);
+      }
+#pragma unroll
+      for (int hh = 0; hh < HG; ++hh) {
+        float x = part[hh];
+        x += __shfl_xor_sync(0xffffffffu, x, 8);
+        x += __shfl_xor_sync(0xffffffffu, x, 4);
+        x += __shfl_xor_sync(0xffffffffu, x, 2);
+        x += __shfl_xor_sync(0xffffffffu, x, 1);
+        sc[u][hh] = valid[u] ? x * p.scale_log2 : -INFINITY;
+      }
+    }
+
+#pragma unroll
+    for (int hh = 0; hh < HG; ++hh) {
+      float mn = m[hh];
+#pragma unroll
+      for (int u = 0; u < U; ++u) mn = fmaxf(mn, sc[u][hh]);
+      if (mn == -INFINITY) continue;
+      const float corr = (m[hh] == -INFINITY) ? 0.0f : exp2f(m[hh] - mn);
+      float pu[U];
+      float psum = 0.0f;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        pu[u] = valid[u] ? exp2f(sc[u][hh] - mn) : 0.0f;
+        psum += pu[u];
+      }
+      l[hh] = l[hh] * corr + psum;
+      m[hh] = mn;
+#pragma unroll
+      for (int ps = 0; ps < PV; ++ps) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[hh][ps][i] *= corr;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          float vf[8];
+          unpack8(vw[u][ps], vf);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[hh][ps][i] = fmaf(pu[u], vf[i], acc[hh][ps][i]);
+        }
+      }
+    }
+  }
+
+  // fold the 8 half-warps of the CTA
+  const int dv = p.dv;
+  float* rm = red;
+  float* rl = red + 8 * HG;
+  float* ra = red + 16 * HG;
+#pragma unroll
+  for (int hh = 0; hh < HG; ++hh) {
+    if (l16 == 0) {
+      rm[hw * HG + hh] = m[hh];
+      rl[hw * HG + hh] = l[hh];
+    }
+#pragma unroll
+    for (int ps = 0; ps < PV; ++ps) {
+      const int e = ps * 128 + l16 * 8;
+      if (e < dv) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ra[((size_t)hw * HG + hh) * dv + e + i] = acc[hh][ps][i];
+      }
+    }
+  }
+  __syncthreads();
+  const int nh = min(HG, g - h0);
+  for (int idx = tid; idx < nh * (dv + 2); idx += 128) {
+    const int hh = idx / (dv + 2), e = idx % (dv + 2);
+    float M = -INFINITY;
+    for (int w = 0; w < 8; ++w) M = fmaxf(M, rm[w * HG + hh]);
+    float val = 0.0f;
+    if (e == 0) {
+      val = M;
+    } else if (M != -INFINITY) {
+      for (int w = 0; w < 8; ++w) {
+        const float mw = rm[w * HG + hh];
+        if (mw == -INFINITY) continue;
+        const float f = exp2f(mw - M);
+        val += f * (e == 1 ? rl[w * HG + hh] : ra[((size_t)w * HG + hh) * dv + (e - 2)]);
+      }
+    }
+    p.partial[(((int64_t)row * g + h0 + hh) * p.splits + split) * (dv + 2) + e] = val;
+  }
+
+  __threadfence();
+  __syncthreads();
+  if (tid == 0)
+    last = atomicInc(&p.counters[row * p.head_groups + hg], p.splits - 1) == (unsigned)(p.splits - 1);
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+
+  // merge the splits of heads h0 .. h0+nh-1 and write the outputs
+  for (int idx = tid; idx < nh * dv; idx += 128) {
+    const int hh = idx / dv, e = idx % dv;
+    const float* pp = p.partial + ((int64_t)row * g + h0 + hh) * p.splits * (dv + 2);
+    float M = -INFINITY;
+    for (int s = 0; s < p.splits; ++s) M = fmaxf(M, __ldcg(pp + (int64_t)s * (dv + 2)));
+    float L = 0.0f, A = 0.0f;
+    for (int s = 0; s < p.splits; ++s) {
+      const float ms = __ldcg(pp + (int64_t)s * (dv + 2));
+      if (ms == -INFINITY) continue;
+      const float f = exp2f(ms - M);
+      L += f * __ldcg(pp + (int64_t)s * (dv + 2) + 1);
+      A += f * __ldcg(pp + (int64_t)s * (dv + 2) + 2 + e);
+    }
+    const float o = A / L;
+    const int64_t oh = (int64_t)b * p.n_q_heads + kvh * g + h0 + hh;
+    if (p.out_bf16) reinterpret_cast<uint16_t*>(p.out)[oh * dv + e] = f32_to_bf16_rn(o);
+    else reinterpret_cast<float*>(p.out)[oh * dv + e] = o;
+    if (e == 0 && p.lse != nullptr) p.lse[oh] = (M + log2f(L)) * 0.69314718055994531f;
+  }
+}
+
+template <int PK, int PV, int HG>
+tls_status launch_attn(const AttnParams& p, int rows, cudaStream_t stream) {
+  constexpr int U = (PK + PV <= 2) ? 4 : 1;
+  const size_t smem = (size_t)(16 * HG + 8 * HG * p.dv) * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<PK, PV, HG, U>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return cuda_check(e, "sparse_decode_attn: set smem attribute");
+  dim3 grid((unsigned)p.splits, (unsigned)p.head_groups, (unsigned)rows);
+  sparse_attn_kernel<PK, PV, HG, U><<<grid, 128, smem, stream>>>(p);
+  return launch_check("sparse_decode_attn launch");
+}
+
+tls_status sparse_attn_impl(const tls_shape& s, const void* q, const tls_kv_view& kv, const int32_t* token_idx,
+                            int k, int out_dtype, void* out, float* lse, uint8_t* ws, const WsLayout& L,
+                            cudaStream_t stream) {
+  AttnParams p;
+  p.q = (const uint16_t*)q;
+  p.k = (const uint16_t*)kv.k;
+  p.v = s.v_offset >= 0 ? (const uint16_t*)kv.k + s.v_offset : (const uint16_t*)kv.v;
+  p.k_stride = kv.k_row_stride;
+  p.v_stride = s.v_offset >= 0 ? kv.k_row_stride : kv.v_row_stride;
+  p.slot_of_block = kv.slot_of_block;
+  p.n_slots = kv.n_slots;
+  p.bs = s.block_size;
+  p.nb = (int)n_blocks(s);
+  p.ctx_len = s.ctx_len;
+  p.token_idx = token_idx;
+  p.k_sel = k;
+  p.n_q_heads = s.n_q_heads;
+  p.n_kv_heads = s.n_kv_heads;
+  p.group = group_of(s);
+  p.dqk = s.qk_dim;
+  p.dv = s.v_dim;
+  p.scale_log2 = s.softmax_scale * 1.4426950408889634f;
+  p.tokens_per_split = L.tokens_per_split;
+  p.splits = L.splits;
+  p.head_groups = L.head_groups;
+  p.partial = reinterpret_cast<float*>(ws + L.partial);
+  p.counters = reinterpret_cast<unsigned*>(ws + L.att_counter);
+  p.out = out;
+  p.out_bf16 = out_dtype == TLS_OUT_BF16;
+  p.lse = lse;
+  const int rows = rows_of(s);
+  const int pk = (s.qk_dim + 127) / 128, pv = (s.v_dim + 127) / 128;
+  const int hg = L.heads_per_cta;
+  if (pk == 1 && pv == 1) {
+    if (hg == 1) return launch_attn<1, 1, 1>(p, rows, stream);
+    if (hg == 2) return launch_attn<1, 1, 2>(p, rows, stream);
+    if (hg == 4) return launch_attn<1, 1, 4>(p, rows, stream);
+    if (hg == 8) return launch_attn<1, 1, 8>(p, rows, stream);
+  } else if (pk <= 2 && pv <= 2) {
+    if (hg == 1) return launch_attn<2, 2, 1>(p, rows, stream);
+    if (hg == 2) return launch_attn<2, 2, 2>(p, rows, stream);
+    if (hg == 4) return launch_attn<2, 2, 4>(p, rows, stream);
+  } else if (pk <= 5 && pv <= 4) {
+    if (hg == 1) return launch_attn<5, 4, 1>(p, rows, stream);
+    if (hg == 2) return launch_attn<5, 4, 2>(p, rows, stream);
+  }
+  return fail(TLS_ERR_UNSUPPORTED, "sparse_decode_attn: no kernel for qk_dim %d, v_dim %d, %d heads per CTA",
+              s.qk_dim, s.v_dim, hg);
+}
+
+// Heads per CTA for the attention kernel: the register budget allows 8 heads
+// at 128-wide rows, 4 at 256 and 2 above.
+int attn_heads_per_cta(const tls_shape& s) {
+  const int g = group_of(s);
+  const int pk = (s.qk_dim + 127) / 128, pv = (s.v_dim + 127) / 128;
+  int cap = (pk == 1 && pv == 1) ? 8 : (pk <= 2 && pv <= 2) ? 4 : 2;
+  int hg = 1;
+  while (hg < g && hg < cap) hg <<= 1;
+  return hg;
+}
+
+}  // namespace tls

@@ -1,0 +1,60 @@
+// Host-side helpers shared by the libtls entry points.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "../../include/tls.h"
+
+namespace tls {
+
+// Sets the thread-local error message and returns `st`.
+tls_status fail(tls_status st, const char* fmt, ...);
+void clear_error();
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Validates the fields every call depends on.
+tls_status check_shape(const tls_shape* s);
+
+inline int64_t n_blocks(const tls_shape& s) { return s.ctx_len / s.block_size; }
+inline int rows_of(const tls_shape& s) { return s.batch * s.n_kv_heads; }
+inline int group_of(const tls_shape& s) { return s.n_q_heads / s.n_kv_heads; }
+
+inline tls_status cuda_check(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return TLS_OK;
+  return fail(TLS_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// Launch-time error (configuration or earlier sticky error).
+inline tls_status launch_check(const char* what) { return cuda_check(cudaGetLastError(), what); }
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Workspace layout shared by the selection and attention entry points.
+struct WsLayout {
+  size_t err;          // int[64] header: error word, location word
+  size_t blk_counter;  // unsigned[rows]
+  size_t tok_counter;  // unsigned[rows]
+  size_t att_counter;  // unsigned[rows]
+  size_t agg;          // float[rows * NB]
+  size_t tscore;       // float[rows * K_b * bs]
+  size_t partial;      // float[rows * G * splits * (Dv + 2)]
+  size_t total;
+  int splits;          // attention split count along the token list
+  int head_groups;     // attention CTAs along the heads of a group
+  int heads_per_cta;
+  int tokens_per_split;
+};
+
+// Plans the attention launch and the workspace for (shape, K_b, k).
+tls_status plan_workspace(const tls_shape& s, int K_b, int k, WsLayout* out);
+
+constexpr int kNumSMs = 148;
+
+}  // namespace tls

@@ -1,0 +1,105 @@
+"""Device-resident state for the decode step, built on the C ABI.
+
+``DecodeState`` owns the device buffers of one attention layer (queries, K/V
+cache, block metadata, INT4 label cache, index lists, output, workspace) and
+calls libtls for every step of the path.  PyTorch is used only to allocate
+device memory and to name the stream.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+from . import tls
+
+
+def _bf16_from_bits(a: np.ndarray, device) -> torch.Tensor:
+    t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16))
+    return t.to(device).view(torch.bfloat16)
+
+
+class DecodeState:
+    """One layer's KV cache and index, resident in HBM, with its step buffers.
+
+    q_bits: uint16 [B, Hq, Dqk]; k_bits: uint16 [B, Hkv, N, Dqk];
+    v_bits: uint16 [B, Hkv, N, Dv] or None (V is the K row slice at v_offset);
+    label_ch: int32 [Hkv, R].  bf16 arrays are passed as their bit patterns.
+    """
+
+    def __init__(self, *, batch, n_q_heads, n_kv_heads, qk_dim, v_dim, v_offset, block_size, n_label, ctx_len,
+                 K_b, k, q_bits, k_bits, v_bits, label_ch, softmax_scale=None, out_dtype=tls.TLS_OUT_F32,
+                 device="cuda", build_index=True, kv_device=None):
+        self.device = torch.device(device)
+        scale = 1.0 / math.sqrt(qk_dim) if softmax_scale is None else softmax_scale
+        self.shape = tls.make_shape(batch, n_q_heads, n_kv_heads, qk_dim, v_dim, v_offset, block_size, n_label,
+                                    ctx_len, scale)
+        self.K_b, self.k = int(K_b), int(k)
+        self.rows = batch * n_kv_heads
+        self.nb = ctx_len // block_size
+        self.out_dtype = out_dtype
+        dev = self.device
+        self.q = _bf16_from_bits(q_bits, dev)
+        self.kc = _bf16_from_bits(k_bits, kv_device or dev) if k_bits is not None else None
+        self.vc = _bf16_from_bits(v_bits, kv_device or dev) if v_bits is not None else None
+        self.label_ch = torch.from_numpy(np.ascontiguousarray(label_ch, dtype=np.int32)).to(dev)
+        self.meta = torch.empty((batch, n_kv_heads, self.nb, 2 * qk_dim), dtype=torch.bfloat16, device=dev)
+        self.codes = torch.empty((batch, n_kv_heads, ctx_len, n_label // 2), dtype=torch.uint8, device=dev)
+        self.scales = torch.empty((batch, n_kv_heads, ctx_len), dtype=torch.float32, device=dev)
+        self.block_idx = torch.empty((batch, n_kv_heads, self.K_b), dtype=torch.int32, device=dev)
+        self.token_idx = torch.empty((batch, n_kv_heads, self.k), dtype=torch.int32, device=dev)
+        self.block_score = torch.empty((batch, n_kv_heads, self.nb), dtype=torch.float32, device=dev)
+        self.token_score = torch.empty((batch, n_kv_heads, self.K_b * block_size), dtype=torch.float32, device=dev)
+        odt = torch.float32 if out_dtype == tls.TLS_OUT_F32 else torch.bfloat16
+        self.out = torch.empty((batch, n_q_heads, v_dim), dtype=odt, device=dev)
+        self.lse = torch.empty((batch, n_q_heads), dtype=torch.float32, device=dev)
+        self.ws_bytes = tls.tls_workspace_bytes(self.shape, self.K_b, self.k)
+        if self.ws_bytes == 0:
+            raise tls.TlsError(tls.TLS_ERR_INVALID_ARG, "tls_workspace_bytes", "invalid shape / K_b / k")
+        self.ws = torch.zeros(self.ws_bytes, dtype=torch.uint8, device=dev)
+        if self.kc is not None:
+            v = self.vc if self.vc is not None else self.kc
+            self.kv = tls.make_kv_view(self.kc, v, qk_dim, v_dim if self.vc is not None else qk_dim)
+        if build_index and self.kc is not None:
+            self.build_index()
+
+    # index build (prefill) -------------------------------------------------
+    def build_index(self, t0: int = 0, t1: int | None = None, stream=None):
+        s = self.shape
+        t1 = s.ctx_len if t1 is None else t1
+        tls.tls_build_block_meta(s, self.kc, s.qk_dim, t0, t1, self.meta, stream)
+        tls.tls_quant_label_cache(s, self.kc, s.qk_dim, self.label_ch, t0, t1, self.codes, self.scales, stream)
+
+    # the per-step path -----------------------------------------------------
+    def select_blocks(self, q=None, keep_scores=False, stream=None):
+        tls.tls_select_blocks(self.shape, self.q if q is None else q, self.meta, self.K_b, self.block_idx,
+                              self.block_score if keep_scores else None, self.ws, self.ws_bytes, stream)
+
+    def select_tokens(self, q=None, block_idx=None, keep_scores=False, stream=None):
+        tls.tls_select_tokens(self.shape, self.q if q is None else q, self.label_ch, self.codes, self.scales,
+                              self.block_idx if block_idx is None else block_idx, self.K_b, self.k, self.token_idx,
+                              self.token_score if keep_scores else None, self.ws, self.ws_bytes, stream)
+
+    def attend(self, q=None, token_idx=None, kv=None, stream=None):
+        tls.tls_sparse_decode_attn(self.shape, self.q if q is None else q, self.kv if kv is None else kv,
+                                   self.token_idx if token_idx is None else token_idx, self.k, self.out_dtype,
+                                   self.out, self.lse, self.ws, self.ws_bytes, stream)
+
+    def step(self, q=None, stream=None):
+        """One synchronous decode step: three kernel launches."""
+        tls.tls_decode_step(self.shape, self.q if q is None else q, self.meta, self.label_ch, self.codes,
+                            self.scales, self.kv, self.K_b, self.k, self.block_idx, self.token_idx, self.out_dtype,
+                            self.out, self.lse, self.ws, self.ws_bytes, stream)
+
+    def check_device_error(self, stream=None) -> int:
+        return tls.tls_workspace_error(self.ws, True, stream)
+
+
+def state_for_config(cfg, q_bits, k_bits, v_bits, label_ch, **kw) -> DecodeState:
+    """DecodeState for a workload description with the fields of synth.WorkloadConfig."""
+    return DecodeState(batch=cfg.batch, n_q_heads=cfg.n_q_heads, n_kv_heads=cfg.n_kv_heads, qk_dim=cfg.qk_dim,
+                       v_dim=cfg.v_dim, v_offset=cfg.v_offset, block_size=cfg.block_size, n_label=cfg.n_label,
+                       ctx_len=cfg.ctx_len, K_b=cfg.K_b, k=cfg.k, q_bits=q_bits, k_bits=k_bits, v_bits=v_bits,
+                       label_ch=label_ch, softmax_scale=cfg.softmax_scale, **kw)
