@@ -201,6 +201,34 @@ TLS_API tls_status tls_decode_step(const tls_shape* shape, const void* q, const 
                            int32_t* block_idx, int32_t* token_idx, int32_t out_dtype,
                            void* out, float* lse, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * Scratch-free variant of tls_sparse_decode_attn (no counterpart in the
+ * paper; it is a convenience of this library).  Same inputs, outputs and
+ * numerics, but it takes no workspace and allocates nothing: the split-K
+ * partials and merge tickets live in one fixed device array of
+ * TLS_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads
+ * the library holds until the process exits.
+ * Meant for callers that cannot allocate device memory: a plug-in inside a
+ * serving runtime that owns the whole HBM budget and offers no allocator, or
+ * a latency-critical decode loop where cudaMalloc (which may synchronise the
+ * device) is not allowed.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - Each call clears the tickets with cudaMemsetAsync on `stream`; it calls
+ *     no cudaMalloc, cudaFree or allocating library routine.
+ *   - All calls share the one array: two calls whose kernels overlap on the
+ *     GPU (e.g. on different streams) race and give wrong results.  Issue them
+ *     on one stream, or use tls_sparse_decode_attn with separate workspaces.
+ *   - Shapes whose scratch exceeds the array (tickets plus
+ *     rows * G * splits * (Dv + 2) floats) return TLS_ERR_CAPACITY and launch
+ *     nothing.
+ */
+#define TLS_NOALLOC_SCRATCH_BYTES (4u << 20)
+TLS_API tls_status tls_sparse_decode_attn_noalloc(const tls_shape* shape, const void* q, const tls_kv_view* kv,
+                                                  const int32_t* token_idx, int32_t k, int32_t out_dtype,
+                                                  void* out, float* lse, void* stream);
+
 /* ------------------------------------------------------------------------
  * Offloaded KV: HBM block cache with incremental transfer (section 2.B).
  * ------------------------------------------------------------------------ */

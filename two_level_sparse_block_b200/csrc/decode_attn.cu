@@ -10,6 +10,8 @@
 // the workspace, and the last CTA of each (row, head group) merges the splits
 // by log-sum-exp and writes the output (fp32 or bf16) and the natural-log lse.
 
+#include <mutex>
+
 #include "device_common.cuh"
 #include "host_common.h"
 
@@ -316,3 +318,88 @@ int attn_heads_per_cta(const tls_shape& s) {
 }
 
 }  // namespace tls
+
+// ---------------------------------------------------------------------------
+// Scratch-free variant of the attention entry point.
+//
+// Some callers cannot hand the library a workspace: code that runs as a
+// plug-in inside a serving runtime that owns the whole HBM budget and exposes
+// no allocator, and latency-critical decode loops where a cudaMalloc (which can
+// synchronise the device and take milliseconds) is not allowed.  For them the
+// split-K partials and the merge tickets live in one file-scope device array
+// of fixed size.  Every GPU that loads the library holds this array until the
+// process exits.  Host code must not pass the array's name to a kernel (on the
+// host it is only a stand-in symbol); the device address is looked up once per
+// device with cudaGetSymbolAddress, on the first call made on that device.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_attn_scratch[TLS_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {nullptr};
+}  // namespace
+
+static tls_status scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return tls::cuda_check(e, "sparse_decode_attn_noalloc: cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return tls::fail(TLS_ERR_UNSUPPORTED, "sparse_decode_attn_noalloc: device id %d", dev);
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_attn_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return tls::cuda_check(e != cudaSuccess ? e : cudaErrorInvalidSymbol,
+                             "sparse_decode_attn_noalloc: cudaGetSymbolAddress");
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return TLS_OK;
+}
+
+extern "C" tls_status tls_sparse_decode_attn_noalloc(const tls_shape* shape, const void* q, const tls_kv_view* kv,
+                                                     const int32_t* token_idx, int32_t k, int32_t out_dtype,
+                                                     void* out, float* lse, void* stream) {
+  using namespace tls;
+  clear_error();
+  tls_status st = check_shape(shape);
+  if (st != TLS_OK) return st;
+  const tls_shape& s = *shape;
+  if (q == nullptr || token_idx == nullptr || out == nullptr || kv == nullptr || kv->k == nullptr)
+    return fail(TLS_ERR_INVALID_ARG, "sparse_decode_attn_noalloc: null pointer");
+  if (!aligned16(q) || !aligned16(kv->k) || (s.v_offset < 0 && (kv->v == nullptr || !aligned16(kv->v))))
+    return fail(TLS_ERR_INVALID_ARG, "sparse_decode_attn_noalloc: q/k/v NULL or not 16-byte aligned");
+  if (kv->k_row_stride < s.qk_dim || kv->k_row_stride % 8 != 0 ||
+      (s.v_offset < 0 && (kv->v_row_stride < s.v_dim || kv->v_row_stride % 8 != 0)))
+    return fail(TLS_ERR_INVALID_ARG, "sparse_decode_attn_noalloc: bad row strides");
+  if (kv->slot_of_block != nullptr && kv->n_slots < 1)
+    return fail(TLS_ERR_INVALID_ARG, "sparse_decode_attn_noalloc: n_slots must be >= 1 with a slot table");
+  if (out_dtype != TLS_OUT_F32 && out_dtype != TLS_OUT_BF16)
+    return fail(TLS_ERR_INVALID_ARG, "sparse_decode_attn_noalloc: bad out_dtype");
+  if (k < 1 || k > s.ctx_len) return fail(TLS_ERR_INVALID_ARG, "sparse_decode_attn_noalloc: k %d out of range", k);
+  const int64_t nb = n_blocks(s);
+  int K_b = (int)((k + s.block_size - 1) / s.block_size);
+  if (K_b > nb) K_b = (int)nb;
+  WsLayout L;
+  st = plan_workspace(s, K_b, k, &L);
+  if (st != TLS_OK) return st;
+  // tickets first, then the partials, inside the static array
+  const size_t ticket_bytes = align_up((size_t)rows_of(s) * L.head_groups * sizeof(unsigned), 256);
+  const size_t partial_bytes = (size_t)rows_of(s) * group_of(s) * L.splits * (s.v_dim + 2) * sizeof(float);
+  if (ticket_bytes + partial_bytes > (size_t)TLS_NOALLOC_SCRATCH_BYTES)
+    return fail(TLS_ERR_CAPACITY,
+                "sparse_decode_attn_noalloc: this shape needs %zu bytes of scratch, above the fixed %u-byte "
+                "array; use tls_sparse_decode_attn with a workspace",
+                ticket_bytes + partial_bytes, (unsigned)TLS_NOALLOC_SCRATCH_BYTES);
+  void* base = nullptr;
+  st = scratch_address(&base);
+  if (st != TLS_OK) return st;
+  // the array keeps the previous call's contents: the tickets must start at zero
+  cudaError_t e = cudaMemsetAsync(base, 0, ticket_bytes, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_check(e, "sparse_decode_attn_noalloc: clear tickets");
+  WsLayout S = L;
+  S.att_counter = 0;
+  S.partial = ticket_bytes;
+  return sparse_attn_impl(s, q, *kv, token_idx, k, out_dtype, out, lse, (uint8_t*)base, S, (cudaStream_t)stream);
+}

@@ -72,6 +72,7 @@ _SIG = {
     "tls_select_blocks": (_I32, [_P, _P, _P, _I32, _P, _P, _P, _SZ, _P]),
     "tls_select_tokens": (_I32, [_P, _P, _P, _P, _P, _P, _I32, _I32, _P, _P, _P, _SZ, _P]),
     "tls_sparse_decode_attn": (_I32, [_P, _P, _P, _P, _I32, _I32, _P, _P, _P, _SZ, _P]),
+    "tls_sparse_decode_attn_noalloc": (_I32, [_P, _P, _P, _P, _I32, _I32, _P, _P, _P]),
     "tls_decode_step": (_I32, [_P, _P, _P, _P, _P, _P, _P, _I32, _I32, _P, _P, _I32, _P, _P, _P, _SZ, _P]),
     "tls_block_cache_create": (_I32, [_P, _P, _P, _I64, _I64, _I32, _P, _P, _P, _P]),
     "tls_block_cache_destroy": (None, [_P]),
@@ -180,6 +181,12 @@ def tls_sparse_decode_attn(shape, q, kv: KvView, token_idx, k, out_dtype, out, l
     _check(lib().tls_sparse_decode_attn(ctypes.byref(shape), _ptr(q), ctypes.byref(kv), _ptr(token_idx), k,
                                         out_dtype, _ptr(out), _ptr(lse), _ptr(ws), ws_bytes, _stream(stream)),
            "tls_sparse_decode_attn")
+
+
+def tls_sparse_decode_attn_noalloc(shape, q, kv: KvView, token_idx, k, out_dtype, out, lse, stream=None):
+    _check(lib().tls_sparse_decode_attn_noalloc(ctypes.byref(shape), _ptr(q), ctypes.byref(kv), _ptr(token_idx), k,
+                                                out_dtype, _ptr(out), _ptr(lse), _stream(stream)),
+           "tls_sparse_decode_attn_noalloc")
 
 
 def tls_decode_step(shape, q, meta, label_ch, codes, scales, kv: KvView, K_b, k, block_idx, token_idx, out_dtype,
