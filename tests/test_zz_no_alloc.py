@@ -60,9 +60,10 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(tls, name):
 
 
 def test_noalloc_rejects_scratch_beyond_its_array(tls):
-    # 512 rows x 8 heads x 2 splits x 130 floats = 4.26 MB > 4 MiB; real buffers are
-    # allocated so that even a wrongly accepted call would stay in bounds
-    B, Hkv, G, D, N, bs, k = 64, 8, 8, 128, 256, 32, 64
+    # 512 rows x 8 heads x 2 splits x 130 floats = 4.26 MB > 4 MiB (256 tokens make two
+    # 128-token splits); real buffers are allocated so that even a wrongly accepted call
+    # would stay in bounds
+    B, Hkv, G, D, N, bs, k = 64, 8, 8, 128, 256, 32, 256
     shape = tls.make_shape(B, Hkv * G, Hkv, D, D, -1, bs, 16, N, D ** -0.5)
     q = torch.zeros((B, Hkv * G, D), dtype=torch.bfloat16, device="cuda")
     kk = torch.zeros((B, Hkv, N, D), dtype=torch.bfloat16, device="cuda")
