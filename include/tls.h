@@ -191,9 +191,18 @@ TLS_API tls_status tls_sparse_decode_attn(const tls_shape* shape, const void* q,
                                   void* out, float* lse, void* ws, size_t ws_bytes, void* stream);
 
 /*
- * One synchronous decode step: tls_select_blocks, tls_select_tokens and
- * tls_sparse_decode_attn in order on `stream` (three kernel launches),
- * sharing one workspace.  block_idx / token_idx are outputs as above.
+ * Levels 1 and 2 together: tls_select_blocks followed by tls_select_tokens
+ * on `stream` (two kernel launches, one shared workspace); the same results
+ * as the two calls.  Arguments as in the two calls.
+ */
+TLS_API tls_status tls_select(const tls_shape* shape, const void* q, const void* meta, const int32_t* label_ch,
+                              const uint8_t* codes, const float* scales, int32_t K_b, int32_t k,
+                              int32_t* block_idx, int32_t* token_idx, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * One synchronous decode step: tls_select then tls_sparse_decode_attn on
+ * `stream` (three kernel launches), sharing one workspace.  block_idx /
+ * token_idx are outputs as above.
  */
 TLS_API tls_status tls_decode_step(const tls_shape* shape, const void* q, const void* meta,
                            const int32_t* label_ch, const uint8_t* codes, const float* scales,

@@ -257,3 +257,44 @@ def test_invalid_arguments_launch_nothing():
         tls.tls_select_blocks(bad, st.q, st.meta, cfg.K_b, st.block_idx, None, st.ws, 16)
     torch.cuda.synchronize()
     assert st.check_device_error() == 0
+
+
+def test_exact_ties_follow_the_lower_index_rule():
+    # keys and queries from {-1, -0.5, 0, 0.5, 1}: every score is a short dyadic
+    # sum, exact in float32, so the GPU and oracle scores are identical and the
+    # many ties must be broken exactly as the rule says (no tie band applies)
+    runtime, tls = _rt()
+    cfg = small("s_exact_ties", batch=2, n_q_heads=8, n_kv_heads=2, ctx_len=1024, block_size=16, K_b=13, k=97,
+                n_label=8, seed=31)
+    rng = np.random.default_rng(31)
+    vals = np.array([-1.0, -0.5, 0.0, 0.5, 1.0], dtype=np.float32)
+    from synth import bf16_bits_from_f32
+    K = bf16_bits_from_f32(rng.choice(vals, size=(2, 2, cfg.ctx_len, cfg.qk_dim)))
+    q = bf16_bits_from_f32(rng.choice(vals, size=(2, 8, cfg.qk_dim)))
+    V = synth.gen_kv(cfg, synth.gen_queries(cfg))[1]
+    lab = synth.gen_label_channels(cfg)
+    st = runtime.state_for_config(cfg, q, K, V, lab)
+    got = run_stages(st)
+    g = cfg.group
+    for b in range(2):
+        for h in range(2):
+            r1 = oracle.decode_row(q[b, h * g:(h + 1) * g], K[b, h], V[b, h], lab[h], cfg.block_size, cfg.K_b,
+                                   cfg.k, cfg.softmax_scale)
+            assert np.array_equal(got["block_score"][b, h], r1["agg"].astype(np.float32))
+            assert got["block_idx"][b, h].tolist() == r1["block_idx"].tolist()
+            r2 = oracle.decode_row(q[b, h * g:(h + 1) * g], K[b, h], V[b, h], lab[h], cfg.block_size, cfg.K_b,
+                                   cfg.k, cfg.softmax_scale, block_idx=got["block_idx"][b, h])
+            assert got["token_idx"][b, h].tolist() == r2["token_idx"].tolist()
+
+
+@pytest.mark.parametrize("cfg", SMALL + [get_config("c1")], ids=lambda c: c.name)
+def test_fused_select_equals_the_two_level_calls(cfg):
+    st, data = make_state(cfg)
+    got = run_stages(st)
+    st.block_idx.fill_(-1)
+    st.token_idx.fill_(-1)
+    st.select()
+    torch.cuda.synchronize()
+    assert st.check_device_error() == 0
+    assert np.array_equal(st.block_idx.cpu().numpy(), got["block_idx"])
+    assert np.array_equal(st.token_idx.cpu().numpy(), got["token_idx"])

@@ -6,18 +6,28 @@
 #include <cstring>
 
 #include "host_common.h"
+#include "token_common.cuh"
 
 namespace tls {
 
+void fill_token_params(TokenParams& p, const tls_shape& s, const void* q, const int32_t* label_ch,
+                       const uint8_t* codes, const float* scales, const int32_t* block_idx, int K_b, int k,
+                       int32_t* token_idx, float* token_score, uint8_t* ws, const WsLayout& L);
 tls_status select_blocks_impl(const tls_shape& s, const void* q, const void* meta, int K_b, int32_t* block_idx,
-                              float* block_score, uint8_t* ws, const WsLayout& L, cudaStream_t stream);
+                              float* block_score, uint8_t* ws, const WsLayout& L, cudaStream_t stream,
+                              const TokenParams* fuse = nullptr, bool* fused = nullptr);
 tls_status select_tokens_impl(const tls_shape& s, const void* q, const int32_t* label_ch, const uint8_t* codes,
                               const float* scales, const int32_t* block_idx, int K_b, int k, int32_t* token_idx,
-                              float* token_score, uint8_t* ws, const WsLayout& L, cudaStream_t stream);
+                              float* token_score, uint8_t* ws, const WsLayout& L, cudaStream_t stream,
+                              bool pdl = false);
 tls_status sparse_attn_impl(const tls_shape& s, const void* q, const tls_kv_view& kv, const int32_t* token_idx,
                             int k, int out_dtype, void* out, float* lse, uint8_t* ws, const WsLayout& L,
                             cudaStream_t stream);
 int attn_heads_per_cta(const tls_shape& s);
+bool attn_tc_supported(const tls_shape& s);
+int attn_tc_plan(int rows, int head_groups, int k, int* tiles, int* n_items, int* n_ctas);
+bool attn_mma_supported(const tls_shape& s);
+int attn_mma_plan(int rows, int k, int* chunks_per_row, int* n_items, int* n_ctas);
 
 namespace {
 thread_local char g_err[512] = {0};
@@ -69,15 +79,27 @@ tls_status plan_workspace(const tls_shape& s, int K_b, int k, WsLayout* out) {
   WsLayout L;
   L.heads_per_cta = attn_heads_per_cta(s);
   L.head_groups = (g + L.heads_per_cta - 1) / L.heads_per_cta;
-  const int target = 4 * kNumSMs;
-  int splits = (target + rows * L.head_groups - 1) / (rows * L.head_groups);
-  const int max_splits = (k + 15) / 16;
-  if (splits > max_splits) splits = max_splits;
-  if (splits < 1) splits = 1;
-  int tps = (k + splits - 1) / splits;
-  tps = (int)align_up((size_t)tps, 8);
-  L.tokens_per_split = tps;
-  L.splits = (k + tps - 1) / tps;
+  L.tiles_per_pair = L.n_items = L.n_ctas = 0;
+  if (attn_mma_supported(s)) {
+    // warp-streaming attention: persistent CTAs over 16-token chunks
+    L.tokens_per_split = 16;
+    L.splits = attn_mma_plan(rows, k, &L.tiles_per_pair, &L.n_items, &L.n_ctas);
+  } else if (attn_tc_supported(s)) {
+    // tensor-core attention: persistent CTAs over 128-token tiles; a split
+    // slot per CTA that shares a (row, head group)
+    L.tokens_per_split = 128;
+    L.splits = attn_tc_plan(rows, L.head_groups, k, &L.tiles_per_pair, &L.n_items, &L.n_ctas);
+  } else {
+    const int target = 4 * kNumSMs;
+    int splits = (target + rows * L.head_groups - 1) / (rows * L.head_groups);
+    int max_splits = (k + 15) / 16;
+    if (max_splits > 64) max_splits = 64;  // the split merge reads at most 64 splits
+    if (splits > max_splits) splits = max_splits;
+    if (splits < 1) splits = 1;
+    int tps = (k + splits - 1) / splits;
+    L.tokens_per_split = (int)align_up((size_t)tps, 8);
+    L.splits = (k + L.tokens_per_split - 1) / L.tokens_per_split;
+  }
   size_t off = 0;
   L.err = off;
   off += 256;
@@ -87,6 +109,7 @@ tls_status plan_workspace(const tls_shape& s, int K_b, int k, WsLayout* out) {
   off = align_up(off + (size_t)rows * 4, 256);
   L.att_counter = off;
   off = align_up(off + (size_t)rows * L.head_groups * 4, 256);
+  if (L.splits > 64) return fail(TLS_ERR_UNSUPPORTED, "attention plan needs %d splits (> 64)", L.splits);
   // regions that depend on fewer arguments come first, so that the offsets
   // a call uses do not depend on arguments it is not given
   L.agg = off;
@@ -216,15 +239,37 @@ extern "C" tls_status tls_sparse_decode_attn(const tls_shape* shape, const void*
                           (cudaStream_t)stream);
 }
 
+extern "C" tls_status tls_select(const tls_shape* shape, const void* q, const void* meta, const int32_t* label_ch,
+                                 const uint8_t* codes, const float* scales, int32_t K_b, int32_t k,
+                                 int32_t* block_idx, int32_t* token_idx, void* ws, size_t ws_bytes, void* stream) {
+  clear_error();
+  tls_status st = check_shape(shape);
+  if (st != TLS_OK) return st;
+  if (q == nullptr || meta == nullptr || label_ch == nullptr || codes == nullptr || scales == nullptr ||
+      block_idx == nullptr || token_idx == nullptr)
+    return fail(TLS_ERR_INVALID_ARG, "select: null pointer");
+  if (!aligned16(q) || !aligned16(meta) || !aligned16(codes))
+    return fail(TLS_ERR_INVALID_ARG, "select: q/meta/codes not 16-byte aligned");
+  WsLayout L;
+  st = check_ws(*shape, K_b, k, ws, ws_bytes, &L);
+  if (st != TLS_OK) return st;
+  TokenParams tp;
+  fill_token_params(tp, *shape, q, label_ch, codes, scales, block_idx, K_b, k, token_idx, nullptr, (uint8_t*)ws, L);
+  bool fused = false;
+  st = select_blocks_impl(*shape, q, meta, K_b, block_idx, nullptr, (uint8_t*)ws, L, (cudaStream_t)stream, &tp,
+                          &fused);
+  if (st != TLS_OK || fused) return st;
+  return select_tokens_impl(*shape, q, label_ch, codes, scales, block_idx, K_b, k, token_idx, nullptr,
+                            (uint8_t*)ws, L, (cudaStream_t)stream, /*pdl=*/true);
+}
+
 extern "C" tls_status tls_decode_step(const tls_shape* shape, const void* q, const void* meta,
                                       const int32_t* label_ch, const uint8_t* codes, const float* scales,
                                       const tls_kv_view* kv, int32_t K_b, int32_t k, int32_t* block_idx,
                                       int32_t* token_idx, int32_t out_dtype, void* out, float* lse, void* ws,
                                       size_t ws_bytes, void* stream) {
-  tls_status st = tls_select_blocks(shape, q, meta, K_b, block_idx, nullptr, ws, ws_bytes, stream);
-  if (st != TLS_OK) return st;
-  st = tls_select_tokens(shape, q, label_ch, codes, scales, block_idx, K_b, k, token_idx, nullptr, ws, ws_bytes,
-                         stream);
+  tls_status st = tls_select(shape, q, meta, label_ch, codes, scales, K_b, k, block_idx, token_idx, ws, ws_bytes,
+                             stream);
   if (st != TLS_OK) return st;
   return tls_sparse_decode_attn(shape, q, kv, token_idx, k, out_dtype, out, lse, ws, ws_bytes, stream);
 }

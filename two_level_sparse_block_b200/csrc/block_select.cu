@@ -30,6 +30,7 @@
 
 #include "device_common.cuh"
 #include "host_common.h"
+#include "token_common.cuh"
 
 namespace tls {
 
@@ -47,6 +48,8 @@ struct BlockScoreParams {
   unsigned* counters;  // workspace [rows]
   int32_t* block_idx;  // [rows, K_b]
   int* err;            // workspace error word
+  int fuse_tokens;     // the last CTA of a row goes on to level 2 (token selection)
+  TokenParams tok;
 };
 
 __device__ __forceinline__ uint32_t relu_bf16x2(uint32_t w) {
@@ -65,14 +68,25 @@ struct BsSmem {
   static constexpr int STAGE_BYTES = kBsStages * (A_BYTES + B_BYTES);
 };
 
-template <int NPAD>
+// Shared-memory bytes the body of a block-score CTA needs: the pipeline
+// stages, or the top-K_b keys, or (fused) the level-2 scores of one row.
+__host__ __device__ inline int bs_body_bytes(int stage_bytes, int nb, int tok_bytes) {
+  int body = stage_bytes;
+  const int sel = nb * 4 + (int)sizeof(TopkScratch);
+  if (sel > body) body = sel;
+  if (tok_bytes > body) body = tok_bytes;
+  return body;
+}
+
+template <int NPAD, int RT>
 __global__ void __launch_bounds__(128, 1)
     block_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, BlockScoreParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   using L = BsSmem<NPAD>;
-  const int sel_bytes = p.nb * 4 + (int)sizeof(TopkScratch);
-  const int body = L::STAGE_BYTES > sel_bytes ? L::STAGE_BYTES : sel_bytes;
+  const int tok_bytes =
+      RT > 0 && p.fuse_tokens ? (p.group * RT + p.tok.n_cand) * 4 + (int)sizeof(TopkScratch) : 0;
+  const int body = bs_body_bytes(L::STAGE_BYTES, p.nb, tok_bytes);
   uint8_t* sA = smem;
   uint8_t* sB = smem + kBsStages * L::A_BYTES;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + ((body + 7) & ~7));
@@ -85,6 +99,7 @@ __global__ void __launch_bounds__(128, 1)
   const int row = blockIdx.y, mt = blockIdx.x;
   const int nk = (2 * p.dqk) / kBsChunk;
   constexpr uint32_t kCols = NPAD < 32 ? 32u : (uint32_t)NPAD;
+  grid_launch_dependents();  // level 2 may be scheduled now; it waits for this grid before reading
 
   if (tid == 0) {
     for (int s = 0; s < kBsStages; ++s) {
@@ -216,6 +231,14 @@ __global__ void __launch_bounds__(128, 1)
   for (int i = tid; i < p.nb; i += 128) keys[i] = float_key(__ldcg(arow + i));
   __syncthreads();
   cta_topk_ascending<128>(keys, p.nb, p.K_b, p.block_idx + (int64_t)row * p.K_b, *ts, [](int i) { return i; });
+  if constexpr (RT > 0) {
+    if (p.fuse_tokens) {
+      // level 2 of this row right away: its block list is in global memory,
+      // written by this CTA (visible to the CTA after the barrier)
+      __syncthreads();
+      token_stage<RT, 128>(p.tok, row, reinterpret_cast<float*>(smem));
+    }
+  }
 }
 
 // CUDA-core variant of the same scores (diagnostic; selected with
@@ -293,24 +316,40 @@ bool use_simt() {
   return v;
 }
 
-template <int NPAD>
+template <int NPAD, int RT>
 tls_status launch_tc(const CUtensorMap& tmap, const BlockScoreParams& p, int rows, cudaStream_t stream) {
   using L = BsSmem<NPAD>;
-  const int sel_bytes = p.nb * 4 + (int)sizeof(TopkScratch);
-  const int body = L::STAGE_BYTES > sel_bytes ? L::STAGE_BYTES : sel_bytes;
+  const int tok_bytes =
+      RT > 0 && p.fuse_tokens ? (p.group * RT + p.tok.n_cand) * 4 + (int)sizeof(TopkScratch) : 0;
+  const int body = bs_body_bytes(L::STAGE_BYTES, p.nb, tok_bytes);
   const size_t smem = 1024 + (size_t)((body + 7) & ~7) + (2 * kBsStages + 1) * 8 + 16;
-  cudaError_t e = cudaFuncSetAttribute(block_score_tc_kernel<NPAD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(block_score_tc_kernel<NPAD, RT>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return cuda_check(e, "select_blocks: set smem attribute");
   dim3 grid((unsigned)((p.nb + kBsTile - 1) / kBsTile), (unsigned)rows);
-  block_score_tc_kernel<NPAD><<<grid, 128, smem, stream>>>(tmap, p);
+  block_score_tc_kernel<NPAD, RT><<<grid, 128, smem, stream>>>(tmap, p);
   return launch_check("select_blocks: block_score_tc launch");
+}
+
+template <int RT>
+tls_status launch_tc_group(const CUtensorMap& tmap, const BlockScoreParams& p, int rows, cudaStream_t stream) {
+  const int g = p.group;
+  if (g <= 16) return launch_tc<16, RT>(tmap, p, rows, stream);
+  if (g <= 32) return launch_tc<32, RT>(tmap, p, rows, stream);
+  if (g <= 64) return launch_tc<64, RT>(tmap, p, rows, stream);
+  if (g <= 128) return launch_tc<128, RT>(tmap, p, rows, stream);
+  if (g <= 256) return launch_tc<256, RT>(tmap, p, rows, stream);
+  return fail(TLS_ERR_UNSUPPORTED, "select_blocks: group size %d > 256", g);
 }
 
 }  // namespace
 
+// Level 1; with `fuse` (level-2 parameters of the same call) the last CTA of
+// each row also runs level 2 when it fits one CTA, and *fused says so.
 tls_status select_blocks_impl(const tls_shape& s, const void* q, const void* meta, int K_b, int32_t* block_idx,
-                              float* block_score, uint8_t* ws, const WsLayout& L, cudaStream_t stream) {
+                              float* block_score, uint8_t* ws, const WsLayout& L, cudaStream_t stream,
+                              const TokenParams* fuse, bool* fused) {
+  if (fused != nullptr) *fused = false;
   const int rows = rows_of(s);
   const int nb = (int)n_blocks(s);
   BlockScoreParams p;
@@ -326,6 +365,7 @@ tls_status select_blocks_impl(const tls_shape& s, const void* q, const void* met
   p.counters = reinterpret_cast<unsigned*>(ws + L.blk_counter);
   p.block_idx = block_idx;
   p.err = reinterpret_cast<int*>(ws + L.err);
+  p.fuse_tokens = 0;
 
   if (use_simt()) {
     const size_t smem = (size_t)p.group * 2 * s.qk_dim * 4 + (size_t)nb * 4 + sizeof(TopkScratch) + 16;
@@ -349,13 +389,8 @@ tls_status select_blocks_impl(const tls_shape& s, const void* q, const void* met
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(TLS_ERR_CUDA, "select_blocks: cuTensorMapEncodeTiled failed (%d)", (int)r);
 
-  const int g = p.group;
-  if (g <= 16) return launch_tc<16>(tmap, p, rows, stream);
-  if (g <= 32) return launch_tc<32>(tmap, p, rows, stream);
-  if (g <= 64) return launch_tc<64>(tmap, p, rows, stream);
-  if (g <= 128) return launch_tc<128>(tmap, p, rows, stream);
-  if (g <= 256) return launch_tc<256>(tmap, p, rows, stream);
-  return fail(TLS_ERR_UNSUPPORTED, "select_blocks: group size %d > 256", g);
+  (void)fuse;  // level 2 runs in its own cluster kernel: a single CTA per row is too narrow for it
+  return launch_tc_group<0>(tmap, p, rows, stream);
 }
 
 }  // namespace tls

@@ -12,30 +12,13 @@
 
 #include <mutex>
 
+#include "attn_common.cuh"
 #include "device_common.cuh"
 #include "host_common.h"
 
 namespace tls {
 
-struct AttnParams {
-  const uint16_t* q;
-  const uint16_t* k;
-  const uint16_t* v;
-  int64_t k_stride, v_stride;
-  const int32_t* slot_of_block;
-  int bs, nb, n_slots;
-  int64_t ctx_len;
-  const int32_t* token_idx;
-  int k_sel;
-  int n_q_heads, n_kv_heads, group, dqk, dv;
-  float scale_log2;
-  int tokens_per_split, splits, head_groups;
-  float* partial;      // workspace [rows][G][splits][dv + 2]
-  unsigned* counters;  // workspace [rows * head_groups]
-  void* out;
-  int out_bf16;
-  float* lse;
-};
+
 
 template <int PK, int PV, int HG, int U>
 __global__ void __launch_bounds__(128) sparse_attn_kernel(AttnParams p) {
@@ -81,6 +64,7 @@ __global__ void __launch_bounds__(128) sparse_attn_kernel(AttnParams p) {
   const int t_begin = split * p.tokens_per_split;
   const int t_end = min(p.k_sel, t_begin + p.tokens_per_split);
   const int32_t* tix = p.token_idx + (int64_t)row * p.k_sel;
+  grid_dependency_wait();  // token lists come from the preceding kernel
 
   for (int base = t_begin; base < t_end; base += 8 * U) {
     uint4 kw[U][PK], vw[U][PV];
@@ -222,26 +206,7 @@ __global__ void __launch_bounds__(128) sparse_attn_kernel(AttnParams p) {
   if (!last) return;
   __threadfence();
 
-  // merge the splits of heads h0 .. h0+nh-1 and write the outputs
-  for (int idx = tid; idx < nh * dv; idx += 128) {
-    const int hh = idx / dv, e = idx % dv;
-    const float* pp = p.partial + ((int64_t)row * g + h0 + hh) * p.splits * (dv + 2);
-    float M = -INFINITY;
-    for (int s = 0; s < p.splits; ++s) M = fmaxf(M, __ldcg(pp + (int64_t)s * (dv + 2)));
-    float L = 0.0f, A = 0.0f;
-    for (int s = 0; s < p.splits; ++s) {
-      const float ms = __ldcg(pp + (int64_t)s * (dv + 2));
-      if (ms == -INFINITY) continue;
-      const float f = exp2f(ms - M);
-      L += f * __ldcg(pp + (int64_t)s * (dv + 2) + 1);
-      A += f * __ldcg(pp + (int64_t)s * (dv + 2) + 2 + e);
-    }
-    const float o = A / L;
-    const int64_t oh = (int64_t)b * p.n_q_heads + kvh * g + h0 + hh;
-    if (p.out_bf16) reinterpret_cast<uint16_t*>(p.out)[oh * dv + e] = f32_to_bf16_rn(o);
-    else reinterpret_cast<float*>(p.out)[oh * dv + e] = o;
-    if (e == 0 && p.lse != nullptr) p.lse[oh] = (M + log2f(L)) * 0.69314718055994531f;
-  }
+  merge_splits(p, row, b, kvh, h0, nh, p.splits, red, 16 * HG + 8 * HG * dv);
 }
 
 template <int PK, int PV, int HG>
@@ -286,7 +251,14 @@ tls_status sparse_attn_impl(const tls_shape& s, const void* q, const tls_kv_view
   p.out = out;
   p.out_bf16 = out_dtype == TLS_OUT_BF16;
   p.lse = lse;
+  p.heads_per_cta = L.heads_per_cta;
+  p.tiles_per_pair = L.tiles_per_pair;
+  p.n_items = L.n_items;
+  p.n_ctas = L.n_ctas;
+  p.err = reinterpret_cast<int*>(ws + L.err);
   const int rows = rows_of(s);
+  if (attn_mma_supported(s)) return launch_attn_mma(p, stream);
+  if (attn_tc_supported(s)) return launch_attn_tc(p, rows, stream);
   const int pk = (s.qk_dim + 127) / 128, pv = (s.v_dim + 127) / 128;
   const int hg = L.heads_per_cta;
   if (pk == 1 && pv == 1) {
@@ -306,10 +278,13 @@ tls_status sparse_attn_impl(const tls_shape& s, const void* q, const tls_kv_view
               s.qk_dim, s.v_dim, hg);
 }
 
-// Heads per CTA for the attention kernel: the register budget allows 8 heads
-// at 128-wide rows, 4 at 256 and 2 above.
+// Heads per CTA for the attention kernel.  The tensor-core kernel takes up to
+// 64 heads (its TMEM and shared-memory budget); for the CUDA-core kernel the
+// register budget allows 8 heads at 128-wide rows, 4 at 256 and 2 above.
 int attn_heads_per_cta(const tls_shape& s) {
   const int g = group_of(s);
+  if (attn_mma_supported(s)) return g;
+  if (attn_tc_supported(s)) return g < 64 ? g : 64;
   const int pk = (s.qk_dim + 127) / 128, pv = (s.v_dim + 127) / 128;
   int cap = (pk == 1 && pv == 1) ? 8 : (pk <= 2 && pv <= 2) ? 4 : 2;
   int hg = 1;

@@ -1,0 +1,389 @@
+// Attention over the chosen tokens for small head groups (G <= 16) with
+// 128-wide K and V rows (AsyncTLS, Italian summary 2.A.2: attention runs on
+// the selected tokens only).
+//
+// At G <= 16 the gather does ~G flop per byte, so the kernel is HBM-bound; the
+// design follows the bandwidth: persistent CTAs (two per SM) over contiguous
+// ranges of 16-token chunks, every warp streaming its own chunks through a
+// 3-stage cp.async ring with no CTA-wide barrier in the steady state.  The
+// dot products run on the tensor cores through warp-level mma.sync
+// (m16n8k16, bf16 -> fp32), whose results stay in registers:
+//   S  = Q . K^T   A = q of the group's heads (rows >= G are zero), B = K rows
+//                  via ldmatrix from a 128B-swizzled stage
+//   softmax        online per head in fp32 registers, base 2
+//   O += P . V     A = P from the S accumulators, split into bf16 hi + lo
+//                  parts (two MMAs: P keeps ~16 significant bits), B = V rows
+//                  via ldmatrix.trans
+// At the end of each (row) segment of its range the CTA folds its warps in
+// shared memory and writes (m, l, O) to the split workspace; the last CTA to
+// finish a row merges the splits by log-sum-exp (attn_common.cuh).
+
+#include "attn_common.cuh"
+#include "device_common.cuh"
+#include "host_common.h"
+
+namespace tls {
+
+constexpr int kMmaWarps = 4;
+constexpr int kChunk = 16;           // tokens per chunk
+constexpr int kChunkBytes = 8192;    // K (4 KB) + V (4 KB) of 16 tokens
+
+// two floats -> bf16x2 (round to nearest even); `a` goes to the low half
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+  return r;
+}
+__device__ __forceinline__ float bf16_lo_f(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi_f(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// 2^x with the hardware approximation (relative error ~2^-22, far below the
+// 2e-3 output tolerance); 2^-inf = 0
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// byte offset of 16-byte unit c (0..15) of token row r (0..15) inside a 4 KB
+// tile of 256-byte rows; the low 3 bits of c are XORed with r so that the 8
+// rows an ldmatrix reads hit 8 different bank groups
+__device__ __forceinline__ uint32_t tile_off(int r, int c) {
+  return (uint32_t)(r * 256 + (((c & 8) | ((c & 7) ^ (r & 7))) << 4));
+}
+
+struct MmaLayout {
+  int off_comb, off_stat, bytes;
+};
+// ring stages per warp: 3 (two chunks in flight while one is computed), so
+// that two CTAs (eight warps) fit on an SM: instruction latency, not memory
+// depth, is what limits a warp here
+__host__ __device__ constexpr int mma_stages(int g) { return 3; }
+__host__ __device__ inline MmaLayout mma_layout(int g) {
+  MmaLayout L;
+  L.off_comb = kMmaWarps * mma_stages(g) * kChunkBytes;    // [warp][h][128] fp32
+  L.off_stat = L.off_comb + kMmaWarps * g * 128 * 4;        // [warp][h] m, then l
+  L.bytes = L.off_stat + 2 * kMmaWarps * 16 * 4 + 16;
+  return L;
+}
+
+template <int NS>
+__global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_kernel(AttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  const int g = p.group;
+  const MmaLayout L = mma_layout(g);
+  float* comb = reinterpret_cast<float*>(sm + L.off_comb);
+  float* cm = reinterpret_cast<float*>(sm + L.off_stat);
+  float* cl = cm + kMmaWarps * 16;
+  __shared__ int s_last;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gq = lane >> 2, tq = lane & 3;  // mma fragment coordinates
+  const int CPR = p.tiles_per_pair;         // chunks per row
+  const int64_t C = p.n_items;
+  const int64_t cta = blockIdx.x;
+  const int64_t c_lo = cta * C / p.n_ctas, c_hi = (cta + 1) * C / p.n_ctas;
+  uint8_t* ring = sm + warp * NS * kChunkBytes;
+  const uint32_t ring_s = smem_u32(ring);
+
+  // this warp's stream: chunks c_lo + warp + 4i
+  const int64_t x0 = c_lo + warp;
+  const int n_mine = x0 < c_hi ? (int)((c_hi - 1 - x0) / kMmaWarps + 1) : 0;
+
+  // raw token index of entry (lane & 15) of chunk x, or -1
+  auto load_tok = [&](int i) -> int {
+    if (i >= n_mine) return -1;
+    const int64_t x = x0 + (int64_t)kMmaWarps * i;
+    const int row = (int)(x / CPR);
+    const int t = (int)(x % CPR) * kChunk + (lane & 15);
+    if (t >= p.k_sel) return -1;
+    return __ldg(p.token_idx + (int64_t)row * p.k_sel + t);
+  };
+  // cp.async of the K and V rows of chunk i (its raw token indices in `tok`) into stage st
+  auto issue = [&](int i, int tok, int st) {
+    if (i < n_mine) {
+      const int row = (int)((x0 + (int64_t)kMmaWarps * i) / CPR);
+      int64_t rid = -1;
+      if (tok >= 0) {
+        const int64_t tk = min(max((int64_t)tok, (int64_t)0), p.ctx_len - 1);
+        if (p.slot_of_block != nullptr) {
+          const int64_t slot =
+              min(max(__ldg(p.slot_of_block + (int64_t)row * p.nb + tk / p.bs), 0), p.n_slots - 1);
+          rid = slot * p.bs + tk % p.bs;
+        } else {
+          rid = (int64_t)row * p.ctx_len + tk;
+        }
+      }
+      const uint32_t kb = ring_s + st * kChunkBytes, vb = kb + 4096;
+      const int c = lane & 15;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int r = (lane >> 4) + 2 * j;
+        const int64_t rr = __shfl_sync(0xffffffffu, rid, r);
+        const bool v = rr >= 0;
+        const uint32_t off = tile_off(r, c);
+        cp_async16(kb + off, p.k + (v ? rr * p.k_stride : 0) + c * 8, v ? 16u : 0u);
+        cp_async16(vb + off, p.v + (v ? rr * p.v_stride : 0) + c * 8, v ? 16u : 0u);
+      }
+    }
+    cp_async_commit();
+  };
+
+  // Q fragments (A operand) of the current row, 8 k-steps
+  uint32_t qa[8][4];
+  float o[16][4];
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f;  // rows gq and gq + 8
+
+  grid_launch_dependents();
+  grid_dependency_wait();  // token lists come from the preceding kernel
+
+  // prologue: stages 0 .. S-2; token indices one chunk further ahead
+  int tok_ahead[NS];
+#pragma unroll
+  for (int s = 0; s < NS; ++s) tok_ahead[s] = load_tok(s);
+#pragma unroll
+  for (int s = 0; s < NS - 1; ++s) issue(s, tok_ahead[s], s);
+  int tok_next = tok_ahead[NS - 1];  // for chunk S-1
+
+  const int row_first = (int)(c_lo / CPR);
+  const int row_last = (int)((c_hi - 1) / CPR);
+  int i = 0;  // position in this warp's stream
+  for (int row = row_first; row <= row_last; ++row) {
+    const int b = row / p.n_kv_heads, kvh = row % p.n_kv_heads;
+    // this row's chunks inside the CTA range
+    const int64_t seg_end = min(c_hi, (int64_t)(row + 1) * CPR);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const int d0 = ks * 16 + 2 * tq;
+      const uint16_t* q0 = p.q + ((int64_t)b * p.n_q_heads + kvh * g + gq) * p.dqk;
+      const uint16_t* q8 = q0 + (int64_t)8 * p.dqk;
+      qa[ks][0] = gq < g ? *reinterpret_cast<const uint32_t*>(q0 + d0) : 0u;
+      qa[ks][1] = gq + 8 < g ? *reinterpret_cast<const uint32_t*>(q8 + d0) : 0u;
+      qa[ks][2] = gq < g ? *reinterpret_cast<const uint32_t*>(q0 + d0 + 8) : 0u;
+      qa[ks][3] = gq + 8 < g ? *reinterpret_cast<const uint32_t*>(q8 + d0 + 8) : 0u;
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.0f;
+    m0 = m1 = -INFINITY;
+    l0 = l1 = 0.0f;
+
+    for (; i < n_mine && x0 + (int64_t)kMmaWarps * i < seg_end; ++i) {
+      // keep S-1 chunks in flight; indices run one chunk further ahead
+      const int tok_after = load_tok(i + NS);
+      issue(i + NS - 1, tok_next, (i + NS - 1) % NS);
+      tok_next = tok_after;
+      cp_async_wait<NS - 1>();
+      __syncwarp();
+
+      const int64_t x = x0 + (int64_t)kMmaWarps * i;
+      const int t_base = (int)(x % CPR) * kChunk;
+      const uint32_t kb = ring_s + (i % NS) * kChunkBytes, vb = kb + 4096;
+
+      // S = Q . K^T for 16 tokens (two n-tiles of 8)
+      float s[2][4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.0f;
+#pragma unroll
+        for (int ks = 0; ks < 8; ks += 2) {
+          // matrices: (k-step ks, units 2ks, 2ks+1), (ks+1, units 2ks+2, 2ks+3)
+          const int mtx = lane >> 3;
+          const uint32_t addr = kb + tile_off(nt * 8 + (lane & 7), ks * 2 + mtx);
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(addr, b0, b1, b2, b3);
+          mma_bf16_16816(s[nt], qa[ks], b0, b1);
+          mma_bf16_16816(s[nt], qa[ks + 1], b2, b3);
+        }
+      }
+      // scale (and mask the tail of the list), online softmax
+      // (rows gq: elements 0,1; rows gq+8: elements 2,3)
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s[nt][e] *= p.scale_log2;
+      if (t_base + kChunk > p.k_sel) {
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (t_base + nt * 8 + 2 * tq + (e & 1) >= p.k_sel) s[nt][e] = -INFINITY;
+      }
+      float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
+      float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+      const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+      // the O rescale is skipped (warp-uniformly) when no row maximum moved
+      if (!__all_sync(0xffffffffu, n0 == m0 && n1 == m1)) {
+        const float c0 = fast_exp2(m0 - n0), c1 = fast_exp2(m1 - n1);  // 0 on the first chunk
+        l0 *= c0;
+        l1 *= c1;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          o[j][0] *= c0;
+          o[j][1] *= c0;
+          o[j][2] *= c1;
+          o[j][3] *= c1;
+        }
+        m0 = n0;
+        m1 = n1;
+      }
+      float pr[2][4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) pr[nt][e] = fast_exp2(s[nt][e] - (e < 2 ? n0 : n1));
+      l0 += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
+      l1 += (pr[0][2] + pr[0][3]) + (pr[1][2] + pr[1][3]);
+      // P as the A operand (k = the 16 tokens), hi and lo parts
+      uint32_t ph[4], pl[4];
+      {
+        const float a[4][2] = {{pr[0][0], pr[0][1]}, {pr[0][2], pr[0][3]}, {pr[1][0], pr[1][1]}, {pr[1][2], pr[1][3]}};
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          ph[r] = pack_bf16(a[r][0], a[r][1]);
+          pl[r] = pack_bf16(a[r][0] - bf16_lo_f(ph[r]), a[r][1] - bf16_hi_f(ph[r]));
+        }
+      }
+      // O += P . V over 16 n-tiles of 8 value columns
+#pragma unroll
+      for (int j = 0; j < 16; j += 2) {
+        // matrices: tokens 0-7 / 8-15 of unit j, then of unit j+1
+        const int mtx = lane >> 3;
+        const uint32_t addr = vb + tile_off((mtx & 1) * 8 + (lane & 7), j + (mtx >> 1));
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(addr, b0, b1, b2, b3);
+        mma_bf16_16816(o[j], ph, b0, b1);
+        mma_bf16_16816(o[j], pl, b0, b1);
+        mma_bf16_16816(o[j + 1], ph, b2, b3);
+        mma_bf16_16816(o[j + 1], pl, b2, b3);
+      }
+      __syncwarp();
+    }
+
+    // fold the warps of the CTA for this row
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    if (tq == 0) {
+      if (gq < g) {
+        cm[warp * 16 + gq] = m0;
+        cl[warp * 16 + gq] = l0;
+      }
+      if (gq + 8 < g) {
+        cm[warp * 16 + gq + 8] = m1;
+        cl[warp * 16 + gq + 8] = l1;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int d = j * 8 + 2 * tq;
+      if (gq < g) {
+        comb[(warp * g + gq) * 128 + d] = o[j][0];
+        comb[(warp * g + gq) * 128 + d + 1] = o[j][1];
+      }
+      if (gq + 8 < g) {
+        comb[(warp * g + gq + 8) * 128 + d] = o[j][2];
+        comb[(warp * g + gq + 8) * 128 + d + 1] = o[j][3];
+      }
+    }
+    __syncthreads();
+    const int64_t first = attn_owner((int64_t)row * CPR, C, p.n_ctas);
+    const int n_part = (int)(attn_owner((int64_t)row * CPR + CPR - 1, C, p.n_ctas) - first + 1);
+    const int slot = (int)(cta - first);
+    for (int idx = tid; idx < g * 130; idx += kMmaWarps * 32) {
+      const int h = idx / 130, e = idx % 130;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kMmaWarps; ++w) M = fmaxf(M, cm[w * 16 + h]);
+      float val = 0.0f;
+      if (e == 0) {
+        val = M;
+      } else if (M != -INFINITY) {
+#pragma unroll
+        for (int w = 0; w < kMmaWarps; ++w) {
+          const float mw = cm[w * 16 + h];
+          if (mw == -INFINITY) continue;
+          const float f = exp2f(mw - M);
+          val += f * (e == 1 ? cl[w * 16 + h] : comb[(w * g + h) * 128 + (e - 2)]);
+        }
+      }
+      p.partial[(((int64_t)row * g + h) * p.splits + slot) * 130 + e] = val;
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = atomicInc(&p.counters[row], (unsigned)(n_part - 1)) == (unsigned)(n_part - 1);
+    __syncthreads();
+    if (s_last) {
+      __threadfence();
+      merge_splits(p, row, b, kvh, 0, g, n_part, comb, kMmaWarps * g * 128);
+    }
+    __syncthreads();  // the fold area is rewritten for the next row
+  }
+  cp_async_wait<0>();
+}
+
+bool attn_mma_supported(const tls_shape& s) {
+  return s.qk_dim == 128 && s.v_dim == 128 && s.v_offset < 0 && group_of(s) <= 16;
+}
+
+// Work partition: chunks of 16 entries of every row's token list, contiguous
+// ranges over two CTAs per SM.  Returns the largest number of CTAs sharing a row.
+int attn_mma_plan(int rows, int k, int* chunks_per_row, int* n_items, int* n_ctas) {
+  const int CPR = (k + kChunk - 1) / kChunk;
+  const int64_t C = (int64_t)rows * CPR;
+  const int64_t want = 2 * (int64_t)kNumSMs;
+  const int64_t byw = (C + kMmaWarps - 1) / kMmaWarps;  // at least a chunk per warp
+  int64_t n = want < byw ? want : byw;
+  if (n > 63 * (int64_t)rows) n = 63 * (int64_t)rows;  // at most 64 splits per row
+  int max_part = 1;
+  for (int64_t r = 0; r < rows; ++r) {
+    const int64_t parts = attn_owner(r * CPR + CPR - 1, C, n) - attn_owner(r * CPR, C, n) + 1;
+    if (parts > max_part) max_part = (int)parts;
+  }
+  *chunks_per_row = CPR;
+  *n_items = (int)C;
+  *n_ctas = (int)n;
+  return max_part;
+}
+
+template <int NS>
+static tls_status launch_mma(const AttnParams& p, cudaStream_t stream) {
+  const MmaLayout L = mma_layout(p.group);
+  const size_t smem = 128 + (size_t)L.bytes;
+  cudaError_t e =
+      cudaFuncSetAttribute(sparse_attn_mma_kernel<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return cuda_check(e, "sparse_decode_attn: set smem attribute");
+  return cuda_check(launch_pdl(sparse_attn_mma_kernel<NS>, dim3(p.n_ctas), dim3(kMmaWarps * 32), smem, stream, p),
+                    "sparse_decode_attn: mma launch");
+}
+
+tls_status launch_attn_mma(const AttnParams& p, cudaStream_t stream) {
+  return launch_mma<3>(p, stream);
+}
+
+}  // namespace tls

@@ -20,6 +20,12 @@ __device__ __forceinline__ void report_error(int* err, int code, int where) {
   }
 }
 
+// Programmatic dependent launch: wait for the preceding kernel of the stream
+// (no-op when the launch carried no programmatic dependency), and let the
+// next kernel be scheduled early.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint64_t global_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
@@ -94,38 +100,83 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int* to
 // keys[0..n) (shared memory) hold float_key(score).  Selects the k largest
 // keys, ties broken towards the lower position, and writes
 // out[j] = map(position) for the selected positions in ascending order.
-// Radix select (four 8-bit digits, most significant first) finds the k-th
-// largest key tau and how many of the keys equal to tau to take; one
-// index-ordered scan then marks the selection and a second one compacts it.
+//
+// 1. The smallest and largest key bound the scores.  If they are finite and
+//    differ, one pass bins every key by value into 256 equal-width bins over
+//    [min, max] (a monotone map, so bins never reorder keys) and finds the
+//    bin that holds the k-th largest key.  Float keys are log-scaled, so this
+//    splits a few-octave range far better than the top bits of the key.
+// 2. The keys of that bin are compacted (warp-aggregated) and the exact
+//    threshold tau and the number of keys equal to tau to take are found
+//    among them: by one warp ranking them pairwise when they are few, else by
+//    radix passes (8 bits at a time) over the compacted keys, or over all
+//    keys if they do not fit.
+// 3. One index-ordered scan marks the selection and a second one compacts it.
 // ----------------------------------------------------------------------------
+constexpr int kTopkCand = 512;
 struct TopkScratch {
   int hist[256];
   int scan[33];
-  uint32_t prefix;
-  int need;  // how many more keys must be taken at the current prefix
+  uint32_t wlo[32], whi[32];
+  uint32_t prefix, mask;
+  int need;   // how many more keys must be taken at the current prefix
+  int ncand;  // keys still in contention, compacted into cand[]
+  uint32_t lo, hi;
+  uint32_t cand[kTopkCand];
 };
+
+__device__ __forceinline__ float key_float(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
 
 template <int NT, typename MapFn>
 __device__ void cta_topk_ascending(const uint32_t* keys, int n, int k, int* out, TopkScratch& sm,
                                    MapFn map) {
-  const int tid = threadIdx.x;
-  if (tid == 0) {
-    sm.prefix = 0;
-    sm.need = k;
-  }
-  uint32_t mask = 0;
-#pragma unroll 1
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = tid; i < 256; i += NT) sm.hist[i] = 0;
-    __syncthreads();
-    const uint32_t prefix = sm.prefix;
+  constexpr int NW = NT / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // smallest and largest key
+  {
+    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
     for (int i = tid; i < n; i += NT) {
-      uint32_t key = keys[i];
-      if ((key & mask) == prefix) atomicAdd(&sm.hist[(key >> shift) & 255u], 1);
+      const uint32_t key = keys[i];
+      lo = min(lo, key);
+      hi = max(hi, key);
+    }
+    lo = __reduce_min_sync(0xffffffffu, lo);
+    hi = __reduce_max_sync(0xffffffffu, hi);
+    if (lane == 0) {
+      sm.wlo[warp] = lo;
+      sm.whi[warp] = hi;
     }
     __syncthreads();
+    if (tid == 0) {
+      for (int w = 1; w < NW; ++w) {
+        lo = min(lo, sm.wlo[w]);
+        hi = max(hi, sm.whi[w]);
+      }
+      const uint32_t diff = lo ^ hi;
+      const uint32_t undecided = diff == 0 ? 0u : (0xFFFFFFFFu >> __clz(diff));
+      sm.mask = ~undecided;
+      sm.prefix = lo & ~undecided;
+      sm.need = k;
+      sm.lo = lo;
+      sm.hi = hi;
+      sm.ncand = -1;  // no compacted set yet
+    }
+    __syncthreads();
+  }
+
+  // 1. value bins over [min, max]
+  const float fmin = key_float(sm.lo), fmax = key_float(sm.hi);
+  const float span = fmax - fmin;
+  if (sm.lo != sm.hi && isfinite(fmin) && isfinite(fmax) && isfinite(span) && span > 0.0f) {
+    const float inv = 256.0f / span;
+    for (int i = tid; i < 256; i += NT) sm.hist[i] = 0;
+    __syncthreads();
+    // value bins are spread over the range, so plain shared atomics rarely collide
+    for (int i = tid; i < n; i += NT) atomicAdd(&sm.hist[min(255, (int)((key_float(keys[i]) - fmin) * inv))], 1);
+    __syncthreads();
     if (tid < 32) {
-      // lane L owns digits [248 - 8L, 255 - 8L] (lane 0 holds the largest)
       int local[8];
       int s = 0;
 #pragma unroll
@@ -136,52 +187,167 @@ __device__ void cta_topk_ascending(const uint32_t* keys, int n, int k, int* out,
       int incl = s;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        int y = __shfl_up_sync(0xffffffffu, incl, o);
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (tid >= o) incl += y;
+      }
+      int above = incl - s;
+      if (above < k && incl >= k) {
+        int d = 0;
+        for (; d < 8; ++d) {
+          if (above + local[d] >= k) break;
+          above += local[d];
+        }
+        sm.hist[0] = 255 - (tid * 8 + d);  // the threshold bin (hist is not read again)
+        sm.need = k - above;
+      }
+    }
+    __syncthreads();
+    const int tbin = sm.hist[0];
+    // 2. compact the keys of the threshold bin
+    if (tid == 0) sm.ncand = 0;
+    __syncthreads();
+    for (int base = 0; base < n; base += NT) {
+      const int i = base + tid;
+      const uint32_t key = i < n ? keys[i] : 0u;
+      const bool hit = i < n && min(255, (int)((key_float(key) - fmin) * inv)) == tbin;
+      const unsigned bal = __ballot_sync(0xffffffffu, hit);
+      int slot0 = 0;
+      if (lane == 0 && bal != 0u) slot0 = atomicAdd(&sm.ncand, __popc(bal));
+      slot0 = __shfl_sync(0xffffffffu, slot0, 0);
+      if (hit) {
+        const int slot = slot0 + __popc(bal & ((1u << lane) - 1u));
+        if (slot < kTopkCand) sm.cand[slot] = key;
+      }
+    }
+    __syncthreads();
+    if (sm.ncand <= 128) {
+      // few keys: warp 0 ranks them pairwise (four per lane)
+      if (tid < 32) {
+        const int nc = sm.ncand, need = sm.need;
+        uint32_t mine[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) mine[j] = lane + 32 * j < nc ? sm.cand[lane + 32 * j] : 0u;
+        int gt[4] = {0, 0, 0, 0}, eq[4] = {0, 0, 0, 0};
+        for (int c = 0; c < nc; ++c) {
+          const uint32_t other = sm.cand[c];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            gt[j] += other > mine[j];
+            eq[j] += other == mine[j];
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (lane + 32 * j < nc && gt[j] < need && need <= gt[j] + eq[j]) {
+            sm.prefix = mine[j];  // every lane that holds tau writes the same values
+            sm.need = need - gt[j];
+          }
+      }
+      __syncthreads();
+      sm.mask = 0xFFFFFFFFu;  // decided (read only after the next barrier)
+    }
+  }
+
+  // 3. radix passes for whatever is still undecided
+  __syncthreads();
+  const bool ranked = sm.ncand >= 0 && sm.ncand <= 128;
+  const uint32_t* src = keys;
+  int nsrc = n;
+  if (!ranked && sm.ncand > 0 && sm.ncand <= kTopkCand) {
+    // restart the radix select inside the compacted bin
+    src = sm.cand;
+    nsrc = sm.ncand;
+  }
+  if (!ranked) {
+    if (tid == 0) {
+      // over all keys the common prefix of min and max is skipped; inside a
+      // compacted bin all 32 bits are decided (sm.need already counts there)
+      uint32_t lo = 0u, hi = 0xFFFFFFFFu;
+      if (src == keys) {
+        lo = sm.lo;
+        hi = sm.hi;
+        sm.need = k;
+      }
+      const uint32_t diff = lo ^ hi;
+      const uint32_t undecided = diff == 0 ? 0u : (0xFFFFFFFFu >> __clz(diff));
+      sm.mask = ~undecided;
+      sm.prefix = lo & ~undecided;
+    }
+    __syncthreads();
+  }
+  int top = ranked ? -1 : 31 - __clz(~sm.mask);  // highest undecided bit, -1 if none (clz(0) = 32)
+#pragma unroll 1
+  while (top >= 0) {
+    const int shift = top >= 7 ? top - 7 : 0;
+    const int width = top - shift + 1;
+    const uint32_t dmask = (1u << width) - 1u;
+    for (int i = tid; i < 256; i += NT) sm.hist[i] = 0;
+    __syncthreads();
+    const uint32_t prefix = sm.prefix, mask = sm.mask;
+    for (int base = 0; base < nsrc; base += NT) {
+      const int i = base + tid;
+      uint32_t key = 0;
+      bool valid = false;
+      if (i < nsrc) {
+        key = src[i];
+        valid = (key & mask) == prefix;
+      }
+      const uint32_t d = valid ? ((key >> shift) & dmask) : 0xFFFFFFFFu;
+      const unsigned peers = __match_any_sync(0xffffffffu, d);
+      if (valid && lane == __ffs(peers) - 1) atomicAdd(&sm.hist[d], __popc(peers));
+    }
+    __syncthreads();
+    if (tid < 32) {
+      int local[8];
+      int s = 0;
+#pragma unroll
+      for (int d = 0; d < 8; ++d) {
+        local[d] = sm.hist[255 - (tid * 8 + d)];
+        s += local[d];
+      }
+      int incl = s;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
         if (tid >= o) incl += y;
       }
       const int need = sm.need;
-      int above = incl - s;  // keys in digits larger than this lane's range
-      bool mine = (above < need) && (incl >= need);
-      unsigned ballot = __ballot_sync(0xffffffffu, mine);
-      if (mine) {
+      int above = incl - s;
+      if (above < need && incl >= need) {
         int d = 0;
         for (; d < 8; ++d) {
           if (above + local[d] >= need) break;
           above += local[d];
         }
-        uint32_t digit = 255u - (uint32_t)(tid * 8 + d);
+        const uint32_t digit = 255u - (uint32_t)(tid * 8 + d);
         sm.prefix = prefix | (digit << shift);
+        sm.mask = mask | (dmask << shift);
         sm.need = need - above;
       }
-      (void)ballot;
     }
-    mask |= 255u << shift;
     __syncthreads();
+    top = shift - 1;
   }
   const uint32_t tau = sm.prefix;
   const int take_eq = sm.need;  // keys equal to tau to take, lowest positions first
 
   // contiguous chunk per thread keeps the scans in position order
   const int per = (n + NT - 1) / NT;
-  const int lo = min(n, tid * per), hi = min(n, lo + per);
-  int eq = 0;
-  for (int i = lo; i < hi; ++i) eq += (keys[i] == tau);
-  int total;
-  int eq_before = block_exclusive_scan<NT>(eq, sm.scan, &total);
-  int sel = 0;
-  {
-    int e = eq_before;
-    for (int i = lo; i < hi; ++i) {
-      uint32_t key = keys[i];
-      if (key > tau) ++sel;
-      else if (key == tau) { if (e < take_eq) ++sel; ++e; }
-    }
+  const int lo_i = min(n, tid * per), hi_i = min(n, lo_i + per);
+  int eq = 0, gt = 0;
+  for (int i = lo_i; i < hi_i; ++i) {
+    const uint32_t key = keys[i];
+    eq += key == tau;
+    gt += key > tau;
   }
-  int pos = block_exclusive_scan<NT>(sel, sm.scan, &total);
+  int total;
+  const int eq_before = block_exclusive_scan<NT>(eq, sm.scan, &total);
+  const int take_here = min(eq, max(0, take_eq - eq_before));
+  int pos = block_exclusive_scan<NT>(gt + take_here, sm.scan, &total);
   {
     int e = eq_before;
-    for (int i = lo; i < hi; ++i) {
-      uint32_t key = keys[i];
+    for (int i = lo_i; i < hi_i; ++i) {
+      const uint32_t key = keys[i];
       bool take = false;
       if (key > tau) take = true;
       else if (key == tau) { take = e < take_eq; ++e; }
@@ -281,13 +447,40 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
   return d;
 }
 
-// Instruction descriptor: kind::f16, bf16 x bf16 -> f32, both K-major.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
+// Shared-memory matrix descriptor for an MN-major operand in the 128-byte
+// swizzled canonical layout: atoms of 8 K-rows x 128 B (64 MN elements);
+// `lbo` = byte distance between atoms along MN, `sbo` = between 8-row K groups.
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// Instruction descriptor: kind::f16, bf16 x bf16 -> f32; K-major operands
+// unless a_mn / b_mn select MN-major.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn = false, bool b_mn = false) {
   return (1u << 4)                      // D format f32
          | (1u << 7)                    // A format bf16
          | (1u << 10)                   // B format bf16
+         | ((a_mn ? 1u : 0u) << 15)     // A major
+         | ((b_mn ? 1u : 0u) << 16)     // B major
          | ((uint32_t)(N >> 3) << 17)   // N / 8
          | ((uint32_t)(M >> 4) << 24);  // M / 16
+}
+
+// 16-byte asynchronous global -> shared copy (L2 only); src_bytes = 0 fills zeros.
+__device__ __forceinline__ void cp_async16(uint32_t saddr, const void* gptr, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(saddr), "l"(gptr), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 __device__ __forceinline__ void tc_mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
@@ -315,6 +508,20 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 32 lanes x 32 bit, 16 consecutive columns per thread (store).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
+      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
+      "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
+      "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15]))
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 }  // namespace tls

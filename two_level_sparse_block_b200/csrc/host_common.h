@@ -9,7 +9,7 @@
 #include <cstdio>
 #include <string>
 
-#include "../../include/tls.h"
+#include "tls.h"
 
 namespace tls {
 
@@ -50,11 +50,32 @@ struct WsLayout {
   int head_groups;     // attention CTAs along the heads of a group
   int heads_per_cta;
   int tokens_per_split;
+  int tiles_per_pair, n_items, n_ctas;  // tensor-core attention work partition
 };
 
 // Plans the attention launch and the workspace for (shape, K_b, k).
 tls_status plan_workspace(const tls_shape& s, int K_b, int k, WsLayout* out);
 
 constexpr int kNumSMs = 148;
+
+// Launches `kernel` with programmatic stream serialization: it may start while
+// the preceding kernel of the stream finishes, and must call
+// griddepcontrol.wait (grid_dependency_wait) before touching that kernel's
+// outputs.  Hides the launch gap between dependent kernels of one step.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
 
 }  // namespace tls

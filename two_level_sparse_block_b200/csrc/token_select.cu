@@ -9,57 +9,16 @@
 // scaled dots), writes the scores to the workspace, and the last CTA of each
 // row to finish runs the deterministic top-k over the row's scores.
 
+#include <cooperative_groups.h>
 #include <cstdlib>
 
 #include "device_common.cuh"
 #include "host_common.h"
+#include "token_common.cuh"
 
 namespace tls {
 
-struct TokenParams {
-  const uint16_t* q;
-  const int32_t* label_ch;
-  const uint8_t* codes;
-  const float* scales;
-  const int32_t* block_idx;
-  int n_q_heads, n_kv_heads, group, dqk, bs, nb;
-  int64_t ctx_len;
-  int K_b, k, n_cand, chunk;
-  float* tscore;        // workspace [rows, n_cand]
-  float* token_score;   // optional copy
-  unsigned* counters;   // workspace [rows]
-  int32_t* token_idx;   // [rows, k]
-};
 
-template <int R>
-__device__ __forceinline__ void load_codes(const uint8_t* p, float (&c)[R]) {
-  uint32_t w[(R + 7) / 8];
-  if constexpr (R == 2) {
-    w[0] = p[0];
-  } else if constexpr (R == 4) {
-    w[0] = *reinterpret_cast<const uint16_t*>(p);
-  } else if constexpr (R == 8) {
-    w[0] = *reinterpret_cast<const uint32_t*>(p);
-  } else if constexpr (R == 16) {
-    const uint2 v = *reinterpret_cast<const uint2*>(p);
-    w[0] = v.x;
-    w[1] = v.y;
-  } else {
-#pragma unroll
-    for (int i = 0; i < R / 32; ++i) {
-      const uint4 v = reinterpret_cast<const uint4*>(p)[i];
-      w[4 * i + 0] = v.x;
-      w[4 * i + 1] = v.y;
-      w[4 * i + 2] = v.z;
-      w[4 * i + 3] = v.w;
-    }
-  }
-#pragma unroll
-  for (int r = 0; r < R; ++r) {
-    const int nib = (int)((w[r / 8] >> (4 * (r % 8))) & 15u);
-    c[r] = (float)((nib ^ 8) - 8);  // sign-extend the 4-bit two's complement code
-  }
-}
 
 template <int R, int NT>
 __global__ void __launch_bounds__(NT) token_select_kernel(TokenParams p) {
@@ -117,12 +76,66 @@ __global__ void __launch_bounds__(NT) token_select_kernel(TokenParams p) {
                          [bidx, bs](int i) { return bidx[i / bs] * bs + (i % bs); });
 }
 
-tls_status select_tokens_impl(const tls_shape& s, const void* q, const int32_t* label_ch, const uint8_t* codes,
-                              const float* scales, const int32_t* block_idx, int K_b, int k, int32_t* token_idx,
-                              float* token_score, uint8_t* ws, const WsLayout& L, cudaStream_t stream) {
-  constexpr int NT = 256;
-  const int rows = rows_of(s);
-  TokenParams p;
+// A cluster of kTokCluster CTAs per row when scoring is light: every CTA
+// scores a contiguous quarter of the candidates into its own shared memory;
+// after a cluster barrier the leader CTA gathers all keys through
+// distributed shared memory, a second barrier lets the others retire, and
+// the leader runs the top-k.
+constexpr int kTokCluster = 4;
+constexpr int kTokThreads = 256;
+
+template <int R>
+__global__ void __cluster_dims__(kTokCluster, 1, 1) __launch_bounds__(kTokThreads)
+    token_select_cluster_kernel(TokenParams p) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  extern __shared__ float sm[];
+  const int rank = (int)cluster.block_rank();
+  const int row = blockIdx.y;
+  const int per = (p.n_cand + kTokCluster - 1) / kTokCluster;
+  float* qlab = sm;                                                   // [G][R]
+  int32_t* bidx = reinterpret_cast<int32_t*>(sm + p.group * R);       // [K_b]
+  uint32_t* mine = reinterpret_cast<uint32_t*>(bidx + p.K_b);         // [per]
+  uint32_t* all = mine + per;                                         // [n_cand] (leader)
+  TopkScratch* ts = reinterpret_cast<TopkScratch*>(all + p.n_cand);
+  grid_launch_dependents();
+  load_qlab<R, kTokThreads>(p, row, qlab);
+  grid_dependency_wait();  // the block lists come from the preceding kernel
+  load_block_list<kTokThreads>(p, row, bidx);
+  __syncthreads();
+  const int c0 = min(p.n_cand, rank * per), c1 = min(p.n_cand, c0 + per);
+  score_candidates<R, kTokThreads>(p, row, qlab, bidx, c0, c1, mine);
+  cluster.sync();
+  if (rank == 0) {
+    // gather the other CTAs' keys through distributed shared memory, eight
+    // independent loads in flight per thread
+    for (int r = 0; r < kTokCluster; ++r) {
+      const uint32_t* __restrict__ src = cluster.map_shared_rank(mine, r);
+      const int b0 = min(p.n_cand, r * per), b1 = min(p.n_cand, b0 + per);
+      for (int i0 = 0; i0 < b1 - b0; i0 += 8 * kTokThreads) {
+        uint32_t v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int i = i0 + u * kTokThreads + (int)threadIdx.x;
+          v[u] = i < b1 - b0 ? src[i] : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int i = i0 + u * kTokThreads + (int)threadIdx.x;
+          if (i < b1 - b0) all[b0 + i] = v[u];
+        }
+      }
+    }
+  }
+  cluster.sync();  // the other CTAs' shared memory may be released after this
+  if (rank != 0) return;
+  cta_topk_ascending<kTokThreads>(all, p.n_cand, p.k, p.token_idx + (int64_t)row * p.k, *ts,
+                                  CandidateToken{bidx, p.bs});
+}
+
+void fill_token_params(TokenParams& p, const tls_shape& s, const void* q, const int32_t* label_ch,
+                       const uint8_t* codes, const float* scales, const int32_t* block_idx, int K_b, int k,
+                       int32_t* token_idx, float* token_score, uint8_t* ws, const WsLayout& L) {
   p.q = (const uint16_t*)q;
   p.label_ch = label_ch;
   p.codes = codes;
@@ -138,6 +151,23 @@ tls_status select_tokens_impl(const tls_shape& s, const void* q, const int32_t* 
   p.K_b = K_b;
   p.k = k;
   p.n_cand = K_b * s.block_size;
+  p.chunk = 0;
+  p.tscore = reinterpret_cast<float*>(ws + L.tscore);
+  p.token_score = token_score;
+  p.counters = reinterpret_cast<unsigned*>(ws + L.tok_counter);
+  p.token_idx = token_idx;
+}
+
+// `pdl`: the preceding kernel of the stream is this library's level-1 kernel,
+// which writes only the block lists (the one input the cluster kernel reads
+// after its dependency wait), so the launch may overlap its tail.
+tls_status select_tokens_impl(const tls_shape& s, const void* q, const int32_t* label_ch, const uint8_t* codes,
+                              const float* scales, const int32_t* block_idx, int K_b, int k, int32_t* token_idx,
+                              float* token_score, uint8_t* ws, const WsLayout& L, cudaStream_t stream, bool pdl) {
+  constexpr int NT = 256;
+  const int rows = rows_of(s);
+  TokenParams p;
+  fill_token_params(p, s, q, label_ch, codes, scales, block_idx, K_b, k, token_idx, token_score, ws, L);
   // enough CTAs for about two waves, at least one candidate per thread
   int chunks = (2 * kNumSMs + rows - 1) / rows;
   int chunk = (p.n_cand + chunks - 1) / chunks;
@@ -151,6 +181,33 @@ tls_status select_tokens_impl(const tls_shape& s, const void* q, const int32_t* 
   p.token_idx = token_idx;
 
   const size_t smem = (size_t)p.group * s.n_label * 4 + (size_t)p.n_cand * 4 + sizeof(TopkScratch) + 16;
+  if (token_stage_fits(p.group, s.n_label, p.n_cand)) {
+    const int per = (p.n_cand + kTokCluster - 1) / kTokCluster;
+    const size_t csmem = ((size_t)p.group * s.n_label + K_b + per + p.n_cand) * 4 + sizeof(TopkScratch) + 16;
+    const dim3 cgrid(kTokCluster, (unsigned)rows);
+    switch (s.n_label) {
+#define TLS_TC_CASE(RR)                                                                                     \
+  case RR: {                                                                                                \
+    cudaError_t e = cudaFuncSetAttribute(token_select_cluster_kernel<RR>,                                   \
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)csmem);          \
+    if (e != cudaSuccess) return cuda_check(e, "select_tokens: set smem attribute");                        \
+    if (pdl)                                                                                                \
+      return cuda_check(launch_pdl(token_select_cluster_kernel<RR>, cgrid, dim3(kTokThreads), csmem, stream, p), \
+                        "select_tokens launch");                                                             \
+    token_select_cluster_kernel<RR><<<cgrid, kTokThreads, csmem, stream>>>(p);                              \
+    return launch_check("select_tokens launch");                                                             \
+  }
+      TLS_TC_CASE(2)
+      TLS_TC_CASE(4)
+      TLS_TC_CASE(8)
+      TLS_TC_CASE(16)
+      TLS_TC_CASE(32)
+      TLS_TC_CASE(64)
+#undef TLS_TC_CASE
+      default:
+        return fail(TLS_ERR_UNSUPPORTED, "select_tokens: n_label %d not built (2,4,8,16,32,64)", s.n_label);
+    }
+  }
   dim3 grid((unsigned)chunks, (unsigned)rows);
   switch (s.n_label) {
 #define TLS_TS_CASE(RR)                                                                                     \

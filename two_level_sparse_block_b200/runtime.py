@@ -82,13 +82,18 @@ class DecodeState:
                               self.block_idx if block_idx is None else block_idx, self.K_b, self.k, self.token_idx,
                               self.token_score if keep_scores else None, self.ws, self.ws_bytes, stream)
 
+    def select(self, q=None, stream=None):
+        """Levels 1 and 2 (tls_select)."""
+        tls.tls_select(self.shape, self.q if q is None else q, self.meta, self.label_ch, self.codes, self.scales,
+                       self.K_b, self.k, self.block_idx, self.token_idx, self.ws, self.ws_bytes, stream)
+
     def attend(self, q=None, token_idx=None, kv=None, stream=None):
         tls.tls_sparse_decode_attn(self.shape, self.q if q is None else q, self.kv if kv is None else kv,
                                    self.token_idx if token_idx is None else token_idx, self.k, self.out_dtype,
                                    self.out, self.lse, self.ws, self.ws_bytes, stream)
 
     def step(self, q=None, stream=None):
-        """One synchronous decode step: three kernel launches."""
+        """One synchronous decode step (tls_select + attention)."""
         tls.tls_decode_step(self.shape, self.q if q is None else q, self.meta, self.label_ch, self.codes,
                             self.scales, self.kv, self.K_b, self.k, self.block_idx, self.token_idx, self.out_dtype,
                             self.out, self.lse, self.ws, self.ws_bytes, stream)

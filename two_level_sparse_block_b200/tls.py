@@ -73,6 +73,7 @@ _SIG = {
     "tls_select_tokens": (_I32, [_P, _P, _P, _P, _P, _P, _I32, _I32, _P, _P, _P, _SZ, _P]),
     "tls_sparse_decode_attn": (_I32, [_P, _P, _P, _P, _I32, _I32, _P, _P, _P, _SZ, _P]),
     "tls_sparse_decode_attn_noalloc": (_I32, [_P, _P, _P, _P, _I32, _I32, _P, _P, _P]),
+    "tls_select": (_I32, [_P, _P, _P, _P, _P, _P, _I32, _I32, _P, _P, _P, _SZ, _P]),
     "tls_decode_step": (_I32, [_P, _P, _P, _P, _P, _P, _P, _I32, _I32, _P, _P, _I32, _P, _P, _P, _SZ, _P]),
     "tls_block_cache_create": (_I32, [_P, _P, _P, _I64, _I64, _I32, _P, _P, _P, _P]),
     "tls_block_cache_destroy": (None, [_P]),
@@ -187,6 +188,12 @@ def tls_sparse_decode_attn_noalloc(shape, q, kv: KvView, token_idx, k, out_dtype
     _check(lib().tls_sparse_decode_attn_noalloc(ctypes.byref(shape), _ptr(q), ctypes.byref(kv), _ptr(token_idx), k,
                                                 out_dtype, _ptr(out), _ptr(lse), _stream(stream)),
            "tls_sparse_decode_attn_noalloc")
+
+
+def tls_select(shape, q, meta, label_ch, codes, scales, K_b, k, block_idx, token_idx, ws, ws_bytes, stream=None):
+    _check(lib().tls_select(ctypes.byref(shape), _ptr(q), _ptr(meta), _ptr(label_ch), _ptr(codes), _ptr(scales),
+                            K_b, k, _ptr(block_idx), _ptr(token_idx), _ptr(ws), ws_bytes, _stream(stream)),
+           "tls_select")
 
 
 def tls_decode_step(shape, q, meta, label_ch, codes, scales, kv: KvView, K_b, k, block_idx, token_idx, out_dtype,
