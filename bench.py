@@ -93,20 +93,31 @@ def load_peaks():
     return 6650.0, "fallback"
 
 
-def kernel_source_hash(name):
-    p = os.path.join(ROOT, "two_level_sparse_block_b200", "csrc", name)
-    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+# Sources compiled into each attention kernel: a recorded ncu traffic figure
+# holds only while all of them are unchanged.
+ATTN_SOURCES = {
+    "sparse_attn_mma_kernel": ("decode_attn_mma.cu", "attn_common.cuh", "device_common.cuh"),
+    "sparse_attn_tc_kernel": ("decode_attn_tc.cu", "attn_common.cuh", "device_common.cuh"),
+    "sparse_attn_kernel": ("decode_attn.cu", "attn_common.cuh", "device_common.cuh"),
+}
 
 
-def recorded_traffic(kernel_file, workload_name):
+def kernel_source_hash(files):
+    h = hashlib.sha256()
+    for name in files:
+        h.update(open(os.path.join(ROOT, "two_level_sparse_block_b200", "csrc", name), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload_name):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
     on the current source of the kernel; otherwise None."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
-    e = d.get(kernel_file, {}).get(workload_name)
-    if not e or e.get("source_sha256_16") != kernel_source_hash(kernel_file):
+    e = d.get(kernel, {}).get(workload_name)
+    if not e or e.get("source_sha256_16") != kernel_source_hash(ATTN_SOURCES[kernel]):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -366,6 +377,7 @@ def main():
     e2e_ms = float(t[0])
 
     ab = algorithmic_bytes(c)
+    attn_kernel = tls.tls_attn_kernel(st.shape)
     peak, peak_kind = load_peaks()
     att_avg_s = att_mean_ms / 1e3
     achieved = ab["attn"] / att_avg_s / 1e9
@@ -384,10 +396,10 @@ def main():
                      "sparse_decode_attn": 1e3 * statistics.mean(att_ms),
                      "note": "stages replayed as separate graphs (each pays its own launch); the step is one graph"},
         "step_hbm": {"algorithmic_bytes": ab["step"], "achieved_gbs": step_gbs, "frac_of_peak": step_gbs / peak},
-        "roofline": {"kernel": "sparse_attn_kernel (decode_attn.cu)", "bound": "hbm", "achieved": achieved,
+        "roofline": {"kernel": attn_kernel, "bound": "hbm", "achieved": achieved,
                      "peak": peak, "peak_source": f"hbm_gbs {peak_kind}", "unit": "GB/s", "frac": achieved / peak,
                      "algorithmic_bytes_per_launch": ab["attn"],
-                     "traffic": recorded_traffic("decode_attn.cu", c.name)},
+                     "traffic": recorded_traffic(attn_kernel, c.name)},
         "gpu_launches": launches_per_step(c) * args.steps,
         "e2e": {"value": world * c.batch / (e2e_ms / 1e3), "unit": "decode tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": int(st.q.numel() * 2), "d2h_bytes_per_step": int(st.out.numel() * st.out.element_size()),

@@ -99,6 +99,16 @@ TLS_API const char* tls_last_error(void);
 TLS_API int32_t tls_version(void);
 
 /*
+ * Name of the attention kernel tls_sparse_decode_attn launches for this
+ * shape: "sparse_attn_mma_kernel" (128-wide heads, at most 16 query heads per
+ * KV head), "sparse_attn_tc_kernel" (128-wide heads, wider groups) or
+ * "sparse_attn_kernel" (every other shape, e.g. the MLA latent cache).  A
+ * static string owned by the library; NULL if the shape is invalid
+ * (tls_last_error says why).  Host only, no device work.
+ */
+TLS_API const char* tls_attn_kernel(const tls_shape* shape);
+
+/*
  * Bytes of device workspace needed by tls_select_blocks, tls_select_tokens,
  * tls_sparse_decode_attn and tls_decode_step for this shape, K_b and k.
  * The workspace must be zero-filled once after allocation; every call that

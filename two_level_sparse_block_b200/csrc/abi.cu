@@ -155,6 +155,13 @@ extern "C" const char* tls_last_error(void) { return g_err; }
 
 extern "C" int32_t tls_version(void) { return 100; }
 
+extern "C" const char* tls_attn_kernel(const tls_shape* shape) {
+  if (check_shape(shape) != TLS_OK) return nullptr;
+  if (attn_mma_supported(*shape)) return "sparse_attn_mma_kernel";
+  if (attn_tc_supported(*shape)) return "sparse_attn_tc_kernel";
+  return "sparse_attn_kernel";
+}
+
 extern "C" size_t tls_workspace_bytes(const tls_shape* shape, int32_t K_b, int32_t k) {
   if (check_shape(shape) != TLS_OK) return 0;
   WsLayout L;

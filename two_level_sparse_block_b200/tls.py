@@ -65,6 +65,7 @@ _SZ = ctypes.c_size_t
 _SIG = {
     "tls_last_error": (ctypes.c_char_p, []),
     "tls_version": (_I32, []),
+    "tls_attn_kernel": (ctypes.c_char_p, [_P]),
     "tls_workspace_bytes": (_SZ, [_P, _I32, _I32]),
     "tls_workspace_error": (_I32, [_P, _I32, _P, _P]),
     "tls_build_block_meta": (_I32, [_P, _P, _I64, _I64, _I64, _P, _P]),
@@ -143,6 +144,14 @@ def tls_last_error() -> str:
 
 def tls_version() -> int:
     return lib().tls_version()
+
+
+def tls_attn_kernel(shape: Shape) -> str:
+    """Name of the attention kernel the dispatch launches for this shape."""
+    r = lib().tls_attn_kernel(ctypes.byref(shape))
+    if r is None:
+        _check(TLS_ERR_INVALID_ARG, "tls_attn_kernel")
+    return r.decode()
 
 
 def tls_workspace_bytes(shape: Shape, K_b: int, k: int) -> int:
