@@ -287,6 +287,34 @@ def test_exact_ties_follow_the_lower_index_rule():
             assert got["token_idx"][b, h].tolist() == r2["token_idx"].tolist()
 
 
+def test_crowded_threshold_takes_the_lowest_positions():
+    # every K row is one of two patterns, so the token scores take exactly two
+    # values; the k-th largest sits among ~half of the 1024 candidates, far more
+    # than the pairwise ranking takes, and ties must fall to the lowest positions
+    runtime, tls = _rt()
+    cfg = small("s_two_valued", batch=1, n_q_heads=4, n_kv_heads=2, ctx_len=2048, block_size=64, K_b=16, k=300,
+                n_label=16, seed=41)
+    rng = np.random.default_rng(41)
+    from synth import bf16_bits_from_f32
+    pat = rng.standard_normal((2, cfg.qk_dim)).astype(np.float32)
+    pick = rng.integers(0, 2, size=(1, 2, cfg.ctx_len))
+    K = bf16_bits_from_f32(pat[pick])
+    q = synth.gen_queries(cfg)
+    V = synth.gen_kv(cfg, q)[1]
+    lab = synth.gen_label_channels(cfg)
+    st = runtime.state_for_config(cfg, q, K, V, lab)
+    got = run_stages(st)
+    g = cfg.group
+    for h in range(2):
+        r2 = oracle.decode_row(q[0, h * g:(h + 1) * g], K[0, h], V[0, h], lab[h], cfg.block_size, cfg.K_b,
+                               cfg.k, cfg.softmax_scale, block_idx=got["block_idx"][0, h])
+        ts = np.asarray(r2["token_score"], dtype=np.float64)
+        vals = np.unique(ts)
+        tau = np.sort(ts)[::-1][cfg.k - 1]
+        assert vals.size == 2 and np.count_nonzero(ts == tau) > 128, "workload lost its construction"
+        assert got["token_idx"][0, h].tolist() == r2["token_idx"].tolist()
+
+
 @pytest.mark.parametrize("cfg", SMALL + [get_config("c1")], ids=lambda c: c.name)
 def test_fused_select_equals_the_two_level_calls(cfg):
     st, data = make_state(cfg)

@@ -110,6 +110,12 @@ __global__ void __launch_bounds__(128, 1)
     flags[0] = 0;
     flags[1] = 0;
     fence_barrier_init();
+  } else if (tid == 32) {
+    // what the epilogue and the row's top-K_b write: prefetching them now
+    // also warms their address translations during the metadata loads
+    prefetch_l2(p.agg + (int64_t)row * p.nb + mt * kBsTile);
+    prefetch_l2(p.counters + row);
+    prefetch_l2(p.block_idx + (int64_t)row * p.K_b);
   }
   if (warp == 0) tmem_alloc(tmem_slot, kCols);
   tc_fence_before();

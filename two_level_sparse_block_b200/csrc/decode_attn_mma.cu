@@ -156,6 +156,18 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_kernel(Attn
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f;  // rows gq and gq + 8
 
   grid_launch_dependents();
+  if (tid == 0 && c_lo < c_hi) {
+    // what the first row end writes (split partials, the row's ticket, the
+    // output and lse rows): prefetching them now also warms their address
+    // translations while the token lists are still being selected
+    const int r0 = (int)(c_lo / CPR);
+    const int64_t f0 = attn_owner((int64_t)r0 * CPR, C, p.n_ctas);
+    prefetch_l2(p.partial + (((int64_t)r0 * g) * p.splits + (cta - f0)) * 130);
+    prefetch_l2(p.counters + r0);
+    const int64_t oh = (int64_t)(r0 / p.n_kv_heads) * p.n_q_heads + (r0 % p.n_kv_heads) * g;
+    prefetch_l2(reinterpret_cast<const uint8_t*>(p.out) + oh * p.dv * (p.out_bf16 ? 2 : 4));
+    if (p.lse != nullptr) prefetch_l2(p.lse + oh);
+  }
   grid_dependency_wait();  // token lists come from the preceding kernel
 
   // prologue: stages 0 .. S-2; token indices one chunk further ahead

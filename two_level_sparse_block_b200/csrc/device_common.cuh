@@ -54,44 +54,18 @@ __device__ __forceinline__ uint16_t f32_to_bf16_rn(float x) {
 // Order-preserving map float -> uint32 (larger float -> larger key).
 // -0 is folded onto +0 and NaN onto -inf so that equal values tie.
 // ----------------------------------------------------------------------------
+// Prefetches the line at p into L2.  Issued early for a buffer a kernel
+// writes only at its end, it also brings the buffer's address translation
+// into the SM's TLBs while the kernel still waits for its inputs.
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 __device__ __forceinline__ uint32_t float_key(float f) {
   if (f != f) f = -INFINITY;
   if (f == 0.0f) f = 0.0f;
   uint32_t u = __float_as_uint(f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-// ----------------------------------------------------------------------------
-// Block-wide exclusive scan of one int per thread.  `scratch` holds >= 33 ints.
-// Returns the exclusive prefix; *total receives the sum over the block.
-// ----------------------------------------------------------------------------
-template <int NT>
-__device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int* total) {
-  constexpr int NW = NT / 32;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) scratch[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    int w = lane < NW ? scratch[lane] : 0;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      int y = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += y;
-    }
-    if (lane < NW) scratch[lane] = w;  // inclusive warp totals
-    if (lane == NW - 1) scratch[32] = w;
-  }
-  __syncthreads();
-  int before = (warp > 0 ? scratch[warp - 1] : 0) + x - v;
-  *total = scratch[32];
-  __syncthreads();
-  return before;
 }
 
 // ----------------------------------------------------------------------------
@@ -106,22 +80,31 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int* to
 //    [min, max] (a monotone map, so bins never reorder keys) and finds the
 //    bin that holds the k-th largest key.  Float keys are log-scaled, so this
 //    splits a few-octave range far better than the top bits of the key.
-// 2. The keys of that bin are compacted (warp-aggregated) and the exact
-//    threshold tau and the number of keys equal to tau to take are found
-//    among them: by one warp ranking them pairwise when they are few, else by
-//    radix passes (8 bits at a time) over the compacted keys, or over all
-//    keys if they do not fit.
-// 3. One index-ordered scan marks the selection and a second one compacts it.
+// 2. The keys of that bin are compacted and the exact threshold tau and the
+//    number of keys equal to tau to take are found among them: by ranking
+//    them pairwise when they are few, else by radix passes (8 bits at a time)
+//    over the compacted keys, or over all keys if they do not fit.
+// 3. Every warp owns a contiguous range of positions.  One ballot pass counts
+//    the keys above and equal to tau per warp; a second one hands out output
+//    slots in position order (ballot prefix counts inside a warp, the warps'
+//    counts before it across warps).
+//
+// The scans of steps 2 and 3 read the keys of four 32-key steps before they
+// vote, so a warp has four shared-memory loads in flight instead of one.
 // ----------------------------------------------------------------------------
 constexpr int kTopkCand = 512;
+constexpr int kTopkRankMax = 128;  // at most this many compacted keys are ranked pairwise
 struct TopkScratch {
   int hist[256];
-  int scan[33];
   uint32_t wlo[32], whi[32];
+  int wgt[32], weq[32];
   uint32_t prefix, mask;
   int need;   // how many more keys must be taken at the current prefix
   int ncand;  // keys still in contention, compacted into cand[]
+  int tbin;   // value bin of the k-th largest key
   uint32_t lo, hi;
+  uint32_t tau;  // threshold found by the pairwise ranking
+  int take;      // keys equal to tau to take, found by the pairwise ranking
   uint32_t cand[kTopkCand];
 };
 
@@ -129,14 +112,27 @@ __device__ __forceinline__ float key_float(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
+// 256 value bins of a (finite) key over [fmin, fmin + 256 / inv]
+__device__ __forceinline__ int topk_value_bin(uint32_t key, float fmin, float inv) {
+  return min(255, (int)((key_float(key) - fmin) * inv));
+}
+
 template <int NT, typename MapFn>
 __device__ void cta_topk_ascending(const uint32_t* keys, int n, int k, int* out, TopkScratch& sm,
                                    MapFn map) {
+  static_assert(NT % 32 == 0 && NT >= kTopkRankMax && NT <= 1024, "CTA size");
   constexpr int NW = NT / 32;
+  constexpr int U = 4;  // 32-key steps batched per warp iteration
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // smallest and largest key
+  const unsigned below = (1u << lane) - 1u;
+  // this warp's contiguous range of positions
+  const int per_w = ((n + NW - 1) / NW + 31) & ~31;
+  const int w_lo = min(n, warp * per_w), w_hi = min(n, w_lo + per_w);
+
+  // 0. smallest and largest key
   {
     uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+#pragma unroll 4
     for (int i = tid; i < n; i += NT) {
       const uint32_t key = keys[i];
       lo = min(lo, key);
@@ -169,12 +165,14 @@ __device__ void cta_topk_ascending(const uint32_t* keys, int n, int k, int* out,
   // 1. value bins over [min, max]
   const float fmin = key_float(sm.lo), fmax = key_float(sm.hi);
   const float span = fmax - fmin;
+  bool ranked = false;
   if (sm.lo != sm.hi && isfinite(fmin) && isfinite(fmax) && isfinite(span) && span > 0.0f) {
     const float inv = 256.0f / span;
     for (int i = tid; i < 256; i += NT) sm.hist[i] = 0;
     __syncthreads();
     // value bins are spread over the range, so plain shared atomics rarely collide
-    for (int i = tid; i < n; i += NT) atomicAdd(&sm.hist[min(255, (int)((key_float(keys[i]) - fmin) * inv))], 1);
+#pragma unroll 4
+    for (int i = tid; i < n; i += NT) atomicAdd(&sm.hist[topk_value_bin(keys[i], fmin, inv)], 1);
     __syncthreads();
     if (tid < 32) {
       int local[8];
@@ -197,68 +195,81 @@ __device__ void cta_topk_ascending(const uint32_t* keys, int n, int k, int* out,
           if (above + local[d] >= k) break;
           above += local[d];
         }
-        sm.hist[0] = 255 - (tid * 8 + d);  // the threshold bin (hist is not read again)
+        sm.tbin = 255 - (tid * 8 + d);
         sm.need = k - above;
       }
+      if (tid == 0) sm.ncand = 0;
     }
     __syncthreads();
-    const int tbin = sm.hist[0];
-    // 2. compact the keys of the threshold bin
-    if (tid == 0) sm.ncand = 0;
-    __syncthreads();
-    for (int base = 0; base < n; base += NT) {
-      const int i = base + tid;
-      const uint32_t key = i < n ? keys[i] : 0u;
-      const bool hit = i < n && min(255, (int)((key_float(key) - fmin) * inv)) == tbin;
-      const unsigned bal = __ballot_sync(0xffffffffu, hit);
-      int slot0 = 0;
-      if (lane == 0 && bal != 0u) slot0 = atomicAdd(&sm.ncand, __popc(bal));
-      slot0 = __shfl_sync(0xffffffffu, slot0, 0);
-      if (hit) {
-        const int slot = slot0 + __popc(bal & ((1u << lane) - 1u));
-        if (slot < kTopkCand) sm.cand[slot] = key;
+    const int tbin = sm.tbin;
+    // 2. compact the keys of the threshold bin (slot order is irrelevant)
+    for (int base = w_lo; base < w_hi; base += 32 * U) {
+      uint32_t kv[U];
+      unsigned bal[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int i = base + 32 * u + lane;
+        kv[u] = i < w_hi ? keys[i] : 0u;
       }
-    }
-    __syncthreads();
-    if (sm.ncand <= 128) {
-      // few keys: warp 0 ranks them pairwise (four per lane)
-      if (tid < 32) {
-        const int nc = sm.ncand, need = sm.need;
-        uint32_t mine[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) mine[j] = lane + 32 * j < nc ? sm.cand[lane + 32 * j] : 0u;
-        int gt[4] = {0, 0, 0, 0}, eq[4] = {0, 0, 0, 0};
-        for (int c = 0; c < nc; ++c) {
-          const uint32_t other = sm.cand[c];
+      for (int u = 0; u < U; ++u) {
+        const int i = base + 32 * u + lane;
+        bal[u] = __ballot_sync(0xffffffffu, i < w_hi && topk_value_bin(kv[u], fmin, inv) == tbin);
+      }
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            gt[j] += other > mine[j];
-            eq[j] += other == mine[j];
-          }
+      for (int u = 0; u < U; ++u) {
+        if (bal[u] == 0u) continue;  // warp-uniform
+        int slot0 = 0;
+        if (lane == 0) slot0 = atomicAdd(&sm.ncand, __popc(bal[u]));
+        slot0 = __shfl_sync(0xffffffffu, slot0, 0);
+        if ((bal[u] >> lane) & 1u) {
+          const int slot = slot0 + __popc(bal[u] & below);
+          if (slot < kTopkCand) sm.cand[slot] = kv[u];
         }
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if (lane + 32 * j < nc && gt[j] < need && need <= gt[j] + eq[j]) {
-            sm.prefix = mine[j];  // every lane that holds tau writes the same values
-            sm.need = need - gt[j];
-          }
       }
-      __syncthreads();
-      sm.mask = 0xFFFFFFFFu;  // decided (read only after the next barrier)
+    }
+    __syncthreads();
+    const int nc = sm.ncand;
+    if (nc <= kTopkRankMax) {
+      // few keys: thread t ranks compacted key t against all of them
+      ranked = true;
+      if (tid < kTopkRankMax) {
+        const int need = sm.need;
+        const uint32_t mine = tid < nc ? sm.cand[tid] : 0u;
+        int gt = 0, eq = 0, c = 0;
+        for (; c + 4 <= nc; c += 4) {
+          const uint32_t o0 = sm.cand[c], o1 = sm.cand[c + 1], o2 = sm.cand[c + 2], o3 = sm.cand[c + 3];
+          gt += (int)(o0 > mine) + (int)(o1 > mine) + (int)(o2 > mine) + (int)(o3 > mine);
+          eq += (int)(o0 == mine) + (int)(o1 == mine) + (int)(o2 == mine) + (int)(o3 == mine);
+        }
+        for (; c < nc; ++c) {
+          const uint32_t o = sm.cand[c];
+          gt += (int)(o > mine);
+          eq += (int)(o == mine);
+        }
+        if (tid < nc && gt < need && need <= gt + eq) {
+          sm.tau = mine;  // every thread that holds tau writes the same values
+          sm.take = need - gt;
+        }
+      }
     }
   }
 
-  // 3. radix passes for whatever is still undecided
+  // radix passes for whatever is still undecided
   __syncthreads();
-  const bool ranked = sm.ncand >= 0 && sm.ncand <= 128;
-  const uint32_t* src = keys;
-  int nsrc = n;
-  if (!ranked && sm.ncand > 0 && sm.ncand <= kTopkCand) {
-    // restart the radix select inside the compacted bin
-    src = sm.cand;
-    nsrc = sm.ncand;
-  }
-  if (!ranked) {
+  uint32_t tau;
+  int take_eq;  // keys equal to tau to take, lowest positions first
+  if (ranked) {
+    tau = sm.tau;
+    take_eq = sm.take;
+  } else {
+    const uint32_t* src = keys;
+    int nsrc = n;
+    if (sm.ncand > 0 && sm.ncand <= kTopkCand) {
+      // restart the radix select inside the compacted bin
+      src = sm.cand;
+      nsrc = sm.ncand;
+    }
     if (tid == 0) {
       // over all keys the common prefix of min and max is skipped; inside a
       // compacted bin all 32 bits are decided (sm.need already counts there)
@@ -274,84 +285,111 @@ __device__ void cta_topk_ascending(const uint32_t* keys, int n, int k, int* out,
       sm.prefix = lo & ~undecided;
     }
     __syncthreads();
-  }
-  int top = ranked ? -1 : 31 - __clz(~sm.mask);  // highest undecided bit, -1 if none (clz(0) = 32)
+    int top = 31 - __clz(~sm.mask);  // highest undecided bit, -1 if none (clz(0) = 32)
 #pragma unroll 1
-  while (top >= 0) {
-    const int shift = top >= 7 ? top - 7 : 0;
-    const int width = top - shift + 1;
-    const uint32_t dmask = (1u << width) - 1u;
-    for (int i = tid; i < 256; i += NT) sm.hist[i] = 0;
-    __syncthreads();
-    const uint32_t prefix = sm.prefix, mask = sm.mask;
-    for (int base = 0; base < nsrc; base += NT) {
-      const int i = base + tid;
-      uint32_t key = 0;
-      bool valid = false;
-      if (i < nsrc) {
-        key = src[i];
-        valid = (key & mask) == prefix;
-      }
-      const uint32_t d = valid ? ((key >> shift) & dmask) : 0xFFFFFFFFu;
-      const unsigned peers = __match_any_sync(0xffffffffu, d);
-      if (valid && lane == __ffs(peers) - 1) atomicAdd(&sm.hist[d], __popc(peers));
-    }
-    __syncthreads();
-    if (tid < 32) {
-      int local[8];
-      int s = 0;
-#pragma unroll
-      for (int d = 0; d < 8; ++d) {
-        local[d] = sm.hist[255 - (tid * 8 + d)];
-        s += local[d];
-      }
-      int incl = s;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (tid >= o) incl += y;
-      }
-      const int need = sm.need;
-      int above = incl - s;
-      if (above < need && incl >= need) {
-        int d = 0;
-        for (; d < 8; ++d) {
-          if (above + local[d] >= need) break;
-          above += local[d];
+    while (top >= 0) {
+      const int shift = top >= 7 ? top - 7 : 0;
+      const int width = top - shift + 1;
+      const uint32_t dmask = (1u << width) - 1u;
+      for (int i = tid; i < 256; i += NT) sm.hist[i] = 0;
+      __syncthreads();
+      const uint32_t prefix = sm.prefix, mask = sm.mask;
+      for (int base = 0; base < nsrc; base += NT) {
+        const int i = base + tid;
+        uint32_t key = 0;
+        bool valid = false;
+        if (i < nsrc) {
+          key = src[i];
+          valid = (key & mask) == prefix;
         }
-        const uint32_t digit = 255u - (uint32_t)(tid * 8 + d);
-        sm.prefix = prefix | (digit << shift);
-        sm.mask = mask | (dmask << shift);
-        sm.need = need - above;
+        const uint32_t d = valid ? ((key >> shift) & dmask) : 0xFFFFFFFFu;
+        const unsigned peers = __match_any_sync(0xffffffffu, d);
+        if (valid && lane == __ffs(peers) - 1) atomicAdd(&sm.hist[d], __popc(peers));
       }
+      __syncthreads();
+      if (tid < 32) {
+        int local[8];
+        int s = 0;
+#pragma unroll
+        for (int d = 0; d < 8; ++d) {
+          local[d] = sm.hist[255 - (tid * 8 + d)];
+          s += local[d];
+        }
+        int incl = s;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (tid >= o) incl += y;
+        }
+        const int need = sm.need;
+        int above = incl - s;
+        if (above < need && incl >= need) {
+          int d = 0;
+          for (; d < 8; ++d) {
+            if (above + local[d] >= need) break;
+            above += local[d];
+          }
+          const uint32_t digit = 255u - (uint32_t)(tid * 8 + d);
+          sm.prefix = prefix | (digit << shift);
+          sm.mask = mask | (dmask << shift);
+          sm.need = need - above;
+        }
+      }
+      __syncthreads();
+      top = shift - 1;
     }
-    __syncthreads();
-    top = shift - 1;
+    tau = sm.prefix;
+    take_eq = sm.need;
   }
-  const uint32_t tau = sm.prefix;
-  const int take_eq = sm.need;  // keys equal to tau to take, lowest positions first
 
-  // contiguous chunk per thread keeps the scans in position order
-  const int per = (n + NT - 1) / NT;
-  const int lo_i = min(n, tid * per), hi_i = min(n, lo_i + per);
-  int eq = 0, gt = 0;
-  for (int i = lo_i; i < hi_i; ++i) {
-    const uint32_t key = keys[i];
-    eq += key == tau;
-    gt += key > tau;
+  // 3. per-warp counts above / equal to tau
+  int cgt = 0, ceq = 0;
+  for (int base = w_lo; base < w_hi; base += 32 * U) {
+    uint32_t kv[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = base + 32 * u + lane;
+      kv[u] = i < w_hi ? keys[i] : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const bool valid = base + 32 * u + lane < w_hi;
+      cgt += __popc(__ballot_sync(0xffffffffu, valid && kv[u] > tau));
+      ceq += __popc(__ballot_sync(0xffffffffu, valid && kv[u] == tau));
+    }
   }
-  int total;
-  const int eq_before = block_exclusive_scan<NT>(eq, sm.scan, &total);
-  const int take_here = min(eq, max(0, take_eq - eq_before));
-  int pos = block_exclusive_scan<NT>(gt + take_here, sm.scan, &total);
-  {
-    int e = eq_before;
-    for (int i = lo_i; i < hi_i; ++i) {
-      const uint32_t key = keys[i];
-      bool take = false;
-      if (key > tau) take = true;
-      else if (key == tau) { take = e < take_eq; ++e; }
-      if (take && pos < k) out[pos++] = map(i);
+  if (lane == 0) {
+    sm.wgt[warp] = cgt;
+    sm.weq[warp] = ceq;
+  }
+  __syncthreads();
+  // keys equal to tau and output slots used by the warps before this one
+  int e_run = 0, p_run = 0;
+  for (int w = 0; w < warp; ++w) {
+    const int e = sm.weq[w];
+    p_run += sm.wgt[w] + min(e, max(0, take_eq - e_run));
+    e_run += e;
+  }
+  // slots in position order
+  for (int base = w_lo; base < w_hi; base += 32 * U) {
+    uint32_t kv[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = base + 32 * u + lane;
+      kv[u] = i < w_hi ? keys[i] : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = base + 32 * u + lane;
+      const bool valid = i < w_hi;
+      const bool q = valid && kv[u] == tau;
+      const unsigned eb = __ballot_sync(0xffffffffu, q);
+      const bool take = (valid && kv[u] > tau) || (q && e_run + __popc(eb & below) < take_eq);
+      const unsigned tb = __ballot_sync(0xffffffffu, take);
+      const int pos = p_run + __popc(tb & below);
+      if (take && pos < k) out[pos] = map(i);
+      e_run += __popc(eb);
+      p_run += __popc(tb);
     }
   }
 }

@@ -12,6 +12,7 @@
 #include <cooperative_groups.h>
 #include <cstdlib>
 
+#include "cluster_topk.cuh"
 #include "device_common.cuh"
 #include "host_common.h"
 #include "token_common.cuh"
@@ -77,10 +78,10 @@ __global__ void __launch_bounds__(NT) token_select_kernel(TokenParams p) {
 }
 
 // A cluster of kTokCluster CTAs per row when scoring is light: every CTA
-// scores a contiguous quarter of the candidates into its own shared memory;
-// after a cluster barrier the leader CTA gathers all keys through
-// distributed shared memory, a second barrier lets the others retire, and
-// the leader runs the top-k.
+// scores a contiguous quarter of the candidates into its own shared memory
+// and the cluster selects the top-k together over distributed shared memory
+// (cluster_topk.cuh).  When the scores are degenerate or too many of them
+// share the threshold bin, the leader CTA gathers all keys and selects alone.
 constexpr int kTokCluster = 4;
 constexpr int kTokThreads = 256;
 
@@ -96,16 +97,24 @@ __global__ void __cluster_dims__(kTokCluster, 1, 1) __launch_bounds__(kTokThread
   float* qlab = sm;                                                   // [G][R]
   int32_t* bidx = reinterpret_cast<int32_t*>(sm + p.group * R);       // [K_b]
   uint32_t* mine = reinterpret_cast<uint32_t*>(bidx + p.K_b);         // [per]
-  uint32_t* all = mine + per;                                         // [n_cand] (leader)
+  uint32_t* all = mine + per;                                         // [n_cand] (leader, fallback)
   TopkScratch* ts = reinterpret_cast<TopkScratch*>(all + p.n_cand);
+  ClusterTopkScratch<kTokCluster>* cts = reinterpret_cast<ClusterTopkScratch<kTokCluster>*>(
+      (reinterpret_cast<uintptr_t>(ts + 1) + 15) & ~uintptr_t(15));
+  cluster_arrive_relaxed();  // completes once every CTA of the cluster has started
   grid_launch_dependents();
   load_qlab<R, kTokThreads>(p, row, qlab);
+  if (threadIdx.x == 0) prefetch_l2(p.token_idx + (int64_t)row * p.k + (int64_t)rank * p.k / kTokCluster);
   grid_dependency_wait();  // the block lists come from the preceding kernel
   load_block_list<kTokThreads>(p, row, bidx);
   __syncthreads();
   const int c0 = min(p.n_cand, rank * per), c1 = min(p.n_cand, c0 + per);
   score_candidates<R, kTokThreads>(p, row, qlab, bidx, c0, c1, mine);
-  cluster.sync();
+  __syncthreads();
+  cluster_wait();
+  int* out = p.token_idx + (int64_t)row * p.k;
+  const CandidateToken map{bidx, p.bs};
+  if (cluster_topk_ascending<kTokThreads, kTokCluster>(mine, c1 - c0, c0, p.k, out, *cts, map)) return;
   if (rank == 0) {
     // gather the other CTAs' keys through distributed shared memory, eight
     // independent loads in flight per thread
@@ -129,8 +138,7 @@ __global__ void __cluster_dims__(kTokCluster, 1, 1) __launch_bounds__(kTokThread
   }
   cluster.sync();  // the other CTAs' shared memory may be released after this
   if (rank != 0) return;
-  cta_topk_ascending<kTokThreads>(all, p.n_cand, p.k, p.token_idx + (int64_t)row * p.k, *ts,
-                                  CandidateToken{bidx, p.bs});
+  cta_topk_ascending<kTokThreads>(all, p.n_cand, p.k, out, *ts, map);
 }
 
 void fill_token_params(TokenParams& p, const tls_shape& s, const void* q, const int32_t* label_ch,
@@ -183,7 +191,8 @@ tls_status select_tokens_impl(const tls_shape& s, const void* q, const int32_t* 
   const size_t smem = (size_t)p.group * s.n_label * 4 + (size_t)p.n_cand * 4 + sizeof(TopkScratch) + 16;
   if (token_stage_fits(p.group, s.n_label, p.n_cand)) {
     const int per = (p.n_cand + kTokCluster - 1) / kTokCluster;
-    const size_t csmem = ((size_t)p.group * s.n_label + K_b + per + p.n_cand) * 4 + sizeof(TopkScratch) + 16;
+    const size_t csmem = ((size_t)p.group * s.n_label + K_b + per + p.n_cand) * 4 + sizeof(TopkScratch) +
+                          sizeof(ClusterTopkScratch<kTokCluster>) + 32;
     const dim3 cgrid(kTokCluster, (unsigned)rows);
     switch (s.n_label) {
 #define TLS_TC_CASE(RR)                                                                                     \
