@@ -19,8 +19,8 @@
  *   - Pointers named "device" point to GPU memory (cudaMalloc / torch CUDA
  *     tensors); "host" pointers point to CPU memory.  The caller owns every
  *     buffer; the library keeps no pointer after a call returns, except the
- *     handles of tls_block_cache_create / tls_engine_create, which keep the
- *     pointers given to them until destroyed.
+ *     handle of tls_block_cache_create, which keeps the pointers given to it
+ *     until destroyed.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Kernel calls are asynchronous on that stream.
  *   - bf16 is IEEE bfloat16 stored as 16-bit words; all tensors are dense,
@@ -210,9 +210,10 @@ TLS_API tls_status tls_select(const tls_shape* shape, const void* q, const void*
                               int32_t* block_idx, int32_t* token_idx, void* ws, size_t ws_bytes, void* stream);
 
 /*
- * One synchronous decode step: tls_select then tls_sparse_decode_attn on
- * `stream` (three kernel launches), sharing one workspace.  block_idx /
- * token_idx are outputs as above.
+ * One decode step: tls_select then tls_sparse_decode_attn on `stream` (three
+ * kernel launches), sharing one workspace; the same results as those calls.
+ * block_idx / token_idx are outputs as above.  Every argument either call
+ * would reject is checked before anything is launched.
  */
 TLS_API tls_status tls_decode_step(const tls_shape* shape, const void* q, const void* meta,
                            const int32_t* label_ch, const uint8_t* codes, const float* scales,

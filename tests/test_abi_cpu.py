@@ -53,8 +53,12 @@ def c2_shape(tls, **kw):
 
 
 def test_attention_dispatch_names_the_kernel_per_shape(tls):
-    assert tls.tls_attn_kernel(c2_shape(tls)) == "sparse_attn_mma_kernel"              # G = 4
-    assert tls.tls_attn_kernel(c2_shape(tls, n_q_heads=128)) == "sparse_attn_mma_kernel"  # G = 16
+    # 128-wide heads, G <= 16: one cluster of CTAs per row when the rows fill the GPU that way
+    assert tls.tls_attn_kernel(c2_shape(tls)) == "sparse_attn_mma_cluster_kernel"              # 64 rows x 4
+    assert tls.tls_attn_kernel(c2_shape(tls, n_q_heads=128)) == "sparse_attn_mma_cluster_kernel"  # G = 16
+    assert tls.tls_attn_kernel(c2_shape(tls, batch=16)) == "sparse_attn_mma_cluster_kernel"     # 128 rows x 2
+    assert tls.tls_attn_kernel(c2_shape(tls, batch=1)) == "sparse_attn_mma_kernel"              # 8 rows: persistent
+    assert tls.tls_attn_kernel(c2_shape(tls, batch=64)) == "sparse_attn_mma_kernel"             # 512 rows
     assert tls.tls_attn_kernel(c2_shape(tls, n_q_heads=64, n_kv_heads=1)) == "sparse_attn_tc_kernel"
     mla = c2_shape(tls, batch=4, n_q_heads=128, n_kv_heads=1, qk_dim=576, v_dim=512, v_offset=0, n_label=32)
     assert tls.tls_attn_kernel(mla) == "sparse_attn_kernel"

@@ -63,6 +63,14 @@ SMALL = [
     small("s_all", ctx_len=512, K_b=32, k=512, seed=18),
 ]
 FULL = [get_config(c) for c in ("c1", "c2", "c3", "c4")]
+# row counts that send the 128-wide, G <= 16 attention to its cluster form
+# (8, 4 and 2 CTAs per row); ragged lists, and in s_cl8 a CTA with no chunk
+CLUSTER = [
+    small("s_cl8", batch=20, n_q_heads=4, n_kv_heads=1, ctx_len=1024, K_b=7, k=97, seed=21),
+    small("s_cl4", batch=16, n_q_heads=16, n_kv_heads=4, ctx_len=2048, K_b=13, k=200, seed=22),
+    small("s_cl4_g1", batch=8, n_q_heads=8, n_kv_heads=8, ctx_len=1024, K_b=8, k=128, seed=23),
+    small("s_cl2_g16", batch=100, n_q_heads=16, n_kv_heads=1, ctx_len=1024, block_size=32, K_b=9, k=270, seed=24),
+]
 
 
 def make_state(cfg, **kw):
@@ -158,6 +166,16 @@ def test_small_shapes_all_rows(cfg):
     for b in range(cfg.batch):
         for h in range(cfg.n_kv_heads):
             check_row(cfg, data, got, st, b, h)
+
+
+@pytest.mark.parametrize("cfg", CLUSTER, ids=lambda c: c.name)
+def test_cluster_attention_sampled_rows(cfg):
+    runtime, tls = _rt()
+    st, data = make_state(cfg)
+    assert tls.tls_attn_kernel(st.shape) == "sparse_attn_mma_cluster_kernel"
+    got = run_stages(st)
+    for b, h in sample_rows(cfg, 6):  # the first and last rows among them
+        check_row(cfg, data, got, st, b, h)
 
 
 @pytest.mark.parametrize("cfg", FULL, ids=lambda c: c.name)
@@ -326,3 +344,21 @@ def test_fused_select_equals_the_two_level_calls(cfg):
     assert st.check_device_error() == 0
     assert np.array_equal(st.block_idx.cpu().numpy(), got["block_idx"])
     assert np.array_equal(st.token_idx.cpu().numpy(), got["token_idx"])
+
+
+@pytest.mark.parametrize("cfg", SMALL + [get_config("c1"), get_config("c2")], ids=lambda c: c.name)
+def test_decode_step_equals_select_then_attend(cfg):
+    # one call for the whole step: the results of the separate calls, bit for bit
+    st, data = make_state(cfg)
+    got = run_stages(st)
+    for t in (st.block_idx, st.token_idx):
+        t.fill_(-1)
+    st.out.fill_(float("nan"))
+    st.lse.fill_(float("nan"))
+    st.step()
+    torch.cuda.synchronize()
+    assert st.check_device_error() == 0
+    assert np.array_equal(st.block_idx.cpu().numpy(), got["block_idx"])
+    assert np.array_equal(st.token_idx.cpu().numpy(), got["token_idx"])
+    assert np.array_equal(st.out.float().cpu().numpy(), got["out"])
+    assert np.array_equal(st.lse.cpu().numpy(), got["lse"])

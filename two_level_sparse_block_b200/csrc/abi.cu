@@ -28,6 +28,7 @@ bool attn_tc_supported(const tls_shape& s);
 int attn_tc_plan(int rows, int head_groups, int k, int* tiles, int* n_items, int* n_ctas);
 bool attn_mma_supported(const tls_shape& s);
 int attn_mma_plan(int rows, int k, int* chunks_per_row, int* n_items, int* n_ctas);
+int attn_mma_cluster_size(int rows);
 
 namespace {
 thread_local char g_err[512] = {0};
@@ -157,7 +158,8 @@ extern "C" int32_t tls_version(void) { return 100; }
 
 extern "C" const char* tls_attn_kernel(const tls_shape* shape) {
   if (check_shape(shape) != TLS_OK) return nullptr;
-  if (attn_mma_supported(*shape)) return "sparse_attn_mma_kernel";
+  if (attn_mma_supported(*shape))
+    return attn_mma_cluster_size(rows_of(*shape)) > 0 ? "sparse_attn_mma_cluster_kernel" : "sparse_attn_mma_kernel";
   if (attn_tc_supported(*shape)) return "sparse_attn_tc_kernel";
   return "sparse_attn_kernel";
 }
@@ -246,10 +248,10 @@ extern "C" tls_status tls_sparse_decode_attn(const tls_shape* shape, const void*
                           (cudaStream_t)stream);
 }
 
-extern "C" tls_status tls_select(const tls_shape* shape, const void* q, const void* meta, const int32_t* label_ch,
-                                 const uint8_t* codes, const float* scales, int32_t K_b, int32_t k,
-                                 int32_t* block_idx, int32_t* token_idx, void* ws, size_t ws_bytes, void* stream) {
-  clear_error();
+// Levels 1 and 2 (the second launched with programmatic dependent launch).
+static tls_status select_impl(const tls_shape* shape, const void* q, const void* meta, const int32_t* label_ch,
+                              const uint8_t* codes, const float* scales, int32_t K_b, int32_t k, int32_t* block_idx,
+                              int32_t* token_idx, void* ws, size_t ws_bytes, void* stream) {
   tls_status st = check_shape(shape);
   if (st != TLS_OK) return st;
   if (q == nullptr || meta == nullptr || label_ch == nullptr || codes == nullptr || scales == nullptr ||
@@ -270,13 +272,28 @@ extern "C" tls_status tls_select(const tls_shape* shape, const void* q, const vo
                             (uint8_t*)ws, L, (cudaStream_t)stream, /*pdl=*/true);
 }
 
+extern "C" tls_status tls_select(const tls_shape* shape, const void* q, const void* meta, const int32_t* label_ch,
+                                 const uint8_t* codes, const float* scales, int32_t K_b, int32_t k,
+                                 int32_t* block_idx, int32_t* token_idx, void* ws, size_t ws_bytes, void* stream) {
+  clear_error();
+  return select_impl(shape, q, meta, label_ch, codes, scales, K_b, k, block_idx, token_idx, ws, ws_bytes, stream);
+}
+
 extern "C" tls_status tls_decode_step(const tls_shape* shape, const void* q, const void* meta,
                                       const int32_t* label_ch, const uint8_t* codes, const float* scales,
                                       const tls_kv_view* kv, int32_t K_b, int32_t k, int32_t* block_idx,
                                       int32_t* token_idx, int32_t out_dtype, void* out, float* lse, void* ws,
                                       size_t ws_bytes, void* stream) {
-  tls_status st = tls_select(shape, q, meta, label_ch, codes, scales, K_b, k, block_idx, token_idx, ws, ws_bytes,
-                             stream);
+  clear_error();
+  // everything the attention checks is checked before anything is launched
+  tls_status st = check_shape(shape);
+  if (st != TLS_OK) return st;
+  st = check_kv(*shape, kv);
+  if (st != TLS_OK) return st;
+  if (out == nullptr) return fail(TLS_ERR_INVALID_ARG, "decode_step: out is NULL");
+  if (out_dtype != TLS_OUT_F32 && out_dtype != TLS_OUT_BF16)
+    return fail(TLS_ERR_INVALID_ARG, "decode_step: out_dtype must be TLS_OUT_F32 or TLS_OUT_BF16");
+  st = select_impl(shape, q, meta, label_ch, codes, scales, K_b, k, block_idx, token_idx, ws, ws_bytes, stream);
   if (st != TLS_OK) return st;
   return tls_sparse_decode_attn(shape, q, kv, token_idx, k, out_dtype, out, lse, ws, ws_bytes, stream);
 }

@@ -123,6 +123,7 @@ bool attn_tc_supported(const tls_shape& s);
 tls_status launch_attn_tc(const AttnParams& p, int rows, cudaStream_t stream);
 // Warp-streaming attention for groups of <= 16 heads (decode_attn_mma.cu).
 bool attn_mma_supported(const tls_shape& s);
-tls_status launch_attn_mma(const AttnParams& p, cudaStream_t stream);
+tls_status launch_attn_mma(const AttnParams& p, int rows, cudaStream_t stream);
+int attn_mma_cluster_size(int rows);
 
 }  // namespace tls

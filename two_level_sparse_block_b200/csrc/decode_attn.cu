@@ -64,7 +64,7 @@ __global__ void __launch_bounds__(128) sparse_attn_kernel(AttnParams p) {
   const int t_begin = split * p.tokens_per_split;
   const int t_end = min(p.k_sel, t_begin + p.tokens_per_split);
   const int32_t* tix = p.token_idx + (int64_t)row * p.k_sel;
-  grid_dependency_wait();  // token lists come from the preceding kernel
+  grid_dependency_wait();  // token lists come from the preceding kernel (read through L2)
 
   for (int base = t_begin; base < t_end; base += 8 * U) {
     uint4 kw[U][PK], vw[U][PV];
@@ -76,7 +76,7 @@ __global__ void __launch_bounds__(128) sparse_attn_kernel(AttnParams p) {
       int64_t krow = 0, vrow = 0;
       if (valid[u]) {
         // indices are clamped so a bad list can never address outside the cache
-        const int64_t tok = min(max((int64_t)tix[t], (int64_t)0), p.ctx_len - 1);
+        const int64_t tok = min(max((int64_t)__ldcg(tix + t), (int64_t)0), p.ctx_len - 1);
         int64_t r;
         if (p.slot_of_block != nullptr) {
           const int64_t slot = min(max(p.slot_of_block[(int64_t)row * p.nb + tok / p.bs], 0), p.n_slots - 1);
@@ -257,7 +257,7 @@ tls_status sparse_attn_impl(const tls_shape& s, const void* q, const tls_kv_view
   p.n_ctas = L.n_ctas;
   p.err = reinterpret_cast<int*>(ws + L.err);
   const int rows = rows_of(s);
-  if (attn_mma_supported(s)) return launch_attn_mma(p, stream);
+  if (attn_mma_supported(s)) return launch_attn_mma(p, rows, stream);
   if (attn_tc_supported(s)) return launch_attn_tc(p, rows, stream);
   const int pk = (s.qk_dim + 127) / 128, pv = (s.v_dim + 127) / 128;
   const int hg = L.heads_per_cta;

@@ -18,6 +18,8 @@
 // shared memory and writes (m, l, O) to the split workspace; the last CTA to
 // finish a row merges the splits by log-sum-exp (attn_common.cuh).
 
+#include <cooperative_groups.h>
+
 #include "attn_common.cuh"
 #include "device_common.cuh"
 #include "host_common.h"
@@ -87,6 +89,212 @@ __host__ __device__ inline MmaLayout mma_layout(int g) {
   return L;
 }
 
+// Q fragments (the A operand of S = Q.K^T, 8 k-steps of 16) of the g heads
+// of row (b, kvh); fragment rows >= g are zero.
+__device__ __forceinline__ void mma_load_q(const AttnParams& p, int b, int kvh, int lane, uint32_t (&qa)[8][4]) {
+  const int g = p.group, gq = lane >> 2, tq = lane & 3;
+  const uint16_t* q0 = p.q + ((int64_t)b * p.n_q_heads + kvh * g + gq) * p.dqk;
+  const uint16_t* q8 = q0 + (int64_t)8 * p.dqk;
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+    const int d0 = ks * 16 + 2 * tq;
+    qa[ks][0] = gq < g ? *reinterpret_cast<const uint32_t*>(q0 + d0) : 0u;
+    qa[ks][1] = gq + 8 < g ? *reinterpret_cast<const uint32_t*>(q8 + d0) : 0u;
+    qa[ks][2] = gq < g ? *reinterpret_cast<const uint32_t*>(q0 + d0 + 8) : 0u;
+    qa[ks][3] = gq + 8 < g ? *reinterpret_cast<const uint32_t*>(q8 + d0 + 8) : 0u;
+  }
+}
+
+// Raw token index of entry (lane & 15) of chunk x of the row's list, or -1
+// past the end of the list.
+__device__ __forceinline__ int mma_chunk_token(const AttnParams& p, int row, int x, int lane) {
+  const int t = x * kChunk + (lane & 15);
+  if (t >= p.k_sel) return -1;
+  // L2 load: the list is written by the preceding kernel while this grid is
+  // already resident (programmatic dependent launch)
+  return __ldcg(p.token_idx + (int64_t)row * p.k_sel + t);
+}
+
+// cp.async of the K and V rows of one chunk into the ring stage at shared
+// address kb (K tile; V tile at kb + 4096).  Entry lane & 15 holds raw token
+// `tok` (-1: the rows are zero-filled); tokens are clamped to the context and
+// slots to the pool.  The caller commits the group.
+__device__ __forceinline__ void mma_issue_rows(const AttnParams& p, int row, int tok, uint32_t kb, int lane) {
+  int64_t rid = -1;
+  if (tok >= 0) {
+    const int64_t tk = min(max((int64_t)tok, (int64_t)0), p.ctx_len - 1);
+    if (p.slot_of_block != nullptr) {
+      const int64_t slot = min(max(__ldg(p.slot_of_block + (int64_t)row * p.nb + tk / p.bs), 0), p.n_slots - 1);
+      rid = slot * p.bs + tk % p.bs;
+    } else {
+      rid = (int64_t)row * p.ctx_len + tk;
+    }
+  }
+  const uint32_t vb = kb + 4096;
+  const int c = lane & 15;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int r = (lane >> 4) + 2 * j;
+    const int64_t rr = __shfl_sync(0xffffffffu, rid, r);
+    const bool v = rr >= 0;
+    const uint32_t off = tile_off(r, c);
+    cp_async16(kb + off, p.k + (v ? rr * p.k_stride : 0) + c * 8, v ? 16u : 0u);
+    cp_async16(vb + off, p.v + (v ? rr * p.v_stride : 0) + c * 8, v ? 16u : 0u);
+  }
+}
+
+// One chunk of 16 tokens (list positions t_base ..) for the fragment rows gq
+// (m0, l0) and gq + 8 (m1, l1): S = Q.K^T scaled to base 2 and masked past the
+// list end, the online softmax update, and O += P.V with P split into bf16
+// hi + lo parts.  K and V tiles of the chunk at shared address kb / kb + 4096.
+__device__ __forceinline__ void mma_chunk(const AttnParams& p, const uint32_t (&qa)[8][4], float (&o)[16][4],
+                                          float& m0, float& m1, float& l0, float& l1, uint32_t kb, int t_base,
+                                          int lane) {
+  const int tq = lane & 3;
+  const uint32_t vb = kb + 4096;
+  // S = Q . K^T for 16 tokens (two n-tiles of 8)
+  float s[2][4];
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+    s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.0f;
+#pragma unroll
+    for (int ks = 0; ks < 8; ks += 2) {
+      // matrices: (k-step ks, units 2ks, 2ks+1), (ks+1, units 2ks+2, 2ks+3)
+      const int mtx = lane >> 3;
+      const uint32_t addr = kb + tile_off(nt * 8 + (lane & 7), ks * 2 + mtx);
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4(addr, b0, b1, b2, b3);
+      mma_bf16_16816(s[nt], qa[ks], b0, b1);
+      mma_bf16_16816(s[nt], qa[ks + 1], b2, b3);
+    }
+  }
+  // scale (and mask the tail of the list), online softmax
+  // (rows gq: elements 0,1; rows gq+8: elements 2,3)
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s[nt][e] *= p.scale_log2;
+  if (t_base + kChunk > p.k_sel) {
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (t_base + nt * 8 + 2 * tq + (e & 1) >= p.k_sel) s[nt][e] = -INFINITY;
+  }
+  float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
+  float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
+  mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+  mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+  mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+  mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+  const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+  // the O rescale is skipped (warp-uniformly) when no row maximum moved
+  if (!__all_sync(0xffffffffu, n0 == m0 && n1 == m1)) {
+    const float c0 = fast_exp2(m0 - n0), c1 = fast_exp2(m1 - n1);  // 0 on the first chunk
+    l0 *= c0;
+    l1 *= c1;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      o[j][0] *= c0;
+      o[j][1] *= c0;
+      o[j][2] *= c1;
+      o[j][3] *= c1;
+    }
+    m0 = n0;
+    m1 = n1;
+  }
+  float pr[2][4];
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) pr[nt][e] = fast_exp2(s[nt][e] - (e < 2 ? n0 : n1));
+  l0 += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
+  l1 += (pr[0][2] + pr[0][3]) + (pr[1][2] + pr[1][3]);
+  // P as the A operand (k = the 16 tokens), hi and lo parts
+  uint32_t ph[4], pl[4];
+  {
+    const float a[4][2] = {{pr[0][0], pr[0][1]}, {pr[0][2], pr[0][3]}, {pr[1][0], pr[1][1]}, {pr[1][2], pr[1][3]}};
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      ph[r] = pack_bf16(a[r][0], a[r][1]);
+      pl[r] = pack_bf16(a[r][0] - bf16_lo_f(ph[r]), a[r][1] - bf16_hi_f(ph[r]));
+    }
+  }
+  // O += P . V over 16 n-tiles of 8 value columns
+#pragma unroll
+  for (int j = 0; j < 16; j += 2) {
+    // matrices: tokens 0-7 / 8-15 of unit j, then of unit j+1
+    const int mtx = lane >> 3;
+    const uint32_t addr = vb + tile_off((mtx & 1) * 8 + (lane & 7), j + (mtx >> 1));
+    uint32_t b0, b1, b2, b3;
+    ldsm_x4_t(addr, b0, b1, b2, b3);
+    mma_bf16_16816(o[j], ph, b0, b1);
+    mma_bf16_16816(o[j], pl, b0, b1);
+    mma_bf16_16816(o[j + 1], ph, b2, b3);
+    mma_bf16_16816(o[j + 1], pl, b2, b3);
+  }
+}
+
+// The CTA's warps fold their (m, l, O) for one row: they write them to
+// shared memory (comb [warp][h][128], cm / cl [warp][16]) and, after a
+// barrier, put(h, e, v) receives for every head h < g the CTA's combined
+// values relative to its own maximum M: e = 0 -> M, e = 1 -> l,
+// e = 2 + d -> O[d].  All threads of the CTA must call it.
+template <typename Put>
+__device__ __forceinline__ void mma_fold(int g, float m0, float m1, float l0, float l1, const float (&o)[16][4],
+                                         float* comb, float* cm, float* cl, Put put) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+  if (tq == 0) {
+    if (gq < g) {
+      cm[warp * 16 + gq] = m0;
+      cl[warp * 16 + gq] = l0;
+    }
+    if (gq + 8 < g) {
+      cm[warp * 16 + gq + 8] = m1;
+      cl[warp * 16 + gq + 8] = l1;
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const int d = j * 8 + 2 * tq;
+    if (gq < g) {
+      comb[(warp * g + gq) * 128 + d] = o[j][0];
+      comb[(warp * g + gq) * 128 + d + 1] = o[j][1];
+    }
+    if (gq + 8 < g) {
+      comb[(warp * g + gq + 8) * 128 + d] = o[j][2];
+      comb[(warp * g + gq + 8) * 128 + d + 1] = o[j][3];
+    }
+  }
+  __syncthreads();
+  for (int idx = tid; idx < g * 130; idx += kMmaWarps * 32) {
+    const int h = idx / 130, e = idx % 130;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kMmaWarps; ++w) M = fmaxf(M, cm[w * 16 + h]);
+    float val = 0.0f;
+    if (e == 0) {
+      val = M;
+    } else if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kMmaWarps; ++w) {
+        const float mw = cm[w * 16 + h];
+        if (mw == -INFINITY) continue;
+        const float f = exp2f(mw - M);
+        val += f * (e == 1 ? cl[w * 16 + h] : comb[(w * g + h) * 128 + (e - 2)]);
+      }
+    }
+    put(h, e, val);
+  }
+}
+
+// Persistent form: every CTA owns a contiguous range of the (row, chunk)
+// items; a row spread over several CTAs is merged by the last of them
+// through the split workspace (attn_common.cuh).
 template <int NS>
 __global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_kernel(AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -99,61 +307,29 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_kernel(Attn
   __shared__ int s_last;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int gq = lane >> 2, tq = lane & 3;  // mma fragment coordinates
-  const int CPR = p.tiles_per_pair;         // chunks per row
+  const int CPR = p.tiles_per_pair;  // chunks per row
   const int64_t C = p.n_items;
   const int64_t cta = blockIdx.x;
   const int64_t c_lo = cta * C / p.n_ctas, c_hi = (cta + 1) * C / p.n_ctas;
-  uint8_t* ring = sm + warp * NS * kChunkBytes;
-  const uint32_t ring_s = smem_u32(ring);
+  const uint32_t ring_s = smem_u32(sm + warp * NS * kChunkBytes);
 
   // this warp's stream: chunks c_lo + warp + 4i
   const int64_t x0 = c_lo + warp;
   const int n_mine = x0 < c_hi ? (int)((c_hi - 1 - x0) / kMmaWarps + 1) : 0;
-
-  // raw token index of entry (lane & 15) of chunk x, or -1
   auto load_tok = [&](int i) -> int {
     if (i >= n_mine) return -1;
     const int64_t x = x0 + (int64_t)kMmaWarps * i;
-    const int row = (int)(x / CPR);
-    const int t = (int)(x % CPR) * kChunk + (lane & 15);
-    if (t >= p.k_sel) return -1;
-    return __ldg(p.token_idx + (int64_t)row * p.k_sel + t);
+    return mma_chunk_token(p, (int)(x / CPR), (int)(x % CPR), lane);
   };
-  // cp.async of the K and V rows of chunk i (its raw token indices in `tok`) into stage st
   auto issue = [&](int i, int tok, int st) {
-    if (i < n_mine) {
-      const int row = (int)((x0 + (int64_t)kMmaWarps * i) / CPR);
-      int64_t rid = -1;
-      if (tok >= 0) {
-        const int64_t tk = min(max((int64_t)tok, (int64_t)0), p.ctx_len - 1);
-        if (p.slot_of_block != nullptr) {
-          const int64_t slot =
-              min(max(__ldg(p.slot_of_block + (int64_t)row * p.nb + tk / p.bs), 0), p.n_slots - 1);
-          rid = slot * p.bs + tk % p.bs;
-        } else {
-          rid = (int64_t)row * p.ctx_len + tk;
-        }
-      }
-      const uint32_t kb = ring_s + st * kChunkBytes, vb = kb + 4096;
-      const int c = lane & 15;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int r = (lane >> 4) + 2 * j;
-        const int64_t rr = __shfl_sync(0xffffffffu, rid, r);
-        const bool v = rr >= 0;
-        const uint32_t off = tile_off(r, c);
-        cp_async16(kb + off, p.k + (v ? rr * p.k_stride : 0) + c * 8, v ? 16u : 0u);
-        cp_async16(vb + off, p.v + (v ? rr * p.v_stride : 0) + c * 8, v ? 16u : 0u);
-      }
-    }
+    if (i < n_mine)
+      mma_issue_rows(p, (int)((x0 + (int64_t)kMmaWarps * i) / CPR), tok, ring_s + st * kChunkBytes, lane);
     cp_async_commit();
   };
 
-  // Q fragments (A operand) of the current row, 8 k-steps
   uint32_t qa[8][4];
   float o[16][4];
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f;  // rows gq and gq + 8
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f;  // fragment rows gq and gq + 8
 
   grid_launch_dependents();
   if (tid == 0 && c_lo < c_hi) {
@@ -185,16 +361,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_kernel(Attn
     const int b = row / p.n_kv_heads, kvh = row % p.n_kv_heads;
     // this row's chunks inside the CTA range
     const int64_t seg_end = min(c_hi, (int64_t)(row + 1) * CPR);
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      const int d0 = ks * 16 + 2 * tq;
-      const uint16_t* q0 = p.q + ((int64_t)b * p.n_q_heads + kvh * g + gq) * p.dqk;
-      const uint16_t* q8 = q0 + (int64_t)8 * p.dqk;
-      qa[ks][0] = gq < g ? *reinterpret_cast<const uint32_t*>(q0 + d0) : 0u;
-      qa[ks][1] = gq + 8 < g ? *reinterpret_cast<const uint32_t*>(q8 + d0) : 0u;
-      qa[ks][2] = gq < g ? *reinterpret_cast<const uint32_t*>(q0 + d0 + 8) : 0u;
-      qa[ks][3] = gq + 8 < g ? *reinterpret_cast<const uint32_t*>(q8 + d0 + 8) : 0u;
-    }
+    mma_load_q(p, b, kvh, lane, qa);
 #pragma unroll
     for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.0f;
     m0 = m1 = -INFINITY;
@@ -207,145 +374,18 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_kernel(Attn
       tok_next = tok_after;
       cp_async_wait<NS - 1>();
       __syncwarp();
-
       const int64_t x = x0 + (int64_t)kMmaWarps * i;
-      const int t_base = (int)(x % CPR) * kChunk;
-      const uint32_t kb = ring_s + (i % NS) * kChunkBytes, vb = kb + 4096;
-
-      // S = Q . K^T for 16 tokens (two n-tiles of 8)
-      float s[2][4];
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.0f;
-#pragma unroll
-        for (int ks = 0; ks < 8; ks += 2) {
-          // matrices: (k-step ks, units 2ks, 2ks+1), (ks+1, units 2ks+2, 2ks+3)
-          const int mtx = lane >> 3;
-          const uint32_t addr = kb + tile_off(nt * 8 + (lane & 7), ks * 2 + mtx);
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(addr, b0, b1, b2, b3);
-          mma_bf16_16816(s[nt], qa[ks], b0, b1);
-          mma_bf16_16816(s[nt], qa[ks + 1], b2, b3);
-        }
-      }
-      // scale (and mask the tail of the list), online softmax
-      // (rows gq: elements 0,1; rows gq+8: elements 2,3)
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) s[nt][e] *= p.scale_log2;
-      if (t_base + kChunk > p.k_sel) {
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            if (t_base + nt * 8 + 2 * tq + (e & 1) >= p.k_sel) s[nt][e] = -INFINITY;
-      }
-      float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
-      float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-      const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
-      // the O rescale is skipped (warp-uniformly) when no row maximum moved
-      if (!__all_sync(0xffffffffu, n0 == m0 && n1 == m1)) {
-        const float c0 = fast_exp2(m0 - n0), c1 = fast_exp2(m1 - n1);  // 0 on the first chunk
-        l0 *= c0;
-        l1 *= c1;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          o[j][0] *= c0;
-          o[j][1] *= c0;
-          o[j][2] *= c1;
-          o[j][3] *= c1;
-        }
-        m0 = n0;
-        m1 = n1;
-      }
-      float pr[2][4];
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) pr[nt][e] = fast_exp2(s[nt][e] - (e < 2 ? n0 : n1));
-      l0 += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
-      l1 += (pr[0][2] + pr[0][3]) + (pr[1][2] + pr[1][3]);
-      // P as the A operand (k = the 16 tokens), hi and lo parts
-      uint32_t ph[4], pl[4];
-      {
-        const float a[4][2] = {{pr[0][0], pr[0][1]}, {pr[0][2], pr[0][3]}, {pr[1][0], pr[1][1]}, {pr[1][2], pr[1][3]}};
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          ph[r] = pack_bf16(a[r][0], a[r][1]);
-          pl[r] = pack_bf16(a[r][0] - bf16_lo_f(ph[r]), a[r][1] - bf16_hi_f(ph[r]));
-        }
-      }
-      // O += P . V over 16 n-tiles of 8 value columns
-#pragma unroll
-      for (int j = 0; j < 16; j += 2) {
-        // matrices: tokens 0-7 / 8-15 of unit j, then of unit j+1
-        const int mtx = lane >> 3;
-        const uint32_t addr = vb + tile_off((mtx & 1) * 8 + (lane & 7), j + (mtx >> 1));
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(addr, b0, b1, b2, b3);
-        mma_bf16_16816(o[j], ph, b0, b1);
-        mma_bf16_16816(o[j], pl, b0, b1);
-        mma_bf16_16816(o[j + 1], ph, b2, b3);
-        mma_bf16_16816(o[j + 1], pl, b2, b3);
-      }
+      mma_chunk(p, qa, o, m0, m1, l0, l1, ring_s + (i % NS) * kChunkBytes, (int)(x % CPR) * kChunk, lane);
       __syncwarp();
     }
 
-    // fold the warps of the CTA for this row
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-    if (tq == 0) {
-      if (gq < g) {
-        cm[warp * 16 + gq] = m0;
-        cl[warp * 16 + gq] = l0;
-      }
-      if (gq + 8 < g) {
-        cm[warp * 16 + gq + 8] = m1;
-        cl[warp * 16 + gq + 8] = l1;
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const int d = j * 8 + 2 * tq;
-      if (gq < g) {
-        comb[(warp * g + gq) * 128 + d] = o[j][0];
-        comb[(warp * g + gq) * 128 + d + 1] = o[j][1];
-      }
-      if (gq + 8 < g) {
-        comb[(warp * g + gq + 8) * 128 + d] = o[j][2];
-        comb[(warp * g + gq + 8) * 128 + d + 1] = o[j][3];
-      }
-    }
-    __syncthreads();
+    // fold the warps of the CTA for this row into its split of the workspace
     const int64_t first = attn_owner((int64_t)row * CPR, C, p.n_ctas);
     const int n_part = (int)(attn_owner((int64_t)row * CPR + CPR - 1, C, p.n_ctas) - first + 1);
     const int slot = (int)(cta - first);
-    for (int idx = tid; idx < g * 130; idx += kMmaWarps * 32) {
-      const int h = idx / 130, e = idx % 130;
-      float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < kMmaWarps; ++w) M = fmaxf(M, cm[w * 16 + h]);
-      float val = 0.0f;
-      if (e == 0) {
-        val = M;
-      } else if (M != -INFINITY) {
-#pragma unroll
-        for (int w = 0; w < kMmaWarps; ++w) {
-          const float mw = cm[w * 16 + h];
-          if (mw == -INFINITY) continue;
-          const float f = exp2f(mw - M);
-          val += f * (e == 1 ? cl[w * 16 + h] : comb[(w * g + h) * 128 + (e - 2)]);
-        }
-      }
-      p.partial[(((int64_t)row * g + h) * p.splits + slot) * 130 + e] = val;
-    }
+    float* part = p.partial + ((int64_t)row * g * p.splits + slot) * 130;
+    mma_fold(g, m0, m1, l0, l1, o, comb, cm, cl,
+             [&](int h, int e, float v) { part[(int64_t)h * p.splits * 130 + e] = v; });
     __threadfence();
     __syncthreads();
     if (tid == 0) s_last = atomicInc(&p.counters[row], (unsigned)(n_part - 1)) == (unsigned)(n_part - 1);
@@ -357,6 +397,99 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_kernel(Attn
     __syncthreads();  // the fold area is rewritten for the next row
   }
   cp_async_wait<0>();
+}
+
+// Cluster form: one cluster of CL = gridDim.x CTAs per row (row =
+// blockIdx.y).  CTA r streams chunks [r * CPR / CL, (r + 1) * CPR / CL) of
+// the row as above; then every CTA folds its warps and writes its partial
+// (M, l, O per head) into the leader's drained cp.async ring over
+// distributed shared memory, and the leader merges the CL partials by
+// log-sum-exp.  No workspace, ticket or device-wide fence.
+template <int NS>
+__global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_cluster_kernel(AttnParams p) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  const int g = p.group;
+  const MmaLayout L = mma_layout(g);
+  float* comb = reinterpret_cast<float*>(sm + L.off_comb);
+  float* cm = reinterpret_cast<float*>(sm + L.off_stat);
+  float* cl = cm + kMmaWarps * 16;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int CL = (int)gridDim.x, rank = (int)blockIdx.x, row = (int)blockIdx.y;
+  const int b = row / p.n_kv_heads, kvh = row % p.n_kv_heads;
+  const int CPR = p.tiles_per_pair;
+  const int c_lo = rank * CPR / CL, c_hi = (rank + 1) * CPR / CL;
+  const uint32_t ring_s = smem_u32(sm + warp * NS * kChunkBytes);
+  const int x0 = c_lo + warp;
+  const int n_mine = x0 < c_hi ? (c_hi - 1 - x0) / kMmaWarps + 1 : 0;
+  auto load_tok = [&](int i) -> int { return i < n_mine ? mma_chunk_token(p, row, x0 + kMmaWarps * i, lane) : -1; };
+  auto issue = [&](int i, int tok, int st) {
+    if (i < n_mine) mma_issue_rows(p, row, tok, ring_s + st * kChunkBytes, lane);
+    cp_async_commit();
+  };
+  const int64_t oh = (int64_t)b * p.n_q_heads + (int64_t)kvh * g;  // first output head of the row
+
+  grid_launch_dependents();
+  if (tid == 0 && rank == 0) {
+    // the leader writes the output and lse rows last: warm them now
+    prefetch_l2(reinterpret_cast<const uint8_t*>(p.out) + oh * p.dv * (p.out_bf16 ? 2 : 4));
+    if (p.lse != nullptr) prefetch_l2(p.lse + oh);
+  }
+  uint32_t qa[8][4];
+  mma_load_q(p, b, kvh, lane, qa);  // q is an input of the step, not of the preceding kernel
+  grid_dependency_wait();           // token lists come from the preceding kernel
+
+  float o[16][4];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.0f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f;
+  int tok_ahead[NS];
+#pragma unroll
+  for (int s = 0; s < NS; ++s) tok_ahead[s] = load_tok(s);
+#pragma unroll
+  for (int s = 0; s < NS - 1; ++s) issue(s, tok_ahead[s], s);
+  int tok_next = tok_ahead[NS - 1];
+  for (int i = 0; i < n_mine; ++i) {
+    const int tok_after = load_tok(i + NS);
+    issue(i + NS - 1, tok_next, (i + NS - 1) % NS);
+    tok_next = tok_after;
+    cp_async_wait<NS - 1>();
+    __syncwarp();
+    mma_chunk(p, qa, o, m0, m1, l0, l1, ring_s + (i % NS) * kChunkBytes, (x0 + kMmaWarps * i) * kChunk, lane);
+    __syncwarp();
+  }
+  cp_async_wait<0>();
+  cluster.sync();  // every CTA (the leader included) is done with its ring
+
+  // partials [CL][g][130] over the leader's ring
+  float* part = reinterpret_cast<float*>(sm);
+  float* dst = cluster.map_shared_rank(part, 0) + (size_t)rank * g * 130;
+  mma_fold(g, m0, m1, l0, l1, o, comb, cm, cl, [&](int h, int e, float v) { dst[h * 130 + e] = v; });
+  cluster.sync();  // the partials have landed; nothing remote is touched after this
+  if (rank != 0) return;
+
+  const int dv = p.dv;
+  for (int idx = tid; idx < g * dv; idx += kMmaWarps * 32) {
+    const int h = idx / dv, e = idx - h * dv;
+    float M = -INFINITY;
+    for (int r = 0; r < CL; ++r) M = fmaxf(M, part[(r * g + h) * 130]);
+    float lsum = 0.0f, acc = 0.0f;
+    for (int r = 0; r < CL; ++r) {
+      const float* pr = part + (r * g + h) * 130;
+      if (pr[0] == -INFINITY) continue;
+      const float f = exp2f(pr[0] - M);
+      lsum += f * pr[1];
+      acc += f * pr[2 + e];
+    }
+    const float val = lsum > 0.0f ? acc / lsum : 0.0f;
+    const int64_t oe = (oh + h) * dv + e;
+    if (p.out_bf16) reinterpret_cast<uint16_t*>(p.out)[oe] = f32_to_bf16_rn(val);
+    else reinterpret_cast<float*>(p.out)[oe] = val;
+    if (e == 0 && p.lse != nullptr) p.lse[oh + h] = (M + log2f(lsum)) * 0.69314718055994531f;
+  }
 }
 
 bool attn_mma_supported(const tls_shape& s) {
@@ -383,10 +516,31 @@ int attn_mma_plan(int rows, int k, int* chunks_per_row, int* n_items, int* n_cta
   return max_part;
 }
 
+// Cluster size of the cluster form for `rows` rows: the largest of 8, 4, 2
+// whose grid (rows x CL CTAs) fills between one and two CTAs per SM; 0 when
+// none does (few rows: the persistent form spreads them over every SM; many
+// rows: one CTA per row and split would not help either).
+int attn_mma_cluster_size(int rows) {
+  for (int cl = 8; cl >= 2; cl /= 2) {
+    const int64_t ctas = (int64_t)rows * cl;
+    if (ctas >= kNumSMs && ctas <= 2 * (int64_t)kNumSMs) return cl;
+  }
+  return 0;
+}
+
 template <int NS>
-static tls_status launch_mma(const AttnParams& p, cudaStream_t stream) {
+static tls_status launch_mma(const AttnParams& p, int rows, cudaStream_t stream) {
   const MmaLayout L = mma_layout(p.group);
   const size_t smem = 128 + (size_t)L.bytes;
+  const int cl = attn_mma_cluster_size(rows);
+  if (cl > 0) {
+    cudaError_t e = cudaFuncSetAttribute(sparse_attn_mma_cluster_kernel<NS>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_check(e, "sparse_decode_attn: set smem attribute");
+    return cuda_check(launch_pdl_cluster(sparse_attn_mma_cluster_kernel<NS>, dim3(cl, rows), dim3(kMmaWarps * 32),
+                                         smem, stream, (unsigned)cl, p),
+                      "sparse_decode_attn: mma cluster launch");
+  }
   cudaError_t e =
       cudaFuncSetAttribute(sparse_attn_mma_kernel<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return cuda_check(e, "sparse_decode_attn: set smem attribute");
@@ -394,8 +548,8 @@ static tls_status launch_mma(const AttnParams& p, cudaStream_t stream) {
                     "sparse_decode_attn: mma launch");
 }
 
-tls_status launch_attn_mma(const AttnParams& p, cudaStream_t stream) {
-  return launch_mma<3>(p, stream);
+tls_status launch_attn_mma(const AttnParams& p, int rows, cudaStream_t stream) {
+  return launch_mma<3>(p, rows, stream);
 }
 
 }  // namespace tls

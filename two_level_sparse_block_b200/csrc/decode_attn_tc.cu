@@ -90,7 +90,7 @@ __global__ void __launch_bounds__(128, 1) sparse_attn_tc_kernel(AttnParams p) {
     const int t = (int)(it % T) * kAttnTile + tid;
     if (t >= p.k_sel) return -1;
     const int64_t tok =
-        min(max((int64_t)__ldg(p.token_idx + (int64_t)row * p.k_sel + t), (int64_t)0), p.ctx_len - 1);
+        min(max((int64_t)__ldcg(p.token_idx + (int64_t)row * p.k_sel + t), (int64_t)0), p.ctx_len - 1);
     if (p.slot_of_block != nullptr) {
       const int64_t slot = min(max(__ldg(p.slot_of_block + (int64_t)row * p.nb + tok / p.bs), 0), p.n_slots - 1);
       return slot * p.bs + tok % p.bs;

@@ -82,7 +82,10 @@ __device__ __forceinline__ void load_qlab(const TokenParams& p, int row, float* 
 // address outside the index, copied to shared memory.
 template <int NT>
 __device__ __forceinline__ void load_block_list(const TokenParams& p, int row, int32_t* sb) {
-  for (int i = threadIdx.x; i < p.K_b; i += NT) sb[i] = min(max(p.block_idx[(int64_t)row * p.K_b + i], 0), p.nb - 1);
+  // L2 loads: the list is written by the preceding kernel while this grid may
+  // already be resident (programmatic dependent launch)
+  for (int i = threadIdx.x; i < p.K_b; i += NT)
+    sb[i] = min(max(__ldcg(p.block_idx + (int64_t)row * p.K_b + i), 0), p.nb - 1);
 }
 
 // Scores of candidates [c0, c1) of one row (candidates in ascending token

@@ -43,7 +43,7 @@ __global__ void __launch_bounds__(NT) token_select_kernel(TokenParams p) {
   const int c1 = min(p.n_cand, c0 + p.chunk);
   float* out = p.tscore + (int64_t)row * p.n_cand;
   for (int i = c0 + tid; i < c1; i += NT) {
-    const int64_t blk = min(max(bidx[i / p.bs], 0), p.nb - 1);  // clamped: never out of bounds
+    const int64_t blk = min(max(__ldcg(bidx + i / p.bs), 0), p.nb - 1);  // clamped: never out of bounds
     const int64_t tok = blk * p.bs + (i % p.bs);
     const int64_t at = (int64_t)row * p.ctx_len + tok;
     float c[R];
