@@ -10,12 +10,8 @@
 
 namespace tls {
 
-void fill_token_params(TokenParams& p, const tls_shape& s, const void* q, const int32_t* label_ch,
-                       const uint8_t* codes, const float* scales, const int32_t* block_idx, int K_b, int k,
-                       int32_t* token_idx, float* token_score, uint8_t* ws, const WsLayout& L);
 tls_status select_blocks_impl(const tls_shape& s, const void* q, const void* meta, int K_b, int32_t* block_idx,
-                              float* block_score, uint8_t* ws, const WsLayout& L, cudaStream_t stream,
-                              const TokenParams* fuse = nullptr, bool* fused = nullptr);
+                              float* block_score, uint8_t* ws, const WsLayout& L, cudaStream_t stream);
 tls_status select_tokens_impl(const tls_shape& s, const void* q, const int32_t* label_ch, const uint8_t* codes,
                               const float* scales, const int32_t* block_idx, int K_b, int k, int32_t* token_idx,
                               float* token_score, uint8_t* ws, const WsLayout& L, cudaStream_t stream,
@@ -262,12 +258,8 @@ static tls_status select_impl(const tls_shape* shape, const void* q, const void*
   WsLayout L;
   st = check_ws(*shape, K_b, k, ws, ws_bytes, &L);
   if (st != TLS_OK) return st;
-  TokenParams tp;
-  fill_token_params(tp, *shape, q, label_ch, codes, scales, block_idx, K_b, k, token_idx, nullptr, (uint8_t*)ws, L);
-  bool fused = false;
-  st = select_blocks_impl(*shape, q, meta, K_b, block_idx, nullptr, (uint8_t*)ws, L, (cudaStream_t)stream, &tp,
-                          &fused);
-  if (st != TLS_OK || fused) return st;
+  st = select_blocks_impl(*shape, q, meta, K_b, block_idx, nullptr, (uint8_t*)ws, L, (cudaStream_t)stream);
+  if (st != TLS_OK) return st;
   return select_tokens_impl(*shape, q, label_ch, codes, scales, block_idx, K_b, k, token_idx, nullptr,
                             (uint8_t*)ws, L, (cudaStream_t)stream, /*pdl=*/true);
 }

@@ -28,9 +28,11 @@
 #include <cstring>
 #include <mutex>
 
+#include <cooperative_groups.h>
+
+#include "cluster_topk.cuh"
 #include "device_common.cuh"
 #include "host_common.h"
-#include "token_common.cuh"
 
 namespace tls {
 
@@ -48,8 +50,6 @@ struct BlockScoreParams {
   unsigned* counters;  // workspace [rows]
   int32_t* block_idx;  // [rows, K_b]
   int* err;            // workspace error word
-  int fuse_tokens;     // the last CTA of a row goes on to level 2 (token selection)
-  TokenParams tok;
 };
 
 __device__ __forceinline__ uint32_t relu_bf16x2(uint32_t w) {
@@ -69,24 +69,26 @@ struct BsSmem {
 };
 
 // Shared-memory bytes the body of a block-score CTA needs: the pipeline
-// stages, or the top-K_b keys, or (fused) the level-2 scores of one row.
-__host__ __device__ inline int bs_body_bytes(int stage_bytes, int nb, int tok_bytes) {
-  int body = stage_bytes;
-  const int sel = nb * 4 + (int)sizeof(TopkScratch);
-  if (sel > body) body = sel;
-  if (tok_bytes > body) body = tok_bytes;
-  return body;
+// stages, which the selection reuses once the MMAs are done (this CTA's
+// keys, the row's keys for a one-CTA selection, the selection scratch).
+template <int CL>
+__host__ __device__ inline int bs_body_bytes(int stage_bytes, int nb) {
+  int sel = (kBsTile + nb) * 4 + (int)sizeof(TopkScratch);
+  if constexpr (CL >= 2) sel += (int)sizeof(ClusterTopkScratch<CL>) + 16;
+  return stage_bytes > sel ? stage_bytes : sel;
 }
 
-template <int NPAD, int RT>
+// CL: how the row's top-K_b is taken.  1: the row is one tile, its CTA
+// selects; 2, 4, 8: the row's CTAs form a cluster and select together over
+// distributed shared memory (cluster_topk.cuh); 0: the last CTA of the row
+// (a ticket) selects from the scores in the workspace.
+template <int NPAD, int CL>
 __global__ void __launch_bounds__(128, 1)
     block_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, BlockScoreParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   using L = BsSmem<NPAD>;
-  const int tok_bytes =
-      RT > 0 && p.fuse_tokens ? (p.group * RT + p.tok.n_cand) * 4 + (int)sizeof(TopkScratch) : 0;
-  const int body = bs_body_bytes(L::STAGE_BYTES, p.nb, tok_bytes);
+  const int body = bs_body_bytes<CL>(L::STAGE_BYTES, p.nb);
   uint8_t* sA = smem;
   uint8_t* sB = smem + kBsStages * L::A_BYTES;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + ((body + 7) & ~7));
@@ -99,6 +101,7 @@ __global__ void __launch_bounds__(128, 1)
   const int row = blockIdx.y, mt = blockIdx.x;
   const int nk = (2 * p.dqk) / kBsChunk;
   constexpr uint32_t kCols = NPAD < 32 ? 32u : (uint32_t)NPAD;
+  if constexpr (CL >= 2) cluster_arrive_relaxed();  // completes once every CTA of the cluster has started
   grid_launch_dependents();  // level 2 may be scheduled now; it waits for this grid before reading
 
   if (tid == 0) {
@@ -196,9 +199,9 @@ __global__ void __launch_bounds__(128, 1)
   bool ok = mbar_wait_bounded(done, 0, kWaitNs) && flags[1] == 0;
   ok = __all_sync(0xffffffffu, ok);
   tc_fence_after();
+  float best = -INFINITY;
   if (ok) {
     const int j = mt * kBsTile + warp * 32 + lane;
-    float best = -INFINITY;
 #pragma unroll
     for (int c0 = 0; c0 < NPAD; c0 += 16) {
       float v[16];
@@ -208,7 +211,7 @@ __global__ void __launch_bounds__(128, 1)
         if (c0 + i < p.group) best = fmaxf(best, v[i]);
     }
     if (j < p.nb) {
-      p.agg[(int64_t)row * p.nb + j] = best;
+      if (CL == 0) p.agg[(int64_t)row * p.nb + j] = best;
       if (p.block_score != nullptr) p.block_score[(int64_t)row * p.nb + j] = best;
     }
   } else if (lane == 0) {
@@ -221,28 +224,54 @@ __global__ void __launch_bounds__(128, 1)
     tmem_dealloc(tmem, kCols);
   }
 
-  // Last CTA of this row selects the top-K_b blocks.
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    unsigned prev = atomicInc(&p.counters[row], gridDim.x - 1);
-    flags[0] = (prev == gridDim.x - 1) ? 1 : 0;
-  }
-  __syncthreads();
-  if (flags[0] == 0) return;
-  __threadfence();
-  uint32_t* keys = reinterpret_cast<uint32_t*>(smem);
-  TopkScratch* ts = reinterpret_cast<TopkScratch*>(keys + p.nb);
-  const float* arow = p.agg + (int64_t)row * p.nb;
-  for (int i = tid; i < p.nb; i += 128) keys[i] = float_key(__ldcg(arow + i));
-  __syncthreads();
-  cta_topk_ascending<128>(keys, p.nb, p.K_b, p.block_idx + (int64_t)row * p.K_b, *ts, [](int i) { return i; });
-  if constexpr (RT > 0) {
-    if (p.fuse_tokens) {
-      // level 2 of this row right away: its block list is in global memory,
-      // written by this CTA (visible to the CTA after the barrier)
-      __syncthreads();
-      token_stage<RT, 128>(p.tok, row, reinterpret_cast<float*>(smem));
+  int32_t* out = p.block_idx + (int64_t)row * p.K_b;
+  if constexpr (CL == 0) {
+    // Last CTA of this row selects the top-K_b blocks.
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+      unsigned prev = atomicInc(&p.counters[row], gridDim.x - 1);
+      flags[0] = (prev == gridDim.x - 1) ? 1 : 0;
+    }
+    __syncthreads();
+    if (flags[0] == 0) return;
+    __threadfence();
+    uint32_t* keys = reinterpret_cast<uint32_t*>(smem);
+    TopkScratch* ts = reinterpret_cast<TopkScratch*>(keys + p.nb);
+    const float* arow = p.agg + (int64_t)row * p.nb;
+    for (int i = tid; i < p.nb; i += 128) keys[i] = float_key(__ldcg(arow + i));
+    __syncthreads();
+    cta_topk_ascending<128>(keys, p.nb, p.K_b, out, *ts, [](int i) { return i; });
+  } else {
+    // the drained stages hold the selection: this CTA's keys, then the row's
+    uint32_t* mine = reinterpret_cast<uint32_t*>(smem);  // [kBsTile]
+    uint32_t* all = mine + kBsTile;                       // [nb]
+    TopkScratch* ts = reinterpret_cast<TopkScratch*>(all + p.nb);
+    const int n_loc = min(kBsTile, p.nb - mt * kBsTile);
+    if (tid < n_loc) mine[tid] = float_key(best);
+    __syncthreads();
+    if constexpr (CL == 1) {
+      cta_topk_ascending<128>(mine, n_loc, p.K_b, out, *ts, [](int i) { return i; });
+    } else {
+      namespace cg = cooperative_groups;
+      cg::cluster_group cluster = cg::this_cluster();
+      auto* cts = reinterpret_cast<ClusterTopkScratch<CL>*>((reinterpret_cast<uintptr_t>(ts + 1) + 15) &
+                                                            ~uintptr_t(15));
+      cluster_wait();
+      if (cluster_topk_ascending<128, CL>(mine, n_loc, mt * kBsTile, p.K_b, out, *cts, [](int i) { return i; }))
+        return;
+      // degenerate scores or a crowded threshold bin: the leader gathers the
+      // row's keys through distributed shared memory and selects alone
+      if (mt == 0) {
+        for (int r = 0; r < CL; ++r) {
+          const uint32_t* src = cluster.map_shared_rank(mine, r);
+          const int b0 = r * kBsTile, n = min(kBsTile, p.nb - b0);
+          for (int i = tid; i < n; i += 128) all[b0 + i] = src[i];
+        }
+      }
+      cluster.sync();  // the other CTAs' shared memory may be released after this
+      if (mt != 0) return;
+      cta_topk_ascending<128>(all, p.nb, p.K_b, out, *ts, [](int i) { return i; });
     }
   }
 }
@@ -322,40 +351,39 @@ bool use_simt() {
   return v;
 }
 
-template <int NPAD, int RT>
+template <int NPAD, int CL>
 tls_status launch_tc(const CUtensorMap& tmap, const BlockScoreParams& p, int rows, cudaStream_t stream) {
   using L = BsSmem<NPAD>;
-  const int tok_bytes =
-      RT > 0 && p.fuse_tokens ? (p.group * RT + p.tok.n_cand) * 4 + (int)sizeof(TopkScratch) : 0;
-  const int body = bs_body_bytes(L::STAGE_BYTES, p.nb, tok_bytes);
+  const int body = bs_body_bytes<CL>(L::STAGE_BYTES, p.nb);
   const size_t smem = 1024 + (size_t)((body + 7) & ~7) + (2 * kBsStages + 1) * 8 + 16;
-  cudaError_t e = cudaFuncSetAttribute(block_score_tc_kernel<NPAD, RT>,
+  cudaError_t e = cudaFuncSetAttribute(block_score_tc_kernel<NPAD, CL>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return cuda_check(e, "select_blocks: set smem attribute");
-  dim3 grid((unsigned)((p.nb + kBsTile - 1) / kBsTile), (unsigned)rows);
-  block_score_tc_kernel<NPAD, RT><<<grid, 128, smem, stream>>>(tmap, p);
+  const dim3 grid((unsigned)((p.nb + kBsTile - 1) / kBsTile), (unsigned)rows);
+  if constexpr (CL >= 2)
+    return cuda_check(launch_cluster(block_score_tc_kernel<NPAD, CL>, grid, dim3(128), smem, stream, (unsigned)CL,
+                                     tmap, p),
+                      "select_blocks: block_score_tc launch");
+  block_score_tc_kernel<NPAD, CL><<<grid, 128, smem, stream>>>(tmap, p);
   return launch_check("select_blocks: block_score_tc launch");
 }
 
-template <int RT>
+template <int CL>
 tls_status launch_tc_group(const CUtensorMap& tmap, const BlockScoreParams& p, int rows, cudaStream_t stream) {
   const int g = p.group;
-  if (g <= 16) return launch_tc<16, RT>(tmap, p, rows, stream);
-  if (g <= 32) return launch_tc<32, RT>(tmap, p, rows, stream);
-  if (g <= 64) return launch_tc<64, RT>(tmap, p, rows, stream);
-  if (g <= 128) return launch_tc<128, RT>(tmap, p, rows, stream);
-  if (g <= 256) return launch_tc<256, RT>(tmap, p, rows, stream);
+  if (g <= 16) return launch_tc<16, CL>(tmap, p, rows, stream);
+  if (g <= 32) return launch_tc<32, CL>(tmap, p, rows, stream);
+  if (g <= 64) return launch_tc<64, CL>(tmap, p, rows, stream);
+  if (g <= 128) return launch_tc<128, CL>(tmap, p, rows, stream);
+  if (g <= 256) return launch_tc<256, CL>(tmap, p, rows, stream);
   return fail(TLS_ERR_UNSUPPORTED, "select_blocks: group size %d > 256", g);
 }
 
 }  // namespace
 
-// Level 1; with `fuse` (level-2 parameters of the same call) the last CTA of
-// each row also runs level 2 when it fits one CTA, and *fused says so.
+// Level 1: block scores and the top-K_b of every row.
 tls_status select_blocks_impl(const tls_shape& s, const void* q, const void* meta, int K_b, int32_t* block_idx,
-                              float* block_score, uint8_t* ws, const WsLayout& L, cudaStream_t stream,
-                              const TokenParams* fuse, bool* fused) {
-  if (fused != nullptr) *fused = false;
+                              float* block_score, uint8_t* ws, const WsLayout& L, cudaStream_t stream) {
   const int rows = rows_of(s);
   const int nb = (int)n_blocks(s);
   BlockScoreParams p;
@@ -371,7 +399,6 @@ tls_status select_blocks_impl(const tls_shape& s, const void* q, const void* met
   p.counters = reinterpret_cast<unsigned*>(ws + L.blk_counter);
   p.block_idx = block_idx;
   p.err = reinterpret_cast<int*>(ws + L.err);
-  p.fuse_tokens = 0;
 
   if (use_simt()) {
     const size_t smem = (size_t)p.group * 2 * s.qk_dim * 4 + (size_t)nb * 4 + sizeof(TopkScratch) + 16;
@@ -395,7 +422,12 @@ tls_status select_blocks_impl(const tls_shape& s, const void* q, const void* met
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(TLS_ERR_CUDA, "select_blocks: cuTensorMapEncodeTiled failed (%d)", (int)r);
 
-  (void)fuse;  // level 2 runs in its own cluster kernel: a single CTA per row is too narrow for it
+  // the row's tiles select together when they fit one cluster
+  const int tiles = (nb + kBsTile - 1) / kBsTile;
+  if (tiles == 1) return launch_tc_group<1>(tmap, p, rows, stream);
+  if (tiles == 2) return launch_tc_group<2>(tmap, p, rows, stream);
+  if (tiles == 4) return launch_tc_group<4>(tmap, p, rows, stream);
+  if (tiles == 8) return launch_tc_group<8>(tmap, p, rows, stream);
   return launch_tc_group<0>(tmap, p, rows, stream);
 }
 

@@ -1,5 +1,5 @@
-// Level-2 pieces shared by the token-select kernels and the fused
-// level-1 + level-2 kernel (AsyncTLS, English summary 2.A Stage 2).
+// Level-2 pieces shared by the token-select kernels (AsyncTLS, English
+// summary 2.A Stage 2).
 #pragma once
 
 #include "device_common.cuh"
@@ -129,26 +129,9 @@ __device__ __forceinline__ void score_candidates(const TokenParams& p, int row, 
   }
 }
 
-// The whole of level 2 for one row in one CTA: scores in shared memory, then
-// the deterministic top-k written as ascending token positions.  `smem`
-// holds G*R + K_b + n_cand words plus a TopkScratch.
-template <int R, int NT>
-__device__ void token_stage(const TokenParams& p, int row, float* smem) {
-  float* qlab = smem;  // [G][R]
-  int32_t* bidx = reinterpret_cast<int32_t*>(smem + p.group * R);  // [K_b]
-  uint32_t* keys = reinterpret_cast<uint32_t*>(bidx + p.K_b);
-  TopkScratch* ts = reinterpret_cast<TopkScratch*>(keys + p.n_cand);
-  load_qlab<R, NT>(p, row, qlab);
-  grid_dependency_wait();
-  load_block_list<NT>(p, row, bidx);
-  __syncthreads();
-  score_candidates<R, NT>(p, row, qlab, bidx, 0, p.n_cand, keys);
-  __syncthreads();
-  cta_topk_ascending<NT>(keys, p.n_cand, p.k, p.token_idx + (int64_t)row * p.k, *ts, CandidateToken{bidx, p.bs});
-}
-
-// Whether level 2 of a row is light enough for one CTA (scores in shared memory).
-__host__ __device__ inline bool token_stage_fits(int group, int n_label, int n_cand) {
+// Whether level 2 of a row is light enough for one 4-CTA cluster (the
+// scores of all candidates in shared memory, no device-wide exchange).
+__host__ __device__ inline bool token_cluster_fits(int group, int n_label, int n_cand) {
   return (int64_t)group * n_label * n_cand <= ((int64_t)1 << 20);
 }
 

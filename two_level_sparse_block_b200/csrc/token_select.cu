@@ -189,7 +189,7 @@ tls_status select_tokens_impl(const tls_shape& s, const void* q, const int32_t* 
   p.token_idx = token_idx;
 
   const size_t smem = (size_t)p.group * s.n_label * 4 + (size_t)p.n_cand * 4 + sizeof(TopkScratch) + 16;
-  if (token_stage_fits(p.group, s.n_label, p.n_cand)) {
+  if (token_cluster_fits(p.group, s.n_label, p.n_cand)) {
     const int per = (p.n_cand + kTokCluster - 1) / kTokCluster;
     const size_t csmem = ((size_t)p.group * s.n_label + K_b + per + p.n_cand) * 4 + sizeof(TopkScratch) +
                           sizeof(ClusterTopkScratch<kTokCluster>) + 32;
