@@ -19,8 +19,8 @@
  *   - Pointers named "device" point to GPU memory (cudaMalloc / torch CUDA
  *     tensors); "host" pointers point to CPU memory.  The caller owns every
  *     buffer; the library keeps no pointer after a call returns, except the
- *     handle of tls_block_cache_create, which keeps the pointers given to it
- *     until destroyed.
+ *     handles of tls_block_cache_create and tls_engine_create, which keep the
+ *     pointers given to them until destroyed.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Kernel calls are asynchronous on that stream.
  *   - bf16 is IEEE bfloat16 stored as 16-bit words; all tensors are dense,
@@ -262,8 +262,9 @@ typedef struct tls_block_cache tls_block_cache;
  * slot_k [n_slots, bs, host_k_row_stride] and slot_v [n_slots, bs,
  * host_v_row_stride] (bf16).  slot_table_dev: device int32 [B, Hkv, NB],
  * written by the library (-1 = not resident); the attention kernel reads it
- * through tls_kv_view.slot_of_block.  The handle allocates two small pinned
- * staging tables (B*Hkv*NB int32 each) and nothing on the device.
+ * through tls_kv_view.slot_of_block.  The handle allocates two small mapped
+ * pinned staging buffers (max(B*Hkv*NB, 4*n_slots) int32 each) and nothing
+ * on the device.
  * Any pointer may be NULL only for host-only use of tls_block_cache_plan.
  */
 TLS_API tls_status tls_block_cache_create(const tls_shape* shape, const void* host_k, const void* host_v,
@@ -292,9 +293,13 @@ TLS_API tls_status tls_block_cache_plan(tls_block_cache* cache, const int32_t* n
 /*
  * Incremental prefetch (section 2.B): plans as tls_block_cache_plan, then
  * issues one cudaMemcpyAsync per copied run of blocks (K and V) from host
- * memory into the chosen slots on copy_stream and one copy of the updated
- * slot table.  The caller must order copy_stream after every kernel still
- * reading a slot that may be evicted (the previous step's attention).
+ * memory into the chosen slots on copy_stream, then updates the device slot
+ * table on copy_stream: the first call writes the whole table, later calls
+ * change only the entries of the copied and the evicted blocks (a small
+ * kernel).  Neither touches a slot or an entry of in_use_block_idx_host, so
+ * an attention reading those blocks may run concurrently.  The caller must
+ * order copy_stream after every other kernel still reading a slot that may
+ * be evicted (e.g. the attention of the step before).
  * *n_copied = blocks copied.  Setting the environment variable
  * TLS_FAULT_INJECT=copy makes the copy step fail with TLS_ERR_COPY before
  * anything is issued (host-side fault injection for tests).
@@ -305,6 +310,66 @@ TLS_API tls_status tls_prefetch_diff(tls_block_cache* cache, const int32_t* new_
 
 /* Copies the host mirror of the slot table (int32 [B, Hkv, NB]) into `table`. */
 TLS_API tls_status tls_block_cache_table(const tls_block_cache* cache, int32_t* table);
+
+/* ------------------------------------------------------------------------
+ * Staggered decode engine over a block cache (section 2.B: staggered
+ * execution with incremental transfer).
+ * ------------------------------------------------------------------------ */
+typedef struct tls_engine tls_engine;
+
+/* Transfer figures of one engine step (see tls_engine_stats). */
+typedef struct tls_engine_step_stats {
+  int64_t step;          /* the step whose transfer T_step these describe; -1 = the prologue (M_{-1}) */
+  int32_t n_copied;      /* blocks copied, summed over rows */
+  int64_t bytes_copied;  /* host -> device bytes of K and V */
+  float copy_ms;         /* copy-stream time of the transfer (block copies and slot-table update) */
+  float exposed_ms;      /* how long the attention of step+1 waited for this transfer past the point it
+                            was otherwise ready to start; -1 when step+1 has not been issued */
+} tls_engine_step_stats;
+
+/*
+ * Creates an engine for one attention layer whose K/V live in `cache` (created
+ * with device buffers).  meta, label_ch, codes, scales: the resident index, as
+ * in tls_select_blocks / tls_select_tokens.  block_idx: device int32
+ * [2, B, Hkv, K_b], the engine's two block lists (M_t and M_{t-1}, alternating).
+ * token_idx: device int32 [B, Hkv, k].  ws/ws_bytes: a workspace of
+ * tls_workspace_bytes(shape, K_b, k) bytes, zero-filled, used by no other call
+ * while the engine lives.  The engine keeps every pointer until destroyed and
+ * allocates two streams, its events and two pinned host copies of a block list.
+ */
+TLS_API tls_status tls_engine_create(const tls_shape* shape, int32_t K_b, int32_t k, const void* meta,
+                             const int32_t* label_ch, const uint8_t* codes, const float* scales,
+                             tls_block_cache* cache, int32_t* block_idx, int32_t* token_idx, void* ws,
+                             size_t ws_bytes, tls_engine** out);
+
+/*
+ * One decode step t with query q (device bf16 [B, Hq, Dqk], ready on
+ * `stream`).  Output as tls_sparse_decode_attn, written on `stream`.  Level 2
+ * and the attention use the blocks chosen at step t-1 (M_{t-1}, resident in
+ * the cache) with q; level 1 chooses M_t from q on the engine's second stream,
+ * and the blocks of M_t not yet resident are copied from host memory on the
+ * engine's copy stream while the attention runs; step t+1's attention waits
+ * for them.  The first step selects M_{-1} from its own q and makes it
+ * resident before attending.  The call waits on the host for level 1 of step
+ * t (to plan the transfer); everything else is asynchronous.  After a failed
+ * step (a copy failure, TLS_ERR_CAPACITY, a launch error) the cache no longer
+ * matches the block lists: every later step returns the same error and the
+ * engine must be destroyed.
+ */
+TLS_API tls_status tls_engine_step(tls_engine* engine, const void* q, int32_t out_dtype, void* out, float* lse,
+                           void* stream);
+
+/* Number of steps taken (-1 for a NULL engine). */
+TLS_API int64_t tls_engine_steps(const tls_engine* engine);
+
+/*
+ * Transfer figures of step `step` (-1 .. steps-1, among the last 255 steps);
+ * waits for the events they need.
+ */
+TLS_API tls_status tls_engine_stats(tls_engine* engine, int64_t step, tls_engine_step_stats* out);
+
+/* Waits for the engine's streams and releases it (not the caller's buffers). */
+TLS_API void tls_engine_destroy(tls_engine* engine);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,161 @@
+"""The staggered engine over an HBM block cache, on the GPU, against the oracle.
+
+Step t: the blocks M_t chosen from q_t (checked against the oracle within the
+tie band), the tokens and the attention of step t within the GPU's M_{t-1}
+with q_t (the oracle's staggered row, re-run on the GPU's sets), and after the
+last step the transfer invariants: every block of M_T is resident, its slot
+holds exactly the host rows of K and V, and the slot table matches the
+cache's host mirror.
+"""
+
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from parity import check_output, check_selection
+
+pytestmark = pytest.mark.gpu
+
+
+def _rt():
+    from two_level_sparse_block_b200 import runtime, tls
+    return runtime, tls
+
+
+def offload(name, **kw):
+    base = dict(name=name, description="small offload shape", batch=1, n_q_heads=16, n_kv_heads=1, qk_dim=128,
+                v_dim=128, v_offset=-1, ctx_len=8192, block_size=64, K_b=16, k=512, n_label=16, seed=31,
+                n_outlier=6, planted_per_row=64, planted_blocks=20, label_from_outliers=True, steps=6,
+                offload=True, n_slots=32, q_drift=0.3)
+    base.update(kw)
+    return synth.WorkloadConfig(**base)
+
+
+ENGINE = [
+    offload("e_g16_persistent"),
+    offload("e_mqa64_tc", n_q_heads=64, seed=32),
+    offload("e_gqa4_cluster", batch=16, n_q_heads=16, n_kv_heads=4, ctx_len=4096, K_b=12, k=384, n_slots=24,
+            seed=33, steps=4),
+]
+
+
+def _dev_q(q_bits):
+    return torch.from_numpy(np.ascontiguousarray(q_bits).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def _rows(cfg, n=3):
+    rows = [(b, h) for b in range(cfg.batch) for h in range(cfg.n_kv_heads)]
+    if len(rows) <= n:
+        return rows
+    rng = np.random.default_rng(cfg.seed)
+    return [rows[0], rows[-1]] + [rows[i] for i in rng.choice(np.arange(1, len(rows) - 1), n - 2, replace=False)]
+
+
+def _orow(cfg, q, K, V, lab, b, h, **kw):
+    g = cfg.group
+    return oracle.decode_row(q[b, h * g:(h + 1) * g], K[b, h], V[b, h], lab[h], cfg.block_size, cfg.K_b, cfg.k,
+                             cfg.softmax_scale, **kw)
+
+
+@pytest.mark.parametrize("cfg", ENGINE, ids=lambda c: c.name)
+def test_engine_follows_the_staggered_oracle(cfg):
+    runtime, tls = _rt()
+    qs = synth.gen_query_trajectory(cfg)
+    K, V, _ = synth.gen_kv(cfg, qs[0])
+    lab = synth.gen_label_channels(cfg)
+    layer = runtime.offloaded_layer_for_config(cfg, K, V, lab)
+    g = cfg.group
+    try:
+        copied = []
+        for t, q in enumerate(qs):
+            layer.step(_dev_q(q))
+            torch.cuda.synchronize()
+            assert layer.check_device_error() == 0
+            m_prev = layer.block_idx[(t + 1) & 1].cpu().numpy()  # M_{t-1} (the prologue's M_{-1} at t = 0)
+            m_cur = layer.block_idx[t & 1].cpu().numpy()         # M_t
+            tok = layer.token_idx.cpu().numpy()
+            out = layer.out.float().cpu().numpy()
+            for b, h in _rows(cfg):
+                where = f"{cfg.name} step {t} row ({b},{h})"
+                # level 1 of step t chooses M_t from q_t
+                r1 = _orow(cfg, q, K, V, lab, b, h)
+                check_selection(m_cur[b, h], r1["agg"], cfg.K_b, where + " M_t")
+                if t == 0:
+                    check_selection(m_prev[b, h], r1["agg"], cfg.K_b, where + " M_-1")
+                # level 2 and attention of step t within the GPU's M_{t-1}, with q_t
+                r2 = _orow(cfg, q, K, V, lab, b, h, block_idx=m_prev[b, h])
+                pos = np.searchsorted(r2["cand"], tok[b, h])
+                assert np.array_equal(r2["cand"][pos], tok[b, h]), f"{where}: token outside M_t-1"
+                check_selection(pos, r2["token_score"], cfg.k, where + " tokens")
+                r3 = _orow(cfg, q, K, V, lab, b, h, block_idx=m_prev[b, h], token_idx=tok[b, h])
+                check_output(out[b, h * g:(h + 1) * g], r3["out"], where + " out")
+            copied.append(m_cur)
+        torch.cuda.synchronize()
+
+        # transfer invariants after the last step
+        table = layer.slot_table.cpu().numpy()
+        mirror = np.empty_like(table)
+        tls.tls_block_cache_table(layer.cache, mirror)
+        assert np.array_equal(table, mirror), "device slot table differs from the host mirror"
+        slot_k = layer.slot_k.view(torch.int16).cpu().numpy().view(np.uint16)
+        slot_v = layer.slot_v.view(torch.int16).cpu().numpy().view(np.uint16)
+        bs = cfg.block_size
+        last = copied[-1]
+        for b in range(cfg.batch):
+            for h in range(cfg.n_kv_heads):
+                for blk in last[b, h]:
+                    s = table[b, h, blk]
+                    assert s >= 0, f"block {blk} of M_T not resident in row ({b},{h})"
+                    assert np.array_equal(slot_k[s], K[b, h, blk * bs:(blk + 1) * bs]), "slot K differs"
+                    assert np.array_equal(slot_v[s], V[b, h, blk * bs:(blk + 1) * bs]), "slot V differs"
+        # occupancy: no slot holds two blocks
+        used = table[table >= 0]
+        assert used.size == np.unique(used).size
+
+        # transfer figures: the prologue copies all of M_{-1}; later steps copy T_t = M_t \ C_t
+        st = layer.stats(-1)
+        assert st.n_copied == cfg.rows * cfg.K_b and st.copy_ms >= 0.0
+        blk_bytes = cfg.block_size * (cfg.qk_dim + cfg.v_dim) * 2
+        for t in range(len(qs) - 1):
+            st = layer.stats(t)
+            assert 0 <= st.n_copied <= cfg.rows * cfg.K_b
+            assert st.bytes_copied == st.n_copied * blk_bytes
+            assert st.copy_ms >= 0.0 and st.exposed_ms >= 0.0
+        assert layer.stats(len(qs) - 1).exposed_ms == -1.0  # no later step has been issued
+    finally:
+        layer.close()
+
+
+def test_engine_copy_failure_is_reported_and_sticks(monkeypatch):
+    # host-side fault injection: the transfer of step 2 fails before anything
+    # is issued; that step and every later one return TLS_ERR_COPY, and the
+    # device stays healthy
+    runtime, tls = _rt()
+    cfg = ENGINE[0]
+    qs = synth.gen_query_trajectory(cfg, 4)
+    K, V, _ = synth.gen_kv(cfg, qs[0])
+    lab = synth.gen_label_channels(cfg)
+    layer = runtime.offloaded_layer_for_config(cfg, K, V, lab)
+    try:
+        layer.step(_dev_q(qs[0]))
+        layer.step(_dev_q(qs[1]))
+        monkeypatch.setenv("TLS_FAULT_INJECT", "copy")
+        with pytest.raises(tls.TlsError) as e:
+            layer.step(_dev_q(qs[2]))
+        assert e.value.status == tls.TLS_ERR_COPY
+        monkeypatch.delenv("TLS_FAULT_INJECT")
+        with pytest.raises(tls.TlsError) as e2:
+            layer.step(_dev_q(qs[3]))
+        assert e2.value.status == tls.TLS_ERR_COPY
+        assert layer.steps_taken() == 2
+        torch.cuda.synchronize()
+        assert layer.check_device_error() == 0
+    finally:
+        layer.close()
+    # the device still runs work after the engine is gone
+    x = torch.ones(1024, device="cuda")
+    assert float(x.sum()) == 1024.0

@@ -5,7 +5,11 @@
 // Host state: a mirror of the device slot table (block -> slot), the owner
 // of every slot and its last use.  Planning is pure host code; the prefetch
 // issues one cudaMemcpyAsync per run of blocks that are adjacent both in host
-// memory and in the slot pool, then one copy of the slot table.
+// memory and in the slot pool, then updates the device slot table.  The first
+// transfer writes the whole table (nothing is resident, so nothing reads it);
+// later ones change only the entries of the copied and the evicted blocks,
+// which the running attention (reading M_{t-1}) never reads, so the update
+// may run concurrently with it.
 
 #include <algorithm>
 #include <cstdlib>
@@ -29,9 +33,11 @@ struct tls_block_cache {
   std::vector<int64_t> owner;       // [n_slots] -> row * nb + block, or -1
   std::vector<int64_t> last_use;    // [n_slots] planning step of the last use
   int64_t step = 0;
-  int32_t* staging[2] = {nullptr, nullptr};  // pinned copies of the table
+  int32_t* staging[2] = {nullptr, nullptr};  // pinned, mapped: the first table, then (entry, value) pairs
   cudaEvent_t staged[2] = {nullptr, nullptr};
   int cur = 0;
+  bool published = false;                     // the device table has been written once
+  std::vector<int2> changes;                  // this plan's (entry, value) table changes
 };
 
 namespace tls {
@@ -95,12 +101,17 @@ tls_status plan(const tls_block_cache& c, const int32_t* new_idx, const int32_t*
 void commit(tls_block_cache& c, const int32_t* new_idx, int K_b, std::vector<Copy>& copies,
             const std::vector<int32_t>& victims) {
   c.step += 1;
+  c.changes.clear();
   for (size_t i = 0; i < copies.size(); ++i) {
     const int32_t s = victims[i];
-    if (c.owner[s] >= 0) c.table[c.owner[s]] = -1;
+    if (c.owner[s] >= 0) {
+      c.table[c.owner[s]] = -1;
+      c.changes.push_back(make_int2((int)c.owner[s], -1));
+    }
     const int64_t key = (int64_t)copies[i].row * c.nb + copies[i].block;
     c.owner[s] = key;
     c.table[key] = s;
+    c.changes.push_back(make_int2((int)key, s));
     copies[i].slot = s;
   }
   for (int r = 0; r < c.rows; ++r)
@@ -110,7 +121,87 @@ void commit(tls_block_cache& c, const int32_t* new_idx, int K_b, std::vector<Cop
     }
 }
 
+// Applies (entry, value) pairs (mapped pinned memory) to the device slot table.
+__global__ void slot_table_update_kernel(int32_t* table, const int2* pairs, int n) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    const int2 pr = pairs[i];
+    table[pr.x] = pr.y;
+  }
+}
+
 }  // namespace
+
+// The incremental prefetch of tls_prefetch_diff without the argument checks
+// (also used by the staggered engine).  *bytes = host -> device bytes of the
+// block copies.
+tls_status prefetch_diff_impl(tls_block_cache* c, const int32_t* new_idx, const int32_t* in_use, int K_b,
+                              cudaStream_t cs, int32_t* n_copied, int64_t* bytes) {
+  if (fault_injected_copy()) return fail(TLS_ERR_COPY, "prefetch_diff: copy failure injected (TLS_FAULT_INJECT=copy)");
+  std::vector<Copy> copies;
+  std::vector<int32_t> victims;
+  tls_status st = plan(*c, new_idx, in_use, K_b, &copies, &victims);
+  if (st != TLS_OK) return st;
+  commit(*c, new_idx, K_b, copies, victims);
+
+  const int bs = c->shape.block_size;
+  const int64_t n = c->shape.ctx_len;
+  const size_t kblk = (size_t)bs * c->hk_stride * 2, vblk = (size_t)bs * c->hv_stride * 2;
+  const bool with_v = c->host_v != nullptr && c->slot_v != nullptr;
+  size_t i = 0;
+  while (i < copies.size()) {
+    size_t j = i + 1;
+    while (j < copies.size() && copies[j].row == copies[i].row &&
+           copies[j].block == copies[j - 1].block + 1 && copies[j].slot == copies[j - 1].slot + 1)
+      ++j;
+    const size_t len = j - i;
+    const int64_t tok0 = (int64_t)copies[i].row * n + (int64_t)copies[i].block * bs;
+    cudaError_t e = cudaMemcpyAsync(c->slot_k + (size_t)copies[i].slot * kblk,
+                                    c->host_k + (size_t)tok0 * c->hk_stride * 2, len * kblk,
+                                    cudaMemcpyHostToDevice, cs);
+    if (e == cudaSuccess && with_v)
+      e = cudaMemcpyAsync(c->slot_v + (size_t)copies[i].slot * vblk, c->host_v + (size_t)tok0 * c->hv_stride * 2,
+                          len * vblk, cudaMemcpyHostToDevice, cs);
+    if (e != cudaSuccess) return fail(TLS_ERR_COPY, "prefetch_diff: block copy failed: %s", cudaGetErrorString(e));
+    i = j;
+  }
+  // publish the table: whole the first time, afterwards only the changed entries
+  const int b = c->cur;
+  cudaError_t e = cudaEventSynchronize(c->staged[b]);  // the staging buffer's previous use is done
+  if (e != cudaSuccess) return cuda_check(e, "prefetch_diff: staging wait");
+  if (!c->published) {
+    std::memcpy(c->staging[b], c->table.data(), c->table.size() * sizeof(int32_t));
+    e = cudaMemcpyAsync(c->table_dev, c->staging[b], c->table.size() * sizeof(int32_t), cudaMemcpyHostToDevice, cs);
+    c->published = true;
+  } else if (!c->changes.empty()) {
+    int2* pairs = reinterpret_cast<int2*>(c->staging[b]);
+    std::memcpy(pairs, c->changes.data(), c->changes.size() * sizeof(int2));
+    const int n_pairs = (int)c->changes.size();
+    slot_table_update_kernel<<<(n_pairs + 255) / 256, 256, 0, cs>>>(c->table_dev, pairs, n_pairs);
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess) e = cudaEventRecord(c->staged[b], cs);
+  if (e != cudaSuccess) return fail(TLS_ERR_COPY, "prefetch_diff: slot table update failed: %s", cudaGetErrorString(e));
+  c->cur ^= 1;
+  *n_copied = (int32_t)copies.size();
+  if (bytes != nullptr) *bytes = (int64_t)copies.size() * (int64_t)(kblk + (with_v ? vblk : 0));
+  return TLS_OK;
+}
+
+// The attention's view of the slot pool of a cache created with device buffers.
+tls_status block_cache_view(const tls_block_cache* c, tls_kv_view* kv) {
+  if (c->slot_k == nullptr || c->table_dev == nullptr || c->host_k == nullptr)
+    return fail(TLS_ERR_INVALID_ARG, "block cache was created without device buffers");
+  const bool own_v = c->shape.v_offset < 0;
+  if (own_v && c->slot_v == nullptr) return fail(TLS_ERR_INVALID_ARG, "block cache has no V slots");
+  kv->k = c->slot_k;
+  kv->v = own_v ? c->slot_v : c->slot_k;
+  kv->k_row_stride = c->hk_stride;
+  kv->v_row_stride = own_v ? c->hv_stride : c->hk_stride;
+  kv->slot_of_block = c->table_dev;
+  kv->n_slots = c->n_slots;
+  return TLS_OK;
+}
+
 }  // namespace tls
 
 using namespace tls;
@@ -144,8 +235,11 @@ extern "C" tls_status tls_block_cache_create(const tls_shape* shape, const void*
   c->owner.assign(n_slots, -1);
   c->last_use.assign(n_slots, 0);
   if (slot_table_dev != nullptr) {
+    // a plan changes at most two entries per copied block and copies at most n_slots blocks
+    const size_t words = std::max(c->table.size(), (size_t)4 * (size_t)n_slots);
     for (int i = 0; i < 2; ++i) {
-      cudaError_t e = cudaHostAlloc((void**)&c->staging[i], c->table.size() * sizeof(int32_t), cudaHostAllocDefault);
+      cudaError_t e = cudaHostAlloc((void**)&c->staging[i], words * sizeof(int32_t),
+                                    cudaHostAllocMapped | cudaHostAllocPortable);
       if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->staged[i], cudaEventDisableTiming);
       if (e != cudaSuccess) {
         tls_block_cache_destroy(c);
@@ -199,45 +293,8 @@ extern "C" tls_status tls_prefetch_diff(tls_block_cache* c, const int32_t* new_b
   if (c->host_k == nullptr || c->slot_k == nullptr || c->table_dev == nullptr)
     return fail(TLS_ERR_INVALID_ARG, "prefetch_diff: cache was created without device buffers");
   if (K_b < 1 || K_b > c->nb) return fail(TLS_ERR_INVALID_ARG, "prefetch_diff: K_b out of range");
-  if (fault_injected_copy()) return fail(TLS_ERR_COPY, "prefetch_diff: copy failure injected (TLS_FAULT_INJECT=copy)");
-  std::vector<Copy> copies;
-  std::vector<int32_t> victims;
-  tls_status st = plan(*c, new_block_idx_host, in_use_block_idx_host, K_b, &copies, &victims);
-  if (st != TLS_OK) return st;
-  commit(*c, new_block_idx_host, K_b, copies, victims);
-
-  cudaStream_t cs = (cudaStream_t)copy_stream;
-  const int bs = c->shape.block_size;
-  const int64_t n = c->shape.ctx_len;
-  const size_t kblk = (size_t)bs * c->hk_stride * 2, vblk = (size_t)bs * c->hv_stride * 2;
-  size_t i = 0;
-  while (i < copies.size()) {
-    size_t j = i + 1;
-    while (j < copies.size() && copies[j].row == copies[i].row &&
-           copies[j].block == copies[j - 1].block + 1 && copies[j].slot == copies[j - 1].slot + 1)
-      ++j;
-    const size_t len = j - i;
-    const int64_t tok0 = (int64_t)copies[i].row * n + (int64_t)copies[i].block * bs;
-    cudaError_t e = cudaMemcpyAsync(c->slot_k + (size_t)copies[i].slot * kblk,
-                                    c->host_k + (size_t)tok0 * c->hk_stride * 2, len * kblk,
-                                    cudaMemcpyHostToDevice, cs);
-    if (e == cudaSuccess && c->host_v != nullptr && c->slot_v != nullptr)
-      e = cudaMemcpyAsync(c->slot_v + (size_t)copies[i].slot * vblk, c->host_v + (size_t)tok0 * c->hv_stride * 2,
-                          len * vblk, cudaMemcpyHostToDevice, cs);
-    if (e != cudaSuccess) return fail(TLS_ERR_COPY, "prefetch_diff: block copy failed: %s", cudaGetErrorString(e));
-    i = j;
-  }
-  // publish the new slot table through a pinned staging copy
-  const int b = c->cur;
-  cudaError_t e = cudaEventSynchronize(c->staged[b]);
-  if (e != cudaSuccess) return cuda_check(e, "prefetch_diff: staging wait");
-  std::memcpy(c->staging[b], c->table.data(), c->table.size() * sizeof(int32_t));
-  e = cudaMemcpyAsync(c->table_dev, c->staging[b], c->table.size() * sizeof(int32_t), cudaMemcpyHostToDevice, cs);
-  if (e == cudaSuccess) e = cudaEventRecord(c->staged[b], cs);
-  if (e != cudaSuccess) return fail(TLS_ERR_COPY, "prefetch_diff: slot table copy failed: %s", cudaGetErrorString(e));
-  c->cur ^= 1;
-  *n_copied = (int32_t)copies.size();
-  return TLS_OK;
+  return prefetch_diff_impl(c, new_block_idx_host, in_use_block_idx_host, K_b, (cudaStream_t)copy_stream, n_copied,
+                            nullptr);
 }
 
 extern "C" tls_status tls_block_cache_table(const tls_block_cache* c, int32_t* table) {

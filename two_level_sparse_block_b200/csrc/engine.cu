@@ -1,0 +1,244 @@
+// Staggered decode engine over an HBM block cache (AsyncTLS, English summary
+// 2.B; Italian 2.B; Japanese 2.B): step t selects its tokens and attends
+// within the blocks chosen at step t-1 (M_{t-1}, already resident), while
+// level 1 chooses M_t on a second stream; only the blocks of M_t that are not
+// resident, T_t = M_t \ C_t, cross PCIe on a copy stream, overlapping step
+// t's attention, and must land before step t+1 attends.
+//
+// Streams: the caller's stream A runs level 2 and the attention; the engine's
+// stream B runs level 1 and the device -> host copy of M_t; stream C copies
+// blocks and updates the slot table.  Per step t (cur = t & 1 holds M_t):
+//   A: event q_t; level 2 over M_{t-1}; event ready_t; wait copy_end_{t-1};
+//      attention over the slot pool; event attn_t
+//   B: wait q_t; level 1 -> M_t; M_t -> pinned host; event sel_t
+//   host: wait sel_t, plan T_t against C_t with M_{t-1} kept (host mirror)
+//   C: wait attn_{t-1} (its slots may be victims now); event copy_start_t;
+//      block copies; slot-table update; event copy_end_t
+// The table update changes only entries of copied and evicted blocks, none of
+// which step t's attention reads, so C may run alongside it.
+
+#include <vector>
+
+#include "host_common.h"
+
+namespace tls {
+tls_status plan_workspace(const tls_shape& s, int K_b, int k, WsLayout* out);
+tls_status select_blocks_impl(const tls_shape& s, const void* q, const void* meta, int K_b, int32_t* block_idx,
+                              float* block_score, uint8_t* ws, const WsLayout& L, cudaStream_t stream);
+tls_status select_tokens_impl(const tls_shape& s, const void* q, const int32_t* label_ch, const uint8_t* codes,
+                              const float* scales, const int32_t* block_idx, int K_b, int k, int32_t* token_idx,
+                              float* token_score, uint8_t* ws, const WsLayout& L, cudaStream_t stream,
+                              bool pdl = false);
+tls_status sparse_attn_impl(const tls_shape& s, const void* q, const tls_kv_view& kv, const int32_t* token_idx,
+                            int k, int out_dtype, void* out, float* lse, uint8_t* ws, const WsLayout& L,
+                            cudaStream_t stream);
+tls_status prefetch_diff_impl(tls_block_cache* c, const int32_t* new_idx, const int32_t* in_use, int K_b,
+                              cudaStream_t cs, int32_t* n_copied, int64_t* bytes);
+tls_status block_cache_view(const tls_block_cache* c, tls_kv_view* kv);
+}  // namespace tls
+
+namespace {
+constexpr int kRing = 256;  // steps whose timing events are kept
+}
+
+struct tls_engine {
+  tls_shape shape;
+  int K_b = 0, k = 0, rows = 0;
+  const void* meta = nullptr;
+  const int32_t* label_ch = nullptr;
+  const uint8_t* codes = nullptr;
+  const float* scales = nullptr;
+  tls_block_cache* cache = nullptr;
+  tls_kv_view kv;
+  uint8_t* ws = nullptr;
+  tls::WsLayout L;
+  int32_t* bidx[2] = {nullptr, nullptr};       // caller's device [rows, K_b] x 2
+  int32_t* token_idx = nullptr;                // caller's device [rows, k]
+  int32_t* host_bidx[2] = {nullptr, nullptr};  // pinned mirrors of bidx
+  cudaStream_t sel = nullptr, copy = nullptr;
+  cudaEvent_t ev_q = nullptr, ev_sel = nullptr, ev_attn[2] = {nullptr, nullptr};
+  cudaEvent_t ready[kRing] = {}, copy_start[kRing] = {}, copy_end[kRing] = {};
+  int32_t n_copied[kRing] = {};
+  int64_t bytes[kRing] = {};
+  int64_t t = 0;
+  tls_status failed = TLS_OK;
+};
+
+using namespace tls;
+
+namespace {
+
+void release(tls_engine* e) {
+  if (e->sel != nullptr) cudaStreamSynchronize(e->sel);
+  if (e->copy != nullptr) cudaStreamSynchronize(e->copy);
+  for (cudaEvent_t* ev : {&e->ev_q, &e->ev_sel, &e->ev_attn[0], &e->ev_attn[1]})
+    if (*ev != nullptr) cudaEventDestroy(*ev);
+  for (int i = 0; i < kRing; ++i)
+    for (cudaEvent_t ev : {e->ready[i], e->copy_start[i], e->copy_end[i]})
+      if (ev != nullptr) cudaEventDestroy(ev);
+  for (int i = 0; i < 2; ++i)
+    if (e->host_bidx[i] != nullptr) cudaFreeHost(e->host_bidx[i]);
+  if (e->sel != nullptr) cudaStreamDestroy(e->sel);
+  if (e->copy != nullptr) cudaStreamDestroy(e->copy);
+  delete e;
+}
+
+}  // namespace
+
+extern "C" tls_status tls_engine_create(const tls_shape* shape, int32_t K_b, int32_t k, const void* meta,
+                                        const int32_t* label_ch, const uint8_t* codes, const float* scales,
+                                        tls_block_cache* cache, int32_t* block_idx, int32_t* token_idx, void* ws,
+                                        size_t ws_bytes, tls_engine** out) {
+  clear_error();
+  tls_status st = check_shape(shape);
+  if (st != TLS_OK) return st;
+  if (out == nullptr || meta == nullptr || label_ch == nullptr || codes == nullptr || scales == nullptr ||
+      cache == nullptr || block_idx == nullptr || token_idx == nullptr)
+    return fail(TLS_ERR_INVALID_ARG, "engine_create: NULL argument");
+  if (!aligned16(meta) || !aligned16(codes)) return fail(TLS_ERR_INVALID_ARG, "engine_create: meta/codes not 16-byte aligned");
+  WsLayout L;
+  st = plan_workspace(*shape, K_b, k, &L);
+  if (st != TLS_OK) return st;
+  if (ws == nullptr || !aligned16(ws)) return fail(TLS_ERR_INVALID_ARG, "engine_create: workspace NULL or not 16-byte aligned");
+  if (ws_bytes < L.total) return fail(TLS_ERR_INVALID_ARG, "engine_create: workspace %zu bytes < required %zu", ws_bytes, L.total);
+  tls_kv_view kv;
+  st = block_cache_view(cache, &kv);
+  if (st != TLS_OK) return st;
+
+  auto* e = new tls_engine();
+  e->shape = *shape;
+  e->K_b = K_b;
+  e->k = k;
+  e->rows = rows_of(*shape);
+  e->meta = meta;
+  e->label_ch = label_ch;
+  e->codes = codes;
+  e->scales = scales;
+  e->cache = cache;
+  e->kv = kv;
+  e->ws = (uint8_t*)ws;
+  e->L = L;
+  e->bidx[0] = block_idx;
+  e->bidx[1] = block_idx + (size_t)e->rows * K_b;
+  e->token_idx = token_idx;
+  cudaError_t ce = cudaSuccess;
+  for (int i = 0; i < 2 && ce == cudaSuccess; ++i)
+    ce = cudaHostAlloc((void**)&e->host_bidx[i], (size_t)e->rows * K_b * sizeof(int32_t), cudaHostAllocDefault);
+  if (ce == cudaSuccess) ce = cudaStreamCreateWithFlags(&e->sel, cudaStreamNonBlocking);
+  if (ce == cudaSuccess) ce = cudaStreamCreateWithFlags(&e->copy, cudaStreamNonBlocking);
+  for (cudaEvent_t* ev : {&e->ev_q, &e->ev_sel, &e->ev_attn[0], &e->ev_attn[1]})
+    if (ce == cudaSuccess) ce = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+  for (int i = 0; i < kRing && ce == cudaSuccess; ++i) {
+    ce = cudaEventCreate(&e->ready[i]);
+    if (ce == cudaSuccess) ce = cudaEventCreate(&e->copy_start[i]);
+    if (ce == cudaSuccess) ce = cudaEventCreate(&e->copy_end[i]);
+  }
+  if (ce != cudaSuccess) {
+    release(e);
+    return cuda_check(ce, "engine_create: streams, events or pinned mirrors");
+  }
+  *out = e;
+  return TLS_OK;
+}
+
+extern "C" void tls_engine_destroy(tls_engine* e) {
+  if (e != nullptr) release(e);
+}
+
+namespace {
+
+tls_status engine_step(tls_engine* e, const void* q, int32_t out_dtype, void* out, float* lse, cudaStream_t A) {
+  const tls_shape& s = e->shape;
+  const size_t list_bytes = (size_t)e->rows * e->K_b * sizeof(int32_t);
+  const int cur = (int)(e->t & 1), prev = cur ^ 1;
+  const int ri = (int)(e->t % kRing), rp = (int)((e->t + kRing - 1) % kRing);
+  tls_status st;
+  if (e->t == 0) {
+    // prologue: M_{-1} from q_0, made resident before the first attention
+    st = select_blocks_impl(s, q, e->meta, e->K_b, e->bidx[prev], nullptr, e->ws, e->L, A);
+    if (st != TLS_OK) return st;
+    cudaError_t ce = cudaMemcpyAsync(e->host_bidx[prev], e->bidx[prev], list_bytes, cudaMemcpyDeviceToHost, A);
+    if (ce == cudaSuccess) ce = cudaStreamSynchronize(A);
+    if (ce == cudaSuccess) ce = cudaEventRecord(e->copy_start[rp], e->copy);
+    if (ce != cudaSuccess) return cuda_check(ce, "engine_step: prologue");
+    st = prefetch_diff_impl(e->cache, e->host_bidx[prev], nullptr, e->K_b, e->copy, &e->n_copied[rp], &e->bytes[rp]);
+    if (st != TLS_OK) return st;
+    ce = cudaEventRecord(e->copy_end[rp], e->copy);
+    if (ce != cudaSuccess) return cuda_check(ce, "engine_step: prologue");
+  }
+  // level 1 for q_t on the select stream: M_t
+  cudaError_t ce = cudaEventRecord(e->ev_q, A);
+  if (ce == cudaSuccess) ce = cudaStreamWaitEvent(e->sel, e->ev_q, 0);
+  if (ce != cudaSuccess) return cuda_check(ce, "engine_step: select stream");
+  st = select_blocks_impl(s, q, e->meta, e->K_b, e->bidx[cur], nullptr, e->ws, e->L, e->sel);
+  if (st != TLS_OK) return st;
+  ce = cudaMemcpyAsync(e->host_bidx[cur], e->bidx[cur], list_bytes, cudaMemcpyDeviceToHost, e->sel);
+  if (ce == cudaSuccess) ce = cudaEventRecord(e->ev_sel, e->sel);
+  if (ce != cudaSuccess) return cuda_check(ce, "engine_step: block list to host");
+  // level 2 within M_{t-1} and the attention over the slot pool, on A
+  st = select_tokens_impl(s, q, e->label_ch, e->codes, e->scales, e->bidx[prev], e->K_b, e->k, e->token_idx, nullptr,
+                          e->ws, e->L, A, /*pdl=*/false);
+  if (st != TLS_OK) return st;
+  ce = cudaEventRecord(e->ready[ri], A);
+  if (ce == cudaSuccess) ce = cudaStreamWaitEvent(A, e->copy_end[rp], 0);  // T_{t-1} has landed
+  if (ce != cudaSuccess) return cuda_check(ce, "engine_step: wait for the transfer");
+  st = sparse_attn_impl(s, q, e->kv, e->token_idx, e->k, out_dtype, out, lse, e->ws, e->L, A);
+  if (st != TLS_OK) return st;
+  ce = cudaEventRecord(e->ev_attn[cur], A);
+  // T_t = M_t \ C_t on the copy stream, after the attention of step t-1 (its
+  // slots may be evicted now), alongside the attention of step t
+  if (ce == cudaSuccess) ce = cudaEventSynchronize(e->ev_sel);
+  if (ce == cudaSuccess) ce = cudaStreamWaitEvent(e->copy, e->ev_attn[prev], 0);
+  if (ce == cudaSuccess) ce = cudaEventRecord(e->copy_start[ri], e->copy);
+  if (ce != cudaSuccess) return cuda_check(ce, "engine_step: copy stream");
+  st = prefetch_diff_impl(e->cache, e->host_bidx[cur], e->host_bidx[prev], e->K_b, e->copy, &e->n_copied[ri],
+                          &e->bytes[ri]);
+  if (st != TLS_OK) return st;
+  ce = cudaEventRecord(e->copy_end[ri], e->copy);
+  if (ce != cudaSuccess) return cuda_check(ce, "engine_step: copy stream");
+  e->t += 1;
+  return TLS_OK;
+}
+
+}  // namespace
+
+extern "C" tls_status tls_engine_step(tls_engine* e, const void* q, int32_t out_dtype, void* out, float* lse,
+                                      void* stream) {
+  clear_error();
+  if (e == nullptr || q == nullptr || out == nullptr) return fail(TLS_ERR_INVALID_ARG, "engine_step: NULL argument");
+  if (!aligned16(q)) return fail(TLS_ERR_INVALID_ARG, "engine_step: q not 16-byte aligned");
+  if (out_dtype != TLS_OUT_F32 && out_dtype != TLS_OUT_BF16)
+    return fail(TLS_ERR_INVALID_ARG, "engine_step: out_dtype must be TLS_OUT_F32 or TLS_OUT_BF16");
+  if (e->failed != TLS_OK)
+    return fail(e->failed, "engine_step: an earlier step failed; the cache no longer matches the block lists");
+  const tls_status st = engine_step(e, q, out_dtype, out, lse, (cudaStream_t)stream);
+  if (st != TLS_OK) e->failed = st;
+  return st;
+}
+
+extern "C" int64_t tls_engine_steps(const tls_engine* e) { return e == nullptr ? -1 : e->t; }
+
+extern "C" tls_status tls_engine_stats(tls_engine* e, int64_t step, tls_engine_step_stats* out) {
+  clear_error();
+  if (e == nullptr || out == nullptr) return fail(TLS_ERR_INVALID_ARG, "engine_stats: NULL argument");
+  if (step < -1 || step >= e->t || step < e->t - (kRing - 1))
+    return fail(TLS_ERR_INVALID_ARG, "engine_stats: step %lld not among the last %d steps taken",
+                (long long)step, kRing - 1);
+  const int si = (int)((step + kRing) % kRing);
+  cudaError_t ce = cudaEventSynchronize(e->copy_end[si]);
+  float copy_ms = 0.0f, exposed_ms = -1.0f;
+  if (ce == cudaSuccess) ce = cudaEventElapsedTime(&copy_ms, e->copy_start[si], e->copy_end[si]);
+  if (ce == cudaSuccess && step + 1 < e->t) {
+    const int ni = (int)((step + 1) % kRing);
+    ce = cudaEventSynchronize(e->ready[ni]);
+    if (ce == cudaSuccess) ce = cudaEventElapsedTime(&exposed_ms, e->ready[ni], e->copy_end[si]);
+    if (exposed_ms < 0.0f) exposed_ms = 0.0f;
+  }
+  if (ce != cudaSuccess) return cuda_check(ce, "engine_stats: events");
+  out->step = step;
+  out->n_copied = e->n_copied[si];
+  out->bytes_copied = e->bytes[si];
+  out->copy_ms = copy_ms;
+  out->exposed_ms = exposed_ms;
+  return TLS_OK;
+}

@@ -108,3 +108,103 @@ def state_for_config(cfg, q_bits, k_bits, v_bits, label_ch, **kw) -> DecodeState
                        v_dim=cfg.v_dim, v_offset=cfg.v_offset, block_size=cfg.block_size, n_label=cfg.n_label,
                        ctx_len=cfg.ctx_len, K_b=cfg.K_b, k=cfg.k, q_bits=q_bits, k_bits=k_bits, v_bits=v_bits,
                        label_ch=label_ch, softmax_scale=cfg.softmax_scale, **kw)
+
+
+class OffloadedLayer:
+    """One layer whose K/V live in pinned host memory behind an HBM block cache,
+    decoded step by step by the staggered engine (tls_engine_*).
+
+    q_bits are not needed to build it; k_bits / v_bits: uint16 [B, Hkv, N, D]
+    bf16 bit patterns (v_bits None for the MLA latent).  The index (block
+    meta, INT4 label cache) is built on the device from a temporary copy of K,
+    which is released afterwards: only the n_slots-block pool holds K/V in HBM.
+    """
+
+    def __init__(self, *, batch, n_q_heads, n_kv_heads, qk_dim, v_dim, v_offset, block_size, n_label, ctx_len,
+                 K_b, k, n_slots, k_bits, v_bits, label_ch, softmax_scale=None, out_dtype=tls.TLS_OUT_F32,
+                 device="cuda"):
+        dev = torch.device(device)
+        self.device = dev
+        scale = 1.0 / math.sqrt(qk_dim) if softmax_scale is None else softmax_scale
+        self.shape = tls.make_shape(batch, n_q_heads, n_kv_heads, qk_dim, v_dim, v_offset, block_size, n_label,
+                                    ctx_len, scale)
+        self.K_b, self.k, self.n_slots = int(K_b), int(k), int(n_slots)
+        self.rows = batch * n_kv_heads
+        self.nb = ctx_len // block_size
+        self.out_dtype = out_dtype
+        # full K/V in pinned host memory
+        self.host_k = torch.from_numpy(np.ascontiguousarray(k_bits).view(np.int16)).pin_memory()
+        self.host_v = (torch.from_numpy(np.ascontiguousarray(v_bits).view(np.int16)).pin_memory()
+                       if v_bits is not None else None)
+        # resident index, built from a temporary device copy of K
+        self.label_ch = torch.from_numpy(np.ascontiguousarray(label_ch, dtype=np.int32)).to(dev)
+        self.meta = torch.empty((batch, n_kv_heads, self.nb, 2 * qk_dim), dtype=torch.bfloat16, device=dev)
+        self.codes = torch.empty((batch, n_kv_heads, ctx_len, n_label // 2), dtype=torch.uint8, device=dev)
+        self.scales = torch.empty((batch, n_kv_heads, ctx_len), dtype=torch.float32, device=dev)
+        kd = self.host_k.to(dev).view(torch.bfloat16)
+        tls.tls_build_block_meta(self.shape, kd, qk_dim, 0, ctx_len, self.meta, None)
+        tls.tls_quant_label_cache(self.shape, kd, qk_dim, self.label_ch, 0, ctx_len, self.codes, self.scales, None)
+        torch.cuda.synchronize(dev)
+        del kd
+        # the HBM block cache
+        self.slot_k = torch.empty((n_slots, block_size, qk_dim), dtype=torch.bfloat16, device=dev)
+        self.slot_v = (torch.empty((n_slots, block_size, v_dim), dtype=torch.bfloat16, device=dev)
+                       if v_bits is not None else None)
+        self.slot_table = torch.full((batch, n_kv_heads, self.nb), -1, dtype=torch.int32, device=dev)
+        self.cache = tls.tls_block_cache_create(self.shape, self.host_k, self.host_v, qk_dim,
+                                                v_dim if v_bits is not None else 0, n_slots, self.slot_k,
+                                                self.slot_v, self.slot_table)
+        self.block_idx = torch.empty((2, batch, n_kv_heads, self.K_b), dtype=torch.int32, device=dev)
+        self.token_idx = torch.empty((batch, n_kv_heads, self.k), dtype=torch.int32, device=dev)
+        odt = torch.float32 if out_dtype == tls.TLS_OUT_F32 else torch.bfloat16
+        self.out = torch.empty((batch, n_q_heads, v_dim), dtype=odt, device=dev)
+        self.lse = torch.empty((batch, n_q_heads), dtype=torch.float32, device=dev)
+        self.ws_bytes = tls.tls_workspace_bytes(self.shape, self.K_b, self.k)
+        self.ws = torch.zeros(self.ws_bytes, dtype=torch.uint8, device=dev)
+        self.engine = tls.tls_engine_create(self.shape, self.K_b, self.k, self.meta, self.label_ch, self.codes,
+                                            self.scales, self.cache, self.block_idx, self.token_idx, self.ws,
+                                            self.ws_bytes)
+
+    def step(self, q, stream=None):
+        """One staggered decode step with q (device bf16 [B, Hq, Dqk]); writes self.out / self.lse."""
+        tls.tls_engine_step(self.engine, q, self.out_dtype, self.out, self.lse, stream)
+
+    def steps_taken(self) -> int:
+        return tls.tls_engine_steps(self.engine)
+
+    def stats(self, step: int):
+        return tls.tls_engine_stats(self.engine, step)
+
+    def blocks_of_step(self, t: int) -> torch.Tensor:
+        """M_t (valid after step t, until step t + 2 overwrites it)."""
+        return self.block_idx[t & 1]
+
+    def check_device_error(self, stream=None) -> int:
+        return tls.tls_workspace_error(self.ws, True, stream)
+
+    def close(self):
+        if getattr(self, "engine", None):
+            tls.tls_engine_destroy(self.engine)
+            self.engine = None
+        if getattr(self, "cache", None):
+            tls.tls_block_cache_destroy(self.cache)
+            self.cache = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def offloaded_layer_for_config(cfg, k_bits, v_bits, label_ch, n_slots=None, **kw) -> OffloadedLayer:
+    """OffloadedLayer for a workload description with the fields of synth.WorkloadConfig.
+
+    The pool is shared by all rows: cfg.n_slots (default 2 * K_b, which always
+    holds M_{t-1} and M_t) slots per (batch row, KV head), unless n_slots
+    gives the pool size itself."""
+    pool = n_slots if n_slots is not None else (cfg.n_slots or 2 * cfg.K_b) * cfg.batch * cfg.n_kv_heads
+    return OffloadedLayer(batch=cfg.batch, n_q_heads=cfg.n_q_heads, n_kv_heads=cfg.n_kv_heads, qk_dim=cfg.qk_dim,
+                          v_dim=cfg.v_dim, v_offset=cfg.v_offset, block_size=cfg.block_size, n_label=cfg.n_label,
+                          ctx_len=cfg.ctx_len, K_b=cfg.K_b, k=cfg.k, n_slots=pool,
+                          k_bits=k_bits, v_bits=v_bits, label_ch=label_ch, softmax_scale=cfg.softmax_scale, **kw)

@@ -47,6 +47,16 @@ class Shape(ctypes.Structure):
     ]
 
 
+class EngineStepStats(ctypes.Structure):
+    _fields_ = [
+        ("step", ctypes.c_int64),
+        ("n_copied", ctypes.c_int32),
+        ("bytes_copied", ctypes.c_int64),
+        ("copy_ms", ctypes.c_float),
+        ("exposed_ms", ctypes.c_float),
+    ]
+
+
 class KvView(ctypes.Structure):
     _fields_ = [
         ("k", ctypes.c_void_p),
@@ -81,6 +91,11 @@ _SIG = {
     "tls_block_cache_plan": (_I32, [_P, _P, _P, _I32, _P, _P, _P, _P]),
     "tls_prefetch_diff": (_I32, [_P, _P, _P, _I32, _P, _P]),
     "tls_block_cache_table": (_I32, [_P, _P]),
+    "tls_engine_create": (_I32, [_P, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "tls_engine_step": (_I32, [_P, _P, _I32, _P, _P, _P]),
+    "tls_engine_steps": (_I64, [_P]),
+    "tls_engine_stats": (_I32, [_P, _I64, _P]),
+    "tls_engine_destroy": (None, [_P]),
 }
 
 _lib = None
@@ -243,3 +258,31 @@ def tls_prefetch_diff(handle, new_block_idx_host, in_use_block_idx_host, K_b, co
 
 def tls_block_cache_table(handle, table):
     _check(lib().tls_block_cache_table(handle, _ptr(table)), "tls_block_cache_table")
+
+
+def tls_engine_create(shape, K_b, k, meta, label_ch, codes, scales, cache, block_idx, token_idx, ws,
+                      ws_bytes) -> int:
+    h = ctypes.c_void_p()
+    _check(lib().tls_engine_create(ctypes.byref(shape), K_b, k, _ptr(meta), _ptr(label_ch), _ptr(codes),
+                                   _ptr(scales), cache, _ptr(block_idx), _ptr(token_idx), _ptr(ws), ws_bytes,
+                                   ctypes.byref(h)), "tls_engine_create")
+    return h.value
+
+
+def tls_engine_step(engine, q, out_dtype, out, lse=None, stream=None):
+    _check(lib().tls_engine_step(engine, _ptr(q), out_dtype, _ptr(out), _ptr(lse), _stream(stream)),
+           "tls_engine_step")
+
+
+def tls_engine_steps(engine) -> int:
+    return lib().tls_engine_steps(engine)
+
+
+def tls_engine_stats(engine, step: int) -> EngineStepStats:
+    st = EngineStepStats()
+    _check(lib().tls_engine_stats(engine, step, ctypes.byref(st)), "tls_engine_stats")
+    return st
+
+
+def tls_engine_destroy(engine):
+    lib().tls_engine_destroy(engine)
