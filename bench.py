@@ -47,6 +47,7 @@ def parse():
     ap.add_argument("--impl", default="tls", choices=["tls", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-offload", action="store_true", help="skip the offload-engine measurement (c4)")
     ap.add_argument("--e2e-steps", type=int, default=300)
     return ap.parse_args()
 
@@ -210,6 +211,60 @@ def time_oracle(cfg, q, K, V, lab, seconds, rows_sample=8):
             "sample": f"{done} (batch row, KV head) decode_row calls over {len(pick)} seeded rows of "
                       f"{cfg.name} in {el:.1f} s; scaled to all {cfg.rows} rows of one step",
             "s_per_step": step_s}
+
+
+def measure_offload_engine(dev, steps=64):
+    """The offload workload (c4): the staggered engine over an HBM block cache of
+    256 slots, K/V in pinned host memory, `steps` consecutive decode steps along
+    the seeded query trajectory.  Steps run back to back (no L2 flush, nothing
+    between them), which leaves the copies the least time to hide."""
+    import synth
+    import torch
+    from two_level_sparse_block_b200 import runtime
+    cfg = synth.get_config("c4")
+    qs = synth.gen_query_trajectory(cfg, steps)
+    K, V, _ = synth.gen_kv(cfg, qs[0])
+    lab = synth.gen_label_channels(cfg)
+    layer = runtime.offloaded_layer_for_config(cfg, K, V, lab)
+    try:
+        qd = [torch.from_numpy(np.ascontiguousarray(q).view(np.int16)).to(dev).view(torch.bfloat16) for q in qs]
+        stream = torch.cuda.current_stream(dev)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        torch.cuda.synchronize(dev)
+        host_s = []
+        for t in range(steps):
+            evs[t][0].record(stream)
+            h0 = time.perf_counter()
+            layer.step(qd[t], stream=stream)
+            host_s.append(time.perf_counter() - h0)
+            evs[t][1].record(stream)
+        torch.cuda.synchronize(dev)
+        if layer.check_device_error() != 0:
+            raise RuntimeError("device error in the offload engine")
+        step_ms = [a.elapsed_time(b) for a, b in evs]
+        st = [layer.stats(t) for t in range(steps - 1)]  # the transfer of step t, awaited by step t + 1
+        copy_ms = sum(x.copy_ms for x in st)
+        exposed_ms = sum(x.exposed_ms for x in st)
+        moved = sum(x.bytes_copied for x in st)
+        blocks = [x.n_copied for x in st]
+        prologue = layer.stats(-1)
+    finally:
+        layer.close()
+    steady = step_ms[1:]
+    return {
+        "workload": cfg.name, "steps": steps, "n_slots": cfg.n_slots * cfg.rows, "K_b": cfg.K_b,
+        "us_per_step_median": 1e3 * statistics.median(steady), "us_per_step_mean": 1e3 * statistics.mean(steady),
+        "us_first_step": 1e3 * step_ms[0], "prologue_blocks": prologue.n_copied,
+        "host_us_per_step_median": 1e6 * statistics.median(host_s[1:]),
+        "transfer_blocks_per_step_mean": statistics.mean(blocks),
+        "transfer_frac_of_K_b_mean": statistics.mean(blocks) / (cfg.K_b * cfg.rows),
+        "h2d_gbs": moved / (copy_ms / 1e3) / 1e9 if copy_ms > 0 else None,
+        "copy_us_per_step_mean": 1e3 * copy_ms / len(st), "exposed_us_per_step_mean": 1e3 * exposed_ms / len(st),
+        "copy_hidden_frac": 1.0 - exposed_ms / copy_ms if copy_ms > 0 else None, "target_hidden_frac": 0.9,
+        "timing": "per step: CUDA events on the caller's stream around tls_engine_step (level 2 + wait for the "
+                  "previous transfer + attention; level 1 runs on the engine's second stream); transfer figures "
+                  "from the engine's copy-stream events",
+    }
 
 
 def run_reference(args, cfg):
@@ -411,6 +466,8 @@ def main():
         "clocks": clocks,
         "wall_s_timed": wall,
     }
+    if rank == 0 and world == 1 and not args.no_offload:
+        line["offload_engine"] = measure_offload_engine(dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = time_oracle(c, q, K, V, lab, args.cpu_seconds)
         line["cpu_baseline"].pop("s_per_step", None)

@@ -53,13 +53,16 @@ def c2_shape(tls, **kw):
 
 
 def test_attention_dispatch_names_the_kernel_per_shape(tls):
-    # 128-wide heads, G <= 16: one cluster of CTAs per row when the rows fill the GPU that way
+    # 128-wide heads: one cluster of CTAs per (row, head group of <= 16 heads) while the grid
+    # fits two CTAs per SM; more rows than that: the persistent form
     assert tls.tls_attn_kernel(c2_shape(tls)) == "sparse_attn_mma_cluster_kernel"              # 64 rows x 4
     assert tls.tls_attn_kernel(c2_shape(tls, n_q_heads=128)) == "sparse_attn_mma_cluster_kernel"  # G = 16
     assert tls.tls_attn_kernel(c2_shape(tls, batch=16)) == "sparse_attn_mma_cluster_kernel"     # 128 rows x 2
-    assert tls.tls_attn_kernel(c2_shape(tls, batch=1)) == "sparse_attn_mma_kernel"              # 8 rows: persistent
+    assert tls.tls_attn_kernel(c2_shape(tls, batch=1)) == "sparse_attn_mma_cluster_kernel"      # 8 rows x 16
     assert tls.tls_attn_kernel(c2_shape(tls, batch=64)) == "sparse_attn_mma_kernel"             # 512 rows
-    assert tls.tls_attn_kernel(c2_shape(tls, n_q_heads=64, n_kv_heads=1)) == "sparse_attn_tc_kernel"
+    # G > 16: head groups of 16 as virtual rows (1 row x 4 groups -> clusters of 8)
+    assert tls.tls_attn_kernel(c2_shape(tls, batch=1, n_q_heads=64, n_kv_heads=1)) == "sparse_attn_mma_cluster_kernel"
+    assert tls.tls_attn_kernel(c2_shape(tls, batch=40, n_q_heads=64, n_kv_heads=1)) == "sparse_attn_mma_kernel"
     mla = c2_shape(tls, batch=4, n_q_heads=128, n_kv_heads=1, qk_dim=576, v_dim=512, v_offset=0, n_label=32)
     assert tls.tls_attn_kernel(mla) == "sparse_attn_kernel"
     assert tls.tls_attn_kernel(c2_shape(tls, qk_dim=64, v_dim=64)) == "sparse_attn_kernel"

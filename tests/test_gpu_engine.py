@@ -159,3 +159,37 @@ def test_engine_copy_failure_is_reported_and_sticks(monkeypatch):
     # the device still runs work after the engine is gone
     x = torch.ones(1024, device="cuda")
     assert float(x.sum()) == 1024.0
+
+
+def test_engine_on_the_offload_workload_sampled_steps():
+    # c4 (MQA, 131072 tokens, 256 slots): three steps of the trajectory, the
+    # row checked against the staggered oracle each step
+    runtime, tls = _rt()
+    cfg = synth.get_config("c4")
+    qs = synth.gen_query_trajectory(cfg, 3)
+    K, V, _ = synth.gen_kv(cfg, qs[0])
+    lab = synth.gen_label_channels(cfg)
+    layer = runtime.offloaded_layer_for_config(cfg, K, V, lab)
+    g = cfg.group
+    try:
+        for t, q in enumerate(qs):
+            layer.step(_dev_q(q))
+            torch.cuda.synchronize()
+            assert layer.check_device_error() == 0
+            m_prev = layer.block_idx[(t + 1) & 1].cpu().numpy()
+            m_cur = layer.block_idx[t & 1].cpu().numpy()
+            tok = layer.token_idx.cpu().numpy()
+            out = layer.out.float().cpu().numpy()
+            where = f"c4 step {t}"
+            r1 = _orow(cfg, q, K, V, lab, 0, 0)
+            check_selection(m_cur[0, 0], r1["agg"], cfg.K_b, where + " M_t")
+            r2 = _orow(cfg, q, K, V, lab, 0, 0, block_idx=m_prev[0, 0])
+            pos = np.searchsorted(r2["cand"], tok[0, 0])
+            assert np.array_equal(r2["cand"][pos], tok[0, 0]), where + ": token outside M_t-1"
+            check_selection(pos, r2["token_score"], cfg.k, where + " tokens")
+            r3 = _orow(cfg, q, K, V, lab, 0, 0, block_idx=m_prev[0, 0], token_idx=tok[0, 0])
+            check_output(out[0, 0:g], r3["out"], where + " out")
+        assert layer.stats(-1).n_copied == cfg.K_b
+        assert all(0 <= layer.stats(t).n_copied <= cfg.K_b for t in range(len(qs) - 1))
+    finally:
+        layer.close()

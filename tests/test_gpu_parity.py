@@ -63,9 +63,12 @@ SMALL = [
     small("s_all", ctx_len=512, K_b=32, k=512, seed=18),
 ]
 FULL = [get_config(c) for c in ("c1", "c2", "c3", "c4")]
-# row counts that send the 128-wide, G <= 16 attention to its cluster form
-# (8, 4 and 2 CTAs per row); ragged lists, and in s_cl8 a CTA with no chunk
+# row counts that send the 128-wide attention to its cluster form (16, 8, 4
+# and 2 CTAs per row); ragged lists, idle CTAs, and a 64-head group split into
+# four virtual rows of 16 heads
 CLUSTER = [
+    small("s_cl16", batch=2, n_q_heads=16, n_kv_heads=2, ctx_len=1024, K_b=9, k=120, seed=25),
+    small("s_hg4_g64", batch=1, n_q_heads=64, n_kv_heads=1, ctx_len=2048, K_b=14, k=200, seed=26),
     small("s_cl8", batch=20, n_q_heads=4, n_kv_heads=1, ctx_len=1024, K_b=7, k=97, seed=21),
     small("s_cl4", batch=16, n_q_heads=16, n_kv_heads=4, ctx_len=2048, K_b=13, k=200, seed=22),
     small("s_cl4_g1", batch=8, n_q_heads=8, n_kv_heads=8, ctx_len=1024, K_b=8, k=128, seed=23),

@@ -18,13 +18,13 @@ tls_status select_tokens_impl(const tls_shape& s, const void* q, const int32_t* 
                               bool pdl = false);
 tls_status sparse_attn_impl(const tls_shape& s, const void* q, const tls_kv_view& kv, const int32_t* token_idx,
                             int k, int out_dtype, void* out, float* lse, uint8_t* ws, const WsLayout& L,
-                            cudaStream_t stream);
+                            cudaStream_t stream, bool pdl = true);
 int attn_heads_per_cta(const tls_shape& s);
 bool attn_tc_supported(const tls_shape& s);
 int attn_tc_plan(int rows, int head_groups, int k, int* tiles, int* n_items, int* n_ctas);
 bool attn_mma_supported(const tls_shape& s);
 int attn_mma_plan(int rows, int k, int* chunks_per_row, int* n_items, int* n_ctas);
-int attn_mma_cluster_size(int rows);
+int attn_mma_cluster_size(int rows, int hpc);
 
 namespace {
 thread_local char g_err[512] = {0};
@@ -80,7 +80,7 @@ tls_status plan_workspace(const tls_shape& s, int K_b, int k, WsLayout* out) {
   if (attn_mma_supported(s)) {
     // warp-streaming attention: persistent CTAs over 16-token chunks
     L.tokens_per_split = 16;
-    L.splits = attn_mma_plan(rows, k, &L.tiles_per_pair, &L.n_items, &L.n_ctas);
+    L.splits = attn_mma_plan(rows * L.head_groups, k, &L.tiles_per_pair, &L.n_items, &L.n_ctas);
   } else if (attn_tc_supported(s)) {
     // tensor-core attention: persistent CTAs over 128-token tiles; a split
     // slot per CTA that shares a (row, head group)
@@ -154,8 +154,11 @@ extern "C" int32_t tls_version(void) { return 100; }
 
 extern "C" const char* tls_attn_kernel(const tls_shape* shape) {
   if (check_shape(shape) != TLS_OK) return nullptr;
-  if (attn_mma_supported(*shape))
-    return attn_mma_cluster_size(rows_of(*shape)) > 0 ? "sparse_attn_mma_cluster_kernel" : "sparse_attn_mma_kernel";
+  if (attn_mma_supported(*shape)) {
+    const int g = group_of(*shape), hpc = g < 16 ? g : 16, head_groups = (g + hpc - 1) / hpc;
+    return attn_mma_cluster_size(rows_of(*shape) * head_groups, hpc) > 0 ? "sparse_attn_mma_cluster_kernel"
+                                                                          : "sparse_attn_mma_kernel";
+  }
   if (attn_tc_supported(*shape)) return "sparse_attn_tc_kernel";
   return "sparse_attn_kernel";
 }

@@ -120,10 +120,10 @@ static __device__ __noinline__ void merge_splits(const AttnParams& p, int row, i
 
 // Tensor-core attention (decode_attn_tc.cu): 128-wide K and V rows.
 bool attn_tc_supported(const tls_shape& s);
-tls_status launch_attn_tc(const AttnParams& p, int rows, cudaStream_t stream);
+tls_status launch_attn_tc(const AttnParams& p, int rows, cudaStream_t stream, bool pdl);
 // Warp-streaming attention for groups of <= 16 heads (decode_attn_mma.cu).
 bool attn_mma_supported(const tls_shape& s);
-tls_status launch_attn_mma(const AttnParams& p, int rows, cudaStream_t stream);
-int attn_mma_cluster_size(int rows);
+tls_status launch_attn_mma(const AttnParams& p, int rows, cudaStream_t stream, bool pdl);
+int attn_mma_cluster_size(int rows, int hpc);
 
 }  // namespace tls

@@ -38,6 +38,11 @@ struct tls_block_cache {
   int cur = 0;
   bool published = false;                     // the device table has been written once
   std::vector<int2> changes;                  // this plan's (entry, value) table changes
+  // Pull path: when K/V are pinned host memory mapped into the device address
+  // space, one kernel reads the planned blocks over PCIe into their slots.
+  const uint8_t* dev_host_k = nullptr;        // device addresses of host_k / host_v
+  const uint8_t* dev_host_v = nullptr;
+  int4* jobs[2] = {nullptr, nullptr};         // pinned, mapped: {tok0 lo, tok0 hi, slot, 0} per copy
 };
 
 namespace tls {
@@ -46,6 +51,23 @@ namespace {
 struct Copy {
   int32_t row, block, slot;
 };
+
+// Device address of [p, p + bytes) when the whole range is pinned host memory
+// mapped into the device address space as one contiguous range; else NULL.
+const uint8_t* mapped_host_range(const void* p, size_t bytes) {
+  if (p == nullptr || bytes == 0) return nullptr;
+  cudaPointerAttributes a, b;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess ||
+      cudaPointerGetAttributes(&b, (const uint8_t*)p + (bytes - 1)) != cudaSuccess) {
+    cudaGetLastError();  // clear the sticky-free error of an unknown pointer
+    return nullptr;
+  }
+  if (a.type != cudaMemoryTypeHost || b.type != cudaMemoryTypeHost || a.devicePointer == nullptr ||
+      b.devicePointer == nullptr)
+    return nullptr;
+  if ((const uint8_t*)b.devicePointer - (const uint8_t*)a.devicePointer != (ptrdiff_t)(bytes - 1)) return nullptr;
+  return (const uint8_t*)a.devicePointer;
+}
 
 bool fault_injected_copy() {
   const char* e = std::getenv("TLS_FAULT_INJECT");
@@ -121,6 +143,47 @@ void commit(tls_block_cache& c, const int32_t* new_idx, int K_b, std::vector<Cop
     }
 }
 
+// Copies planned blocks from mapped pinned host memory into their slots: CTA
+// j takes job j (a block's bs rows of K and of V, contiguous on both sides),
+// 16-byte loads, eight in flight per thread; then the slot-table changes.
+// The consumers (the next attention) start after the whole kernel, so the
+// order of the two parts does not matter.
+constexpr int kPullThreads = 256;
+__global__ void __launch_bounds__(kPullThreads) block_pull_kernel(const uint8_t* host_k, const uint8_t* host_v,
+                                                                  uint8_t* slot_k, uint8_t* slot_v, int64_t kblk,
+                                                                  int64_t vblk, int64_t k_row_bytes,
+                                                                  int64_t v_row_bytes, const int4* jobs, int n_jobs,
+                                                                  int32_t* table, const int2* pairs, int n_pairs) {
+  if ((int)blockIdx.x < n_jobs) {
+    const int4 jb = jobs[blockIdx.x];
+    const int64_t tok0 = (int64_t)(uint32_t)jb.x | ((int64_t)jb.y << 32);
+    const int64_t slot = jb.z;
+    for (int part = 0; part < 2; ++part) {
+      const uint8_t* src = part == 0 ? host_k + tok0 * k_row_bytes : (host_v ? host_v + tok0 * v_row_bytes : nullptr);
+      uint8_t* dst = part == 0 ? slot_k + slot * kblk : (slot_v ? slot_v + slot * vblk : nullptr);
+      if (src == nullptr || dst == nullptr) continue;
+      const int64_t n16 = (part == 0 ? kblk : vblk) / 16;
+      const uint4* s4 = reinterpret_cast<const uint4*>(src);
+      uint4* d4 = reinterpret_cast<uint4*>(dst);
+      for (int64_t i0 = threadIdx.x; i0 < n16; i0 += 8 * kPullThreads) {
+        uint4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int64_t i = i0 + (int64_t)u * kPullThreads;
+          if (i < n16) v[u] = __ldcv(s4 + i);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int64_t i = i0 + (int64_t)u * kPullThreads;
+          if (i < n16) d4[i] = v[u];
+        }
+      }
+    }
+  }
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < n_pairs; i += kPullThreads) table[pairs[i].x] = pairs[i].y;
+}
+
 // Applies (entry, value) pairs (mapped pinned memory) to the device slot table.
 __global__ void slot_table_update_kernel(int32_t* table, const int2* pairs, int n) {
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
@@ -147,40 +210,64 @@ tls_status prefetch_diff_impl(tls_block_cache* c, const int32_t* new_idx, const 
   const int64_t n = c->shape.ctx_len;
   const size_t kblk = (size_t)bs * c->hk_stride * 2, vblk = (size_t)bs * c->hv_stride * 2;
   const bool with_v = c->host_v != nullptr && c->slot_v != nullptr;
-  size_t i = 0;
-  while (i < copies.size()) {
-    size_t j = i + 1;
-    while (j < copies.size() && copies[j].row == copies[i].row &&
-           copies[j].block == copies[j - 1].block + 1 && copies[j].slot == copies[j - 1].slot + 1)
-      ++j;
-    const size_t len = j - i;
-    const int64_t tok0 = (int64_t)copies[i].row * n + (int64_t)copies[i].block * bs;
-    cudaError_t e = cudaMemcpyAsync(c->slot_k + (size_t)copies[i].slot * kblk,
-                                    c->host_k + (size_t)tok0 * c->hk_stride * 2, len * kblk,
-                                    cudaMemcpyHostToDevice, cs);
-    if (e == cudaSuccess && with_v)
-      e = cudaMemcpyAsync(c->slot_v + (size_t)copies[i].slot * vblk, c->host_v + (size_t)tok0 * c->hv_stride * 2,
-                          len * vblk, cudaMemcpyHostToDevice, cs);
-    if (e != cudaSuccess) return fail(TLS_ERR_COPY, "prefetch_diff: block copy failed: %s", cudaGetErrorString(e));
-    i = j;
-  }
-  // publish the table: whole the first time, afterwards only the changed entries
   const int b = c->cur;
-  cudaError_t e = cudaEventSynchronize(c->staged[b]);  // the staging buffer's previous use is done
+  cudaError_t e = cudaEventSynchronize(c->staged[b]);  // the staging buffers' previous use is done
   if (e != cudaSuccess) return cuda_check(e, "prefetch_diff: staging wait");
-  if (!c->published) {
+  // the first transfer publishes the whole table (nothing is resident, so nothing reads it)
+  const bool first = !c->published;
+  if (first) {
     std::memcpy(c->staging[b], c->table.data(), c->table.size() * sizeof(int32_t));
     e = cudaMemcpyAsync(c->table_dev, c->staging[b], c->table.size() * sizeof(int32_t), cudaMemcpyHostToDevice, cs);
+    if (e != cudaSuccess) return fail(TLS_ERR_COPY, "prefetch_diff: slot table copy failed: %s", cudaGetErrorString(e));
     c->published = true;
-  } else if (!c->changes.empty()) {
-    int2* pairs = reinterpret_cast<int2*>(c->staging[b]);
-    std::memcpy(pairs, c->changes.data(), c->changes.size() * sizeof(int2));
-    const int n_pairs = (int)c->changes.size();
-    slot_table_update_kernel<<<(n_pairs + 255) / 256, 256, 0, cs>>>(c->table_dev, pairs, n_pairs);
-    e = cudaGetLastError();
   }
-  if (e == cudaSuccess) e = cudaEventRecord(c->staged[b], cs);
-  if (e != cudaSuccess) return fail(TLS_ERR_COPY, "prefetch_diff: slot table update failed: %s", cudaGetErrorString(e));
+  const int n_pairs = first ? 0 : (int)c->changes.size();
+  if (c->dev_host_k != nullptr) {
+    // one kernel pulls every planned block over PCIe and applies the table changes
+    int4* jobs = c->jobs[b];
+    for (size_t i = 0; i < copies.size(); ++i) {
+      const int64_t tok0 = (int64_t)copies[i].row * n + (int64_t)copies[i].block * bs;
+      jobs[i] = make_int4((int)(uint32_t)(tok0 & 0xFFFFFFFF), (int)(tok0 >> 32), copies[i].slot, 0);
+    }
+    int2* pairs = first ? nullptr : reinterpret_cast<int2*>(c->staging[b]);
+    if (pairs != nullptr) std::memcpy(pairs, c->changes.data(), (size_t)n_pairs * sizeof(int2));
+    const int grid = copies.empty() ? 1 : (int)copies.size();
+    if (!copies.empty() || n_pairs > 0) {
+      block_pull_kernel<<<grid, kPullThreads, 0, cs>>>(c->dev_host_k, with_v ? c->dev_host_v : nullptr, c->slot_k,
+                                                        with_v ? c->slot_v : nullptr, (int64_t)kblk, (int64_t)vblk,
+                                                        c->hk_stride * 2, c->hv_stride * 2, jobs,
+                                                        (int)copies.size(), c->table_dev, pairs, n_pairs);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return fail(TLS_ERR_COPY, "prefetch_diff: pull kernel launch failed: %s", cudaGetErrorString(e));
+    }
+  } else {
+    // one cudaMemcpyAsync per run of blocks adjacent in host memory and in the pool
+    size_t i = 0;
+    while (i < copies.size()) {
+      size_t j = i + 1;
+      while (j < copies.size() && copies[j].row == copies[i].row &&
+             copies[j].block == copies[j - 1].block + 1 && copies[j].slot == copies[j - 1].slot + 1)
+        ++j;
+      const size_t len = j - i;
+      const int64_t tok0 = (int64_t)copies[i].row * n + (int64_t)copies[i].block * bs;
+      e = cudaMemcpyAsync(c->slot_k + (size_t)copies[i].slot * kblk, c->host_k + (size_t)tok0 * c->hk_stride * 2,
+                          len * kblk, cudaMemcpyHostToDevice, cs);
+      if (e == cudaSuccess && with_v)
+        e = cudaMemcpyAsync(c->slot_v + (size_t)copies[i].slot * vblk, c->host_v + (size_t)tok0 * c->hv_stride * 2,
+                            len * vblk, cudaMemcpyHostToDevice, cs);
+      if (e != cudaSuccess) return fail(TLS_ERR_COPY, "prefetch_diff: block copy failed: %s", cudaGetErrorString(e));
+      i = j;
+    }
+    if (n_pairs > 0) {
+      int2* pairs = reinterpret_cast<int2*>(c->staging[b]);
+      std::memcpy(pairs, c->changes.data(), (size_t)n_pairs * sizeof(int2));
+      slot_table_update_kernel<<<(n_pairs + 255) / 256, 256, 0, cs>>>(c->table_dev, pairs, n_pairs);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return fail(TLS_ERR_COPY, "prefetch_diff: table update launch failed: %s", cudaGetErrorString(e));
+    }
+  }
+  e = cudaEventRecord(c->staged[b], cs);
+  if (e != cudaSuccess) return cuda_check(e, "prefetch_diff: staging event");
   c->cur ^= 1;
   *n_copied = (int32_t)copies.size();
   if (bytes != nullptr) *bytes = (int64_t)copies.size() * (int64_t)(kblk + (with_v ? vblk : 0));
@@ -234,6 +321,27 @@ extern "C" tls_status tls_block_cache_create(const tls_shape* shape, const void*
   c->table.assign((size_t)c->rows * c->nb, -1);
   c->owner.assign(n_slots, -1);
   c->last_use.assign(n_slots, 0);
+  if (slot_table_dev != nullptr && host_k != nullptr && slot_k != nullptr) {
+    // the pull path needs 16-byte-aligned rows and both tensors mapped
+    const size_t tokens = (size_t)c->rows * (size_t)shape->ctx_len;
+    const bool aligned = aligned16(host_k) && host_k_row_stride % 8 == 0 &&
+                         (c->host_v == nullptr || (aligned16(host_v) && host_v_row_stride % 8 == 0));
+    const uint8_t* dk = aligned ? mapped_host_range(host_k, tokens * (size_t)host_k_row_stride * 2) : nullptr;
+    const uint8_t* dv =
+        (dk != nullptr && c->host_v != nullptr) ? mapped_host_range(host_v, tokens * (size_t)host_v_row_stride * 2)
+                                                : nullptr;
+    if (dk != nullptr && (c->host_v == nullptr || dv != nullptr)) {
+      cudaError_t e = cudaSuccess;
+      for (int i = 0; i < 2 && e == cudaSuccess; ++i)
+        e = cudaHostAlloc((void**)&c->jobs[i], (size_t)n_slots * sizeof(int4), cudaHostAllocMapped | cudaHostAllocPortable);
+      if (e != cudaSuccess) {
+        tls_block_cache_destroy(c);
+        return cuda_check(e, "block_cache_create: pinned job lists");
+      }
+      c->dev_host_k = dk;
+      c->dev_host_v = dv;
+    }
+  }
   if (slot_table_dev != nullptr) {
     // a plan changes at most two entries per copied block and copies at most n_slots blocks
     const size_t words = std::max(c->table.size(), (size_t)4 * (size_t)n_slots);
@@ -259,6 +367,7 @@ extern "C" void tls_block_cache_destroy(tls_block_cache* c) {
       cudaEventDestroy(c->staged[i]);
     }
     if (c->staging[i] != nullptr) cudaFreeHost(c->staging[i]);
+    if (c->jobs[i] != nullptr) cudaFreeHost(c->jobs[i]);
   }
   delete c;
 }

@@ -223,7 +223,7 @@ tls_status launch_attn(const AttnParams& p, int rows, cudaStream_t stream) {
 
 tls_status sparse_attn_impl(const tls_shape& s, const void* q, const tls_kv_view& kv, const int32_t* token_idx,
                             int k, int out_dtype, void* out, float* lse, uint8_t* ws, const WsLayout& L,
-                            cudaStream_t stream) {
+                            cudaStream_t stream, bool pdl) {
   AttnParams p;
   p.q = (const uint16_t*)q;
   p.k = (const uint16_t*)kv.k;
@@ -257,8 +257,8 @@ tls_status sparse_attn_impl(const tls_shape& s, const void* q, const tls_kv_view
   p.n_ctas = L.n_ctas;
   p.err = reinterpret_cast<int*>(ws + L.err);
   const int rows = rows_of(s);
-  if (attn_mma_supported(s)) return launch_attn_mma(p, rows, stream);
-  if (attn_tc_supported(s)) return launch_attn_tc(p, rows, stream);
+  if (attn_mma_supported(s)) return launch_attn_mma(p, rows, stream, pdl);
+  if (attn_tc_supported(s)) return launch_attn_tc(p, rows, stream, pdl);
   const int pk = (s.qk_dim + 127) / 128, pv = (s.v_dim + 127) / 128;
   const int hg = L.heads_per_cta;
   if (pk == 1 && pv == 1) {
@@ -283,7 +283,7 @@ tls_status sparse_attn_impl(const tls_shape& s, const void* q, const tls_kv_view
 // register budget allows 8 heads at 128-wide rows, 4 at 256 and 2 above.
 int attn_heads_per_cta(const tls_shape& s) {
   const int g = group_of(s);
-  if (attn_mma_supported(s)) return g;
+  if (attn_mma_supported(s)) return g < 16 ? g : 16;
   if (attn_tc_supported(s)) return g < 64 ? g : 64;
   const int pk = (s.qk_dim + 127) / 128, pv = (s.v_dim + 127) / 128;
   int cap = (pk == 1 && pv == 1) ? 8 : (pk <= 2 && pv <= 2) ? 4 : 2;
@@ -376,5 +376,6 @@ extern "C" tls_status tls_sparse_decode_attn_noalloc(const tls_shape* shape, con
   WsLayout S = L;
   S.att_counter = 0;
   S.partial = ticket_bytes;
-  return sparse_attn_impl(s, q, *kv, token_idx, k, out_dtype, out, lse, (uint8_t*)base, S, (cudaStream_t)stream);
+  return sparse_attn_impl(s, q, *kv, token_idx, k, out_dtype, out, lse, (uint8_t*)base, S, (cudaStream_t)stream,
+                          /*pdl=*/true);
 }

@@ -89,11 +89,12 @@ __host__ __device__ inline MmaLayout mma_layout(int g) {
   return L;
 }
 
-// Q fragments (the A operand of S = Q.K^T, 8 k-steps of 16) of the g heads
-// of row (b, kvh); fragment rows >= g are zero.
-__device__ __forceinline__ void mma_load_q(const AttnParams& p, int b, int kvh, int lane, uint32_t (&qa)[8][4]) {
-  const int g = p.group, gq = lane >> 2, tq = lane & 3;
-  const uint16_t* q0 = p.q + ((int64_t)b * p.n_q_heads + kvh * g + gq) * p.dqk;
+// Q fragments (the A operand of S = Q.K^T, 8 k-steps of 16) of heads
+// h0 .. h0+g-1 of the group of row (b, kvh); fragment rows >= g are zero.
+__device__ __forceinline__ void mma_load_q(const AttnParams& p, int b, int kvh, int h0, int g, int lane,
+                                           uint32_t (&qa)[8][4]) {
+  const int gq = lane >> 2, tq = lane & 3;
+  const uint16_t* q0 = p.q + ((int64_t)b * p.n_q_heads + (int64_t)kvh * p.group + h0 + gq) * p.dqk;
   const uint16_t* q8 = q0 + (int64_t)8 * p.dqk;
 #pragma unroll
   for (int ks = 0; ks < 8; ++ks) {
@@ -299,8 +300,8 @@ template <int NS>
 __global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_kernel(AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-  const int g = p.group;
-  const MmaLayout L = mma_layout(g);
+  const int HPC = p.heads_per_cta, HG = p.head_groups;  // heads of a CTA item, head groups per row
+  const MmaLayout L = mma_layout(HPC);
   float* comb = reinterpret_cast<float*>(sm + L.off_comb);
   float* cm = reinterpret_cast<float*>(sm + L.off_stat);
   float* cl = cm + kMmaWarps * 16;
@@ -316,14 +317,15 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_kernel(Attn
   // this warp's stream: chunks c_lo + warp + 4i
   const int64_t x0 = c_lo + warp;
   const int n_mine = x0 < c_hi ? (int)((c_hi - 1 - x0) / kMmaWarps + 1) : 0;
+  // items are (virtual row, chunk); virtual row vr = (row, head group vr % HG)
   auto load_tok = [&](int i) -> int {
     if (i >= n_mine) return -1;
     const int64_t x = x0 + (int64_t)kMmaWarps * i;
-    return mma_chunk_token(p, (int)(x / CPR), (int)(x % CPR), lane);
+    return mma_chunk_token(p, (int)(x / CPR) / HG, (int)(x % CPR), lane);
   };
   auto issue = [&](int i, int tok, int st) {
     if (i < n_mine)
-      mma_issue_rows(p, (int)((x0 + (int64_t)kMmaWarps * i) / CPR), tok, ring_s + st * kChunkBytes, lane);
+      mma_issue_rows(p, (int)((x0 + (int64_t)kMmaWarps * i) / CPR) / HG, tok, ring_s + st * kChunkBytes, lane);
     cp_async_commit();
   };
 
@@ -336,11 +338,11 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_kernel(Attn
     // what the first row end writes (split partials, the row's ticket, the
     // output and lse rows): prefetching them now also warms their address
     // translations while the token lists are still being selected
-    const int r0 = (int)(c_lo / CPR);
-    const int64_t f0 = attn_owner((int64_t)r0 * CPR, C, p.n_ctas);
-    prefetch_l2(p.partial + (((int64_t)r0 * g) * p.splits + (cta - f0)) * 130);
-    prefetch_l2(p.counters + r0);
-    const int64_t oh = (int64_t)(r0 / p.n_kv_heads) * p.n_q_heads + (r0 % p.n_kv_heads) * g;
+    const int v0 = (int)(c_lo / CPR), r0 = v0 / HG, h00 = (v0 % HG) * HPC;
+    const int64_t f0 = attn_owner((int64_t)v0 * CPR, C, p.n_ctas);
+    prefetch_l2(p.partial + (((int64_t)r0 * p.group + h00) * p.splits + (cta - f0)) * 130);
+    prefetch_l2(p.counters + v0);
+    const int64_t oh = (int64_t)(r0 / p.n_kv_heads) * p.n_q_heads + (int64_t)(r0 % p.n_kv_heads) * p.group + h00;
     prefetch_l2(reinterpret_cast<const uint8_t*>(p.out) + oh * p.dv * (p.out_bf16 ? 2 : 4));
     if (p.lse != nullptr) prefetch_l2(p.lse + oh);
   }
@@ -354,14 +356,15 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_kernel(Attn
   for (int s = 0; s < NS - 1; ++s) issue(s, tok_ahead[s], s);
   int tok_next = tok_ahead[NS - 1];  // for chunk S-1
 
-  const int row_first = (int)(c_lo / CPR);
-  const int row_last = (int)((c_hi - 1) / CPR);
+  const int vrow_first = (int)(c_lo / CPR);
+  const int vrow_last = (int)((c_hi - 1) / CPR);
   int i = 0;  // position in this warp's stream
-  for (int row = row_first; row <= row_last; ++row) {
+  for (int vr = vrow_first; vr <= vrow_last; ++vr) {
+    const int row = vr / HG, h0 = (vr % HG) * HPC, g = min(HPC, p.group - h0);
     const int b = row / p.n_kv_heads, kvh = row % p.n_kv_heads;
-    // this row's chunks inside the CTA range
-    const int64_t seg_end = min(c_hi, (int64_t)(row + 1) * CPR);
-    mma_load_q(p, b, kvh, lane, qa);
+    // this virtual row's chunks inside the CTA range
+    const int64_t seg_end = min(c_hi, (int64_t)(vr + 1) * CPR);
+    mma_load_q(p, b, kvh, h0, g, lane, qa);
 #pragma unroll
     for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.0f;
     m0 = m1 = -INFINITY;
@@ -379,20 +382,20 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_kernel(Attn
       __syncwarp();
     }
 
-    // fold the warps of the CTA for this row into its split of the workspace
-    const int64_t first = attn_owner((int64_t)row * CPR, C, p.n_ctas);
-    const int n_part = (int)(attn_owner((int64_t)row * CPR + CPR - 1, C, p.n_ctas) - first + 1);
+    // fold the warps of the CTA for this virtual row into its split of the workspace
+    const int64_t first = attn_owner((int64_t)vr * CPR, C, p.n_ctas);
+    const int n_part = (int)(attn_owner((int64_t)vr * CPR + CPR - 1, C, p.n_ctas) - first + 1);
     const int slot = (int)(cta - first);
-    float* part = p.partial + ((int64_t)row * g * p.splits + slot) * 130;
+    float* part = p.partial + (((int64_t)row * p.group + h0) * p.splits + slot) * 130;
     mma_fold(g, m0, m1, l0, l1, o, comb, cm, cl,
              [&](int h, int e, float v) { part[(int64_t)h * p.splits * 130 + e] = v; });
     __threadfence();
     __syncthreads();
-    if (tid == 0) s_last = atomicInc(&p.counters[row], (unsigned)(n_part - 1)) == (unsigned)(n_part - 1);
+    if (tid == 0) s_last = atomicInc(&p.counters[vr], (unsigned)(n_part - 1)) == (unsigned)(n_part - 1);
     __syncthreads();
     if (s_last) {
       __threadfence();
-      merge_splits(p, row, b, kvh, 0, g, n_part, comb, kMmaWarps * g * 128);
+      merge_splits(p, row, b, kvh, h0, g, n_part, comb, kMmaWarps * HPC * 128);
     }
     __syncthreads();  // the fold area is rewritten for the next row
   }
@@ -411,14 +414,16 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_cluster_ker
   cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-  const int g = p.group;
-  const MmaLayout L = mma_layout(g);
+  const int HPC = p.heads_per_cta, HG = p.head_groups;
+  const MmaLayout L = mma_layout(HPC);
   float* comb = reinterpret_cast<float*>(sm + L.off_comb);
   float* cm = reinterpret_cast<float*>(sm + L.off_stat);
   float* cl = cm + kMmaWarps * 16;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int CL = (int)gridDim.x, rank = (int)blockIdx.x, row = (int)blockIdx.y;
+  // blockIdx.y is the virtual row (row, head group): heads h0 .. h0+g-1
+  const int CL = (int)gridDim.x, rank = (int)blockIdx.x, vr = (int)blockIdx.y;
+  const int row = vr / HG, h0 = (vr % HG) * HPC, g = min(HPC, p.group - h0);
   const int b = row / p.n_kv_heads, kvh = row % p.n_kv_heads;
   const int CPR = p.tiles_per_pair;
   const int c_lo = rank * CPR / CL, c_hi = (rank + 1) * CPR / CL;
@@ -430,7 +435,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_cluster_ker
     if (i < n_mine) mma_issue_rows(p, row, tok, ring_s + st * kChunkBytes, lane);
     cp_async_commit();
   };
-  const int64_t oh = (int64_t)b * p.n_q_heads + (int64_t)kvh * g;  // first output head of the row
+  const int64_t oh = (int64_t)b * p.n_q_heads + (int64_t)kvh * p.group + h0;  // first output head
 
   grid_launch_dependents();
   if (tid == 0 && rank == 0) {
@@ -439,7 +444,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_cluster_ker
     if (p.lse != nullptr) prefetch_l2(p.lse + oh);
   }
   uint32_t qa[8][4];
-  mma_load_q(p, b, kvh, lane, qa);  // q is an input of the step, not of the preceding kernel
+  mma_load_q(p, b, kvh, h0, g, lane, qa);  // q is an input of the step, not of the preceding kernel
   grid_dependency_wait();           // token lists come from the preceding kernel
 
   float o[16][4];
@@ -492,9 +497,9 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_cluster_ker
   }
 }
 
-bool attn_mma_supported(const tls_shape& s) {
-  return s.qk_dim == 128 && s.v_dim == 128 && s.v_offset < 0 && group_of(s) <= 16;
-}
+// 128-wide K and V rows, any group size: groups above 16 heads are split
+// into head groups of at most 16, each its own virtual row.
+bool attn_mma_supported(const tls_shape& s) { return s.qk_dim == 128 && s.v_dim == 128 && s.v_offset < 0; }
 
 // Work partition: chunks of 16 entries of every row's token list, contiguous
 // ranges over two CTAs per SM.  Returns the largest number of CTAs sharing a row.
@@ -516,40 +521,45 @@ int attn_mma_plan(int rows, int k, int* chunks_per_row, int* n_items, int* n_cta
   return max_part;
 }
 
-// Cluster size of the cluster form for `rows` rows: the largest of 8, 4, 2
-// whose grid (rows x CL CTAs) fills between one and two CTAs per SM; 0 when
-// none does (few rows: the persistent form spreads them over every SM; many
-// rows: one CTA per row and split would not help either).
-int attn_mma_cluster_size(int rows) {
-  for (int cl = 8; cl >= 2; cl /= 2) {
-    const int64_t ctas = (int64_t)rows * cl;
-    if (ctas >= kNumSMs && ctas <= 2 * (int64_t)kNumSMs) return cl;
+// Cluster size of the cluster form for `rows` virtual rows of `hpc` heads:
+// the largest of 16, 8, 4, 2 whose grid (rows x CL CTAs) fits two CTAs per
+// SM and whose CL partials fit the leader's ring (CL * hpc * 130 floats);
+// 0 when even CL = 2 does not fit (many rows: the persistent form).
+int attn_mma_cluster_size(int rows, int hpc) {
+  const int ring_floats = kMmaWarps * mma_stages(hpc) * kChunkBytes / 4;
+  for (int cl = 16; cl >= 2; cl /= 2) {
+    if ((int64_t)rows * cl > 2 * (int64_t)kNumSMs) continue;
+    if ((int64_t)cl * hpc * 130 > ring_floats) continue;
+    return cl;
   }
   return 0;
 }
 
 template <int NS>
-static tls_status launch_mma(const AttnParams& p, int rows, cudaStream_t stream) {
-  const MmaLayout L = mma_layout(p.group);
+static tls_status launch_mma(const AttnParams& p, int rows, cudaStream_t stream, bool pdl) {
+  const MmaLayout L = mma_layout(p.heads_per_cta);
   const size_t smem = 128 + (size_t)L.bytes;
-  const int cl = attn_mma_cluster_size(rows);
+  rows *= p.head_groups;  // virtual rows (row, head group)
+  const int cl = attn_mma_cluster_size(rows, p.heads_per_cta);
   if (cl > 0) {
     cudaError_t e = cudaFuncSetAttribute(sparse_attn_mma_cluster_kernel<NS>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return cuda_check(e, "sparse_decode_attn: set smem attribute");
-    return cuda_check(launch_pdl_cluster(sparse_attn_mma_cluster_kernel<NS>, dim3(cl, rows), dim3(kMmaWarps * 32),
-                                         smem, stream, (unsigned)cl, p),
+    if (e == cudaSuccess && cl > 8)  // 16-CTA clusters are beyond the portable size
+      e = cudaFuncSetAttribute(sparse_attn_mma_cluster_kernel<NS>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return cuda_check(e, "sparse_decode_attn: set cluster attributes");
+    return cuda_check(launch_ex(sparse_attn_mma_cluster_kernel<NS>, dim3(cl, rows), dim3(kMmaWarps * 32), smem, stream,
+                                pdl, (unsigned)cl, p),
                       "sparse_decode_attn: mma cluster launch");
   }
   cudaError_t e =
       cudaFuncSetAttribute(sparse_attn_mma_kernel<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return cuda_check(e, "sparse_decode_attn: set smem attribute");
-  return cuda_check(launch_pdl(sparse_attn_mma_kernel<NS>, dim3(p.n_ctas), dim3(kMmaWarps * 32), smem, stream, p),
+  return cuda_check(launch_ex(sparse_attn_mma_kernel<NS>, dim3(p.n_ctas), dim3(kMmaWarps * 32), smem, stream, pdl, 0u, p),
                     "sparse_decode_attn: mma launch");
 }
 
-tls_status launch_attn_mma(const AttnParams& p, int rows, cudaStream_t stream) {
-  return launch_mma<3>(p, rows, stream);
+tls_status launch_attn_mma(const AttnParams& p, int rows, cudaStream_t stream, bool pdl) {
+  return launch_mma<3>(p, rows, stream, pdl);
 }
 
 }  // namespace tls

@@ -348,22 +348,22 @@ int attn_tc_plan(int rows, int head_groups, int k, int* tiles, int* n_items, int
 }
 
 template <int NPAD, int NS>
-static tls_status launch_tc(const AttnParams& p, cudaStream_t stream) {
+static tls_status launch_tc(const AttnParams& p, cudaStream_t stream, bool pdl) {
   const AttnTcLayout L = attn_tc_layout(NPAD, p.heads_per_cta, NS);
   const size_t smem = 1024 + (size_t)L.bytes;
   cudaError_t e = cudaFuncSetAttribute(sparse_attn_tc_kernel<NPAD, NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return cuda_check(e, "sparse_decode_attn: set smem attribute");
-  return cuda_check(launch_pdl(sparse_attn_tc_kernel<NPAD, NS>, dim3(p.n_ctas), dim3(128), smem, stream, p),
+  return cuda_check(launch_ex(sparse_attn_tc_kernel<NPAD, NS>, dim3(p.n_ctas), dim3(128), smem, stream, pdl, 0u, p),
                     "sparse_decode_attn: tc launch");
 }
 
-tls_status launch_attn_tc(const AttnParams& p, int rows, cudaStream_t stream) {
+tls_status launch_attn_tc(const AttnParams& p, int rows, cudaStream_t stream, bool pdl) {
   (void)rows;
   switch (attn_tc_npad(p.heads_per_cta)) {
-    case 16: return launch_tc<16, 3>(p, stream);
-    case 32: return launch_tc<32, 3>(p, stream);
-    default: return launch_tc<64, 2>(p, stream);
+    case 16: return launch_tc<16, 3>(p, stream, pdl);
+    case 32: return launch_tc<32, 3>(p, stream, pdl);
+    default: return launch_tc<64, 2>(p, stream, pdl);
   }
 }
 

@@ -31,7 +31,7 @@ tls_status select_tokens_impl(const tls_shape& s, const void* q, const int32_t* 
                               bool pdl = false);
 tls_status sparse_attn_impl(const tls_shape& s, const void* q, const tls_kv_view& kv, const int32_t* token_idx,
                             int k, int out_dtype, void* out, float* lse, uint8_t* ws, const WsLayout& L,
-                            cudaStream_t stream);
+                            cudaStream_t stream, bool pdl = true);
 tls_status prefetch_diff_impl(tls_block_cache* c, const int32_t* new_idx, const int32_t* in_use, int K_b,
                               cudaStream_t cs, int32_t* n_copied, int64_t* bytes);
 tls_status block_cache_view(const tls_block_cache* c, tls_kv_view* kv);
@@ -124,8 +124,12 @@ extern "C" tls_status tls_engine_create(const tls_shape* shape, int32_t K_b, int
   cudaError_t ce = cudaSuccess;
   for (int i = 0; i < 2 && ce == cudaSuccess; ++i)
     ce = cudaHostAlloc((void**)&e->host_bidx[i], (size_t)e->rows * K_b * sizeof(int32_t), cudaHostAllocDefault);
-  if (ce == cudaSuccess) ce = cudaStreamCreateWithFlags(&e->sel, cudaStreamNonBlocking);
-  if (ce == cudaSuccess) ce = cudaStreamCreateWithFlags(&e->copy, cudaStreamNonBlocking);
+  // the select and copy streams get the highest priority: their small grids
+  // are on the critical path of the next step, the attention is not
+  int least = 0, greatest = 0;
+  if (ce == cudaSuccess) ce = cudaDeviceGetStreamPriorityRange(&least, &greatest);
+  if (ce == cudaSuccess) ce = cudaStreamCreateWithPriority(&e->sel, cudaStreamNonBlocking, greatest);
+  if (ce == cudaSuccess) ce = cudaStreamCreateWithPriority(&e->copy, cudaStreamNonBlocking, greatest);
   for (cudaEvent_t* ev : {&e->ev_q, &e->ev_sel, &e->ev_attn[0], &e->ev_attn[1]})
     if (ce == cudaSuccess) ce = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
   for (int i = 0; i < kRing && ce == cudaSuccess; ++i) {
@@ -182,7 +186,9 @@ tls_status engine_step(tls_engine* e, const void* q, int32_t out_dtype, void* ou
   ce = cudaEventRecord(e->ready[ri], A);
   if (ce == cudaSuccess) ce = cudaStreamWaitEvent(A, e->copy_end[rp], 0);  // T_{t-1} has landed
   if (ce != cudaSuccess) return cuda_check(ce, "engine_step: wait for the transfer");
-  st = sparse_attn_impl(s, q, e->kv, e->token_idx, e->k, out_dtype, out, lse, e->ws, e->L, A);
+  // a plain launch: an early-resident attention would hold every SM while it
+  // waits, starving level 1 on the select stream and the block pulls
+  st = sparse_attn_impl(s, q, e->kv, e->token_idx, e->k, out_dtype, out, lse, e->ws, e->L, A, /*pdl=*/false);
   if (st != TLS_OK) return st;
   ce = cudaEventRecord(e->ev_attn[cur], A);
   // T_t = M_t \ C_t on the copy stream, after the attention of step t-1 (its
