@@ -99,7 +99,6 @@ def load_peaks():
 ATTN_SOURCES = {
     "sparse_attn_mma_kernel": ("decode_attn_mma.cu", "attn_common.cuh", "device_common.cuh"),
     "sparse_attn_mma_cluster_kernel": ("decode_attn_mma.cu", "attn_common.cuh", "device_common.cuh"),
-    "sparse_attn_tc_kernel": ("decode_attn_tc.cu", "attn_common.cuh", "device_common.cuh"),
     "sparse_attn_kernel": ("decode_attn.cu", "attn_common.cuh", "device_common.cuh"),
 }
 

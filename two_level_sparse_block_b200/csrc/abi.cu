@@ -20,8 +20,6 @@ tls_status sparse_attn_impl(const tls_shape& s, const void* q, const tls_kv_view
                             int k, int out_dtype, void* out, float* lse, uint8_t* ws, const WsLayout& L,
                             cudaStream_t stream, bool pdl = true);
 int attn_heads_per_cta(const tls_shape& s);
-bool attn_tc_supported(const tls_shape& s);
-int attn_tc_plan(int rows, int head_groups, int k, int* tiles, int* n_items, int* n_ctas);
 bool attn_mma_supported(const tls_shape& s);
 int attn_mma_plan(int rows, int k, int* chunks_per_row, int* n_items, int* n_ctas);
 int attn_mma_cluster_size(int rows, int hpc);
@@ -81,11 +79,6 @@ tls_status plan_workspace(const tls_shape& s, int K_b, int k, WsLayout* out) {
     // warp-streaming attention: persistent CTAs over 16-token chunks
     L.tokens_per_split = 16;
     L.splits = attn_mma_plan(rows * L.head_groups, k, &L.tiles_per_pair, &L.n_items, &L.n_ctas);
-  } else if (attn_tc_supported(s)) {
-    // tensor-core attention: persistent CTAs over 128-token tiles; a split
-    // slot per CTA that shares a (row, head group)
-    L.tokens_per_split = 128;
-    L.splits = attn_tc_plan(rows, L.head_groups, k, &L.tiles_per_pair, &L.n_items, &L.n_ctas);
   } else {
     const int target = 4 * kNumSMs;
     int splits = (target + rows * L.head_groups - 1) / (rows * L.head_groups);
@@ -159,7 +152,6 @@ extern "C" const char* tls_attn_kernel(const tls_shape* shape) {
     return attn_mma_cluster_size(rows_of(*shape) * head_groups, hpc) > 0 ? "sparse_attn_mma_cluster_kernel"
                                                                           : "sparse_attn_mma_kernel";
   }
-  if (attn_tc_supported(*shape)) return "sparse_attn_tc_kernel";
   return "sparse_attn_kernel";
 }
 

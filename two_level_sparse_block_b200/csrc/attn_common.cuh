@@ -19,7 +19,7 @@ struct AttnParams {
   int n_q_heads, n_kv_heads, group, dqk, dv;
   float scale_log2;
   int tokens_per_split, splits, head_groups, heads_per_cta;
-  int tiles_per_pair, n_items, n_ctas;  // tensor-core kernel: work partition
+  int tiles_per_pair, n_items, n_ctas;  // mma attention: chunks per (virtual) row, items, persistent CTAs
   int* err;            // workspace error word
   float* partial;      // workspace [rows][G][splits][dv + 2]
   unsigned* counters;  // workspace [rows * head_groups]
@@ -118,9 +118,6 @@ static __device__ __noinline__ void merge_splits(const AttnParams& p, int row, i
   }
 }
 
-// Tensor-core attention (decode_attn_tc.cu): 128-wide K and V rows.
-bool attn_tc_supported(const tls_shape& s);
-tls_status launch_attn_tc(const AttnParams& p, int rows, cudaStream_t stream, bool pdl);
 // Warp-streaming attention for groups of <= 16 heads (decode_attn_mma.cu).
 bool attn_mma_supported(const tls_shape& s);
 tls_status launch_attn_mma(const AttnParams& p, int rows, cudaStream_t stream, bool pdl);

@@ -50,7 +50,7 @@ struct WsLayout {
   int head_groups;     // attention CTAs along the heads of a group
   int heads_per_cta;
   int tokens_per_split;
-  int tiles_per_pair, n_items, n_ctas;  // tensor-core attention work partition
+  int tiles_per_pair, n_items, n_ctas;  // mma attention: chunks per (virtual) row, items, persistent CTAs
 };
 
 // Plans the attention launch and the workspace for (shape, K_b, k).
