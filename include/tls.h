@@ -236,14 +236,14 @@ TLS_API tls_status tls_decode_step(const tls_shape* shape, const void* q, const 
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before any stream capture.
- *   - Each call clears the tickets with cudaMemsetAsync on `stream`; it calls
- *     no cudaMalloc, cudaFree or allocating library routine.
+ *   - Each call clears the error word and the tickets with cudaMemsetAsync on
+ *     `stream`; it calls no cudaMalloc, cudaFree or allocating library routine.
  *   - All calls share the one array: two calls whose kernels overlap on the
  *     GPU (e.g. on different streams) race and give wrong results.  Issue them
  *     on one stream, or use tls_sparse_decode_attn with separate workspaces.
- *   - Shapes whose scratch exceeds the array (tickets plus
- *     rows * G * splits * (Dv + 2) floats) return TLS_ERR_CAPACITY and launch
- *     nothing.
+ *   - Shapes whose scratch exceeds the array (a 256-byte error header, the
+ *     tickets and rows * G * splits * (Dv + 2) floats) return
+ *     TLS_ERR_CAPACITY and launch nothing.
  */
 #define TLS_NOALLOC_SCRATCH_BYTES (4u << 20)
 TLS_API tls_status tls_sparse_decode_attn_noalloc(const tls_shape* shape, const void* q, const tls_kv_view* kv,

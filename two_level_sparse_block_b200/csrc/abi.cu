@@ -104,6 +104,9 @@ tls_status plan_workspace(const tls_shape& s, int K_b, int k, WsLayout* out) {
   // a call uses do not depend on arguments it is not given
   L.agg = off;
   off = align_up(off + (size_t)rows * nb * 4, 256);
+  const int npad = block_score_npad(g);
+  L.qprime = off;
+  if (npad >= 64) off = align_up(off + (size_t)rows * npad * 2 * s.qk_dim * 2, 256);
   L.partial = off;
   off = align_up(off + (size_t)rows * g * L.splits * (s.v_dim + 2) * 4, 256);
   L.tscore = off;

@@ -82,9 +82,31 @@ __host__ __device__ inline int bs_body_bytes(int stage_bytes, int nb) {
 // selects; 2, 4, 8: the row's CTAs form a cluster and select together over
 // distributed shared memory (cluster_topk.cuh); 0: the last CTA of the row
 // (a ticket) selects from the scores in the workspace.
+// Q' = [relu(q_h), min(q_h, 0)] of every row, bf16 [rows * npad][2 * Dqk]
+// (rows h >= G zero): the level-1 B operand, written once per step for wide
+// groups so that each level-1 CTA loads it by TMA instead of rebuilding it.
+// One CTA per (row, padded head): eight bf16 per thread, one 16-byte load and
+// two 16-byte stores (Dqk is a multiple of 32).
+__global__ void __launch_bounds__(128) block_query_prep_kernel(const uint16_t* q, int n_q_heads, int n_kv_heads,
+                                                                int g, int dqk, int npad, uint16_t* qp) {
+  const int row = blockIdx.x, h = blockIdx.y, b = row / n_kv_heads, kvh = row % n_kv_heads;
+  const uint4* src = reinterpret_cast<const uint4*>(q + ((int64_t)b * n_q_heads + (int64_t)kvh * g + h) * dqk);
+  uint4* out = reinterpret_cast<uint4*>(qp + ((int64_t)row * npad + h) * 2 * dqk);
+  const int n8 = dqk / 8;
+  for (int i = threadIdx.x; i < n8; i += blockDim.x) {
+    const uint4 x = h < g ? src[i] : make_uint4(0u, 0u, 0u, 0u);
+    out[i] = make_uint4(relu_bf16x2(x.x), relu_bf16x2(x.y), relu_bf16x2(x.z), relu_bf16x2(x.w));
+    out[n8 + i] = make_uint4(min0_bf16x2(x.x), min0_bf16x2(x.y), min0_bf16x2(x.z), min0_bf16x2(x.w));
+  }
+}
+
+// QT: the B operand (Q') comes from global memory by TMA (wide groups)
+// instead of being built by warps 2-3 in every CTA.
 template <int NPAD, int CL>
 __global__ void __launch_bounds__(128, 1)
-    block_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, BlockScoreParams p) {
+    block_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUtensorMap qmap,
+                          BlockScoreParams p) {
+  constexpr bool QT = NPAD >= 64;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   using L = BsSmem<NPAD>;
@@ -106,7 +128,7 @@ __global__ void __launch_bounds__(128, 1)
 
   if (tid == 0) {
     for (int s = 0; s < kBsStages; ++s) {
-      mbar_init(&full[s], 1 + 64);
+      mbar_init(&full[s], QT ? 1 : 1 + 64);
       mbar_init(&empty[s], 1);
     }
     mbar_init(done, 1);
@@ -135,8 +157,9 @@ __global__ void __launch_bounds__(128, 1)
           flags[1] = 1;
           break;
         }
-        mbar_arrive_expect_tx(&full[s], L::A_BYTES);
+        mbar_arrive_expect_tx(&full[s], L::A_BYTES + (QT ? L::B_BYTES : 0));
         tma_load_2d(sA + s * L::A_BYTES, &tmap, &full[s], kc * kBsChunk, row * p.nb + mt * kBsTile);
+        if constexpr (QT) tma_load_2d(sB + s * L::B_BYTES, &qmap, &full[s], kc * kBsChunk, row * NPAD);
       }
     }
   } else if (warp == 1) {
@@ -162,7 +185,7 @@ __global__ void __launch_bounds__(128, 1)
       }
       if (ok) tc_commit(done);
     }
-  } else {
+  } else if (!QT) {
     // Q' producers: row h of a stage holds Q'[h, kc*64 .. kc*64+63] as eight
     // 16-byte chunks, chunk c stored at position c ^ (h % 8) (128B swizzle).
     const int t = tid - 64;
@@ -352,7 +375,8 @@ bool use_simt() {
 }
 
 template <int NPAD, int CL>
-tls_status launch_tc(const CUtensorMap& tmap, const BlockScoreParams& p, int rows, cudaStream_t stream) {
+tls_status launch_tc(const CUtensorMap& tmap, const CUtensorMap& qmap, const BlockScoreParams& p, int rows,
+                     cudaStream_t stream) {
   using L = BsSmem<NPAD>;
   const int body = bs_body_bytes<CL>(L::STAGE_BYTES, p.nb);
   const size_t smem = 1024 + (size_t)((body + 7) & ~7) + (2 * kBsStages + 1) * 8 + 16;
@@ -362,20 +386,21 @@ tls_status launch_tc(const CUtensorMap& tmap, const BlockScoreParams& p, int row
   const dim3 grid((unsigned)((p.nb + kBsTile - 1) / kBsTile), (unsigned)rows);
   if constexpr (CL >= 2)
     return cuda_check(launch_cluster(block_score_tc_kernel<NPAD, CL>, grid, dim3(128), smem, stream, (unsigned)CL,
-                                     tmap, p),
+                                     tmap, qmap, p),
                       "select_blocks: block_score_tc launch");
-  block_score_tc_kernel<NPAD, CL><<<grid, 128, smem, stream>>>(tmap, p);
+  block_score_tc_kernel<NPAD, CL><<<grid, 128, smem, stream>>>(tmap, qmap, p);
   return launch_check("select_blocks: block_score_tc launch");
 }
 
 template <int CL>
-tls_status launch_tc_group(const CUtensorMap& tmap, const BlockScoreParams& p, int rows, cudaStream_t stream) {
+tls_status launch_tc_group(const CUtensorMap& tmap, const CUtensorMap& qmap, const BlockScoreParams& p, int rows,
+                           cudaStream_t stream) {
   const int g = p.group;
-  if (g <= 16) return launch_tc<16, CL>(tmap, p, rows, stream);
-  if (g <= 32) return launch_tc<32, CL>(tmap, p, rows, stream);
-  if (g <= 64) return launch_tc<64, CL>(tmap, p, rows, stream);
-  if (g <= 128) return launch_tc<128, CL>(tmap, p, rows, stream);
-  if (g <= 256) return launch_tc<256, CL>(tmap, p, rows, stream);
+  if (g <= 16) return launch_tc<16, CL>(tmap, qmap, p, rows, stream);
+  if (g <= 32) return launch_tc<32, CL>(tmap, qmap, p, rows, stream);
+  if (g <= 64) return launch_tc<64, CL>(tmap, qmap, p, rows, stream);
+  if (g <= 128) return launch_tc<128, CL>(tmap, qmap, p, rows, stream);
+  if (g <= 256) return launch_tc<256, CL>(tmap, qmap, p, rows, stream);
   return fail(TLS_ERR_UNSUPPORTED, "select_blocks: group size %d > 256", g);
 }
 
@@ -421,14 +446,31 @@ tls_status select_blocks_impl(const tls_shape& s, const void* q, const void* met
                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(TLS_ERR_CUDA, "select_blocks: cuTensorMapEncodeTiled failed (%d)", (int)r);
+  // wide groups: Q' written once per step, loaded by TMA in every CTA
+  CUtensorMap qmap = tmap;  // unused below 64 padded heads
+  const int npad = block_score_npad(p.group);
+  if (npad >= 64) {
+    uint16_t* qp = reinterpret_cast<uint16_t*>(ws + L.qprime);
+    block_query_prep_kernel<<<dim3(rows, npad), 128, 0, stream>>>((const uint16_t*)q, s.n_q_heads, s.n_kv_heads,
+                                                                   p.group, s.qk_dim, npad, qp);
+    tls_status lst = launch_check("select_blocks: query prep launch");
+    if (lst != TLS_OK) return lst;
+    const cuuint64_t qdims[2] = {(cuuint64_t)(2 * s.qk_dim), (cuuint64_t)rows * (cuuint64_t)npad};
+    const cuuint64_t qstrides[1] = {(cuuint64_t)(2 * s.qk_dim) * 2};
+    const cuuint32_t qbox[2] = {(cuuint32_t)kBsChunk, (cuuint32_t)npad};
+    r = g_encode(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, qp, qdims, qstrides, qbox, estr,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(TLS_ERR_CUDA, "select_blocks: cuTensorMapEncodeTiled (Q') failed (%d)", (int)r);
+  }
 
   // the row's tiles select together when they fit one cluster
   const int tiles = (nb + kBsTile - 1) / kBsTile;
-  if (tiles == 1) return launch_tc_group<1>(tmap, p, rows, stream);
-  if (tiles == 2) return launch_tc_group<2>(tmap, p, rows, stream);
-  if (tiles == 4) return launch_tc_group<4>(tmap, p, rows, stream);
-  if (tiles == 8) return launch_tc_group<8>(tmap, p, rows, stream);
-  return launch_tc_group<0>(tmap, p, rows, stream);
+  if (tiles == 1) return launch_tc_group<1>(tmap, qmap, p, rows, stream);
+  if (tiles == 2) return launch_tc_group<2>(tmap, qmap, p, rows, stream);
+  if (tiles == 4) return launch_tc_group<4>(tmap, qmap, p, rows, stream);
+  if (tiles == 8) return launch_tc_group<8>(tmap, qmap, p, rows, stream);
+  return launch_tc_group<0>(tmap, qmap, p, rows, stream);
 }
 
 }  // namespace tls

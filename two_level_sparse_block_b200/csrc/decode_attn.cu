@@ -357,23 +357,25 @@ extern "C" tls_status tls_sparse_decode_attn_noalloc(const tls_shape* shape, con
   WsLayout L;
   st = plan_workspace(s, K_b, k, &L);
   if (st != TLS_OK) return st;
-  // tickets first, then the partials, inside the static array
+  // the error word (256-byte header), the tickets, then the partials, inside the static array
+  const size_t header = 256;
   const size_t ticket_bytes = align_up((size_t)rows_of(s) * L.head_groups * sizeof(unsigned), 256);
   const size_t partial_bytes = (size_t)rows_of(s) * group_of(s) * L.splits * (s.v_dim + 2) * sizeof(float);
-  if (ticket_bytes + partial_bytes > (size_t)TLS_NOALLOC_SCRATCH_BYTES)
+  if (header + ticket_bytes + partial_bytes > (size_t)TLS_NOALLOC_SCRATCH_BYTES)
     return fail(TLS_ERR_CAPACITY,
                 "sparse_decode_attn_noalloc: this shape needs %zu bytes of scratch, above the fixed %u-byte "
                 "array; use tls_sparse_decode_attn with a workspace",
-                ticket_bytes + partial_bytes, (unsigned)TLS_NOALLOC_SCRATCH_BYTES);
+                header + ticket_bytes + partial_bytes, (unsigned)TLS_NOALLOC_SCRATCH_BYTES);
   void* base = nullptr;
   st = scratch_address(&base);
   if (st != TLS_OK) return st;
-  // the array keeps the previous call's contents: the tickets must start at zero
-  cudaError_t e = cudaMemsetAsync(base, 0, ticket_bytes, (cudaStream_t)stream);
+  // the array keeps the previous call's contents: error word and tickets must start at zero
+  cudaError_t e = cudaMemsetAsync(base, 0, header + ticket_bytes, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_check(e, "sparse_decode_attn_noalloc: clear tickets");
   WsLayout S = L;
-  S.att_counter = 0;
-  S.partial = ticket_bytes;
+  S.err = 0;
+  S.att_counter = header;
+  S.partial = header + ticket_bytes;
   return sparse_attn_impl(s, q, *kv, token_idx, k, out_dtype, out, lse, (uint8_t*)base, S, (cudaStream_t)stream,
                           /*pdl=*/true);
 }

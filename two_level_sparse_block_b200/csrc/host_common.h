@@ -25,6 +25,8 @@ tls_status check_shape(const tls_shape* s);
 inline int64_t n_blocks(const tls_shape& s) { return s.ctx_len / s.block_size; }
 inline int rows_of(const tls_shape& s) { return s.batch * s.n_kv_heads; }
 inline int group_of(const tls_shape& s) { return s.n_q_heads / s.n_kv_heads; }
+// Heads of a KV group padded to the level-1 GEMM's N (16, 32, 64, 128 or 256).
+inline int block_score_npad(int g) { return g <= 16 ? 16 : g <= 32 ? 32 : g <= 64 ? 64 : g <= 128 ? 128 : 256; }
 
 inline tls_status cuda_check(cudaError_t e, const char* what) {
   if (e == cudaSuccess) return TLS_OK;
@@ -43,6 +45,7 @@ struct WsLayout {
   size_t tok_counter;  // unsigned[rows]
   size_t att_counter;  // unsigned[rows]
   size_t agg;          // float[rows * NB]
+  size_t qprime;       // bf16[rows * NPAD * 2 * Dqk] when NPAD >= 64 (level-1 B operand), else empty
   size_t tscore;       // float[rows * K_b * bs]
   size_t partial;      // float[rows * G * splits * (Dv + 2)]
   size_t total;
