@@ -102,8 +102,10 @@ TLS_API int32_t tls_version(void);
  * Name of the attention kernel tls_sparse_decode_attn launches for this
  * shape: "sparse_attn_mma_cluster_kernel" or "sparse_attn_mma_kernel" for
  * 128-wide K and V rows (one cluster of CTAs per row and head group of <= 16
- * heads while such a grid fits two CTAs per SM; else persistent CTAs), and
- * "sparse_attn_kernel" for every other shape (e.g. the MLA latent cache).  A
+ * heads while such a grid fits two CTAs per SM; else persistent CTAs),
+ * "sparse_attn_mla_kernel" for the MLA latent cache (Dqk 576, Dv 512 taken
+ * from the same row, G a multiple of 16), and "sparse_attn_kernel" for every
+ * other shape.  A
  * static string owned by the library; NULL if the shape is invalid
  * (tls_last_error says why).  Host only, no device work.
  */

@@ -59,6 +59,10 @@ SMALL = [
     small("s_g16_bs32", n_q_heads=16, n_kv_heads=1, block_size=32, ctx_len=4096, K_b=20, k=640, seed=15),
     small("s_mla", batch=2, n_q_heads=16, n_kv_heads=1, qk_dim=576, v_dim=512, v_offset=0, ctx_len=1024,
           block_size=64, K_b=6, k=200, n_label=32, n_outlier=0, label_from_outliers=False, kv_std=0.7071, seed=16),
+    small("s_mla_g32", batch=2, n_q_heads=32, n_kv_heads=1, qk_dim=576, v_dim=512, v_offset=0, ctx_len=2048,
+          block_size=64, K_b=7, k=333, n_label=32, n_outlier=0, label_from_outliers=False, kv_std=0.7071, seed=19),
+    small("s_mla_g8_simt", batch=1, n_q_heads=8, n_kv_heads=1, qk_dim=576, v_dim=512, v_offset=0, ctx_len=1024,
+          block_size=64, K_b=5, k=150, n_label=32, n_outlier=0, label_from_outliers=False, kv_std=0.7071, seed=20),
     small("s_k_eq_1", K_b=1, k=1, seed=17),
     small("s_all", ctx_len=512, K_b=32, k=512, seed=18),
 ]

@@ -23,6 +23,8 @@ int attn_heads_per_cta(const tls_shape& s);
 bool attn_mma_supported(const tls_shape& s);
 int attn_mma_plan(int rows, int k, int* chunks_per_row, int* n_items, int* n_ctas);
 int attn_mma_cluster_size(int rows, int hpc);
+bool attn_mla_supported(const tls_shape& s);
+int attn_mla_tokens_per_split(int k);
 
 namespace {
 thread_local char g_err[512] = {0};
@@ -79,6 +81,10 @@ tls_status plan_workspace(const tls_shape& s, int K_b, int k, WsLayout* out) {
     // warp-streaming attention: persistent CTAs over 16-token chunks
     L.tokens_per_split = 16;
     L.splits = attn_mma_plan(rows * L.head_groups, k, &L.tiles_per_pair, &L.n_items, &L.n_ctas);
+  } else if (attn_mla_supported(s)) {
+    // MLA: 8 token splits per (row, head block) merged inside a cluster; no workspace partials
+    L.tokens_per_split = attn_mla_tokens_per_split(k);
+    L.splits = 1;
   } else {
     const int target = 4 * kNumSMs;
     int splits = (target + rows * L.head_groups - 1) / (rows * L.head_groups);
@@ -155,6 +161,7 @@ extern "C" const char* tls_attn_kernel(const tls_shape* shape) {
     return attn_mma_cluster_size(rows_of(*shape) * head_groups, hpc) > 0 ? "sparse_attn_mma_cluster_kernel"
                                                                           : "sparse_attn_mma_kernel";
   }
+  if (attn_mla_supported(*shape)) return "sparse_attn_mla_kernel";
   return "sparse_attn_kernel";
 }
 

@@ -121,6 +121,10 @@ static __device__ __noinline__ void merge_splits(const AttnParams& p, int row, i
 // Warp-streaming attention for groups of <= 16 heads (decode_attn_mma.cu).
 bool attn_mma_supported(const tls_shape& s);
 tls_status launch_attn_mma(const AttnParams& p, int rows, cudaStream_t stream, bool pdl);
+// MLA latent attention (decode_attn_mla.cu): Dqk 576, Dv 512 = the row's first 512, G % 16 == 0.
+bool attn_mla_supported(const tls_shape& s);
+int attn_mla_tokens_per_split(int k);
+tls_status launch_attn_mla(const AttnParams& p, int rows, cudaStream_t stream, bool pdl);
 int attn_mma_cluster_size(int rows, int hpc);
 
 }  // namespace tls

@@ -258,6 +258,7 @@ tls_status sparse_attn_impl(const tls_shape& s, const void* q, const tls_kv_view
   p.err = reinterpret_cast<int*>(ws + L.err);
   const int rows = rows_of(s);
   if (attn_mma_supported(s)) return launch_attn_mma(p, rows, stream, pdl);
+  if (attn_mla_supported(s)) return launch_attn_mla(p, rows, stream, pdl);
   const int pk = (s.qk_dim + 127) / 128, pv = (s.v_dim + 127) / 128;
   const int hg = L.heads_per_cta;
   if (pk == 1 && pv == 1) {
@@ -283,6 +284,7 @@ tls_status sparse_attn_impl(const tls_shape& s, const void* q, const tls_kv_view
 int attn_heads_per_cta(const tls_shape& s) {
   const int g = group_of(s);
   if (attn_mma_supported(s)) return g < 16 ? g : 16;
+  if (attn_mla_supported(s)) return 16;
   const int pk = (s.qk_dim + 127) / 128, pv = (s.v_dim + 127) / 128;
   int cap = (pk == 1 && pv == 1) ? 8 : (pk <= 2 && pv <= 2) ? 4 : 2;
   int hg = 1;
