@@ -48,6 +48,7 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-offload", action="store_true", help="skip the offload-engine measurement (c4)")
+    ap.add_argument("--no-other-configs", action="store_true", help="skip the c1 / c3 step measurements")
     ap.add_argument("--e2e-steps", type=int, default=300)
     return ap.parse_args()
 
@@ -82,8 +83,10 @@ def algorithmic_bytes(cfg):
 
 def launches_per_step(cfg):
     """Kernels one step launches: level 1 (block scores + top-K_b), level 2
-    (token scores + top-k) and the attention kernel."""
-    return 3
+    (token scores + top-k) and the attention kernel, plus the query-prep
+    kernel of level 1 for groups padded to 64 heads or more."""
+    g = cfg.n_q_heads // cfg.n_kv_heads
+    return 3 + (1 if g > 32 else 0)
 
 
 def load_peaks():
@@ -211,6 +214,54 @@ def time_oracle(cfg, q, K, V, lab, seconds, rows_sample=8):
             "sample": f"{done} (batch row, KV head) decode_row calls over {len(pick)} seeded rows of "
                       f"{cfg.name} in {el:.1f} s; scaled to all {cfg.rows} rows of one step",
             "s_per_step": step_s}
+
+
+def measure_config(name, dev, steps=200, warmup=10):
+    """One more workload measured like the headline: tls_decode_step replayed
+    from a CUDA graph, L2 flushed (write + read of 256 MB) before each step,
+    CUDA events around each replay."""
+    import synth
+    import torch
+    from two_level_sparse_block_b200 import runtime, tls
+    c = synth.get_config(name)
+    q = synth.gen_queries(c)
+    K, V, _ = synth.gen_kv(c, q)
+    lab = synth.gen_label_channels(c)
+    st = runtime.state_for_config(c, q, K, V, lab, device=dev)
+    del K, V
+    flush = torch.empty(64 << 20, dtype=torch.float32, device=dev)
+    flush_rd = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+    cap = torch.cuda.Stream(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(cap):
+        st.step(stream=cap)
+        with torch.cuda.graph(g, stream=cap):
+            st.step(stream=cap)
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    times = []
+    for i in range(warmup + steps):
+        flush.fill_(float(i))
+        torch.sum(flush_rd, dim=0, out=sink)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+        if i >= warmup:
+            times.append((a, b))
+    torch.cuda.synchronize(dev)
+    if st.check_device_error() != 0:
+        raise RuntimeError(f"device error in {name}")
+    ts = [x.elapsed_time(y) for x, y in times]
+    ms = statistics.mean(ts)  # (event ticks are coarse: the mean, not the median, averages them out)
+    ab = algorithmic_bytes(c)
+    del g
+    return {"us_per_step": ms * 1e3, "us_per_step_median": statistics.median(ts) * 1e3,
+            "decode_tokens_per_s": c.batch / (ms / 1e3),
+            "algorithmic_bytes": ab["step"], "achieved_gbs": ab["step"] / (ms / 1e3) / 1e9,
+            "attention_kernel": tls.tls_attn_kernel(st.shape), "steps": steps,
+            "l2": "flushed before every step (write + read of 256 MB)"}
 
 
 def measure_offload_engine(dev, steps=64):
@@ -468,6 +519,8 @@ def main():
     }
     if rank == 0 and world == 1 and not args.no_offload:
         line["offload_engine"] = measure_offload_engine(dev)
+    if rank == 0 and world == 1 and not args.no_other_configs:
+        line["other_configs"] = {n: measure_config(n, dev) for n in ("c1", "c3") if n != c.name}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = time_oracle(c, q, K, V, lab, args.cpu_seconds)
         line["cpu_baseline"].pop("s_per_step", None)

@@ -340,6 +340,77 @@ def test_crowded_threshold_takes_the_lowest_positions():
         assert got["token_idx"][0, h].tolist() == r2["token_idx"].tolist()
 
 
+def _crowd_depth(scores, k, levels=3):
+    """Levels of 256 sub-bins (float32 arithmetic, as the cluster selection
+    bins) needed before the bin of the k-th largest score holds <= 128."""
+    s = np.asarray(scores, dtype=np.float32)
+    lo, inv = np.float32(s.min()), np.float32(256.0) / np.float32(s.max() - s.min())
+    cell = np.ones(s.size, dtype=bool)
+    need = k
+    for lv in range(levels):
+        b = np.clip(((s - lo) * inv).astype(np.int64), 0, 255)
+        cnt = np.bincount(b[cell], minlength=256)
+        above = 0
+        for tb in range(255, -1, -1):
+            if above + cnt[tb] >= need:
+                break
+            above += cnt[tb]
+        need -= above
+        if cnt[tb] <= 128:
+            return lv
+        cell &= b == tb
+        lo, inv = np.float32(lo + np.float32(tb) / inv), np.float32(inv * np.float32(256.0))
+    return levels
+
+
+# a few tokens with K rows 1e4 times the rest stretch the score range so far
+# that all other candidates share one value bin: the cluster selections (16
+# and 8 CTAs a row at level 2, several at level 1) must split that bin with
+# sub-bins instead of handing the row to one CTA
+DENSE = [
+    small("s_dense_cl16", batch=1, n_q_heads=16, n_kv_heads=1, ctx_len=16384, block_size=64, K_b=128, k=4096,
+          seed=43),
+    small("s_dense_cl8_r32", batch=2, n_q_heads=64, n_kv_heads=2, ctx_len=8192, block_size=64, K_b=64, k=2000,
+          n_label=32, seed=44),
+]
+
+
+@pytest.mark.parametrize("cfg", DENSE, ids=lambda c: c.name)
+def test_dense_threshold_splits_with_sub_bins(cfg):
+    runtime, tls = _rt()
+    from synth import bf16_bits_from_f32
+    q, K, V, lab = gen_case(cfg)
+    Kf = f32_from_bf16_bits(K)
+    rng = np.random.default_rng(cfg.seed)
+    for b in range(cfg.batch):
+        for h in range(cfg.n_kv_heads):
+            Kf[b, h, rng.choice(cfg.ctx_len, 4, replace=False)] *= 1.0e4
+    K = bf16_bits_from_f32(Kf)
+    data = (q, K, V, lab)
+    st = runtime.state_for_config(cfg, q, K, V, lab)
+    got = run_stages(st)
+    bs = cfg.block_size
+    deepest = 0
+    for b in range(cfg.batch):
+        for h in range(cfg.n_kv_heads):
+            where = f"{cfg.name} row ({b},{h})"
+            # both selections are the exact top-k of the GPU's own float32
+            # scores (ties to the lower position): the decision in one precision
+            bsc = got["block_score"][b, h]
+            assert got["block_idx"][b, h].tolist() == oracle.topk_ascending(bsc, cfg.K_b).tolist(), where + " blocks"
+            gb = got["block_idx"][b, h]
+            cand = (gb[:, None] * bs + np.arange(bs)[None, :]).reshape(-1)
+            ts = got["token_score"][b, h]
+            pos = np.searchsorted(cand, got["token_idx"][b, h])
+            assert np.array_equal(cand[pos], got["token_idx"][b, h]), where + ": token outside the chosen blocks"
+            assert pos.tolist() == oracle.topk_ascending(ts, cfg.k).tolist(), where + " tokens"
+            deepest = max(deepest, _crowd_depth(ts, cfg.k))
+            # and the scores, tokens and output are the oracle's
+            check_row(cfg, data, got, st, b, h)
+    assert deepest >= 1, "workload lost its construction: no sub-bins needed"
+    assert st.check_device_error() == 0
+
+
 @pytest.mark.parametrize("cfg", SMALL + [get_config("c1")], ids=lambda c: c.name)
 def test_fused_select_equals_the_two_level_calls(cfg):
     st, data = make_state(cfg)

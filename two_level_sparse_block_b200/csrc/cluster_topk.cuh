@@ -14,7 +14,9 @@
 //
 //   1. key range: local min / max, pushed; barrier
 //   2. 256 value bins over the range: local histogram, pushed; barrier
-//   3. every CTA sums the histograms and finds the bin of the k-th key
+//   3. every CTA sums the histograms and finds the bin of the k-th key; if
+//      that bin holds more than kTopkRankMax keys, steps 2-3 repeat with 256
+//      sub-bins of it (at most kTopkLevels levels in all)
 //   4. the local keys of that bin are compacted and pushed; barrier
 //   5. every CTA ranks the (few) candidates pairwise: tau and how many keys
 //      equal to tau to take
@@ -24,7 +26,8 @@
 //
 // Returns false, uniformly over the cluster and with nothing written, when
 // the keys cannot be binned (not finite, or all equal) or the threshold bin
-// holds more than kTopkRankMax keys; the caller then selects with one CTA.
+// still holds more than kTopkRankMax keys after the last level of sub-bins
+// (keys equal over a wide run); the caller then selects with one CTA.
 // On both return paths the other CTAs' shared memory is still alive until
 // the caller's next cluster barrier.
 //
@@ -39,11 +42,20 @@
 
 namespace tls {
 
+constexpr int kTopkLevels = 3;
+
+// bin of a key at a sub-bin level: the bounds are rounded, so a key of the
+// parent bin may fall just outside [fmin, fmin + 256 / inv]; clamping keeps
+// the map monotone in the key, which is all the selection relies on
+__device__ __forceinline__ int topk_sub_bin(uint32_t key, float fmin, float inv) {
+  return max(0, min(255, (int)((key_float(key) - fmin) * inv)));
+}
+
 template <int CL>
 struct alignas(16) ClusterTopkScratch {
   // written by the cluster's CTAs (index = writer's rank)
   uint32_t lo[CL], hi[CL];
-  int hist[CL][256];
+  int hist[2][CL][256];  // alternate levels use alternate halves
   int ncand[CL];
   alignas(16) uint32_t cand[CL][kTopkRankMax];  // rows read as uint4
   int tot_gt[CL], tot_eq[CL];
@@ -51,8 +63,10 @@ struct alignas(16) ClusterTopkScratch {
   int hsum[256];
   uint32_t wlo[32], whi[32];
   int wgt[32], weq[32];
-  int tbin, need, nloc, take;
+  int tbin, need, tcount, nloc, take;
   uint32_t tau;
+  float lmin[kTopkLevels], linv[kTopkLevels];
+  int lbin[kTopkLevels];
   uint32_t lcand[kTopkRankMax];
 };
 
@@ -109,61 +123,92 @@ __device__ bool cluster_topk_ascending(const uint32_t* keys, int n_loc, int pos0
   const float fmin = key_float(glo), fmax = key_float(ghi);
   const float span = fmax - fmin;
   if (!(glo != ghi && isfinite(fmin) && isfinite(fmax) && isfinite(span) && span > 0.0f)) return false;
-  const float inv = 256.0f / span;
-
-  // 2. local histogram, pushed to every CTA
-  for (int i = tid; i < 256; i += NT) sm.hsum[i] = 0;
-  __syncthreads();
-  for (int i = tid; i < n_loc; i += NT) atomicAdd(&sm.hsum[topk_value_bin(keys[i], fmin, inv)], 1);
-  __syncthreads();
-  for (int i = tid; i < 256 * CL; i += NT) {
-    const int j = i >> 8, b = i & 255;
-    *cluster.map_shared_rank(&sm.hist[rank][b], j) = sm.hsum[b];
+  if (tid == 0) {
+    sm.lmin[0] = fmin;
+    sm.linv[0] = 256.0f / span;
   }
-  cluster.sync();
+  // whether a key lies in the threshold bins of levels 0 .. upto - 1
+  auto in_cell = [&](uint32_t key, int upto) {
+    bool m = true;
+    for (int l = 0; l < upto; ++l) m = m && topk_sub_bin(key, sm.lmin[l], sm.linv[l]) == sm.lbin[l];
+    return m;
+  };
 
-  // 3. the bin of the k-th largest key (every CTA finds the same)
-  for (int b = tid; b < 256; b += NT) {
-    int s = 0;
-#pragma unroll
-    for (int j = 0; j < CL; ++j) s += sm.hist[j][b];
-    sm.hsum[b] = s;
-  }
-  __syncthreads();
-  if (tid < 32) {
-    int local[8];
-    int s = 0;
-#pragma unroll
-    for (int d = 0; d < 8; ++d) {
-      local[d] = sm.hsum[255 - (tid * 8 + d)];
-      s += local[d];
+  int lv = 0, need = k;
+  for (;;) {
+    // 2. local histogram of the keys in the current cell, pushed to every CTA
+    for (int i = tid; i < 256; i += NT) sm.hsum[i] = 0;
+    __syncthreads();
+    const float lmin = sm.lmin[lv], linv = sm.linv[lv];
+    for (int i = tid; i < n_loc; i += NT) {
+      const uint32_t key = keys[i];
+      if (in_cell(key, lv)) atomicAdd(&sm.hsum[topk_sub_bin(key, lmin, linv)], 1);
     }
-    int incl = s;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (tid >= o) incl += y;
+    __syncthreads();
+    for (int i = tid; i < 256 * CL; i += NT) {
+      const int j = i >> 8, b = i & 255;
+      *cluster.map_shared_rank(&sm.hist[lv & 1][rank][b], j) = sm.hsum[b];
     }
-    int above = incl - s;
-    if (above < k && incl >= k) {
-      int d = 0;
-      for (; d < 8; ++d) {
-        if (above + local[d] >= k) break;
-        above += local[d];
+    cluster.sync();
+
+    // 3. the bin of the need-th largest key of the cell (every CTA finds the same)
+    for (int b = tid; b < 256; b += NT) {
+      int s = 0;
+#pragma unroll
+      for (int j = 0; j < CL; ++j) s += sm.hist[lv & 1][j][b];
+      sm.hsum[b] = s;
+    }
+    __syncthreads();
+    if (tid < 32) {
+      int local[8];
+      int s = 0;
+#pragma unroll
+      for (int d = 0; d < 8; ++d) {
+        local[d] = sm.hsum[255 - (tid * 8 + d)];
+        s += local[d];
       }
-      sm.tbin = 255 - (tid * 8 + d);
-      sm.need = k - above;
+      int incl = s;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (tid >= o) incl += y;
+      }
+      int above = incl - s;
+      if (above < need && incl >= need) {
+        int d = 0;
+        for (; d < 8; ++d) {
+          if (above + local[d] >= need) break;
+          above += local[d];
+        }
+        const int tb = 255 - (tid * 8 + d);
+        sm.tbin = tb;
+        sm.need = need - above;
+        sm.tcount = local[d];
+        sm.lbin[lv] = tb;
+        if (lv + 1 < kTopkLevels) {
+          // sub-bins of the threshold bin for the next level
+          sm.lmin[lv + 1] = lmin + (float)tb / linv;
+          sm.linv[lv + 1] = linv * 256.0f;
+        }
+      }
+      if (tid == 0) sm.nloc = 0;
     }
-    if (tid == 0) sm.nloc = 0;
+    __syncthreads();
+    // (hsum is cleared by the next level before every thread could read it,
+    // so the bin's count travels in its own field)
+    need = sm.need;
+    if (sm.tcount <= kTopkRankMax) break;  // uniform over the cluster
+    if (lv + 1 == kTopkLevels || !isfinite(sm.lmin[lv + 1]) || !isfinite(sm.linv[lv + 1])) return false;
+    ++lv;
   }
-  __syncthreads();
   const int tbin = sm.tbin;
+  const float bmin = sm.lmin[lv], binv = sm.linv[lv];
 
   // 4. local keys of that bin, pushed to every CTA
   for (int base = 0; base < n_loc; base += NT) {
     const int i = base + tid;
     const uint32_t key = i < n_loc ? keys[i] : 0u;
-    const bool hit = i < n_loc && topk_value_bin(key, fmin, inv) == tbin;
+    const bool hit = i < n_loc && topk_sub_bin(key, bmin, binv) == tbin && in_cell(key, lv);
     const unsigned bal = __ballot_sync(0xffffffffu, hit);
     if (bal == 0u) continue;  // warp-uniform
     int slot0 = 0;
@@ -191,7 +236,6 @@ __device__ bool cluster_topk_ascending(const uint32_t* keys, int n_loc, int pos0
   for (int j = 0; j < CL; ++j) nc += sm.ncand[j];
   if (nc > kTopkRankMax) return false;
   if (tid < nc) {
-    const int need = sm.need;
     int t = tid, jj = 0;
     while (t >= sm.ncand[jj]) t -= sm.ncand[jj++];
     const uint32_t mine = sm.cand[jj][t];

@@ -129,6 +129,137 @@ __device__ __forceinline__ void score_candidates(const TokenParams& p, int row, 
   }
 }
 
+// Token scores on the tensor cores for wide groups (G >= 16, R = 16 or 32):
+// per warp step 16 candidates, S[cand, head] = code[cand, :] . qlab[head, :]
+// as m16n8k16 bf16 MMAs with fp32 accumulation (M = 16 candidates, N = 8
+// heads per n-tile, K = the R label channels).  INT4 codes are integers in
+// [-7, 7], exact in bf16, and qlab holds bf16 values, so every product is
+// exact.  Then the max over the group's heads (n-tiles and lanes), times the
+// token's scale.  Same output as score_candidates.
+__device__ __forceinline__ uint32_t tok_pack_bf16(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// the two INT4 codes of one byte (low nibble = even channel) as bf16x2
+__device__ __forceinline__ uint32_t tok_codes_bf16x2(uint32_t byte) {
+  const int lo = (int)((byte & 0xFu) ^ 8u) - 8, hi = (int)(((byte >> 4) & 0xFu) ^ 8u) - 8;
+  return tok_pack_bf16((float)lo, (float)hi);
+}
+__device__ __forceinline__ void tok_mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+template <int R, int NT, int NTILE>
+__device__ __forceinline__ void score_candidates_tc(const TokenParams& p, int row, const float* qlab,
+                                                    const int32_t* bidx, int c0, int c1, uint32_t* keys) {
+  static_assert(R == 16 || R == 32, "label channels for the tensor-core scorer");
+  constexpr int KS = R / 16, NW = NT / 32;
+  const int g = p.group;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
+  // B fragments: n-tile j holds heads 8j .. 8j + 7 (zero beyond G)
+  uint32_t bq[NTILE][KS][2];
+#pragma unroll
+  for (int j = 0; j < NTILE; ++j) {
+    const int h = 8 * j + gq;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      const float* qh = qlab + h * R + ks * 16 + 2 * tq;
+      bq[j][ks][0] = h < g ? tok_pack_bf16(qh[0], qh[1]) : 0u;
+      bq[j][ks][1] = h < g ? tok_pack_bf16(qh[8], qh[9]) : 0u;
+    }
+  }
+  const CandidateToken map{bidx, p.bs};
+  // U steps of 16 candidates per warp iteration: all their code and scale
+  // loads are in flight before the first MMA
+  constexpr int U = 4;
+  for (int base0 = c0 + warp * 16; base0 < c1; base0 += NW * 16 * U) {
+    uint32_t w[U][2][KS * 2];  // code words of fragment rows gq, gq + 8
+    float sc[U][2];
+    bool ok[U][2];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int base = base0 + u * NW * 16;
+#pragma unroll
+      for (int hlf = 0; hlf < 2; ++hlf) {
+        const int i = base + gq + 8 * hlf;
+        ok[u][hlf] = i < c1;
+        const int64_t at = (int64_t)row * p.ctx_len + (ok[u][hlf] ? map(i) : 0);
+        if constexpr (R == 16) {
+          const uint2 c = ok[u][hlf] ? *reinterpret_cast<const uint2*>(p.codes + at * 8) : make_uint2(0u, 0u);
+          w[u][hlf][0] = c.x;
+          w[u][hlf][1] = c.y;
+        } else {
+          const uint4 c = ok[u][hlf] ? *reinterpret_cast<const uint4*>(p.codes + at * 16) : make_uint4(0u, 0u, 0u, 0u);
+          w[u][hlf][0] = c.x;
+          w[u][hlf][1] = c.y;
+          w[u][hlf][2] = c.z;
+          w[u][hlf][3] = c.w;
+        }
+        sc[u][hlf] = ok[u][hlf] ? p.scales[at] : 0.0f;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int base = base0 + u * NW * 16;
+      if (base >= c1) break;  // warp-uniform
+      float acc[NTILE][4];
+#pragma unroll
+      for (int j = 0; j < NTILE; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        // channels 16 ks + 2 tq, +1 are byte 8 ks + tq; channels + 8, + 9 are byte 8 ks + tq + 4
+        const uint32_t lo0 = (w[u][0][2 * ks] >> (8 * tq)) & 0xFFu, hi0 = (w[u][0][2 * ks + 1] >> (8 * tq)) & 0xFFu;
+        const uint32_t lo1 = (w[u][1][2 * ks] >> (8 * tq)) & 0xFFu, hi1 = (w[u][1][2 * ks + 1] >> (8 * tq)) & 0xFFu;
+        const uint32_t a[4] = {tok_codes_bf16x2(lo0), tok_codes_bf16x2(lo1), tok_codes_bf16x2(hi0),
+                               tok_codes_bf16x2(hi1)};
+#pragma unroll
+        for (int j = 0; j < NTILE; ++j) tok_mma(acc[j], a, bq[j][ks][0], bq[j][ks][1]);
+      }
+      // max over the group's heads: fragment columns 2 tq, 2 tq + 1 of every n-tile, then the 4 lanes of a row
+      float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < NTILE; ++j) {
+        const int h = 8 * j + 2 * tq;
+        if (h < g) {
+          mx0 = fmaxf(mx0, acc[j][0]);
+          mx1 = fmaxf(mx1, acc[j][2]);
+        }
+        if (h + 1 < g) {
+          mx0 = fmaxf(mx0, acc[j][1]);
+          mx1 = fmaxf(mx1, acc[j][3]);
+        }
+      }
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+      if (tq == 0) {
+#pragma unroll
+        for (int hlf = 0; hlf < 2; ++hlf) {
+          if (!ok[u][hlf]) continue;
+          const int i = base + gq + 8 * hlf;
+          const float score = sc[u][hlf] * (hlf == 0 ? mx0 : mx1);
+          keys[i - c0] = float_key(score);
+          if (p.token_score != nullptr) p.token_score[(int64_t)row * p.n_cand + i] = score;
+        }
+      }
+    }
+  }
+}
+
+// CTAs per row of the cluster kernel: 4, or (tensor-core scoring only) 8 / 16
+// while the rows leave most SMs idle and every CTA keeps 512 candidates or more.
+__host__ __device__ inline int token_cluster_size(int rows, int n_cand, bool tc) {
+  int cl = 4;
+  while (tc && cl < 16 && (int64_t)rows * cl * 2 <= 148 && n_cand >= cl * 2 * 512) cl *= 2;
+  return cl;
+}
+
 // Whether level 2 of a row is light enough for one 4-CTA cluster (the
 // scores of all candidates in shared memory, no device-wide exchange).
 __host__ __device__ inline bool token_cluster_fits(int group, int n_label, int n_cand) {

@@ -77,48 +77,51 @@ __global__ void __launch_bounds__(NT) token_select_kernel(TokenParams p) {
                          [bidx, bs](int i) { return bidx[i / bs] * bs + (i % bs); });
 }
 
-// A cluster of kTokCluster CTAs per row when scoring is light: every CTA
-// scores a contiguous quarter of the candidates into its own shared memory
-// and the cluster selects the top-k together over distributed shared memory
-// (cluster_topk.cuh).  When the scores are degenerate or too many of them
-// share the threshold bin, the leader CTA gathers all keys and selects alone.
-constexpr int kTokCluster = 4;
+// A cluster of CTAs per row when scoring is light: every CTA scores a
+// contiguous share of the candidates into its own shared memory and the
+// cluster selects the top-k together over distributed shared memory
+// (cluster_topk.cuh).  When the scores are degenerate (a wide run of equal
+// keys at the threshold), the leader CTA gathers all keys and selects alone.
 constexpr int kTokThreads = 256;
 
-template <int R>
-__global__ void __cluster_dims__(kTokCluster, 1, 1) __launch_bounds__(kTokThreads)
-    token_select_cluster_kernel(TokenParams p) {
+// NTILE > 0: scores on the tensor cores (score_candidates_tc, heads in
+// NTILE n-tiles of 8); 0: on the CUDA cores.  CL CTAs (the launch's cluster
+// size) share a row: 4 when there are enough rows to fill the GPU, up to 16
+// when a few long rows would leave it idle.
+template <int R, int NTILE, int CL>
+__global__ void __launch_bounds__(kTokThreads) token_select_cluster_kernel(TokenParams p) {
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ float sm[];
   const int rank = (int)cluster.block_rank();
   const int row = blockIdx.y;
-  const int per = (p.n_cand + kTokCluster - 1) / kTokCluster;
+  const int per = (p.n_cand + CL - 1) / CL;
   float* qlab = sm;                                                   // [G][R]
   int32_t* bidx = reinterpret_cast<int32_t*>(sm + p.group * R);       // [K_b]
   uint32_t* mine = reinterpret_cast<uint32_t*>(bidx + p.K_b);         // [per]
   uint32_t* all = mine + per;                                         // [n_cand] (leader, fallback)
   TopkScratch* ts = reinterpret_cast<TopkScratch*>(all + p.n_cand);
-  ClusterTopkScratch<kTokCluster>* cts = reinterpret_cast<ClusterTopkScratch<kTokCluster>*>(
-      (reinterpret_cast<uintptr_t>(ts + 1) + 15) & ~uintptr_t(15));
+  ClusterTopkScratch<CL>* cts =
+      reinterpret_cast<ClusterTopkScratch<CL>*>((reinterpret_cast<uintptr_t>(ts + 1) + 15) & ~uintptr_t(15));
   cluster_arrive_relaxed();  // completes once every CTA of the cluster has started
   grid_launch_dependents();
   load_qlab<R, kTokThreads>(p, row, qlab);
-  if (threadIdx.x == 0) prefetch_l2(p.token_idx + (int64_t)row * p.k + (int64_t)rank * p.k / kTokCluster);
+  if (threadIdx.x == 0) prefetch_l2(p.token_idx + (int64_t)row * p.k + (int64_t)rank * p.k / CL);
   grid_dependency_wait();  // the block lists come from the preceding kernel
   load_block_list<kTokThreads>(p, row, bidx);
   __syncthreads();
   const int c0 = min(p.n_cand, rank * per), c1 = min(p.n_cand, c0 + per);
-  score_candidates<R, kTokThreads>(p, row, qlab, bidx, c0, c1, mine);
+  if constexpr (NTILE > 0) score_candidates_tc<R, kTokThreads, NTILE>(p, row, qlab, bidx, c0, c1, mine);
+  else score_candidates<R, kTokThreads>(p, row, qlab, bidx, c0, c1, mine);
   __syncthreads();
   cluster_wait();
   int* out = p.token_idx + (int64_t)row * p.k;
   const CandidateToken map{bidx, p.bs};
-  if (cluster_topk_ascending<kTokThreads, kTokCluster>(mine, c1 - c0, c0, p.k, out, *cts, map)) return;
+  if (cluster_topk_ascending<kTokThreads, CL>(mine, c1 - c0, c0, p.k, out, *cts, map)) return;
   if (rank == 0) {
     // gather the other CTAs' keys through distributed shared memory, eight
     // independent loads in flight per thread
-    for (int r = 0; r < kTokCluster; ++r) {
+    for (int r = 0; r < CL; ++r) {
       const uint32_t* __restrict__ src = cluster.map_shared_rank(mine, r);
       const int b0 = min(p.n_cand, r * per), b1 = min(p.n_cand, b0 + per);
       for (int i0 = 0; i0 < b1 - b0; i0 += 8 * kTokThreads) {
@@ -189,30 +192,51 @@ tls_status select_tokens_impl(const tls_shape& s, const void* q, const int32_t* 
   p.token_idx = token_idx;
 
   const size_t smem = (size_t)p.group * s.n_label * 4 + (size_t)p.n_cand * 4 + sizeof(TopkScratch) + 16;
-  if (token_cluster_fits(p.group, s.n_label, p.n_cand)) {
-    const int per = (p.n_cand + kTokCluster - 1) / kTokCluster;
-    const size_t csmem = ((size_t)p.group * s.n_label + K_b + per + p.n_cand) * 4 + sizeof(TopkScratch) +
-                          sizeof(ClusterTopkScratch<kTokCluster>) + 32;
-    const dim3 cgrid(kTokCluster, (unsigned)rows);
+  // wide groups score on the tensor cores, which keeps any candidate count in one cluster
+  const bool tc = p.group >= 16 && p.group <= 128 && (s.n_label == 16 || s.n_label == 32);
+  if (tc || token_cluster_fits(p.group, s.n_label, p.n_cand)) {
+    const int cl = token_cluster_size(rows, p.n_cand, tc);
+    const int per = (p.n_cand + cl - 1) / cl;
+    const size_t cts_bytes = cl == 16 ? sizeof(ClusterTopkScratch<16>)
+                             : cl == 8 ? sizeof(ClusterTopkScratch<8>)
+                                       : sizeof(ClusterTopkScratch<4>);
+    const size_t csmem =
+        ((size_t)p.group * s.n_label + K_b + per + p.n_cand) * 4 + sizeof(TopkScratch) + cts_bytes + 32;
+    const int ntile = p.group <= 16 ? 2 : p.group <= 32 ? 4 : p.group <= 64 ? 8 : 16;
+    auto launch = [&](auto kernel) -> tls_status {
+      cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)csmem);
+      if (e == cudaSuccess && cl > 8)  // 16-CTA clusters are beyond the portable size
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e != cudaSuccess) return cuda_check(e, "select_tokens: set kernel attributes");
+      return cuda_check(launch_ex(kernel, dim3((unsigned)cl, (unsigned)rows), dim3(kTokThreads), csmem, stream, pdl,
+                                  (unsigned)cl, p),
+                        "select_tokens launch");
+    };
+    auto by_cl = [&](auto k4, auto k8, auto k16) -> tls_status {
+      return cl == 16 ? launch(k16) : cl == 8 ? launch(k8) : launch(k4);
+    };
+#define TLS_TC(RR, NN) \
+  by_cl(token_select_cluster_kernel<RR, NN, 4>, token_select_cluster_kernel<RR, NN, 8>, token_select_cluster_kernel<RR, NN, 16>)
+    if (tc) {
+      if (s.n_label == 16) {
+        if (ntile == 2) return TLS_TC(16, 2);
+        if (ntile == 4) return TLS_TC(16, 4);
+        if (ntile == 8) return TLS_TC(16, 8);
+        return TLS_TC(16, 16);
+      }
+      if (ntile == 2) return TLS_TC(32, 2);
+      if (ntile == 4) return TLS_TC(32, 4);
+      if (ntile == 8) return TLS_TC(32, 8);
+      return TLS_TC(32, 16);
+    }
+#undef TLS_TC
     switch (s.n_label) {
-#define TLS_TC_CASE(RR)                                                                                     \
-  case RR: {                                                                                                \
-    cudaError_t e = cudaFuncSetAttribute(token_select_cluster_kernel<RR>,                                   \
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)csmem);          \
-    if (e != cudaSuccess) return cuda_check(e, "select_tokens: set smem attribute");                        \
-    if (pdl)                                                                                                \
-      return cuda_check(launch_pdl(token_select_cluster_kernel<RR>, cgrid, dim3(kTokThreads), csmem, stream, p), \
-                        "select_tokens launch");                                                             \
-    token_select_cluster_kernel<RR><<<cgrid, kTokThreads, csmem, stream>>>(p);                              \
-    return launch_check("select_tokens launch");                                                             \
-  }
-      TLS_TC_CASE(2)
-      TLS_TC_CASE(4)
-      TLS_TC_CASE(8)
-      TLS_TC_CASE(16)
-      TLS_TC_CASE(32)
-      TLS_TC_CASE(64)
-#undef TLS_TC_CASE
+      case 2: return launch(token_select_cluster_kernel<2, 0, 4>);
+      case 4: return launch(token_select_cluster_kernel<4, 0, 4>);
+      case 8: return launch(token_select_cluster_kernel<8, 0, 4>);
+      case 16: return launch(token_select_cluster_kernel<16, 0, 4>);
+      case 32: return launch(token_select_cluster_kernel<32, 0, 4>);
+      case 64: return launch(token_select_cluster_kernel<64, 0, 4>);
       default:
         return fail(TLS_ERR_UNSUPPORTED, "select_tokens: n_label %d not built (2,4,8,16,32,64)", s.n_label);
     }
