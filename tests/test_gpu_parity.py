@@ -364,12 +364,14 @@ def _crowd_depth(scores, k, levels=3):
 
 
 # a few tokens with K rows 1e4 times the rest stretch the score range so far
-# that all other candidates share one value bin: the cluster selections (16
-# and 8 CTAs a row at level 2, several at level 1) must split that bin with
-# sub-bins instead of handing the row to one CTA
+# that all other candidates share one value bin: the selections (level 2 in
+# one CTA a row, or in clusters of 16 and 8 CTAs; level 1 over several CTAs)
+# must split that bin with sub-bins instead of falling back
 DENSE = [
-    small("s_dense_cl16", batch=1, n_q_heads=16, n_kv_heads=1, ctx_len=16384, block_size=64, K_b=128, k=4096,
+    small("s_dense_row_g16", batch=1, n_q_heads=16, n_kv_heads=1, ctx_len=16384, block_size=64, K_b=128, k=4096,
           seed=43),
+    small("s_dense_cl16_g32", batch=1, n_q_heads=32, n_kv_heads=1, ctx_len=16384, block_size=64, K_b=128,
+          k=4096, seed=45),
     small("s_dense_cl8_r32", batch=2, n_q_heads=64, n_kv_heads=2, ctx_len=8192, block_size=64, K_b=64, k=2000,
           n_label=32, seed=44),
 ]

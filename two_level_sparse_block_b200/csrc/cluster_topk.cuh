@@ -42,15 +42,6 @@
 
 namespace tls {
 
-constexpr int kTopkLevels = 3;
-
-// bin of a key at a sub-bin level: the bounds are rounded, so a key of the
-// parent bin may fall just outside [fmin, fmin + 256 / inv]; clamping keeps
-// the map monotone in the key, which is all the selection relies on
-__device__ __forceinline__ int topk_sub_bin(uint32_t key, float fmin, float inv) {
-  return max(0, min(255, (int)((key_float(key) - fmin) * inv)));
-}
-
 template <int CL>
 struct alignas(16) ClusterTopkScratch {
   // written by the cluster's CTAs (index = writer's rank)

@@ -105,6 +105,7 @@ struct TopkScratch {
   uint32_t lo, hi;
   uint32_t tau;  // threshold found by the pairwise ranking
   int take;      // keys equal to tau to take, found by the pairwise ranking
+  int tcount;    // keys in the threshold bin (cta_topk_regs)
   uint32_t cand[kTopkCand];
 };
 
@@ -115,6 +116,19 @@ __device__ __forceinline__ float key_float(uint32_t k) {
 // 256 value bins of a (finite) key over [fmin, fmin + 256 / inv]
 __device__ __forceinline__ int topk_value_bin(uint32_t key, float fmin, float inv) {
   return min(255, (int)((key_float(key) - fmin) * inv));
+}
+
+__device__ __forceinline__ uint32_t smem_addr32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+constexpr int kTopkLevels = 3;  // levels of 256 sub-bins before a selection gives up on value bins
+
+// bin of a key at a sub-bin level: the bounds are rounded, so a key of the
+// parent bin may fall just outside [fmin, fmin + 256 / inv]; clamping keeps
+// the map monotone in the key, which is all the selection relies on
+__device__ __forceinline__ int topk_sub_bin(uint32_t key, float fmin, float inv) {
+  return max(0, min(255, (int)((key_float(key) - fmin) * inv)));
 }
 
 template <int NT, typename MapFn>
@@ -392,6 +406,239 @@ __device__ void cta_topk_ascending(const uint32_t* keys, int n, int k, int* out,
       p_run += __popc(tb);
     }
   }
+}
+
+// Same selection as cta_topk_ascending for n <= KPT * NT keys, with every
+// thread holding KPT consecutive positions in registers: a handful of CTA
+// barriers, prefix counts by warp scans instead of shared counters, and
+// sub-bins (up to three levels of 256) instead of radix passes.
+//   0. key range (warp reductions, every thread folds the warp results)
+//   1. value-bin histogram of the keys still in the threshold cell; the bin
+//      of the need-th key narrows the cell; repeat while it holds > 128 keys
+//   2. the cell's keys compacted at scanned offsets
+//   3. pairwise ranking of those: tau and how many keys equal to it to take
+//   4. counts above / equal to tau scanned over the CTA, then each thread
+//      writes its own taken positions
+// Degenerate keys (all equal, not finite, or a wide run of equal keys at the
+// threshold) go to cta_topk_ascending.  `keys` is shared memory, 16-byte
+// aligned when KPT is a multiple of 4; its first k words are overwritten (the
+// output is staged there).
+template <int NT, int KPT, typename MapFn>
+__device__ void cta_topk_regs(const uint32_t* keys, int n, int k, int* out, TopkScratch& sm, MapFn map) {
+  static_assert(NT % 32 == 0 && NT >= kTopkRankMax && NT <= 1024 && KPT >= 1 && KPT <= 32, "shape");
+  constexpr int NW = NT / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int p0 = tid * KPT;
+  uint32_t kv[KPT];
+  uint32_t cell = 0u;  // bit j: key j is valid and still in the threshold cell
+  if constexpr (KPT % 4 == 0) {
+    if (p0 + KPT <= n) {
+#pragma unroll
+      for (int j = 0; j < KPT; j += 4) {
+        const uint4 v = *reinterpret_cast<const uint4*>(keys + p0 + j);
+        kv[j] = v.x;
+        kv[j + 1] = v.y;
+        kv[j + 2] = v.z;
+        kv[j + 3] = v.w;
+      }
+      cell = KPT == 32 ? 0xFFFFFFFFu : (1u << KPT) - 1u;
+    } else {
+#pragma unroll
+      for (int j = 0; j < KPT; ++j) {
+        kv[j] = p0 + j < n ? keys[p0 + j] : 0u;
+        if (p0 + j < n) cell |= 1u << j;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {
+      kv[j] = p0 + j < n ? keys[p0 + j] : 0u;
+      if (p0 + j < n) cell |= 1u << j;
+    }
+  }
+
+  // 0. key range
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    if ((cell >> j) & 1u) {
+      lo = min(lo, kv[j]);
+      hi = max(hi, kv[j]);
+    }
+  }
+  lo = __reduce_min_sync(0xffffffffu, lo);
+  hi = __reduce_max_sync(0xffffffffu, hi);
+  if (lane == 0) {
+    sm.wlo[warp] = lo;
+    sm.whi[warp] = hi;
+  }
+  for (int i = tid; i < 256; i += NT) sm.hist[i] = 0;
+  __syncthreads();
+  // every warp folds the warp results, one per lane
+  lo = __reduce_min_sync(0xffffffffu, lane < NW ? sm.wlo[lane] : 0xFFFFFFFFu);
+  hi = __reduce_max_sync(0xffffffffu, lane < NW ? sm.whi[lane] : 0u);
+  const float fmin = key_float(lo), fmax = key_float(hi);
+  const float span = fmax - fmin;
+  bool ok = lo != hi && isfinite(fmin) && isfinite(fmax) && isfinite(span) && span > 0.0f;  // uniform
+  float lmin = fmin, linv = ok ? 256.0f / span : 0.0f;
+  int need = k;
+
+  // 1. levels of value bins
+  for (int lv = 0; ok; ++lv) {
+#pragma unroll
+    for (int j = 0; j < KPT; ++j)
+      if ((cell >> j) & 1u) atomicAdd(&sm.hist[topk_sub_bin(kv[j], lmin, linv)], 1);
+    __syncthreads();
+    if (warp == 0) {
+      int local[8];
+      int s = 0;
+#pragma unroll
+      for (int d = 0; d < 8; ++d) {
+        local[d] = sm.hist[255 - (lane * 8 + d)];
+        s += local[d];
+      }
+      int incl = s;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int above = incl - s;
+      if (above < need && incl >= need) {
+        int d = 0;
+        for (; d < 8; ++d) {
+          if (above + local[d] >= need) break;
+          above += local[d];
+        }
+        sm.tbin = 255 - (lane * 8 + d);
+        sm.need = need - above;
+        sm.tcount = local[d];
+      }
+    }
+    __syncthreads();
+    const int tb = sm.tbin;
+    need = sm.need;
+#pragma unroll
+    for (int j = 0; j < KPT; ++j)
+      if (((cell >> j) & 1u) && topk_sub_bin(kv[j], lmin, linv) != tb) cell &= ~(1u << j);
+    if (sm.tcount <= kTopkRankMax) break;
+    // sub-bins of the threshold bin
+    lmin = lmin + (float)tb / linv;
+    linv = linv * 256.0f;
+    ok = lv + 1 < kTopkLevels && isfinite(lmin) && isfinite(linv);
+    // every thread has read the scan results; the histogram is free again
+    for (int i = tid; i < 256; i += NT) sm.hist[i] = 0;
+    __syncthreads();
+  }
+  if (!ok) {
+    __syncthreads();  // the scratch fields read above are rewritten by the fallback
+    cta_topk_ascending<NT>(keys, n, k, out, sm, map);
+    return;
+  }
+
+  // 2. compaction of the threshold cell at scanned offsets
+  {
+    const int c = __popc(cell);
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) sm.wgt[warp] = incl;
+    __syncthreads();
+    int off = incl - c + (int)__reduce_add_sync(0xffffffffu, lane < warp ? (unsigned)sm.wgt[lane] : 0u);
+#pragma unroll
+    for (int j = 0; j < KPT; ++j)
+      if ((cell >> j) & 1u) sm.cand[off++] = kv[j];
+    __syncthreads();
+  }
+
+  // 3. pairwise ranking inside the cell: TPC adjacent threads per key, thread
+  // `part` comparing the 16-byte chunks part, part + TPC, ... (the TPC lanes
+  // of a key read adjacent chunks: no bank conflicts)
+  {
+    constexpr int TPC = NT / kTopkRankMax;  // 1, 2, 4 or 8
+    constexpr int NCH = kTopkRankMax / 4 / TPC;  // chunks per thread
+    const int nc = sm.tcount;
+    const int c = tid / TPC, part = tid % TPC;
+    if (c < nc) {
+      const uint32_t mine = sm.cand[c];
+      int gt = 0, eq = 0;
+      const bool vec = (smem_addr32(sm.cand) & 15u) == 0u;  // (the scratch may sit anywhere 4-byte aligned)
+#pragma unroll
+      for (int q = 0; q < NCH; ++q) {
+        const int i0 = 4 * (q * TPC + part);
+        uint32_t o[4];
+        if (vec) {
+          const uint4 v = *reinterpret_cast<const uint4*>(sm.cand + i0);
+          o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+        } else {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) o[u] = sm.cand[i0 + u];
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const bool in = i0 + u < nc;
+          gt += (int)(in && o[u] > mine);
+          eq += (int)(in && o[u] == mine);
+        }
+      }
+      // the TPC lanes of a key are adjacent and all inside the c < nc branch
+      const unsigned grp = TPC == 32 ? 0xffffffffu : (((1u << TPC) - 1u) << (lane & ~(TPC - 1)));
+#pragma unroll
+      for (int o = 1; o < TPC; o <<= 1) {
+        gt += __shfl_xor_sync(grp, gt, o);
+        eq += __shfl_xor_sync(grp, eq, o);
+      }
+      if (part == 0 && gt < need && need <= gt + eq) {
+        sm.tau = mine;  // every thread that holds tau writes the same values
+        sm.take = need - gt;
+      }
+    }
+  }
+  __syncthreads();
+  const uint32_t tau = sm.tau;
+  const int take_eq = sm.take;
+
+  // 4. counts above / equal to tau before this thread, then the stores
+  int gt = 0, eq = 0;
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    const bool valid = p0 + j < n;
+    gt += (int)(valid && kv[j] > tau);
+    eq += (int)(valid && kv[j] == tau);
+  }
+  const int v = gt | (eq << 16);  // n <= 32768: neither half overflows
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) sm.weq[warp] = incl;
+  __syncthreads();
+  const int pre = incl - v + (int)__reduce_add_sync(0xffffffffu, lane < warp ? (unsigned)sm.weq[lane] : 0u);
+  int e_run = pre >> 16;
+  int slot = (pre & 0xFFFF) + min(e_run, take_eq);
+  // taken positions staged in shared memory (over the keys, which every
+  // thread holds in registers by now), then written out coalesced
+  int* stage = reinterpret_cast<int*>(const_cast<uint32_t*>(keys));
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    if (p0 + j >= n) continue;
+    bool take = kv[j] > tau;
+    if (kv[j] == tau) {
+      take = e_run < take_eq;
+      ++e_run;
+    }
+    if (take) {
+      if (slot < k) stage[slot] = p0 + j;
+      ++slot;
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < k; i += NT) out[i] = map(stage[i]);
 }
 
 // ----------------------------------------------------------------------------

@@ -44,10 +44,13 @@ __device__ __forceinline__ void load_codes(const uint8_t* p, float (&c)[R]) {
       w[4 * i + 3] = v.w;
     }
   }
+  // sign-extend the 4-bit two's complement codes without integer-to-float
+  // conversions: with v = nibble ^ 8, the float bit pattern 0x4B000000 | v is
+  // 2^23 + v, and subtracting 2^23 + 8 leaves v - 8 exactly
 #pragma unroll
   for (int r = 0; r < R; ++r) {
-    const int nib = (int)((w[r / 8] >> (4 * (r % 8))) & 15u);
-    c[r] = (float)((nib ^ 8) - 8);  // sign-extend the 4-bit two's complement code
+    const uint32_t v = ((w[r / 8] >> (4 * (r % 8))) & 15u) ^ 8u;
+    c[r] = __uint_as_float(0x4B000000u | v) - 8388616.0f;
   }
 }
 
@@ -129,6 +132,32 @@ __device__ __forceinline__ void score_candidates(const TokenParams& p, int row, 
   }
 }
 
+// Codes and scales of every candidate of a row copied to shared memory in
+// candidate order (block by block, 16-byte asynchronous copies, all in flight
+// at once), so that scoring waits on one round trip to memory instead of one
+// per batch of candidates.  Needs bs * R / 2 and bs * 4 to be multiples of 16
+// and 16-byte aligned codes and scales (token_row_kernel_fits).
+// Blocks [j0, j1) of the row's list are staged; candidate j0 * bs lands at
+// index 0.
+template <int R, int NT>
+__device__ __forceinline__ void stage_candidate_codes(const TokenParams& p, int row, const int32_t* bidx, int j0,
+                                                      int j1, uint8_t* scodes, float* sscales) {
+  const int cpb = p.bs * (R / 2) / 16;  // 16-byte chunks of codes per block
+  const int per = cpb + p.bs * 4 / 16;  // ... and of scales
+  const uint32_t sc0 = smem_addr32(scodes), ss0 = smem_addr32(sscales);
+  for (int i = threadIdx.x; i < (j1 - j0) * per; i += NT) {
+    const int j = i / per, c = i - j * per;
+    const int64_t tok0 = (int64_t)row * p.ctx_len + (int64_t)bidx[j0 + j] * p.bs;
+    if (c < cpb)
+      cp_async16(sc0 + (uint32_t)(j * p.bs * (R / 2) + c * 16), p.codes + tok0 * (R / 2) + c * 16, 16u);
+    else
+      cp_async16(ss0 + (uint32_t)(j * p.bs * 4 + (c - cpb) * 16),
+                 reinterpret_cast<const uint8_t*>(p.scales + tok0) + (c - cpb) * 16, 16u);
+  }
+  cp_async_commit();
+  cp_async_wait<0>();
+}
+
 // Token scores on the tensor cores for wide groups (G >= 16, R = 16 or 32):
 // per warp step 16 candidates, S[cand, head] = code[cand, :] . qlab[head, :]
 // as m16n8k16 bf16 MMAs with fp32 accumulation (M = 16 candidates, N = 8
@@ -141,10 +170,16 @@ __device__ __forceinline__ uint32_t tok_pack_bf16(float lo, float hi) {
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
-// the two INT4 codes of one byte (low nibble = even channel) as bf16x2
+// the two INT4 codes of one byte (low nibble = even channel) as bf16x2,
+// without integer-to-float conversions: with v = nibble ^ 8, the bf16 bit
+// pattern 0x4300 | v is 128 + v (v < 128 fits the 7 mantissa bits at
+// exponent 7), and subtracting 136 (bf16 0x4308) leaves v - 8, the two's
+// complement code, exactly
 __device__ __forceinline__ uint32_t tok_codes_bf16x2(uint32_t byte) {
-  const int lo = (int)((byte & 0xFu) ^ 8u) - 8, hi = (int)(((byte >> 4) & 0xFu) ^ 8u) - 8;
-  return tok_pack_bf16((float)lo, (float)hi);
+  const uint32_t t = ((byte & 0xFu) | ((byte & 0xF0u) << 12)) ^ 0x43084308u;
+  uint32_t r;
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(t), "r"(0x43084308u));
+  return r;
 }
 __device__ __forceinline__ void tok_mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -154,9 +189,14 @@ __device__ __forceinline__ void tok_mma(float (&d)[4], const uint32_t (&a)[4], u
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-template <int R, int NT, int NTILE>
+// STAGED: the codes and scales of candidates [c0, c1) were copied, in
+// candidate order from index 0, to shared memory (scodes, sscales) by
+// stage_candidate_codes.
+template <int R, int NT, int NTILE, bool STAGED = false>
 __device__ __forceinline__ void score_candidates_tc(const TokenParams& p, int row, const float* qlab,
-                                                    const int32_t* bidx, int c0, int c1, uint32_t* keys) {
+                                                    const int32_t* bidx, int c0, int c1, uint32_t* keys,
+                                                    const uint8_t* scodes = nullptr,
+                                                    const float* sscales = nullptr) {
   static_assert(R == 16 || R == 32, "label channels for the tensor-core scorer");
   constexpr int KS = R / 16, NW = NT / 32;
   const int g = p.group;
@@ -175,8 +215,9 @@ __device__ __forceinline__ void score_candidates_tc(const TokenParams& p, int ro
   }
   const CandidateToken map{bidx, p.bs};
   // U steps of 16 candidates per warp iteration: all their code and scale
-  // loads are in flight before the first MMA
-  constexpr int U = 4;
+  // loads are in flight before the first MMA (fewer in 1024-thread CTAs,
+  // which have 64 registers a thread)
+  constexpr int U = STAGED ? 2 : NT >= 1024 ? 2 : 4;
   for (int base0 = c0 + warp * 16; base0 < c1; base0 += NW * 16 * U) {
     uint32_t w[U][2][KS * 2];  // code words of fragment rows gq, gq + 8
     float sc[U][2];
@@ -188,19 +229,21 @@ __device__ __forceinline__ void score_candidates_tc(const TokenParams& p, int ro
       for (int hlf = 0; hlf < 2; ++hlf) {
         const int i = base + gq + 8 * hlf;
         ok[u][hlf] = i < c1;
-        const int64_t at = (int64_t)row * p.ctx_len + (ok[u][hlf] ? map(i) : 0);
+        const int64_t at = STAGED ? (ok[u][hlf] ? i - c0 : 0) : (int64_t)row * p.ctx_len + (ok[u][hlf] ? map(i) : 0);
+        const uint8_t* cb = STAGED ? scodes : p.codes;
+        const float* sb = STAGED ? sscales : p.scales;
         if constexpr (R == 16) {
-          const uint2 c = ok[u][hlf] ? *reinterpret_cast<const uint2*>(p.codes + at * 8) : make_uint2(0u, 0u);
+          const uint2 c = ok[u][hlf] ? *reinterpret_cast<const uint2*>(cb + at * 8) : make_uint2(0u, 0u);
           w[u][hlf][0] = c.x;
           w[u][hlf][1] = c.y;
         } else {
-          const uint4 c = ok[u][hlf] ? *reinterpret_cast<const uint4*>(p.codes + at * 16) : make_uint4(0u, 0u, 0u, 0u);
+          const uint4 c = ok[u][hlf] ? *reinterpret_cast<const uint4*>(cb + at * 16) : make_uint4(0u, 0u, 0u, 0u);
           w[u][hlf][0] = c.x;
           w[u][hlf][1] = c.y;
           w[u][hlf][2] = c.z;
           w[u][hlf][3] = c.w;
         }
-        sc[u][hlf] = ok[u][hlf] ? p.scales[at] : 0.0f;
+        sc[u][hlf] = ok[u][hlf] ? sb[at] : 0.0f;
       }
     }
 #pragma unroll
@@ -250,6 +293,24 @@ __device__ __forceinline__ void score_candidates_tc(const TokenParams& p, int ro
       }
     }
   }
+}
+
+// Whether level 2 runs as the row-cluster kernel: tensor-core scoring of a
+// narrow group (G <= 16, 16 or 32 label channels) over at most 8192
+// candidates, kept in registers by the leader's top-k, with the candidates'
+// codes and scales staged in shared memory by 16-byte copies (block size a
+// multiple of 4; the caller also checks 16-byte aligned codes and scales).
+__host__ __device__ inline bool token_row_kernel_fits(int group, int n_label, int n_cand, int bs) {
+  return group <= 16 && (n_label == 16 || n_label == 32) && n_cand <= 8192 && bs % 4 == 0;
+}
+
+// CTAs per row of the row-cluster kernel: 4, 2 or 1, as many as keep every
+// CTA at 8 blocks or more and the grid within two CTAs per SM.
+__host__ __device__ inline int token_row_cluster_size(int rows, int K_b, int bs) {
+  int cl = 4;
+  while (cl > 1 && ((int64_t)rows * cl > 2 * 148 || K_b < 8 * cl)) cl /= 2;
+  (void)bs;
+  return cl;
 }
 
 // CTAs per row of the cluster kernel: 4, or (tensor-core scoring only) 8 / 16
