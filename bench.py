@@ -49,6 +49,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-offload", action="store_true", help="skip the offload-engine measurement (c4)")
     ap.add_argument("--no-other-configs", action="store_true", help="skip the c1 / c3 step measurements")
+    ap.add_argument("--no-staggered", action="store_true", help="skip the staggered-schedule measurement")
     ap.add_argument("--e2e-steps", type=int, default=300)
     return ap.parse_args()
 
@@ -264,6 +265,50 @@ def measure_config(name, dev, steps=200, warmup=10):
             "l2": "flushed before every step (write + read of 256 MB)"}
 
 
+def measure_staggered(st, dev, flush_l2, steps, warmup=6):
+    """The staggered schedule over the same HBM-resident layer (ResidentEngine):
+    step t runs level 2 and the attention within M_{t-1} while level 1 chooses
+    M_t on a second stream, joined at the end of the step.  Two graphs (the two
+    parities of the block lists) replayed alternately, L2 flushed before every
+    step as for the headline, CUDA events around each replay."""
+    import torch
+    from two_level_sparse_block_b200 import runtime
+    eng = runtime.ResidentEngine(st)
+    cap = torch.cuda.Stream(dev)
+    graphs = []
+    with torch.cuda.stream(cap):
+        eng.step(stream=cap)  # step 0, with the prologue (M_{-1})
+        for _ in range(2):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap):
+                eng.step(stream=cap)
+            graphs.append(g)
+    stream = torch.cuda.current_stream(dev)
+    stream.wait_stream(cap)
+    torch.cuda.synchronize(dev)
+    evs = []
+    for i in range(warmup + steps):
+        flush_l2(i)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        graphs[i & 1].replay()
+        b.record(stream)
+        if i >= warmup:
+            evs.append((a, b))
+    torch.cuda.synchronize(dev)
+    err = eng.check_device_error()
+    del graphs
+    eng.close()
+    if err != 0:
+        raise RuntimeError(f"device error {err} in the staggered engine")
+    ts = [a.elapsed_time(b) for a, b in evs]
+    ms = statistics.mean(ts)
+    return {"us_per_step": ms * 1e3, "us_per_step_median": statistics.median(ts) * 1e3,
+            "decode_tokens_per_s": st.shape.batch / (ms / 1e3), "steps": steps,
+            "schedule": "step t: level 2 + attention within M_{t-1} on the caller's stream, level 1 for q_t "
+                        "on a second stream; one graph per step parity, L2 flushed before every step"}
+
+
 def measure_offload_engine(dev, steps=64):
     """The offload workload (c4): the staggered engine over an HBM block cache of
     256 slots, K/V in pinned host memory, `steps` consecutive decode steps along
@@ -457,6 +502,7 @@ def main():
     step_ms = [e[0].elapsed_time(e[1]) for e in evs]
     # stage breakdown (separate graphs, so each stage also pays its own launch)
     sel_ms, att_ms = stage_times(min(args.steps, 500))
+    staggered = measure_staggered(st, dev, flush_l2, min(args.steps, 500)) if not args.no_staggered else None
     total_ms = sum(step_ms)
     t = torch.tensor([total_ms, statistics.mean(att_ms)], dtype=torch.float64, device=dev)
     if world > 1:
@@ -506,6 +552,7 @@ def main():
                      "note": "tls_select and tls_sparse_decode_attn replayed as separate graphs (each pays its own "
                              "launch, the attention reads K and V from HBM); the step is one tls_decode_step graph"},
         "step_hbm": {"algorithmic_bytes": ab["step"], "achieved_gbs": step_gbs, "frac_of_peak": step_gbs / peak},
+        "staggered_engine": staggered,
         "roofline": {"kernel": attn_kernel, "bound": "hbm", "achieved": achieved,
                      "peak": peak, "peak_source": f"hbm_gbs {peak_kind}", "unit": "GB/s", "frac": achieved / peak,
                      "algorithmic_bytes_per_launch": ab["attn"],

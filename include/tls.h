@@ -346,6 +346,19 @@ TLS_API tls_status tls_engine_create(const tls_shape* shape, int32_t K_b, int32_
                              size_t ws_bytes, tls_engine** out);
 
 /*
+ * Creates an engine whose K/V are resident in HBM (`kv`, a dense view as in
+ * tls_sparse_decode_attn; no block cache, no transfers): the staggered
+ * schedule alone.  Other arguments and ownership as tls_engine_create; the
+ * engine allocates one stream and its events.  Its steps never wait on the
+ * host, so a step may be captured into a CUDA graph on its stream (each step
+ * forks level 1 onto the engine's stream and joins it back before returning).
+ */
+TLS_API tls_status tls_engine_create_resident(const tls_shape* shape, int32_t K_b, int32_t k, const void* meta,
+                                      const int32_t* label_ch, const uint8_t* codes, const float* scales,
+                                      const tls_kv_view* kv, int32_t* block_idx, int32_t* token_idx, void* ws,
+                                      size_t ws_bytes, tls_engine** out);
+
+/*
  * One decode step t with query q (device bf16 [B, Hq, Dqk], ready on
  * `stream`).  Output as tls_sparse_decode_attn, written on `stream`.  Level 2
  * and the attention use the blocks chosen at step t-1 (M_{t-1}, resident in
@@ -354,7 +367,11 @@ TLS_API tls_status tls_engine_create(const tls_shape* shape, int32_t K_b, int32_
  * engine's copy stream while the attention runs; step t+1's attention waits
  * for them.  The first step selects M_{-1} from its own q and makes it
  * resident before attending.  The call waits on the host for level 1 of step
- * t (to plan the transfer); everything else is asynchronous.  After a failed
+ * t (to plan the transfer); everything else is asynchronous.  A resident
+ * engine (tls_engine_create_resident) has no transfer and no host wait: on
+ * `stream` it records q_t, runs level 2 over M_{t-1} and the attention, and
+ * waits for level 1 of step t (engine stream, after q_t) before returning, so
+ * the next step's level 2 finds M_t complete.  After a failed
  * step (a copy failure, TLS_ERR_CAPACITY, a launch error) the cache no longer
  * matches the block lists: every later step returns the same error and the
  * engine must be destroyed.
@@ -367,7 +384,8 @@ TLS_API int64_t tls_engine_steps(const tls_engine* engine);
 
 /*
  * Transfer figures of step `step` (-1 .. steps-1, among the last 255 steps);
- * waits for the events they need.
+ * waits for the events they need.  A resident engine reports no transfer
+ * (zero blocks, bytes and times).
  */
 TLS_API tls_status tls_engine_stats(tls_engine* engine, int64_t step, tls_engine_step_stats* out);
 

@@ -193,3 +193,90 @@ def test_engine_on_the_offload_workload_sampled_steps():
         assert all(0 <= layer.stats(t).n_copied <= cfg.K_b for t in range(len(qs) - 1))
     finally:
         layer.close()
+
+
+# ---------------------------------------------------------------------------
+# resident engine: the same stagger over HBM-resident K/V, no transfers
+# ---------------------------------------------------------------------------
+
+def _resident(cfg, qs):
+    runtime, tls = _rt()
+    K, V, _ = synth.gen_kv(cfg, qs[0])
+    lab = synth.gen_label_channels(cfg)
+    st = runtime.state_for_config(cfg, qs[0], K, V, lab)
+    return runtime, st, (K, V, lab)
+
+
+@pytest.mark.parametrize("cfg", ENGINE, ids=lambda c: c.name)
+def test_resident_engine_follows_the_staggered_oracle(cfg):
+    qs = synth.gen_query_trajectory(cfg)
+    runtime, st, (K, V, lab) = _resident(cfg, qs)
+    eng = runtime.ResidentEngine(st)
+    g = cfg.group
+    try:
+        for t, q in enumerate(qs):
+            eng.step(_dev_q(q))
+            torch.cuda.synchronize()
+            assert eng.check_device_error() == 0
+            m_prev = eng.block_idx[(t + 1) & 1].cpu().numpy()
+            m_cur = eng.block_idx[t & 1].cpu().numpy()
+            tok = eng.token_idx.cpu().numpy()
+            out = eng.out.float().cpu().numpy()
+            for b, h in _rows(cfg):
+                where = f"{cfg.name} resident step {t} row ({b},{h})"
+                r1 = _orow(cfg, q, K, V, lab, b, h)
+                check_selection(m_cur[b, h], r1["agg"], cfg.K_b, where + " M_t")
+                if t == 0:
+                    check_selection(m_prev[b, h], r1["agg"], cfg.K_b, where + " M_-1")
+                r2 = _orow(cfg, q, K, V, lab, b, h, block_idx=m_prev[b, h])
+                pos = np.searchsorted(r2["cand"], tok[b, h])
+                assert np.array_equal(r2["cand"][pos], tok[b, h]), f"{where}: token outside M_t-1"
+                check_selection(pos, r2["token_score"], cfg.k, where + " tokens")
+                r3 = _orow(cfg, q, K, V, lab, b, h, block_idx=m_prev[b, h], token_idx=tok[b, h])
+                check_output(out[b, h * g:(h + 1) * g], r3["out"], where + " out")
+        assert eng.steps_taken() == len(qs)
+        st0 = runtime.tls.tls_engine_stats(eng.engine, 0)
+        assert st0.n_copied == 0 and st0.bytes_copied == 0
+    finally:
+        eng.close()
+
+
+def test_resident_engine_steps_replay_from_graphs():
+    # steps 1 and 2 captured into two graphs (the two parities of the block
+    # lists), then replayed alternately: every step equals the eager engine's,
+    # bit for bit
+    cfg = ENGINE[2]
+    qs = synth.gen_query_trajectory(cfg, 6)
+    runtime, st, _ = _resident(cfg, qs)
+    eager = runtime.ResidentEngine(st)
+    want = []
+    for q in qs:
+        eager.step(_dev_q(q))
+        torch.cuda.synchronize()
+        want.append((eager.token_idx.clone(), eager.out.clone(), eager.lse.clone()))
+    eager.close()
+
+    eng = runtime.ResidentEngine(st)
+    s = torch.cuda.Stream()
+    qbuf = _dev_q(qs[0]).clone()
+    graphs = []
+    try:
+        with torch.cuda.stream(s):
+            eng.step(qbuf, stream=s)  # step 0 (with the prologue) eagerly
+            s.synchronize()
+            assert torch.equal(eng.token_idx, want[0][0]) and torch.equal(eng.out, want[0][1])
+            for _ in range(2):
+                gr = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gr, stream=s):
+                    eng.step(qbuf, stream=s)
+                graphs.append(gr)
+            for t in range(1, len(qs)):
+                qbuf.copy_(_dev_q(qs[t]))
+                graphs[(t - 1) & 1].replay()
+                s.synchronize()
+                assert torch.equal(eng.token_idx, want[t][0]), f"step {t}: token lists differ"
+                assert torch.equal(eng.out, want[t][1]) and torch.equal(eng.lse, want[t][2]), f"step {t}: output"
+        assert eng.check_device_error() == 0
+    finally:
+        del graphs
+        eng.close()

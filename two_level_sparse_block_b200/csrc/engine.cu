@@ -16,6 +16,13 @@
 //      block copies; slot-table update; event copy_end_t
 // The table update changes only entries of copied and evicted blocks, none of
 // which step t's attention reads, so C may run alongside it.
+//
+// A resident engine (K/V in HBM, no cache) keeps only the stagger, with no
+// host wait: A: event q_t; B: wait q_t, level 1 -> M_t, event sel_t; A: level 2
+// over M_{t-1}, attention, wait sel_t.  Level 1 of step t overwrites the list
+// level 2 read at step t-1, which A finished before recording q_t; level 2 of
+// step t+1 reads M_t, which the join at the end of step t completes.  Every
+// step forks and joins within itself, so it can be captured into a graph.
 
 #include <vector>
 
@@ -48,7 +55,7 @@ struct tls_engine {
   const int32_t* label_ch = nullptr;
   const uint8_t* codes = nullptr;
   const float* scales = nullptr;
-  tls_block_cache* cache = nullptr;
+  tls_block_cache* cache = nullptr;  // null: resident K/V (kv is a dense view)
   tls_kv_view kv;
   uint8_t* ws = nullptr;
   tls::WsLayout L;
@@ -85,15 +92,16 @@ void release(tls_engine* e) {
 
 }  // namespace
 
-extern "C" tls_status tls_engine_create(const tls_shape* shape, int32_t K_b, int32_t k, const void* meta,
-                                        const int32_t* label_ch, const uint8_t* codes, const float* scales,
-                                        tls_block_cache* cache, int32_t* block_idx, int32_t* token_idx, void* ws,
-                                        size_t ws_bytes, tls_engine** out) {
+namespace {
+
+tls_status engine_create(const tls_shape* shape, int32_t K_b, int32_t k, const void* meta, const int32_t* label_ch,
+                         const uint8_t* codes, const float* scales, tls_block_cache* cache, const tls_kv_view* dense,
+                         int32_t* block_idx, int32_t* token_idx, void* ws, size_t ws_bytes, tls_engine** out) {
   clear_error();
   tls_status st = check_shape(shape);
   if (st != TLS_OK) return st;
   if (out == nullptr || meta == nullptr || label_ch == nullptr || codes == nullptr || scales == nullptr ||
-      cache == nullptr || block_idx == nullptr || token_idx == nullptr)
+      (cache == nullptr && dense == nullptr) || block_idx == nullptr || token_idx == nullptr)
     return fail(TLS_ERR_INVALID_ARG, "engine_create: NULL argument");
   if (!aligned16(meta) || !aligned16(codes)) return fail(TLS_ERR_INVALID_ARG, "engine_create: meta/codes not 16-byte aligned");
   WsLayout L;
@@ -102,8 +110,14 @@ extern "C" tls_status tls_engine_create(const tls_shape* shape, int32_t K_b, int
   if (ws == nullptr || !aligned16(ws)) return fail(TLS_ERR_INVALID_ARG, "engine_create: workspace NULL or not 16-byte aligned");
   if (ws_bytes < L.total) return fail(TLS_ERR_INVALID_ARG, "engine_create: workspace %zu bytes < required %zu", ws_bytes, L.total);
   tls_kv_view kv;
-  st = block_cache_view(cache, &kv);
-  if (st != TLS_OK) return st;
+  if (cache != nullptr) {
+    st = block_cache_view(cache, &kv);
+    if (st != TLS_OK) return st;
+  } else {
+    kv = *dense;
+    if (kv.k == nullptr || kv.slot_of_block != nullptr || !aligned16(kv.k) || (kv.v != nullptr && !aligned16(kv.v)))
+      return fail(TLS_ERR_INVALID_ARG, "engine_create_resident: kv must be a dense view with 16-byte aligned K/V");
+  }
 
   auto* e = new tls_engine();
   e->shape = *shape;
@@ -122,17 +136,17 @@ extern "C" tls_status tls_engine_create(const tls_shape* shape, int32_t K_b, int
   e->bidx[1] = block_idx + (size_t)e->rows * K_b;
   e->token_idx = token_idx;
   cudaError_t ce = cudaSuccess;
-  for (int i = 0; i < 2 && ce == cudaSuccess; ++i)
+  for (int i = 0; i < 2 && ce == cudaSuccess && cache != nullptr; ++i)
     ce = cudaHostAlloc((void**)&e->host_bidx[i], (size_t)e->rows * K_b * sizeof(int32_t), cudaHostAllocDefault);
   // the select and copy streams get the highest priority: their small grids
   // are on the critical path of the next step, the attention is not
   int least = 0, greatest = 0;
   if (ce == cudaSuccess) ce = cudaDeviceGetStreamPriorityRange(&least, &greatest);
   if (ce == cudaSuccess) ce = cudaStreamCreateWithPriority(&e->sel, cudaStreamNonBlocking, greatest);
-  if (ce == cudaSuccess) ce = cudaStreamCreateWithPriority(&e->copy, cudaStreamNonBlocking, greatest);
+  if (ce == cudaSuccess && cache != nullptr) ce = cudaStreamCreateWithPriority(&e->copy, cudaStreamNonBlocking, greatest);
   for (cudaEvent_t* ev : {&e->ev_q, &e->ev_sel, &e->ev_attn[0], &e->ev_attn[1]})
     if (ce == cudaSuccess) ce = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
-  for (int i = 0; i < kRing && ce == cudaSuccess; ++i) {
+  for (int i = 0; i < kRing && ce == cudaSuccess && cache != nullptr; ++i) {
     ce = cudaEventCreate(&e->ready[i]);
     if (ce == cudaSuccess) ce = cudaEventCreate(&e->copy_start[i]);
     if (ce == cudaSuccess) ce = cudaEventCreate(&e->copy_end[i]);
@@ -145,13 +159,72 @@ extern "C" tls_status tls_engine_create(const tls_shape* shape, int32_t K_b, int
   return TLS_OK;
 }
 
+}  // namespace
+
+extern "C" tls_status tls_engine_create(const tls_shape* shape, int32_t K_b, int32_t k, const void* meta,
+                                        const int32_t* label_ch, const uint8_t* codes, const float* scales,
+                                        tls_block_cache* cache, int32_t* block_idx, int32_t* token_idx, void* ws,
+                                        size_t ws_bytes, tls_engine** out) {
+  if (cache == nullptr) {
+    clear_error();
+    return fail(TLS_ERR_INVALID_ARG, "engine_create: NULL cache (resident K/V: tls_engine_create_resident)");
+  }
+  return engine_create(shape, K_b, k, meta, label_ch, codes, scales, cache, nullptr, block_idx, token_idx, ws,
+                       ws_bytes, out);
+}
+
+extern "C" tls_status tls_engine_create_resident(const tls_shape* shape, int32_t K_b, int32_t k, const void* meta,
+                                                 const int32_t* label_ch, const uint8_t* codes, const float* scales,
+                                                 const tls_kv_view* kv, int32_t* block_idx, int32_t* token_idx,
+                                                 void* ws, size_t ws_bytes, tls_engine** out) {
+  if (kv == nullptr) {
+    clear_error();
+    return fail(TLS_ERR_INVALID_ARG, "engine_create_resident: NULL kv");
+  }
+  return engine_create(shape, K_b, k, meta, label_ch, codes, scales, nullptr, kv, block_idx, token_idx, ws, ws_bytes,
+                       out);
+}
+
 extern "C" void tls_engine_destroy(tls_engine* e) {
   if (e != nullptr) release(e);
 }
 
 namespace {
 
+tls_status resident_step(tls_engine* e, const void* q, int32_t out_dtype, void* out, float* lse, cudaStream_t A) {
+  const tls_shape& s = e->shape;
+  const int cur = (int)(e->t & 1), prev = cur ^ 1;
+  tls_status st;
+  // prologue: M_{-1} from q_0
+  if (e->t == 0) {
+    st = select_blocks_impl(s, q, e->meta, e->K_b, e->bidx[prev], nullptr, e->ws, e->L, A);
+    if (st != TLS_OK) return st;
+  }
+  // fork: level 1 for q_t on the select stream, after everything A has issued
+  cudaError_t ce = cudaEventRecord(e->ev_q, A);
+  if (ce == cudaSuccess) ce = cudaStreamWaitEvent(e->sel, e->ev_q, 0);
+  if (ce != cudaSuccess) return cuda_check(ce, "engine_step: select stream");
+  st = select_blocks_impl(s, q, e->meta, e->K_b, e->bidx[cur], nullptr, e->ws, e->L, e->sel);
+  if (st != TLS_OK) return st;
+  ce = cudaEventRecord(e->ev_sel, e->sel);
+  if (ce != cudaSuccess) return cuda_check(ce, "engine_step: select stream");
+  // level 2 within M_{t-1} and the attention, on A
+  st = select_tokens_impl(s, q, e->label_ch, e->codes, e->scales, e->bidx[prev], e->K_b, e->k, e->token_idx, nullptr,
+                          e->ws, e->L, A, /*pdl=*/false);
+  if (st != TLS_OK) return st;
+  // programmatic launch after level 2, as in the synchronous step (a plain
+  // launch measured slower: level 1 still competes with level 2 for the SMs)
+  st = sparse_attn_impl(s, q, e->kv, e->token_idx, e->k, out_dtype, out, lse, e->ws, e->L, A, /*pdl=*/true);
+  if (st != TLS_OK) return st;
+  // join: M_t is complete before anything A issues next
+  ce = cudaStreamWaitEvent(A, e->ev_sel, 0);
+  if (ce != cudaSuccess) return cuda_check(ce, "engine_step: join");
+  e->t += 1;
+  return TLS_OK;
+}
+
 tls_status engine_step(tls_engine* e, const void* q, int32_t out_dtype, void* out, float* lse, cudaStream_t A) {
+  if (e->cache == nullptr) return resident_step(e, q, out_dtype, out, lse, A);
   const tls_shape& s = e->shape;
   const size_t list_bytes = (size_t)e->rows * e->K_b * sizeof(int32_t);
   const int cur = (int)(e->t & 1), prev = cur ^ 1;
@@ -230,6 +303,14 @@ extern "C" tls_status tls_engine_stats(tls_engine* e, int64_t step, tls_engine_s
   if (step < -1 || step >= e->t || step < e->t - (kRing - 1))
     return fail(TLS_ERR_INVALID_ARG, "engine_stats: step %lld not among the last %d steps taken",
                 (long long)step, kRing - 1);
+  if (e->cache == nullptr) {  // resident K/V: nothing is transferred
+    out->step = step;
+    out->n_copied = 0;
+    out->bytes_copied = 0;
+    out->copy_ms = 0.0f;
+    out->exposed_ms = step + 1 < e->t ? 0.0f : -1.0f;
+    return TLS_OK;
+  }
   const int si = (int)((step + kRing) % kRing);
   cudaError_t ce = cudaEventSynchronize(e->copy_end[si]);
   float copy_ms = 0.0f, exposed_ms = -1.0f;

@@ -102,6 +102,55 @@ class DecodeState:
         return tls.tls_workspace_error(self.ws, True, stream)
 
 
+class ResidentEngine:
+    """The staggered schedule over a DecodeState's HBM-resident K/V and index
+    (tls_engine_create_resident): step t selects tokens and attends within
+    the blocks chosen at step t-1 while level 1 chooses M_t on a second
+    stream.  Its own block lists (two), token list, output and workspace; the
+    state's buffers are left alone.  A step never waits on the host and may be
+    captured into a CUDA graph."""
+
+    def __init__(self, st: DecodeState):
+        self.st = st
+        dev = st.device
+        s = st.shape
+        self.K_b, self.k = st.K_b, st.k
+        self.block_idx = torch.empty((2, s.batch, s.n_kv_heads, self.K_b), dtype=torch.int32, device=dev)
+        self.token_idx = torch.empty((s.batch, s.n_kv_heads, self.k), dtype=torch.int32, device=dev)
+        self.out = torch.empty_like(st.out)
+        self.lse = torch.empty_like(st.lse)
+        self.out_dtype = st.out_dtype
+        self.ws_bytes = tls.tls_workspace_bytes(s, self.K_b, self.k)
+        self.ws = torch.zeros(self.ws_bytes, dtype=torch.uint8, device=dev)
+        self.engine = tls.tls_engine_create_resident(s, self.K_b, self.k, st.meta, st.label_ch, st.codes, st.scales,
+                                                     st.kv, self.block_idx, self.token_idx, self.ws, self.ws_bytes)
+
+    def step(self, q=None, stream=None):
+        """One staggered step with q (default: the state's q); writes self.out / self.lse."""
+        tls.tls_engine_step(self.engine, self.st.q if q is None else q, self.out_dtype, self.out, self.lse, stream)
+
+    def steps_taken(self) -> int:
+        return tls.tls_engine_steps(self.engine)
+
+    def blocks_of_step(self, t: int) -> torch.Tensor:
+        """M_t (valid after step t, until step t + 2 overwrites it)."""
+        return self.block_idx[t & 1]
+
+    def check_device_error(self, stream=None) -> int:
+        return tls.tls_workspace_error(self.ws, True, stream)
+
+    def close(self):
+        if getattr(self, "engine", None):
+            tls.tls_engine_destroy(self.engine)
+            self.engine = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
 def state_for_config(cfg, q_bits, k_bits, v_bits, label_ch, **kw) -> DecodeState:
     """DecodeState for a workload description with the fields of synth.WorkloadConfig."""
     return DecodeState(batch=cfg.batch, n_q_heads=cfg.n_q_heads, n_kv_heads=cfg.n_kv_heads, qk_dim=cfg.qk_dim,

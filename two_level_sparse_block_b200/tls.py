@@ -92,6 +92,7 @@ _SIG = {
     "tls_prefetch_diff": (_I32, [_P, _P, _P, _I32, _P, _P]),
     "tls_block_cache_table": (_I32, [_P, _P]),
     "tls_engine_create": (_I32, [_P, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "tls_engine_create_resident": (_I32, [_P, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "tls_engine_step": (_I32, [_P, _P, _I32, _P, _P, _P]),
     "tls_engine_steps": (_I64, [_P]),
     "tls_engine_stats": (_I32, [_P, _I64, _P]),
@@ -266,6 +267,15 @@ def tls_engine_create(shape, K_b, k, meta, label_ch, codes, scales, cache, block
     _check(lib().tls_engine_create(ctypes.byref(shape), K_b, k, _ptr(meta), _ptr(label_ch), _ptr(codes),
                                    _ptr(scales), cache, _ptr(block_idx), _ptr(token_idx), _ptr(ws), ws_bytes,
                                    ctypes.byref(h)), "tls_engine_create")
+    return h.value
+
+
+def tls_engine_create_resident(shape, K_b, k, meta, label_ch, codes, scales, kv: KvView, block_idx, token_idx, ws,
+                               ws_bytes) -> int:
+    h = ctypes.c_void_p()
+    _check(lib().tls_engine_create_resident(ctypes.byref(shape), K_b, k, _ptr(meta), _ptr(label_ch), _ptr(codes),
+                                            _ptr(scales), ctypes.byref(kv), _ptr(block_idx), _ptr(token_idx),
+                                            _ptr(ws), ws_bytes, ctypes.byref(h)), "tls_engine_create_resident")
     return h.value
 
 
