@@ -50,6 +50,7 @@ def parse():
     ap.add_argument("--no-offload", action="store_true", help="skip the offload-engine measurement (c4)")
     ap.add_argument("--no-other-configs", action="store_true", help="skip the c1 / c3 step measurements")
     ap.add_argument("--no-staggered", action="store_true", help="skip the staggered-schedule measurement")
+    ap.add_argument("--no-c5", action="store_true", help="skip the c5 per-layer measurements")
     ap.add_argument("--e2e-steps", type=int, default=300)
     return ap.parse_args()
 
@@ -217,19 +218,11 @@ def time_oracle(cfg, q, K, V, lab, seconds, rows_sample=8):
             "s_per_step": step_s}
 
 
-def measure_config(name, dev, steps=200, warmup=10):
-    """One more workload measured like the headline: tls_decode_step replayed
-    from a CUDA graph, L2 flushed (write + read of 256 MB) before each step,
-    CUDA events around each replay."""
-    import synth
+def time_step_graph(st, dev, steps=200, warmup=10):
+    """tls_decode_step of a DecodeState replayed from a CUDA graph, L2 flushed
+    (write + read of 256 MB) before each step, CUDA events around each replay.
+    Returns the per-step times in ms."""
     import torch
-    from two_level_sparse_block_b200 import runtime, tls
-    c = synth.get_config(name)
-    q = synth.gen_queries(c)
-    K, V, _ = synth.gen_kv(c, q)
-    lab = synth.gen_label_channels(c)
-    st = runtime.state_for_config(c, q, K, V, lab, device=dev)
-    del K, V
     flush = torch.empty(64 << 20, dtype=torch.float32, device=dev)
     flush_rd = torch.ones(64 << 20, dtype=torch.float32, device=dev)
     sink = torch.empty((), dtype=torch.float32, device=dev)
@@ -253,11 +246,24 @@ def measure_config(name, dev, steps=200, warmup=10):
             times.append((a, b))
     torch.cuda.synchronize(dev)
     if st.check_device_error() != 0:
-        raise RuntimeError(f"device error in {name}")
-    ts = [x.elapsed_time(y) for x, y in times]
+        raise RuntimeError("device error in a timed step")
+    del g
+    return [x.elapsed_time(y) for x, y in times]
+
+
+def measure_config(name, dev, steps=200, warmup=10):
+    """One more workload measured like the headline (time_step_graph)."""
+    import synth
+    from two_level_sparse_block_b200 import runtime, tls
+    c = synth.get_config(name)
+    q = synth.gen_queries(c)
+    K, V, _ = synth.gen_kv(c, q)
+    lab = synth.gen_label_channels(c)
+    st = runtime.state_for_config(c, q, K, V, lab, device=dev)
+    del K, V
+    ts = time_step_graph(st, dev, steps, warmup)
     ms = statistics.mean(ts)  # (event ticks are coarse: the mean, not the median, averages them out)
     ab = algorithmic_bytes(c)
-    del g
     return {"us_per_step": ms * 1e3, "us_per_step_median": statistics.median(ts) * 1e3,
             "decode_tokens_per_s": c.batch / (ms / 1e3),
             "algorithmic_bytes": ab["step"], "achieved_gbs": ab["step"] / (ms / 1e3) / 1e9,
@@ -309,19 +315,25 @@ def measure_staggered(st, dev, flush_l2, steps, warmup=6):
                         "on a second stream; one graph per step parity, L2 flushed before every step"}
 
 
-def measure_offload_engine(dev, steps=64):
-    """The offload workload (c4): the staggered engine over an HBM block cache of
-    256 slots, K/V in pinned host memory, `steps` consecutive decode steps along
-    the seeded query trajectory.  Steps run back to back (no L2 flush, nothing
-    between them), which leaves the copies the least time to hide."""
+def measure_offload_engine(dev, steps=64, name="c4", data=None):
+    """An offload workload (c4 by default): the staggered engine over an HBM
+    block cache (2 K_b slots a row unless the workload names a count), K/V in
+    pinned host memory, `steps` consecutive decode steps along the seeded query
+    trajectory.  Steps run back to back (no L2 flush, nothing between them),
+    which leaves the copies the least time to hide.  data: (q trajectory, K, V,
+    label channels) already generated, or None."""
     import synth
     import torch
     from two_level_sparse_block_b200 import runtime
-    cfg = synth.get_config("c4")
-    qs = synth.gen_query_trajectory(cfg, steps)
-    K, V, _ = synth.gen_kv(cfg, qs[0])
-    lab = synth.gen_label_channels(cfg)
+    cfg = synth.get_config(name)
+    if data is None:
+        qs = synth.gen_query_trajectory(cfg, steps)
+        K, V, _ = synth.gen_kv(cfg, qs[0])
+        lab = synth.gen_label_channels(cfg)
+    else:
+        qs, K, V, lab = data
     layer = runtime.offloaded_layer_for_config(cfg, K, V, lab)
+    del K, V
     try:
         qd = [torch.from_numpy(np.ascontiguousarray(q).view(np.int16)).to(dev).view(torch.bfloat16) for q in qs]
         stream = torch.cuda.current_stream(dev)
@@ -348,7 +360,7 @@ def measure_offload_engine(dev, steps=64):
         layer.close()
     steady = step_ms[1:]
     return {
-        "workload": cfg.name, "steps": steps, "n_slots": cfg.n_slots * cfg.rows, "K_b": cfg.K_b,
+        "workload": cfg.name, "steps": steps, "n_slots": (cfg.n_slots or 2 * cfg.K_b) * cfg.rows, "K_b": cfg.K_b,
         "us_per_step_median": 1e3 * statistics.median(steady), "us_per_step_mean": 1e3 * statistics.mean(steady),
         "us_first_step": 1e3 * step_ms[0], "prologue_blocks": prologue.n_copied,
         "host_us_per_step_median": 1e6 * statistics.median(host_s[1:]),
@@ -361,6 +373,38 @@ def measure_offload_engine(dev, steps=64):
                   "previous transfer + attention; level 1 runs on the engine's second stream); transfer figures "
                   "from the engine's copy-stream events",
     }
+
+
+def measure_c5(dev, steps_resident=50, steps_offload=24, n_resident=20):
+    """The 36-layer workload (c5), one layer of it measured two ways: resident in
+    HBM (time_step_graph) and offloaded to pinned host memory behind the
+    staggered engine (measure_offload_engine, 2 K_b slots a row).  Each layer's
+    KV is 8 GB, so the 36 layers (290 GB) cannot all be resident: the step is
+    reported as n_resident resident layers plus the rest offloaded, each layer
+    at its measured time (layers run one after another and share nothing)."""
+    import synth
+    from two_level_sparse_block_b200 import runtime
+    c = synth.get_config("c5")
+    qs = synth.gen_query_trajectory(c, steps_offload)
+    K, V, _ = synth.gen_kv(c, qs[0])
+    lab = synth.gen_label_channels(c)
+    st = runtime.state_for_config(c, qs[0], K, V, lab, device=dev)
+    ts = time_step_graph(st, dev, steps_resident, 5)
+    del st
+    import torch
+    torch.cuda.empty_cache()
+    off = measure_offload_engine(dev, steps_offload, "c5", (qs, K, V, lab))
+    res_us = statistics.mean(ts) * 1e3
+    off_us = off["us_per_step_mean"]
+    n_layers = 36
+    step_us = n_resident * res_us + (n_layers - n_resident) * off_us
+    ab = algorithmic_bytes(c)
+    return {"layers": n_layers, "layer_kv_bytes": 2 * c.rows * c.ctx_len * c.qk_dim * 2,
+            "resident_layer_us": res_us, "resident_layer_achieved_gbs": ab["step"] / (res_us / 1e6) / 1e9,
+            "offloaded_layer": off, "n_resident_layers": n_resident,
+            "step_us_composed": step_us, "decode_tokens_per_s_composed": c.batch / (step_us / 1e6),
+            "composition": f"{n_resident} layers resident in HBM (each layer's 8 GB KV plus index; about 20 fit "
+                           f"in 180 GB) + {n_layers - n_resident} offloaded, each at its measured per-layer time"}
 
 
 def run_reference(args, cfg):
@@ -566,6 +610,8 @@ def main():
     }
     if rank == 0 and world == 1 and not args.no_offload:
         line["offload_engine"] = measure_offload_engine(dev)
+    if rank == 0 and world == 1 and not args.no_c5:
+        line["c5_layers"] = measure_c5(dev)
     if rank == 0 and world == 1 and not args.no_other_configs:
         line["other_configs"] = {n: measure_config(n, dev) for n in ("c1", "c3") if n != c.name}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
