@@ -73,15 +73,14 @@ struct BsSmem {
 // keys, the row's keys for a one-CTA selection, the selection scratch).
 template <int CL>
 __host__ __device__ inline int bs_body_bytes(int stage_bytes, int nb) {
-  int sel = (kBsTile + nb) * 4 + (int)sizeof(TopkScratch);
-  if constexpr (CL >= 2) sel += (int)sizeof(ClusterTopkScratch<CL>) + 16;
+  const int sel = (kBsTile + nb) * 4 + (int)sizeof(TopkScratch);
   return stage_bytes > sel ? stage_bytes : sel;
 }
 
 // CL: how the row's top-K_b is taken.  1: the row is one tile, its CTA
-// selects; 2, 4, 8: the row's CTAs form a cluster and select together over
-// distributed shared memory (cluster_topk.cuh); 0: the last CTA of the row
-// (a ticket) selects from the scores in the workspace.
+// selects; 2, 4, 8: the row's CTAs form a cluster, push their keys into the
+// leader's shared memory, and the leader selects (cta_topk_regs); 0: the last
+// CTA of the row (a ticket) selects from the scores in the workspace.
 // Q' = [relu(q_h), min(q_h, 0)] of every row, bf16 [rows * npad][2 * Dqk]
 // (rows h >= G zero): the level-1 B operand, written once per step for wide
 // groups so that each level-1 CTA loads it by TMA instead of rebuilding it.
@@ -264,7 +263,8 @@ __global__ void __launch_bounds__(128, 1)
     const float* arow = p.agg + (int64_t)row * p.nb;
     for (int i = tid; i < p.nb; i += 128) keys[i] = float_key(__ldcg(arow + i));
     __syncthreads();
-    cta_topk_ascending<128>(keys, p.nb, p.K_b, out, *ts, [](int i) { return i; });
+    if (p.nb <= 128 * 16) cta_topk_regs<128, 16>(keys, p.nb, p.K_b, out, *ts, [](int i) { return i; });
+    else cta_topk_ascending<128>(keys, p.nb, p.K_b, out, *ts, [](int i) { return i; });
   } else {
     // the drained stages hold the selection: this CTA's keys, then the row's
     uint32_t* mine = reinterpret_cast<uint32_t*>(smem);  // [kBsTile]
@@ -276,25 +276,16 @@ __global__ void __launch_bounds__(128, 1)
     if constexpr (CL == 1) {
       cta_topk_ascending<128>(mine, n_loc, p.K_b, out, *ts, [](int i) { return i; });
     } else {
+      // every CTA pushes its keys into the leader's row array; after one
+      // cluster barrier the leader selects alone with the keys in registers
       namespace cg = cooperative_groups;
       cg::cluster_group cluster = cg::this_cluster();
-      auto* cts = reinterpret_cast<ClusterTopkScratch<CL>*>((reinterpret_cast<uintptr_t>(ts + 1) + 15) &
-                                                            ~uintptr_t(15));
       cluster_wait();
-      if (cluster_topk_ascending<128, CL>(mine, n_loc, mt * kBsTile, p.K_b, out, *cts, [](int i) { return i; }))
-        return;
-      // degenerate scores or a crowded threshold bin: the leader gathers the
-      // row's keys through distributed shared memory and selects alone
-      if (mt == 0) {
-        for (int r = 0; r < CL; ++r) {
-          const uint32_t* src = cluster.map_shared_rank(mine, r);
-          const int b0 = r * kBsTile, n = min(kBsTile, p.nb - b0);
-          for (int i = tid; i < n; i += 128) all[b0 + i] = src[i];
-        }
-      }
-      cluster.sync();  // the other CTAs' shared memory may be released after this
+      uint32_t* dst = cluster.map_shared_rank(all, 0) + mt * kBsTile;
+      if (tid < n_loc) dst[tid] = mine[tid];
+      cluster.sync();  // the leader's keys are complete; no remote access after this
       if (mt != 0) return;
-      cta_topk_ascending<128>(all, p.nb, p.K_b, out, *ts, [](int i) { return i; });
+      cta_topk_regs<128, CL>(all, p.nb, p.K_b, out, *ts, [](int i) { return i; });
     }
   }
 }

@@ -131,8 +131,11 @@ __device__ __forceinline__ int topk_sub_bin(uint32_t key, float fmin, float inv)
   return max(0, min(255, (int)((key_float(key) - fmin) * inv)));
 }
 
+// Out of line: it is the fallback of the other selections, and its code
+// inlined into their kernels would sit between their hot phases and the
+// instruction fetch.
 template <int NT, typename MapFn>
-__device__ void cta_topk_ascending(const uint32_t* keys, int n, int k, int* out, TopkScratch& sm,
+__device__ __noinline__ void cta_topk_ascending(const uint32_t* keys, int n, int k, int* out, TopkScratch& sm,
                                    MapFn map) {
   static_assert(NT % 32 == 0 && NT >= kTopkRankMax && NT <= 1024, "CTA size");
   constexpr int NW = NT / 32;
@@ -555,34 +558,39 @@ __device__ void cta_topk_regs(const uint32_t* keys, int n, int k, int* out, Topk
   }
 
   // 3. pairwise ranking inside the cell: TPC adjacent threads per key, thread
-  // `part` comparing the 16-byte chunks part, part + TPC, ... (the TPC lanes
-  // of a key read adjacent chunks: no bank conflicts)
+  // `part` comparing the 16-byte chunks part, part + TPC, ... that hold
+  // candidates (the TPC lanes of a key read adjacent chunks: no bank
+  // conflicts), four chunk loads in flight at a time
   {
     constexpr int TPC = NT / kTopkRankMax;  // 1, 2, 4 or 8
-    constexpr int NCH = kTopkRankMax / 4 / TPC;  // chunks per thread
     const int nc = sm.tcount;
     const int c = tid / TPC, part = tid % TPC;
     if (c < nc) {
       const uint32_t mine = sm.cand[c];
-      int gt = 0, eq = 0;
+      const int nq = (nc + 4 * TPC - 1) / (4 * TPC);  // chunks per thread
       const bool vec = (smem_addr32(sm.cand) & 15u) == 0u;  // (the scratch may sit anywhere 4-byte aligned)
-#pragma unroll
-      for (int q = 0; q < NCH; ++q) {
-        const int i0 = 4 * (q * TPC + part);
-        uint32_t o[4];
-        if (vec) {
-          const uint4 v = *reinterpret_cast<const uint4*>(sm.cand + i0);
-          o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
-        } else {
-#pragma unroll
-          for (int u = 0; u < 4; ++u) o[u] = sm.cand[i0 + u];
-        }
+      int gt = 0, eq = 0;
+      for (int q0 = 0; q0 < nq; q0 += 4) {
+        uint32_t o[4][4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const bool in = i0 + u < nc;
-          gt += (int)(in && o[u] > mine);
-          eq += (int)(in && o[u] == mine);
+          const int i0 = 4 * ((q0 + u) * TPC + part);
+          if (q0 + u < nq && vec) {
+            const uint4 v = *reinterpret_cast<const uint4*>(sm.cand + i0);
+            o[u][0] = v.x; o[u][1] = v.y; o[u][2] = v.z; o[u][3] = v.w;
+          } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[u][e] = q0 + u < nq ? sm.cand[i0 + e] : 0u;
+          }
         }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const bool in = q0 + u < nq && 4 * ((q0 + u) * TPC + part) + e < nc;
+            gt += (int)(in && o[u][e] > mine);
+            eq += (int)(in && o[u][e] == mine);
+          }
       }
       // the TPC lanes of a key are adjacent and all inside the c < nc branch
       const unsigned grp = TPC == 32 ? 0xffffffffu : (((1u << TPC) - 1u) << (lane & ~(TPC - 1)));
