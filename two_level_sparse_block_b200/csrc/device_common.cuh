@@ -423,9 +423,9 @@ __device__ __noinline__ void cta_topk_ascending(const uint32_t* keys, int n, int
 //   4. counts above / equal to tau scanned over the CTA, then each thread
 //      writes its own taken positions
 // Degenerate keys (all equal, not finite, or a wide run of equal keys at the
-// threshold) go to cta_topk_ascending.  `keys` is shared memory, 16-byte
-// aligned when KPT is a multiple of 4; its first k words are overwritten (the
-// output is staged there).
+// threshold) go to cta_topk_ascending.  `keys` is shared memory (read with
+// 16-byte loads when it is 16-byte aligned and KPT a multiple of 4); its first
+// k words are overwritten (the output is staged there).
 template <int NT, int KPT, typename MapFn>
 __device__ void cta_topk_regs(const uint32_t* keys, int n, int k, int* out, TopkScratch& sm, MapFn map) {
   static_assert(NT % 32 == 0 && NT >= kTopkRankMax && NT <= 1024 && KPT >= 1 && KPT <= 32, "shape");
@@ -435,7 +435,7 @@ __device__ void cta_topk_regs(const uint32_t* keys, int n, int k, int* out, Topk
   uint32_t kv[KPT];
   uint32_t cell = 0u;  // bit j: key j is valid and still in the threshold cell
   if constexpr (KPT % 4 == 0) {
-    if (p0 + KPT <= n) {
+    if (p0 + KPT <= n && (smem_addr32(keys) & 15u) == 0u) {
 #pragma unroll
       for (int j = 0; j < KPT; j += 4) {
         const uint4 v = *reinterpret_cast<const uint4*>(keys + p0 + j);
