@@ -50,9 +50,12 @@ __device__ __forceinline__ uint32_t mla_off(int r, int u) {
 // exchange [2][kMlaWarps][16 x 16] fp32, then m/l [16] x 2
 constexpr int kMlaOffS = kMlaStages * kMlaStageBytes;
 constexpr int kMlaOffStat = kMlaOffS + 2 * kMlaWarps * 256 * 4;
-constexpr int kMlaSmem = kMlaOffStat + 2 * kMlaHeads * 4;
-// after the loop the ring holds this CTA's partial O [16][512] fp32 (32 KB)
-static_assert(kMlaHeads * kMlaV * 4 <= kMlaStages * kMlaStageBytes, "partial O must fit the ring");
+constexpr int kMlaOffRid = kMlaOffStat + 2 * kMlaHeads * 4;  // then the split's row ids, int64 each
+constexpr int kMlaSmem = kMlaOffRid;
+// after the loop the ring holds this CTA's partial O [16][512] fp32 (rows
+// padded to 520 floats, so the 8 rows a warp store touches hit 8 banks)
+constexpr int kMlaOStride = kMlaV + 8;
+static_assert(kMlaHeads * kMlaOStride * 4 <= kMlaStages * kMlaStageBytes, "partial O must fit the ring");
 
 __device__ __forceinline__ uint32_t mla_pack_bf16(float a, float b) {
   uint32_t r;
@@ -102,10 +105,8 @@ __device__ __forceinline__ void mla_issue(const AttnParams& p, int64_t rid, uint
   }
 }
 
-// Row id of entry (lane & 15) of the chunk at list position t_base, or -1.
-__device__ __forceinline__ int64_t mla_rid(const AttnParams& p, int row, int t_base, int t_end) {
-  const int t = t_base + (threadIdx.x & 15);
-  if (t >= t_end) return -1;
+// Row id (index into the K/V rows) of list entry t of the row, t < k.
+__device__ __forceinline__ int64_t mla_rid(const AttnParams& p, int row, int t) {
   // L2 load: the list is written by the preceding kernel while this grid is
   // already resident (programmatic dependent launch)
   const int64_t tk = min(max((int64_t)__ldcg(p.token_idx + (int64_t)row * p.k_sel + t), (int64_t)0), p.ctx_len - 1);
@@ -123,9 +124,9 @@ __global__ void __launch_bounds__(kMlaWarps * 32, 2) sparse_attn_mla_kernel(Attn
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   const uint32_t ring = smem_u32(sm);
-  float* sS = reinterpret_cast<float*>(sm + kMlaOffS);     // [2][warp][lane * 8 + i]
+  float* sS = reinterpret_cast<float*>(sm + kMlaOffS);     // [2][warp][i * 32 + lane]
   float* sM = reinterpret_cast<float*>(sm + kMlaOffStat);  // m [16], then l [16]
-  float* sO = reinterpret_cast<float*>(sm);                // after the loop: O [16][512]
+  float* sO = reinterpret_cast<float*>(sm);                // after the loop: O [16][kMlaOStride]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gq = lane >> 2, tq = lane & 3;
@@ -157,6 +158,12 @@ __global__ void __launch_bounds__(kMlaWarps * 32, 2) sparse_attn_mla_kernel(Attn
     }
   }
   grid_dependency_wait();  // token lists come from the preceding kernel
+  // the row ids of this split's entries, padded with -1 (zero-fill) to whole
+  // chunks: one round trip to the list now instead of one per chunk in the loop
+  int64_t* srid = reinterpret_cast<int64_t*>(sm + kMlaOffRid);
+  for (int i = tid; i < n_chunks * kMlaChunk; i += kMlaWarps * 32)
+    srid[i] = t_lo + i < t_hi ? mla_rid(p, row, t_lo + i) : (int64_t)-1;
+  __syncthreads();
 
   float o[16][4];
 #pragma unroll
@@ -165,7 +172,7 @@ __global__ void __launch_bounds__(kMlaWarps * 32, 2) sparse_attn_mla_kernel(Attn
 
 #pragma unroll
   for (int s = 0; s < NS - 1; ++s) {
-    if (s < n_chunks) mla_issue(p, mla_rid(p, row, t_lo + s * kMlaChunk, t_hi), ring + s * kMlaStageBytes);
+    if (s < n_chunks) mla_issue(p, srid[s * kMlaChunk + (lane & 15)], ring + s * kMlaStageBytes);
     cp_async_commit();
   }
   for (int c = 0; c < n_chunks; ++c) {
@@ -173,7 +180,7 @@ __global__ void __launch_bounds__(kMlaWarps * 32, 2) sparse_attn_mla_kernel(Attn
     __syncthreads();          // everyone's have; every warp is past chunk c - 1
     {
       const int cn = c + NS - 1;  // refill the stage chunk c - 1 used
-      if (cn < n_chunks) mla_issue(p, mla_rid(p, row, t_lo + cn * kMlaChunk, t_hi), ring + (cn % NS) * kMlaStageBytes);
+      if (cn < n_chunks) mla_issue(p, srid[cn * kMlaChunk + (lane & 15)], ring + (cn % NS) * kMlaStageBytes);
       cp_async_commit();
     }
     const uint32_t st = ring + (c % NS) * kMlaStageBytes;
@@ -202,11 +209,12 @@ __global__ void __launch_bounds__(kMlaWarps * 32, 2) sparse_attn_mla_kernel(Attn
       }
     }
     // the four partial S summed in a fixed order: every warp holds the same S
-    float* mine = sS + ((c & 1) * kMlaWarps + warp) * 256 + lane * 8;
+    // (element i of lane l at [i][l]: consecutive lanes, consecutive banks)
+    float* mine = sS + ((c & 1) * kMlaWarps + warp) * 256 + lane;
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) mine[nt * 4 + e] = s[nt][e];
+      for (int e = 0; e < 4; ++e) mine[(nt * 4 + e) * 32] = s[nt][e];
     __syncthreads();
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
@@ -214,7 +222,7 @@ __global__ void __launch_bounds__(kMlaWarps * 32, 2) sparse_attn_mla_kernel(Attn
       for (int e = 0; e < 4; ++e) {
         float v = 0.0f;
 #pragma unroll
-        for (int w = 0; w < kMlaWarps; ++w) v += sS[((c & 1) * kMlaWarps + w) * 256 + lane * 8 + nt * 4 + e];
+        for (int w = 0; w < kMlaWarps; ++w) v += sS[((c & 1) * kMlaWarps + w) * 256 + (nt * 4 + e) * 32 + lane];
         s[nt][e] = v * p.scale_log2;
       }
     if (t_base + kMlaChunk > t_hi) {
@@ -284,10 +292,10 @@ __global__ void __launch_bounds__(kMlaWarps * 32, 2) sparse_attn_mla_kernel(Attn
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
     const int d = 128 * warp + j * 8 + 2 * tq;
-    sO[gq * kMlaV + d] = o[j][0];
-    sO[gq * kMlaV + d + 1] = o[j][1];
-    sO[(gq + 8) * kMlaV + d] = o[j][2];
-    sO[(gq + 8) * kMlaV + d + 1] = o[j][3];
+    sO[gq * kMlaOStride + d] = o[j][0];
+    sO[gq * kMlaOStride + d + 1] = o[j][1];
+    sO[(gq + 8) * kMlaOStride + d] = o[j][2];
+    sO[(gq + 8) * kMlaOStride + d + 1] = o[j][3];
   }
   if (warp == 0 && tq == 0) {
     sM[gq] = m0;
@@ -331,7 +339,7 @@ __global__ void __launch_bounds__(kMlaWarps * 32, 2) sparse_attn_mla_kernel(Attn
     const int h = idx >> 6, d = 64 * split + (idx & 63);
     float v[kMlaSplits];
 #pragma unroll
-    for (int j = 0; j < kMlaSplits; ++j) v[j] = j < CL ? cluster.map_shared_rank(sO, j)[h * kMlaV + d] : 0.0f;
+    for (int j = 0; j < kMlaSplits; ++j) v[j] = j < CL ? cluster.map_shared_rank(sO, j)[h * kMlaOStride + d] : 0.0f;
     float acc = 0.0f;
 #pragma unroll
     for (int j = 0; j < kMlaSplits; ++j) acc = fmaf(sW[h * kMlaSplits + j], v[j], acc);
@@ -353,7 +361,7 @@ int attn_mla_tokens_per_split(int k) {
 }
 
 tls_status launch_attn_mla(const AttnParams& p, int rows, cudaStream_t stream, bool pdl) {
-  const size_t smem = 128 + (size_t)kMlaSmem;
+  const size_t smem = 128 + (size_t)kMlaSmem + (size_t)p.tokens_per_split * 8;
   cudaError_t e = cudaFuncSetAttribute(sparse_attn_mla_kernel<kMlaStages>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return cuda_check(e, "sparse_decode_attn: set smem attribute");
