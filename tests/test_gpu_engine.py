@@ -280,3 +280,35 @@ def test_resident_engine_steps_replay_from_graphs():
     finally:
         del graphs
         eng.close()
+
+
+def test_resident_engine_on_the_headline_workload_sampled_rows():
+    # c2 (Qwen3-8B shape, 32K context) through the resident engine, the path
+    # the benchmark times: level 2 on half the SMs beside level 1; three steps
+    # of a q trajectory, sampled rows checked against the staggered oracle
+    cfg = synth.get_config("c2")
+    qs = synth.gen_query_trajectory(cfg, 3)
+    runtime, st, (K, V, lab) = _resident(cfg, qs)
+    eng = runtime.ResidentEngine(st)
+    g = cfg.group
+    try:
+        for t, q in enumerate(qs):
+            eng.step(_dev_q(q))
+            torch.cuda.synchronize()
+            assert eng.check_device_error() == 0
+            m_prev = eng.block_idx[(t + 1) & 1].cpu().numpy()
+            m_cur = eng.block_idx[t & 1].cpu().numpy()
+            tok = eng.token_idx.cpu().numpy()
+            out = eng.out.float().cpu().numpy()
+            for b, h in _rows(cfg, 2):
+                where = f"c2 resident step {t} row ({b},{h})"
+                r1 = _orow(cfg, q, K, V, lab, b, h)
+                check_selection(m_cur[b, h], r1["agg"], cfg.K_b, where + " M_t")
+                r2 = _orow(cfg, q, K, V, lab, b, h, block_idx=m_prev[b, h])
+                pos = np.searchsorted(r2["cand"], tok[b, h])
+                assert np.array_equal(r2["cand"][pos], tok[b, h]), f"{where}: token outside M_t-1"
+                check_selection(pos, r2["token_score"], cfg.k, where + " tokens")
+                r3 = _orow(cfg, q, K, V, lab, b, h, block_idx=m_prev[b, h], token_idx=tok[b, h])
+                check_output(out[b, h * g:(h + 1) * g], r3["out"], where + " out")
+    finally:
+        eng.close()

@@ -15,7 +15,7 @@ tls_status select_blocks_impl(const tls_shape& s, const void* q, const void* met
 tls_status select_tokens_impl(const tls_shape& s, const void* q, const int32_t* label_ch, const uint8_t* codes,
                               const float* scales, const int32_t* block_idx, int K_b, int k, int32_t* token_idx,
                               float* token_score, uint8_t* ws, const WsLayout& L, cudaStream_t stream,
-                              bool pdl = false);
+                              bool pdl = false, bool lean = false);
 tls_status sparse_attn_impl(const tls_shape& s, const void* q, const tls_kv_view& kv, const int32_t* token_idx,
                             int k, int out_dtype, void* out, float* lse, uint8_t* ws, const WsLayout& L,
                             cudaStream_t stream, bool pdl = true);

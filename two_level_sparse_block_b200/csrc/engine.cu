@@ -18,8 +18,8 @@
 // which step t's attention reads, so C may run alongside it.
 //
 // A resident engine (K/V in HBM, no cache) keeps only the stagger, with no
-// host wait: A: event q_t; B: wait q_t, level 1 -> M_t, event sel_t; A: level 2
-// over M_{t-1}, attention, wait sel_t.  Level 1 of step t overwrites the list
+// host wait: A: event q_t, level 2 over M_{t-1}; B: wait q_t, level 1 -> M_t,
+// event sel_t; A: attention, wait sel_t.  Level 1 of step t overwrites the list
 // level 2 read at step t-1, which A finished before recording q_t; level 2 of
 // step t+1 reads M_t, which the join at the end of step t completes.  Every
 // step forks and joins within itself, so it can be captured into a graph.
@@ -35,7 +35,7 @@ tls_status select_blocks_impl(const tls_shape& s, const void* q, const void* met
 tls_status select_tokens_impl(const tls_shape& s, const void* q, const int32_t* label_ch, const uint8_t* codes,
                               const float* scales, const int32_t* block_idx, int K_b, int k, int32_t* token_idx,
                               float* token_score, uint8_t* ws, const WsLayout& L, cudaStream_t stream,
-                              bool pdl = false);
+                              bool pdl = false, bool lean = false);
 tls_status sparse_attn_impl(const tls_shape& s, const void* q, const tls_kv_view& kv, const int32_t* token_idx,
                             int k, int out_dtype, void* out, float* lse, uint8_t* ws, const WsLayout& L,
                             cudaStream_t stream, bool pdl = true);
@@ -200,20 +200,24 @@ tls_status resident_step(tls_engine* e, const void* q, int32_t out_dtype, void* 
     st = select_blocks_impl(s, q, e->meta, e->K_b, e->bidx[prev], nullptr, e->ws, e->L, A);
     if (st != TLS_OK) return st;
   }
-  // fork: level 1 for q_t on the select stream, after everything A has issued
+  // level 2 within M_{t-1} first, on A (it is on the critical path; launched
+  // first, its CTAs are placed first), on at most half the SMs, which leaves
+  // level 1 the other half
   cudaError_t ce = cudaEventRecord(e->ev_q, A);
-  if (ce == cudaSuccess) ce = cudaStreamWaitEvent(e->sel, e->ev_q, 0);
+  if (ce != cudaSuccess) return cuda_check(ce, "engine_step: q event");
+  st = select_tokens_impl(s, q, e->label_ch, e->codes, e->scales, e->bidx[prev], e->K_b, e->k, e->token_idx, nullptr,
+                          e->ws, e->L, A, /*pdl=*/false, /*lean=*/true);
+  if (st != TLS_OK) return st;
+  // fork: level 1 for q_t on the select stream, after what A had issued
+  // before level 2 (it writes M_t, which no kernel of this step reads)
+  ce = cudaStreamWaitEvent(e->sel, e->ev_q, 0);
   if (ce != cudaSuccess) return cuda_check(ce, "engine_step: select stream");
   st = select_blocks_impl(s, q, e->meta, e->K_b, e->bidx[cur], nullptr, e->ws, e->L, e->sel);
   if (st != TLS_OK) return st;
   ce = cudaEventRecord(e->ev_sel, e->sel);
   if (ce != cudaSuccess) return cuda_check(ce, "engine_step: select stream");
-  // level 2 within M_{t-1} and the attention, on A
-  st = select_tokens_impl(s, q, e->label_ch, e->codes, e->scales, e->bidx[prev], e->K_b, e->k, e->token_idx, nullptr,
-                          e->ws, e->L, A, /*pdl=*/false);
-  if (st != TLS_OK) return st;
-  // programmatic launch after level 2, as in the synchronous step (a plain
-  // launch measured slower: level 1 still competes with level 2 for the SMs)
+  // programmatic launch: level 2 lets the attention's CTAs in only once it has
+  // scored, so they do not hold the SMs level 1 needs for long
   st = sparse_attn_impl(s, q, e->kv, e->token_idx, e->k, out_dtype, out, lse, e->ws, e->L, A, /*pdl=*/true);
   if (st != TLS_OK) return st;
   // join: M_t is complete before anything A issues next

@@ -305,11 +305,10 @@ __host__ __device__ inline bool token_row_kernel_fits(int group, int n_label, in
 }
 
 // CTAs per row of the row-cluster kernel: 4, 2 or 1, as many as keep every
-// CTA at 8 blocks or more and the grid within two CTAs per SM.
-__host__ __device__ inline int token_row_cluster_size(int rows, int K_b, int bs) {
+// CTA at 8 blocks or more and the grid within `max_ctas` CTAs.
+__host__ __device__ inline int token_row_cluster_size(int rows, int K_b, int max_ctas) {
   int cl = 4;
-  while (cl > 1 && ((int64_t)rows * cl > 2 * 148 || K_b < 8 * cl)) cl /= 2;
-  (void)bs;
+  while (cl > 1 && ((int64_t)rows * cl > max_ctas || K_b < 8 * cl)) cl /= 2;
   return cl;
 }
 

@@ -169,7 +169,6 @@ __global__ void __launch_bounds__(kRowThreads, KPT <= 8 ? 2 : 1) token_select_ro
   int32_t* bidx = reinterpret_cast<int32_t*>(qlab + p.group * R);                 // [K_b]
   TopkScratch* ts = reinterpret_cast<TopkScratch*>(bidx + ((p.K_b + 3) & ~3));
   if (cl > 1) cluster_arrive_relaxed();  // completes once every CTA of the cluster has started
-  grid_launch_dependents();
   load_qlab<R, kRowThreads>(p, row, qlab);
   if (threadIdx.x == 0 && rank == 0) prefetch_l2(p.token_idx + (int64_t)row * p.k);
   grid_dependency_wait();  // the block lists come from the preceding kernel
@@ -178,6 +177,10 @@ __global__ void __launch_bounds__(kRowThreads, KPT <= 8 ? 2 : 1) token_select_ro
   stage_candidate_codes<R, kRowThreads>(p, row, bidx, j0, j1, scodes, sscales);
   __syncthreads();
   score_candidates_tc<R, kRowThreads, NTILE, true>(p, row, qlab, bidx, c0, c1, keys, scodes, sscales);
+  // the next grid (the attention) may become resident from here: only the
+  // selection is left, and earlier it would hold SMs a concurrent level 1
+  // needs
+  grid_launch_dependents();
   __syncthreads();
   if (cl > 1) {
     cluster_wait();
@@ -219,12 +222,15 @@ void fill_token_params(TokenParams& p, const tls_shape& s, const void* q, const 
   p.token_idx = token_idx;
 }
 
+// `lean`: the row kernel on at most half the SMs (the other half is left to
+// a level-1 grid running beside it, as in the resident stagger).
 // `pdl`: the preceding kernel of the stream is this library's level-1 kernel,
 // which writes only the block lists (the one input the cluster kernel reads
 // after its dependency wait), so the launch may overlap its tail.
 tls_status select_tokens_impl(const tls_shape& s, const void* q, const int32_t* label_ch, const uint8_t* codes,
                               const float* scales, const int32_t* block_idx, int K_b, int k, int32_t* token_idx,
-                              float* token_score, uint8_t* ws, const WsLayout& L, cudaStream_t stream, bool pdl) {
+                              float* token_score, uint8_t* ws, const WsLayout& L, cudaStream_t stream, bool pdl,
+                              bool lean) {
   constexpr int NT = 256;
   const int rows = rows_of(s);
   TokenParams p;
@@ -246,7 +252,7 @@ tls_status select_tokens_impl(const tls_shape& s, const void* q, const int32_t* 
       ((reinterpret_cast<uintptr_t>(codes) | reinterpret_cast<uintptr_t>(scales)) & 15u) == 0) {
     const int kpt = p.n_cand <= 2 * kRowThreads ? 2 : p.n_cand <= 4 * kRowThreads ? 4
                   : p.n_cand <= 8 * kRowThreads ? 8 : 16;
-    const int cl = token_row_cluster_size(rows, K_b, s.block_size);
+    const int cl = token_row_cluster_size(rows, K_b, lean ? kNumSMs / 2 : 2 * kNumSMs);
     const int bpc = (K_b + cl - 1) / cl;
     const size_t rsmem = (size_t)kpt * kRowThreads * 4 + (size_t)bpc * s.block_size * (s.n_label / 2 + 4) +
                          ((size_t)p.group * s.n_label + ((K_b + 3) & ~3)) * 4 + sizeof(TopkScratch);
