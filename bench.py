@@ -49,8 +49,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-offload", action="store_true", help="skip the offload-engine measurement (c4)")
     ap.add_argument("--no-other-configs", action="store_true", help="skip the c1 / c3 step measurements")
-    ap.add_argument("--no-staggered", action="store_true", help="skip the staggered-schedule measurement")
     ap.add_argument("--no-c5", action="store_true", help="skip the c5 per-layer measurements")
+    ap.add_argument("--no-staggered", action="store_true",
+                    help="time the synchronous step (tls_decode_step) as the headline instead of the staggered one")
     ap.add_argument("--e2e-steps", type=int, default=300)
     return ap.parse_args()
 
@@ -271,50 +272,6 @@ def measure_config(name, dev, steps=200, warmup=10):
             "l2": "flushed before every step (write + read of 256 MB)"}
 
 
-def measure_staggered(st, dev, flush_l2, steps, warmup=6):
-    """The staggered schedule over the same HBM-resident layer (ResidentEngine):
-    step t runs level 2 and the attention within M_{t-1} while level 1 chooses
-    M_t on a second stream, joined at the end of the step.  Two graphs (the two
-    parities of the block lists) replayed alternately, L2 flushed before every
-    step as for the headline, CUDA events around each replay."""
-    import torch
-    from two_level_sparse_block_b200 import runtime
-    eng = runtime.ResidentEngine(st)
-    cap = torch.cuda.Stream(dev)
-    graphs = []
-    with torch.cuda.stream(cap):
-        eng.step(stream=cap)  # step 0, with the prologue (M_{-1})
-        for _ in range(2):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=cap):
-                eng.step(stream=cap)
-            graphs.append(g)
-    stream = torch.cuda.current_stream(dev)
-    stream.wait_stream(cap)
-    torch.cuda.synchronize(dev)
-    evs = []
-    for i in range(warmup + steps):
-        flush_l2(i)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        graphs[i & 1].replay()
-        b.record(stream)
-        if i >= warmup:
-            evs.append((a, b))
-    torch.cuda.synchronize(dev)
-    err = eng.check_device_error()
-    del graphs
-    eng.close()
-    if err != 0:
-        raise RuntimeError(f"device error {err} in the staggered engine")
-    ts = [a.elapsed_time(b) for a, b in evs]
-    ms = statistics.mean(ts)
-    return {"us_per_step": ms * 1e3, "us_per_step_median": statistics.median(ts) * 1e3,
-            "decode_tokens_per_s": st.shape.batch / (ms / 1e3), "steps": steps,
-            "schedule": "step t: level 2 + attention within M_{t-1} on the caller's stream, level 1 for q_t "
-                        "on a second stream; one graph per step parity, L2 flushed before every step"}
-
-
 def measure_offload_engine(dev, steps=64, name="c4", data=None):
     """An offload workload (c4 by default): the staggered engine over an HBM
     block cache (2 K_b slots a row unless the workload names a count), K/V in
@@ -470,36 +427,51 @@ def main():
         torch.sum(flush_rd, dim=0, out=sink)
     torch.cuda.synchronize(dev)
 
-    # The step (tls_decode_step: block scores + top-K_b, token scores + top-k,
-    # attention) is captured once into a CUDA graph and replayed, so the timed
-    # loop spends no host time per kernel and the events measure the GPU
-    # alone.  Two more graphs hold tls_select and tls_sparse_decode_attn for
-    # the per-stage times (the attention alone, K and V read from HBM).
+    # The timed step is the hot path as the method schedules it: the resident
+    # staggered engine (tls_engine_create_resident / tls_engine_step), where
+    # step t runs level 2 and the attention within the blocks chosen at step
+    # t-1 while level 1 chooses M_t for q_t beside them.  Its steps are
+    # captured into two CUDA graphs (the two parities of its block lists) and
+    # replayed alternately, so the timed loop spends no host time per kernel
+    # and the events measure the GPU alone.  The synchronous step
+    # (tls_decode_step: levels 1, 2 and the attention in order) is captured
+    # too and timed beside it, and two more graphs hold tls_select and
+    # tls_sparse_decode_attn for the per-stage times (the attention alone, K
+    # and V read from HBM).
+    eng = runtime.ResidentEngine(st)
     cap = torch.cuda.Stream(dev)
     cap.wait_stream(stream)
     g_step, g_sel, g_att = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    g_stag = [torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()]
     with torch.cuda.stream(cap):
         st.step(stream=cap)
         st.select(stream=cap)
         st.attend(stream=cap)
+        eng.step(stream=cap)  # step 0 with its prologue (M_{-1} from q_0)
         with torch.cuda.graph(g_step, stream=cap):
             st.step(stream=cap)
         with torch.cuda.graph(g_sel, stream=cap):
             st.select(stream=cap)
         with torch.cuda.graph(g_att, stream=cap):
             st.attend(stream=cap)
+        for g in g_stag:
+            with torch.cuda.graph(g, stream=cap):
+                eng.step(stream=cap)
     stream.wait_stream(cap)
     torch.cuda.synchronize(dev)
 
     def step_events(n):
         return [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
 
-    def timed_steps(n, evs):
+    def timed_steps(n, evs, synchronous=False):
         for i in range(n):
             flush_l2(i)
             e = evs[i]
             e[0].record(stream)
-            g_step.replay()
+            if synchronous:
+                g_step.replay()
+            else:
+                g_stag[i & 1].replay()
             e[1].record(stream)
 
     def stage_times(n):
@@ -514,10 +486,12 @@ def main():
         torch.cuda.synchronize(dev)
         return ([e[0].elapsed_time(e[1]) for e in evs], [e[1].elapsed_time(e[2]) for e in evs])
 
+    sync_headline = args.no_staggered
     warm = step_events(args.warmup)
     timed_steps(args.warmup, warm)
+    timed_steps(args.warmup, warm, synchronous=True)
     torch.cuda.synchronize(dev)
-    if st.check_device_error() != 0:
+    if st.check_device_error() != 0 or eng.check_device_error() != 0:
         raise RuntimeError("device error during warm-up")
 
     evs = step_events(args.steps)
@@ -533,25 +507,33 @@ def main():
     sampler.start()
     time.sleep(0.3)
     wall0 = time.perf_counter()
-    timed_steps(args.steps, evs)
+    timed_steps(args.steps, evs, synchronous=sync_headline)
     torch.cuda.synchronize(dev)
     wall = time.perf_counter() - wall0
     clocks = sampler.stop()
     if world > 1:
         dist.barrier()
-    err = st.check_device_error()
+    err = st.check_device_error() if sync_headline else eng.check_device_error()
     if err != 0:
         raise RuntimeError(f"device error {err} during the timed steps")
 
     step_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    # the synchronous step, timed the same way (untimed by the headline)
+    n_sync = min(args.steps, 500)
+    sync_evs = step_events(n_sync)
+    timed_steps(n_sync, sync_evs, synchronous=True)
+    torch.cuda.synchronize(dev)
+    if st.check_device_error() != 0:
+        raise RuntimeError("device error in the synchronous steps")
+    sync_ms = [e[0].elapsed_time(e[1]) for e in sync_evs]
     # stage breakdown (separate graphs, so each stage also pays its own launch)
-    sel_ms, att_ms = stage_times(min(args.steps, 500))
-    staggered = measure_staggered(st, dev, flush_l2, min(args.steps, 500)) if not args.no_staggered else None
+    sel_ms, att_ms = stage_times(n_sync)
     total_ms = sum(step_ms)
-    t = torch.tensor([total_ms, statistics.mean(att_ms)], dtype=torch.float64, device=dev)
+    t = torch.tensor([total_ms, statistics.mean(att_ms), statistics.mean(sync_ms)], dtype=torch.float64,
+                     device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, att_mean_ms = float(t[0]), float(t[1])
+    total_ms, att_mean_ms, sync_mean_ms = float(t[0]), float(t[1]), float(t[2])
     ms_per_step = total_ms / args.steps
     value = world * c.batch / (ms_per_step / 1e3)
 
@@ -565,8 +547,8 @@ def main():
         flush_l2(i)
         e2e_ev[i][0].record(stream)
         q_dev.copy_(q_host, non_blocking=True)
-        st.step(q=q_dev, stream=stream)
-        out_host.copy_(st.out, non_blocking=True)
+        eng.step(q=q_dev, stream=stream)
+        out_host.copy_(eng.out, non_blocking=True)
         e2e_ev[i][1].record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = sum(e[0].elapsed_time(e[1]) for e in e2e_ev) / args.e2e_steps
@@ -591,12 +573,18 @@ def main():
                    "k": c.k, "label_channels": c.n_label, "parallelism": f"weak x{world} (independent batches)",
                    "l2": "between timed steps (untimed): write a 256 MB buffer, then read another 256 MB buffer; "
                          "every step starts with none of its lines in L2 and no dirty line to write back"},
+        "schedule": ("synchronous step (tls_decode_step), one graph" if sync_headline else
+                     "the method's staggered step (tls_engine_step on a resident engine): level 2 and the "
+                     "attention within the blocks chosen at step t-1, level 1 for q_t beside them on a second "
+                     "stream; two graphs (block-list parities) replayed alternately"),
+        "synchronous_step": {"us_per_step": sync_mean_ms * 1e3, "decode_tokens_per_s": world * c.batch /
+                             (sync_mean_ms / 1e3), "steps": n_sync,
+                             "path": "tls_decode_step (levels 1, 2 and the attention in order), one graph"},
         "stage_us": {"select (levels 1+2)": 1e3 * statistics.mean(sel_ms),
                      "sparse_decode_attn": 1e3 * statistics.mean(att_ms),
                      "note": "tls_select and tls_sparse_decode_attn replayed as separate graphs (each pays its own "
-                             "launch, the attention reads K and V from HBM); the step is one tls_decode_step graph"},
+                             "launch, the attention reads K and V from HBM)"},
         "step_hbm": {"algorithmic_bytes": ab["step"], "achieved_gbs": step_gbs, "frac_of_peak": step_gbs / peak},
-        "staggered_engine": staggered,
         "roofline": {"kernel": attn_kernel, "bound": "hbm", "achieved": achieved,
                      "peak": peak, "peak_source": f"hbm_gbs {peak_kind}", "unit": "GB/s", "frac": achieved / peak,
                      "algorithmic_bytes_per_launch": ab["attn"],
@@ -604,7 +592,8 @@ def main():
         "gpu_launches": launches_per_step(c) * args.steps,
         "e2e": {"value": world * c.batch / (e2e_ms / 1e3), "unit": "decode tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": int(st.q.numel() * 2), "d2h_bytes_per_step": int(st.out.numel() * st.out.element_size()),
-                "path": "tls_decode_step via the Python binding, q from pinned host, out to pinned host"},
+                "path": "tls_engine_step (resident engine) via the Python binding, one call per step, q from "
+                        "pinned host, out to pinned host"},
         "clocks": clocks,
         "wall_s_timed": wall,
     }

@@ -371,8 +371,7 @@ tls_status launch_tc(const CUtensorMap& tmap, const CUtensorMap& qmap, const Blo
   using L = BsSmem<NPAD>;
   const int body = bs_body_bytes<CL>(L::STAGE_BYTES, p.nb);
   const size_t smem = 1024 + (size_t)((body + 7) & ~7) + (2 * kBsStages + 1) * 8 + 16;
-  cudaError_t e = cudaFuncSetAttribute(block_score_tc_kernel<NPAD, CL>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = kernel_attrs((const void*)block_score_tc_kernel<NPAD, CL>, smem);
   if (e != cudaSuccess) return cuda_check(e, "select_blocks: set smem attribute");
   const dim3 grid((unsigned)((p.nb + kBsTile - 1) / kBsTile), (unsigned)rows);
   if constexpr (CL >= 2)
@@ -418,8 +417,7 @@ tls_status select_blocks_impl(const tls_shape& s, const void* q, const void* met
 
   if (use_simt()) {
     const size_t smem = (size_t)p.group * 2 * s.qk_dim * 4 + (size_t)nb * 4 + sizeof(TopkScratch) + 16;
-    cudaError_t e = cudaFuncSetAttribute(block_score_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    cudaError_t e = kernel_attrs((const void*)block_score_simt_kernel, smem);
     if (e != cudaSuccess) return cuda_check(e, "select_blocks: set smem attribute");
     dim3 grid((unsigned)((nb + 127) / 128), (unsigned)rows);
     block_score_simt_kernel<<<grid, 128, smem, stream>>>((const uint16_t*)meta, p);

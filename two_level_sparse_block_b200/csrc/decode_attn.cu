@@ -213,8 +213,7 @@ template <int PK, int PV, int HG>
 tls_status launch_attn(const AttnParams& p, int rows, cudaStream_t stream) {
   constexpr int U = (PK + PV <= 2) ? 4 : 1;
   const size_t smem = (size_t)(16 * HG + 8 * HG * p.dv) * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<PK, PV, HG, U>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = kernel_attrs((const void*)sparse_attn_kernel<PK, PV, HG, U>, smem);
   if (e != cudaSuccess) return cuda_check(e, "sparse_decode_attn: set smem attribute");
   dim3 grid((unsigned)p.splits, (unsigned)p.head_groups, (unsigned)rows);
   sparse_attn_kernel<PK, PV, HG, U><<<grid, 128, smem, stream>>>(p);

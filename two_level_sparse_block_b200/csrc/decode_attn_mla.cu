@@ -362,8 +362,7 @@ int attn_mla_tokens_per_split(int k) {
 
 tls_status launch_attn_mla(const AttnParams& p, int rows, cudaStream_t stream, bool pdl) {
   const size_t smem = 128 + (size_t)kMlaSmem + (size_t)p.tokens_per_split * 8;
-  cudaError_t e = cudaFuncSetAttribute(sparse_attn_mla_kernel<kMlaStages>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = kernel_attrs((const void*)sparse_attn_mla_kernel<kMlaStages>, smem);
   if (e != cudaSuccess) return cuda_check(e, "sparse_decode_attn: set smem attribute");
   const dim3 grid(kMlaSplits, (unsigned)(p.group / kMlaHeads), (unsigned)rows);
   return cuda_check(launch_ex(sparse_attn_mla_kernel<kMlaStages>, grid, dim3(kMlaWarps * 32), smem, stream, pdl,

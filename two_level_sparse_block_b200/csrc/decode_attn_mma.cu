@@ -542,17 +542,14 @@ static tls_status launch_mma(const AttnParams& p, int rows, cudaStream_t stream,
   rows *= p.head_groups;  // virtual rows (row, head group)
   const int cl = attn_mma_cluster_size(rows, p.heads_per_cta);
   if (cl > 0) {
-    cudaError_t e = cudaFuncSetAttribute(sparse_attn_mma_cluster_kernel<NS>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e == cudaSuccess && cl > 8)  // 16-CTA clusters are beyond the portable size
-      e = cudaFuncSetAttribute(sparse_attn_mma_cluster_kernel<NS>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    // 16-CTA clusters are beyond the portable size
+    cudaError_t e = kernel_attrs((const void*)sparse_attn_mma_cluster_kernel<NS>, smem, cl > 8);
     if (e != cudaSuccess) return cuda_check(e, "sparse_decode_attn: set cluster attributes");
     return cuda_check(launch_ex(sparse_attn_mma_cluster_kernel<NS>, dim3(cl, rows), dim3(kMmaWarps * 32), smem, stream,
                                 pdl, (unsigned)cl, p),
                       "sparse_decode_attn: mma cluster launch");
   }
-  cudaError_t e =
-      cudaFuncSetAttribute(sparse_attn_mma_kernel<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = kernel_attrs((const void*)sparse_attn_mma_kernel<NS>, smem);
   if (e != cudaSuccess) return cuda_check(e, "sparse_decode_attn: set smem attribute");
   return cuda_check(launch_ex(sparse_attn_mma_kernel<NS>, dim3(p.n_ctas), dim3(kMmaWarps * 32), smem, stream, pdl, 0u, p),
                     "sparse_decode_attn: mma launch");

@@ -7,7 +7,9 @@
 
 #include <cstdarg>
 #include <cstdio>
+#include <mutex>
 #include <string>
+#include <unordered_map>
 
 #include "tls.h"
 
@@ -69,6 +71,38 @@ constexpr int kNumSMs = 148;
 // may start before the preceding kernel of the stream ends; it calls
 // griddepcontrol.wait before reading that kernel's output) and optional
 // thread-block clusters of cluster_x CTAs along x (cluster_x <= 1: none).
+// cudaFuncSetAttribute once per kernel, device and value (the dynamic shared
+// memory limit only ever rises): a launch path that runs every decode step
+// should not pay the driver calls each time.
+inline cudaError_t kernel_attrs(const void* fn, size_t smem_bytes, bool nonportable_cluster = false) {
+  struct Key {
+    const void* fn;
+    int dev;
+    bool operator==(const Key& o) const { return fn == o.fn && dev == o.dev; }
+  };
+  struct KeyHash {
+    size_t operator()(const Key& k) const { return std::hash<const void*>()(k.fn) * 31u + (size_t)k.dev; }
+  };
+  static std::mutex mu;
+  static std::unordered_map<Key, std::pair<size_t, bool>, KeyHash> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  auto& d = done[Key{fn, dev}];
+  if (smem_bytes > d.first) {
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes);
+    if (e != cudaSuccess) return e;
+    d.first = smem_bytes;
+  }
+  if (nonportable_cluster && !d.second) {
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+    d.second = true;
+  }
+  return cudaSuccess;
+}
+
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
                              bool pdl, unsigned cluster_x, Args... args) {

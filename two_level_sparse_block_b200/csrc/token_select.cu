@@ -257,7 +257,7 @@ tls_status select_tokens_impl(const tls_shape& s, const void* q, const int32_t* 
     const size_t rsmem = (size_t)kpt * kRowThreads * 4 + (size_t)bpc * s.block_size * (s.n_label / 2 + 4) +
                          ((size_t)p.group * s.n_label + ((K_b + 3) & ~3)) * 4 + sizeof(TopkScratch);
     auto launch = [&](auto kernel) -> tls_status {
-      cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem);
+      cudaError_t e = kernel_attrs((const void*)kernel, rsmem);
       if (e != cudaSuccess) return cuda_check(e, "select_tokens: set kernel attributes");
       return cuda_check(launch_ex(kernel, dim3((unsigned)cl, (unsigned)rows), dim3(kRowThreads), rsmem, stream, pdl,
                                   (unsigned)cl, p),
@@ -285,9 +285,8 @@ tls_status select_tokens_impl(const tls_shape& s, const void* q, const int32_t* 
         ((size_t)p.group * s.n_label + K_b + per + p.n_cand) * 4 + sizeof(TopkScratch) + cts_bytes + 32;
     const int ntile = p.group <= 16 ? 2 : p.group <= 32 ? 4 : p.group <= 64 ? 8 : 16;
     auto launch = [&](auto kernel) -> tls_status {
-      cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)csmem);
-      if (e == cudaSuccess && cl > 8)  // 16-CTA clusters are beyond the portable size
-        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      // 16-CTA clusters are beyond the portable size
+      cudaError_t e = kernel_attrs((const void*)kernel, csmem, cl > 8);
       if (e != cudaSuccess) return cuda_check(e, "select_tokens: set kernel attributes");
       return cuda_check(launch_ex(kernel, dim3((unsigned)cl, (unsigned)rows), dim3(kTokThreads), csmem, stream, pdl,
                                   (unsigned)cl, p),
@@ -326,8 +325,7 @@ tls_status select_tokens_impl(const tls_shape& s, const void* q, const int32_t* 
   switch (s.n_label) {
 #define TLS_TS_CASE(RR)                                                                                     \
   case RR: {                                                                                                \
-    cudaError_t e =                                                                                         \
-        cudaFuncSetAttribute(token_select_kernel<RR, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
+    cudaError_t e = kernel_attrs((const void*)token_select_kernel<RR, NT>, smem);                          \
     if (e != cudaSuccess) return cuda_check(e, "select_tokens: set smem attribute");                        \
     token_select_kernel<RR, NT><<<grid, NT, smem, stream>>>(p);                                             \
     break;                                                                                                  \
