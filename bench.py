@@ -579,25 +579,50 @@ def main():
     ms_per_step = total_ms / args.steps
     value = world * c.batch / (ms_per_step / 1e3)
 
-    # end to end through the public API: pinned host q in, host out back, every step
+    # end to end through the public API: pinned host q in, host out back, every
+    # step.  As a serving loop runs it: the host -> device copy of q, the
+    # engine step and the device -> host copy of the output captured together
+    # into graphs (one per block-list parity) and replayed; and, for
+    # reference, the same three calls issued eagerly every step.
     q_host = torch.empty(st.q.shape, dtype=torch.bfloat16).pin_memory()
     q_host.copy_(st.q.cpu())
     out_host = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
-    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.e2e_steps)]
     q_dev = torch.empty_like(st.q)
-    for i in range(args.e2e_steps):
-        flush_l2(i)
-        e2e_ev[i][0].record(stream)
-        q_dev.copy_(q_host, non_blocking=True)
-        eng.step(q=q_dev, stream=stream)
-        out_host.copy_(eng.out, non_blocking=True)
-        e2e_ev[i][1].record(stream)
+    g_e2e = [torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()]
+    cap.wait_stream(stream)
+    with torch.cuda.stream(cap):
+        for g in g_e2e:
+            with torch.cuda.graph(g, stream=cap):
+                q_dev.copy_(q_host, non_blocking=True)
+                eng.step(q=q_dev, stream=cap)
+                out_host.copy_(eng.out, non_blocking=True)
+    stream.wait_stream(cap)
     torch.cuda.synchronize(dev)
-    e2e_ms = sum(e[0].elapsed_time(e[1]) for e in e2e_ev) / args.e2e_steps
-    t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+
+    def e2e_times(n, eager):
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
+        for i in range(n):
+            flush_l2(i)
+            evs[i][0].record(stream)
+            if eager:
+                q_dev.copy_(q_host, non_blocking=True)
+                eng.step(q=q_dev, stream=stream)
+                out_host.copy_(eng.out, non_blocking=True)
+            else:
+                g_e2e[i & 1].replay()
+            evs[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        return sum(e[0].elapsed_time(e[1]) for e in evs) / n
+
+    e2e_ms = e2e_times(args.e2e_steps, eager=False)
+    e2e_eager_ms = e2e_times(args.e2e_steps, eager=True)
+    if eng.check_device_error() != 0:
+        raise RuntimeError("device error in the end-to-end steps")
+    t = torch.tensor([e2e_ms, e2e_eager_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_ms = float(t[0])
+    e2e_ms, e2e_eager_ms = float(t[0]), float(t[1])
+    del g_e2e
 
     ab = algorithmic_bytes(c)
     attn_kernel = tls.tls_attn_kernel(st.shape)
@@ -634,8 +659,11 @@ def main():
         "gpu_launches": launches_per_step(c) * args.steps,
         "e2e": {"value": world * c.batch / (e2e_ms / 1e3), "unit": "decode tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": int(st.q.numel() * 2), "d2h_bytes_per_step": int(st.out.numel() * st.out.element_size()),
-                "path": "tls_engine_step (resident engine) via the Python binding, one call per step, q from "
-                        "pinned host, out to pinned host"},
+                "path": "tls_engine_step (resident engine) via the Python binding, q copied in from pinned host "
+                        "and the output copied back to pinned host every step, the three captured together in "
+                        "graphs (one per block-list parity) and replayed",
+                "eager_ms_per_step": e2e_eager_ms,
+                "eager_path": "the same three calls issued from Python every step, no graph"},
         "clocks": clocks,
         "wall_s_timed": wall,
     }
