@@ -150,10 +150,10 @@ __global__ void __launch_bounds__(kTokThreads) token_select_cluster_kernel(Token
 // cores and pushes the keys into the leader's shared memory; the leader then
 // selects with the register-resident top-k (cta_topk_regs), CTA barriers
 // only.  For narrow groups (G <= 16) and rows of at most 8192 candidates.
-constexpr int kRowThreads = 512;
+constexpr int kRowThreads = 512;  // the default CTA; 1024 when a row has one CTA of its own (`lean`)
 
-template <int R, int NTILE, int KPT>
-__global__ void __launch_bounds__(kRowThreads, KPT <= 8 ? 2 : 1) token_select_row_kernel(TokenParams p) {
+template <int R, int NTILE, int KPT, int NT>
+__global__ void __launch_bounds__(NT, NT >= 1024 || KPT > 8 ? 1 : 2) token_select_row_kernel(TokenParams p) {
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
   const int cl = (int)cluster.num_blocks(), rank = (int)cluster.block_rank();
@@ -162,21 +162,21 @@ __global__ void __launch_bounds__(kRowThreads, KPT <= 8 ? 2 : 1) token_select_ro
   const int j0 = min(p.K_b, rank * bpc), j1 = min(p.K_b, j0 + bpc);
   const int c0 = j0 * p.bs, c1 = j1 * p.bs;
   extern __shared__ __align__(16) uint32_t smw[];
-  uint32_t* keys = smw;                                                           // [KPT * kRowThreads]
-  uint8_t* scodes = reinterpret_cast<uint8_t*>(smw + KPT * kRowThreads);          // [bpc * bs][R / 2]
+  uint32_t* keys = smw;                                                           // [KPT * NT]
+  uint8_t* scodes = reinterpret_cast<uint8_t*>(smw + KPT * NT);          // [bpc * bs][R / 2]
   float* sscales = reinterpret_cast<float*>(scodes + (size_t)bpc * p.bs * (R / 2));  // [bpc * bs]
   float* qlab = sscales + bpc * p.bs;                                             // [G][R]
   int32_t* bidx = reinterpret_cast<int32_t*>(qlab + p.group * R);                 // [K_b]
   TopkScratch* ts = reinterpret_cast<TopkScratch*>(bidx + ((p.K_b + 3) & ~3));
   if (cl > 1) cluster_arrive_relaxed();  // completes once every CTA of the cluster has started
-  load_qlab<R, kRowThreads>(p, row, qlab);
+  load_qlab<R, NT>(p, row, qlab);
   if (threadIdx.x == 0 && rank == 0) prefetch_l2(p.token_idx + (int64_t)row * p.k);
   grid_dependency_wait();  // the block lists come from the preceding kernel
-  load_block_list<kRowThreads>(p, row, bidx);
+  load_block_list<NT>(p, row, bidx);
   __syncthreads();
-  stage_candidate_codes<R, kRowThreads>(p, row, bidx, j0, j1, scodes, sscales);
+  stage_candidate_codes<R, NT>(p, row, bidx, j0, j1, scodes, sscales);
   __syncthreads();
-  score_candidates_tc<R, kRowThreads, NTILE, true>(p, row, qlab, bidx, c0, c1, keys, scodes, sscales);
+  score_candidates_tc<R, NT, NTILE, true>(p, row, qlab, bidx, c0, c1, keys, scodes, sscales);
   // the next grid (the attention) may become resident from here: only the
   // selection is left, and earlier it would hold SMs a concurrent level 1
   // needs
@@ -188,13 +188,13 @@ __global__ void __launch_bounds__(kRowThreads, KPT <= 8 ? 2 : 1) token_select_ro
       // keys of [c0, c1) into the leader's array (bs is a multiple of 4: whole 16-byte units)
       uint4* dst = reinterpret_cast<uint4*>(cluster.map_shared_rank(keys, 0) + c0);
       const uint4* src = reinterpret_cast<const uint4*>(keys);
-      for (int i = threadIdx.x; i < (c1 - c0) / 4; i += kRowThreads) dst[i] = src[i];
+      for (int i = threadIdx.x; i < (c1 - c0) / 4; i += NT) dst[i] = src[i];
     }
     cluster.sync();  // the leader's keys are complete; no remote access after this
     if (rank != 0) return;
   }
   const CandidateToken map{bidx, p.bs};
-  cta_topk_regs<kRowThreads, KPT>(keys, p.n_cand, p.k, p.token_idx + (int64_t)row * p.k, *ts, map);
+  cta_topk_regs<NT, KPT>(keys, p.n_cand, p.k, p.token_idx + (int64_t)row * p.k, *ts, map);
 }
 
 void fill_token_params(TokenParams& p, const tls_shape& s, const void* q, const int32_t* label_ch,
@@ -250,25 +250,29 @@ tls_status select_tokens_impl(const tls_shape& s, const void* q, const int32_t* 
   const size_t smem = (size_t)p.group * s.n_label * 4 + (size_t)p.n_cand * 4 + sizeof(TopkScratch) + 16;
   if (token_row_kernel_fits(p.group, s.n_label, p.n_cand, s.block_size) &&
       ((reinterpret_cast<uintptr_t>(codes) | reinterpret_cast<uintptr_t>(scales)) & 15u) == 0) {
-    const int kpt = p.n_cand <= 2 * kRowThreads ? 2 : p.n_cand <= 4 * kRowThreads ? 4
-                  : p.n_cand <= 8 * kRowThreads ? 8 : 16;
     const int cl = token_row_cluster_size(rows, K_b, lean ? kNumSMs / 2 : 2 * kNumSMs);
+    // a row alone in its CTA gets 1024 threads: twice the warps to score it
+    const int nt = (cl == 1 && p.n_cand <= 8 * 1024) ? 1024 : kRowThreads;
+    const int kpt = p.n_cand <= 2 * nt ? 2 : p.n_cand <= 4 * nt ? 4 : p.n_cand <= 8 * nt ? 8 : 16;
     const int bpc = (K_b + cl - 1) / cl;
-    const size_t rsmem = (size_t)kpt * kRowThreads * 4 + (size_t)bpc * s.block_size * (s.n_label / 2 + 4) +
+    const size_t rsmem = (size_t)kpt * nt * 4 + (size_t)bpc * s.block_size * (s.n_label / 2 + 4) +
                          ((size_t)p.group * s.n_label + ((K_b + 3) & ~3)) * 4 + sizeof(TopkScratch);
     auto launch = [&](auto kernel) -> tls_status {
       cudaError_t e = kernel_attrs((const void*)kernel, rsmem);
       if (e != cudaSuccess) return cuda_check(e, "select_tokens: set kernel attributes");
-      return cuda_check(launch_ex(kernel, dim3((unsigned)cl, (unsigned)rows), dim3(kRowThreads), rsmem, stream, pdl,
+      return cuda_check(launch_ex(kernel, dim3((unsigned)cl, (unsigned)rows), dim3((unsigned)nt), rsmem, stream, pdl,
                                   (unsigned)cl, p),
                         "select_tokens launch");
     };
-    auto by_kpt = [&](auto k2, auto k4, auto k8, auto k16) -> tls_status {
+    auto by_kpt = [&](auto k2, auto k4, auto k8, auto k16, auto w2, auto w4, auto w8) -> tls_status {
+      if (nt == 1024) return kpt == 2 ? launch(w2) : kpt == 4 ? launch(w4) : launch(w8);
       return kpt == 2 ? launch(k2) : kpt == 4 ? launch(k4) : kpt == 8 ? launch(k8) : launch(k16);
     };
 #define TLS_ROW(RR, NN)                                                                                     \
-  by_kpt(token_select_row_kernel<RR, NN, 2>, token_select_row_kernel<RR, NN, 4>, token_select_row_kernel<RR, NN, 8>, \
-         token_select_row_kernel<RR, NN, 16>)
+  by_kpt(token_select_row_kernel<RR, NN, 2, 512>, token_select_row_kernel<RR, NN, 4, 512>,                  \
+         token_select_row_kernel<RR, NN, 8, 512>, token_select_row_kernel<RR, NN, 16, 512>,                 \
+         token_select_row_kernel<RR, NN, 2, 1024>, token_select_row_kernel<RR, NN, 4, 1024>,                \
+         token_select_row_kernel<RR, NN, 8, 1024>)
     if (s.n_label == 16) return p.group <= 8 ? TLS_ROW(16, 1) : TLS_ROW(16, 2);
     return p.group <= 8 ? TLS_ROW(32, 1) : TLS_ROW(32, 2);
 #undef TLS_ROW
