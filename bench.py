@@ -67,6 +67,22 @@ def workload(cfg, rank):
     return c, q, K, V, lab
 
 
+def max_over_ranks(values, world, device=None):
+    """Each timing (ms) as the slowest rank saw it: the job's step time is set
+    by its last rank.  One all-reduce (MAX) over the process group."""
+    import torch
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
+def job_tokens_per_s(world, batch, ms_per_step):
+    """Whole-job decode tokens/s: every rank decodes its own batch of `batch` rows per step."""
+    return world * batch / (ms_per_step / 1e3)
+
+
 def algorithmic_bytes(cfg):
     """Bytes the step must move: metadata, candidate label codes+scales,
     gathered K/V rows, queries, index lists and the fp32 output."""
@@ -570,14 +586,10 @@ def main():
     sync_ms = [e[0].elapsed_time(e[1]) for e in sync_evs]
     # stage breakdown (separate graphs, so each stage also pays its own launch)
     sel_ms, att_ms = stage_times(n_sync)
-    total_ms = sum(step_ms)
-    t = torch.tensor([total_ms, statistics.mean(att_ms), statistics.mean(sync_ms)], dtype=torch.float64,
-                     device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, att_mean_ms, sync_mean_ms = float(t[0]), float(t[1]), float(t[2])
+    total_ms, att_mean_ms, sync_mean_ms = max_over_ranks(
+        [sum(step_ms), statistics.mean(att_ms), statistics.mean(sync_ms)], world, dev)
     ms_per_step = total_ms / args.steps
-    value = world * c.batch / (ms_per_step / 1e3)
+    value = job_tokens_per_s(world, c.batch, ms_per_step)
 
     # end to end through the public API: pinned host q in, host out back, every
     # step.  As a serving loop runs it: the host -> device copy of q, the
@@ -618,10 +630,7 @@ def main():
     e2e_eager_ms = e2e_times(args.e2e_steps, eager=True)
     if eng.check_device_error() != 0:
         raise RuntimeError("device error in the end-to-end steps")
-    t = torch.tensor([e2e_ms, e2e_eager_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_ms, e2e_eager_ms = float(t[0]), float(t[1])
+    e2e_ms, e2e_eager_ms = max_over_ranks([e2e_ms, e2e_eager_ms], world, dev)
     del g_e2e
 
     ab = algorithmic_bytes(c)
@@ -644,8 +653,8 @@ def main():
                      "the method's staggered step (tls_engine_step on a resident engine): level 2 and the "
                      "attention within the blocks chosen at step t-1, level 1 for q_t beside them on a second "
                      "stream; two graphs (block-list parities) replayed alternately"),
-        "synchronous_step": {"us_per_step": sync_mean_ms * 1e3, "decode_tokens_per_s": world * c.batch /
-                             (sync_mean_ms / 1e3), "steps": n_sync,
+        "synchronous_step": {"us_per_step": sync_mean_ms * 1e3,
+                             "decode_tokens_per_s": job_tokens_per_s(world, c.batch, sync_mean_ms), "steps": n_sync,
                              "path": "tls_decode_step (levels 1, 2 and the attention in order), one graph"},
         "stage_us": {"select (levels 1+2)": 1e3 * statistics.mean(sel_ms),
                      "sparse_decode_attn": 1e3 * statistics.mean(att_ms),
@@ -657,7 +666,7 @@ def main():
                      "algorithmic_bytes_per_launch": ab["attn"],
                      "traffic": recorded_traffic(attn_kernel, c.name)},
         "gpu_launches": launches_per_step(c) * args.steps,
-        "e2e": {"value": world * c.batch / (e2e_ms / 1e3), "unit": "decode tokens/s", "ms_per_step": e2e_ms,
+        "e2e": {"value": job_tokens_per_s(world, c.batch, e2e_ms), "unit": "decode tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": int(st.q.numel() * 2), "d2h_bytes_per_step": int(st.out.numel() * st.out.element_size()),
                 "path": "tls_engine_step (resident engine) via the Python binding, q copied in from pinned host "
                         "and the output copied back to pinned host every step, the three captured together in "
