@@ -422,6 +422,66 @@ def measure_c5(dev, steps_resident=50, steps_offload=24, n_resident=20):
                            f"in 180 GB) + {n_layers - n_resident} offloaded, each at its measured per-layer time"}
 
 
+def measure_c5_loop(dev, steps=6, n_resident=20, n_layers=36):
+    """The 36-layer workload (c5) as one decode loop: per step, n_resident
+    layers with their KV in HBM (resident staggered engines) and the rest
+    offloaded to pinned host memory behind their own block caches (offload
+    engines), layer after layer on one stream, each layer with its own q
+    trajectory.  Every layer decodes the same seeded 8 GB KV (one HBM copy for
+    the resident layers, one pinned host copy for the offloaded ones, one
+    index), since 36 distinct copies (290 GB) fit neither memory; each layer
+    keeps its own block lists, token lists, slot pool and transfers.  Every
+    layer reads more than L2 holds, so consecutive layers share no cached
+    lines.  CUDA events around each whole decode step."""
+    import synth
+    import torch
+    from two_level_sparse_block_b200 import runtime
+    c = synth.get_config("c5")
+    qs = [synth.gen_query_trajectory(c, steps, layer=l) for l in range(n_layers)]
+    K, V, _ = synth.gen_kv(c, qs[0][0])
+    lab = synth.gen_label_channels(c)
+    st = runtime.state_for_config(c, qs[0][0], K, V, lab, device=dev)
+    resident = [runtime.ResidentEngine(st) for _ in range(n_resident)]
+    first = runtime.offloaded_layer_for_config(c, K, V, lab)
+    del K, V
+    offloaded = [first] + [runtime.offloaded_layer_for_config(c, None, None, lab, share_from=first)
+                           for _ in range(n_layers - n_resident - 1)]
+    try:
+        qd = [[torch.from_numpy(np.ascontiguousarray(q).view(np.int16)).to(dev).view(torch.bfloat16) for q in ql]
+              for ql in qs]
+        stream = torch.cuda.current_stream(dev)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        torch.cuda.synchronize(dev)
+        for t in range(steps):
+            evs[t][0].record(stream)
+            for l in range(n_layers):
+                if l < n_resident:
+                    resident[l].step(q=qd[l][t], stream=stream)
+                else:
+                    offloaded[l - n_resident].step(qd[l][t], stream=stream)
+            evs[t][1].record(stream)
+        torch.cuda.synchronize(dev)
+        if any(e.check_device_error() != 0 for e in resident) or any(o.check_device_error() != 0 for o in offloaded):
+            raise RuntimeError("device error in the 36-layer loop")
+        step_ms = [a.elapsed_time(b) for a, b in evs]
+        moved = [sum(o.stats(t).bytes_copied for o in offloaded) for t in range(steps - 1)]
+        blocks = [sum(o.stats(t).n_copied for o in offloaded) for t in range(steps - 1)]
+    finally:
+        for e in resident:
+            e.close()
+        for o in offloaded:
+            o.close()
+    steady = step_ms[1:]  # the first step also makes every offloaded layer's M_{-1} resident
+    ms = statistics.mean(steady)
+    return {"layers": n_layers, "n_resident_layers": n_resident, "steps": steps,
+            "ms_per_step_mean": ms, "decode_tokens_per_s": c.batch / (ms / 1e3),
+            "ms_first_step": step_ms[0], "h2d_bytes_per_step_mean": statistics.mean(moved),
+            "transfer_blocks_per_step_mean": statistics.mean(blocks),
+            "h2d_gbs_needed": statistics.mean(moved) / (ms / 1e3) / 1e9,
+            "timing": "CUDA events around each decode step (36 layer steps issued back to back on one stream; "
+                      "each offloaded layer's call waits on the host for its level 1)"}
+
+
 def run_reference(args, cfg):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -680,6 +740,7 @@ def main():
         line["offload_engine"] = measure_offload_engine(dev)
     if rank == 0 and world == 1 and not args.no_c5:
         line["c5_layers"] = measure_c5(dev)
+        line["c5_layers"]["loop_36_layers"] = measure_c5_loop(dev)
     if rank == 0 and world == 1 and not args.no_other_configs:
         line["other_configs"] = {n: measure_config(n, dev) for n in ("c1", "c3") if n != c.name}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -171,7 +171,7 @@ class OffloadedLayer:
 
     def __init__(self, *, batch, n_q_heads, n_kv_heads, qk_dim, v_dim, v_offset, block_size, n_label, ctx_len,
                  K_b, k, n_slots, k_bits, v_bits, label_ch, softmax_scale=None, out_dtype=tls.TLS_OUT_F32,
-                 device="cuda"):
+                 device="cuda", share_from=None):
         dev = torch.device(device)
         self.device = dev
         scale = 1.0 / math.sqrt(qk_dim) if softmax_scale is None else softmax_scale
@@ -181,27 +181,36 @@ class OffloadedLayer:
         self.rows = batch * n_kv_heads
         self.nb = ctx_len // block_size
         self.out_dtype = out_dtype
-        # full K/V in pinned host memory
-        self.host_k = torch.from_numpy(np.ascontiguousarray(k_bits).view(np.int16)).pin_memory()
-        self.host_v = (torch.from_numpy(np.ascontiguousarray(v_bits).view(np.int16)).pin_memory()
-                       if v_bits is not None else None)
-        # resident index, built from a temporary device copy of K
-        self.label_ch = torch.from_numpy(np.ascontiguousarray(label_ch, dtype=np.int32)).to(dev)
-        self.meta = torch.empty((batch, n_kv_heads, self.nb, 2 * qk_dim), dtype=torch.bfloat16, device=dev)
-        self.codes = torch.empty((batch, n_kv_heads, ctx_len, n_label // 2), dtype=torch.uint8, device=dev)
-        self.scales = torch.empty((batch, n_kv_heads, ctx_len), dtype=torch.float32, device=dev)
-        kd = self.host_k.to(dev).view(torch.bfloat16)
-        tls.tls_build_block_meta(self.shape, kd, qk_dim, 0, ctx_len, self.meta, None)
-        tls.tls_quant_label_cache(self.shape, kd, qk_dim, self.label_ch, 0, ctx_len, self.codes, self.scales, None)
-        torch.cuda.synchronize(dev)
-        del kd
+        if share_from is not None:
+            # another layer object over the same host K/V and index (its own
+            # cache, block lists and engine): the pinned buffers and the index
+            # are shared, read-only
+            for name in ("host_k", "host_v", "label_ch", "meta", "codes", "scales"):
+                setattr(self, name, getattr(share_from, name))
+        else:
+            # full K/V in pinned host memory
+            self.host_k = torch.from_numpy(np.ascontiguousarray(k_bits).view(np.int16)).pin_memory()
+            self.host_v = (torch.from_numpy(np.ascontiguousarray(v_bits).view(np.int16)).pin_memory()
+                           if v_bits is not None else None)
+            # resident index, built from a temporary device copy of K
+            self.label_ch = torch.from_numpy(np.ascontiguousarray(label_ch, dtype=np.int32)).to(dev)
+            self.meta = torch.empty((batch, n_kv_heads, self.nb, 2 * qk_dim), dtype=torch.bfloat16, device=dev)
+            self.codes = torch.empty((batch, n_kv_heads, ctx_len, n_label // 2), dtype=torch.uint8, device=dev)
+            self.scales = torch.empty((batch, n_kv_heads, ctx_len), dtype=torch.float32, device=dev)
+            kd = self.host_k.to(dev).view(torch.bfloat16)
+            tls.tls_build_block_meta(self.shape, kd, qk_dim, 0, ctx_len, self.meta, None)
+            tls.tls_quant_label_cache(self.shape, kd, qk_dim, self.label_ch, 0, ctx_len, self.codes, self.scales,
+                                      None)
+            torch.cuda.synchronize(dev)
+            del kd
+        with_v = self.host_v is not None
         # the HBM block cache
         self.slot_k = torch.empty((n_slots, block_size, qk_dim), dtype=torch.bfloat16, device=dev)
         self.slot_v = (torch.empty((n_slots, block_size, v_dim), dtype=torch.bfloat16, device=dev)
-                       if v_bits is not None else None)
+                       if with_v else None)
         self.slot_table = torch.full((batch, n_kv_heads, self.nb), -1, dtype=torch.int32, device=dev)
         self.cache = tls.tls_block_cache_create(self.shape, self.host_k, self.host_v, qk_dim,
-                                                v_dim if v_bits is not None else 0, n_slots, self.slot_k,
+                                                v_dim if with_v else 0, n_slots, self.slot_k,
                                                 self.slot_v, self.slot_table)
         self.block_idx = torch.empty((2, batch, n_kv_heads, self.K_b), dtype=torch.int32, device=dev)
         self.token_idx = torch.empty((batch, n_kv_heads, self.k), dtype=torch.int32, device=dev)
