@@ -352,6 +352,10 @@ TLS_API tls_status tls_engine_create(const tls_shape* shape, int32_t K_b, int32_
  * engine allocates one stream and its events.  Its steps never wait on the
  * host, so a step may be captured into a CUDA graph on its stream (each step
  * forks level 1 onto the engine's stream and joins it back before returning).
+ * A captured step keeps the block-list parity of the step it was captured
+ * at (it writes M_t into one of the two lists and reads M_{t-1} from the
+ * other): capture two consecutive steps and replay the two graphs
+ * alternately.  Captures count as steps in tls_engine_steps; replays do not.
  */
 TLS_API tls_status tls_engine_create_resident(const tls_shape* shape, int32_t K_b, int32_t k, const void* meta,
                                       const int32_t* label_ch, const uint8_t* codes, const float* scales,
