@@ -112,6 +112,21 @@ TLS_API int32_t tls_version(void);
 TLS_API const char* tls_attn_kernel(const tls_shape* shape);
 
 /*
+ * Name of the level-2 kernel tls_select_tokens (staggered = 0: as in
+ * tls_select and tls_decode_step) or a resident engine's step (staggered !=
+ * 0, which keeps level 2 to half the SMs) takes for this shape, K_b and k,
+ * for 16-byte aligned codes and scales: "token_select_row_kernel",
+ * "token_select_cluster_kernel" or "token_select_kernel".  cluster_ctas and
+ * cta_threads (nullable, host) receive its CTAs per row (a thread-block
+ * cluster when more than one) and threads per CTA.  A static string owned by
+ * the library; NULL if the arguments are invalid (tls_last_error says why).
+ * Host only, no device work.
+ */
+TLS_API const char* tls_token_kernel(const tls_shape* shape, int32_t K_b, int32_t k, int32_t staggered,
+                                     int32_t* cluster_ctas, int32_t* cta_threads);
+
+/*
+ * Bytes of device workspace needed by tls_select_blocks, tls_select_tokens,/*
  * Bytes of device workspace needed by tls_select_blocks, tls_select_tokens,
  * tls_sparse_decode_attn and tls_decode_step for this shape, K_b and k.
  * The workspace must be zero-filled once after allocation; every call that

@@ -72,6 +72,30 @@ def test_attention_dispatch_names_the_kernel_per_shape(tls):
         tls.tls_attn_kernel(c2_shape(tls, n_q_heads=30))
 
 
+def test_level2_dispatch_names_the_kernel_per_workload(tls):
+    # narrow groups (G <= 16, 16/32 label channels, <= 8192 candidates): the row kernel, up to 4
+    # CTAs per row within two CTAs per SM, or one 1024-thread CTA per row when the resident
+    # stagger keeps level 2 to half the SMs; wide groups: 16-CTA clusters for few long rows
+    import synth
+    want = {"c1": (("token_select_row_kernel", 2, 512), ("token_select_row_kernel", 2, 512)),
+            "c2": (("token_select_row_kernel", 4, 512), ("token_select_row_kernel", 1, 1024)),
+            "c3": (("token_select_cluster_kernel", 16, 256), ("token_select_cluster_kernel", 16, 256)),
+            "c4": (("token_select_cluster_kernel", 16, 256), ("token_select_cluster_kernel", 16, 256)),
+            "c5": (("token_select_row_kernel", 2, 512), ("token_select_row_kernel", 1, 1024))}
+    for name, (sync, stag) in want.items():
+        c = synth.get_config(name)
+        shape = tls.make_shape(c.batch, c.n_q_heads, c.n_kv_heads, c.qk_dim, c.v_dim, c.v_offset, c.block_size,
+                               c.n_label, c.ctx_len, c.softmax_scale)
+        assert tls.tls_token_kernel(shape, c.K_b, c.k) == sync, name
+        assert tls.tls_token_kernel(shape, c.K_b, c.k, staggered=True) == stag, name
+    # label channels the tensor-core scorer does not take, or too many candidates for a row
+    assert tls.tls_token_kernel(c2_shape(tls, n_label=8), 64, 2048)[0] == "token_select_cluster_kernel"
+    assert tls.tls_token_kernel(c2_shape(tls), 256, 2048)[0] == "token_select_cluster_kernel"  # G*R*cand = 2^20
+    assert tls.tls_token_kernel(c2_shape(tls, n_label=32), 256, 2048)[0] == "token_select_kernel"  # 2^21
+    with pytest.raises(tls.TlsError):
+        tls.tls_token_kernel(c2_shape(tls), 64, 4097)  # k > K_b * bs
+
+
 def test_workspace_validation(tls):
     s = c2_shape(tls)
     a = tls.tls_workspace_bytes(s, 64, 2048)

@@ -165,6 +165,18 @@ extern "C" const char* tls_attn_kernel(const tls_shape* shape) {
   return "sparse_attn_kernel";
 }
 
+extern "C" const char* tls_token_kernel(const tls_shape* shape, int32_t K_b, int32_t k, int32_t staggered,
+                                        int32_t* cluster_ctas, int32_t* cta_threads) {
+  clear_error();
+  if (check_shape(shape) != TLS_OK) return nullptr;
+  WsLayout L;
+  if (plan_workspace(*shape, K_b, k, &L) != TLS_OK) return nullptr;
+  const TokenDispatch d = token_dispatch(*shape, K_b, staggered != 0, true);
+  if (cluster_ctas != nullptr) *cluster_ctas = d.cl;
+  if (cta_threads != nullptr) *cta_threads = d.threads;
+  return d.name;
+}
+
 extern "C" size_t tls_workspace_bytes(const tls_shape* shape, int32_t K_b, int32_t k) {
   if (check_shape(shape) != TLS_OK) return 0;
   WsLayout L;

@@ -71,6 +71,15 @@ constexpr int kNumSMs = 148;
 // may start before the preceding kernel of the stream ends; it calls
 // griddepcontrol.wait before reading that kernel's output) and optional
 // thread-block clusters of cluster_x CTAs along x (cluster_x <= 1: none).
+// The level-2 kernel a call takes (token_select.cu decides it).
+struct TokenDispatch {
+  enum Kind { kRow, kCluster, kChunked } kind;
+  const char* name;  // static string
+  int cl;            // CTAs per row (a cluster when > 1)
+  int threads;       // threads per CTA
+};
+TokenDispatch token_dispatch(const tls_shape& s, int K_b, bool lean, bool aligned);
+
 // cudaFuncSetAttribute once per kernel, device and value (the dynamic shared
 // memory limit only ever rises): a launch path that runs every decode step
 // should not pay the driver calls each time.

@@ -197,6 +197,23 @@ __global__ void __launch_bounds__(NT, NT >= 1024 || KPT > 8 ? 1 : 2) token_selec
   cta_topk_regs<NT, KPT>(keys, p.n_cand, p.k, p.token_idx + (int64_t)row * p.k, *ts, map);
 }
 
+// Which level-2 kernel a call takes, its CTAs per row and threads per CTA
+// (`lean` as in select_tokens_impl; `aligned`: codes and scales 16-byte
+// aligned).  The one place the choice is made.
+TokenDispatch token_dispatch(const tls_shape& s, int K_b, bool lean, bool aligned) {
+  const int rows = rows_of(s), g = group_of(s), n_cand = K_b * s.block_size;
+  if (aligned && token_row_kernel_fits(g, s.n_label, n_cand, s.block_size)) {
+    const int cl = token_row_cluster_size(rows, K_b, lean ? kNumSMs / 2 : 2 * kNumSMs);
+    // a row alone in its CTA gets 1024 threads: twice the warps to score it
+    const int nt = (cl == 1 && n_cand <= 8 * 1024) ? 1024 : kRowThreads;
+    return {TokenDispatch::kRow, "token_select_row_kernel", cl, nt};
+  }
+  const bool tc = g >= 16 && g <= 128 && (s.n_label == 16 || s.n_label == 32);
+  if (tc || token_cluster_fits(g, s.n_label, n_cand))
+    return {TokenDispatch::kCluster, "token_select_cluster_kernel", token_cluster_size(rows, n_cand, tc), kTokThreads};
+  return {TokenDispatch::kChunked, "token_select_kernel", 1, 256};
+}
+
 void fill_token_params(TokenParams& p, const tls_shape& s, const void* q, const int32_t* label_ch,
                        const uint8_t* codes, const float* scales, const int32_t* block_idx, int K_b, int k,
                        int32_t* token_idx, float* token_score, uint8_t* ws, const WsLayout& L) {
@@ -248,11 +265,10 @@ tls_status select_tokens_impl(const tls_shape& s, const void* q, const int32_t* 
   p.token_idx = token_idx;
 
   const size_t smem = (size_t)p.group * s.n_label * 4 + (size_t)p.n_cand * 4 + sizeof(TopkScratch) + 16;
-  if (token_row_kernel_fits(p.group, s.n_label, p.n_cand, s.block_size) &&
-      ((reinterpret_cast<uintptr_t>(codes) | reinterpret_cast<uintptr_t>(scales)) & 15u) == 0) {
-    const int cl = token_row_cluster_size(rows, K_b, lean ? kNumSMs / 2 : 2 * kNumSMs);
-    // a row alone in its CTA gets 1024 threads: twice the warps to score it
-    const int nt = (cl == 1 && p.n_cand <= 8 * 1024) ? 1024 : kRowThreads;
+  const TokenDispatch d = token_dispatch(
+      s, K_b, lean, ((reinterpret_cast<uintptr_t>(codes) | reinterpret_cast<uintptr_t>(scales)) & 15u) == 0);
+  if (d.kind == TokenDispatch::kRow) {
+    const int cl = d.cl, nt = d.threads;
     const int kpt = p.n_cand <= 2 * nt ? 2 : p.n_cand <= 4 * nt ? 4 : p.n_cand <= 8 * nt ? 8 : 16;
     const int bpc = (K_b + cl - 1) / cl;
     const size_t rsmem = (size_t)kpt * nt * 4 + (size_t)bpc * s.block_size * (s.n_label / 2 + 4) +
@@ -279,8 +295,8 @@ tls_status select_tokens_impl(const tls_shape& s, const void* q, const int32_t* 
   }
   // wide groups score on the tensor cores, which keeps any candidate count in one cluster
   const bool tc = p.group >= 16 && p.group <= 128 && (s.n_label == 16 || s.n_label == 32);
-  if (tc || token_cluster_fits(p.group, s.n_label, p.n_cand)) {
-    const int cl = token_cluster_size(rows, p.n_cand, tc);
+  if (d.kind == TokenDispatch::kCluster) {
+    const int cl = d.cl;
     const int per = (p.n_cand + cl - 1) / cl;
     const size_t cts_bytes = cl == 16 ? sizeof(ClusterTopkScratch<16>)
                              : cl == 8 ? sizeof(ClusterTopkScratch<8>)

@@ -76,6 +76,7 @@ _SIG = {
     "tls_last_error": (ctypes.c_char_p, []),
     "tls_version": (_I32, []),
     "tls_attn_kernel": (ctypes.c_char_p, [_P]),
+    "tls_token_kernel": (ctypes.c_char_p, [_P, _I32, _I32, _I32, _P, _P]),
     "tls_workspace_bytes": (_SZ, [_P, _I32, _I32]),
     "tls_workspace_error": (_I32, [_P, _I32, _P, _P]),
     "tls_build_block_meta": (_I32, [_P, _P, _I64, _I64, _I64, _P, _P]),
@@ -160,6 +161,16 @@ def tls_last_error() -> str:
 
 def tls_version() -> int:
     return lib().tls_version()
+
+
+def tls_token_kernel(shape: Shape, K_b: int, k: int, staggered: bool = False):
+    """(name, CTAs per row, threads per CTA) of the level-2 kernel for this shape, K_b and k;
+    staggered: as a resident engine's step launches it."""
+    cl, nt = ctypes.c_int32(), ctypes.c_int32()
+    r = lib().tls_token_kernel(ctypes.byref(shape), K_b, k, 1 if staggered else 0, ctypes.byref(cl), ctypes.byref(nt))
+    if r is None:
+        _check(TLS_ERR_INVALID_ARG, "tls_token_kernel")
+    return r.decode(), cl.value, nt.value
 
 
 def tls_attn_kernel(shape: Shape) -> str:
