@@ -120,6 +120,16 @@ def test_entry_points_reject_null_arguments_without_a_gpu(tls):
     with pytest.raises(tls.TlsError) as e:
         tls.tls_build_block_meta(s, None, 128, 0, 64, None, stream=0)
     assert e.value.status == tls.TLS_ERR_INVALID_ARG
+    # the engines: a NULL cache (offloaded form) or a NULL / non-dense view (resident form)
+    with pytest.raises(tls.TlsError) as e:
+        tls.tls_engine_create(s, 64, 2048, None, None, None, None, None, None, None, None, 0)
+    assert e.value.status == tls.TLS_ERR_INVALID_ARG
+    lib = tls.lib()
+    h = ctypes.c_void_p()
+    assert lib.tls_engine_create_resident(ctypes.byref(s), 64, 2048, None, None, None, None, None, None, None, None, 0,
+                                          ctypes.byref(h)) == tls.TLS_ERR_INVALID_ARG
+    assert b"NULL" in lib.tls_last_error()
+    assert tls.tls_engine_steps(None) == -1
 
 
 def _trajectory(nb, K_b, steps, seed):
