@@ -3,11 +3,20 @@
 // key channels quantised to INT4, then the top-K_t tokens).
 //
 // Candidates of a row are the bs tokens of each of its K_b chosen blocks, in
-// ascending token order.  A grid of (chunks, rows) CTAs scores them:
+// ascending token order, scored as
 //     score(t) = s_t * max_h sum_r qlab[h, r] * code_{t, r}
 // (s_t >= 0, so scaling after the max is the same as taking the max of the
-// scaled dots), writes the scores to the workspace, and the last CTA of each
-// row to finish runs the deterministic top-k over the row's scores.
+// scaled dots), then the deterministic top-k.  Three kernels, chosen by
+// token_dispatch:
+//   token_select_row_kernel      narrow groups (G <= 16, 16 or 32 label
+//                                channels, <= 8192 candidates): up to 4 CTAs
+//                                a row stage and score, the leader selects
+//   token_select_cluster_kernel  wider groups or other channel counts: a
+//                                cluster of 4 to 16 CTAs scores and selects
+//                                together over distributed shared memory
+//   token_select_kernel          the rest: a grid of (chunks, rows) CTAs
+//                                writes the scores to the workspace and the
+//                                last CTA of each row selects
 
 #include <cooperative_groups.h>
 #include <cstdlib>
@@ -18,8 +27,6 @@
 #include "token_common.cuh"
 
 namespace tls {
-
-
 
 template <int R, int NT>
 __global__ void __launch_bounds__(NT) token_select_kernel(TokenParams p) {
