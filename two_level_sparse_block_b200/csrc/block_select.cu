@@ -13,10 +13,15 @@
 //   warp 0 lane 0   TMA producer: 128 x 64 bf16 metadata tiles, 128B swizzle
 //   warp 1 lane 0   MMA issuer: tcgen05.mma kind::f16, fp32 accumulator in TMEM
 //   warps 2-3       build the Q' tile of each stage in the same swizzled layout
+//                   (for 64 padded heads or more a prep kernel writes Q' once
+//                   per step and warp 0 loads it by TMA as well)
 //   all warps       epilogue: tcgen05.ld one accumulator row per thread,
 //                   max over the G real heads -> agg[row, j]
-// The last CTA of a row to finish (atomic ticket in the workspace) runs the
-// deterministic top-K_b over the row's NB scores, read back from L2.
+// The deterministic top-K_b over the row's NB scores: a row of one tile is
+// selected by its CTA; the 2, 4 or 8 CTAs of a longer row form a cluster and
+// push their keys into the leader's shared memory, which selects; longer
+// rows go through the workspace, and the last CTA of the row to finish
+// (atomic ticket) selects from the scores read back from L2.
 //
 // Every mbarrier wait is bounded (2 s); on expiry the workspace error word
 // is set and the CTA skips the rest of its work, frees its TMEM and returns.
