@@ -126,7 +126,6 @@ TLS_API const char* tls_token_kernel(const tls_shape* shape, int32_t K_b, int32_
                                      int32_t* cluster_ctas, int32_t* cta_threads);
 
 /*
- * Bytes of device workspace needed by tls_select_blocks, tls_select_tokens,/*
  * Bytes of device workspace needed by tls_select_blocks, tls_select_tokens,
  * tls_sparse_decode_attn and tls_decode_step for this shape, K_b and k.
  * The workspace must be zero-filled once after allocation; every call that
@@ -142,6 +141,9 @@ TLS_API size_t tls_workspace_bytes(const tls_shape* shape, int32_t K_b, int32_t 
  * Reads (and, if clear != 0, zeroes) the workspace error word on `stream`,
  * synchronising that stream.  *code = 0 when no kernel reported an error;
  * otherwise a TLS_ERR_* value set by a kernel whose bounded wait ran out.
+ * ws = NULL reads the error word of tls_sparse_decode_attn_noalloc's fixed
+ * array on the current device instead (each call of that entry point clears
+ * it first, so it reports the last call's kernels).
  */
 TLS_API tls_status tls_workspace_error(const void* ws, int32_t clear, int32_t* code, void* stream);
 
@@ -250,11 +252,14 @@ TLS_API tls_status tls_decode_step(const tls_shape* shape, const void* q, const 
  * serving runtime that owns the whole HBM budget and offers no allocator, or
  * a latency-critical decode loop where cudaMalloc (which may synchronise the
  * device) is not allowed.
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *   - The first call in a device's CUDA context looks up the array's device
+ *     address (cudaGetSymbolAddress) with that device current and keeps it for
+ *     that device and context; make that first call before any stream
+ *     capture.  A context created later (e.g. after cudaDeviceReset) is looked
+ *     up again on its own first call.
  *   - Each call clears the error word and the tickets with cudaMemsetAsync on
  *     `stream`; it calls no cudaMalloc, cudaFree or allocating library routine.
+ *   - tls_workspace_error(NULL, ...) reads the error word of the last call.
  *   - All calls share the one array: two calls whose kernels overlap on the
  *     GPU (e.g. on different streams) race and give wrong results.  Issue them
  *     on one stream, or use tls_sparse_decode_attn with separate workspaces.
@@ -310,21 +315,29 @@ TLS_API tls_status tls_block_cache_plan(tls_block_cache* cache, const int32_t* n
 
 /*
  * Incremental prefetch (section 2.B): plans as tls_block_cache_plan, then
- * issues one cudaMemcpyAsync per copied run of blocks (K and V) from host
- * memory into the chosen slots on copy_stream, then updates the device slot
- * table on copy_stream: the first call writes the whole table, later calls
- * change only the entries of the copied and the evicted blocks (a small
- * kernel).  Neither touches a slot or an entry of in_use_block_idx_host, so
- * an attention reading those blocks may run concurrently.  The caller must
- * order copy_stream after every other kernel still reading a slot that may
- * be evicted (e.g. the attention of the step before).
+ * queues on copy_stream the copies of the planned blocks (K and V) from host
+ * memory into their slots -- one kernel that reads them from mapped pinned
+ * memory, or else one cudaMemcpyAsync per run of adjacent blocks -- and the
+ * slot-table update: the first call writes the whole table, later calls
+ * change only the entries of the copied and the evicted blocks.  Neither
+ * touches a slot or an entry of in_use_block_idx_host, so an attention
+ * reading those blocks may run concurrently.  The caller must order
+ * copy_stream after every other kernel still reading a slot that may be
+ * evicted (e.g. the attention of the step before).
+ * done_event: optional cudaEvent_t (as void*), recorded on copy_stream after
+ * the copies and the table update; a stream that makes the next attention
+ * waits on it (cudaStreamWaitEvent) before reading the new blocks.  NULL:
+ * the caller orders its work after copy_stream itself.
+ * The host mirror is updated only once all device work is queued.  A failure
+ * after some of it was queued marks the cache failed: that call and every
+ * later tls_prefetch_diff or tls_block_cache_plan return TLS_ERR_COPY.
  * *n_copied = blocks copied.  Setting the environment variable
  * TLS_FAULT_INJECT=copy makes the copy step fail with TLS_ERR_COPY before
  * anything is issued (host-side fault injection for tests).
  */
 TLS_API tls_status tls_prefetch_diff(tls_block_cache* cache, const int32_t* new_block_idx_host,
                              const int32_t* in_use_block_idx_host, int32_t K_b,
-                             void* copy_stream, int32_t* n_copied);
+                             void* copy_stream, void* done_event, int32_t* n_copied);
 
 /* Copies the host mirror of the slot table (int32 [B, Hkv, NB]) into `table`. */
 TLS_API tls_status tls_block_cache_table(const tls_block_cache* cache, int32_t* table);

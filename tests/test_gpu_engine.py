@@ -195,6 +195,54 @@ def test_engine_on_the_offload_workload_sampled_steps():
         layer.close()
 
 
+def test_engine_on_the_36_layer_workload_sampled_steps():
+    # c5's layer shape (batch 16, 32:8 heads, 122880 tokens, K_b 96, k 3072)
+    # behind the offload engine with its 2 * K_b slots per row (24576 in all):
+    # three steps of the trajectory, sampled rows against the staggered oracle
+    runtime, tls = _rt()
+    cfg = synth.get_config("c5")
+    qs = synth.gen_query_trajectory(cfg, 3)
+    K, V, _ = synth.gen_kv(cfg, qs[0])
+    lab = synth.gen_label_channels(cfg)
+    layer = runtime.offloaded_layer_for_config(cfg, K, V, lab)
+    g = cfg.group
+    try:
+        for t, q in enumerate(qs):
+            layer.step(_dev_q(q))
+            torch.cuda.synchronize()
+            assert layer.check_device_error() == 0
+            m_prev = layer.block_idx[(t + 1) & 1].cpu().numpy()
+            m_cur = layer.block_idx[t & 1].cpu().numpy()
+            tok = layer.token_idx.cpu().numpy()
+            out = layer.out.float().cpu().numpy()
+            for b, h in _rows(cfg, 3):
+                where = f"c5 step {t} row ({b},{h})"
+                r1 = _orow(cfg, q, K, V, lab, b, h)
+                check_selection(m_cur[b, h], r1["agg"], cfg.K_b, where + " M_t")
+                r2 = _orow(cfg, q, K, V, lab, b, h, block_idx=m_prev[b, h])
+                pos = np.searchsorted(r2["cand"], tok[b, h])
+                assert np.array_equal(r2["cand"][pos], tok[b, h]), where + ": token outside M_t-1"
+                check_selection(pos, r2["token_score"], cfg.k, where + " tokens")
+                r3 = _orow(cfg, q, K, V, lab, b, h, block_idx=m_prev[b, h], token_idx=tok[b, h])
+                check_output(out[b, h * g:(h + 1) * g], r3["out"], where + " out")
+        assert layer.stats(-1).n_copied == cfg.rows * cfg.K_b
+        assert all(0 <= layer.stats(t).n_copied <= cfg.rows * cfg.K_b for t in range(len(qs) - 1))
+        # the slot table agrees with the host mirror, and sampled slots hold their blocks
+        table = layer.slot_table.cpu().numpy()
+        mirror = np.empty_like(table)
+        tls.tls_block_cache_table(layer.cache, mirror)
+        assert np.array_equal(table, mirror)
+        last = layer.block_idx[(len(qs) - 1) & 1].cpu().numpy()
+        bs = cfg.block_size
+        for b, h in _rows(cfg, 3):
+            for blk in last[b, h][:: 17]:
+                s = int(table[b, h, blk])
+                got = layer.slot_k[s].view(torch.int16).cpu().numpy().view(np.uint16)
+                assert s >= 0 and np.array_equal(got, K[b, h, blk * bs:(blk + 1) * bs])
+    finally:
+        layer.close()
+
+
 # ---------------------------------------------------------------------------
 # resident engine: the same stagger over HBM-resident K/V, no transfers
 # ---------------------------------------------------------------------------
@@ -312,3 +360,60 @@ def test_resident_engine_on_the_headline_workload_sampled_rows():
                 check_output(out[b, h * g:(h + 1) * g], r3["out"], where + " out")
     finally:
         eng.close()
+
+
+def test_prefetch_diff_records_its_done_event():
+    # the plain C call: plan T_t = M_t \ C_t, queue the copies on a copy stream
+    # and record the caller's event after them; work ordered after the event
+    # sees every block of M_t in its slot (three rounds, the last one evicting)
+    runtime, tls = _rt()
+    cfg = ENGINE[2]
+    q = synth.gen_queries(cfg)
+    K, V, _ = synth.gen_kv(cfg, q)
+    rows, nb, bs, K_b = cfg.rows, cfg.n_blocks, cfg.block_size, cfg.K_b
+    n_slots = 2 * rows * K_b
+    host_k = torch.from_numpy(np.ascontiguousarray(K).view(np.int16)).pin_memory()
+    host_v = torch.from_numpy(np.ascontiguousarray(V).view(np.int16)).pin_memory()
+    slot_k = torch.zeros((n_slots, bs, cfg.qk_dim), dtype=torch.bfloat16, device="cuda")
+    slot_v = torch.zeros((n_slots, bs, cfg.v_dim), dtype=torch.bfloat16, device="cuda")
+    table = torch.full((cfg.batch, cfg.n_kv_heads, nb), -1, dtype=torch.int32, device="cuda")
+    shape = tls.make_shape(cfg.batch, cfg.n_q_heads, cfg.n_kv_heads, cfg.qk_dim, cfg.v_dim, -1, bs, cfg.n_label,
+                           cfg.ctx_len, cfg.softmax_scale)
+    cache = tls.tls_block_cache_create(shape, host_k, host_v, cfg.qk_dim, cfg.v_dim, n_slots, slot_k, slot_v, table)
+    rng = np.random.default_rng(7)
+    copy_stream = torch.cuda.Stream()
+    try:
+        prev = None
+        resident = np.zeros((cfg.batch, cfg.n_kv_heads, nb), dtype=bool)
+        evicted = 0
+        for rnd in range(3):
+            m = np.stack([np.sort(rng.choice(nb, K_b, replace=False)) for _ in range(rows)]).astype(np.int32)
+            m = m.reshape(cfg.batch, cfg.n_kv_heads, K_b)
+            done = torch.cuda.Event()
+            done.record(copy_stream)  # the event exists before the library records it
+            n = tls.tls_prefetch_diff(cache, m, prev, K_b, copy_stream, done)
+            torch.cuda.current_stream().wait_event(done)
+            tab = table.cpu().numpy()  # ordered after the event on the current stream
+            sk = slot_k.view(torch.int16).cpu().numpy().view(np.uint16)
+            sv = slot_v.view(torch.int16).cpu().numpy().view(np.uint16)
+            # |T_t| = |M_t \ C_t| summed over rows, C_t = the blocks resident before the call
+            want = sum(len(oracle.plan_transfer(m[b, h], np.flatnonzero(resident[b, h])))
+                       for b in range(cfg.batch) for h in range(cfg.n_kv_heads))
+            assert n == want
+            now = tab >= 0
+            evicted += int(np.count_nonzero(resident & ~now))
+            resident = now
+            for b in range(cfg.batch):
+                for h in range(cfg.n_kv_heads):
+                    if prev is not None:
+                        assert np.all(tab[b, h, prev[b, h]] >= 0), "a block of M_t-1 was evicted"
+                    for blk in m[b, h]:
+                        sl = tab[b, h, blk]
+                        assert sl >= 0
+                        assert np.array_equal(sk[sl], K[b, h, blk * bs:(blk + 1) * bs])
+                        assert np.array_equal(sv[sl], V[b, h, blk * bs:(blk + 1) * bs])
+            prev = m
+        assert evicted > 0, "the workload lost its construction: nothing was evicted"
+    finally:
+        torch.cuda.synchronize()
+        tls.tls_block_cache_destroy(cache)

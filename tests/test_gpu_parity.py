@@ -35,7 +35,7 @@ def _rt():
     return runtime, tls
 
 
-@functools.lru_cache(maxsize=4)
+@functools.lru_cache(maxsize=2)
 def gen_case(cfg):
     q = synth.gen_queries(cfg)
     K, V, planted = synth.gen_kv(cfg, q)
@@ -66,7 +66,9 @@ SMALL = [
     small("s_k_eq_1", K_b=1, k=1, seed=17),
     small("s_all", ctx_len=512, K_b=32, k=512, seed=18),
 ]
-FULL = [get_config(c) for c in ("c1", "c2", "c3", "c4")]
+FULL = [get_config(c) for c in ("c1", "c2", "c3", "c4", "c5")]
+# rows the oracle checks per full-size workload (the first and last among them)
+FULL_ROWS = {"c1": 1, "c2": 8, "c3": 4, "c4": 1, "c5": 6}
 # row counts that send the 128-wide attention to its cluster form (16, 8, 4
 # and 2 CTAs per row); ragged lists, idle CTAs, and a 64-head group split into
 # four virtual rows of 16 heads
@@ -189,7 +191,7 @@ def test_cluster_attention_sampled_rows(cfg):
 def test_full_size_sampled_rows(cfg):
     st, data = make_state(cfg)
     got = run_stages(st)
-    for b, h in sample_rows(cfg):
+    for b, h in sample_rows(cfg, FULL_ROWS[cfg.name[:2]]):
         check_row(cfg, data, got, st, b, h)
     # the fused step gives the same lists and outputs as the three calls
     st.step()
@@ -442,3 +444,50 @@ def test_decode_step_equals_select_then_attend(cfg):
     assert np.array_equal(st.token_idx.cpu().numpy(), got["token_idx"])
     assert np.array_equal(st.out.float().cpu().numpy(), got["out"])
     assert np.array_equal(st.lse.cpu().numpy(), got["lse"])
+
+
+# more virtual rows than two CTAs per SM hold in clusters: the persistent
+# attention (contiguous ranges of 16-token chunks, ticket merge through the
+# workspace), with rows split across CTAs and CTAs spanning rows
+PERSISTENT = [
+    small("s_persist_g4", batch=80, n_q_heads=8, n_kv_heads=2, ctx_len=1024, K_b=9, k=133, seed=51),
+    small("s_persist_g64", batch=40, n_q_heads=64, n_kv_heads=1, ctx_len=1024, K_b=10, k=150, seed=52),
+]
+
+
+@pytest.mark.parametrize("cfg", PERSISTENT, ids=lambda c: c.name)
+def test_persistent_attention_sampled_rows(cfg):
+    runtime, tls = _rt()
+    st, data = make_state(cfg)
+    assert tls.tls_attn_kernel(st.shape) == "sparse_attn_mma_kernel"
+    got = run_stages(st)
+    for b, h in sample_rows(cfg, 8):
+        check_row(cfg, data, got, st, b, h)
+    # and once more through the fused step: the tickets reset after every call
+    st.out.fill_(float("nan"))
+    st.step()
+    torch.cuda.synchronize()
+    assert st.check_device_error() == 0
+    assert np.array_equal(st.out.float().cpu().numpy(), got["out"])
+
+
+# level-2 work too heavy for one cluster on the CUDA cores (G * R * candidates
+# above 2^20, label channels the tensor-core scorer does not take): scores go
+# to the workspace and the last CTA of each row selects
+CHUNKED = [
+    small("s_chunked_r64", batch=2, n_q_heads=16, n_kv_heads=2, ctx_len=8192, block_size=64, K_b=64, k=1500,
+          n_label=64, seed=53),
+    small("s_chunked_r8_g32", batch=1, n_q_heads=64, n_kv_heads=2, ctx_len=16384, block_size=64, K_b=128, k=3000,
+          n_label=8, seed=54),
+]
+
+
+@pytest.mark.parametrize("cfg", CHUNKED, ids=lambda c: c.name)
+def test_chunked_level2_all_rows(cfg):
+    runtime, tls = _rt()
+    st, data = make_state(cfg)
+    assert tls.tls_token_kernel(st.shape, cfg.K_b, cfg.k)[0] == "token_select_kernel"
+    got = run_stages(st)
+    for b in range(cfg.batch):
+        for h in range(cfg.n_kv_heads):
+            check_row(cfg, data, got, st, b, h)

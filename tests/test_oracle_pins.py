@@ -151,6 +151,16 @@ def test_int4_worked_example():
     assert oracle.unpack_codes(oracle.pack_codes(codes)).tolist() == codes.tolist()
 
 
+def test_int4_exact_halves_round_to_even():
+    # x / s lands exactly on n + 1/2 for seven of the eight channels: the codes
+    # pin the tie rule (half to even), which no random input exercises
+    g = GOLD["int4_ties"]
+    kb = bits([g["x"]])
+    codes, scales = oracle.quant_label(kb, np.arange(len(g["x"])))
+    assert scales[0] == np.float32(g["scale"])
+    assert codes[0].tolist() == g["codes"]
+
+
 def test_int4_round_trip_within_half_step():
     rng = np.random.default_rng(3)
     kb = rand_bits(rng, (2000, 40), 5.0)

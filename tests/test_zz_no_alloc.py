@@ -57,6 +57,8 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(tls, name):
         check_output(out.cpu().numpy(), ref_out.cpu().numpy(), f"{name} noalloc out")
         assert np.max(np.abs(lse.cpu().numpy() - ref_lse.cpu().numpy())) <= 1e-4 * max(1.0, float(ref_lse.abs().max()))
         assert torch.equal(out, ref_out)
+        # the array's error word (read through tls_workspace_error with no workspace) stays clear
+        assert tls.tls_workspace_error(None) == 0
 
 
 def test_noalloc_rejects_scratch_beyond_its_array(tls):

@@ -186,7 +186,14 @@ extern "C" size_t tls_workspace_bytes(const tls_shape* shape, int32_t K_b, int32
 
 extern "C" tls_status tls_workspace_error(const void* ws, int32_t clear, int32_t* code, void* stream) {
   clear_error();
-  if (ws == nullptr || code == nullptr) return fail(TLS_ERR_INVALID_ARG, "workspace_error: NULL argument");
+  if (code == nullptr) return fail(TLS_ERR_INVALID_ARG, "workspace_error: NULL code");
+  if (ws == nullptr) {
+    // the scratch-free attention's array on the current device
+    void* base = nullptr;
+    tls_status st = noalloc_scratch(&base);
+    if (st != TLS_OK) return st;
+    ws = base;
+  }
   int32_t words[2] = {0, 0};
   cudaStream_t cs = (cudaStream_t)stream;
   tls_status st = cuda_check(cudaMemcpyAsync(words, ws, sizeof(words), cudaMemcpyDeviceToHost, cs),

@@ -37,12 +37,15 @@ struct tls_block_cache {
   cudaEvent_t staged[2] = {nullptr, nullptr};
   int cur = 0;
   bool published = false;                     // the device table has been written once
-  std::vector<int2> changes;                  // this plan's (entry, value) table changes
   // Pull path: when K/V are pinned host memory mapped into the device address
   // space, one kernel reads the planned blocks over PCIe into their slots.
   const uint8_t* dev_host_k = nullptr;        // device addresses of host_k / host_v
   const uint8_t* dev_host_v = nullptr;
   int4* jobs[2] = {nullptr, nullptr};         // pinned, mapped: {tok0 lo, tok0 hi, slot, 0} per copy
+  // set when a transfer failed after some of its device work was queued: the
+  // slots may no longer hold what the host mirror says, so every later
+  // transfer or plan returns this status
+  tls_status failed = TLS_OK;
 };
 
 namespace tls {
@@ -120,21 +123,29 @@ tls_status plan(const tls_block_cache& c, const int32_t* new_idx, const int32_t*
   return TLS_OK;
 }
 
-void commit(tls_block_cache& c, const int32_t* new_idx, int K_b, std::vector<Copy>& copies,
-            const std::vector<int32_t>& victims) {
-  c.step += 1;
-  c.changes.clear();
+// The slot-table changes a plan makes, as (entry, value) pairs, without
+// changing the cache: each copied block's entry gets its victim slot, and the
+// block a victim held (if any) loses its entry.  The new blocks are not
+// resident and the evicted ones are, so no entry appears twice.
+void assign_slots(const tls_block_cache& c, std::vector<Copy>& copies, const std::vector<int32_t>& victims,
+                  std::vector<int2>* changes) {
+  changes->clear();
   for (size_t i = 0; i < copies.size(); ++i) {
     const int32_t s = victims[i];
-    if (c.owner[s] >= 0) {
-      c.table[c.owner[s]] = -1;
-      c.changes.push_back(make_int2((int)c.owner[s], -1));
-    }
-    const int64_t key = (int64_t)copies[i].row * c.nb + copies[i].block;
-    c.owner[s] = key;
-    c.table[key] = s;
-    c.changes.push_back(make_int2((int)key, s));
+    if (c.owner[s] >= 0) changes->push_back(make_int2((int)c.owner[s], -1));
+    changes->push_back(make_int2((int)((int64_t)copies[i].row * c.nb + copies[i].block), s));
     copies[i].slot = s;
+  }
+}
+
+// Applies a plan to the host mirror (after its device work was queued).
+void commit(tls_block_cache& c, const int32_t* new_idx, int K_b, const std::vector<Copy>& copies) {
+  c.step += 1;
+  for (const Copy& cp : copies) {
+    if (c.owner[cp.slot] >= 0) c.table[c.owner[cp.slot]] = -1;
+    const int64_t key = (int64_t)cp.row * c.nb + cp.block;
+    c.owner[cp.slot] = key;
+    c.table[key] = cp.slot;
   }
   for (int r = 0; r < c.rows; ++r)
     for (int i = 0; i < K_b; ++i) {
@@ -199,12 +210,15 @@ __global__ void slot_table_update_kernel(int32_t* table, const int2* pairs, int 
 // block copies.
 tls_status prefetch_diff_impl(tls_block_cache* c, const int32_t* new_idx, const int32_t* in_use, int K_b,
                               cudaStream_t cs, int32_t* n_copied, int64_t* bytes) {
+  if (c->failed != TLS_OK)
+    return fail(c->failed, "prefetch_diff: an earlier transfer failed; the slots no longer match the host mirror");
   if (fault_injected_copy()) return fail(TLS_ERR_COPY, "prefetch_diff: copy failure injected (TLS_FAULT_INJECT=copy)");
   std::vector<Copy> copies;
   std::vector<int32_t> victims;
   tls_status st = plan(*c, new_idx, in_use, K_b, &copies, &victims);
   if (st != TLS_OK) return st;
-  commit(*c, new_idx, K_b, copies, victims);
+  std::vector<int2> changes;
+  assign_slots(*c, copies, victims, &changes);
 
   const int bs = c->shape.block_size;
   const int64_t n = c->shape.ctx_len;
@@ -213,15 +227,20 @@ tls_status prefetch_diff_impl(tls_block_cache* c, const int32_t* new_idx, const 
   const int b = c->cur;
   cudaError_t e = cudaEventSynchronize(c->staged[b]);  // the staging buffers' previous use is done
   if (e != cudaSuccess) return cuda_check(e, "prefetch_diff: staging wait");
+  // from here on device work is queued: a failure leaves the cache failed
+  auto queue_failed = [&](const char* what, cudaError_t err) {
+    c->failed = TLS_ERR_COPY;
+    return fail(TLS_ERR_COPY, "prefetch_diff: %s: %s", what, cudaGetErrorString(err));
+  };
   // the first transfer publishes the whole table (nothing is resident, so nothing reads it)
   const bool first = !c->published;
   if (first) {
     std::memcpy(c->staging[b], c->table.data(), c->table.size() * sizeof(int32_t));
+    for (const int2& ch : changes) c->staging[b][ch.x] = ch.y;
     e = cudaMemcpyAsync(c->table_dev, c->staging[b], c->table.size() * sizeof(int32_t), cudaMemcpyHostToDevice, cs);
-    if (e != cudaSuccess) return fail(TLS_ERR_COPY, "prefetch_diff: slot table copy failed: %s", cudaGetErrorString(e));
-    c->published = true;
+    if (e != cudaSuccess) return queue_failed("slot table copy failed", e);
   }
-  const int n_pairs = first ? 0 : (int)c->changes.size();
+  const int n_pairs = first ? 0 : (int)changes.size();
   if (c->dev_host_k != nullptr) {
     // one kernel pulls every planned block over PCIe and applies the table changes
     int4* jobs = c->jobs[b];
@@ -230,7 +249,7 @@ tls_status prefetch_diff_impl(tls_block_cache* c, const int32_t* new_idx, const 
       jobs[i] = make_int4((int)(uint32_t)(tok0 & 0xFFFFFFFF), (int)(tok0 >> 32), copies[i].slot, 0);
     }
     int2* pairs = first ? nullptr : reinterpret_cast<int2*>(c->staging[b]);
-    if (pairs != nullptr) std::memcpy(pairs, c->changes.data(), (size_t)n_pairs * sizeof(int2));
+    if (pairs != nullptr) std::memcpy(pairs, changes.data(), (size_t)n_pairs * sizeof(int2));
     const int grid = copies.empty() ? 1 : (int)copies.size();
     if (!copies.empty() || n_pairs > 0) {
       block_pull_kernel<<<grid, kPullThreads, 0, cs>>>(c->dev_host_k, with_v ? c->dev_host_v : nullptr, c->slot_k,
@@ -238,7 +257,7 @@ tls_status prefetch_diff_impl(tls_block_cache* c, const int32_t* new_idx, const 
                                                         c->hk_stride * 2, c->hv_stride * 2, jobs,
                                                         (int)copies.size(), c->table_dev, pairs, n_pairs);
       e = cudaGetLastError();
-      if (e != cudaSuccess) return fail(TLS_ERR_COPY, "prefetch_diff: pull kernel launch failed: %s", cudaGetErrorString(e));
+      if (e != cudaSuccess) return queue_failed("pull kernel launch failed", e);
     }
   } else {
     // one cudaMemcpyAsync per run of blocks adjacent in host memory and in the pool
@@ -255,19 +274,22 @@ tls_status prefetch_diff_impl(tls_block_cache* c, const int32_t* new_idx, const 
       if (e == cudaSuccess && with_v)
         e = cudaMemcpyAsync(c->slot_v + (size_t)copies[i].slot * vblk, c->host_v + (size_t)tok0 * c->hv_stride * 2,
                             len * vblk, cudaMemcpyHostToDevice, cs);
-      if (e != cudaSuccess) return fail(TLS_ERR_COPY, "prefetch_diff: block copy failed: %s", cudaGetErrorString(e));
+      if (e != cudaSuccess) return queue_failed("block copy failed", e);
       i = j;
     }
     if (n_pairs > 0) {
       int2* pairs = reinterpret_cast<int2*>(c->staging[b]);
-      std::memcpy(pairs, c->changes.data(), (size_t)n_pairs * sizeof(int2));
+      std::memcpy(pairs, changes.data(), (size_t)n_pairs * sizeof(int2));
       slot_table_update_kernel<<<(n_pairs + 255) / 256, 256, 0, cs>>>(c->table_dev, pairs, n_pairs);
       e = cudaGetLastError();
-      if (e != cudaSuccess) return fail(TLS_ERR_COPY, "prefetch_diff: table update launch failed: %s", cudaGetErrorString(e));
+      if (e != cudaSuccess) return queue_failed("table update launch failed", e);
     }
   }
   e = cudaEventRecord(c->staged[b], cs);
-  if (e != cudaSuccess) return cuda_check(e, "prefetch_diff: staging event");
+  if (e != cudaSuccess) return queue_failed("staging event", e);
+  // everything is queued: the host mirror follows
+  if (first) c->published = true;
+  commit(*c, new_idx, K_b, copies);
   c->cur ^= 1;
   *n_copied = (int32_t)copies.size();
   if (bytes != nullptr) *bytes = (int64_t)copies.size() * (int64_t)(kblk + (with_v ? vblk : 0));
@@ -379,11 +401,15 @@ extern "C" tls_status tls_block_cache_plan(tls_block_cache* c, const int32_t* ne
   if (c == nullptr || new_block_idx == nullptr || n_copy == nullptr)
     return fail(TLS_ERR_INVALID_ARG, "block_cache_plan: NULL argument");
   if (K_b < 1 || K_b > c->nb) return fail(TLS_ERR_INVALID_ARG, "block_cache_plan: K_b out of range");
+  if (c->failed != TLS_OK)
+    return fail(c->failed, "block_cache_plan: an earlier transfer failed; the slots no longer match the host mirror");
   std::vector<Copy> copies;
   std::vector<int32_t> victims;
   tls_status st = plan(*c, new_block_idx, in_use_block_idx, K_b, &copies, &victims);
   if (st != TLS_OK) return st;
-  commit(*c, new_block_idx, K_b, copies, victims);
+  std::vector<int2> changes;
+  assign_slots(*c, copies, victims, &changes);
+  commit(*c, new_block_idx, K_b, copies);
   for (size_t i = 0; i < copies.size(); ++i) {
     if (copy_row) copy_row[i] = copies[i].row;
     if (copy_block) copy_block[i] = copies[i].block;
@@ -395,15 +421,18 @@ extern "C" tls_status tls_block_cache_plan(tls_block_cache* c, const int32_t* ne
 
 extern "C" tls_status tls_prefetch_diff(tls_block_cache* c, const int32_t* new_block_idx_host,
                                         const int32_t* in_use_block_idx_host, int32_t K_b, void* copy_stream,
-                                        int32_t* n_copied) {
+                                        void* done_event, int32_t* n_copied) {
   clear_error();
   if (c == nullptr || new_block_idx_host == nullptr || n_copied == nullptr)
     return fail(TLS_ERR_INVALID_ARG, "prefetch_diff: NULL argument");
   if (c->host_k == nullptr || c->slot_k == nullptr || c->table_dev == nullptr)
     return fail(TLS_ERR_INVALID_ARG, "prefetch_diff: cache was created without device buffers");
   if (K_b < 1 || K_b > c->nb) return fail(TLS_ERR_INVALID_ARG, "prefetch_diff: K_b out of range");
-  return prefetch_diff_impl(c, new_block_idx_host, in_use_block_idx_host, K_b, (cudaStream_t)copy_stream, n_copied,
-                            nullptr);
+  tls_status st = prefetch_diff_impl(c, new_block_idx_host, in_use_block_idx_host, K_b, (cudaStream_t)copy_stream,
+                                     n_copied, nullptr);
+  if (st != TLS_OK || done_event == nullptr) return st;
+  cudaError_t e = cudaEventRecord((cudaEvent_t)done_event, (cudaStream_t)copy_stream);
+  return e == cudaSuccess ? TLS_OK : cuda_check(e, "prefetch_diff: done event");
 }
 
 extern "C" tls_status tls_block_cache_table(const tls_block_cache* c, int32_t* table) {

@@ -29,8 +29,6 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
-#include <cstdlib>
-#include <cstring>
 #include <mutex>
 
 #include <cooperative_groups.h>
@@ -295,53 +293,6 @@ __global__ void __launch_bounds__(128, 1)
   }
 }
 
-// CUDA-core variant of the same scores (diagnostic; selected with
-// TLS_BLOCK_SCORE_KERNEL=simt).  One thread per block, Q' in shared memory.
-__global__ void __launch_bounds__(128) block_score_simt_kernel(const uint16_t* __restrict__ meta, BlockScoreParams p) {
-  extern __shared__ float qs[];  // [G][2*dqk] as float, then select scratch
-  const int tid = threadIdx.x;
-  const int row = blockIdx.y;
-  const int g = p.group, k2 = 2 * p.dqk;
-  const int b = row / p.n_kv_heads, kvh = row % p.n_kv_heads;
-  const uint16_t* qg = p.q + ((int64_t)b * p.n_q_heads + (int64_t)kvh * g) * p.dqk;
-  for (int i = tid; i < g * k2; i += 128) {
-    const int h = i / k2, e = i % k2;
-    const float x = __uint_as_float((uint32_t)qg[(int64_t)h * p.dqk + (e < p.dqk ? e : e - p.dqk)] << 16);
-    qs[i] = e < p.dqk ? fmaxf(x, 0.0f) : fminf(x, 0.0f);
-  }
-  __syncthreads();
-  const int j = blockIdx.x * 128 + tid;
-  if (j < p.nb) {
-    const uint16_t* m = meta + ((int64_t)row * p.nb + j) * k2;
-    float best = -INFINITY;
-    for (int h = 0; h < g; ++h) {
-      float acc = 0.0f;
-      for (int e = 0; e < k2; e += 8) {
-        float f[8];
-        unpack8(*reinterpret_cast<const uint4*>(m + e), f);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc = fmaf(qs[h * k2 + e + i], f[i], acc);
-      }
-      best = fmaxf(best, acc);
-    }
-    p.agg[(int64_t)row * p.nb + j] = best;
-    if (p.block_score != nullptr) p.block_score[(int64_t)row * p.nb + j] = best;
-  }
-  __threadfence();
-  __syncthreads();
-  __shared__ int last;
-  if (tid == 0) last = atomicInc(&p.counters[row], gridDim.x - 1) == gridDim.x - 1;
-  __syncthreads();
-  if (!last) return;
-  __threadfence();
-  uint32_t* keys = reinterpret_cast<uint32_t*>(qs + (size_t)g * k2);
-  TopkScratch* ts = reinterpret_cast<TopkScratch*>(keys + p.nb);
-  const float* arow = p.agg + (int64_t)row * p.nb;
-  for (int i = tid; i < p.nb; i += 128) keys[i] = float_key(__ldcg(arow + i));
-  __syncthreads();
-  cta_topk_ascending<128>(keys, p.nb, p.K_b, p.block_idx + (int64_t)row * p.K_b, *ts, [](int i) { return i; });
-}
-
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
@@ -360,14 +311,6 @@ tls_status get_encoder() {
   });
   if (g_encode == nullptr) return fail(TLS_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   return TLS_OK;
-}
-
-bool use_simt() {
-  static const bool v = [] {
-    const char* e = std::getenv("TLS_BLOCK_SCORE_KERNEL");
-    return e != nullptr && std::strcmp(e, "simt") == 0;
-  }();
-  return v;
 }
 
 template <int NPAD, int CL>
@@ -419,15 +362,6 @@ tls_status select_blocks_impl(const tls_shape& s, const void* q, const void* met
   p.counters = reinterpret_cast<unsigned*>(ws + L.blk_counter);
   p.block_idx = block_idx;
   p.err = reinterpret_cast<int*>(ws + L.err);
-
-  if (use_simt()) {
-    const size_t smem = (size_t)p.group * 2 * s.qk_dim * 4 + (size_t)nb * 4 + sizeof(TopkScratch) + 16;
-    cudaError_t e = kernel_attrs((const void*)block_score_simt_kernel, smem);
-    if (e != cudaSuccess) return cuda_check(e, "select_blocks: set smem attribute");
-    dim3 grid((unsigned)((nb + 127) / 128), (unsigned)rows);
-    block_score_simt_kernel<<<grid, 128, smem, stream>>>((const uint16_t*)meta, p);
-    return launch_check("select_blocks: block_score_simt launch");
-  }
 
   tls_status st = get_encoder();
   if (st != TLS_OK) return st;

@@ -11,6 +11,8 @@
 // by log-sum-exp and writes the output (fp32 or bf16) and the natural-log lse.
 
 #include <mutex>
+#include <utility>
+#include <vector>
 
 #include "attn_common.cuh"
 #include "device_common.cuh"
@@ -309,28 +311,55 @@ int attn_heads_per_cta(const tls_shape& s) {
 static __device__ __align__(256) unsigned char g_attn_scratch[TLS_NOALLOC_SCRATCH_BYTES];
 
 namespace {
-constexpr int kMaxDevices = 64;
+// The array's device address, looked up once per (device, CUDA context): a
+// context created anew (the primary context after cudaDeviceReset, or a
+// context of the caller's own) loads the module again at another address.
+struct ScratchKey {
+  int dev;
+  void* ctx;
+};
 std::mutex g_scratch_mu;
-void* g_scratch_ptr[kMaxDevices] = {nullptr};
+std::vector<std::pair<ScratchKey, void*>> g_scratch_ptr;
+using CtxGetCurrentFn = int (*)(void**);
+CtxGetCurrentFn g_ctx_current = nullptr;
+std::once_flag g_ctx_once;
 }  // namespace
 
-static tls_status scratch_address(void** out) {
+namespace tls {
+tls_status noalloc_scratch(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return tls::cuda_check(e, "sparse_decode_attn_noalloc: cudaGetDevice");
-  if (dev < 0 || dev >= kMaxDevices) return tls::fail(TLS_ERR_UNSUPPORTED, "sparse_decode_attn_noalloc: device id %d", dev);
+  if (e != cudaSuccess) return cuda_check(e, "sparse_decode_attn_noalloc: cudaGetDevice");
+  std::call_once(g_ctx_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_current = reinterpret_cast<CtxGetCurrentFn>(fn);
+  });
+  if (g_ctx_current == nullptr) return fail(TLS_ERR_CUDA, "sparse_decode_attn_noalloc: cuCtxGetCurrent unavailable");
+  void* ctx = nullptr;
+  if (g_ctx_current(&ctx) != 0) return fail(TLS_ERR_CUDA, "sparse_decode_attn_noalloc: cuCtxGetCurrent failed");
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_attn_scratch);
-    if (e != cudaSuccess || p == nullptr)
-      return tls::cuda_check(e != cudaSuccess ? e : cudaErrorInvalidSymbol,
-                             "sparse_decode_attn_noalloc: cudaGetSymbolAddress");
-    g_scratch_ptr[dev] = p;
-  }
-  *out = g_scratch_ptr[dev];
+  if (ctx != nullptr)
+    for (auto& kv : g_scratch_ptr)
+      if (kv.first.dev == dev && kv.first.ctx == ctx) {
+        *out = kv.second;
+        return TLS_OK;
+      }
+  // the lookup also makes the device's primary context current when no
+  // context was; the context it ran in keys the cached address
+  void* p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_attn_scratch);
+  if (e != cudaSuccess || p == nullptr)
+    return cuda_check(e != cudaSuccess ? e : cudaErrorInvalidSymbol, "sparse_decode_attn_noalloc: cudaGetSymbolAddress");
+  if (g_ctx_current(&ctx) != 0 || ctx == nullptr)
+    return fail(TLS_ERR_CUDA, "sparse_decode_attn_noalloc: no current context after the lookup");
+  g_scratch_ptr.push_back({ScratchKey{dev, ctx}, p});
+  *out = p;
   return TLS_OK;
 }
+}  // namespace tls
 
 extern "C" tls_status tls_sparse_decode_attn_noalloc(const tls_shape* shape, const void* q, const tls_kv_view* kv,
                                                      const int32_t* token_idx, int32_t k, int32_t out_dtype,
@@ -368,7 +397,7 @@ extern "C" tls_status tls_sparse_decode_attn_noalloc(const tls_shape* shape, con
                 "array; use tls_sparse_decode_attn with a workspace",
                 header + ticket_bytes + partial_bytes, (unsigned)TLS_NOALLOC_SCRATCH_BYTES);
   void* base = nullptr;
-  st = scratch_address(&base);
+  st = noalloc_scratch(&base);
   if (st != TLS_OK) return st;
   // the array keeps the previous call's contents: error word and tickets must start at zero
   cudaError_t e = cudaMemsetAsync(base, 0, header + ticket_bytes, (cudaStream_t)stream);

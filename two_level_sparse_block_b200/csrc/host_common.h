@@ -58,6 +58,10 @@ struct WsLayout {
   int tiles_per_pair, n_items, n_ctas;  // mma attention: chunks per (virtual) row, items, persistent CTAs
 };
 
+// Device address of the scratch-free entry point's static array on the
+// current device and context (looked up once per device and context).
+tls_status noalloc_scratch(void** out);
+
 // Plans the attention launch and the workspace for (shape, K_b, k).
 tls_status plan_workspace(const tls_shape& s, int K_b, int k, WsLayout* out);
 

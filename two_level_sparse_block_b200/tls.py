@@ -90,7 +90,7 @@ _SIG = {
     "tls_block_cache_create": (_I32, [_P, _P, _P, _I64, _I64, _I32, _P, _P, _P, _P]),
     "tls_block_cache_destroy": (None, [_P]),
     "tls_block_cache_plan": (_I32, [_P, _P, _P, _I32, _P, _P, _P, _P]),
-    "tls_prefetch_diff": (_I32, [_P, _P, _P, _I32, _P, _P]),
+    "tls_prefetch_diff": (_I32, [_P, _P, _P, _I32, _P, _P, _P]),
     "tls_block_cache_table": (_I32, [_P, _P]),
     "tls_engine_create": (_I32, [_P, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "tls_engine_create_resident": (_I32, [_P, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
@@ -186,6 +186,7 @@ def tls_workspace_bytes(shape: Shape, K_b: int, k: int) -> int:
 
 
 def tls_workspace_error(ws, clear=True, stream=None) -> int:
+    """Error word of a workspace, or (ws=None) of the scratch-free attention's array."""
     code = ctypes.c_int32(0)
     _check(lib().tls_workspace_error(_ptr(ws), int(bool(clear)), ctypes.byref(code), _stream(stream)),
            "tls_workspace_error")
@@ -261,10 +262,13 @@ def tls_block_cache_plan(handle, new_block_idx, in_use_block_idx, K_b, copy_row=
     return n.value
 
 
-def tls_prefetch_diff(handle, new_block_idx_host, in_use_block_idx_host, K_b, copy_stream=None) -> int:
+def tls_prefetch_diff(handle, new_block_idx_host, in_use_block_idx_host, K_b, copy_stream=None,
+                      done_event=None) -> int:
+    """done_event: optional torch.cuda.Event (or raw cudaEvent_t) recorded on copy_stream after the copies."""
     n = ctypes.c_int32(0)
+    ev = getattr(done_event, "cuda_event", done_event)
     _check(lib().tls_prefetch_diff(handle, _ptr(new_block_idx_host), _ptr(in_use_block_idx_host), K_b,
-                                   _stream(copy_stream), ctypes.byref(n)), "tls_prefetch_diff")
+                                   _stream(copy_stream), ev, ctypes.byref(n)), "tls_prefetch_diff")
     return n.value
 
 
