@@ -34,6 +34,14 @@ Readings where the pages are silent (each is listed in the design notes):
   * Ties: higher score first, then lower index; index lists come out ascending.
   * Staggering: attend(t) uses blocks chosen with q_{t-1}, tokens and
     attention with q_t.
+  * A sequence holds its first n tokens; its blocks are the ceil(n / bs)
+    blocks those tokens fall in, the last one possibly partial, whose index
+    is the max/min of the keys it holds.  Candidates are the held positions
+    of the chosen blocks; a selection asked for more than there are takes
+    them all.  Attention over no token gives a zero output and lse -inf.
+  * Operator baselines [EN 4]: full attention (every held token), block
+    selection alone (every token of the top-K_b blocks, Quest) and token
+    selection alone (the top-k over every held token, Double Sparsity).
 
 Pins (tests that tie each function to something other than itself) are in
 tests/test_oracle_pins.py.  Parity of the *quality* of a selection (does it
@@ -61,6 +69,9 @@ __all__ = [
     "decode_row",
     "staggered_row",
     "plan_transfer",
+    "dense_row",
+    "quest_row",
+    "ds_row",
 ]
 
 
@@ -77,13 +88,14 @@ def widen_bf16(bits: np.ndarray) -> np.ndarray:
 def block_meta(k_bits: np.ndarray, block_size: int):
     """Per-block, per-channel max and min of the keys of one (row, KV head).
 
-    k_bits: uint16 [N, D] with N a multiple of block_size.
-    Returns (kmax, kmin) as float64 [N/block_size, D]; both are bf16 values
-    (max/min selects an input, so no rounding happens).
+    k_bits: uint16 [N, D], the tokens the sequence holds.  Block j holds
+    tokens j*bs .. min(N, (j+1)*bs) - 1, so the last block may be partial.
+    Returns (kmax, kmin) as float64 [ceil(N/block_size), D]; both are bf16
+    values (max/min selects an input, so no rounding happens).
     """
     k = widen_bf16(k_bits)
     n, d = k.shape
-    nb = n // block_size
+    nb = -(-n // block_size)
     kmax = np.empty((nb, d))
     kmin = np.empty((nb, d))
     for j in range(nb):
@@ -168,10 +180,12 @@ def topk_ascending(scores: np.ndarray, k: int) -> np.ndarray:
 # Level 2: token scores inside the chosen blocks and top-k  [EN 2A-2], [JA 2A]
 # --------------------------------------------------------------------------
 
-def candidate_tokens(block_idx: np.ndarray, block_size: int) -> np.ndarray:
-    """All token positions of the chosen blocks, ascending."""
+def candidate_tokens(block_idx: np.ndarray, block_size: int, n_tokens: int | None = None) -> np.ndarray:
+    """All token positions of the chosen blocks that the sequence holds
+    (below n_tokens, when given), ascending."""
     b = np.sort(np.asarray(block_idx, dtype=np.int64))
-    return (b[:, None] * block_size + np.arange(block_size)[None, :]).ravel()
+    c = (b[:, None] * block_size + np.arange(block_size)[None, :]).ravel()
+    return c if n_tokens is None else c[c < n_tokens]
 
 
 def token_scores(q: np.ndarray, label_ch: np.ndarray, codes: np.ndarray,
@@ -194,8 +208,11 @@ def token_scores(q: np.ndarray, label_ch: np.ndarray, codes: np.ndarray,
 def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, softmax_scale: float):
     """Softmax attention of G heads over n rows; returns (out [G, Dv], lse [G]).
 
-    lse is the natural log of sum_t exp(scale * q.k_t).
+    lse is the natural log of sum_t exp(scale * q.k_t).  With no row the
+    output is zero and lse is -inf (an empty sum).
     """
+    if k.shape[0] == 0:
+        return np.zeros((q.shape[0], v.shape[1])), np.full(q.shape[0], -np.inf)
     logits = softmax_scale * (q @ k.T)  # [G, n]
     m = logits.max(axis=1, keepdims=True)
     p = np.exp(logits - m)
@@ -236,7 +253,7 @@ def decode_row(q_bits_group: np.ndarray, k_bits: np.ndarray, v_bits: np.ndarray 
     agg = group_max(per_head)
     if block_idx is None:
         block_idx = topk_ascending(agg, K_b)
-    cand = candidate_tokens(block_idx, block_size)
+    cand = candidate_tokens(block_idx, block_size, k_bits.shape[0])
     ts = token_scores(q, label_ch, codes, scales, cand)
     if token_idx is None:
         token_idx = cand[topk_ascending(ts, k)]
@@ -267,6 +284,31 @@ def plan_transfer(new_blocks, resident_blocks) -> np.ndarray:
     m = set(int(b) for b in new_blocks)
     c = set(int(b) for b in resident_blocks)
     return np.asarray(sorted(m - c), dtype=np.int64)
+
+
+# --------------------------------------------------------------------------
+# Operator baselines  [EN 4] (full attention, Quest alone, Double Sparsity alone)
+# --------------------------------------------------------------------------
+
+def dense_row(q_bits_group, k_bits, v_bits, softmax_scale, v_offset=-1, v_dim=None):
+    """Full attention of the group's heads over every token the sequence holds."""
+    kf = widen_bf16(k_bits)
+    vf = kf[:, v_offset:v_offset + v_dim] if v_bits is None else widen_bf16(v_bits)
+    return attention(widen_bf16(q_bits_group), kf, vf, softmax_scale)
+
+
+def quest_row(q_bits_group, k_bits, v_bits, label_ch, block_size, K_b, softmax_scale, block_idx=None, **kw):
+    """Block selection alone: level 1, then attention over every token of the
+    K_b blocks (a token budget of K_b * bs takes every candidate)."""
+    return decode_row(q_bits_group, k_bits, v_bits, label_ch, block_size, K_b, K_b * block_size, softmax_scale,
+                      block_idx=block_idx, **kw)
+
+
+def ds_row(q_bits_group, k_bits, v_bits, label_ch, block_size, k, softmax_scale, token_idx=None, **kw):
+    """Token selection alone: level 2 over every block of the sequence, then attention."""
+    nb = -(-k_bits.shape[0] // block_size)
+    return decode_row(q_bits_group, k_bits, v_bits, label_ch, block_size, nb, k, softmax_scale,
+                      block_idx=np.arange(nb), token_idx=token_idx, **kw)
 
 
 def softmax_scale_for(qk_dim: int) -> float:

@@ -343,3 +343,122 @@ def test_c1_planted_tokens_carry_the_largest_exact_logits():
         mine = row.planted_pos[row.planted_head == h]
         assert mine.size == cfg.planted_per_row // cfg.group
         assert logits[h, mine].mean() > np.quantile(logits[h, ~mask], 0.999)
+
+
+# ---------------------------------------------------------------- ragged sequences, partial blocks
+
+def test_block_meta_partial_last_block_brute_force():
+    # 37 tokens in blocks of 8: four full blocks and one holding tokens 32..36
+    rng = np.random.default_rng(61)
+    kb = rand_bits(rng, (37, 6))
+    kmax, kmin = oracle.block_meta(kb, 8)
+    assert kmax.shape == (5, 6)
+    k = f32_from_bf16_bits(kb).astype(np.float64)
+    for j in range(5):
+        rows = range(8 * j, min(37, 8 * j + 8))
+        for c in range(6):
+            assert kmax[j, c] == max(float(k[t, c]) for t in rows)
+            assert kmin[j, c] == min(float(k[t, c]) for t in rows)
+
+
+def test_block_meta_grows_by_running_max_min():
+    # adding one token at a time changes only its block, whose max/min is the
+    # channel-wise max/min of the old one and the new key (a fresh block: the key)
+    rng = np.random.default_rng(62)
+    kb = rand_bits(rng, (29, 4))
+    k = f32_from_bf16_bits(kb).astype(np.float64)
+    for n in range(1, 29):
+        a_max, a_min = oracle.block_meta(kb[:n], 5)
+        b_max, b_min = oracle.block_meta(kb[:n + 1], 5)
+        j = n // 5
+        if n % 5 == 0:
+            assert np.array_equal(b_max[j], k[n]) and np.array_equal(b_min[j], k[n])
+        else:
+            assert np.array_equal(b_max[j], np.maximum(a_max[j], k[n]))
+            assert np.array_equal(b_min[j], np.minimum(a_min[j], k[n]))
+        assert np.array_equal(b_max[:j], a_max[:j]) and np.array_equal(b_min[:j], a_min[:j])
+
+
+def test_candidates_are_the_held_positions_of_the_chosen_blocks():
+    c = oracle.candidate_tokens(np.array([4, 0, 2]), 4, n_tokens=18)
+    assert c.tolist() == [0, 1, 2, 3, 8, 9, 10, 11, 16, 17]
+    assert oracle.candidate_tokens(np.array([1]), 4).tolist() == [4, 5, 6, 7]
+
+
+def test_short_sequence_takes_every_block_and_candidate():
+    # fewer blocks than K_b and fewer candidates than k: both levels take all,
+    # and the step is then full attention over the held tokens
+    rng = np.random.default_rng(63)
+    g, d, n, bs = 3, 16, 21, 8
+    q = rand_bits(rng, (g, d))
+    kb = rand_bits(rng, (n, d))
+    vb = rand_bits(rng, (n, d))
+    lab = np.array([1, 5, 7, 12])
+    r = oracle.decode_row(q, kb, vb, lab, bs, K_b=9, k=500, softmax_scale=0.25)
+    assert r["block_idx"].tolist() == [0, 1, 2]
+    assert r["token_idx"].tolist() == list(range(n))
+    qq = torch.from_numpy(f32_from_bf16_bits(q).astype(np.float64))
+    kk = torch.from_numpy(f32_from_bf16_bits(kb).astype(np.float64))
+    vv = torch.from_numpy(f32_from_bf16_bits(vb).astype(np.float64))
+    ref = torch.nn.functional.scaled_dot_product_attention(qq[:, None, :], kk[None].expand(g, -1, -1),
+                                                           vv[None].expand(g, -1, -1), scale=0.25)[:, 0, :]
+    assert np.allclose(r["out"], ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_empty_sequence_gives_zero_output_and_no_selection():
+    q = bits([[1.0, 2.0]])
+    r = oracle.decode_row(q, np.zeros((0, 2), np.uint16), np.zeros((0, 2), np.uint16), np.array([0, 1]), 4,
+                          K_b=2, k=3, softmax_scale=1.0)
+    assert r["block_idx"].size == 0 and r["token_idx"].size == 0
+    assert r["out"].tolist() == [[0.0, 0.0]] and r["lse"][0] == -np.inf
+
+
+# ---------------------------------------------------------------- operator baselines
+
+def test_dense_row_is_softmax_attention():
+    rng = np.random.default_rng(64)
+    g, d, n = 4, 24, 57
+    q, kb, vb = rand_bits(rng, (g, d)), rand_bits(rng, (n, d)), rand_bits(rng, (n, 16))
+    out, lse = oracle.dense_row(q, kb, vb, 0.2)
+    qq = torch.from_numpy(f32_from_bf16_bits(q).astype(np.float64))
+    kk = torch.from_numpy(f32_from_bf16_bits(kb).astype(np.float64))
+    vv = torch.from_numpy(f32_from_bf16_bits(vb).astype(np.float64))
+    ref = torch.nn.functional.scaled_dot_product_attention(qq[:, None, :], kk[None].expand(g, -1, -1),
+                                                           vv[None].expand(g, -1, -1), scale=0.2)[:, 0, :]
+    assert np.allclose(out, ref.numpy(), rtol=1e-12, atol=1e-12)
+    assert np.allclose(lse, torch.logsumexp(0.2 * qq @ kk.T, dim=1).numpy(), rtol=1e-12)
+    # the MLA form: V is the K row slice
+    out2, _ = oracle.dense_row(q, kb, None, 0.2, v_offset=4, v_dim=8)
+    ref2 = torch.softmax(0.2 * qq @ kk.T, dim=1) @ kk[:, 4:12]
+    assert np.allclose(out2, ref2.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_quest_row_attends_every_token_of_its_blocks():
+    rng = np.random.default_rng(65)
+    g, d, n, bs, K_b = 2, 16, 90, 8, 4
+    q, kb, vb = rand_bits(rng, (g, d)), rand_bits(rng, (n, d)), rand_bits(rng, (n, d))
+    lab = np.array([0, 3, 9, 15])
+    r = oracle.quest_row(q, kb, vb, lab, bs, K_b, 0.25)
+    meta = oracle.block_meta(kb, bs)
+    agg = oracle.block_scores(f32_from_bf16_bits(q).astype(np.float64), *meta).max(axis=0)
+    assert r["block_idx"].tolist() == sorted(np.argsort(-agg, kind="stable")[:K_b].tolist())
+    want = [t for b in r["block_idx"] for t in range(b * bs, min(n, b * bs + bs))]
+    assert r["token_idx"].tolist() == want
+    ref, _ = oracle.dense_row(q, kb[want], vb[want], 0.25)
+    assert np.allclose(r["out"], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_ds_row_with_every_token_is_full_attention():
+    rng = np.random.default_rng(66)
+    g, d, n, bs = 3, 16, 45, 8
+    q, kb, vb = rand_bits(rng, (g, d)), rand_bits(rng, (n, d)), rand_bits(rng, (n, d))
+    lab = np.array([2, 3, 11, 13])
+    r = oracle.ds_row(q, kb, vb, lab, bs, n, 0.3)
+    assert r["block_idx"].tolist() == list(range(6)) and r["token_idx"].tolist() == list(range(n))
+    ref, _ = oracle.dense_row(q, kb, vb, 0.3)
+    assert np.allclose(r["out"], ref, rtol=1e-12, atol=1e-12)
+    # with a smaller budget: the top-k of the label scores over every held token
+    r2 = oracle.ds_row(q, kb, vb, lab, bs, 10, 0.3)
+    codes, scales = oracle.quant_label(kb, lab)
+    ts = oracle.token_scores(f32_from_bf16_bits(q).astype(np.float64), lab, codes, scales, np.arange(n))
+    assert r2["token_idx"].tolist() == sorted(sorted(range(n), key=lambda t: (-ts[t], t))[:10])
