@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--no-offload", action="store_true", help="skip the offload-engine measurement (c4)")
     ap.add_argument("--no-other-configs", action="store_true", help="skip the c1 / c3 step measurements")
     ap.add_argument("--no-c5", action="store_true", help="skip the c5 per-layer measurements")
+    ap.add_argument("--no-baselines", action="store_true",
+                    help="skip the operator baselines (full attention, block or token selection alone)")
     ap.add_argument("--no-staggered", action="store_true",
                     help="time the synchronous step (tls_decode_step) as the headline instead of the staggered one")
     ap.add_argument("--e2e-steps", type=int, default=300)
@@ -197,9 +199,54 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- CPU oracle arm
 
-def time_oracle(cfg, q, K, V, lab, seconds, rows_sample=8):
+def _oracle_rows(args):
+    """Worker of the oracle timing: decode_row over its rows until `seconds`
+    have passed; returns (rows done, seconds).  Rows are (q of the group, K,
+    V, label channels, meta, label cache), or (b, kvh) pairs that the worker
+    regenerates from the seeded generator first (untimed)."""
+    rows, cfg_fields, seconds = args
+    import oracle
+    import synth
+    cfg = synth.WorkloadConfig(**cfg_fields)
+    g = cfg.group
+    if rows and len(rows[0]) == 2:
+        q = synth.gen_queries(cfg)
+        lab_all = synth.gen_label_channels(cfg)
+        made = []
+        for b, h in rows:
+            r = synth.gen_row(cfg, b, h, q)
+            made.append((q[b, h * g:(h + 1) * g], r.k, r.v, lab_all[h], oracle.block_meta(r.k, cfg.block_size),
+                         oracle.quant_label(r.k, lab_all[h])))
+        rows = made
+    done = 0
+    t0 = time.perf_counter()
+    while True:
+        qg, kb, vb, lab, meta, label = rows[done % len(rows)]
+        oracle.decode_row(qg, kb, vb, lab, cfg.block_size, cfg.K_b, cfg.k, cfg.softmax_scale,
+                          v_offset=cfg.v_offset, v_dim=cfg.v_dim, meta=meta, label=label)
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= seconds and done >= len(rows):
+            return done, el
+
+
+def cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+def time_oracle(cfg, q, K, V, lab, seconds, rows_sample=8, all_cores=True):
     """Times the float64 oracle's per-step path (levels 1, 2 and attention;
-    the index build is prepared outside the timed region, as on the GPU)."""
+    the index build is prepared outside the timed region, as on the GPU):
+    single-threaded, and (all_cores) with one single-threaded process per host
+    core working on the sampled rows at once (a spawn pool, so no CUDA state is
+    forked)."""
+    import dataclasses
     import oracle
     try:
         import threadpoolctl
@@ -213,26 +260,47 @@ def time_oracle(cfg, q, K, V, lab, seconds, rows_sample=8):
     prepared = []
     for b, h in pick:
         kb = K[b, h]
-        prepared.append((b, h, oracle.block_meta(kb, cfg.block_size), oracle.quant_label(kb, lab[h])))
-    done = 0
-    t0 = time.perf_counter()
-    while True:
-        b, h, meta, label = prepared[done % len(prepared)]
-        oracle.decode_row(q[b, h * g:(h + 1) * g], K[b, h], None if V is None else V[b, h], lab[h], cfg.block_size,
-                          cfg.K_b, cfg.k, cfg.softmax_scale, v_offset=cfg.v_offset, v_dim=cfg.v_dim, meta=meta,
-                          label=label)
-        done += 1
-        el = time.perf_counter() - t0
-        if el >= seconds and done >= len(prepared):
-            break
+        prepared.append((q[b, h * g:(h + 1) * g], kb, None if V is None else V[b, h], lab[h],
+                         oracle.block_meta(kb, cfg.block_size), oracle.quant_label(kb, lab[h])))
+    fields = dataclasses.asdict(cfg)
+    done, el = _oracle_rows((prepared, fields, seconds))
     if limiter is not None:
         limiter.unregister()
     per_row = el / done
     step_s = per_row * cfg.rows
-    return {"value": cfg.batch / step_s, "unit": "decode tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{done} (batch row, KV head) decode_row calls over {len(pick)} seeded rows of "
-                      f"{cfg.name} in {el:.1f} s; scaled to all {cfg.rows} rows of one step",
-            "s_per_step": step_s}
+    res = {"value": cfg.batch / step_s, "unit": "decode tokens/s", "cores": 1, "kind": "oracle",
+           "sample": f"{done} (batch row, KV head) decode_row calls over {len(pick)} seeded rows of "
+                     f"{cfg.name} in {el:.1f} s; scaled to all {cfg.rows} rows of one step",
+           "s_per_step": step_s, "nproc": os.cpu_count(), "cpu_model": cpu_model()}
+    if all_cores and (os.cpu_count() or 1) > 1:
+        import multiprocessing as mp
+        n = min(os.cpu_count(), 64)
+        saved = {k: os.environ.get(k) for k in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")}
+        for k in saved:
+            os.environ[k] = "1"
+        try:
+            ctx = mp.get_context("spawn")
+            with ctx.Pool(n) as pool:
+                # each worker regenerates two of the sampled rows (the arrays are too large to ship)
+                work = [([pick[(2 * i + j) % len(pick)] for j in range(2)], fields, seconds) for i in range(n)]
+                t0 = time.perf_counter()
+                outs = pool.map(_oracle_rows, work)
+                wall = time.perf_counter() - t0
+        finally:
+            for k, v in saved.items():
+                if v is None:
+                    os.environ.pop(k, None)
+                else:
+                    os.environ[k] = v
+        rows_done = sum(d for d, _ in outs)
+        span = max(e for _, e in outs)
+        step_all = span / rows_done * cfg.rows
+        res["all_cores"] = {"value": cfg.batch / step_all, "unit": "decode tokens/s", "cores": n,
+                            "sample": f"{n} single-threaded processes (of {os.cpu_count()} host threads), each "
+                                      f"decoding two of the sampled rows for {seconds:.0f} s ({rows_done} "
+                                      f"decode_row calls, {wall:.1f} s wall with regeneration); scaled to all "
+                                      f"{cfg.rows} rows of one step"}
+    return res
 
 
 def time_step_graph(st, dev, steps=200, warmup=10):
@@ -306,6 +374,60 @@ def time_staggered_graphs(st, dev, steps=200, warmup=10):
     return [x.elapsed_time(y) for x, y in times]
 
 
+def time_graph(fn, dev, steps=100, warmup=5):
+    """Mean ms of fn() captured into a CUDA graph and replayed, L2 flushed
+    (write + read of 256 MB) before each replay, CUDA events around it."""
+    import torch
+    flush = torch.empty(64 << 20, dtype=torch.float32, device=dev)
+    flush_rd = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+    cap = torch.cuda.Stream(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(cap):
+        fn(cap)
+        with torch.cuda.graph(g, stream=cap):
+            fn(cap)
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    times = []
+    for i in range(warmup + steps):
+        flush.fill_(float(i))
+        torch.sum(flush_rd, dim=0, out=sink)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+        if i >= warmup:
+            times.append((a, b))
+    torch.cuda.synchronize(dev)
+    del g
+    return statistics.mean(x.elapsed_time(y) for x, y in times)
+
+
+def measure_baselines(st, cfg, dev, staggered_us=None, steps=100):
+    """The operator comparison of the pages (English summary 4, Efficiency) on
+    this GPU: the two-level step against full attention (every token), block
+    selection alone (Quest: every token of the K_b blocks) and token selection
+    alone (Double Sparsity: the top-k over every token), each one graph replay
+    with a cold L2, same inputs."""
+    two = 1e3 * time_graph(lambda s: st.step(stream=s), dev, steps)
+    full = 1e3 * time_graph(lambda s: st.dense(stream=s), dev, steps)
+    quest = 1e3 * time_graph(lambda s: st.quest(stream=s), dev, steps)
+    ds = 1e3 * time_graph(lambda s: st.ds(stream=s), dev, steps)
+    if st.check_device_error() != 0:
+        raise RuntimeError("device error in the baselines")
+    best = min(two, staggered_us) if staggered_us else two
+    return {"workload": cfg.name, "two_level_us": two, "two_level_staggered_us": staggered_us,
+            "full_attention_us": full, "quest_only_us": quest, "ds_only_us": ds,
+            "speedup_vs_full": full / best, "speedup_vs_ds": ds / best, "speedup_vs_quest": quest / best,
+            "budgets": {"two_level": f"K_b {cfg.K_b}, k {cfg.k}", "quest_only": f"K_b {cfg.K_b} (all {cfg.K_b * cfg.block_size} tokens of them)",
+                        "ds_only": f"k {cfg.k} of all {cfg.ctx_len} tokens", "full": f"all {cfg.ctx_len} tokens"},
+            "speedups_use": "the faster of the synchronous and the staggered two-level step",
+            "pages": "operator speedups quoted for context (GPU unstated): GQA 1.2-4.0x vs Double Sparsity and "
+                     "1.7-6.2x vs full attention; MLA 1.9-4.0x and 3.3-10.0x (English summary 4)",
+            "timing": "each path one CUDA graph, L2 flushed before every replay, mean of CUDA-event times"}
+
+
 def measure_config(name, dev, steps=200, warmup=10):
     """One more workload measured like the headline (time_step_graph)."""
     import synth
@@ -320,7 +442,9 @@ def measure_config(name, dev, steps=200, warmup=10):
     ts = time_step_graph(st, dev, steps, warmup)
     ms = statistics.mean(tss)  # (event ticks are coarse: the mean, not the median, averages them out)
     ab = algorithmic_bytes(c)
+    base = measure_baselines(st, c, dev, ms * 1e3) if name == "c3" else None
     return {"us_per_step": ms * 1e3, "us_per_step_median": statistics.median(tss) * 1e3,
+            "baselines": base,
             "decode_tokens_per_s": c.batch / (ms / 1e3),
             "algorithmic_bytes": ab["step"], "achieved_gbs": ab["step"] / (ms / 1e3) / 1e9,
             "synchronous_us_per_step": statistics.mean(ts) * 1e3,
@@ -328,6 +452,26 @@ def measure_config(name, dev, steps=200, warmup=10):
             "schedule": "staggered step (resident engine), as the headline; synchronous_us_per_step: "
                         "tls_decode_step",
             "l2": "flushed before every step (write + read of 256 MB)"}
+
+
+def pcie_h2d_peak(dev, nbytes=256 << 20, reps=5):
+    """Host -> device bandwidth of one large copy from pinned memory (best of
+    reps, CUDA events): the copy engines' ceiling the block transfers are
+    compared against."""
+    import torch
+    src = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    dst = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    best = None
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        dst.copy_(src, non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = a.elapsed_time(b)
+        best = ms if best is None else min(best, ms)
+    return nbytes / (best / 1e3) / 1e9
 
 
 def measure_offload_engine(dev, steps=64, name="c4", data=None):
@@ -347,11 +491,29 @@ def measure_offload_engine(dev, steps=64, name="c4", data=None):
         lab = synth.gen_label_channels(cfg)
     else:
         qs, K, V, lab = data
+    qd = [torch.from_numpy(np.ascontiguousarray(q).view(np.int16)).to(dev).view(torch.bfloat16) for q in qs]
+    stream = torch.cuda.current_stream(dev)
+    # the same layer and q trajectory with its K/V resident in HBM (the
+    # resident engine: the same stagger, no transfer), issued the same way: the
+    # step time the transfers would add to if they were not hidden
+    st = runtime.state_for_config(cfg, qs[0], K, V, lab, device=dev)
+    eng = runtime.ResidentEngine(st)
+    try:
+        r_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        torch.cuda.synchronize(dev)
+        for t in range(steps):
+            r_evs[t][0].record(stream)
+            eng.step(q=qd[t], stream=stream)
+            r_evs[t][1].record(stream)
+        torch.cuda.synchronize(dev)
+        resident_ms = [a.elapsed_time(b) for a, b in r_evs][1:]
+    finally:
+        eng.close()
+        del st
+        torch.cuda.empty_cache()
     layer = runtime.offloaded_layer_for_config(cfg, K, V, lab)
     del K, V
     try:
-        qd = [torch.from_numpy(np.ascontiguousarray(q).view(np.int16)).to(dev).view(torch.bfloat16) for q in qs]
-        stream = torch.cuda.current_stream(dev)
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
         torch.cuda.synchronize(dev)
         host_s = []
@@ -374,19 +536,30 @@ def measure_offload_engine(dev, steps=64, name="c4", data=None):
     finally:
         layer.close()
     steady = step_ms[1:]
+    peak = pcie_h2d_peak(dev)
+    copy_us = 1e3 * copy_ms / len(st)
+    added_us = max(0.0, 1e3 * (statistics.mean(steady) - statistics.mean(resident_ms)))
+    h2d = moved / (copy_ms / 1e3) / 1e9 if copy_ms > 0 else None
     return {
         "workload": cfg.name, "steps": steps, "n_slots": (cfg.n_slots or 2 * cfg.K_b) * cfg.rows, "K_b": cfg.K_b,
+        "resident_us_per_step_mean": 1e3 * statistics.mean(resident_ms),
+        "added_us_per_step_vs_resident": added_us,
+        "hidden_frac_vs_resident": (1.0 - min(1.0, added_us / copy_us)) if copy_us > 0 else None,
+        "pcie_peak_gbs": peak, "h2d_frac_of_pcie_peak": (h2d / peak) if h2d else None,
         "us_per_step_median": 1e3 * statistics.median(steady), "us_per_step_mean": 1e3 * statistics.mean(steady),
         "us_first_step": 1e3 * step_ms[0], "prologue_blocks": prologue.n_copied,
         "host_us_per_step_median": 1e6 * statistics.median(host_s[1:]),
         "transfer_blocks_per_step_mean": statistics.mean(blocks),
         "transfer_frac_of_K_b_mean": statistics.mean(blocks) / (cfg.K_b * cfg.rows),
-        "h2d_gbs": moved / (copy_ms / 1e3) / 1e9 if copy_ms > 0 else None,
-        "copy_us_per_step_mean": 1e3 * copy_ms / len(st), "exposed_us_per_step_mean": 1e3 * exposed_ms / len(st),
+        "h2d_gbs": h2d,
+        "copy_us_per_step_mean": copy_us, "exposed_us_per_step_mean": 1e3 * exposed_ms / len(st),
         "copy_hidden_frac": 1.0 - exposed_ms / copy_ms if copy_ms > 0 else None, "target_hidden_frac": 0.9,
         "timing": "per step: CUDA events on the caller's stream around tls_engine_step (level 2 + wait for the "
                   "previous transfer + attention; level 1 runs on the engine's second stream); transfer figures "
-                  "from the engine's copy-stream events",
+                  "from the engine's copy-stream events.  copy_hidden_frac counts the time the attention waited "
+                  "on a transfer past its own readiness; hidden_frac_vs_resident compares the step with the same "
+                  "layer and q trajectory over HBM-resident K/V (resident engine, no transfer): 1 - (step time "
+                  "added by offloading) / (copy-stream time)",
     }
 
 
@@ -489,11 +662,11 @@ def run_reference(args, cfg):
     cfg, q, K, V, lab = workload(cfg, 0)
     per_step = max(0.5, args.cpu_seconds / max(1, args.steps))
     for _ in range(args.warmup):
-        time_oracle(cfg, q, K, V, lab, 0.0, rows_sample=1)
+        time_oracle(cfg, q, K, V, lab, 0.0, rows_sample=1, all_cores=False)
     t = []
     res = None
     for _ in range(args.steps):
-        res = time_oracle(cfg, q, K, V, lab, per_step, rows_sample=2)
+        res = time_oracle(cfg, q, K, V, lab, per_step, rows_sample=2, all_cores=False)
         t.append(res["s_per_step"])
     step_s = statistics.mean(t)
     value = cfg.batch / step_s
@@ -736,6 +909,8 @@ def main():
         "clocks": clocks,
         "wall_s_timed": wall,
     }
+    if rank == 0 and world == 1 and not args.no_baselines:
+        line["baselines"] = measure_baselines(st, c, dev, ms_per_step * 1e3)
     if rank == 0 and world == 1 and not args.no_offload:
         line["offload_engine"] = measure_offload_engine(dev)
     if rank == 0 and world == 1 and not args.no_c5:

@@ -32,8 +32,16 @@
  *     reported through the workspace error word (tls_workspace_error).
  *   - Shapes: B batch, Hq query heads, Hkv KV heads (Hq % Hkv == 0,
  *     G = Hq / Hkv heads share one KV head), Dqk key dim, Dv value dim,
- *     N context length, bs block size, NB = N / bs, R label channels,
+ *     N context capacity, bs block size, NB = N / bs, R label channels,
  *     "row" = one (batch, KV head) pair, rows = B * Hkv.
+ *   - Ragged batches and partial blocks: sequence b holds len_b tokens,
+ *     positions 0 .. len_b - 1 (tls_shape.seq_lens; all N when NULL).  Its
+ *     blocks are j < ceil(len_b / bs); the last one may be partial.  Positions
+ *     >= len_b are never scored, selected or attended.  When a sequence has
+ *     fewer blocks than K_b, or its chosen blocks fewer tokens than k, the
+ *     valid entries of its list come first (ascending) and the rest are -1.
+ *     A sequence with len_b = 0 gets empty (all -1) lists, a zero output and
+ *     lse = -inf.
  */
 #ifndef TLS_H
 #define TLS_H
@@ -71,8 +79,11 @@ typedef struct tls_shape {
                            slice [v_offset, v_offset + v_dim) (MLA shared latent) */
   int32_t block_size;   /* bs: tokens per block, multiple of 8, <= 256 */
   int32_t n_label;      /* R: label channels, even, 2..64, <= qk_dim */
-  int64_t ctx_len;      /* N: multiple of block_size */
+  int64_t ctx_len;      /* N: capacity of every sequence in tokens (the row stride of K/V and
+                           of the index), a multiple of block_size */
   float softmax_scale;  /* logits are softmax_scale * q.k (e.g. 1/sqrt(Dqk)) */
+  const int32_t* seq_lens; /* optional device int32 [B]: tokens present in each sequence, 0..N
+                              (values outside are clamped); NULL: every sequence holds N */
 } tls_shape;
 
 /* Output element type of tls_sparse_decode_attn. */
@@ -149,19 +160,22 @@ TLS_API tls_status tls_workspace_error(const void* ws, int32_t clear, int32_t* c
 
 /*
  * Index build, part 1 (Stage 1 block-level index; Italian 2.A.1 max/min of
- * the keys).  For every row and every block j with t0 <= j*bs < t1:
- *   meta[row, j, c]       = max over the block's tokens of K[row, t, c]
- *   meta[row, j, Dqk + c] = min over the block's tokens of K[row, t, c]
- * k: device bf16, row r's token t at k + (r*N + t) * k_row_stride.
- * meta: device bf16 [B, Hkv, NB, 2*Dqk].  t0, t1 multiples of bs,
- * 0 <= t0 < t1 <= N.  The values are exact (max/min picks an input).
+ * the keys).  For every row and every block j with t0 <= j*bs < t1 that
+ * holds a token below e = min(t1, len_b):
+ *   meta[row, j, c]       = max over the block's tokens t < e of K[row, t, c]
+ *   meta[row, j, Dqk + c] = min over the block's tokens t < e of K[row, t, c]
+ * (so a partial last block covers the tokens it holds; blocks with none are
+ * left untouched).  k: device bf16, row r's token t at
+ * k + (r*N + t) * k_row_stride.  meta: device bf16 [B, Hkv, NB, 2*Dqk].
+ * t0 a multiple of bs, 0 <= t0 < t1 <= N.  The values are exact (max/min
+ * picks an input).
  */
 TLS_API tls_status tls_build_block_meta(const tls_shape* shape, const void* k, int64_t k_row_stride,
                                 int64_t t0, int64_t t1, void* meta, void* stream);
 
 /*
  * Index build, part 2 (Stage 2: channel selection + INT4 keys).  For every
- * row and token t0 <= t < t1, with x_r = K[row, t, label_ch[h, r]]:
+ * row and token t0 <= t < min(t1, len_b), with x_r = K[row, t, label_ch[h, r]]:
  *   s = max_r |x_r| / 7                  (float32, IEEE division)
  *   code_r = rint(x_r / s) in [-7, 7]    (float32, ties to even; s = 0 -> 0)
  * codes: device uint8 [B, Hkv, N, R/2]; byte j holds code 2j in its low
@@ -180,9 +194,10 @@ TLS_API tls_status tls_quant_label_cache(const tls_shape* shape, const void* k, 
  * a row combine by max: agg[row, j] = max_h S[h, j].  Then the K_b blocks
  * with the largest agg (ties: lower block index) are written ascending.
  * q: device bf16 [B, Hq, Dqk] (16-byte aligned); meta as built above
- * (16-byte aligned).  block_idx: device int32 [B, Hkv, K_b].
- * block_score: optional device float32 [B, Hkv, NB] receiving agg.
- * 1 <= K_b <= NB, NB <= 16384.
+ * (16-byte aligned).  block_idx: device int32 [B, Hkv, K_b]; only blocks
+ * holding tokens of the sequence compete (the list is padded with -1 past
+ * them).  block_score: optional device float32 [B, Hkv, NB] receiving agg
+ * (-inf for blocks past the sequence).  1 <= K_b <= NB, NB <= 16384.
  */
 TLS_API tls_status tls_select_blocks(const tls_shape* shape, const void* q, const void* meta, int32_t K_b,
                              int32_t* block_idx, float* block_score,
@@ -193,11 +208,13 @@ TLS_API tls_status tls_select_blocks(const tls_shape* shape, const void* q, cons
  * blocks (candidates in ascending token order),
  *   score(t) = max_h  s_t * sum_r q_h[label_ch[h_kv, r]] * code_{t, r}
  * then the k best candidates (ties: lower token index) are written
- * ascending as absolute token positions.
- * block_idx: device int32 [B, Hkv, K_b], ascending per row (as written by
- * tls_select_blocks).  token_idx: device int32 [B, Hkv, k].
- * token_score: optional device float32 [B, Hkv, K_b*bs] receiving the
- * candidate scores.  1 <= k <= K_b*bs <= 16384.
+ * ascending as absolute token positions.  Candidates are the positions
+ * below len_b of the listed blocks; entries -1 of the list end it.
+ * block_idx: device int32 [B, Hkv, K_b], ascending per row with any -1 at
+ * the end (as written by tls_select_blocks).  token_idx: device int32
+ * [B, Hkv, k], padded with -1 past the candidates.  token_score: optional
+ * device float32 [B, Hkv, K_b*bs] receiving the candidate scores (-inf past
+ * the candidates).  1 <= k <= K_b*bs <= 524288.
  */
 TLS_API tls_status tls_select_tokens(const tls_shape* shape, const void* q, const int32_t* label_ch,
                              const uint8_t* codes, const float* scales, const int32_t* block_idx,
@@ -213,8 +230,10 @@ TLS_API tls_status tls_select_tokens(const tls_shape* shape, const void* q, cons
  * the token list with a log-sum-exp merge inside the same launch.
  * out: device [B, Hq, Dv], float32 (out_dtype TLS_OUT_F32) or bf16
  * (TLS_OUT_BF16, round to nearest even).  lse: optional device float32 [B, Hq].
- * Token indices must lie in [0, N); with a slot table, every block they fall
- * in must map to a slot in [0, n_slots) (not checked on the device).
+ * Entries outside [0, len_b) (the -1 padding of a selection) are skipped;
+ * with a slot table, every block a valid entry falls in must map to a slot
+ * in [0, n_slots) (slots are clamped into the pool on the device).  A row
+ * with no valid entry gets a zero output and lse = -inf.  1 <= k <= N.
  */
 TLS_API tls_status tls_sparse_decode_attn(const tls_shape* shape, const void* q, const tls_kv_view* kv,
                                   const int32_t* token_idx, int32_t k, int32_t out_dtype,
@@ -240,6 +259,67 @@ TLS_API tls_status tls_decode_step(const tls_shape* shape, const void* q, const 
                            const tls_kv_view* kv, int32_t K_b, int32_t k,
                            int32_t* block_idx, int32_t* token_idx, int32_t out_dtype,
                            void* out, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Operator baselines (English summary 4, Efficiency: the method is compared
+ * with full attention and with each level alone -- Quest's block selection,
+ * Double Sparsity's token selection).  Same numerics and output conventions
+ * as tls_sparse_decode_attn; each takes a workspace of the size given.
+ * ------------------------------------------------------------------------ */
+
+/*
+ * Full attention: every token a sequence holds (positions 0 .. len_b - 1),
+ * with no selection.  Workspace: tls_workspace_bytes(shape, NB, N).
+ */
+TLS_API tls_status tls_dense_decode_attn(const tls_shape* shape, const void* q, const tls_kv_view* kv,
+                                         int32_t out_dtype, void* out, float* lse, void* ws, size_t ws_bytes,
+                                         void* stream);
+
+/*
+ * Block selection alone (Quest): level 1 as tls_select_blocks writes
+ * block_idx, then attention over every token of the K_b chosen blocks
+ * (K_b * bs positions, no level 2).  Two launches.  Workspace:
+ * tls_workspace_bytes(shape, K_b, K_b * bs).
+ */
+TLS_API tls_status tls_quest_decode_step(const tls_shape* shape, const void* q, const void* meta,
+                                         const tls_kv_view* kv, int32_t K_b, int32_t* block_idx,
+                                         int32_t out_dtype, void* out, float* lse, void* ws, size_t ws_bytes,
+                                         void* stream);
+
+/*
+ * Token selection alone (Double Sparsity): level 2 over every token of the
+ * sequence (K_b = NB, no level 1) writes token_idx (k entries), then the
+ * attention over them.  Two launches.  Workspace:
+ * tls_workspace_bytes(shape, NB, k).
+ */
+TLS_API tls_status tls_ds_decode_step(const tls_shape* shape, const void* q, const int32_t* label_ch,
+                                      const uint8_t* codes, const float* scales, const tls_kv_view* kv, int32_t k,
+                                      int32_t* token_idx, int32_t out_dtype, void* out, float* lse, void* ws,
+                                      size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Appending the decoded token (English summary 2.A: the KV cache is split
+ * into blocks with a block-level index and an INT4 label cache; a decode step
+ * adds one token to each sequence, and with it to the index).
+ * ------------------------------------------------------------------------ */
+
+/*
+ * For every sequence b with t = seq_lens[b] < N and every KV head h: writes
+ * k_new[b, h] as K row t and v_new[b, h] as V row t (through kv: dense, or
+ * the slot of block t / bs in the slot table, which must be >= 0), updates
+ * the block-level index of block t / bs -- meta = (k, k) when t starts the
+ * block, else the channel-wise max / min with k -- quantises the token's
+ * label channels into codes / scales (as tls_quant_label_cache), and then
+ * sets seq_lens[b] = t + 1.  A full sequence (seq_lens[b] >= N) is left
+ * unchanged.  One launch; the result equals building the index over the
+ * grown sequence.
+ * seq_lens: device int32 [B] (in/out; shape->seq_lens is ignored).
+ * k_new: device bf16 [B, Hkv, Dqk]; v_new: device bf16 [B, Hkv, Dv], NULL
+ * when v_offset >= 0 (the value is the K row slice).  kv.k / kv.v are written.
+ */
+TLS_API tls_status tls_append_kv(const tls_shape* shape, int32_t* seq_lens, const void* k_new, const void* v_new,
+                                 const tls_kv_view* kv, void* meta, const int32_t* label_ch, uint8_t* codes,
+                                 float* scales, void* stream);
 
 /*
  * Scratch-free variant of tls_sparse_decode_attn (no counterpart in the
@@ -403,10 +483,14 @@ TLS_API tls_status tls_engine_create_resident(const tls_shape* shape, int32_t K_
  * engine (tls_engine_create_resident) has no transfer and no host wait: on
  * `stream` it records q_t, runs level 2 over M_{t-1} and the attention, and
  * waits for level 1 of step t (engine stream, after q_t) before returning, so
- * the next step's level 2 finds M_t complete.  After a failed
- * step (a copy failure, TLS_ERR_CAPACITY, a launch error) the cache no longer
- * matches the block lists: every later step returns the same error and the
- * engine must be destroyed.
+ * the next step's level 2 finds M_t complete.  The host waits (for level 1
+ * of the step, and for the prologue's block list) have a deadline:
+ * TLS_HOST_WAIT_MS milliseconds from the environment at engine creation, else
+ * 10 s; when it passes the step returns TLS_ERR_TIMEOUT (the device work
+ * completes on its own).  After a failed step (a timeout, a copy failure,
+ * TLS_ERR_CAPACITY, a launch error) the cache no longer matches the block
+ * lists: every later step returns the same error and the engine must be
+ * destroyed.
  */
 TLS_API tls_status tls_engine_step(tls_engine* engine, const void* q, int32_t out_dtype, void* out, float* lse,
                            void* stream);

@@ -161,6 +161,37 @@ def test_engine_copy_failure_is_reported_and_sticks(monkeypatch):
     assert float(x.sum()) == 1024.0
 
 
+def test_engine_host_wait_times_out_and_sticks(monkeypatch):
+    # host-side deadline: with TLS_HOST_WAIT_MS = 50, a step whose level 1 is
+    # held back ~1 s (a bounded spin kernel queued on the step's stream before
+    # it) returns TLS_ERR_TIMEOUT instead of blocking; later steps return the
+    # same status, and the device drains and stays healthy
+    runtime, tls = _rt()
+    monkeypatch.setenv("TLS_HOST_WAIT_MS", "50")
+    cfg = ENGINE[0]
+    qs = synth.gen_query_trajectory(cfg, 3)
+    K, V, _ = synth.gen_kv(cfg, qs[0])
+    lab = synth.gen_label_channels(cfg)
+    layer = runtime.offloaded_layer_for_config(cfg, K, V, lab)
+    try:
+        layer.step(_dev_q(qs[0]))
+        torch.cuda.synchronize()
+        q1 = _dev_q(qs[1])
+        torch.cuda._sleep(2_000_000_000)  # about a second of GPU clock cycles, then it ends
+        with pytest.raises(tls.TlsError) as e:
+            layer.step(q1)
+        assert e.value.status == tls.TLS_ERR_TIMEOUT
+        with pytest.raises(tls.TlsError) as e2:
+            layer.step(_dev_q(qs[2]))
+        assert e2.value.status == tls.TLS_ERR_TIMEOUT
+        torch.cuda.synchronize()
+        assert layer.check_device_error() == 0
+    finally:
+        layer.close()
+    x = torch.ones(1024, device="cuda")
+    assert float(x.sum()) == 1024.0
+
+
 def test_engine_on_the_offload_workload_sampled_steps():
     # c4 (MQA, 131072 tokens, 256 slots): three steps of the trajectory, the
     # row checked against the staggered oracle each step

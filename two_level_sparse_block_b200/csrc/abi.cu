@@ -3,22 +3,16 @@
 // decode_attn.cu; the index build in index_build.cu; the block cache and
 // incremental prefetch in block_cache.cu.
 
+#include <chrono>
+#include <cstdlib>
 #include <cstring>
+#include <thread>
 
 #include "host_common.h"
 #include "token_common.cuh"
 
 namespace tls {
 
-tls_status select_blocks_impl(const tls_shape& s, const void* q, const void* meta, int K_b, int32_t* block_idx,
-                              float* block_score, uint8_t* ws, const WsLayout& L, cudaStream_t stream);
-tls_status select_tokens_impl(const tls_shape& s, const void* q, const int32_t* label_ch, const uint8_t* codes,
-                              const float* scales, const int32_t* block_idx, int K_b, int k, int32_t* token_idx,
-                              float* token_score, uint8_t* ws, const WsLayout& L, cudaStream_t stream,
-                              bool pdl = false, bool lean = false);
-tls_status sparse_attn_impl(const tls_shape& s, const void* q, const tls_kv_view& kv, const int32_t* token_idx,
-                            int k, int out_dtype, void* out, float* lse, uint8_t* ws, const WsLayout& L,
-                            cudaStream_t stream, bool pdl = true);
 int attn_heads_per_cta(const tls_shape& s);
 bool attn_mma_supported(const tls_shape& s);
 int attn_mma_plan(int rows, int k, int* chunks_per_row, int* n_items, int* n_ctas);
@@ -39,6 +33,27 @@ tls_status fail(tls_status st, const char* fmt, ...) {
 }
 
 void clear_error() { g_err[0] = 0; }
+
+tls_status wait_event_deadline(cudaEvent_t ev, double timeout_ms, const char* what) {
+  const auto t0 = std::chrono::steady_clock::now();
+  for (;;) {
+    const cudaError_t e = cudaEventQuery(ev);
+    if (e == cudaSuccess) return TLS_OK;
+    if (e != cudaErrorNotReady) return cuda_check(e, what);
+    const double ms = std::chrono::duration<double, std::milli>(std::chrono::steady_clock::now() - t0).count();
+    if (ms > timeout_ms) return fail(TLS_ERR_TIMEOUT, "%s: no completion within %.0f ms", what, timeout_ms);
+    std::this_thread::yield();
+  }
+}
+
+double host_wait_ms() {
+  const char* v = std::getenv("TLS_HOST_WAIT_MS");
+  if (v != nullptr) {
+    const double x = std::atof(v);
+    if (x > 0.0) return x;
+  }
+  return 10000.0;
+}
 
 tls_status check_shape(const tls_shape* p) {
   if (p == nullptr) return fail(TLS_ERR_INVALID_ARG, "shape is NULL");
@@ -71,7 +86,8 @@ tls_status plan_workspace(const tls_shape& s, int K_b, int k, WsLayout* out) {
   if (K_b < 1 || K_b > nb) return fail(TLS_ERR_INVALID_ARG, "K_b %d must be in [1, NB=%lld]", K_b, (long long)nb);
   if (nb > 16384) return fail(TLS_ERR_UNSUPPORTED, "NB %lld above 16384", (long long)nb);
   const int64_t n_cand = (int64_t)K_b * s.block_size;
-  if (n_cand > 16384) return fail(TLS_ERR_UNSUPPORTED, "K_b*block_size %lld above 16384", (long long)n_cand);
+  if (n_cand > kMaxListLen) return fail(TLS_ERR_UNSUPPORTED, "K_b*block_size %lld above %lld", (long long)n_cand,
+                                        (long long)kMaxListLen);
   if (k < 1 || k > n_cand) return fail(TLS_ERR_INVALID_ARG, "k %d must be in [1, K_b*bs=%lld]", k, (long long)n_cand);
   WsLayout L;
   L.heads_per_cta = attn_heads_per_cta(s);
@@ -128,6 +144,15 @@ static tls_status check_ws(const tls_shape& s, int K_b, int k, void* ws, size_t 
   if (ws == nullptr || !aligned16(ws)) return fail(TLS_ERR_INVALID_ARG, "workspace NULL or not 16-byte aligned");
   if (ws_bytes < L->total)
     return fail(TLS_ERR_INVALID_ARG, "workspace %zu bytes < required %zu", ws_bytes, L->total);
+  return TLS_OK;
+}
+
+// Level 2 takes at most kMaxCandidates candidates per row.
+static tls_status check_candidates(const tls_shape& s, int K_b) {
+  const int64_t n_cand = (int64_t)K_b * s.block_size;
+  if (n_cand > kMaxCandidates)
+    return fail(TLS_ERR_UNSUPPORTED, "level 2 takes at most %lld candidates per row (K_b*bs = %lld)",
+                (long long)kMaxCandidates, (long long)n_cand);
   return TLS_OK;
 }
 
@@ -239,6 +264,8 @@ extern "C" tls_status tls_select_tokens(const tls_shape* shape, const void* q, c
   WsLayout L;
   st = check_ws(*shape, K_b, k, ws, ws_bytes, &L);
   if (st != TLS_OK) return st;
+  st = check_candidates(*shape, K_b);
+  if (st != TLS_OK) return st;
   return select_tokens_impl(*shape, q, label_ch, codes, scales, block_idx, K_b, k, token_idx, token_score,
                             (uint8_t*)ws, L, (cudaStream_t)stream);
 }
@@ -282,6 +309,8 @@ static tls_status select_impl(const tls_shape* shape, const void* q, const void*
   WsLayout L;
   st = check_ws(*shape, K_b, k, ws, ws_bytes, &L);
   if (st != TLS_OK) return st;
+  st = check_candidates(*shape, K_b);
+  if (st != TLS_OK) return st;
   st = select_blocks_impl(*shape, q, meta, K_b, block_idx, nullptr, (uint8_t*)ws, L, (cudaStream_t)stream);
   if (st != TLS_OK) return st;
   return select_tokens_impl(*shape, q, label_ch, codes, scales, block_idx, K_b, k, token_idx, nullptr,
@@ -312,4 +341,80 @@ extern "C" tls_status tls_decode_step(const tls_shape* shape, const void* q, con
   st = select_impl(shape, q, meta, label_ch, codes, scales, K_b, k, block_idx, token_idx, ws, ws_bytes, stream);
   if (st != TLS_OK) return st;
   return tls_sparse_decode_attn(shape, q, kv, token_idx, k, out_dtype, out, lse, ws, ws_bytes, stream);
+}
+
+// ---------------------------------------------------------------------------
+// Operator baselines: full attention, block selection alone, token selection
+// alone (English summary 4, Efficiency).
+// ---------------------------------------------------------------------------
+
+static tls_status check_attn_args(const tls_shape* shape, const void* q, const tls_kv_view* kv, int32_t out_dtype,
+                                  const void* out, const char* who) {
+  tls_status st = check_shape(shape);
+  if (st != TLS_OK) return st;
+  st = check_kv(*shape, kv);
+  if (st != TLS_OK) return st;
+  if (q == nullptr || out == nullptr) return fail(TLS_ERR_INVALID_ARG, "%s: null pointer", who);
+  if (!aligned16(q)) return fail(TLS_ERR_INVALID_ARG, "%s: q not 16-byte aligned", who);
+  if (out_dtype != TLS_OUT_F32 && out_dtype != TLS_OUT_BF16)
+    return fail(TLS_ERR_INVALID_ARG, "%s: out_dtype must be TLS_OUT_F32 or TLS_OUT_BF16", who);
+  return TLS_OK;
+}
+
+extern "C" tls_status tls_dense_decode_attn(const tls_shape* shape, const void* q, const tls_kv_view* kv,
+                                            int32_t out_dtype, void* out, float* lse, void* ws, size_t ws_bytes,
+                                            void* stream) {
+  clear_error();
+  tls_status st = check_attn_args(shape, q, kv, out_dtype, out, "dense_decode_attn");
+  if (st != TLS_OK) return st;
+  const int nb = (int)n_blocks(*shape);
+  if (shape->ctx_len > kMaxListLen) return fail(TLS_ERR_UNSUPPORTED, "dense_decode_attn: ctx_len above 2^24");
+  WsLayout L;
+  st = check_ws(*shape, nb, (int)shape->ctx_len, ws, ws_bytes, &L);
+  if (st != TLS_OK) return st;
+  return sparse_attn_impl(*shape, q, *kv, nullptr, (int)shape->ctx_len, out_dtype, out, lse, (uint8_t*)ws, L,
+                          (cudaStream_t)stream, /*pdl=*/true, kListAll);
+}
+
+extern "C" tls_status tls_quest_decode_step(const tls_shape* shape, const void* q, const void* meta,
+                                            const tls_kv_view* kv, int32_t K_b, int32_t* block_idx,
+                                            int32_t out_dtype, void* out, float* lse, void* ws, size_t ws_bytes,
+                                            void* stream) {
+  clear_error();
+  tls_status st = check_attn_args(shape, q, kv, out_dtype, out, "quest_decode_step");
+  if (st != TLS_OK) return st;
+  if (meta == nullptr || block_idx == nullptr) return fail(TLS_ERR_INVALID_ARG, "quest_decode_step: null pointer");
+  if (!aligned16(meta)) return fail(TLS_ERR_INVALID_ARG, "quest_decode_step: meta not 16-byte aligned");
+  const int64_t k = (int64_t)K_b * shape->block_size;
+  if (K_b < 1 || k > kMaxListLen) return fail(TLS_ERR_INVALID_ARG, "quest_decode_step: K_b %d out of range", K_b);
+  WsLayout L;
+  st = check_ws(*shape, K_b, (int)k, ws, ws_bytes, &L);
+  if (st != TLS_OK) return st;
+  st = select_blocks_impl(*shape, q, meta, K_b, block_idx, nullptr, (uint8_t*)ws, L, (cudaStream_t)stream);
+  if (st != TLS_OK) return st;
+  return sparse_attn_impl(*shape, q, *kv, nullptr, (int)k, out_dtype, out, lse, (uint8_t*)ws, L,
+                          (cudaStream_t)stream, /*pdl=*/true, kListBlocks, block_idx, K_b);
+}
+
+extern "C" tls_status tls_ds_decode_step(const tls_shape* shape, const void* q, const int32_t* label_ch,
+                                         const uint8_t* codes, const float* scales, const tls_kv_view* kv, int32_t k,
+                                         int32_t* token_idx, int32_t out_dtype, void* out, float* lse, void* ws,
+                                         size_t ws_bytes, void* stream) {
+  clear_error();
+  tls_status st = check_attn_args(shape, q, kv, out_dtype, out, "ds_decode_step");
+  if (st != TLS_OK) return st;
+  if (label_ch == nullptr || codes == nullptr || scales == nullptr || token_idx == nullptr)
+    return fail(TLS_ERR_INVALID_ARG, "ds_decode_step: null pointer");
+  if (!aligned16(codes)) return fail(TLS_ERR_INVALID_ARG, "ds_decode_step: codes not 16-byte aligned");
+  const int nb = (int)n_blocks(*shape);
+  WsLayout L;
+  st = check_ws(*shape, nb, k, ws, ws_bytes, &L);
+  if (st != TLS_OK) return st;
+  st = check_candidates(*shape, nb);
+  if (st != TLS_OK) return st;
+  // level 2 over every block (no list), then the attention over its choice
+  st = select_tokens_impl(*shape, q, label_ch, codes, scales, nullptr, nb, k, token_idx, nullptr, (uint8_t*)ws, L,
+                          (cudaStream_t)stream);
+  if (st != TLS_OK) return st;
+  return sparse_attn_impl(*shape, q, *kv, token_idx, k, out_dtype, out, lse, (uint8_t*)ws, L, (cudaStream_t)stream);
 }

@@ -26,7 +26,38 @@ struct AttnParams {
   void* out;
   int out_bf16;
   float* lse;
+  const int32_t* seq_lens;  // optional [B]: tokens per sequence (later positions are skipped)
+  int list_mode;            // kListTokens, kListAll or kListBlocks
+  const int32_t* blocks;    // kListBlocks: [rows, K_b] block list
+  int K_b;
 };
+
+// Token of entry t (< k_sel) of row `row`'s list, or -1 when the entry is no
+// token of the sequence (padding of a selection, a position >= len).  List
+// reads go through L2: the list may be written by the preceding kernel while
+// this grid is already resident (programmatic dependent launch).
+__device__ __forceinline__ int attn_token(const AttnParams& p, int row, int t, int64_t len) {
+  int64_t tok;
+  if (p.list_mode == kListAll) {
+    tok = t;
+  } else if (p.list_mode == kListBlocks) {
+    const int blk = __ldcg(p.blocks + (int64_t)row * p.K_b + t / p.bs);
+    tok = blk < 0 ? -1 : (int64_t)blk * p.bs + t % p.bs;
+  } else {
+    tok = __ldcg(p.token_idx + (int64_t)row * p.k_sel + t);
+  }
+  return (tok >= 0 && tok < len) ? (int)tok : -1;
+}
+
+// Row id (index of the K/V row) of token `tok` of row `row` (tok >= 0): the
+// dense layout, or its block's slot in the pool (clamped into the pool).
+__device__ __forceinline__ int64_t attn_row_id(const AttnParams& p, int row, int64_t tok) {
+  if (p.slot_of_block != nullptr) {
+    const int64_t slot = min(max(__ldg(p.slot_of_block + (int64_t)row * p.nb + tok / p.bs), 0), p.n_slots - 1);
+    return slot * p.bs + tok % p.bs;
+  }
+  return (int64_t)row * p.ctx_len + tok;
+}
 
 // Owner of work item `item` when CTA c takes items [c*W/n, (c+1)*W/n).
 __host__ __device__ inline int64_t attn_owner(int64_t item, int64_t n_items, int64_t n_ctas) {
@@ -74,7 +105,7 @@ static __device__ __noinline__ void merge_splits(const AttnParams& p, int row, i
         L += f * l[s];
         m[s] = f;
       }
-      const float inv = 1.0f / L;
+      const float inv = L > 0.0f ? 1.0f / L : 0.0f;  // a row with no token: zero output
       for (int s = 0; s < n_splits; ++s) m[s] *= inv;
       m[kMergeMaxSplits] = (M + log2f(L)) * 0.69314718055994531f;
     }

@@ -87,7 +87,8 @@ tls_status plan(const tls_block_cache& c, const int32_t* new_idx, const int32_t*
   for (int r = 0; r < c.rows; ++r) {
     for (int i = 0; i < K_b; ++i) {
       const int32_t blk = new_idx[(int64_t)r * K_b + i];
-      if (blk < 0 || blk >= c.nb) return fail(TLS_ERR_INVALID_ARG, "plan: block %d out of range in row %d", blk, r);
+      if (blk < 0) continue;  // the -1 padding of a sequence with fewer than K_b blocks
+      if (blk >= c.nb) return fail(TLS_ERR_INVALID_ARG, "plan: block %d out of range in row %d", blk, r);
       const int64_t key = (int64_t)r * c.nb + blk;
       if (seen[key]) return fail(TLS_ERR_INVALID_ARG, "plan: block %d repeated in row %d", blk, r);
       seen[key] = 1;
@@ -149,8 +150,9 @@ void commit(tls_block_cache& c, const int32_t* new_idx, int K_b, const std::vect
   }
   for (int r = 0; r < c.rows; ++r)
     for (int i = 0; i < K_b; ++i) {
-      const int32_t s = c.table[(int64_t)r * c.nb + new_idx[(int64_t)r * K_b + i]];
-      c.last_use[s] = c.step;
+      const int32_t blk = new_idx[(int64_t)r * K_b + i];
+      if (blk < 0) continue;
+      c.last_use[c.table[(int64_t)r * c.nb + blk]] = c.step;
     }
 }
 
@@ -225,8 +227,10 @@ tls_status prefetch_diff_impl(tls_block_cache* c, const int32_t* new_idx, const 
   const size_t kblk = (size_t)bs * c->hk_stride * 2, vblk = (size_t)bs * c->hv_stride * 2;
   const bool with_v = c->host_v != nullptr && c->slot_v != nullptr;
   const int b = c->cur;
-  cudaError_t e = cudaEventSynchronize(c->staged[b]);  // the staging buffers' previous use is done
-  if (e != cudaSuccess) return cuda_check(e, "prefetch_diff: staging wait");
+  // the staging buffers' previous use is done
+  st = wait_event_deadline(c->staged[b], host_wait_ms(), "prefetch_diff: staging buffers");
+  if (st != TLS_OK) return st;
+  cudaError_t e = cudaSuccess;
   // from here on device work is queued: a failure leaves the cache failed
   auto queue_failed = [&](const char* what, cudaError_t err) {
     c->failed = TLS_ERR_COPY;

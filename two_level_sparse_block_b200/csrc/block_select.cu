@@ -53,6 +53,9 @@ struct BlockScoreParams {
   unsigned* counters;  // workspace [rows]
   int32_t* block_idx;  // [rows, K_b]
   int* err;            // workspace error word
+  const int32_t* seq_lens;  // optional [B]: tokens per sequence (blocks past them do not compete)
+  int64_t ctx_len;
+  int bs;
 };
 
 __device__ __forceinline__ uint32_t relu_bf16x2(uint32_t w) {
@@ -124,6 +127,9 @@ __global__ void __launch_bounds__(128, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int row = blockIdx.y, mt = blockIdx.x;
   const int nk = (2 * p.dqk) / kBsChunk;
+  // blocks of this row's sequence: only they compete (a suffix of the row)
+  const int nbr = (int)((seq_len_of(p.seq_lens, row / p.n_kv_heads, p.ctx_len) + p.bs - 1) / p.bs);
+  const int kk = min(p.K_b, nbr);  // entries selected; the rest of the list is -1
   constexpr uint32_t kCols = NPAD < 32 ? 32u : (uint32_t)NPAD;
   if constexpr (CL >= 2) cluster_arrive_relaxed();  // completes once every CTA of the cluster has started
   grid_launch_dependents();  // level 2 may be scheduled now; it waits for this grid before reading
@@ -237,7 +243,7 @@ __global__ void __launch_bounds__(128, 1)
     }
     if (j < p.nb) {
       if (CL == 0) p.agg[(int64_t)row * p.nb + j] = best;
-      if (p.block_score != nullptr) p.block_score[(int64_t)row * p.nb + j] = best;
+      if (p.block_score != nullptr) p.block_score[(int64_t)row * p.nb + j] = j < nbr ? best : -INFINITY;
     }
   } else if (lane == 0) {
     report_error(p.err, kErrTimeout, 104);
@@ -264,20 +270,23 @@ __global__ void __launch_bounds__(128, 1)
     uint32_t* keys = reinterpret_cast<uint32_t*>(smem);
     TopkScratch* ts = reinterpret_cast<TopkScratch*>(keys + p.nb);
     const float* arow = p.agg + (int64_t)row * p.nb;
-    for (int i = tid; i < p.nb; i += 128) keys[i] = float_key(__ldcg(arow + i));
+    for (int i = tid; i < nbr; i += 128) keys[i] = float_key(__ldcg(arow + i));
+    pad_list(out, kk, p.K_b);
     __syncthreads();
-    if (p.nb <= 128 * 16) cta_topk_regs<128, 16>(keys, p.nb, p.K_b, out, *ts, [](int i) { return i; });
-    else cta_topk_ascending<128>(keys, p.nb, p.K_b, out, *ts, [](int i) { return i; });
+    if (kk == 0) return;
+    if (nbr <= 128 * 16) cta_topk_regs<128, 16>(keys, nbr, kk, out, *ts, [](int i) { return i; });
+    else cta_topk_ascending<128>(keys, nbr, kk, out, *ts, [](int i) { return i; });
   } else {
     // the drained stages hold the selection: this CTA's keys, then the row's
     uint32_t* mine = reinterpret_cast<uint32_t*>(smem);  // [kBsTile]
     uint32_t* all = mine + kBsTile;                       // [nb]
     TopkScratch* ts = reinterpret_cast<TopkScratch*>(all + p.nb);
-    const int n_loc = min(kBsTile, p.nb - mt * kBsTile);
+    const int n_loc = max(0, min(kBsTile, nbr - mt * kBsTile));  // this CTA's competing blocks
     if (tid < n_loc) mine[tid] = float_key(best);
+    if (mt == 0) pad_list(out, kk, p.K_b);
     __syncthreads();
     if constexpr (CL == 1) {
-      cta_topk_ascending<128>(mine, n_loc, p.K_b, out, *ts, [](int i) { return i; });
+      if (kk > 0) cta_topk_ascending<128>(mine, n_loc, kk, out, *ts, [](int i) { return i; });
     } else {
       // every CTA pushes its keys into the leader's row array; after one
       // cluster barrier the leader selects alone with the keys in registers
@@ -287,8 +296,8 @@ __global__ void __launch_bounds__(128, 1)
       uint32_t* dst = cluster.map_shared_rank(all, 0) + mt * kBsTile;
       if (tid < n_loc) dst[tid] = mine[tid];
       cluster.sync();  // the leader's keys are complete; no remote access after this
-      if (mt != 0) return;
-      cta_topk_regs<128, CL>(all, p.nb, p.K_b, out, *ts, [](int i) { return i; });
+      if (mt != 0 || kk == 0) return;
+      cta_topk_regs<128, CL>(all, nbr, kk, out, *ts, [](int i) { return i; });
     }
   }
 }
@@ -362,6 +371,9 @@ tls_status select_blocks_impl(const tls_shape& s, const void* q, const void* met
   p.counters = reinterpret_cast<unsigned*>(ws + L.blk_counter);
   p.block_idx = block_idx;
   p.err = reinterpret_cast<int*>(ws + L.err);
+  p.seq_lens = s.seq_lens;
+  p.ctx_len = s.ctx_len;
+  p.bs = s.block_size;
 
   tls_status st = get_encoder();
   if (st != TLS_OK) return st;

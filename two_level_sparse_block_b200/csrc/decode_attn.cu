@@ -65,7 +65,7 @@ __global__ void __launch_bounds__(128) sparse_attn_kernel(AttnParams p) {
 
   const int t_begin = split * p.tokens_per_split;
   const int t_end = min(p.k_sel, t_begin + p.tokens_per_split);
-  const int32_t* tix = p.token_idx + (int64_t)row * p.k_sel;
+  const int64_t len = seq_len_of(p.seq_lens, b, p.ctx_len);
   grid_dependency_wait();  // token lists come from the preceding kernel (read through L2)
 
   for (int base = t_begin; base < t_end; base += 8 * U) {
@@ -74,18 +74,13 @@ __global__ void __launch_bounds__(128) sparse_attn_kernel(AttnParams p) {
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int t = base + u * 8 + hw;
-      valid[u] = t < t_end;
+      // entries that are no token of the sequence are skipped, so a bad list
+      // can never address outside the cache
+      const int tok = t < t_end ? attn_token(p, row, t, len) : -1;
+      valid[u] = tok >= 0;
       int64_t krow = 0, vrow = 0;
       if (valid[u]) {
-        // indices are clamped so a bad list can never address outside the cache
-        const int64_t tok = min(max((int64_t)__ldcg(tix + t), (int64_t)0), p.ctx_len - 1);
-        int64_t r;
-        if (p.slot_of_block != nullptr) {
-          const int64_t slot = min(max(p.slot_of_block[(int64_t)row * p.nb + tok / p.bs], 0), p.n_slots - 1);
-          r = slot * p.bs + tok % p.bs;
-        } else {
-          r = (int64_t)row * p.ctx_len + tok;
-        }
+        const int64_t r = attn_row_id(p, row, tok);
         krow = r * p.k_stride;
         vrow = r * p.v_stride;
       }
@@ -224,7 +219,7 @@ tls_status launch_attn(const AttnParams& p, int rows, cudaStream_t stream) {
 
 tls_status sparse_attn_impl(const tls_shape& s, const void* q, const tls_kv_view& kv, const int32_t* token_idx,
                             int k, int out_dtype, void* out, float* lse, uint8_t* ws, const WsLayout& L,
-                            cudaStream_t stream, bool pdl) {
+                            cudaStream_t stream, bool pdl, int list_mode, const int32_t* blocks, int K_b) {
   AttnParams p;
   p.q = (const uint16_t*)q;
   p.k = (const uint16_t*)kv.k;
@@ -257,6 +252,10 @@ tls_status sparse_attn_impl(const tls_shape& s, const void* q, const tls_kv_view
   p.n_items = L.n_items;
   p.n_ctas = L.n_ctas;
   p.err = reinterpret_cast<int*>(ws + L.err);
+  p.seq_lens = s.seq_lens;
+  p.list_mode = list_mode;
+  p.blocks = blocks;
+  p.K_b = K_b;
   const int rows = rows_of(s);
   if (attn_mma_supported(s)) return launch_attn_mma(p, rows, stream, pdl);
   if (attn_mla_supported(s)) return launch_attn_mla(p, rows, stream, pdl);

@@ -105,16 +105,11 @@ __device__ __forceinline__ void mla_issue(const AttnParams& p, int64_t rid, uint
   }
 }
 
-// Row id (index into the K/V rows) of list entry t of the row, t < k.
-__device__ __forceinline__ int64_t mla_rid(const AttnParams& p, int row, int t) {
-  // L2 load: the list is written by the preceding kernel while this grid is
-  // already resident (programmatic dependent launch)
-  const int64_t tk = min(max((int64_t)__ldcg(p.token_idx + (int64_t)row * p.k_sel + t), (int64_t)0), p.ctx_len - 1);
-  if (p.slot_of_block != nullptr) {
-    const int64_t slot = min(max(__ldg(p.slot_of_block + (int64_t)row * p.nb + tk / p.bs), 0), p.n_slots - 1);
-    return slot * p.bs + tk % p.bs;
-  }
-  return (int64_t)row * p.ctx_len + tk;
+// Row id (index into the K/V rows) of list entry t of the row (t < k), or -1
+// when the entry is no token of the sequence (len tokens).
+__device__ __forceinline__ int64_t mla_rid(const AttnParams& p, int row, int t, int64_t len) {
+  const int tok = attn_token(p, row, t, len);
+  return tok < 0 ? (int64_t)-1 : attn_row_id(p, row, tok);
 }
 
 template <int NS>
@@ -157,13 +152,23 @@ __global__ void __launch_bounds__(kMlaWarps * 32, 2) sparse_attn_mla_kernel(Attn
       qa[ks][3] = *reinterpret_cast<const uint32_t*>(q8 + d0 + 8);
     }
   }
+  const int64_t len = seq_len_of(p.seq_lens, b, p.ctx_len);
   grid_dependency_wait();  // token lists come from the preceding kernel
-  // the row ids of this split's entries, padded with -1 (zero-fill) to whole
-  // chunks: one round trip to the list now instead of one per chunk in the loop
+  // a token list: the row ids of this split's entries, padded with -1
+  // (zero-fill) to whole chunks -- one round trip to the list now instead of
+  // one per chunk in the loop; other lists are computed where they are used
   int64_t* srid = reinterpret_cast<int64_t*>(sm + kMlaOffRid);
-  for (int i = tid; i < n_chunks * kMlaChunk; i += kMlaWarps * 32)
-    srid[i] = t_lo + i < t_hi ? mla_rid(p, row, t_lo + i) : (int64_t)-1;
-  __syncthreads();
+  const bool staged = p.list_mode == kListTokens;
+  if (staged) {
+    for (int i = tid; i < n_chunks * kMlaChunk; i += kMlaWarps * 32)
+      srid[i] = t_lo + i < t_hi ? mla_rid(p, row, t_lo + i, len) : (int64_t)-1;
+    __syncthreads();
+  }
+  // row id of entry i of this split (-1: no token, rows zero-filled and masked)
+  auto rid_at = [&](int i) -> int64_t {
+    if (staged) return srid[i];
+    return t_lo + i < t_hi ? mla_rid(p, row, t_lo + i, len) : (int64_t)-1;
+  };
 
   float o[16][4];
 #pragma unroll
@@ -172,7 +177,7 @@ __global__ void __launch_bounds__(kMlaWarps * 32, 2) sparse_attn_mla_kernel(Attn
 
 #pragma unroll
   for (int s = 0; s < NS - 1; ++s) {
-    if (s < n_chunks) mla_issue(p, srid[s * kMlaChunk + (lane & 15)], ring + s * kMlaStageBytes);
+    if (s < n_chunks) mla_issue(p, rid_at(s * kMlaChunk + (lane & 15)), ring + s * kMlaStageBytes);
     cp_async_commit();
   }
   for (int c = 0; c < n_chunks; ++c) {
@@ -180,11 +185,12 @@ __global__ void __launch_bounds__(kMlaWarps * 32, 2) sparse_attn_mla_kernel(Attn
     __syncthreads();          // everyone's have; every warp is past chunk c - 1
     {
       const int cn = c + NS - 1;  // refill the stage chunk c - 1 used
-      if (cn < n_chunks) mla_issue(p, srid[cn * kMlaChunk + (lane & 15)], ring + (cn % NS) * kMlaStageBytes);
+      if (cn < n_chunks) mla_issue(p, rid_at(cn * kMlaChunk + (lane & 15)), ring + (cn % NS) * kMlaStageBytes);
       cp_async_commit();
     }
     const uint32_t st = ring + (c % NS) * kMlaStageBytes;
-    const int t_base = t_lo + c * kMlaChunk;
+    // the chunk's entries that are tokens (bit e: entry e)
+    const uint32_t vm = __ballot_sync(0xffffffffu, rid_at(c * kMlaChunk + (lane & 15)) >= 0) & 0xFFFFu;
 
     // partial S over this warp's 144 dims: 16 heads x 16 tokens
     float s[2][4];
@@ -225,12 +231,12 @@ __global__ void __launch_bounds__(kMlaWarps * 32, 2) sparse_attn_mla_kernel(Attn
         for (int w = 0; w < kMlaWarps; ++w) v += sS[((c & 1) * kMlaWarps + w) * 256 + (nt * 4 + e) * 32 + lane];
         s[nt][e] = v * p.scale_log2;
       }
-    if (t_base + kMlaChunk > t_hi) {
+    if (vm != 0xFFFFu) {
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          if (t_base + nt * 8 + 2 * tq + (e & 1) >= t_hi) s[nt][e] = -INFINITY;
+          if (!((vm >> (nt * 8 + 2 * tq + (e & 1))) & 1u)) s[nt][e] = -INFINITY;
     }
     // online softmax (rows gq: elements 0, 1; rows gq + 8: elements 2, 3)
     float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
@@ -241,7 +247,8 @@ __global__ void __launch_bounds__(kMlaWarps * 32, 2) sparse_attn_mla_kernel(Attn
     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
     const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
     if (!__all_sync(0xffffffffu, n0 == m0 && n1 == m1)) {
-      const float c0 = mla_exp2(m0 - n0), c1 = mla_exp2(m1 - n1);
+      // 1 where the maximum did not move (also while a row has seen no token)
+      const float c0 = n0 == m0 ? 1.0f : mla_exp2(m0 - n0), c1 = n1 == m1 ? 1.0f : mla_exp2(m1 - n1);
       l0 *= c0;
       l1 *= c1;
 #pragma unroll
@@ -254,11 +261,13 @@ __global__ void __launch_bounds__(kMlaWarps * 32, 2) sparse_attn_mla_kernel(Attn
       m0 = n0;
       m1 = n1;
     }
+    // a row with no token so far keeps max -inf: its masked scores give 0
+    const float z0 = n0 == -INFINITY ? 0.0f : n0, z1 = n1 == -INFINITY ? 0.0f : n1;
     float pr[2][4];
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) pr[nt][e] = mla_exp2(s[nt][e] - (e < 2 ? n0 : n1));
+      for (int e = 0; e < 4; ++e) pr[nt][e] = mla_exp2(s[nt][e] - (e < 2 ? z0 : z1));
     l0 += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
     l1 += (pr[0][2] + pr[0][3]) + (pr[1][2] + pr[1][3]);
     uint32_t ph[4], pl[4];
@@ -361,7 +370,8 @@ int attn_mla_tokens_per_split(int k) {
 }
 
 tls_status launch_attn_mla(const AttnParams& p, int rows, cudaStream_t stream, bool pdl) {
-  const size_t smem = 128 + (size_t)kMlaSmem + (size_t)p.tokens_per_split * 8;
+  // staged row ids only for a token list
+  const size_t smem = 128 + (size_t)kMlaSmem + (p.list_mode == kListTokens ? (size_t)p.tokens_per_split * 8 : 0);
   cudaError_t e = kernel_attrs((const void*)sparse_attn_mla_kernel<kMlaStages>, smem);
   if (e != cudaSuccess) return cuda_check(e, "sparse_decode_attn: set smem attribute");
   const dim3 grid(kMlaSplits, (unsigned)(p.group / kMlaHeads), (unsigned)rows);

@@ -106,31 +106,26 @@ __device__ __forceinline__ void mma_load_q(const AttnParams& p, int b, int kvh, 
   }
 }
 
-// Raw token index of entry (lane & 15) of chunk x of the row's list, or -1
-// past the end of the list.
-__device__ __forceinline__ int mma_chunk_token(const AttnParams& p, int row, int x, int lane) {
+// Token of entry (lane & 15) of chunk x of the row's list, or -1 past the end
+// of the list or when the entry is no token of the sequence (len tokens).
+__device__ __forceinline__ int mma_chunk_token(const AttnParams& p, int row, int x, int lane, int64_t len) {
   const int t = x * kChunk + (lane & 15);
   if (t >= p.k_sel) return -1;
-  // L2 load: the list is written by the preceding kernel while this grid is
-  // already resident (programmatic dependent launch)
-  return __ldcg(p.token_idx + (int64_t)row * p.k_sel + t);
+  return attn_token(p, row, t, len);
+}
+
+// The chunk's 16 entries that are tokens (bit e: entry e), from the lane
+// values of mma_chunk_token; all lanes of the warp call it.
+__device__ __forceinline__ uint32_t mma_valid_mask(int tok) {
+  return __ballot_sync(0xffffffffu, tok >= 0) & 0xFFFFu;
 }
 
 // cp.async of the K and V rows of one chunk into the ring stage at shared
-// address kb (K tile; V tile at kb + 4096).  Entry lane & 15 holds raw token
-// `tok` (-1: the rows are zero-filled); tokens are clamped to the context and
-// slots to the pool.  The caller commits the group.
+// address kb (K tile; V tile at kb + 4096).  Entry lane & 15 holds token
+// `tok` (-1: the rows are zero-filled and the scores masked); slots are
+// clamped to the pool.  The caller commits the group.
 __device__ __forceinline__ void mma_issue_rows(const AttnParams& p, int row, int tok, uint32_t kb, int lane) {
-  int64_t rid = -1;
-  if (tok >= 0) {
-    const int64_t tk = min(max((int64_t)tok, (int64_t)0), p.ctx_len - 1);
-    if (p.slot_of_block != nullptr) {
-      const int64_t slot = min(max(__ldg(p.slot_of_block + (int64_t)row * p.nb + tk / p.bs), 0), p.n_slots - 1);
-      rid = slot * p.bs + tk % p.bs;
-    } else {
-      rid = (int64_t)row * p.ctx_len + tk;
-    }
-  }
+  const int64_t rid = tok >= 0 ? attn_row_id(p, row, tok) : -1;
   const uint32_t vb = kb + 4096;
   const int c = lane & 15;
 #pragma unroll
@@ -144,12 +139,13 @@ __device__ __forceinline__ void mma_issue_rows(const AttnParams& p, int row, int
   }
 }
 
-// One chunk of 16 tokens (list positions t_base ..) for the fragment rows gq
-// (m0, l0) and gq + 8 (m1, l1): S = Q.K^T scaled to base 2 and masked past the
-// list end, the online softmax update, and O += P.V with P split into bf16
-// hi + lo parts.  K and V tiles of the chunk at shared address kb / kb + 4096.
+// One chunk of 16 list entries for the fragment rows gq (m0, l0) and gq + 8
+// (m1, l1): S = Q.K^T scaled to base 2 and masked where the entry is no token
+// (bit e of vm clear: past the list end, or padding), the online softmax
+// update, and O += P.V with P split into bf16 hi + lo parts.  K and V tiles
+// of the chunk at shared address kb / kb + 4096.
 __device__ __forceinline__ void mma_chunk(const AttnParams& p, const uint32_t (&qa)[8][4], float (&o)[16][4],
-                                          float& m0, float& m1, float& l0, float& l1, uint32_t kb, int t_base,
+                                          float& m0, float& m1, float& l0, float& l1, uint32_t kb, uint32_t vm,
                                           int lane) {
   const int tq = lane & 3;
   const uint32_t vb = kb + 4096;
@@ -175,12 +171,12 @@ __device__ __forceinline__ void mma_chunk(const AttnParams& p, const uint32_t (&
   for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
     for (int e = 0; e < 4; ++e) s[nt][e] *= p.scale_log2;
-  if (t_base + kChunk > p.k_sel) {
+  if (vm != 0xFFFFu) {
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e)
-        if (t_base + nt * 8 + 2 * tq + (e & 1) >= p.k_sel) s[nt][e] = -INFINITY;
+        if (!((vm >> (nt * 8 + 2 * tq + (e & 1))) & 1u)) s[nt][e] = -INFINITY;
   }
   float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
   float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
@@ -191,7 +187,9 @@ __device__ __forceinline__ void mma_chunk(const AttnParams& p, const uint32_t (&
   const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
   // the O rescale is skipped (warp-uniformly) when no row maximum moved
   if (!__all_sync(0xffffffffu, n0 == m0 && n1 == m1)) {
-    const float c0 = fast_exp2(m0 - n0), c1 = fast_exp2(m1 - n1);  // 0 on the first chunk
+    // 0 on a row's first token; 1 where the maximum did not move (also while
+    // a row has seen no token at all: both -inf)
+    const float c0 = n0 == m0 ? 1.0f : fast_exp2(m0 - n0), c1 = n1 == m1 ? 1.0f : fast_exp2(m1 - n1);
     l0 *= c0;
     l1 *= c1;
 #pragma unroll
@@ -204,11 +202,13 @@ __device__ __forceinline__ void mma_chunk(const AttnParams& p, const uint32_t (&
     m0 = n0;
     m1 = n1;
   }
+  // a row with no token so far keeps max -inf: its masked scores give 2^-inf = 0
+  const float z0 = n0 == -INFINITY ? 0.0f : n0, z1 = n1 == -INFINITY ? 0.0f : n1;
   float pr[2][4];
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) pr[nt][e] = fast_exp2(s[nt][e] - (e < 2 ? n0 : n1));
+    for (int e = 0; e < 4; ++e) pr[nt][e] = fast_exp2(s[nt][e] - (e < 2 ? z0 : z1));
   l0 += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
   l1 += (pr[0][2] + pr[0][3]) + (pr[1][2] + pr[1][3]);
   // P as the A operand (k = the 16 tokens), hi and lo parts
@@ -321,7 +321,8 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_kernel(Attn
   auto load_tok = [&](int i) -> int {
     if (i >= n_mine) return -1;
     const int64_t x = x0 + (int64_t)kMmaWarps * i;
-    return mma_chunk_token(p, (int)(x / CPR) / HG, (int)(x % CPR), lane);
+    const int r = (int)(x / CPR) / HG;
+    return mma_chunk_token(p, r, (int)(x % CPR), lane, seq_len_of(p.seq_lens, r / p.n_kv_heads, p.ctx_len));
   };
   auto issue = [&](int i, int tok, int st) {
     if (i < n_mine)
@@ -348,12 +349,17 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_kernel(Attn
   }
   grid_dependency_wait();  // token lists come from the preceding kernel
 
-  // prologue: stages 0 .. S-2; token indices one chunk further ahead
+  // prologue: stages 0 .. S-2; token indices one chunk further ahead; vq
+  // queues the issued chunks' token masks, 16 bits each, oldest lowest
   int tok_ahead[NS];
 #pragma unroll
   for (int s = 0; s < NS; ++s) tok_ahead[s] = load_tok(s);
+  uint64_t vq = 0;
 #pragma unroll
-  for (int s = 0; s < NS - 1; ++s) issue(s, tok_ahead[s], s);
+  for (int s = 0; s < NS - 1; ++s) {
+    issue(s, tok_ahead[s], s);
+    vq |= (uint64_t)mma_valid_mask(tok_ahead[s]) << (16 * s);
+  }
   int tok_next = tok_ahead[NS - 1];  // for chunk S-1
 
   const int vrow_first = (int)(c_lo / CPR);
@@ -374,11 +380,13 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_kernel(Attn
       // keep S-1 chunks in flight; indices run one chunk further ahead
       const int tok_after = load_tok(i + NS);
       issue(i + NS - 1, tok_next, (i + NS - 1) % NS);
+      vq |= (uint64_t)mma_valid_mask(tok_next) << (16 * (NS - 1));
       tok_next = tok_after;
       cp_async_wait<NS - 1>();
       __syncwarp();
-      const int64_t x = x0 + (int64_t)kMmaWarps * i;
-      mma_chunk(p, qa, o, m0, m1, l0, l1, ring_s + (i % NS) * kChunkBytes, (int)(x % CPR) * kChunk, lane);
+      const uint32_t vm = (uint32_t)(vq & 0xFFFFu);
+      vq >>= 16;
+      mma_chunk(p, qa, o, m0, m1, l0, l1, ring_s + (i % NS) * kChunkBytes, vm, lane);
       __syncwarp();
     }
 
@@ -430,7 +438,10 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_cluster_ker
   const uint32_t ring_s = smem_u32(sm + warp * NS * kChunkBytes);
   const int x0 = c_lo + warp;
   const int n_mine = x0 < c_hi ? (c_hi - 1 - x0) / kMmaWarps + 1 : 0;
-  auto load_tok = [&](int i) -> int { return i < n_mine ? mma_chunk_token(p, row, x0 + kMmaWarps * i, lane) : -1; };
+  const int64_t len = seq_len_of(p.seq_lens, b, p.ctx_len);
+  auto load_tok = [&](int i) -> int {
+    return i < n_mine ? mma_chunk_token(p, row, x0 + kMmaWarps * i, lane, len) : -1;
+  };
   auto issue = [&](int i, int tok, int st) {
     if (i < n_mine) mma_issue_rows(p, row, tok, ring_s + st * kChunkBytes, lane);
     cp_async_commit();
@@ -454,16 +465,23 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_cluster_ker
   int tok_ahead[NS];
 #pragma unroll
   for (int s = 0; s < NS; ++s) tok_ahead[s] = load_tok(s);
+  uint64_t vq = 0;  // token masks of the issued chunks, 16 bits each, oldest lowest
 #pragma unroll
-  for (int s = 0; s < NS - 1; ++s) issue(s, tok_ahead[s], s);
+  for (int s = 0; s < NS - 1; ++s) {
+    issue(s, tok_ahead[s], s);
+    vq |= (uint64_t)mma_valid_mask(tok_ahead[s]) << (16 * s);
+  }
   int tok_next = tok_ahead[NS - 1];
   for (int i = 0; i < n_mine; ++i) {
     const int tok_after = load_tok(i + NS);
     issue(i + NS - 1, tok_next, (i + NS - 1) % NS);
+    vq |= (uint64_t)mma_valid_mask(tok_next) << (16 * (NS - 1));
     tok_next = tok_after;
     cp_async_wait<NS - 1>();
     __syncwarp();
-    mma_chunk(p, qa, o, m0, m1, l0, l1, ring_s + (i % NS) * kChunkBytes, (x0 + kMmaWarps * i) * kChunk, lane);
+    const uint32_t vm = (uint32_t)(vq & 0xFFFFu);
+    vq >>= 16;
+    mma_chunk(p, qa, o, m0, m1, l0, l1, ring_s + (i % NS) * kChunkBytes, vm, lane);
     __syncwarp();
   }
   cp_async_wait<0>();

@@ -26,6 +26,21 @@ __device__ __forceinline__ void report_error(int* err, int code, int where) {
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+// Tokens sequence b holds: seq_lens[b] clamped into [0, cap], or cap when
+// there is no length array.  Read through L2 (an earlier kernel of the stream
+// may have written it).
+__device__ __forceinline__ int64_t seq_len_of(const int32_t* seq_lens, int b, int64_t cap) {
+  if (seq_lens == nullptr) return cap;
+  const int64_t v = __ldcg(seq_lens + b);
+  return v < 0 ? 0 : (v > cap ? cap : v);
+}
+
+// -1 into out[from, to) (the padding of a selection with fewer valid entries
+// than asked for); all threads of the CTA may call it.
+__device__ __forceinline__ void pad_list(int32_t* out, int from, int to) {
+  for (int i = from + (int)threadIdx.x; i < to; i += (int)blockDim.x) out[i] = -1;
+}
+
 __device__ __forceinline__ uint64_t global_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));

@@ -30,15 +30,6 @@
 
 namespace tls {
 tls_status plan_workspace(const tls_shape& s, int K_b, int k, WsLayout* out);
-tls_status select_blocks_impl(const tls_shape& s, const void* q, const void* meta, int K_b, int32_t* block_idx,
-                              float* block_score, uint8_t* ws, const WsLayout& L, cudaStream_t stream);
-tls_status select_tokens_impl(const tls_shape& s, const void* q, const int32_t* label_ch, const uint8_t* codes,
-                              const float* scales, const int32_t* block_idx, int K_b, int k, int32_t* token_idx,
-                              float* token_score, uint8_t* ws, const WsLayout& L, cudaStream_t stream,
-                              bool pdl = false, bool lean = false);
-tls_status sparse_attn_impl(const tls_shape& s, const void* q, const tls_kv_view& kv, const int32_t* token_idx,
-                            int k, int out_dtype, void* out, float* lse, uint8_t* ws, const WsLayout& L,
-                            cudaStream_t stream, bool pdl = true);
 tls_status prefetch_diff_impl(tls_block_cache* c, const int32_t* new_idx, const int32_t* in_use, int K_b,
                               cudaStream_t cs, int32_t* n_copied, int64_t* bytes);
 tls_status block_cache_view(const tls_block_cache* c, tls_kv_view* kv);
@@ -69,6 +60,7 @@ struct tls_engine {
   int64_t bytes[kRing] = {};
   int64_t t = 0;
   tls_status failed = TLS_OK;
+  double wait_ms = 10000.0;  // deadline of the host waits (TLS_HOST_WAIT_MS)
 };
 
 using namespace tls;
@@ -132,6 +124,7 @@ tls_status engine_create(const tls_shape* shape, int32_t K_b, int32_t k, const v
   e->kv = kv;
   e->ws = (uint8_t*)ws;
   e->L = L;
+  e->wait_ms = host_wait_ms();
   e->bidx[0] = block_idx;
   e->bidx[1] = block_idx + (size_t)e->rows * K_b;
   e->token_idx = token_idx;
@@ -239,8 +232,11 @@ tls_status engine_step(tls_engine* e, const void* q, int32_t out_dtype, void* ou
     st = select_blocks_impl(s, q, e->meta, e->K_b, e->bidx[prev], nullptr, e->ws, e->L, A);
     if (st != TLS_OK) return st;
     cudaError_t ce = cudaMemcpyAsync(e->host_bidx[prev], e->bidx[prev], list_bytes, cudaMemcpyDeviceToHost, A);
-    if (ce == cudaSuccess) ce = cudaStreamSynchronize(A);
-    if (ce == cudaSuccess) ce = cudaEventRecord(e->copy_start[rp], e->copy);
+    if (ce == cudaSuccess) ce = cudaEventRecord(e->ev_sel, A);
+    if (ce != cudaSuccess) return cuda_check(ce, "engine_step: prologue");
+    st = wait_event_deadline(e->ev_sel, e->wait_ms, "engine_step: prologue block list");
+    if (st != TLS_OK) return st;
+    ce = cudaEventRecord(e->copy_start[rp], e->copy);
     if (ce != cudaSuccess) return cuda_check(ce, "engine_step: prologue");
     st = prefetch_diff_impl(e->cache, e->host_bidx[prev], nullptr, e->K_b, e->copy, &e->n_copied[rp], &e->bytes[rp]);
     if (st != TLS_OK) return st;
@@ -270,8 +266,10 @@ tls_status engine_step(tls_engine* e, const void* q, int32_t out_dtype, void* ou
   ce = cudaEventRecord(e->ev_attn[cur], A);
   // T_t = M_t \ C_t on the copy stream, after the attention of step t-1 (its
   // slots may be evicted now), alongside the attention of step t
-  if (ce == cudaSuccess) ce = cudaEventSynchronize(e->ev_sel);
-  if (ce == cudaSuccess) ce = cudaStreamWaitEvent(e->copy, e->ev_attn[prev], 0);
+  if (ce != cudaSuccess) return cuda_check(ce, "engine_step: attention event");
+  st = wait_event_deadline(e->ev_sel, e->wait_ms, "engine_step: level 1 of this step");
+  if (st != TLS_OK) return st;
+  ce = cudaStreamWaitEvent(e->copy, e->ev_attn[prev], 0);
   if (ce == cudaSuccess) ce = cudaEventRecord(e->copy_start[ri], e->copy);
   if (ce != cudaSuccess) return cuda_check(ce, "engine_step: copy stream");
   st = prefetch_diff_impl(e->cache, e->host_bidx[cur], e->host_bidx[prev], e->K_b, e->copy, &e->n_copied[ri],
@@ -316,13 +314,15 @@ extern "C" tls_status tls_engine_stats(tls_engine* e, int64_t step, tls_engine_s
     return TLS_OK;
   }
   const int si = (int)((step + kRing) % kRing);
-  cudaError_t ce = cudaEventSynchronize(e->copy_end[si]);
+  tls_status st = wait_event_deadline(e->copy_end[si], e->wait_ms, "engine_stats: transfer");
+  if (st != TLS_OK) return st;
   float copy_ms = 0.0f, exposed_ms = -1.0f;
-  if (ce == cudaSuccess) ce = cudaEventElapsedTime(&copy_ms, e->copy_start[si], e->copy_end[si]);
+  cudaError_t ce = cudaEventElapsedTime(&copy_ms, e->copy_start[si], e->copy_end[si]);
   if (ce == cudaSuccess && step + 1 < e->t) {
     const int ni = (int)((step + 1) % kRing);
-    ce = cudaEventSynchronize(e->ready[ni]);
-    if (ce == cudaSuccess) ce = cudaEventElapsedTime(&exposed_ms, e->ready[ni], e->copy_end[si]);
+    st = wait_event_deadline(e->ready[ni], e->wait_ms, "engine_stats: next step");
+    if (st != TLS_OK) return st;
+    ce = cudaEventElapsedTime(&exposed_ms, e->ready[ni], e->copy_end[si]);
     if (exposed_ms < 0.0f) exposed_ms = 0.0f;
   }
   if (ce != cudaSuccess) return cuda_check(ce, "engine_stats: events");

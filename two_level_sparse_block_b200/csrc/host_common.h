@@ -25,6 +25,9 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 tls_status check_shape(const tls_shape* s);
 
 inline int64_t n_blocks(const tls_shape& s) { return s.ctx_len / s.block_size; }
+// Largest candidate count of level 2 (K_b * bs) and list length of the attention.
+constexpr int64_t kMaxCandidates = (int64_t)1 << 19;
+constexpr int64_t kMaxListLen = (int64_t)1 << 24;
 inline int rows_of(const tls_shape& s) { return s.batch * s.n_kv_heads; }
 inline int group_of(const tls_shape& s) { return s.n_q_heads / s.n_kv_heads; }
 // Heads of a KV group padded to the level-1 GEMM's N (16, 32, 64, 128 or 256).
@@ -39,6 +42,15 @@ inline tls_status cuda_check(cudaError_t e, const char* what) {
 inline tls_status launch_check(const char* what) { return cuda_check(cudaGetLastError(), what); }
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Host waits with a deadline.  wait_event_deadline polls cudaEventQuery,
+// yielding the thread between polls, until the event has completed
+// (TLS_OK), the runtime reports an error (TLS_ERR_CUDA) or timeout_ms have
+// passed (TLS_ERR_TIMEOUT; the device work it waited for keeps running and
+// completes on its own).  host_wait_ms: the deadline the library's host waits
+// use, TLS_HOST_WAIT_MS from the environment when set (> 0), else 10 s.
+tls_status wait_event_deadline(cudaEvent_t ev, double timeout_ms, const char* what);
+double host_wait_ms();
 
 // Workspace layout shared by the selection and attention entry points.
 struct WsLayout {
@@ -66,6 +78,30 @@ tls_status noalloc_scratch(void** out);
 tls_status plan_workspace(const tls_shape& s, int K_b, int k, WsLayout* out);
 
 constexpr int kNumSMs = 148;
+
+// Where entry t of a row's attention list comes from: the token list
+// (token_idx), every position in order (t itself: full attention), or the
+// tokens of a block list in order (blocks[t / bs] * bs + t % bs: block
+// selection alone).
+enum { kListTokens = 0, kListAll = 1, kListBlocks = 2 };
+
+// The launch paths behind the entry points (arguments already checked).
+// Level 1: scores and top-K_b of every row into block_idx.
+tls_status select_blocks_impl(const tls_shape& s, const void* q, const void* meta, int K_b, int32_t* block_idx,
+                              float* block_score, uint8_t* ws, const WsLayout& L, cudaStream_t stream);
+// Level 2 within block_idx (NULL: every block, K_b = NB).  `lean`: on at most
+// half the SMs (beside a level-1 grid); `pdl`: launched as a programmatic
+// dependent of the stream's preceding kernel.
+tls_status select_tokens_impl(const tls_shape& s, const void* q, const int32_t* label_ch, const uint8_t* codes,
+                              const float* scales, const int32_t* block_idx, int K_b, int k, int32_t* token_idx,
+                              float* token_score, uint8_t* ws, const WsLayout& L, cudaStream_t stream,
+                              bool pdl = false, bool lean = false);
+// Attention over k list entries per row; list_mode 0: token_idx, 1: every
+// position (full attention), 2: the tokens of the block list `blocks` [rows, K_b].
+tls_status sparse_attn_impl(const tls_shape& s, const void* q, const tls_kv_view& kv, const int32_t* token_idx,
+                            int k, int out_dtype, void* out, float* lse, uint8_t* ws, const WsLayout& L,
+                            cudaStream_t stream, bool pdl = true, int list_mode = 0, const int32_t* blocks = nullptr,
+                            int K_b = 0);
 
 // Launches `kernel` with programmatic stream serialization: it may start while
 // the preceding kernel of the stream finishes, and must call

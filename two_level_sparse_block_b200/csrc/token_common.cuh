@@ -19,6 +19,7 @@ struct TokenParams {
   float* token_score;   // optional copy
   unsigned* counters;   // workspace [rows]
   int32_t* token_idx;   // [rows, k]
+  const int32_t* seq_lens;  // optional [B]: tokens per sequence (later positions are not candidates)
 };
 
 template <int R>
@@ -82,21 +83,48 @@ __device__ __forceinline__ void load_qlab(const TokenParams& p, int row, float* 
 }
 
 // The row's chosen blocks, clamped into [0, NB) so a bad list can never
-// address outside the index, copied to shared memory.
+// address outside the index, copied to shared memory (block_idx NULL: every
+// block, 0 .. K_b - 1).  Returns how many entries are blocks (not the -1 that
+// ends a list); every thread of the CTA must call it, and it ends with a CTA
+// barrier, after which sb is complete.
 template <int NT>
-__device__ __forceinline__ void load_block_list(const TokenParams& p, int row, int32_t* sb) {
-  // L2 loads: the list is written by the preceding kernel while this grid may
-  // already be resident (programmatic dependent launch)
-  for (int i = threadIdx.x; i < p.K_b; i += NT)
-    sb[i] = min(max(__ldcg(p.block_idx + (int64_t)row * p.K_b + i), 0), p.nb - 1);
+__device__ __forceinline__ int load_block_list(const TokenParams& p, int row, int32_t* sb) {
+  int nvb = 0;
+  for (int base = 0; base < p.K_b; base += NT) {
+    const int i = base + (int)threadIdx.x;
+    bool valid = false;
+    if (i < p.K_b) {
+      // L2 loads: the list is written by the preceding kernel while this grid
+      // may already be resident (programmatic dependent launch)
+      const int v = p.block_idx == nullptr ? i : __ldcg(p.block_idx + (int64_t)row * p.K_b + i);
+      valid = v >= 0;
+      sb[i] = min(max(v, 0), p.nb - 1);
+    }
+    nvb += __syncthreads_count(valid);
+  }
+  return nvb;
+}
+
+// Candidates of a row that are tokens of its sequence: the lists are
+// ascending with any -1 at the end and only the sequence's last block can be
+// partial, so they are a prefix of the candidate order -- every position of
+// the nvb listed blocks, less the part of the highest one past the sequence.
+__device__ __forceinline__ int valid_candidates(const TokenParams& p, int row, const int32_t* sb, int nvb) {
+  if (nvb <= 0) return 0;
+  const int64_t len = seq_len_of(p.seq_lens, row / p.n_kv_heads, p.ctx_len);
+  const int64_t all = (int64_t)nvb * p.bs;
+  const int64_t end = (int64_t)(sb[nvb - 1] + 1) * p.bs;  // one past the highest listed block
+  const int64_t n = all - (end > len ? end - len : 0);
+  return (int)(n < 0 ? 0 : n);
 }
 
 // Scores of candidates [c0, c1) of one row (candidates in ascending token
 // order), score(t) = s_t * max_h sum_r qlab[h, r] * code_{t, r}, stored as
-// order-preserving keys at keys[i - c0].
+// order-preserving keys at keys[i - c0] (n_valid: candidates that are tokens
+// of the sequence; the optional score copy gets -inf past them).
 template <int R, int NT>
 __device__ __forceinline__ void score_candidates(const TokenParams& p, int row, const float* qlab,
-                                                 const int32_t* bidx, int c0, int c1, uint32_t* keys) {
+                                                 const int32_t* bidx, int c0, int c1, uint32_t* keys, int n_valid) {
   constexpr int U = 4;  // candidates per thread whose loads are in flight together
   const int g = p.group;
   const int tid = threadIdx.x;
@@ -126,7 +154,7 @@ __device__ __forceinline__ void score_candidates(const TokenParams& p, int row, 
         }
         const float score = sc[u] * best;
         keys[i - c0] = float_key(score);
-        if (p.token_score != nullptr) p.token_score[(int64_t)row * p.n_cand + i] = score;
+        if (p.token_score != nullptr) p.token_score[(int64_t)row * p.n_cand + i] = i < n_valid ? score : -INFINITY;
       }
     }
   }
@@ -195,7 +223,7 @@ __device__ __forceinline__ void tok_mma(float (&d)[4], const uint32_t (&a)[4], u
 template <int R, int NT, int NTILE, bool STAGED = false>
 __device__ __forceinline__ void score_candidates_tc(const TokenParams& p, int row, const float* qlab,
                                                     const int32_t* bidx, int c0, int c1, uint32_t* keys,
-                                                    const uint8_t* scodes = nullptr,
+                                                    int n_valid, const uint8_t* scodes = nullptr,
                                                     const float* sscales = nullptr) {
   static_assert(R == 16 || R == 32, "label channels for the tensor-core scorer");
   constexpr int KS = R / 16, NW = NT / 32;
@@ -288,7 +316,8 @@ __device__ __forceinline__ void score_candidates_tc(const TokenParams& p, int ro
           const int i = base + gq + 8 * hlf;
           const float score = sc[u][hlf] * (hlf == 0 ? mx0 : mx1);
           keys[i - c0] = float_key(score);
-          if (p.token_score != nullptr) p.token_score[(int64_t)row * p.n_cand + i] = score;
+          if (p.token_score != nullptr)
+            p.token_score[(int64_t)row * p.n_cand + i] = i < n_valid ? score : -INFINITY;
         }
       }
     }
@@ -314,11 +343,22 @@ __host__ __device__ inline int token_row_cluster_size(int rows, int K_b, int max
 
 // CTAs per row of the cluster kernel: 4, or (tensor-core scoring only) 8 / 16
 // while the rows leave most SMs idle and every CTA keeps 512 candidates or more.
+// Rows whose candidates exceed 4 * kTokMaxPerCta take more CTAs still (up to
+// 16), so that a CTA's keys stay within kTokMaxPerCta.
+constexpr int kTokMaxPerCta = 8192;
 __host__ __device__ inline int token_cluster_size(int rows, int n_cand, bool tc) {
   int cl = 4;
   while (tc && cl < 16 && (int64_t)rows * cl * 2 <= 148 && n_cand >= cl * 2 * 512) cl *= 2;
+  while (cl < 16 && n_cand > cl * kTokMaxPerCta) cl *= 2;
   return cl;
 }
+
+// Candidates per row above which the cluster kernel's degenerate fallback
+// gathers the keys in the workspace instead of the leader's shared memory, and
+// above which the chunked kernel (all keys of a row in one CTA) is not used.
+constexpr int kTokSmemKeysMax = 24576;
+// Largest candidate count level 2 takes (16 CTAs of 4 * kTokMaxPerCta keys).
+constexpr int kTokMaxCand = 16 * 4 * kTokMaxPerCta;
 
 // Whether level 2 of a row is light enough for one 4-CTA cluster (the
 // scores of all candidates in shared memory, no device-wide exchange).

@@ -31,27 +31,24 @@ namespace tls {
 template <int R, int NT>
 __global__ void __launch_bounds__(NT) token_select_kernel(TokenParams p) {
   extern __shared__ float sm[];
-  float* qlab = sm;  // [G][R]
+  float* qlab = sm;                                                 // [G][R]
+  int32_t* sb = reinterpret_cast<int32_t*>(sm + p.group * R);       // [K_b]
+  uint32_t* keys = reinterpret_cast<uint32_t*>(sb + p.K_b);         // [n_cand] (last CTA)
+  TopkScratch* ts = reinterpret_cast<TopkScratch*>(
+      (reinterpret_cast<uintptr_t>(keys + p.n_cand) + 15) & ~uintptr_t(15));
   __shared__ int last;
   const int tid = threadIdx.x;
   const int row = blockIdx.y;
-  const int g = p.group;
-  const int b = row / p.n_kv_heads, kvh = row % p.n_kv_heads;
-  const uint16_t* qg = p.q + ((int64_t)b * p.n_q_heads + (int64_t)kvh * g) * p.dqk;
-  for (int i = tid; i < g * R; i += NT) {
-    const int h = i / R, r = i % R;
-    const int ch = min(max(p.label_ch[kvh * R + r], 0), p.dqk - 1);  // clamped: never out of bounds
-    qlab[i] = __uint_as_float((uint32_t)qg[(int64_t)h * p.dqk + ch] << 16);
-  }
-  __syncthreads();
+  load_qlab<R, NT>(p, row, qlab);
+  const int nvb = load_block_list<NT>(p, row, sb);  // ends with a CTA barrier
+  const int n_valid = valid_candidates(p, row, sb, nvb);
 
-  const int32_t* bidx = p.block_idx + (int64_t)row * p.K_b;
   const int c0 = blockIdx.x * p.chunk;
   const int c1 = min(p.n_cand, c0 + p.chunk);
   float* out = p.tscore + (int64_t)row * p.n_cand;
+  const int g = p.group;
   for (int i = c0 + tid; i < c1; i += NT) {
-    const int64_t blk = min(max(__ldcg(bidx + i / p.bs), 0), p.nb - 1);  // clamped: never out of bounds
-    const int64_t tok = blk * p.bs + (i % p.bs);
+    const int64_t tok = (int64_t)sb[i / p.bs] * p.bs + (i % p.bs);
     const int64_t at = (int64_t)row * p.ctx_len + tok;
     float c[R];
     load_codes<R>(p.codes + at * (R / 2), c);
@@ -66,7 +63,7 @@ __global__ void __launch_bounds__(NT) token_select_kernel(TokenParams p) {
     }
     const float score = s * best;
     out[i] = score;
-    if (p.token_score != nullptr) p.token_score[(int64_t)row * p.n_cand + i] = score;
+    if (p.token_score != nullptr) p.token_score[(int64_t)row * p.n_cand + i] = i < n_valid ? score : -INFINITY;
   }
 
   __threadfence();
@@ -75,13 +72,13 @@ __global__ void __launch_bounds__(NT) token_select_kernel(TokenParams p) {
   __syncthreads();
   if (!last) return;
   __threadfence();
-  uint32_t* keys = reinterpret_cast<uint32_t*>(sm + g * R);
-  TopkScratch* ts = reinterpret_cast<TopkScratch*>(keys + p.n_cand);
-  for (int i = tid; i < p.n_cand; i += NT) keys[i] = float_key(__ldcg(out + i));
+  for (int i = tid; i < n_valid; i += NT) keys[i] = float_key(__ldcg(out + i));
+  const int kk = min(p.k, n_valid);
+  int32_t* dst = p.token_idx + (int64_t)row * p.k;
+  pad_list(dst, kk, p.k);
   __syncthreads();
-  const int bs = p.bs;
-  cta_topk_ascending<NT>(keys, p.n_cand, p.k, p.token_idx + (int64_t)row * p.k, *ts,
-                         [bidx, bs](int i) { return bidx[i / bs] * bs + (i % bs); });
+  if (kk == 0) return;
+  cta_topk_ascending<NT>(keys, n_valid, kk, dst, *ts, CandidateToken{sb, p.bs});
 }
 
 // A cluster of CTAs per row when scoring is light: every CTA scores a
@@ -95,7 +92,10 @@ constexpr int kTokThreads = 256;
 // NTILE n-tiles of 8); 0: on the CUDA cores.  CL CTAs (the launch's cluster
 // size) share a row: 4 when there are enough rows to fill the GPU, up to 16
 // when a few long rows would leave it idle.
-template <int R, int NTILE, int CL>
+// BIG: the row has too many candidates for one CTA's shared memory to hold
+// all their keys; the degenerate fallback then gathers them in the workspace
+// (tscore, as keys) instead of the leader's shared memory.
+template <int R, int NTILE, int CL, bool BIG>
 __global__ void __launch_bounds__(kTokThreads) token_select_cluster_kernel(TokenParams p) {
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
@@ -106,8 +106,8 @@ __global__ void __launch_bounds__(kTokThreads) token_select_cluster_kernel(Token
   float* qlab = sm;                                                   // [G][R]
   int32_t* bidx = reinterpret_cast<int32_t*>(sm + p.group * R);       // [K_b]
   uint32_t* mine = reinterpret_cast<uint32_t*>(bidx + p.K_b);         // [per]
-  uint32_t* all = mine + per;                                         // [n_cand] (leader, fallback)
-  TopkScratch* ts = reinterpret_cast<TopkScratch*>(all + p.n_cand);
+  uint32_t* all = mine + per;                                         // [n_cand] (leader, fallback; not BIG)
+  TopkScratch* ts = reinterpret_cast<TopkScratch*>(BIG ? all : all + p.n_cand);
   ClusterTopkScratch<CL>* cts =
       reinterpret_cast<ClusterTopkScratch<CL>*>((reinterpret_cast<uintptr_t>(ts + 1) + 15) & ~uintptr_t(15));
   cluster_arrive_relaxed();  // completes once every CTA of the cluster has started
@@ -115,22 +115,36 @@ __global__ void __launch_bounds__(kTokThreads) token_select_cluster_kernel(Token
   load_qlab<R, kTokThreads>(p, row, qlab);
   if (threadIdx.x == 0) prefetch_l2(p.token_idx + (int64_t)row * p.k + (int64_t)rank * p.k / CL);
   grid_dependency_wait();  // the block lists come from the preceding kernel
-  load_block_list<kTokThreads>(p, row, bidx);
-  __syncthreads();
+  const int nvb = load_block_list<kTokThreads>(p, row, bidx);  // ends with a CTA barrier
+  const int n_valid = valid_candidates(p, row, bidx, nvb);
   const int c0 = min(p.n_cand, rank * per), c1 = min(p.n_cand, c0 + per);
-  if constexpr (NTILE > 0) score_candidates_tc<R, kTokThreads, NTILE>(p, row, qlab, bidx, c0, c1, mine);
-  else score_candidates<R, kTokThreads>(p, row, qlab, bidx, c0, c1, mine);
+  if constexpr (NTILE > 0) score_candidates_tc<R, kTokThreads, NTILE>(p, row, qlab, bidx, c0, c1, mine, n_valid);
+  else score_candidates<R, kTokThreads>(p, row, qlab, bidx, c0, c1, mine, n_valid);
   __syncthreads();
   cluster_wait();
   int* out = p.token_idx + (int64_t)row * p.k;
   const CandidateToken map{bidx, p.bs};
-  if (cluster_topk_ascending<kTokThreads, CL>(mine, c1 - c0, c0, p.k, out, *cts, map)) return;
-  if (rank == 0) {
+  // only the candidates that are tokens of the sequence compete (a prefix)
+  const int kk = min(p.k, n_valid);
+  const int n_loc = max(0, min(c1, n_valid) - c0);
+  if (rank == 0) pad_list(out, kk, p.k);
+  if (kk == 0) {
+    cluster.sync();  // no CTA leaves while another may still read its shared memory
+    return;
+  }
+  if (cluster_topk_ascending<kTokThreads, CL>(mine, n_loc, c0, kk, out, *cts, map)) return;
+  uint32_t* keys = all;
+  if constexpr (BIG) {
+    // every CTA writes its keys into the row's workspace scores (as keys)
+    keys = reinterpret_cast<uint32_t*>(p.tscore + (int64_t)row * p.n_cand);
+    for (int i = threadIdx.x; i < n_loc; i += kTokThreads) keys[c0 + i] = mine[i];
+    __threadfence();
+  } else if (rank == 0) {
     // gather the other CTAs' keys through distributed shared memory, eight
     // independent loads in flight per thread
     for (int r = 0; r < CL; ++r) {
       const uint32_t* __restrict__ src = cluster.map_shared_rank(mine, r);
-      const int b0 = min(p.n_cand, r * per), b1 = min(p.n_cand, b0 + per);
+      const int b0 = min(n_valid, r * per), b1 = min(n_valid, b0 + per);
       for (int i0 = 0; i0 < b1 - b0; i0 += 8 * kTokThreads) {
         uint32_t v[8];
 #pragma unroll
@@ -146,9 +160,9 @@ __global__ void __launch_bounds__(kTokThreads) token_select_cluster_kernel(Token
       }
     }
   }
-  cluster.sync();  // the other CTAs' shared memory may be released after this
+  cluster.sync();  // the other CTAs' shared memory (or workspace keys) may be released / read after this
   if (rank != 0) return;
-  cta_topk_ascending<kTokThreads>(all, p.n_cand, p.k, out, *ts, map);
+  cta_topk_ascending<kTokThreads>(keys, n_valid, kk, out, *ts, map);
 }
 
 // A small cluster per row (the launch's cluster size CL, 1 to 4): each CTA
@@ -179,11 +193,11 @@ __global__ void __launch_bounds__(NT, NT >= 1024 || KPT > 8 ? 1 : 2) token_selec
   load_qlab<R, NT>(p, row, qlab);
   if (threadIdx.x == 0 && rank == 0) prefetch_l2(p.token_idx + (int64_t)row * p.k);
   grid_dependency_wait();  // the block lists come from the preceding kernel
-  load_block_list<NT>(p, row, bidx);
-  __syncthreads();
+  const int nvb = load_block_list<NT>(p, row, bidx);  // ends with a CTA barrier
+  const int n_valid = valid_candidates(p, row, bidx, nvb);
   stage_candidate_codes<R, NT>(p, row, bidx, j0, j1, scodes, sscales);
   __syncthreads();
-  score_candidates_tc<R, NT, NTILE, true>(p, row, qlab, bidx, c0, c1, keys, scodes, sscales);
+  score_candidates_tc<R, NT, NTILE, true>(p, row, qlab, bidx, c0, c1, keys, n_valid, scodes, sscales);
   // the next grid (the attention) may become resident from here: only the
   // selection is left, and earlier it would hold SMs a concurrent level 1
   // needs
@@ -200,8 +214,13 @@ __global__ void __launch_bounds__(NT, NT >= 1024 || KPT > 8 ? 1 : 2) token_selec
     cluster.sync();  // the leader's keys are complete; no remote access after this
     if (rank != 0) return;
   }
+  // only the candidates that are tokens of the sequence compete (a prefix)
+  const int kk = min(p.k, n_valid);
+  int32_t* out = p.token_idx + (int64_t)row * p.k;
+  pad_list(out, kk, p.k);
+  if (kk == 0) return;
   const CandidateToken map{bidx, p.bs};
-  cta_topk_regs<NT, KPT>(keys, p.n_cand, p.k, p.token_idx + (int64_t)row * p.k, *ts, map);
+  cta_topk_regs<NT, KPT>(keys, n_valid, kk, out, *ts, map);
 }
 
 // Which level-2 kernel a call takes, its CTAs per row and threads per CTA
@@ -216,7 +235,9 @@ TokenDispatch token_dispatch(const tls_shape& s, int K_b, bool lean, bool aligne
     return {TokenDispatch::kRow, "token_select_row_kernel", cl, nt};
   }
   const bool tc = g >= 16 && g <= 128 && (s.n_label == 16 || s.n_label == 32);
-  if (tc || token_cluster_fits(g, s.n_label, n_cand))
+  // rows too long for one CTA's shared memory go to clusters whatever the
+  // scoring load (each CTA keeps at most kTokMaxPerCta * 4 keys)
+  if (tc || token_cluster_fits(g, s.n_label, n_cand) || n_cand > kTokSmemKeysMax)
     return {TokenDispatch::kCluster, "token_select_cluster_kernel", token_cluster_size(rows, n_cand, tc), kTokThreads};
   return {TokenDispatch::kChunked, "token_select_kernel", 1, 256};
 }
@@ -244,6 +265,7 @@ void fill_token_params(TokenParams& p, const tls_shape& s, const void* q, const 
   p.token_score = token_score;
   p.counters = reinterpret_cast<unsigned*>(ws + L.tok_counter);
   p.token_idx = token_idx;
+  p.seq_lens = s.seq_lens;
 }
 
 // `lean`: the row kernel on at most half the SMs (the other half is left to
@@ -271,7 +293,7 @@ tls_status select_tokens_impl(const tls_shape& s, const void* q, const int32_t* 
   p.counters = reinterpret_cast<unsigned*>(ws + L.tok_counter);
   p.token_idx = token_idx;
 
-  const size_t smem = (size_t)p.group * s.n_label * 4 + (size_t)p.n_cand * 4 + sizeof(TopkScratch) + 16;
+  const size_t smem = ((size_t)p.group * s.n_label + K_b + p.n_cand) * 4 + sizeof(TopkScratch) + 32;
   const TokenDispatch d = token_dispatch(
       s, K_b, lean, ((reinterpret_cast<uintptr_t>(codes) | reinterpret_cast<uintptr_t>(scales)) & 15u) == 0);
   if (d.kind == TokenDispatch::kRow) {
@@ -305,11 +327,12 @@ tls_status select_tokens_impl(const tls_shape& s, const void* q, const int32_t* 
   if (d.kind == TokenDispatch::kCluster) {
     const int cl = d.cl;
     const int per = (p.n_cand + cl - 1) / cl;
+    const bool big = p.n_cand > kTokSmemKeysMax;  // the fallback gathers keys in the workspace
     const size_t cts_bytes = cl == 16 ? sizeof(ClusterTopkScratch<16>)
                              : cl == 8 ? sizeof(ClusterTopkScratch<8>)
                                        : sizeof(ClusterTopkScratch<4>);
-    const size_t csmem =
-        ((size_t)p.group * s.n_label + K_b + per + p.n_cand) * 4 + sizeof(TopkScratch) + cts_bytes + 32;
+    const size_t csmem = ((size_t)p.group * s.n_label + K_b + per + (big ? 0 : p.n_cand)) * 4 +
+                         sizeof(TopkScratch) + cts_bytes + 32;
     const int ntile = p.group <= 16 ? 2 : p.group <= 32 ? 4 : p.group <= 64 ? 8 : 16;
     auto launch = [&](auto kernel) -> tls_status {
       // 16-CTA clusters are beyond the portable size
@@ -319,11 +342,14 @@ tls_status select_tokens_impl(const tls_shape& s, const void* q, const int32_t* 
                                   (unsigned)cl, p),
                         "select_tokens launch");
     };
-    auto by_cl = [&](auto k4, auto k8, auto k16) -> tls_status {
+    auto by_cl = [&](auto k4, auto k8, auto k16, auto b4, auto b8, auto b16) -> tls_status {
+      if (big) return cl == 16 ? launch(b16) : cl == 8 ? launch(b8) : launch(b4);
       return cl == 16 ? launch(k16) : cl == 8 ? launch(k8) : launch(k4);
     };
-#define TLS_TC(RR, NN) \
-  by_cl(token_select_cluster_kernel<RR, NN, 4>, token_select_cluster_kernel<RR, NN, 8>, token_select_cluster_kernel<RR, NN, 16>)
+#define TLS_TC(RR, NN)                                                                                      \
+  by_cl(token_select_cluster_kernel<RR, NN, 4, false>, token_select_cluster_kernel<RR, NN, 8, false>,       \
+        token_select_cluster_kernel<RR, NN, 16, false>, token_select_cluster_kernel<RR, NN, 4, true>,        \
+        token_select_cluster_kernel<RR, NN, 8, true>, token_select_cluster_kernel<RR, NN, 16, true>)
     if (tc) {
       if (s.n_label == 16) {
         if (ntile == 2) return TLS_TC(16, 2);
@@ -336,17 +362,17 @@ tls_status select_tokens_impl(const tls_shape& s, const void* q, const int32_t* 
       if (ntile == 8) return TLS_TC(32, 8);
       return TLS_TC(32, 16);
     }
-#undef TLS_TC
     switch (s.n_label) {
-      case 2: return launch(token_select_cluster_kernel<2, 0, 4>);
-      case 4: return launch(token_select_cluster_kernel<4, 0, 4>);
-      case 8: return launch(token_select_cluster_kernel<8, 0, 4>);
-      case 16: return launch(token_select_cluster_kernel<16, 0, 4>);
-      case 32: return launch(token_select_cluster_kernel<32, 0, 4>);
-      case 64: return launch(token_select_cluster_kernel<64, 0, 4>);
+      case 2: return TLS_TC(2, 0);
+      case 4: return TLS_TC(4, 0);
+      case 8: return TLS_TC(8, 0);
+      case 16: return TLS_TC(16, 0);
+      case 32: return TLS_TC(32, 0);
+      case 64: return TLS_TC(64, 0);
       default:
         return fail(TLS_ERR_UNSUPPORTED, "select_tokens: n_label %d not built (2,4,8,16,32,64)", s.n_label);
     }
+#undef TLS_TC
   }
   dim3 grid((unsigned)chunks, (unsigned)rows);
   switch (s.n_label) {

@@ -31,11 +31,15 @@ class DecodeState:
 
     def __init__(self, *, batch, n_q_heads, n_kv_heads, qk_dim, v_dim, v_offset, block_size, n_label, ctx_len,
                  K_b, k, q_bits, k_bits, v_bits, label_ch, softmax_scale=None, out_dtype=tls.TLS_OUT_F32,
-                 device="cuda", build_index=True, kv_device=None):
+                 device="cuda", build_index=True, kv_device=None, seq_lens=None):
         self.device = torch.device(device)
         scale = 1.0 / math.sqrt(qk_dim) if softmax_scale is None else softmax_scale
+        # seq_lens: tokens present per sequence (int [B]); None: every sequence holds ctx_len
+        self.seq_lens = (torch.as_tensor(np.asarray(seq_lens, dtype=np.int32)).to(self.device)
+                         if seq_lens is not None else None)
         self.shape = tls.make_shape(batch, n_q_heads, n_kv_heads, qk_dim, v_dim, v_offset, block_size, n_label,
-                                    ctx_len, scale)
+                                    ctx_len, scale, self.seq_lens)
+        self._baseline_ws = {}
         self.K_b, self.k = int(K_b), int(k)
         self.rows = batch * n_kv_heads
         self.nb = ctx_len // block_size
@@ -100,6 +104,55 @@ class DecodeState:
 
     def check_device_error(self, stream=None) -> int:
         return tls.tls_workspace_error(self.ws, True, stream)
+
+    # per-token append ---------------------------------------------------------
+    def append(self, k_new, v_new=None, stream=None):
+        """Appends one decoded token to every sequence (tls_append_kv): device bf16 k_new [B, Hkv, Dqk],
+        v_new [B, Hkv, Dv] (None for the MLA latent); needs seq_lens."""
+        if self.seq_lens is None:
+            raise ValueError("append needs a state created with seq_lens")
+        v = self.vc if self.vc is not None else self.kc
+        kv = tls.make_kv_view(self.kc, v, self.shape.qk_dim, self.shape.v_dim if self.vc is not None else self.shape.qk_dim)
+        tls.tls_append_kv(self.shape, self.seq_lens, k_new, v_new, kv, self.meta, self.label_ch, self.codes,
+                          self.scales, stream)
+
+    # operator baselines (full attention, block selection alone, token selection alone)
+    def _ws_for(self, K_b, k):
+        key = (K_b, k)
+        if key not in self._baseline_ws:
+            n = tls.tls_workspace_bytes(self.shape, K_b, k)
+            if n == 0:
+                raise tls.TlsError(tls.TLS_ERR_INVALID_ARG, "tls_workspace_bytes", f"K_b {K_b}, k {k}")
+            self._baseline_ws[key] = (torch.zeros(n, dtype=torch.uint8, device=self.device), n)
+        return self._baseline_ws[key]
+
+    def dense(self, q=None, stream=None):
+        """Full attention over every token of each sequence (tls_dense_decode_attn) into out / lse."""
+        ws, n = self._ws_for(self.nb, self.shape.ctx_len)
+        tls.tls_dense_decode_attn(self.shape, self.q if q is None else q, self.kv, self.out_dtype, self.out, self.lse,
+                                  ws, n, stream)
+
+    def quest(self, q=None, K_b=None, block_idx=None, stream=None):
+        """Block selection alone (tls_quest_decode_step): K_b blocks, every token of them attended."""
+        K_b = self.K_b if K_b is None else K_b
+        if block_idx is None:
+            block_idx = self.block_idx if K_b == self.K_b else torch.empty(
+                (self.shape.batch, self.shape.n_kv_heads, K_b), dtype=torch.int32, device=self.device)
+        ws, n = self._ws_for(K_b, K_b * self.shape.block_size)
+        tls.tls_quest_decode_step(self.shape, self.q if q is None else q, self.meta, self.kv, K_b, block_idx,
+                                  self.out_dtype, self.out, self.lse, ws, n, stream)
+        return block_idx
+
+    def ds(self, q=None, k=None, token_idx=None, stream=None):
+        """Token selection alone over every token (tls_ds_decode_step): k tokens attended."""
+        k = self.k if k is None else k
+        if token_idx is None:
+            token_idx = self.token_idx if k == self.k else torch.empty(
+                (self.shape.batch, self.shape.n_kv_heads, k), dtype=torch.int32, device=self.device)
+        ws, n = self._ws_for(self.nb, k)
+        tls.tls_ds_decode_step(self.shape, self.q if q is None else q, self.label_ch, self.codes, self.scales,
+                               self.kv, k, token_idx, self.out_dtype, self.out, self.lse, ws, n, stream)
+        return token_idx
 
 
 class ResidentEngine:

@@ -44,6 +44,7 @@ class Shape(ctypes.Structure):
         ("n_label", ctypes.c_int32),
         ("ctx_len", ctypes.c_int64),
         ("softmax_scale", ctypes.c_float),
+        ("seq_lens", ctypes.c_void_p),
     ]
 
 
@@ -85,6 +86,10 @@ _SIG = {
     "tls_select_tokens": (_I32, [_P, _P, _P, _P, _P, _P, _I32, _I32, _P, _P, _P, _SZ, _P]),
     "tls_sparse_decode_attn": (_I32, [_P, _P, _P, _P, _I32, _I32, _P, _P, _P, _SZ, _P]),
     "tls_sparse_decode_attn_noalloc": (_I32, [_P, _P, _P, _P, _I32, _I32, _P, _P, _P]),
+    "tls_dense_decode_attn": (_I32, [_P, _P, _P, _I32, _P, _P, _P, _SZ, _P]),
+    "tls_quest_decode_step": (_I32, [_P, _P, _P, _P, _I32, _P, _I32, _P, _P, _P, _SZ, _P]),
+    "tls_ds_decode_step": (_I32, [_P, _P, _P, _P, _P, _P, _I32, _P, _I32, _P, _P, _P, _SZ, _P]),
+    "tls_append_kv": (_I32, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "tls_select": (_I32, [_P, _P, _P, _P, _P, _P, _I32, _I32, _P, _P, _P, _SZ, _P]),
     "tls_decode_step": (_I32, [_P, _P, _P, _P, _P, _P, _P, _I32, _I32, _P, _P, _I32, _P, _P, _P, _SZ, _P]),
     "tls_block_cache_create": (_I32, [_P, _P, _P, _I64, _I64, _I32, _P, _P, _P, _P]),
@@ -146,13 +151,21 @@ def _check(status: int, where: str):
 
 
 def make_shape(batch, n_q_heads, n_kv_heads, qk_dim, v_dim, v_offset, block_size, n_label, ctx_len,
-               softmax_scale) -> Shape:
-    return Shape(batch, n_q_heads, n_kv_heads, qk_dim, v_dim, v_offset, block_size, n_label, ctx_len,
-                 softmax_scale)
+               softmax_scale, seq_lens=None) -> Shape:
+    """seq_lens: optional device int32 tensor [B] of tokens per sequence (the shape keeps its address)."""
+    shape = Shape(batch, n_q_heads, n_kv_heads, qk_dim, v_dim, v_offset, block_size, n_label, ctx_len,
+                  softmax_scale, _ptr(seq_lens))
+    shape._keep = seq_lens  # the shape holds its address
+    return shape
 
 
 def make_kv_view(k, v, k_row_stride, v_row_stride, slot_of_block=None, n_slots=0) -> KvView:
-    return KvView(_ptr(k), _ptr(v), int(k_row_stride), int(v_row_stride), _ptr(slot_of_block), int(n_slots))
+    """The view holds device addresses; it also keeps the tensors it was made
+    from alive, so a temporary (e.g. a slot table made inline) is not freed
+    while the view may still be passed to a call."""
+    view = KvView(_ptr(k), _ptr(v), int(k_row_stride), int(v_row_stride), _ptr(slot_of_block), int(n_slots))
+    view._keep = (k, v, slot_of_block)
+    return view
 
 
 def tls_last_error() -> str:
@@ -225,6 +238,31 @@ def tls_sparse_decode_attn_noalloc(shape, q, kv: KvView, token_idx, k, out_dtype
     _check(lib().tls_sparse_decode_attn_noalloc(ctypes.byref(shape), _ptr(q), ctypes.byref(kv), _ptr(token_idx), k,
                                                 out_dtype, _ptr(out), _ptr(lse), _stream(stream)),
            "tls_sparse_decode_attn_noalloc")
+
+
+def tls_dense_decode_attn(shape, q, kv: KvView, out_dtype, out, lse, ws, ws_bytes, stream=None):
+    _check(lib().tls_dense_decode_attn(ctypes.byref(shape), _ptr(q), ctypes.byref(kv), out_dtype, _ptr(out), _ptr(lse),
+                                       _ptr(ws), ws_bytes, _stream(stream)), "tls_dense_decode_attn")
+
+
+def tls_quest_decode_step(shape, q, meta, kv: KvView, K_b, block_idx, out_dtype, out, lse, ws, ws_bytes,
+                          stream=None):
+    _check(lib().tls_quest_decode_step(ctypes.byref(shape), _ptr(q), _ptr(meta), ctypes.byref(kv), K_b,
+                                       _ptr(block_idx), out_dtype, _ptr(out), _ptr(lse), _ptr(ws), ws_bytes,
+                                       _stream(stream)), "tls_quest_decode_step")
+
+
+def tls_ds_decode_step(shape, q, label_ch, codes, scales, kv: KvView, k, token_idx, out_dtype, out, lse, ws, ws_bytes,
+                       stream=None):
+    _check(lib().tls_ds_decode_step(ctypes.byref(shape), _ptr(q), _ptr(label_ch), _ptr(codes), _ptr(scales),
+                                    ctypes.byref(kv), k, _ptr(token_idx), out_dtype, _ptr(out), _ptr(lse), _ptr(ws),
+                                    ws_bytes, _stream(stream)), "tls_ds_decode_step")
+
+
+def tls_append_kv(shape, seq_lens, k_new, v_new, kv: KvView, meta, label_ch, codes, scales, stream=None):
+    _check(lib().tls_append_kv(ctypes.byref(shape), _ptr(seq_lens), _ptr(k_new), _ptr(v_new), ctypes.byref(kv),
+                               _ptr(meta), _ptr(label_ch), _ptr(codes), _ptr(scales), _stream(stream)),
+           "tls_append_kv")
 
 
 def tls_select(shape, q, meta, label_ch, codes, scales, K_b, k, block_idx, token_idx, ws, ws_bytes, stream=None):
