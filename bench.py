@@ -124,7 +124,6 @@ ATTN_SOURCES = {
     "sparse_attn_mma_kernel": ("decode_attn_mma.cu", "attn_common.cuh", "device_common.cuh"),
     "sparse_attn_mma_cluster_kernel": ("decode_attn_mma.cu", "attn_common.cuh", "device_common.cuh"),
     "sparse_attn_mla_kernel": ("decode_attn_mla.cu", "attn_common.cuh", "device_common.cuh"),
-    "sparse_attn_mla_tc_kernel": ("decode_attn_mla_tc.cu", "attn_common.cuh", "device_common.cuh"),
     "sparse_attn_kernel": ("decode_attn.cu", "attn_common.cuh", "device_common.cuh"),
 }
 

@@ -114,10 +114,9 @@ TLS_API int32_t tls_version(void);
  * shape: "sparse_attn_mma_cluster_kernel" or "sparse_attn_mma_kernel" for
  * 128-wide K and V rows (one cluster of CTAs per row and head group of <= 16
  * heads while such a grid fits two CTAs per SM; else persistent CTAs),
- * "sparse_attn_mla_tc_kernel" for the MLA latent cache (Dqk 576, Dv 512 taken
- * from the same row) with G a multiple of 128 (tcgen05, the 128 heads as the
- * MMA's M), "sparse_attn_mla_kernel" for other MLA groups that are a multiple
- * of 16, and "sparse_attn_kernel" for every other shape.  A
+ * "sparse_attn_mla_kernel" for the MLA latent cache (Dqk 576, Dv 512 taken
+ * from the same row, G a multiple of 16), and "sparse_attn_kernel" for every
+ * other shape.  A
  * static string owned by the library; NULL if the shape is invalid
  * (tls_last_error says why).  Host only, no device work.
  */

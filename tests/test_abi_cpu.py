@@ -64,7 +64,7 @@ def test_attention_dispatch_names_the_kernel_per_shape(tls):
     assert tls.tls_attn_kernel(c2_shape(tls, batch=1, n_q_heads=64, n_kv_heads=1)) == "sparse_attn_mma_cluster_kernel"
     assert tls.tls_attn_kernel(c2_shape(tls, batch=40, n_q_heads=64, n_kv_heads=1)) == "sparse_attn_mma_kernel"
     mla = c2_shape(tls, batch=4, n_q_heads=128, n_kv_heads=1, qk_dim=576, v_dim=512, v_offset=0, n_label=32)
-    assert tls.tls_attn_kernel(mla) == "sparse_attn_mla_tc_kernel"  # G = 128: tcgen05
+    assert tls.tls_attn_kernel(mla) == "sparse_attn_mla_kernel"
     assert tls.tls_attn_kernel(c2_shape(tls, batch=4, n_q_heads=32, n_kv_heads=1, qk_dim=576, v_dim=512, v_offset=0,
                                         n_label=32)) == "sparse_attn_mla_kernel"  # G = 32
     assert tls.tls_attn_kernel(c2_shape(tls, batch=4, n_q_heads=8, n_kv_heads=1, qk_dim=576, v_dim=512, v_offset=0,

@@ -18,7 +18,6 @@ bool attn_mma_supported(const tls_shape& s);
 int attn_mma_plan(int rows, int k, int* chunks_per_row, int* n_items, int* n_ctas);
 int attn_mma_cluster_size(int rows, int hpc);
 bool attn_mla_supported(const tls_shape& s);
-bool attn_mla_tc_supported(const tls_shape& s);
 int attn_mla_tokens_per_split(int k);
 
 namespace {
@@ -187,7 +186,6 @@ extern "C" const char* tls_attn_kernel(const tls_shape* shape) {
     return attn_mma_cluster_size(rows_of(*shape) * head_groups, hpc) > 0 ? "sparse_attn_mma_cluster_kernel"
                                                                           : "sparse_attn_mma_kernel";
   }
-  if (attn_mla_tc_supported(*shape)) return "sparse_attn_mla_tc_kernel";
   if (attn_mla_supported(*shape)) return "sparse_attn_mla_kernel";
   return "sparse_attn_kernel";
 }

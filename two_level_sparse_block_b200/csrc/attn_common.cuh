@@ -157,8 +157,5 @@ bool attn_mla_supported(const tls_shape& s);
 int attn_mla_tokens_per_split(int k);
 tls_status launch_attn_mla(const AttnParams& p, int rows, cudaStream_t stream, bool pdl);
 int attn_mma_cluster_size(int rows, int hpc);
-// MLA latent attention on tcgen05 (decode_attn_mla_tc.cu): Dqk 576, Dv 512, G % 128 == 0.
-bool attn_mla_tc_supported(const tls_shape& s);
-tls_status launch_attn_mla_tc(const AttnParams& p, int rows, cudaStream_t stream, bool pdl);
 
 }  // namespace tls

@@ -322,27 +322,6 @@ tls_status get_encoder() {
   return TLS_OK;
 }
 
-}  // namespace
-
-// 2-D bf16 tensor map of a row-major [rows][cols] tensor (row stride
-// cols * 2 bytes), tiles of box_cols x box_rows, 128-byte swizzle.
-tls_status encode_bf16_2d_sw128(void* tmap, const void* base, uint64_t cols, uint64_t rows, uint32_t box_cols,
-                                uint32_t box_rows) {
-  tls_status st = get_encoder();
-  if (st != TLS_OK) return st;
-  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  const cuuint32_t box[2] = {box_cols, box_rows};
-  const cuuint32_t estr[2] = {1, 1};
-  CUresult r = g_encode(reinterpret_cast<CUtensorMap*>(tmap), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-                        const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(TLS_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
-  return TLS_OK;
-}
-
-namespace {
-
 template <int NPAD, int CL>
 tls_status launch_tc(const CUtensorMap& tmap, const CUtensorMap& qmap, const BlockScoreParams& p, int rows,
                      cudaStream_t stream) {

@@ -258,7 +258,6 @@ tls_status sparse_attn_impl(const tls_shape& s, const void* q, const tls_kv_view
   p.K_b = K_b;
   const int rows = rows_of(s);
   if (attn_mma_supported(s)) return launch_attn_mma(p, rows, stream, pdl);
-  if (attn_mla_tc_supported(s)) return launch_attn_mla_tc(p, rows, stream, pdl);
   if (attn_mla_supported(s)) return launch_attn_mla(p, rows, stream, pdl);
   const int pk = (s.qk_dim + 127) / 128, pv = (s.v_dim + 127) / 128;
   const int hg = L.heads_per_cta;

@@ -74,12 +74,6 @@ struct WsLayout {
 // current device and context (looked up once per device and context).
 tls_status noalloc_scratch(void** out);
 
-// Encodes a 2-D bf16 tensor map (128 bytes of CUtensorMap at tmap) of a
-// row-major [rows][cols] tensor with box_cols x box_rows tiles and 128-byte
-// swizzle (the driver's encoder, found once through the runtime).
-tls_status encode_bf16_2d_sw128(void* tmap, const void* base, uint64_t cols, uint64_t rows, uint32_t box_cols,
-                                uint32_t box_rows);
-
 // Plans the attention launch and the workspace for (shape, K_b, k).
 tls_status plan_workspace(const tls_shape& s, int K_b, int k, WsLayout* out);
 
