@@ -200,6 +200,74 @@ def test_paged_kv_of_a_ragged_batch():
     assert torch.equal(st.out, dense)
 
 
+# token lists holding -1 entries with every sequence full (no seq_lens): the
+# attention skips them wherever they stand.  Shapes reaching the cluster and
+# persistent tensor-core kernels, the MLA kernel and the CUDA-core kernel.
+HOLES = [
+    (shape_cfg("h_gqa4_cluster", ctx_len=1024), "sparse_attn_mma_cluster_kernel"),
+    (shape_cfg("h_gqa4_persistent", batch=80, ctx_len=1024, K_b=9, k=133, seed=77), "sparse_attn_mma_kernel"),
+    (RAGGED[1][0], "sparse_attn_mla_kernel"),
+    (RAGGED[3][0], "sparse_attn_kernel"),
+]
+
+
+@pytest.mark.parametrize("case", HOLES, ids=lambda c: c[0].name)
+def test_minus_one_entries_are_skipped(case):
+    runtime, tls = _rt()
+    cfg, kernel = case
+    q = synth.gen_queries(cfg)
+    K, V, _ = synth.gen_kv(cfg, q)
+    lab = synth.gen_label_channels(cfg)
+    st = runtime.state_for_config(cfg, q, K, V, lab)
+    assert tls.tls_attn_kernel(st.shape) == kernel
+    st.select()
+    torch.cuda.synchronize()
+    lists = st.token_idx.cpu().numpy().reshape(cfg.rows, cfg.k).copy()
+    rng = np.random.default_rng(cfg.seed + 1)
+    for r in range(cfg.rows):
+        kind = r % 4
+        if kind == 0:      # a padded tail
+            lists[r, cfg.k // 2:] = -1
+        elif kind == 1:    # the first 16 entries (a whole chunk) and every 7th entry
+            lists[r, :16] = -1
+            lists[r, ::7] = -1
+        elif kind == 2:    # scattered holes, some out of range
+            hole = rng.random(cfg.k) < 0.3
+            lists[r, hole] = rng.choice([-1, -5, cfg.ctx_len, cfg.ctx_len + 9], int(hole.sum()))
+    lists[1 % cfg.rows] = -1  # a row with no token
+    st.token_idx.copy_(torch.from_numpy(lists.reshape(st.token_idx.shape)).cuda())
+    st.attend()
+    torch.cuda.synchronize()
+    assert st.check_device_error() == 0
+    out = st.out.float().cpu().numpy()
+    lse = st.lse.cpu().numpy()
+    g = cfg.group
+    for r in _rows_sample(cfg):
+        b, h = divmod(r, cfg.n_kv_heads)
+        where = f"{cfg.name} row ({b},{h})"
+        keep = lists[r][(lists[r] >= 0) & (lists[r] < cfg.ctx_len)]
+        o = out[b, h * g:(h + 1) * g]
+        ls = lse[b, h * g:(h + 1) * g]
+        if keep.size == 0:
+            assert np.all(o == 0.0) and np.all(np.isneginf(ls)), f"{where}: empty list"
+            continue
+        kf = f32_from_bf16_bits(K[b, h, keep]).astype(np.float64)
+        vf = kf[:, cfg.v_offset:cfg.v_offset + cfg.v_dim] if V is None else \
+            f32_from_bf16_bits(V[b, h, keep]).astype(np.float64)
+        ref_out, ref_lse = oracle.attention(f32_from_bf16_bits(q[b, h * g:(h + 1) * g]).astype(np.float64), kf, vf,
+                                            cfg.softmax_scale)
+        check_output(o, ref_out, where + " out")
+        assert np.max(np.abs(ls - ref_lse)) <= 1e-4 * max(1.0, np.max(np.abs(ref_lse))), f"{where}: lse"
+
+
+def _rows_sample(cfg, n=12):
+    rows = list(range(cfg.rows))
+    if len(rows) <= n:
+        return rows
+    pick = set(np.random.default_rng(cfg.seed).choice(len(rows), n, replace=False).tolist()) | {0, 1, 2, 3}
+    return sorted(pick)
+
+
 APPEND = [
     (shape_cfg("a_gqa4", batch=4, ctx_len=256, block_size=16, K_b=6, k=40, seed=81), [100, 63, 64, 0], 22),
     (shape_cfg("a_mla", batch=2, n_q_heads=16, n_kv_heads=1, qk_dim=576, v_dim=512, v_offset=0, ctx_len=512,

@@ -106,24 +106,43 @@ __device__ __forceinline__ void mma_load_q(const AttnParams& p, int b, int kvh, 
   }
 }
 
-// Token of entry (lane & 15) of chunk x of the row's list, or -1 past the end
-// of the list or when the entry is no token of the sequence (len tokens).
-__device__ __forceinline__ int mma_chunk_token(const AttnParams& p, int row, int x, int lane, int64_t len) {
+// Raw list entry (lane & 15) of chunk x of the row's list, or -1 past the
+// end of the list: the token (a token list), the position (every position),
+// or the block holding the position (a block list).  Nothing is computed on
+// the loaded value here: the load runs a chunk ahead of its use, and any
+// arithmetic on it would make the warp wait for it at once.  RAGGED covers
+// every list form; otherwise the list is a token list.
+template <bool RAGGED>
+__device__ __forceinline__ int mma_list_raw(const AttnParams& p, int row, int x, int lane) {
   const int t = x * kChunk + (lane & 15);
   if (t >= p.k_sel) return -1;
-  return attn_token(p, row, t, len);
+  // L2 loads: the list is written by the preceding kernel while this grid is
+  // already resident (programmatic dependent launch)
+  if (!RAGGED || p.list_mode == kListTokens) return __ldcg(p.token_idx + (int64_t)row * p.k_sel + t);
+  if (p.list_mode == kListAll) return t;
+  return __ldcg(p.blocks + (int64_t)row * p.K_b + t / p.bs);
+}
+
+// Token of a raw entry of chunk x (lane & 15), or -1 when it is none of the
+// sequence's len tokens (list padding, past the list end, out of range).
+template <bool RAGGED>
+__device__ __forceinline__ int mma_list_token(const AttnParams& p, int raw, int x, int lane, int64_t len) {
+  if (raw < 0) return -1;
+  int64_t tok = raw;
+  if (RAGGED && p.list_mode == kListBlocks) tok = (int64_t)raw * p.bs + (x * kChunk + (lane & 15)) % p.bs;
+  return tok < len ? (int)tok : -1;
 }
 
 // The chunk's 16 entries that are tokens (bit e: entry e), from the lane
-// values of mma_chunk_token; all lanes of the warp call it.
+// values of mma_list_token; all lanes of the warp call it.
 __device__ __forceinline__ uint32_t mma_valid_mask(int tok) {
   return __ballot_sync(0xffffffffu, tok >= 0) & 0xFFFFu;
 }
 
 // cp.async of the K and V rows of one chunk into the ring stage at shared
 // address kb (K tile; V tile at kb + 4096).  Entry lane & 15 holds token
-// `tok` (-1: the rows are zero-filled and the scores masked); slots are
-// clamped to the pool.  The caller commits the group.
+// `tok` in [0, N) (-1: the rows are zero-filled and the scores masked);
+// slots are clamped to the pool.  The caller commits the group.
 __device__ __forceinline__ void mma_issue_rows(const AttnParams& p, int row, int tok, uint32_t kb, int lane) {
   const int64_t rid = tok >= 0 ? attn_row_id(p, row, tok) : -1;
   const uint32_t vb = kb + 4096;
@@ -296,7 +315,7 @@ __device__ __forceinline__ void mma_fold(int g, float m0, float m1, float l0, fl
 // Persistent form: every CTA owns a contiguous range of the (row, chunk)
 // items; a row spread over several CTAs is merged by the last of them
 // through the split workspace (attn_common.cuh).
-template <int NS>
+template <int NS, bool RAGGED>
 __global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_kernel(AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
@@ -321,13 +340,20 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_kernel(Attn
   auto load_tok = [&](int i) -> int {
     if (i >= n_mine) return -1;
     const int64_t x = x0 + (int64_t)kMmaWarps * i;
-    const int r = (int)(x / CPR) / HG;
-    return mma_chunk_token(p, r, (int)(x % CPR), lane, seq_len_of(p.seq_lens, r / p.n_kv_heads, p.ctx_len));
+    return mma_list_raw<RAGGED>(p, (int)(x / CPR) / HG, (int)(x % CPR), lane);
   };
-  auto issue = [&](int i, int tok, int st) {
-    if (i < n_mine)
-      mma_issue_rows(p, (int)((x0 + (int64_t)kMmaWarps * i) / CPR) / HG, tok, ring_s + st * kChunkBytes, lane);
+  // issues chunk i from its raw list entry; returns the chunk's token mask
+  auto issue = [&](int i, int raw, int st) -> uint32_t {
+    int tok = -1;
+    if (i < n_mine) {
+      const int64_t x = x0 + (int64_t)kMmaWarps * i;
+      const int r = (int)(x / CPR) / HG;
+      tok = mma_list_token<RAGGED>(p, raw, (int)(x % CPR), lane,
+                                   RAGGED ? seq_len_of(p.seq_lens, r / p.n_kv_heads, p.ctx_len) : p.ctx_len);
+      mma_issue_rows(p, r, tok, ring_s + st * kChunkBytes, lane);
+    }
     cp_async_commit();
+    return mma_valid_mask(tok);
   };
 
   uint32_t qa[8][4];
@@ -356,10 +382,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_kernel(Attn
   for (int s = 0; s < NS; ++s) tok_ahead[s] = load_tok(s);
   uint64_t vq = 0;
 #pragma unroll
-  for (int s = 0; s < NS - 1; ++s) {
-    issue(s, tok_ahead[s], s);
-    vq |= (uint64_t)mma_valid_mask(tok_ahead[s]) << (16 * s);
-  }
+  for (int s = 0; s < NS - 1; ++s) vq |= (uint64_t)issue(s, tok_ahead[s], s) << (16 * s);
   int tok_next = tok_ahead[NS - 1];  // for chunk S-1
 
   const int vrow_first = (int)(c_lo / CPR);
@@ -379,8 +402,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_kernel(Attn
     for (; i < n_mine && x0 + (int64_t)kMmaWarps * i < seg_end; ++i) {
       // keep S-1 chunks in flight; indices run one chunk further ahead
       const int tok_after = load_tok(i + NS);
-      issue(i + NS - 1, tok_next, (i + NS - 1) % NS);
-      vq |= (uint64_t)mma_valid_mask(tok_next) << (16 * (NS - 1));
+      vq |= (uint64_t)issue(i + NS - 1, tok_next, (i + NS - 1) % NS) << (16 * (NS - 1));
       tok_next = tok_after;
       cp_async_wait<NS - 1>();
       __syncwarp();
@@ -416,7 +438,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_kernel(Attn
 // (M, l, O per head) into the leader's drained cp.async ring over
 // distributed shared memory, and the leader merges the CL partials by
 // log-sum-exp.  No workspace, ticket or device-wide fence.
-template <int NS>
+template <int NS, bool RAGGED>
 __global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_cluster_kernel(AttnParams p) {
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
@@ -438,13 +460,17 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_cluster_ker
   const uint32_t ring_s = smem_u32(sm + warp * NS * kChunkBytes);
   const int x0 = c_lo + warp;
   const int n_mine = x0 < c_hi ? (c_hi - 1 - x0) / kMmaWarps + 1 : 0;
-  const int64_t len = seq_len_of(p.seq_lens, b, p.ctx_len);
-  auto load_tok = [&](int i) -> int {
-    return i < n_mine ? mma_chunk_token(p, row, x0 + kMmaWarps * i, lane, len) : -1;
-  };
-  auto issue = [&](int i, int tok, int st) {
-    if (i < n_mine) mma_issue_rows(p, row, tok, ring_s + st * kChunkBytes, lane);
+  const int64_t len = RAGGED ? seq_len_of(p.seq_lens, b, p.ctx_len) : p.ctx_len;
+  auto load_tok = [&](int i) -> int { return i < n_mine ? mma_list_raw<RAGGED>(p, row, x0 + kMmaWarps * i, lane) : -1; };
+  // issues chunk i from its raw list entry; returns the chunk's token mask
+  auto issue = [&](int i, int raw, int st) -> uint32_t {
+    int tok = -1;
+    if (i < n_mine) {
+      tok = mma_list_token<RAGGED>(p, raw, x0 + kMmaWarps * i, lane, len);
+      mma_issue_rows(p, row, tok, ring_s + st * kChunkBytes, lane);
+    }
     cp_async_commit();
+    return mma_valid_mask(tok);
   };
   const int64_t oh = (int64_t)b * p.n_q_heads + (int64_t)kvh * p.group + h0;  // first output head
 
@@ -467,15 +493,11 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_cluster_ker
   for (int s = 0; s < NS; ++s) tok_ahead[s] = load_tok(s);
   uint64_t vq = 0;  // token masks of the issued chunks, 16 bits each, oldest lowest
 #pragma unroll
-  for (int s = 0; s < NS - 1; ++s) {
-    issue(s, tok_ahead[s], s);
-    vq |= (uint64_t)mma_valid_mask(tok_ahead[s]) << (16 * s);
-  }
+  for (int s = 0; s < NS - 1; ++s) vq |= (uint64_t)issue(s, tok_ahead[s], s) << (16 * s);
   int tok_next = tok_ahead[NS - 1];
   for (int i = 0; i < n_mine; ++i) {
     const int tok_after = load_tok(i + NS);
-    issue(i + NS - 1, tok_next, (i + NS - 1) % NS);
-    vq |= (uint64_t)mma_valid_mask(tok_next) << (16 * (NS - 1));
+    vq |= (uint64_t)issue(i + NS - 1, tok_next, (i + NS - 1) % NS) << (16 * (NS - 1));
     tok_next = tok_after;
     cp_async_wait<NS - 1>();
     __syncwarp();
@@ -553,7 +575,7 @@ int attn_mma_cluster_size(int rows, int hpc) {
   return 0;
 }
 
-template <int NS>
+template <int NS, bool RAGGED>
 static tls_status launch_mma(const AttnParams& p, int rows, cudaStream_t stream, bool pdl) {
   const MmaLayout L = mma_layout(p.heads_per_cta);
   const size_t smem = 128 + (size_t)L.bytes;
@@ -561,20 +583,25 @@ static tls_status launch_mma(const AttnParams& p, int rows, cudaStream_t stream,
   const int cl = attn_mma_cluster_size(rows, p.heads_per_cta);
   if (cl > 0) {
     // 16-CTA clusters are beyond the portable size
-    cudaError_t e = kernel_attrs((const void*)sparse_attn_mma_cluster_kernel<NS>, smem, cl > 8);
+    cudaError_t e = kernel_attrs((const void*)sparse_attn_mma_cluster_kernel<NS, RAGGED>, smem, cl > 8);
     if (e != cudaSuccess) return cuda_check(e, "sparse_decode_attn: set cluster attributes");
-    return cuda_check(launch_ex(sparse_attn_mma_cluster_kernel<NS>, dim3(cl, rows), dim3(kMmaWarps * 32), smem, stream,
-                                pdl, (unsigned)cl, p),
+    return cuda_check(launch_ex(sparse_attn_mma_cluster_kernel<NS, RAGGED>, dim3(cl, rows), dim3(kMmaWarps * 32), smem,
+                                stream, pdl, (unsigned)cl, p),
                       "sparse_decode_attn: mma cluster launch");
   }
-  cudaError_t e = kernel_attrs((const void*)sparse_attn_mma_kernel<NS>, smem);
+  cudaError_t e = kernel_attrs((const void*)sparse_attn_mma_kernel<NS, RAGGED>, smem);
   if (e != cudaSuccess) return cuda_check(e, "sparse_decode_attn: set smem attribute");
-  return cuda_check(launch_ex(sparse_attn_mma_kernel<NS>, dim3(p.n_ctas), dim3(kMmaWarps * 32), smem, stream, pdl, 0u, p),
-                    "sparse_decode_attn: mma launch");
+  return cuda_check(
+      launch_ex(sparse_attn_mma_kernel<NS, RAGGED>, dim3(p.n_ctas), dim3(kMmaWarps * 32), smem, stream, pdl, 0u, p),
+      "sparse_decode_attn: mma launch");
 }
 
+// A token list with every sequence full (no per-sequence lengths) takes the
+// kernels built for that case alone; the others read the list form and the
+// lengths at run time.  Both skip entries that are no token.
 tls_status launch_attn_mma(const AttnParams& p, int rows, cudaStream_t stream, bool pdl) {
-  return launch_mma<3>(p, rows, stream, pdl);
+  if (p.seq_lens == nullptr && p.list_mode == kListTokens) return launch_mma<3, false>(p, rows, stream, pdl);
+  return launch_mma<3, true>(p, rows, stream, pdl);
 }
 
 }  // namespace tls
