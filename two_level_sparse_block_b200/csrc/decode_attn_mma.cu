@@ -29,6 +29,7 @@ namespace tls {
 constexpr int kMmaWarps = 4;
 constexpr int kChunk = 16;           // tokens per chunk
 constexpr int kChunkBytes = 8192;    // K (4 KB) + V (4 KB) of 16 tokens
+constexpr int kMmaDv = 128;          // K and V row width of these kernels
 
 // two floats -> bf16x2 (round to nearest even); `a` goes to the low half
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
@@ -84,8 +85,8 @@ __host__ __device__ constexpr int mma_stages(int g) { return 3; }
 __host__ __device__ inline MmaLayout mma_layout(int g) {
   MmaLayout L;
   L.off_comb = kMmaWarps * mma_stages(g) * kChunkBytes;    // [warp][h][128] fp32
-  L.off_stat = L.off_comb + kMmaWarps * g * 128 * 4;        // [warp][h] m, then l
-  L.bytes = L.off_stat + 2 * kMmaWarps * 16 * 4 + 16;
+  L.off_stat = L.off_comb + kMmaWarps * g * 128 * 4;        // [warp][h] m, then l; [h] M, then l
+  L.bytes = L.off_stat + (2 * kMmaWarps + 2) * 16 * 4 + 16;
   return L;
 }
 
@@ -312,6 +313,61 @@ __device__ __forceinline__ void mma_fold(int g, float m0, float m1, float l0, fl
   }
 }
 
+// The CTA's warps fold their (m, l) for one row into factors: afterwards
+// comb [warp][h][128] holds each warp's O (relative to its own maximum),
+// cm [warp][h] the factor 2^(m_w - M) that brings it to the CTA's maximum
+// M = hm[h] (0 for a warp that saw no token), and hl[h] the CTA's l
+// relative to M.  All threads of the CTA call it.
+__device__ __forceinline__ void mma_fold_factors(int g, float m0, float m1, float l0, float l1,
+                                                 const float (&o)[16][4], float* comb, float* cm, float* cl,
+                                                 float* hm, float* hl) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+  if (tq == 0) {
+    if (gq < g) {
+      cm[warp * 16 + gq] = m0;
+      cl[warp * 16 + gq] = l0;
+    }
+    if (gq + 8 < g) {
+      cm[warp * 16 + gq + 8] = m1;
+      cl[warp * 16 + gq + 8] = l1;
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const int d = j * 8 + 2 * tq;
+    if (gq < g) *reinterpret_cast<float2*>(comb + (warp * g + gq) * 128 + d) = make_float2(o[j][0], o[j][1]);
+    if (gq + 8 < g) *reinterpret_cast<float2*>(comb + (warp * g + gq + 8) * 128 + d) = make_float2(o[j][2], o[j][3]);
+  }
+  __syncthreads();
+  if (tid < g) {
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kMmaWarps; ++w) M = fmaxf(M, cm[w * 16 + tid]);
+    float L = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kMmaWarps; ++w) {
+      const float mw = cm[w * 16 + tid];
+      const float f = mw == -INFINITY ? 0.0f : exp2f(mw - M);
+      cm[w * 16 + tid] = f;
+      L += f * cl[w * 16 + tid];
+    }
+    hm[tid] = M;
+    hl[tid] = L;
+  }
+  __syncthreads();
+}
+
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 // Persistent form: every CTA owns a contiguous range of the (row, chunk)
 // items; a row spread over several CTAs is merged by the last of them
 // through the split workspace (attn_common.cuh).
@@ -434,10 +490,11 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_kernel(Attn
 
 // Cluster form: one cluster of CL = gridDim.x CTAs per row (row =
 // blockIdx.y).  CTA r streams chunks [r * CPR / CL, (r + 1) * CPR / CL) of
-// the row as above; then every CTA folds its warps and writes its partial
-// (M, l, O per head) into the leader's drained cp.async ring over
-// distributed shared memory, and the leader merges the CL partials by
-// log-sum-exp.  No workspace, ticket or device-wide fence.
+// the row as above; then every CTA folds its warps, and CTA j merges output
+// columns [j * 128 / CL, (j + 1) * 128 / CL) of every head by log-sum-exp:
+// each CTA writes that slice of its folded O, with its (M, l) per head, into
+// CTA j's drained cp.async ring over distributed shared memory.  Two cluster
+// barriers; no workspace, ticket or device-wide fence.
 template <int NS, bool RAGGED>
 __global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_cluster_kernel(AttnParams p) {
   namespace cg = cooperative_groups;
@@ -475,10 +532,11 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_cluster_ker
   const int64_t oh = (int64_t)b * p.n_q_heads + (int64_t)kvh * p.group + h0;  // first output head
 
   grid_launch_dependents();
-  if (tid == 0 && rank == 0) {
-    // the leader writes the output and lse rows last: warm them now
-    prefetch_l2(reinterpret_cast<const uint8_t*>(p.out) + oh * p.dv * (p.out_bf16 ? 2 : 4));
-    if (p.lse != nullptr) prefetch_l2(p.lse + oh);
+  if (tid == 0) {
+    // every CTA writes its column slice of the output rows last (the leader
+    // the lse values too): warm them now
+    prefetch_l2(reinterpret_cast<const uint8_t*>(p.out) + (oh * kMmaDv + rank * (kMmaDv / CL)) * (p.out_bf16 ? 2 : 4));
+    if (p.lse != nullptr && rank == 0) prefetch_l2(p.lse + oh);
   }
   uint32_t qa[8][4];
   mma_load_q(p, b, kvh, h0, g, lane, qa);  // q is an input of the step, not of the preceding kernel
@@ -507,33 +565,56 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 2) sparse_attn_mma_cluster_ker
     __syncwarp();
   }
   cp_async_wait<0>();
-  cluster.sync();  // every CTA (the leader included) is done with its ring
+  // barrier 1, split: arrive once this CTA's ring is drained, fold the warps
+  // meanwhile, and wait before writing into the other CTAs' rings
+  cluster_arrive_release();
+  float* hm = cl + kMmaWarps * 16;
+  float* hl = hm + 16;
+  mma_fold_factors(g, m0, m1, l0, l1, o, comb, cm, cl, hm, hl);
+  // CTA j merges output columns [j W, (j + 1) W) of every head: it receives
+  // from every CTA r that slice of r's folded O and r's (M, l), in its own
+  // drained ring
+  const int W = kMmaDv / CL;
+  float* recv = reinterpret_cast<float*>(sm);  // [CL][g][W]
+  float* recv_ml = recv + CL * g * W;          // [CL][g] (M, l)
+  cluster_wait_acquire();
+  for (int idx = tid; idx < g * kMmaDv; idx += kMmaWarps * 32) {
+    const int h = idx / kMmaDv, e = idx - h * kMmaDv;
+    float v = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kMmaWarps; ++w) v += cm[w * 16 + h] * comb[(w * g + h) * kMmaDv + e];
+    const int j = e / W;
+    cluster.map_shared_rank(recv, j)[(rank * g + h) * W + (e - j * W)] = v;
+  }
+  for (int idx = tid; idx < g * CL; idx += kMmaWarps * 32) {
+    const int j = idx / g, h = idx - j * g;
+    float* dst = cluster.map_shared_rank(recv_ml, j) + (rank * g + h) * 2;
+    dst[0] = hm[h];
+    dst[1] = hl[h];
+  }
+  cluster_arrive_release();
+  cluster_wait_acquire();  // every slice has landed; nothing remote is touched after this
 
-  // partials [CL][g][130] over the leader's ring
-  float* part = reinterpret_cast<float*>(sm);
-  float* dst = cluster.map_shared_rank(part, 0) + (size_t)rank * g * 130;
-  mma_fold(g, m0, m1, l0, l1, o, comb, cm, cl, [&](int h, int e, float v) { dst[h * 130 + e] = v; });
-  cluster.sync();  // the partials have landed; nothing remote is touched after this
-  if (rank != 0) return;
-
-  const int dv = p.dv;
-  for (int idx = tid; idx < g * dv; idx += kMmaWarps * 32) {
-    const int h = idx / dv, e = idx - h * dv;
+  for (int idx = tid; idx < g * W; idx += kMmaWarps * 32) {
+    const int h = idx / W, c = idx - h * W;
     float M = -INFINITY;
-    for (int r = 0; r < CL; ++r) M = fmaxf(M, part[(r * g + h) * 130]);
+    for (int r = 0; r < CL; ++r) M = fmaxf(M, recv_ml[(r * g + h) * 2]);
     float lsum = 0.0f, acc = 0.0f;
-    for (int r = 0; r < CL; ++r) {
-      const float* pr = part + (r * g + h) * 130;
-      if (pr[0] == -INFINITY) continue;
-      const float f = exp2f(pr[0] - M);
-      lsum += f * pr[1];
-      acc += f * pr[2 + e];
+    if (M != -INFINITY) {
+      for (int r = 0; r < CL; ++r) {
+        const float mr = recv_ml[(r * g + h) * 2];
+        if (mr == -INFINITY) continue;
+        const float f = exp2f(mr - M);
+        lsum += f * recv_ml[(r * g + h) * 2 + 1];
+        acc += f * recv[(r * g + h) * W + c];
+      }
     }
     const float val = lsum > 0.0f ? acc / lsum : 0.0f;
-    const int64_t oe = (oh + h) * dv + e;
+    const int64_t oe = (oh + h) * kMmaDv + rank * W + c;
     if (p.out_bf16) reinterpret_cast<uint16_t*>(p.out)[oe] = f32_to_bf16_rn(val);
     else reinterpret_cast<float*>(p.out)[oe] = val;
-    if (e == 0 && p.lse != nullptr) p.lse[oh + h] = (M + log2f(lsum)) * 0.69314718055994531f;
+    if (rank == 0 && c == 0 && p.lse != nullptr)
+      p.lse[oh + h] = lsum > 0.0f ? (M + log2f(lsum)) * 0.69314718055994531f : -INFINITY;
   }
 }
 
@@ -563,13 +644,13 @@ int attn_mma_plan(int rows, int k, int* chunks_per_row, int* n_items, int* n_cta
 
 // Cluster size of the cluster form for `rows` virtual rows of `hpc` heads:
 // the largest of 16, 8, 4, 2 whose grid (rows x CL CTAs) fits two CTAs per
-// SM and whose CL partials fit the leader's ring (CL * hpc * 130 floats);
+// SM and whose merge slices fit a CTA's ring (hpc * (128 + 2 CL) floats);
 // 0 when even CL = 2 does not fit (many rows: the persistent form).
 int attn_mma_cluster_size(int rows, int hpc) {
   const int ring_floats = kMmaWarps * mma_stages(hpc) * kChunkBytes / 4;
   for (int cl = 16; cl >= 2; cl /= 2) {
     if ((int64_t)rows * cl > 2 * (int64_t)kNumSMs) continue;
-    if ((int64_t)cl * hpc * 130 > ring_floats) continue;
+    if ((int64_t)hpc * (kMmaDv + 2 * cl) > ring_floats) continue;
     return cl;
   }
   return 0;
