@@ -78,6 +78,7 @@ tls_status noalloc_scratch(void** out);
 tls_status plan_workspace(const tls_shape& s, int K_b, int k, WsLayout* out);
 
 constexpr int kNumSMs = 148;
+constexpr size_t kMaxDynSmem = 227 * 1024;  // dynamic shared memory a CTA may opt into
 
 // Where entry t of a row's attention list comes from: the token list
 // (token_idx), every position in order (t itself: full attention), or the
@@ -122,7 +123,11 @@ TokenDispatch token_dispatch(const tls_shape& s, int K_b, bool lean, bool aligne
 
 // cudaFuncSetAttribute once per kernel, device and value (the dynamic shared
 // memory limit only ever rises): a launch path that runs every decode step
-// should not pay the driver calls each time.
+// should not pay the driver calls each time.  Every kernel also prefers the
+// largest shared-memory carve-out: an SM configured for a kernel with little
+// shared memory cannot take a CTA of a concurrent kernel that needs more (the
+// staggered step runs level 1 beside level 2), and none of these kernels
+// keeps data in L1.
 inline cudaError_t kernel_attrs(const void* fn, size_t smem_bytes, bool nonportable_cluster = false) {
   struct Key {
     const void* fn;
@@ -133,21 +138,30 @@ inline cudaError_t kernel_attrs(const void* fn, size_t smem_bytes, bool nonporta
     size_t operator()(const Key& k) const { return std::hash<const void*>()(k.fn) * 31u + (size_t)k.dev; }
   };
   static std::mutex mu;
-  static std::unordered_map<Key, std::pair<size_t, bool>, KeyHash> done;
+  struct Set {
+    size_t smem = 0;
+    bool nonportable = false, carveout = false;
+  };
+  static std::unordered_map<Key, Set, KeyHash> done;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lock(mu);
-  auto& d = done[Key{fn, dev}];
-  if (smem_bytes > d.first) {
+  Set& d = done[Key{fn, dev}];
+  if (!d.carveout) {
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    d.carveout = true;
+  }
+  if (smem_bytes > d.smem) {
     e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes);
     if (e != cudaSuccess) return e;
-    d.first = smem_bytes;
+    d.smem = smem_bytes;
   }
-  if (nonportable_cluster && !d.second) {
+  if (nonportable_cluster && !d.nonportable) {
     e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
-    d.second = true;
+    d.nonportable = true;
   }
   return cudaSuccess;
 }

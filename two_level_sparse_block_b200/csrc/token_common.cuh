@@ -87,22 +87,38 @@ __device__ __forceinline__ void load_qlab(const TokenParams& p, int row, float* 
 // block, 0 .. K_b - 1).  Returns how many entries are blocks (not the -1 that
 // ends a list); every thread of the CTA must call it, and it ends with a CTA
 // barrier, after which sb is complete.
-template <int NT>
-__device__ __forceinline__ int load_block_list(const TokenParams& p, int row, int32_t* sb) {
+// `pre` runs once in every thread while the first list loads are in flight,
+// before the barrier (work that waits on other loads of the same thread).
+template <int NT, typename Pre>
+__device__ __forceinline__ int load_block_list(const TokenParams& p, int row, int32_t* sb, Pre pre) {
   int nvb = 0;
   for (int base = 0; base < p.K_b; base += NT) {
     const int i = base + (int)threadIdx.x;
-    bool valid = false;
-    if (i < p.K_b) {
-      // L2 loads: the list is written by the preceding kernel while this grid
-      // may already be resident (programmatic dependent launch)
-      const int v = p.block_idx == nullptr ? i : __ldcg(p.block_idx + (int64_t)row * p.K_b + i);
-      valid = v >= 0;
-      sb[i] = min(max(v, 0), p.nb - 1);
-    }
-    nvb += __syncthreads_count(valid);
+    int v = -1;
+    // L2 loads: the list is written by the preceding kernel while this grid
+    // may already be resident (programmatic dependent launch)
+    if (i < p.K_b) v = p.block_idx == nullptr ? i : __ldcg(p.block_idx + (int64_t)row * p.K_b + i);
+    if (base == 0) pre();
+    if (i < p.K_b) sb[i] = min(max(v, 0), p.nb - 1);
+    nvb += __syncthreads_count(i < p.K_b && v >= 0);
   }
   return nvb;
+}
+template <int NT>
+__device__ __forceinline__ int load_block_list(const TokenParams& p, int row, int32_t* sb) {
+  return load_block_list<NT>(p, row, sb, [] {});
+}
+
+// The group's query rows (G x Dqk bf16, contiguous in q) copied into shared
+// memory by 16-byte async copies, committed as one group (q 16-byte aligned,
+// Dqk a multiple of 8).
+template <int NT>
+__device__ __forceinline__ void stage_query_rows(const TokenParams& p, int row, uint16_t* sq) {
+  const int g = p.group, b = row / p.n_kv_heads, kvh = row % p.n_kv_heads;
+  const uint16_t* qg = p.q + ((int64_t)b * p.n_q_heads + (int64_t)kvh * g) * p.dqk;
+  const uint32_t s0 = smem_addr32(sq);
+  for (int i = threadIdx.x; i < g * p.dqk / 8; i += NT) cp_async16(s0 + (uint32_t)i * 16u, qg + (int64_t)i * 8, 16u);
+  cp_async_commit();
 }
 
 // Candidates of a row that are tokens of its sequence: the lists are

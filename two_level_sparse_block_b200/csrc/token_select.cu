@@ -189,11 +189,25 @@ __global__ void __launch_bounds__(NT, NT >= 1024 || KPT > 8 ? 1 : 2) token_selec
   float* qlab = sscales + bpc * p.bs;                                             // [G][R]
   int32_t* bidx = reinterpret_cast<int32_t*>(qlab + p.group * R);                 // [K_b]
   TopkScratch* ts = reinterpret_cast<TopkScratch*>(bidx + ((p.K_b + 3) & ~3));
+  int32_t* slab = reinterpret_cast<int32_t*>(ts + 1);                             // [R] label channels
+  uint16_t* sq = reinterpret_cast<uint16_t*>(
+      (reinterpret_cast<uintptr_t>(slab + R) + 15) & ~uintptr_t(15));             // [G][Dqk] query rows
   if (cl > 1) cluster_arrive_relaxed();  // completes once every CTA of the cluster has started
-  load_qlab<R, NT>(p, row, qlab);
+  // the query rows and the label channels (inputs of the step) are loaded
+  // while the block list is: one memory round trip for the three
+  stage_query_rows<NT>(p, row, sq);
+  const int kvh = row % p.n_kv_heads;
+  const int lab = threadIdx.x < R ? __ldg(p.label_ch + kvh * R + threadIdx.x) : 0;
   if (threadIdx.x == 0 && rank == 0) prefetch_l2(p.token_idx + (int64_t)row * p.k);
   grid_dependency_wait();  // the block lists come from the preceding kernel
-  const int nvb = load_block_list<NT>(p, row, bidx);  // ends with a CTA barrier
+  const int nvb = load_block_list<NT>(p, row, bidx, [&] {
+    if (threadIdx.x < R) slab[threadIdx.x] = min(max(lab, 0), p.dqk - 1);  // clamped: never out of bounds
+    cp_async_wait<0>();
+  });  // ends with a CTA barrier
+  for (int i = threadIdx.x; i < p.group * R; i += NT) {
+    const int h = i / R, r = i - h * R;
+    qlab[i] = __uint_as_float((uint32_t)sq[h * p.dqk + slab[r]] << 16);
+  }
   const int n_valid = valid_candidates(p, row, bidx, nvb);
   stage_candidate_codes<R, NT>(p, row, bidx, j0, j1, scodes, sscales);
   __syncthreads();
@@ -223,8 +237,20 @@ __global__ void __launch_bounds__(NT, NT >= 1024 || KPT > 8 ? 1 : 2) token_selec
   cta_topk_regs<NT, KPT>(keys, n_valid, kk, out, *ts, map);
 }
 
+// Dynamic shared memory of the row kernel with cl CTAs of nt threads a row:
+// keys, staged codes and scales, qlab, the block list, the top-k scratch,
+// the label channels and the group's query rows.
+size_t token_row_smem(const tls_shape& s, int K_b, int cl, int nt) {
+  const int n_cand = K_b * s.block_size, g = group_of(s);
+  const int kpt = n_cand <= 2 * nt ? 2 : n_cand <= 4 * nt ? 4 : n_cand <= 8 * nt ? 8 : 16;
+  const int bpc = (K_b + cl - 1) / cl;
+  return (size_t)kpt * nt * 4 + (size_t)bpc * s.block_size * (s.n_label / 2 + 4) +
+         ((size_t)g * s.n_label + ((K_b + 3) & ~3)) * 4 + sizeof(TopkScratch) + (size_t)s.n_label * 4 + 16 +
+         (size_t)g * s.qk_dim * 2;
+}
+
 // Which level-2 kernel a call takes, its CTAs per row and threads per CTA
-// (`lean` as in select_tokens_impl; `aligned`: codes and scales 16-byte
+// (`lean` as in select_tokens_impl; `aligned`: q, codes and scales 16-byte
 // aligned).  The one place the choice is made.
 TokenDispatch token_dispatch(const tls_shape& s, int K_b, bool lean, bool aligned) {
   const int rows = rows_of(s), g = group_of(s), n_cand = K_b * s.block_size;
@@ -232,7 +258,7 @@ TokenDispatch token_dispatch(const tls_shape& s, int K_b, bool lean, bool aligne
     const int cl = token_row_cluster_size(rows, K_b, lean ? kNumSMs / 2 : 2 * kNumSMs);
     // a row alone in its CTA gets 1024 threads: twice the warps to score it
     const int nt = (cl == 1 && n_cand <= 8 * 1024) ? 1024 : kRowThreads;
-    return {TokenDispatch::kRow, "token_select_row_kernel", cl, nt};
+    if (token_row_smem(s, K_b, cl, nt) <= kMaxDynSmem) return {TokenDispatch::kRow, "token_select_row_kernel", cl, nt};
   }
   const bool tc = g >= 16 && g <= 128 && (s.n_label == 16 || s.n_label == 32);
   // rows too long for one CTA's shared memory go to clusters whatever the
@@ -294,14 +320,13 @@ tls_status select_tokens_impl(const tls_shape& s, const void* q, const int32_t* 
   p.token_idx = token_idx;
 
   const size_t smem = ((size_t)p.group * s.n_label + K_b + p.n_cand) * 4 + sizeof(TopkScratch) + 32;
-  const TokenDispatch d = token_dispatch(
-      s, K_b, lean, ((reinterpret_cast<uintptr_t>(codes) | reinterpret_cast<uintptr_t>(scales)) & 15u) == 0);
+  const TokenDispatch d = token_dispatch(s, K_b, lean,
+                                         ((reinterpret_cast<uintptr_t>(codes) | reinterpret_cast<uintptr_t>(scales) |
+                                           reinterpret_cast<uintptr_t>(q)) & 15u) == 0);
   if (d.kind == TokenDispatch::kRow) {
     const int cl = d.cl, nt = d.threads;
     const int kpt = p.n_cand <= 2 * nt ? 2 : p.n_cand <= 4 * nt ? 4 : p.n_cand <= 8 * nt ? 8 : 16;
-    const int bpc = (K_b + cl - 1) / cl;
-    const size_t rsmem = (size_t)kpt * nt * 4 + (size_t)bpc * s.block_size * (s.n_label / 2 + 4) +
-                         ((size_t)p.group * s.n_label + ((K_b + 3) & ~3)) * 4 + sizeof(TopkScratch);
+    const size_t rsmem = token_row_smem(s, K_b, cl, nt);
     auto launch = [&](auto kernel) -> tls_status {
       cudaError_t e = kernel_attrs((const void*)kernel, rsmem);
       if (e != cudaSuccess) return cuda_check(e, "select_tokens: set kernel attributes");
