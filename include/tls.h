@@ -382,7 +382,8 @@ TLS_API void tls_block_cache_destroy(tls_block_cache* cache);
  * resident blocks.  Each block of T_t gets a victim slot that holds no block
  * of in_use_block_idx[row] (the blocks the running attention reads, M_{t-1})
  * nor of M_t, preferring free slots, then the least recently used, then the
- * lower slot.  The plan is committed to the cache's host mirror.
+ * lower slot; copy i (in row, then list order) takes the i-th victim in slot
+ * order.  The plan is committed to the cache's host mirror.
  * new_block_idx, in_use_block_idx: host int32 [B, Hkv, K_b] (in_use may be
  * NULL for none).  copy_row/copy_block/copy_slot: host int32 arrays of
  * capacity B*Hkv*K_b receiving the plan (may be NULL); *n_copy = |T_t| summed
@@ -419,7 +420,37 @@ TLS_API tls_status tls_prefetch_diff(tls_block_cache* cache, const int32_t* new_
                              const int32_t* in_use_block_idx_host, int32_t K_b,
                              void* copy_stream, void* done_event, int32_t* n_copied);
 
-/* Copies the host mirror of the slot table (int32 [B, Hkv, NB]) into `table`. */
+/*
+ * Incremental prefetch planned on the device (section 2.B), for block lists
+ * that live on the device (as level 1 writes them): one kernel of one CTA
+ * plans T_t = M_t \ C_t and its victims from new_block_idx_dev (M_t) and
+ * in_use_block_idx_dev (M_{t-1}, may be NULL), updates the device slot table
+ * and the cache state, and a second kernel pulls the planned blocks from
+ * mapped pinned host memory into their slots -- both on copy_stream, with no
+ * host wait.  The plan is the one tls_block_cache_plan makes (the same
+ * victims and slots; the tables of the two paths are equal).
+ * Each row of new_block_idx_dev must hold distinct blocks in [0, NB),
+ * ascending, with any -1 at the end.  n_copied_dev: optional int32 in device
+ * or mapped pinned memory, written on the device with the number of copied
+ * blocks, or -1 when the plan failed (a list that breaks the rule above:
+ * TLS_ERR_INVALID_ARG; too few evictable slots: TLS_ERR_CAPACITY); a failed
+ * plan changes nothing, and the cache then returns that status from every
+ * later transfer, plan or engine step.  done_event as in tls_prefetch_diff.
+ * Needs a cache whose K/V are mapped pinned host memory (the pull path),
+ * n_slots <= 32768 and B*Hkv*K_b <= 65536 (else TLS_ERR_UNSUPPORTED).  From
+ * the first call on, the device holds the cache state: the host calls
+ * (tls_block_cache_plan, tls_prefetch_diff, tls_block_cache_table) first
+ * wait for the device to finish (cudaDeviceSynchronize) and read it back.
+ * TLS_FAULT_INJECT=copy fails the call with TLS_ERR_COPY before anything is
+ * queued.
+ */
+TLS_API tls_status tls_prefetch_diff_device(tls_block_cache* cache, const int32_t* new_block_idx_dev,
+                                            const int32_t* in_use_block_idx_dev, int32_t K_b, void* copy_stream,
+                                            void* done_event, int32_t* n_copied_dev);
+
+/* Copies the slot table (int32 [B, Hkv, NB]) into `table`: the host mirror,
+ * or, once the device plans the cache, the device table after a
+ * cudaDeviceSynchronize. */
 TLS_API tls_status tls_block_cache_table(const tls_block_cache* cache, int32_t* table);
 
 /* ------------------------------------------------------------------------
@@ -478,8 +509,14 @@ TLS_API tls_status tls_engine_create_resident(const tls_shape* shape, int32_t K_
  * and the blocks of M_t not yet resident are copied from host memory on the
  * engine's copy stream while the attention runs; step t+1's attention waits
  * for them.  The first step selects M_{-1} from its own q and makes it
- * resident before attending.  The call waits on the host for level 1 of step
- * t (to plan the transfer); everything else is asynchronous.  A resident
+ * resident before attending.  When the cache allows it (as for
+ * tls_prefetch_diff_device), the transfer is planned on the device
+ * (tls_prefetch_diff_device on the copy stream, after level 1 and after the
+ * attention of step t-1) and the call does not wait on the host at all; else,
+ * or with TLS_ENGINE_PLANNER=host in the environment at engine creation, the
+ * call waits on the host for level 1 of step t to plan it (tls_prefetch_diff).
+ * A failed device plan is seen by the next step (or tls_engine_stats), which
+ * returns its status.  A resident
  * engine (tls_engine_create_resident) has no transfer and no host wait: on
  * `stream` it records q_t, runs level 2 over M_{t-1} and the attention, and
  * waits for level 1 of step t (engine stream, after q_t) before returning, so

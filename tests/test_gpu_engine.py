@@ -61,9 +61,11 @@ def _orow(cfg, q, K, V, lab, b, h, **kw):
                              cfg.softmax_scale, **kw)
 
 
+@pytest.mark.parametrize("planner", ["device", "host"])
 @pytest.mark.parametrize("cfg", ENGINE, ids=lambda c: c.name)
-def test_engine_follows_the_staggered_oracle(cfg):
+def test_engine_follows_the_staggered_oracle(cfg, planner, monkeypatch):
     runtime, tls = _rt()
+    monkeypatch.setenv("TLS_ENGINE_PLANNER", planner)
     qs = synth.gen_query_trajectory(cfg)
     K, V, _ = synth.gen_kv(cfg, qs[0])
     lab = synth.gen_label_channels(cfg)
@@ -168,6 +170,7 @@ def test_engine_host_wait_times_out_and_sticks(monkeypatch):
     # same status, and the device drains and stays healthy
     runtime, tls = _rt()
     monkeypatch.setenv("TLS_HOST_WAIT_MS", "50")
+    monkeypatch.setenv("TLS_ENGINE_PLANNER", "host")  # the device planner has no host wait
     cfg = ENGINE[0]
     qs = synth.gen_query_trajectory(cfg, 3)
     K, V, _ = synth.gen_kv(cfg, qs[0])
@@ -448,3 +451,128 @@ def test_prefetch_diff_records_its_done_event():
     finally:
         torch.cuda.synchronize()
         tls.tls_block_cache_destroy(cache)
+
+
+def _cache_pair(tls, cfg, n_slots):
+    # two caches over the same pinned K/V: one planned on the host, one on the device
+    q = synth.gen_queries(cfg)
+    K, V, _ = synth.gen_kv(cfg, q)
+    bs, nb = cfg.block_size, cfg.n_blocks
+    host_k = torch.from_numpy(np.ascontiguousarray(K).view(np.int16)).pin_memory()
+    host_v = torch.from_numpy(np.ascontiguousarray(V).view(np.int16)).pin_memory()
+    shape = tls.make_shape(cfg.batch, cfg.n_q_heads, cfg.n_kv_heads, cfg.qk_dim, cfg.v_dim, -1, bs, cfg.n_label,
+                           cfg.ctx_len, cfg.softmax_scale)
+    out = []
+    for _ in range(2):
+        slot_k = torch.zeros((n_slots, bs, cfg.qk_dim), dtype=torch.bfloat16, device="cuda")
+        slot_v = torch.zeros((n_slots, bs, cfg.v_dim), dtype=torch.bfloat16, device="cuda")
+        table = torch.full((cfg.batch, cfg.n_kv_heads, nb), -1, dtype=torch.int32, device="cuda")
+        cache = tls.tls_block_cache_create(shape, host_k, host_v, cfg.qk_dim, cfg.v_dim, n_slots, slot_k, slot_v,
+                                           table)
+        out.append((cache, slot_k, slot_v, table))
+    return K, V, host_k, host_v, out
+
+
+def test_device_planner_evicts_what_the_host_planner_evicts():
+    # the same churning sequence of block lists through tls_prefetch_diff (host
+    # plan) and tls_prefetch_diff_device (device plan): after every round both
+    # caches have the same slot table (the same victims -- free slots, then
+    # least recently used, then lower slot -- taken in slot order) and copied
+    # as many; every resident block's slot holds its K and V rows
+    runtime, tls = _rt()
+    cfg = ENGINE[2]
+    rows, nb, bs, K_b = cfg.rows, cfg.n_blocks, cfg.block_size, cfg.K_b
+    n_slots = 2 * rows * K_b + 5
+    K, V, host_k, host_v, caches = _cache_pair(tls, cfg, n_slots)
+    (hc, _, _, htab), (dc, dk, dv, dtab) = caches
+    rng = np.random.default_rng(11)
+    stream = torch.cuda.Stream()
+    n_dev = torch.zeros(1, dtype=torch.int32, device="cuda")
+    try:
+        prev = None
+        base = np.stack([np.sort(rng.choice(nb, K_b, replace=False)) for _ in range(rows)])
+        for rnd in range(12):
+            # a drifting selection: a few blocks of each row change per round
+            m = base.copy()
+            for r in range(rows):
+                keep = rng.choice(K_b, K_b - 3, replace=False)
+                fresh = rng.choice(np.setdiff1d(np.arange(nb), m[r]), 3, replace=False)
+                m[r] = np.sort(np.concatenate([m[r][keep], fresh]))
+            base = m
+            mm = m.astype(np.int32).reshape(cfg.batch, cfg.n_kv_heads, K_b)
+            n_host = tls.tls_prefetch_diff(hc, mm, prev, K_b, stream)
+            md = torch.from_numpy(mm).cuda()
+            pd = None if prev is None else torch.from_numpy(prev).cuda()
+            torch.cuda.synchronize()
+            tls.tls_prefetch_diff_device(dc, md, pd, K_b, stream, None, n_dev)
+            torch.cuda.synchronize()
+            assert int(n_dev.item()) == n_host, f"round {rnd}: copied {int(n_dev.item())} vs {n_host}"
+            th = np.empty((cfg.batch, cfg.n_kv_heads, nb), dtype=np.int32)
+            td = np.empty_like(th)
+            tls.tls_block_cache_table(hc, th)
+            tls.tls_block_cache_table(dc, td)
+            assert np.array_equal(th, td), f"round {rnd}: slot tables differ"
+            used = td[td >= 0]
+            assert used.size == np.unique(used).size and used.max() < n_slots
+            prev = mm
+        sk = dk.view(torch.int16).cpu().numpy().view(np.uint16)
+        sv = dv.view(torch.int16).cpu().numpy().view(np.uint16)
+        td = dtab.cpu().numpy()
+        for b in range(cfg.batch):
+            for h in range(cfg.n_kv_heads):
+                for blk in np.flatnonzero(td[b, h] >= 0):
+                    s = td[b, h, blk]
+                    assert np.array_equal(sk[s], K[b, h, blk * bs:(blk + 1) * bs])
+                    assert np.array_equal(sv[s], V[b, h, blk * bs:(blk + 1) * bs])
+        # the host path reads the device state back and continues from it
+        m = np.stack([np.sort(rng.choice(nb, K_b, replace=False)) for _ in range(rows)]).astype(np.int32)
+        mm = m.reshape(cfg.batch, cfg.n_kv_heads, K_b)
+        n1 = tls.tls_prefetch_diff(dc, mm, prev, K_b, stream)
+        n2 = tls.tls_prefetch_diff(hc, mm, prev, K_b, stream)
+        assert n1 == n2
+    finally:
+        for c in caches:
+            tls.tls_block_cache_destroy(c[0])
+
+
+def test_device_planner_failures_stick():
+    # too few evictable slots, and a list that is not ascending: the plan
+    # changes nothing, writes -1, and the cache refuses every later transfer
+    runtime, tls = _rt()
+    cfg = ENGINE[2]
+    rows, nb, K_b = cfg.rows, cfg.n_blocks, cfg.K_b
+    stream = torch.cuda.Stream()
+    n_dev = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rng = np.random.default_rng(12)
+    for kind in ("capacity", "order"):
+        n_slots = rows * K_b + (0 if kind == "capacity" else rows * K_b)
+        _, _, _, _, caches = _cache_pair(tls, cfg, n_slots)
+        try:
+            cache = caches[1][0]
+            m = np.stack([np.sort(rng.choice(nb, K_b, replace=False)) for _ in range(rows)]).astype(np.int32)
+            tls.tls_prefetch_diff_device(cache, torch.from_numpy(m).cuda(), None, K_b, stream, None, n_dev)
+            torch.cuda.synchronize()
+            assert int(n_dev.item()) == rows * K_b
+            table0 = np.empty((cfg.batch, cfg.n_kv_heads, nb), dtype=np.int32)
+            tls.tls_block_cache_table(cache, table0)
+            m2 = np.stack([np.sort(rng.choice(np.setdiff1d(np.arange(nb), m[r]), K_b, replace=False))
+                           for r in range(rows)]).astype(np.int32)
+            if kind == "order":
+                m2 = m2[:, ::-1].copy()  # descending
+            tls.tls_prefetch_diff_device(cache, torch.from_numpy(m2).cuda(), torch.from_numpy(m).cuda(), K_b,
+                                         stream, None, n_dev)
+            torch.cuda.synchronize()
+            assert int(n_dev.item()) == -1
+            table1 = np.empty_like(table0)
+            tls.tls_block_cache_table(cache, table1)
+            assert np.array_equal(table0, table1), "a failed plan changed the table"
+            want = tls.TLS_ERR_CAPACITY if kind == "capacity" else tls.TLS_ERR_INVALID_ARG
+            with pytest.raises(tls.TlsError) as e:
+                tls.tls_prefetch_diff_device(cache, torch.from_numpy(m).cuda(), None, K_b, stream, None, n_dev)
+            assert e.value.status == want
+            with pytest.raises(tls.TlsError) as e2:
+                tls.tls_prefetch_diff(cache, m, None, K_b, stream)
+            assert e2.value.status == want
+        finally:
+            for c in caches:
+                tls.tls_block_cache_destroy(c[0])

@@ -16,6 +16,7 @@
 #include <cstring>
 #include <vector>
 
+#include "device_common.cuh"
 #include "host_common.h"
 
 struct tls_block_cache {
@@ -46,6 +47,18 @@ struct tls_block_cache {
   // slots may no longer hold what the host mirror says, so every later
   // transfer or plan returns this status
   tls_status failed = TLS_OK;
+  // Device planning (tls_prefetch_diff_device, the engine): the plan kernel
+  // keeps the owner and last-use arrays on the device; while `device_owned`
+  // the device copies (and the device slot table) are the cache state, and a
+  // host path first downloads them.
+  bool device_owned = false;
+  int64_t* owner_dev = nullptr;
+  int64_t* last_use_dev = nullptr;
+  int4* jobs_dev = nullptr;      // [rows * K_b max] {tok0 lo, tok0 hi, slot, list entry}
+  int32_t* victims_dev = nullptr;
+  int32_t* n_jobs_dev = nullptr;
+  int32_t* dev_failed = nullptr;  // pinned, mapped: set by a plan that found too few evictable slots
+  int max_entries = 0;            // rows * K_b the device arrays were sized for
 };
 
 namespace tls {
@@ -120,7 +133,9 @@ tls_status plan(const tls_block_cache& c, const int32_t* new_idx, const int32_t*
   if (cand.size() < copies->size())
     return fail(TLS_ERR_CAPACITY, "plan: %zu blocks to copy but only %zu evictable slots", copies->size(),
                 cand.size());
+  // copy i (row, then list order) takes the i-th victim in slot order
   victims->assign(cand.begin(), cand.begin() + copies->size());
+  std::sort(victims->begin(), victims->end());
   return TLS_OK;
 }
 
@@ -162,39 +177,56 @@ void commit(tls_block_cache& c, const int32_t* new_idx, int K_b, const std::vect
 // The consumers (the next attention) start after the whole kernel, so the
 // order of the two parts does not matter.
 constexpr int kPullThreads = 256;
+// One job: the block's bs rows of K (and of V) from host memory into its slot.
+__device__ __forceinline__ void pull_block(const uint8_t* host_k, const uint8_t* host_v, uint8_t* slot_k,
+                                           uint8_t* slot_v, int64_t kblk, int64_t vblk, int64_t k_row_bytes,
+                                           int64_t v_row_bytes, int4 jb) {
+  const int64_t tok0 = (int64_t)(uint32_t)jb.x | ((int64_t)jb.y << 32);
+  const int64_t slot = jb.z;
+  for (int part = 0; part < 2; ++part) {
+    const uint8_t* src = part == 0 ? host_k + tok0 * k_row_bytes : (host_v ? host_v + tok0 * v_row_bytes : nullptr);
+    uint8_t* dst = part == 0 ? slot_k + slot * kblk : (slot_v ? slot_v + slot * vblk : nullptr);
+    if (src == nullptr || dst == nullptr) continue;
+    const int64_t n16 = (part == 0 ? kblk : vblk) / 16;
+    const uint4* s4 = reinterpret_cast<const uint4*>(src);
+    uint4* d4 = reinterpret_cast<uint4*>(dst);
+    for (int64_t i0 = threadIdx.x; i0 < n16; i0 += 8 * kPullThreads) {
+      uint4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int64_t i = i0 + (int64_t)u * kPullThreads;
+        if (i < n16) v[u] = __ldcv(s4 + i);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int64_t i = i0 + (int64_t)u * kPullThreads;
+        if (i < n16) d4[i] = v[u];
+      }
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kPullThreads) block_pull_kernel(const uint8_t* host_k, const uint8_t* host_v,
                                                                   uint8_t* slot_k, uint8_t* slot_v, int64_t kblk,
                                                                   int64_t vblk, int64_t k_row_bytes,
                                                                   int64_t v_row_bytes, const int4* jobs, int n_jobs,
                                                                   int32_t* table, const int2* pairs, int n_pairs) {
-  if ((int)blockIdx.x < n_jobs) {
-    const int4 jb = jobs[blockIdx.x];
-    const int64_t tok0 = (int64_t)(uint32_t)jb.x | ((int64_t)jb.y << 32);
-    const int64_t slot = jb.z;
-    for (int part = 0; part < 2; ++part) {
-      const uint8_t* src = part == 0 ? host_k + tok0 * k_row_bytes : (host_v ? host_v + tok0 * v_row_bytes : nullptr);
-      uint8_t* dst = part == 0 ? slot_k + slot * kblk : (slot_v ? slot_v + slot * vblk : nullptr);
-      if (src == nullptr || dst == nullptr) continue;
-      const int64_t n16 = (part == 0 ? kblk : vblk) / 16;
-      const uint4* s4 = reinterpret_cast<const uint4*>(src);
-      uint4* d4 = reinterpret_cast<uint4*>(dst);
-      for (int64_t i0 = threadIdx.x; i0 < n16; i0 += 8 * kPullThreads) {
-        uint4 v[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int64_t i = i0 + (int64_t)u * kPullThreads;
-          if (i < n16) v[u] = __ldcv(s4 + i);
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int64_t i = i0 + (int64_t)u * kPullThreads;
-          if (i < n16) d4[i] = v[u];
-        }
-      }
-    }
-  }
+  if ((int)blockIdx.x < n_jobs)
+    pull_block(host_k, host_v, slot_k, slot_v, kblk, vblk, k_row_bytes, v_row_bytes, jobs[blockIdx.x]);
   if (blockIdx.x == 0)
     for (int i = threadIdx.x; i < n_pairs; i += kPullThreads) table[pairs[i].x] = pairs[i].y;
+}
+
+// The device plan's jobs: a fixed grid strides over the *n_jobs jobs the
+// plan kernel wrote (the table is already updated).
+__global__ void __launch_bounds__(kPullThreads) block_pull_jobs_kernel(const uint8_t* host_k, const uint8_t* host_v,
+                                                                       uint8_t* slot_k, uint8_t* slot_v, int64_t kblk,
+                                                                       int64_t vblk, int64_t k_row_bytes,
+                                                                       int64_t v_row_bytes, const int4* jobs,
+                                                                       const int32_t* n_jobs) {
+  const int n = *n_jobs;
+  for (int j = blockIdx.x; j < n; j += gridDim.x)
+    pull_block(host_k, host_v, slot_k, slot_v, kblk, vblk, k_row_bytes, v_row_bytes, jobs[j]);
 }
 
 // Applies (entry, value) pairs (mapped pinned memory) to the device slot table.
@@ -205,19 +237,326 @@ __global__ void slot_table_update_kernel(int32_t* table, const int2* pairs, int 
   }
 }
 
+// ---------------------------------------------------------------------------
+// Device planning: the same plan as plan() + assign_slots() + commit(), made
+// by one CTA from the device block lists, so no host wait sits between level
+// 1 and the transfer.  Victims are the host plan's set: a slot's key is
+// highest when it is free, then higher the longer it has not been used, and
+// 0 when a block of M_t or M_{t-1} holds it; the n_copy largest keys win,
+// ties to the lower slot (the CTA top-k's rule).  Copy i (in row, then list
+// order) takes the i-th victim in slot order, as in the host plan, so both
+// leave the same table.
+constexpr int kPlanThreads = 1024;
+constexpr int kPlanMaxSlots = 32768;    // keys in shared memory
+constexpr int kPlanMaxEntries = 65536;  // rows * K_b
+
+struct PlanParams {
+  int32_t* table;
+  int64_t* owner;
+  int64_t* last_use;
+  const int32_t* new_idx;  // M_t [rows, K_b]
+  const int32_t* in_use;   // M_{t-1} [rows, K_b] or NULL
+  int rows, nb, K_b, n_slots, bs;
+  int64_t ctx_len, step;   // step: the plan's number (last use of M_t's slots)
+  int4* jobs;
+  int32_t* victims;
+  int32_t* n_jobs;
+  int32_t* n_out;    // optional: n_copy, or -1 when the plan failed
+  int32_t* failed;   // mapped pinned flag, sticky
+};
+
+// Exclusive prefix of v over the CTA; *total receives the sum.  All threads call it.
+__device__ __forceinline__ int plan_block_scan(int v, int* warp_sums, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sums[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < kPlanThreads / 32 ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    warp_sums[lane] = w;  // inclusive
+  }
+  __syncthreads();
+  const int before = (warp > 0 ? warp_sums[warp - 1] : 0) + x - v;
+  *total = warp_sums[kPlanThreads / 32 - 1];
+  __syncthreads();  // warp_sums may be reused
+  return before;
+}
+
+__global__ void __launch_bounds__(kPlanThreads, 1) block_plan_kernel(PlanParams p) {
+  extern __shared__ __align__(16) uint32_t pkeys[];  // [n_slots]
+  TopkScratch* ts = reinterpret_cast<TopkScratch*>(pkeys + ((p.n_slots + 3) & ~3));
+  __shared__ int warp_sums[32];
+  __shared__ int bad;
+  const int tid = threadIdx.x;
+  const int E = p.rows * p.K_b;
+  if (*reinterpret_cast<volatile int32_t*>(p.failed) != 0) {
+    if (tid == 0) {
+      *p.n_jobs = 0;
+      if (p.n_out != nullptr) *p.n_out = -1;
+    }
+    return;
+  }
+  if (tid == 0) bad = 0;
+  // 1. keys: free slots highest, then by the age of their last use
+  const uint32_t kFree = float_key(33554432.0f), kKept = float_key(0.0f);
+  for (int s = tid; s < p.n_slots; s += kPlanThreads) {
+    const int64_t age = p.step - p.last_use[s];
+    pkeys[s] = p.owner[s] < 0 ? kFree : float_key((float)(age < 1 ? 1 : (age > 16777215 ? 16777215 : age)));
+  }
+  __syncthreads();
+  // 2. slots holding a block of M_t or M_{t-1} are kept; M_t must list
+  //    distinct blocks in [0, NB) in ascending order (as level 1 writes it)
+  for (int j = tid; j < E; j += kPlanThreads) {
+    const int r = j / p.K_b;
+    const int blk = p.new_idx[j];
+    if (blk >= p.nb) bad = 1;
+    if (blk >= 0 && j % p.K_b > 0) {
+      const int prv = p.new_idx[j - 1];
+      if (prv >= blk || prv < 0) bad = 1;
+    }
+    if (blk >= 0 && blk < p.nb) {
+      const int s = p.table[(int64_t)r * p.nb + blk];
+      if (s >= 0 && s < p.n_slots) pkeys[s] = kKept;
+    }
+    if (p.in_use != nullptr) {
+      const int ub = p.in_use[j];
+      if (ub >= 0 && ub < p.nb) {
+        const int s = p.table[(int64_t)r * p.nb + ub];
+        if (s >= 0 && s < p.n_slots) pkeys[s] = kKept;
+      }
+    }
+  }
+  __syncthreads();
+  // 3. T_t in row, then list order: each thread a contiguous range of entries
+  const int per = (E + kPlanThreads - 1) / kPlanThreads;
+  const int j0 = min(E, tid * per), j1 = min(E, j0 + per);
+  int cnt = 0, avail = 0;
+  for (int j = j0; j < j1; ++j) {
+    const int blk = p.new_idx[j];
+    if (blk >= 0 && blk < p.nb && p.table[(int64_t)(j / p.K_b) * p.nb + blk] < 0) ++cnt;
+  }
+  for (int s = tid; s < p.n_slots; s += kPlanThreads) avail += pkeys[s] != kKept;
+  int n_copy = 0, n_avail = 0;
+  const int base = plan_block_scan(cnt, warp_sums, &n_copy);
+  plan_block_scan(avail, warp_sums, &n_avail);
+  if (bad != 0 || n_copy > n_avail) {
+    // nothing changes; the cache refuses later plans
+    if (tid == 0) {
+      *reinterpret_cast<volatile int32_t*>(p.failed) = bad != 0 ? 2 : 1;
+      *p.n_jobs = 0;
+      if (p.n_out != nullptr) *p.n_out = -1;
+    }
+    return;
+  }
+  int pos = base;
+  for (int j = j0; j < j1; ++j) {
+    const int blk = p.new_idx[j];
+    if (blk >= 0 && blk < p.nb && p.table[(int64_t)(j / p.K_b) * p.nb + blk] < 0) {
+      const int64_t tok0 = (int64_t)(j / p.K_b) * p.ctx_len + (int64_t)blk * p.bs;
+      p.jobs[pos++] = make_int4((int)(uint32_t)(tok0 & 0xFFFFFFFF), (int)(tok0 >> 32), 0, j);
+    }
+  }
+  // 4. the victims: the n_copy largest keys, ascending slots
+  if (n_copy > 0) cta_topk_ascending<kPlanThreads>(pkeys, p.n_slots, n_copy, p.victims, *ts, [](int i) { return i; });
+  __syncthreads();
+  // 5. copy i takes victim i: the evicted block loses its entry, the copied
+  //    one gets the slot (no entry is touched twice: copied blocks are not
+  //    resident, evicted ones are)
+  for (int i = tid; i < n_copy; i += kPlanThreads) {
+    const int slot = p.victims[i];
+    const int j = p.jobs[i].w;
+    const int64_t key = (int64_t)(j / p.K_b) * p.nb + p.new_idx[j];
+    const int64_t old = p.owner[slot];
+    if (old >= 0) p.table[old] = -1;
+    p.table[key] = slot;
+    p.owner[slot] = key;
+    p.jobs[i].z = slot;
+  }
+  __syncthreads();
+  // 6. every block of M_t is resident now: its slot was used at this step
+  for (int j = tid; j < E; j += kPlanThreads) {
+    const int blk = p.new_idx[j];
+    if (blk < 0 || blk >= p.nb) continue;
+    const int s = p.table[(int64_t)(j / p.K_b) * p.nb + blk];
+    if (s >= 0 && s < p.n_slots) p.last_use[s] = p.step;
+  }
+  if (tid == 0) {
+    *p.n_jobs = n_copy;
+    if (p.n_out != nullptr) *p.n_out = n_copy;
+  }
+}
+
+// The host mirror follows the device state again (after device plans): the
+// device work is drained and the table, owners and last uses are copied back.
+tls_status sync_host_mirror(tls_block_cache& c) {
+  if (!c.device_owned) return TLS_OK;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess)
+    e = cudaMemcpy(c.table.data(), c.table_dev, c.table.size() * sizeof(int32_t), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess)
+    e = cudaMemcpy(c.owner.data(), c.owner_dev, c.owner.size() * sizeof(int64_t), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess)
+    e = cudaMemcpy(c.last_use.data(), c.last_use_dev, c.last_use.size() * sizeof(int64_t), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) {
+    c.failed = TLS_ERR_COPY;
+    return fail(TLS_ERR_COPY, "block cache: reading the device state back failed: %s", cudaGetErrorString(e));
+  }
+  c.device_owned = false;
+  return TLS_OK;
+}
+
+// A device plan that failed leaves the flag set: the cache is failed from then on.
+tls_status device_plan_status(tls_block_cache& c) {
+  if (c.dev_failed != nullptr && c.failed == TLS_OK) {
+    const int32_t f = *reinterpret_cast<volatile int32_t*>(c.dev_failed);
+    if (f != 0) c.failed = f == 2 ? TLS_ERR_INVALID_ARG : TLS_ERR_CAPACITY;
+  }
+  if (c.failed != TLS_OK)
+    return fail(c.failed, c.failed == TLS_ERR_CAPACITY
+                              ? "block cache: a device plan found too few evictable slots"
+                              : c.failed == TLS_ERR_INVALID_ARG
+                                    ? "block cache: a device plan got a block list that is not ascending and in range"
+                                    : "block cache: an earlier transfer failed; the slots no longer match the block lists");
+  return TLS_OK;
+}
+
 }  // namespace
+
+// Whether device planning serves this cache for K_b blocks per row, and its
+// device arrays (allocated once, sized for the largest K_b asked for); the
+// host mirror's state is uploaded when the device takes over.
+tls_status block_cache_device_ready(tls_block_cache* c, int K_b) {
+  if (c->dev_host_k == nullptr || c->slot_k == nullptr || c->table_dev == nullptr)
+    return fail(TLS_ERR_UNSUPPORTED, "device planning needs K/V in mapped pinned host memory and device slots");
+  const int64_t entries = (int64_t)c->rows * K_b;
+  if (c->n_slots > kPlanMaxSlots || entries > kPlanMaxEntries)
+    return fail(TLS_ERR_UNSUPPORTED, "device planning takes at most %d slots and %d list entries", kPlanMaxSlots,
+                kPlanMaxEntries);
+  cudaError_t e = cudaSuccess;
+  if (c->owner_dev == nullptr) {
+    e = cudaMalloc((void**)&c->owner_dev, (size_t)c->n_slots * sizeof(int64_t));
+    if (e == cudaSuccess) e = cudaMalloc((void**)&c->last_use_dev, (size_t)c->n_slots * sizeof(int64_t));
+    if (e == cudaSuccess) e = cudaMalloc((void**)&c->n_jobs_dev, sizeof(int32_t));
+    if (e == cudaSuccess)
+      e = cudaHostAlloc((void**)&c->dev_failed, sizeof(int32_t), cudaHostAllocMapped | cudaHostAllocPortable);
+    if (e == cudaSuccess) *c->dev_failed = 0;
+  }
+  if (e == cudaSuccess && entries > c->max_entries) {
+    if (c->jobs_dev != nullptr) cudaFree(c->jobs_dev);
+    if (c->victims_dev != nullptr) cudaFree(c->victims_dev);
+    c->jobs_dev = nullptr;
+    c->victims_dev = nullptr;
+    e = cudaMalloc((void**)&c->jobs_dev, (size_t)entries * sizeof(int4));
+    if (e == cudaSuccess) e = cudaMalloc((void**)&c->victims_dev, (size_t)entries * sizeof(int32_t));
+    if (e == cudaSuccess) c->max_entries = (int)entries;
+  }
+  if (e == cudaSuccess && !c->device_owned) {
+    e = cudaDeviceSynchronize();  // queued host-planned transfers land first
+    if (e == cudaSuccess)
+      e = cudaMemcpy(c->table_dev, c->table.data(), c->table.size() * sizeof(int32_t), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess)
+      e = cudaMemcpy(c->owner_dev, c->owner.data(), c->owner.size() * sizeof(int64_t), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess)
+      e = cudaMemcpy(c->last_use_dev, c->last_use.data(), c->last_use.size() * sizeof(int64_t),
+                     cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) {
+      c->device_owned = true;
+      c->published = true;
+    }
+  }
+  if (e != cudaSuccess) return cuda_check(e, "block cache: device planning state");
+  return TLS_OK;
+}
+
+// The cache's status: a failed transfer or device plan (sticky).
+tls_status block_cache_check(tls_block_cache* c) { return device_plan_status(*c); }
+
+// Bytes one block occupies in the pool (K and, when the cache has them, V rows).
+int64_t block_cache_block_bytes(const tls_block_cache* c) {
+  const int64_t kblk = (int64_t)c->shape.block_size * c->hk_stride * 2;
+  const int64_t vblk = (int64_t)c->shape.block_size * c->hv_stride * 2;
+  return kblk + (c->host_v != nullptr && c->slot_v != nullptr ? vblk : 0);
+}
+
+// The incremental prefetch planned on the device: one plan kernel (one CTA)
+// reads M_t and M_{t-1} from device memory and updates the slot table, the
+// owners and the last uses; a pull kernel copies its jobs.  n_out (device or
+// mapped memory, may be NULL) receives the number of copied blocks, or -1
+// when the plan failed (the cache is failed from then on).
+tls_status prefetch_device_impl(tls_block_cache* c, const int32_t* new_dev, const int32_t* in_use_dev, int K_b,
+                                cudaStream_t cs, int32_t* n_out, cudaEvent_t planned) {
+  tls_status st = device_plan_status(*c);
+  if (st != TLS_OK) return st;
+  if (fault_injected_copy()) return fail(TLS_ERR_COPY, "prefetch_diff: copy failure injected (TLS_FAULT_INJECT=copy)");
+  st = block_cache_device_ready(c, K_b);
+  if (st != TLS_OK) return st;
+  c->step += 1;
+  PlanParams p;
+  p.table = c->table_dev;
+  p.owner = c->owner_dev;
+  p.last_use = c->last_use_dev;
+  p.new_idx = new_dev;
+  p.in_use = in_use_dev;
+  p.rows = c->rows;
+  p.nb = c->nb;
+  p.K_b = K_b;
+  p.n_slots = c->n_slots;
+  p.bs = c->shape.block_size;
+  p.ctx_len = c->shape.ctx_len;
+  p.step = c->step;
+  p.jobs = c->jobs_dev;
+  p.victims = c->victims_dev;
+  p.n_jobs = c->n_jobs_dev;
+  p.n_out = n_out;
+  int32_t* dflag = nullptr;
+  cudaError_t e = cudaHostGetDevicePointer((void**)&dflag, c->dev_failed, 0);
+  p.failed = dflag;
+  const size_t smem = (size_t)((c->n_slots + 3) & ~3) * 4 + sizeof(TopkScratch) + 16;
+  if (e == cudaSuccess) e = kernel_attrs((const void*)block_plan_kernel, smem);
+  if (e != cudaSuccess) return cuda_check(e, "prefetch_diff_device: plan kernel setup");
+  block_plan_kernel<<<1, kPlanThreads, smem, cs>>>(p);
+  e = cudaGetLastError();
+  if (e == cudaSuccess && planned != nullptr) e = cudaEventRecord(planned, cs);  // the lists have been read
+  const int64_t kblk = (int64_t)c->shape.block_size * c->hk_stride * 2;
+  const int64_t vblk = (int64_t)c->shape.block_size * c->hv_stride * 2;
+  const bool with_v = c->host_v != nullptr && c->slot_v != nullptr;
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)c->rows * K_b, 4 * (int64_t)kNumSMs));
+  if (e == cudaSuccess) {
+    block_pull_jobs_kernel<<<grid, kPullThreads, 0, cs>>>(c->dev_host_k, with_v ? c->dev_host_v : nullptr, c->slot_k,
+                                                          with_v ? c->slot_v : nullptr, kblk, vblk, c->hk_stride * 2,
+                                                          c->hv_stride * 2, c->jobs_dev, c->n_jobs_dev);
+    e = cudaGetLastError();
+  }
+  if (e != cudaSuccess) {
+    c->failed = TLS_ERR_COPY;
+    return fail(TLS_ERR_COPY, "prefetch_diff_device: launch failed: %s", cudaGetErrorString(e));
+  }
+  return TLS_OK;
+}
 
 // The incremental prefetch of tls_prefetch_diff without the argument checks
 // (also used by the staggered engine).  *bytes = host -> device bytes of the
 // block copies.
 tls_status prefetch_diff_impl(tls_block_cache* c, const int32_t* new_idx, const int32_t* in_use, int K_b,
                               cudaStream_t cs, int32_t* n_copied, int64_t* bytes) {
-  if (c->failed != TLS_OK)
-    return fail(c->failed, "prefetch_diff: an earlier transfer failed; the slots no longer match the host mirror");
+  tls_status st = device_plan_status(*c);
+  if (st != TLS_OK) return st;
   if (fault_injected_copy()) return fail(TLS_ERR_COPY, "prefetch_diff: copy failure injected (TLS_FAULT_INJECT=copy)");
+  st = sync_host_mirror(*c);
+  if (st != TLS_OK) return st;
   std::vector<Copy> copies;
   std::vector<int32_t> victims;
-  tls_status st = plan(*c, new_idx, in_use, K_b, &copies, &victims);
+  st = plan(*c, new_idx, in_use, K_b, &copies, &victims);
   if (st != TLS_OK) return st;
   std::vector<int2> changes;
   assign_slots(*c, copies, victims, &changes);
@@ -395,6 +734,15 @@ extern "C" void tls_block_cache_destroy(tls_block_cache* c) {
     if (c->staging[i] != nullptr) cudaFreeHost(c->staging[i]);
     if (c->jobs[i] != nullptr) cudaFreeHost(c->jobs[i]);
   }
+  if (c->owner_dev != nullptr) {
+    cudaDeviceSynchronize();  // no plan or pull kernel may still use the arrays
+    cudaFree(c->owner_dev);
+    cudaFree(c->last_use_dev);
+    cudaFree(c->n_jobs_dev);
+    cudaFreeHost(c->dev_failed);
+  }
+  if (c->jobs_dev != nullptr) cudaFree(c->jobs_dev);
+  if (c->victims_dev != nullptr) cudaFree(c->victims_dev);
   delete c;
 }
 
@@ -405,11 +753,13 @@ extern "C" tls_status tls_block_cache_plan(tls_block_cache* c, const int32_t* ne
   if (c == nullptr || new_block_idx == nullptr || n_copy == nullptr)
     return fail(TLS_ERR_INVALID_ARG, "block_cache_plan: NULL argument");
   if (K_b < 1 || K_b > c->nb) return fail(TLS_ERR_INVALID_ARG, "block_cache_plan: K_b out of range");
-  if (c->failed != TLS_OK)
-    return fail(c->failed, "block_cache_plan: an earlier transfer failed; the slots no longer match the host mirror");
+  tls_status st = device_plan_status(*c);
+  if (st != TLS_OK) return st;
+  st = sync_host_mirror(*c);
+  if (st != TLS_OK) return st;
   std::vector<Copy> copies;
   std::vector<int32_t> victims;
-  tls_status st = plan(*c, new_block_idx, in_use_block_idx, K_b, &copies, &victims);
+  st = plan(*c, new_block_idx, in_use_block_idx, K_b, &copies, &victims);
   if (st != TLS_OK) return st;
   std::vector<int2> changes;
   assign_slots(*c, copies, victims, &changes);
@@ -442,6 +792,26 @@ extern "C" tls_status tls_prefetch_diff(tls_block_cache* c, const int32_t* new_b
 extern "C" tls_status tls_block_cache_table(const tls_block_cache* c, int32_t* table) {
   clear_error();
   if (c == nullptr || table == nullptr) return fail(TLS_ERR_INVALID_ARG, "block_cache_table: NULL argument");
+  if (c->device_owned) {
+    // the device table is the state: read it once the queued work is done
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess)
+      e = cudaMemcpy(table, c->table_dev, c->table.size() * sizeof(int32_t), cudaMemcpyDeviceToHost);
+    return e == cudaSuccess ? TLS_OK : cuda_check(e, "block_cache_table: reading the device table");
+  }
   std::memcpy(table, c->table.data(), c->table.size() * sizeof(int32_t));
   return TLS_OK;
+}
+
+extern "C" tls_status tls_prefetch_diff_device(tls_block_cache* c, const int32_t* new_block_idx_dev,
+                                               const int32_t* in_use_block_idx_dev, int32_t K_b, void* copy_stream,
+                                               void* done_event, int32_t* n_copied_dev) {
+  clear_error();
+  if (c == nullptr || new_block_idx_dev == nullptr) return fail(TLS_ERR_INVALID_ARG, "prefetch_diff_device: NULL argument");
+  if (K_b < 1 || K_b > c->nb) return fail(TLS_ERR_INVALID_ARG, "prefetch_diff_device: K_b out of range");
+  tls_status st = prefetch_device_impl(c, new_block_idx_dev, in_use_block_idx_dev, K_b, (cudaStream_t)copy_stream,
+                                       n_copied_dev, nullptr);
+  if (st != TLS_OK || done_event == nullptr) return st;
+  cudaError_t e = cudaEventRecord((cudaEvent_t)done_event, (cudaStream_t)copy_stream);
+  return e == cudaSuccess ? TLS_OK : cuda_check(e, "prefetch_diff_device: done event");
 }

@@ -24,6 +24,8 @@
 // step t+1 reads M_t, which the join at the end of step t completes.  Every
 // step forks and joins within itself, so it can be captured into a graph.
 
+#include <cstdlib>
+#include <cstring>
 #include <vector>
 
 #include "host_common.h"
@@ -33,6 +35,11 @@ tls_status plan_workspace(const tls_shape& s, int K_b, int k, WsLayout* out);
 tls_status prefetch_diff_impl(tls_block_cache* c, const int32_t* new_idx, const int32_t* in_use, int K_b,
                               cudaStream_t cs, int32_t* n_copied, int64_t* bytes);
 tls_status block_cache_view(const tls_block_cache* c, tls_kv_view* kv);
+tls_status block_cache_device_ready(tls_block_cache* c, int K_b);
+tls_status prefetch_device_impl(tls_block_cache* c, const int32_t* new_dev, const int32_t* in_use_dev, int K_b,
+                                cudaStream_t cs, int32_t* n_out, cudaEvent_t planned);
+int64_t block_cache_block_bytes(const tls_block_cache* c);
+tls_status block_cache_check(tls_block_cache* c);
 }  // namespace tls
 
 namespace {
@@ -58,6 +65,11 @@ struct tls_engine {
   cudaEvent_t ready[kRing] = {}, copy_start[kRing] = {}, copy_end[kRing] = {};
   int32_t n_copied[kRing] = {};
   int64_t bytes[kRing] = {};
+  // device planning: the plan kernel writes each step's block count here
+  bool device_plan = false;
+  int32_t* n_copied_map = nullptr;  // pinned, mapped [kRing]
+  int32_t* n_copied_dev = nullptr;  // its device address
+  cudaEvent_t ev_planned = nullptr;  // after the plan kernel, before the pull
   int64_t t = 0;
   tls_status failed = TLS_OK;
   double wait_ms = 10000.0;  // deadline of the host waits (TLS_HOST_WAIT_MS)
@@ -70,8 +82,9 @@ namespace {
 void release(tls_engine* e) {
   if (e->sel != nullptr) cudaStreamSynchronize(e->sel);
   if (e->copy != nullptr) cudaStreamSynchronize(e->copy);
-  for (cudaEvent_t* ev : {&e->ev_q, &e->ev_sel, &e->ev_attn[0], &e->ev_attn[1]})
+  for (cudaEvent_t* ev : {&e->ev_q, &e->ev_sel, &e->ev_attn[0], &e->ev_attn[1], &e->ev_planned})
     if (*ev != nullptr) cudaEventDestroy(*ev);
+  if (e->n_copied_map != nullptr) cudaFreeHost(e->n_copied_map);
   for (int i = 0; i < kRing; ++i)
     for (cudaEvent_t ev : {e->ready[i], e->copy_start[i], e->copy_end[i]})
       if (ev != nullptr) cudaEventDestroy(ev);
@@ -148,6 +161,29 @@ tls_status engine_create(const tls_shape* shape, int32_t K_b, int32_t k, const v
     release(e);
     return cuda_check(ce, "engine_create: streams, events or pinned mirrors");
   }
+  // the transfer is planned on the device when the cache allows it (K/V in
+  // mapped pinned memory, pool and lists within the plan kernel's sizes);
+  // TLS_ENGINE_PLANNER=host keeps the host planner
+  const char* planner = std::getenv("TLS_ENGINE_PLANNER");
+  if (cache != nullptr && !(planner != nullptr && std::strcmp(planner, "host") == 0)) {
+    st = block_cache_device_ready(cache, K_b);
+    if (st == TLS_OK) {
+      ce = cudaHostAlloc((void**)&e->n_copied_map, kRing * sizeof(int32_t), cudaHostAllocMapped | cudaHostAllocPortable);
+      if (ce == cudaSuccess) ce = cudaHostGetDevicePointer((void**)&e->n_copied_dev, e->n_copied_map, 0);
+      if (ce == cudaSuccess) ce = cudaEventCreateWithFlags(&e->ev_planned, cudaEventDisableTiming);
+      if (ce != cudaSuccess) {
+        release(e);
+        return cuda_check(ce, "engine_create: device planning buffers");
+      }
+      for (int i = 0; i < kRing; ++i) e->n_copied_map[i] = 0;
+      e->device_plan = true;
+    } else if (st == TLS_ERR_UNSUPPORTED) {
+      clear_error();  // the host planner serves this cache
+    } else {
+      release(e);
+      return st;
+    }
+  }
   *out = e;
   return TLS_OK;
 }
@@ -220,8 +256,73 @@ tls_status resident_step(tls_engine* e, const void* q, int32_t out_dtype, void* 
   return TLS_OK;
 }
 
+// The offloaded step with the transfer planned on the device: no host wait.
+// Beside the host-planned order, two device-side waits take the place of the
+// host's: level 2 waits for the level 1 of the step before (it reads M_{t-1}),
+// and level 1 waits for the plan kernel of the step before (which read the
+// list level 1 now overwrites).
+tls_status device_step(tls_engine* e, const void* q, int32_t out_dtype, void* out, float* lse, cudaStream_t A) {
+  const tls_shape& s = e->shape;
+  const int cur = (int)(e->t & 1), prev = cur ^ 1;
+  const int ri = (int)(e->t % kRing), rp = (int)((e->t + kRing - 1) % kRing);
+  tls_status st = block_cache_check(e->cache);  // a failed plan of an earlier step stops the engine
+  if (st != TLS_OK) return st;
+  cudaError_t ce;
+  if (e->t == 0) {
+    // prologue: M_{-1} from q_0 on A, pulled in on the copy stream
+    st = select_blocks_impl(s, q, e->meta, e->K_b, e->bidx[prev], nullptr, e->ws, e->L, A);
+    if (st != TLS_OK) return st;
+    ce = cudaEventRecord(e->ev_sel, A);
+    if (ce == cudaSuccess) ce = cudaStreamWaitEvent(e->copy, e->ev_sel, 0);
+    if (ce == cudaSuccess) ce = cudaEventRecord(e->copy_start[rp], e->copy);
+    if (ce != cudaSuccess) return cuda_check(ce, "engine_step: prologue");
+    e->n_copied_map[rp] = 0;
+    st = prefetch_device_impl(e->cache, e->bidx[prev], nullptr, e->K_b, e->copy, e->n_copied_dev + rp, e->ev_planned);
+    if (st != TLS_OK) return st;
+    ce = cudaEventRecord(e->copy_end[rp], e->copy);
+    if (ce != cudaSuccess) return cuda_check(ce, "engine_step: prologue");
+  }
+  // M_{t-1} (written by level 1 of the step before) is complete before level 2
+  ce = cudaStreamWaitEvent(A, e->ev_sel, 0);
+  if (ce == cudaSuccess) ce = cudaEventRecord(e->ev_q, A);
+  // level 1 for q_t on the select stream: M_t, once the plan of the step
+  // before has read the list it overwrites
+  if (ce == cudaSuccess) ce = cudaStreamWaitEvent(e->sel, e->ev_q, 0);
+  if (ce == cudaSuccess) ce = cudaStreamWaitEvent(e->sel, e->ev_planned, 0);
+  if (ce != cudaSuccess) return cuda_check(ce, "engine_step: select stream");
+  st = select_blocks_impl(s, q, e->meta, e->K_b, e->bidx[cur], nullptr, e->ws, e->L, e->sel);
+  if (st != TLS_OK) return st;
+  ce = cudaEventRecord(e->ev_sel, e->sel);
+  if (ce != cudaSuccess) return cuda_check(ce, "engine_step: select stream");
+  // level 2 within M_{t-1} and the attention over the slot pool, on A
+  st = select_tokens_impl(s, q, e->label_ch, e->codes, e->scales, e->bidx[prev], e->K_b, e->k, e->token_idx, nullptr,
+                          e->ws, e->L, A, /*pdl=*/false);
+  if (st != TLS_OK) return st;
+  ce = cudaEventRecord(e->ready[ri], A);
+  if (ce == cudaSuccess) ce = cudaStreamWaitEvent(A, e->copy_end[rp], 0);  // T_{t-1} has landed
+  if (ce != cudaSuccess) return cuda_check(ce, "engine_step: wait for the transfer");
+  st = sparse_attn_impl(s, q, e->kv, e->token_idx, e->k, out_dtype, out, lse, e->ws, e->L, A, /*pdl=*/false);
+  if (st != TLS_OK) return st;
+  ce = cudaEventRecord(e->ev_attn[cur], A);
+  // T_t on the copy stream, once M_t is chosen and the attention of step t-1
+  // (whose slots may be evicted now) is done; alongside the attention of step t
+  if (ce == cudaSuccess) ce = cudaStreamWaitEvent(e->copy, e->ev_sel, 0);
+  if (ce == cudaSuccess) ce = cudaStreamWaitEvent(e->copy, e->ev_attn[prev], 0);
+  if (ce == cudaSuccess) ce = cudaEventRecord(e->copy_start[ri], e->copy);
+  if (ce != cudaSuccess) return cuda_check(ce, "engine_step: copy stream");
+  e->n_copied_map[ri] = 0;
+  st = prefetch_device_impl(e->cache, e->bidx[cur], e->bidx[prev], e->K_b, e->copy, e->n_copied_dev + ri,
+                            e->ev_planned);
+  if (st != TLS_OK) return st;
+  ce = cudaEventRecord(e->copy_end[ri], e->copy);
+  if (ce != cudaSuccess) return cuda_check(ce, "engine_step: copy stream");
+  e->t += 1;
+  return TLS_OK;
+}
+
 tls_status engine_step(tls_engine* e, const void* q, int32_t out_dtype, void* out, float* lse, cudaStream_t A) {
   if (e->cache == nullptr) return resident_step(e, q, out_dtype, out, lse, A);
+  if (e->device_plan) return device_step(e, q, out_dtype, out, lse, A);
   const tls_shape& s = e->shape;
   const size_t list_bytes = (size_t)e->rows * e->K_b * sizeof(int32_t);
   const int cur = (int)(e->t & 1), prev = cur ^ 1;
@@ -316,6 +417,17 @@ extern "C" tls_status tls_engine_stats(tls_engine* e, int64_t step, tls_engine_s
   const int si = (int)((step + kRing) % kRing);
   tls_status st = wait_event_deadline(e->copy_end[si], e->wait_ms, "engine_stats: transfer");
   if (st != TLS_OK) return st;
+  int32_t n_copied = e->n_copied[si];
+  int64_t bytes_copied = e->bytes[si];
+  if (e->device_plan) {
+    // written by the step's plan kernel, which ran before copy_end
+    n_copied = *reinterpret_cast<volatile int32_t*>(e->n_copied_map + si);
+    if (n_copied < 0) {
+      st = block_cache_check(e->cache);
+      return st != TLS_OK ? st : fail(TLS_ERR_CAPACITY, "engine_stats: the plan of step %lld failed", (long long)step);
+    }
+    bytes_copied = (int64_t)n_copied * block_cache_block_bytes(e->cache);
+  }
   float copy_ms = 0.0f, exposed_ms = -1.0f;
   cudaError_t ce = cudaEventElapsedTime(&copy_ms, e->copy_start[si], e->copy_end[si]);
   if (ce == cudaSuccess && step + 1 < e->t) {
@@ -327,8 +439,8 @@ extern "C" tls_status tls_engine_stats(tls_engine* e, int64_t step, tls_engine_s
   }
   if (ce != cudaSuccess) return cuda_check(ce, "engine_stats: events");
   out->step = step;
-  out->n_copied = e->n_copied[si];
-  out->bytes_copied = e->bytes[si];
+  out->n_copied = n_copied;
+  out->bytes_copied = bytes_copied;
   out->copy_ms = copy_ms;
   out->exposed_ms = exposed_ms;
   return TLS_OK;

@@ -96,6 +96,7 @@ _SIG = {
     "tls_block_cache_destroy": (None, [_P]),
     "tls_block_cache_plan": (_I32, [_P, _P, _P, _I32, _P, _P, _P, _P]),
     "tls_prefetch_diff": (_I32, [_P, _P, _P, _I32, _P, _P, _P]),
+    "tls_prefetch_diff_device": (_I32, [_P, _P, _P, _I32, _P, _P, _P]),
     "tls_block_cache_table": (_I32, [_P, _P]),
     "tls_engine_create": (_I32, [_P, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "tls_engine_create_resident": (_I32, [_P, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
@@ -308,6 +309,15 @@ def tls_prefetch_diff(handle, new_block_idx_host, in_use_block_idx_host, K_b, co
     _check(lib().tls_prefetch_diff(handle, _ptr(new_block_idx_host), _ptr(in_use_block_idx_host), K_b,
                                    _stream(copy_stream), ev, ctypes.byref(n)), "tls_prefetch_diff")
     return n.value
+
+
+def tls_prefetch_diff_device(handle, new_block_idx_dev, in_use_block_idx_dev, K_b, copy_stream=None,
+                             done_event=None, n_copied_dev=None):
+    """Device block lists (torch int32 tensors); n_copied_dev: optional device int32 tensor written with
+    the number of copied blocks (-1: the plan failed)."""
+    ev = getattr(done_event, "cuda_event", done_event)
+    _check(lib().tls_prefetch_diff_device(handle, _ptr(new_block_idx_dev), _ptr(in_use_block_idx_dev), K_b,
+                                          _stream(copy_stream), ev, _ptr(n_copied_dev)), "tls_prefetch_diff_device")
 
 
 def tls_block_cache_table(handle, table):
