@@ -554,8 +554,10 @@ def measure_offload_engine(dev, steps=64, name="c4", data=None):
         "h2d_gbs": h2d,
         "copy_us_per_step_mean": copy_us, "exposed_us_per_step_mean": 1e3 * exposed_ms / len(st),
         "copy_hidden_frac": 1.0 - exposed_ms / copy_ms if copy_ms > 0 else None, "target_hidden_frac": 0.9,
+        "planner": "device (tls_prefetch_diff_device on the copy stream: the step call never waits on the host)",
         "timing": "per step: CUDA events on the caller's stream around tls_engine_step (level 2 + wait for the "
-                  "previous transfer + attention; level 1 runs on the engine's second stream); transfer figures "
+                  "previous transfer + attention; level 1 runs on the engine's second stream), so the step time "
+                  "is the device's, and host_us_per_step the call's own time; transfer figures "
                   "from the engine's copy-stream events.  copy_hidden_frac counts the time the attention waited "
                   "on a transfer past its own readiness; hidden_frac_vs_resident compares the step with the same "
                   "layer and q trajectory over HBM-resident K/V (resident engine, no transfer): 1 - (step time "
@@ -652,7 +654,7 @@ def measure_c5_loop(dev, steps=6, n_resident=20, n_layers=36):
             "transfer_blocks_per_step_mean": statistics.mean(blocks),
             "h2d_gbs_needed": statistics.mean(moved) / (ms / 1e3) / 1e9,
             "timing": "CUDA events around each decode step (36 layer steps issued back to back on one stream; "
-                      "each offloaded layer's call waits on the host for its level 1)"}
+                      "each offloaded layer's transfer is planned on the device, so no call waits on the host)"}
 
 
 def run_reference(args, cfg):

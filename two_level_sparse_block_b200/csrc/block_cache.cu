@@ -191,7 +191,7 @@ __device__ __forceinline__ void pull_block(const uint8_t* host_k, const uint8_t*
     const uint4* s4 = reinterpret_cast<const uint4*>(src);
     uint4* d4 = reinterpret_cast<uint4*>(dst);
     for (int64_t i0 = threadIdx.x; i0 < n16; i0 += 8 * kPullThreads) {
-      uint4 v[8];
+        uint4 v[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const int64_t i = i0 + (int64_t)u * kPullThreads;
@@ -246,7 +246,7 @@ __global__ void slot_table_update_kernel(int32_t* table, const int2* pairs, int 
 // ties to the lower slot (the CTA top-k's rule).  Copy i (in row, then list
 // order) takes the i-th victim in slot order, as in the host plan, so both
 // leave the same table.
-constexpr int kPlanThreads = 1024;
+constexpr int kPlanThreads = 256;  // small enough to start beside the step's other kernels
 constexpr int kPlanMaxSlots = 32768;    // keys in shared memory
 constexpr int kPlanMaxEntries = 65536;  // rows * K_b
 
