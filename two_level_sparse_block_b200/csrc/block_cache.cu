@@ -187,7 +187,34 @@ __device__ __forceinline__ void pull_block(const uint8_t* host_k, const uint8_t*
     const uint8_t* src = part == 0 ? host_k + tok0 * k_row_bytes : (host_v ? host_v + tok0 * v_row_bytes : nullptr);
     uint8_t* dst = part == 0 ? slot_k + slot * kblk : (slot_v ? slot_v + slot * vblk : nullptr);
     if (src == nullptr || dst == nullptr) continue;
-    const int64_t n16 = (part == 0 ? kblk : vblk) / 16;
+    const int64_t bytes = part == 0 ? kblk : vblk;
+    if (((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst) | (uintptr_t)bytes) & 31u) == 0) {
+      // 32-byte loads: half the requests of 16-byte ones over PCIe
+      const int64_t n32 = bytes / 32;
+      for (int64_t i0 = threadIdx.x; i0 < n32; i0 += 4 * kPullThreads) {
+        uint32_t v[4][8];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int64_t i = i0 + (int64_t)u * kPullThreads;
+          if (i < n32)
+            asm volatile("ld.global.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                         : "=r"(v[u][0]), "=r"(v[u][1]), "=r"(v[u][2]), "=r"(v[u][3]), "=r"(v[u][4]), "=r"(v[u][5]),
+                           "=r"(v[u][6]), "=r"(v[u][7])
+                         : "l"(src + i * 32));
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int64_t i = i0 + (int64_t)u * kPullThreads;
+          if (i < n32) {
+            uint4* d = reinterpret_cast<uint4*>(dst + i * 32);
+            d[0] = make_uint4(v[u][0], v[u][1], v[u][2], v[u][3]);
+            d[1] = make_uint4(v[u][4], v[u][5], v[u][6], v[u][7]);
+          }
+        }
+      }
+      continue;
+    }
+    const int64_t n16 = bytes / 16;
     const uint4* s4 = reinterpret_cast<const uint4*>(src);
     uint4* d4 = reinterpret_cast<uint4*>(dst);
     for (int64_t i0 = threadIdx.x; i0 < n16; i0 += 8 * kPullThreads) {
@@ -246,7 +273,7 @@ __global__ void slot_table_update_kernel(int32_t* table, const int2* pairs, int 
 // ties to the lower slot (the CTA top-k's rule).  Copy i (in row, then list
 // order) takes the i-th victim in slot order, as in the host plan, so both
 // leave the same table.
-constexpr int kPlanThreads = 256;  // small enough to start beside the step's other kernels
+constexpr int kPlanThreads = 512;  // small enough to start beside the step's other kernels
 constexpr int kPlanMaxSlots = 32768;    // keys in shared memory
 constexpr int kPlanMaxEntries = 65536;  // rows * K_b
 
@@ -293,12 +320,15 @@ __device__ __forceinline__ int plan_block_scan(int v, int* warp_sums, int* total
 }
 
 __global__ void __launch_bounds__(kPlanThreads, 1) block_plan_kernel(PlanParams p) {
-  extern __shared__ __align__(16) uint32_t pkeys[];  // [n_slots]
-  TopkScratch* ts = reinterpret_cast<TopkScratch*>(pkeys + ((p.n_slots + 3) & ~3));
+  extern __shared__ __align__(16) uint32_t pkeys[];  // [n_slots], then need flags [rows * K_b]
+  uint8_t* needf = reinterpret_cast<uint8_t*>(pkeys + ((p.n_slots + 3) & ~3));
+  const int E = p.rows * p.K_b;
+  TopkScratch* ts = reinterpret_cast<TopkScratch*>(needf + ((E + 15) & ~15));
   __shared__ int warp_sums[32];
   __shared__ int bad;
   const int tid = threadIdx.x;
-  const int E = p.rows * p.K_b;
+  const int32_t* __restrict__ new_idx = p.new_idx;
+  const int32_t* __restrict__ in_use = p.in_use;
   if (*reinterpret_cast<volatile int32_t*>(p.failed) != 0) {
     if (tid == 0) {
       *p.n_jobs = 0;
@@ -309,42 +339,35 @@ __global__ void __launch_bounds__(kPlanThreads, 1) block_plan_kernel(PlanParams 
   if (tid == 0) bad = 0;
   // 1. keys: free slots highest, then by the age of their last use
   const uint32_t kFree = float_key(33554432.0f), kKept = float_key(0.0f);
+#pragma unroll 4
   for (int s = tid; s < p.n_slots; s += kPlanThreads) {
     const int64_t age = p.step - p.last_use[s];
     pkeys[s] = p.owner[s] < 0 ? kFree : float_key((float)(age < 1 ? 1 : (age > 16777215 ? 16777215 : age)));
   }
   __syncthreads();
-  // 2. slots holding a block of M_t or M_{t-1} are kept; M_t must list
-  //    distinct blocks in [0, NB) in ascending order (as level 1 writes it)
+  // 2. slots holding a block of M_t or M_{t-1} are kept, and the blocks of
+  //    M_t that are not resident flagged; M_t must list distinct blocks in
+  //    [0, NB) in ascending order (as level 1 writes it)
+#pragma unroll 4
   for (int j = tid; j < E; j += kPlanThreads) {
-    const int r = j / p.K_b;
-    const int blk = p.new_idx[j];
-    if (blk >= p.nb) bad = 1;
-    if (blk >= 0 && j % p.K_b > 0) {
-      const int prv = p.new_idx[j - 1];
-      if (prv >= blk || prv < 0) bad = 1;
-    }
-    if (blk >= 0 && blk < p.nb) {
-      const int s = p.table[(int64_t)r * p.nb + blk];
-      if (s >= 0 && s < p.n_slots) pkeys[s] = kKept;
-    }
-    if (p.in_use != nullptr) {
-      const int ub = p.in_use[j];
-      if (ub >= 0 && ub < p.nb) {
-        const int s = p.table[(int64_t)r * p.nb + ub];
-        if (s >= 0 && s < p.n_slots) pkeys[s] = kKept;
-      }
-    }
+    const int64_t r = j / p.K_b;
+    const int blk = new_idx[j];
+    const int prv = j % p.K_b > 0 ? new_idx[j - 1] : -1;
+    const int ub = in_use != nullptr ? in_use[j] : -1;
+    const bool ok = blk >= 0 && blk < p.nb;
+    if (blk >= p.nb || (blk >= 0 && j % p.K_b > 0 && (prv >= blk || prv < 0))) bad = 1;
+    const int s = ok ? p.table[r * p.nb + blk] : -1;
+    const int su = (ub >= 0 && ub < p.nb) ? p.table[r * p.nb + ub] : -1;
+    if (s >= 0 && s < p.n_slots) pkeys[s] = kKept;
+    if (su >= 0 && su < p.n_slots) pkeys[su] = kKept;
+    needf[j] = ok && s < 0;
   }
   __syncthreads();
   // 3. T_t in row, then list order: each thread a contiguous range of entries
   const int per = (E + kPlanThreads - 1) / kPlanThreads;
   const int j0 = min(E, tid * per), j1 = min(E, j0 + per);
   int cnt = 0, avail = 0;
-  for (int j = j0; j < j1; ++j) {
-    const int blk = p.new_idx[j];
-    if (blk >= 0 && blk < p.nb && p.table[(int64_t)(j / p.K_b) * p.nb + blk] < 0) ++cnt;
-  }
+  for (int j = j0; j < j1; ++j) cnt += needf[j];
   for (int s = tid; s < p.n_slots; s += kPlanThreads) avail += pkeys[s] != kKept;
   int n_copy = 0, n_avail = 0;
   const int base = plan_block_scan(cnt, warp_sums, &n_copy);
@@ -360,11 +383,9 @@ __global__ void __launch_bounds__(kPlanThreads, 1) block_plan_kernel(PlanParams 
   }
   int pos = base;
   for (int j = j0; j < j1; ++j) {
-    const int blk = p.new_idx[j];
-    if (blk >= 0 && blk < p.nb && p.table[(int64_t)(j / p.K_b) * p.nb + blk] < 0) {
-      const int64_t tok0 = (int64_t)(j / p.K_b) * p.ctx_len + (int64_t)blk * p.bs;
-      p.jobs[pos++] = make_int4((int)(uint32_t)(tok0 & 0xFFFFFFFF), (int)(tok0 >> 32), 0, j);
-    }
+    if (!needf[j]) continue;
+    const int64_t tok0 = (int64_t)(j / p.K_b) * p.ctx_len + (int64_t)new_idx[j] * p.bs;
+    p.jobs[pos++] = make_int4((int)(uint32_t)(tok0 & 0xFFFFFFFF), (int)(tok0 >> 32), 0, j);
   }
   // 4. the victims: the n_copy largest keys, ascending slots
   if (n_copy > 0) cta_topk_ascending<kPlanThreads>(pkeys, p.n_slots, n_copy, p.victims, *ts, [](int i) { return i; });
@@ -375,7 +396,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) block_plan_kernel(PlanParams 
   for (int i = tid; i < n_copy; i += kPlanThreads) {
     const int slot = p.victims[i];
     const int j = p.jobs[i].w;
-    const int64_t key = (int64_t)(j / p.K_b) * p.nb + p.new_idx[j];
+    const int64_t key = (int64_t)(j / p.K_b) * p.nb + new_idx[j];
     const int64_t old = p.owner[slot];
     if (old >= 0) p.table[old] = -1;
     p.table[key] = slot;
@@ -384,10 +405,10 @@ __global__ void __launch_bounds__(kPlanThreads, 1) block_plan_kernel(PlanParams 
   }
   __syncthreads();
   // 6. every block of M_t is resident now: its slot was used at this step
+#pragma unroll 4
   for (int j = tid; j < E; j += kPlanThreads) {
-    const int blk = p.new_idx[j];
-    if (blk < 0 || blk >= p.nb) continue;
-    const int s = p.table[(int64_t)(j / p.K_b) * p.nb + blk];
+    const int blk = new_idx[j];
+    const int s = (blk >= 0 && blk < p.nb) ? p.table[(int64_t)(j / p.K_b) * p.nb + blk] : -1;
     if (s >= 0 && s < p.n_slots) p.last_use[s] = p.step;
   }
   if (tid == 0) {
@@ -521,7 +542,8 @@ tls_status prefetch_device_impl(tls_block_cache* c, const int32_t* new_dev, cons
   int32_t* dflag = nullptr;
   cudaError_t e = cudaHostGetDevicePointer((void**)&dflag, c->dev_failed, 0);
   p.failed = dflag;
-  const size_t smem = (size_t)((c->n_slots + 3) & ~3) * 4 + sizeof(TopkScratch) + 16;
+  const size_t smem = (size_t)((c->n_slots + 3) & ~3) * 4 + (size_t)((c->rows * K_b + 15) & ~15) +
+                      sizeof(TopkScratch) + 16;
   if (e == cudaSuccess) e = kernel_attrs((const void*)block_plan_kernel, smem);
   if (e != cudaSuccess) return cuda_check(e, "prefetch_diff_device: plan kernel setup");
   block_plan_kernel<<<1, kPlanThreads, smem, cs>>>(p);
