@@ -238,6 +238,7 @@ extern "C" tls_status tls_workspace_error(const void* ws, int32_t clear, int32_t
 extern "C" tls_status tls_select_blocks(const tls_shape* shape, const void* q, const void* meta, int32_t K_b,
                                         int32_t* block_idx, float* block_score, void* ws, size_t ws_bytes,
                                         void* stream) {
+  NvtxRange nvtx_range("tls_select_blocks");
   clear_error();
   tls_status st = check_shape(shape);
   if (st != TLS_OK) return st;
@@ -254,6 +255,7 @@ extern "C" tls_status tls_select_tokens(const tls_shape* shape, const void* q, c
                                         const uint8_t* codes, const float* scales, const int32_t* block_idx,
                                         int32_t K_b, int32_t k, int32_t* token_idx, float* token_score, void* ws,
                                         size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("tls_select_tokens");
   clear_error();
   tls_status st = check_shape(shape);
   if (st != TLS_OK) return st;
@@ -273,6 +275,7 @@ extern "C" tls_status tls_select_tokens(const tls_shape* shape, const void* q, c
 extern "C" tls_status tls_sparse_decode_attn(const tls_shape* shape, const void* q, const tls_kv_view* kv,
                                              const int32_t* token_idx, int32_t k, int32_t out_dtype, void* out,
                                              float* lse, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("tls_sparse_decode_attn");
   clear_error();
   tls_status st = check_shape(shape);
   if (st != TLS_OK) return st;
@@ -320,6 +323,7 @@ static tls_status select_impl(const tls_shape* shape, const void* q, const void*
 extern "C" tls_status tls_select(const tls_shape* shape, const void* q, const void* meta, const int32_t* label_ch,
                                  const uint8_t* codes, const float* scales, int32_t K_b, int32_t k,
                                  int32_t* block_idx, int32_t* token_idx, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("tls_select");
   clear_error();
   return select_impl(shape, q, meta, label_ch, codes, scales, K_b, k, block_idx, token_idx, ws, ws_bytes, stream);
 }
@@ -329,6 +333,7 @@ extern "C" tls_status tls_decode_step(const tls_shape* shape, const void* q, con
                                       const tls_kv_view* kv, int32_t K_b, int32_t k, int32_t* block_idx,
                                       int32_t* token_idx, int32_t out_dtype, void* out, float* lse, void* ws,
                                       size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("tls_decode_step");
   clear_error();
   // everything the attention checks is checked before anything is launched
   tls_status st = check_shape(shape);
@@ -364,6 +369,7 @@ static tls_status check_attn_args(const tls_shape* shape, const void* q, const t
 extern "C" tls_status tls_dense_decode_attn(const tls_shape* shape, const void* q, const tls_kv_view* kv,
                                             int32_t out_dtype, void* out, float* lse, void* ws, size_t ws_bytes,
                                             void* stream) {
+  NvtxRange nvtx_range("tls_dense_decode_attn");
   clear_error();
   tls_status st = check_attn_args(shape, q, kv, out_dtype, out, "dense_decode_attn");
   if (st != TLS_OK) return st;
@@ -380,6 +386,7 @@ extern "C" tls_status tls_quest_decode_step(const tls_shape* shape, const void* 
                                             const tls_kv_view* kv, int32_t K_b, int32_t* block_idx,
                                             int32_t out_dtype, void* out, float* lse, void* ws, size_t ws_bytes,
                                             void* stream) {
+  NvtxRange nvtx_range("tls_quest_decode_step");
   clear_error();
   tls_status st = check_attn_args(shape, q, kv, out_dtype, out, "quest_decode_step");
   if (st != TLS_OK) return st;
@@ -400,6 +407,7 @@ extern "C" tls_status tls_ds_decode_step(const tls_shape* shape, const void* q, 
                                          const uint8_t* codes, const float* scales, const tls_kv_view* kv, int32_t k,
                                          int32_t* token_idx, int32_t out_dtype, void* out, float* lse, void* ws,
                                          size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("tls_ds_decode_step");
   clear_error();
   tls_status st = check_attn_args(shape, q, kv, out_dtype, out, "ds_decode_step");
   if (st != TLS_OK) return st;

@@ -771,6 +771,7 @@ extern "C" void tls_block_cache_destroy(tls_block_cache* c) {
 extern "C" tls_status tls_block_cache_plan(tls_block_cache* c, const int32_t* new_block_idx,
                                            const int32_t* in_use_block_idx, int32_t K_b, int32_t* copy_row,
                                            int32_t* copy_block, int32_t* copy_slot, int32_t* n_copy) {
+  NvtxRange nvtx_range("tls_block_cache_plan");
   clear_error();
   if (c == nullptr || new_block_idx == nullptr || n_copy == nullptr)
     return fail(TLS_ERR_INVALID_ARG, "block_cache_plan: NULL argument");
@@ -798,6 +799,7 @@ extern "C" tls_status tls_block_cache_plan(tls_block_cache* c, const int32_t* ne
 extern "C" tls_status tls_prefetch_diff(tls_block_cache* c, const int32_t* new_block_idx_host,
                                         const int32_t* in_use_block_idx_host, int32_t K_b, void* copy_stream,
                                         void* done_event, int32_t* n_copied) {
+  NvtxRange nvtx_range("tls_prefetch_diff");
   clear_error();
   if (c == nullptr || new_block_idx_host == nullptr || n_copied == nullptr)
     return fail(TLS_ERR_INVALID_ARG, "prefetch_diff: NULL argument");
@@ -828,6 +830,7 @@ extern "C" tls_status tls_block_cache_table(const tls_block_cache* c, int32_t* t
 extern "C" tls_status tls_prefetch_diff_device(tls_block_cache* c, const int32_t* new_block_idx_dev,
                                                const int32_t* in_use_block_idx_dev, int32_t K_b, void* copy_stream,
                                                void* done_event, int32_t* n_copied_dev) {
+  NvtxRange nvtx_range("tls_prefetch_diff_device");
   clear_error();
   if (c == nullptr || new_block_idx_dev == nullptr) return fail(TLS_ERR_INVALID_ARG, "prefetch_diff_device: NULL argument");
   if (K_b < 1 || K_b > c->nb) return fail(TLS_ERR_INVALID_ARG, "prefetch_diff_device: K_b out of range");

@@ -363,6 +363,7 @@ tls_status noalloc_scratch(void** out) {
 extern "C" tls_status tls_sparse_decode_attn_noalloc(const tls_shape* shape, const void* q, const tls_kv_view* kv,
                                                      const int32_t* token_idx, int32_t k, int32_t out_dtype,
                                                      void* out, float* lse, void* stream) {
+  tls::NvtxRange nvtx_range("tls_sparse_decode_attn_noalloc");
   using namespace tls;
   clear_error();
   tls_status st = check_shape(shape);

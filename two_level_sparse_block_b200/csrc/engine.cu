@@ -386,6 +386,7 @@ tls_status engine_step(tls_engine* e, const void* q, int32_t out_dtype, void* ou
 
 extern "C" tls_status tls_engine_step(tls_engine* e, const void* q, int32_t out_dtype, void* out, float* lse,
                                       void* stream) {
+  NvtxRange nvtx_range("tls_engine_step");
   clear_error();
   if (e == nullptr || q == nullptr || out == nullptr) return fail(TLS_ERR_INVALID_ARG, "engine_step: NULL argument");
   if (!aligned16(q)) return fail(TLS_ERR_INVALID_ARG, "engine_step: q not 16-byte aligned");

@@ -12,8 +12,18 @@
 #include <unordered_map>
 
 #include "tls.h"
+#include <nvtx3/nvToolsExt.h>
 
 namespace tls {
+
+// An NVTX range around one library call, named for the entry point (seen by
+// Nsight Systems and other NVTX tools; a few nanoseconds without a tool).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // Sets the thread-local error message and returns `st`.
 tls_status fail(tls_status st, const char* fmt, ...);

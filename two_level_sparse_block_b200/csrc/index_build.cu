@@ -198,6 +198,7 @@ using namespace tls;
 
 extern "C" tls_status tls_build_block_meta(const tls_shape* shape, const void* k, int64_t k_row_stride,
                                            int64_t t0, int64_t t1, void* meta, void* stream) {
+  NvtxRange nvtx_range("tls_build_block_meta");
   clear_error();
   tls_status st = check_shape(shape);
   if (st != TLS_OK) return st;
@@ -224,6 +225,7 @@ extern "C" tls_status tls_build_block_meta(const tls_shape* shape, const void* k
 extern "C" tls_status tls_quant_label_cache(const tls_shape* shape, const void* k, int64_t k_row_stride,
                                             const int32_t* label_ch, int64_t t0, int64_t t1, uint8_t* codes,
                                             float* scales, void* stream) {
+  NvtxRange nvtx_range("tls_quant_label_cache");
   clear_error();
   tls_status st = check_shape(shape);
   if (st != TLS_OK) return st;
@@ -260,6 +262,7 @@ extern "C" tls_status tls_quant_label_cache(const tls_shape* shape, const void* 
 extern "C" tls_status tls_append_kv(const tls_shape* shape, int32_t* seq_lens, const void* k_new, const void* v_new,
                                     const tls_kv_view* kv, void* meta, const int32_t* label_ch, uint8_t* codes,
                                     float* scales, void* stream) {
+  NvtxRange nvtx_range("tls_append_kv");
   clear_error();
   tls_status st = check_shape(shape);
   if (st != TLS_OK) return st;
