@@ -536,6 +536,14 @@ TLS_API tls_status tls_engine_step(tls_engine* engine, const void* q, int32_t ou
 TLS_API int64_t tls_engine_steps(const tls_engine* engine);
 
 /*
+ * Kernel launches of one steady-state step (-1 for a NULL engine): level 1,
+ * level 2 and the attention (plus level 1's query preparation for groups of
+ * more than 32 heads); an offloaded engine adds the transfer's plan and pull
+ * kernels (device planner) or its pull kernel (host planner).
+ */
+TLS_API int32_t tls_engine_step_kernels(const tls_engine* engine);
+
+/*
  * Transfer figures of step `step` (-1 .. steps-1, among the last 255 steps);
  * waits for the events they need.  A resident engine reports no transfer
  * (zero blocks, bytes and times).

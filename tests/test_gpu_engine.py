@@ -289,11 +289,22 @@ def _resident(cfg, qs):
     return runtime, st, (K, V, lab)
 
 
-@pytest.mark.parametrize("cfg", ENGINE, ids=lambda c: c.name)
+# more resident shapes: 8 heads a group; 512 blocks with 32 label channels and
+# an odd K_b; 4096 candidates and 2048 tokens a row
+RESIDENT = [
+    offload("f_g8", n_q_heads=8, ctx_len=4096, block_size=32, K_b=16, k=256, seed=34, steps=4),
+    offload("f_r32_two_passes", batch=4, n_q_heads=16, n_kv_heads=4, ctx_len=16384, block_size=32, K_b=23, k=300,
+            n_label=32, seed=35, steps=4),
+    offload("f_c2_rows", batch=2, n_q_heads=8, n_kv_heads=2, ctx_len=32768, K_b=64, k=2048, seed=36, steps=3),
+]
+
+
+@pytest.mark.parametrize("cfg", ENGINE + RESIDENT, ids=lambda c: c.name)
 def test_resident_engine_follows_the_staggered_oracle(cfg):
     qs = synth.gen_query_trajectory(cfg)
     runtime, st, (K, V, lab) = _resident(cfg, qs)
     eng = runtime.ResidentEngine(st)
+    assert eng.step_kernels() == 3 + (1 if cfg.group > 32 else 0)
     g = cfg.group
     try:
         for t, q in enumerate(qs):

@@ -58,15 +58,6 @@ struct BlockScoreParams {
   int bs;
 };
 
-__device__ __forceinline__ uint32_t relu_bf16x2(uint32_t w) {
-  uint32_t neg = (w & 0x80008000u) >> 15;  // 1 in each negative half
-  return w & ~(neg * 0xFFFFu);
-}
-__device__ __forceinline__ uint32_t min0_bf16x2(uint32_t w) {
-  uint32_t neg = (w & 0x80008000u) >> 15;
-  return w & (neg * 0xFFFFu);
-}
-
 template <int NPAD>
 struct BsSmem {
   static constexpr int A_BYTES = kBsTile * 128;

@@ -664,6 +664,17 @@ __device__ void cta_topk_regs(const uint32_t* keys, int n, int k, int* out, Topk
   for (int i = tid; i < k; i += NT) out[i] = map(stage[i]);
 }
 
+// The two halves of a block score's query operand [relu(q), min(q, 0)] on a
+// pair of bf16 values (exact: a sign test per half).
+__device__ __forceinline__ uint32_t relu_bf16x2(uint32_t w) {
+  uint32_t neg = (w & 0x80008000u) >> 15;  // 1 in each negative half
+  return w & ~(neg * 0xFFFFu);
+}
+__device__ __forceinline__ uint32_t min0_bf16x2(uint32_t w) {
+  uint32_t neg = (w & 0x80008000u) >> 15;
+  return w & (neg * 0xFFFFu);
+}
+
 // ----------------------------------------------------------------------------
 // mbarrier / TMA / tcgen05 wrappers (PTX ISA 8.7, sm_100a)
 // ----------------------------------------------------------------------------

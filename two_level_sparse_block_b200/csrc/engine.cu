@@ -401,6 +401,16 @@ extern "C" tls_status tls_engine_step(tls_engine* e, const void* q, int32_t out_
 
 extern "C" int64_t tls_engine_steps(const tls_engine* e) { return e == nullptr ? -1 : e->t; }
 
+extern "C" int32_t tls_engine_step_kernels(const tls_engine* e) {
+  if (e == nullptr) return -1;
+  // level 1 (with its query preparation for groups padded to 64 heads or
+  // more), level 2, the attention; offloaded: the transfer's plan and pull
+  // (device planner) or its one pull kernel (host planner)
+  const int n = 3 + (group_of(e->shape) > 32 ? 1 : 0);
+  if (e->cache == nullptr) return n;
+  return n + (e->device_plan ? 2 : 1);
+}
+
 extern "C" tls_status tls_engine_stats(tls_engine* e, int64_t step, tls_engine_step_stats* out) {
   clear_error();
   if (e == nullptr || out == nullptr) return fail(TLS_ERR_INVALID_ARG, "engine_stats: NULL argument");

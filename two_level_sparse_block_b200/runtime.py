@@ -185,6 +185,10 @@ class ResidentEngine:
     def steps_taken(self) -> int:
         return tls.tls_engine_steps(self.engine)
 
+    def step_kernels(self) -> int:
+        """Kernel launches of one step (tls_engine_step_kernels)."""
+        return tls.tls_engine_step_kernels(self.engine)
+
     def blocks_of_step(self, t: int) -> torch.Tensor:
         """M_t (valid after step t, until step t + 2 overwrites it)."""
         return self.block_idx[t & 1]

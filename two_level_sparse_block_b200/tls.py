@@ -102,6 +102,7 @@ _SIG = {
     "tls_engine_create_resident": (_I32, [_P, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "tls_engine_step": (_I32, [_P, _P, _I32, _P, _P, _P]),
     "tls_engine_steps": (_I64, [_P]),
+    "tls_engine_step_kernels": (_I32, [_P]),
     "tls_engine_stats": (_I32, [_P, _I64, _P]),
     "tls_engine_destroy": (None, [_P]),
 }
@@ -349,6 +350,10 @@ def tls_engine_step(engine, q, out_dtype, out, lse=None, stream=None):
 
 def tls_engine_steps(engine) -> int:
     return lib().tls_engine_steps(engine)
+
+
+def tls_engine_step_kernels(engine) -> int:
+    return lib().tls_engine_step_kernels(engine)
 
 
 def tls_engine_stats(engine, step: int) -> EngineStepStats:
