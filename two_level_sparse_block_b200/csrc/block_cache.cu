@@ -177,58 +177,66 @@ void commit(tls_block_cache& c, const int32_t* new_idx, int K_b, const std::vect
 // The consumers (the next attention) start after the whole kernel, so the
 // order of the two parts does not matter.
 constexpr int kPullThreads = 256;
-// One job: the block's bs rows of K (and of V) from host memory into its slot.
+// One job: the block's bs rows of K (and of V) from host memory into its
+// slot.  The loads of both parts are issued together (one PCIe round trip
+// for a block when the CTA's loads cover it), 32 bytes each where every
+// address and size is 32-byte aligned, else 16.
 __device__ __forceinline__ void pull_block(const uint8_t* host_k, const uint8_t* host_v, uint8_t* slot_k,
                                            uint8_t* slot_v, int64_t kblk, int64_t vblk, int64_t k_row_bytes,
                                            int64_t v_row_bytes, int4 jb) {
   const int64_t tok0 = (int64_t)(uint32_t)jb.x | ((int64_t)jb.y << 32);
   const int64_t slot = jb.z;
-  for (int part = 0; part < 2; ++part) {
-    const uint8_t* src = part == 0 ? host_k + tok0 * k_row_bytes : (host_v ? host_v + tok0 * v_row_bytes : nullptr);
-    uint8_t* dst = part == 0 ? slot_k + slot * kblk : (slot_v ? slot_v + slot * vblk : nullptr);
-    if (src == nullptr || dst == nullptr) continue;
-    const int64_t bytes = part == 0 ? kblk : vblk;
-    if (((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst) | (uintptr_t)bytes) & 31u) == 0) {
-      // 32-byte loads: half the requests of 16-byte ones over PCIe
-      const int64_t n32 = bytes / 32;
-      for (int64_t i0 = threadIdx.x; i0 < n32; i0 += 4 * kPullThreads) {
-        uint32_t v[4][8];
+  const uint8_t* src0 = host_k + tok0 * k_row_bytes;
+  uint8_t* dst0 = slot_k + slot * kblk;
+  const bool with_v = host_v != nullptr && slot_v != nullptr;
+  const uint8_t* src1 = with_v ? host_v + tok0 * v_row_bytes : src0;
+  uint8_t* dst1 = with_v ? slot_v + slot * vblk : dst0;
+  const int64_t n1 = with_v ? vblk : 0;
+  const uintptr_t al = reinterpret_cast<uintptr_t>(src0) | reinterpret_cast<uintptr_t>(dst0) |
+                       reinterpret_cast<uintptr_t>(src1) | reinterpret_cast<uintptr_t>(dst1) | (uintptr_t)kblk |
+                       (uintptr_t)n1;
+  if ((al & 31u) == 0) {
+    // 32-byte units: K's first, then V's
+    const int64_t a0 = kblk / 32, tot = a0 + n1 / 32;
+    for (int64_t i0 = threadIdx.x; i0 < tot; i0 += 4 * kPullThreads) {
+      uint32_t v[4][8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int64_t i = i0 + (int64_t)u * kPullThreads;
-          if (i < n32)
-            asm volatile("ld.global.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-                         : "=r"(v[u][0]), "=r"(v[u][1]), "=r"(v[u][2]), "=r"(v[u][3]), "=r"(v[u][4]), "=r"(v[u][5]),
-                           "=r"(v[u][6]), "=r"(v[u][7])
-                         : "l"(src + i * 32));
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int64_t i = i0 + (int64_t)u * kPullThreads;
-          if (i < n32) {
-            uint4* d = reinterpret_cast<uint4*>(dst + i * 32);
-            d[0] = make_uint4(v[u][0], v[u][1], v[u][2], v[u][3]);
-            d[1] = make_uint4(v[u][4], v[u][5], v[u][6], v[u][7]);
-          }
+      for (int u = 0; u < 4; ++u) {
+        const int64_t i = i0 + (int64_t)u * kPullThreads;
+        if (i < tot) {
+          const uint8_t* sp = i < a0 ? src0 + i * 32 : src1 + (i - a0) * 32;
+          asm volatile("ld.global.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                       : "=r"(v[u][0]), "=r"(v[u][1]), "=r"(v[u][2]), "=r"(v[u][3]), "=r"(v[u][4]), "=r"(v[u][5]),
+                         "=r"(v[u][6]), "=r"(v[u][7])
+                       : "l"(sp));
         }
       }
-      continue;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t i = i0 + (int64_t)u * kPullThreads;
+        if (i < tot) {
+          uint4* d = reinterpret_cast<uint4*>(i < a0 ? dst0 + i * 32 : dst1 + (i - a0) * 32);
+          d[0] = make_uint4(v[u][0], v[u][1], v[u][2], v[u][3]);
+          d[1] = make_uint4(v[u][4], v[u][5], v[u][6], v[u][7]);
+        }
+      }
     }
-    const int64_t n16 = bytes / 16;
-    const uint4* s4 = reinterpret_cast<const uint4*>(src);
-    uint4* d4 = reinterpret_cast<uint4*>(dst);
-    for (int64_t i0 = threadIdx.x; i0 < n16; i0 += 8 * kPullThreads) {
-        uint4 v[8];
+    return;
+  }
+  // 16-byte units (rows 16-byte aligned: checked at cache creation)
+  const int64_t a0 = kblk / 16, tot = a0 + n1 / 16;
+  for (int64_t i0 = threadIdx.x; i0 < tot; i0 += 8 * kPullThreads) {
+    uint4 v[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int64_t i = i0 + (int64_t)u * kPullThreads;
-        if (i < n16) v[u] = __ldcv(s4 + i);
-      }
+    for (int u = 0; u < 8; ++u) {
+      const int64_t i = i0 + (int64_t)u * kPullThreads;
+      if (i < tot)
+        v[u] = __ldcv(reinterpret_cast<const uint4*>(i < a0 ? src0 + i * 16 : src1 + (i - a0) * 16));
+    }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int64_t i = i0 + (int64_t)u * kPullThreads;
-        if (i < n16) d4[i] = v[u];
-      }
+    for (int u = 0; u < 8; ++u) {
+      const int64_t i = i0 + (int64_t)u * kPullThreads;
+      if (i < tot) *reinterpret_cast<uint4*>(i < a0 ? dst0 + i * 16 : dst1 + (i - a0) * 16) = v[u];
     }
   }
 }
@@ -251,6 +259,7 @@ __global__ void __launch_bounds__(kPullThreads) block_pull_jobs_kernel(const uin
                                                                        int64_t vblk, int64_t k_row_bytes,
                                                                        int64_t v_row_bytes, const int4* jobs,
                                                                        const int32_t* n_jobs) {
+  grid_dependency_wait();  // the plan kernel's jobs (programmatic dependent launch)
   const int n = *n_jobs;
   for (int j = blockIdx.x; j < n; j += gridDim.x)
     pull_block(host_k, host_v, slot_k, slot_v, kblk, vblk, k_row_bytes, v_row_bytes, jobs[j]);
@@ -387,9 +396,110 @@ __global__ void __launch_bounds__(kPlanThreads, 1) block_plan_kernel(PlanParams 
     const int64_t tok0 = (int64_t)(j / p.K_b) * p.ctx_len + (int64_t)new_idx[j] * p.bs;
     p.jobs[pos++] = make_int4((int)(uint32_t)(tok0 & 0xFFFFFFFF), (int)(tok0 >> 32), 0, j);
   }
-  // 4. the victims: the n_copy largest keys, ascending slots
-  if (n_copy > 0) cta_topk_ascending<kPlanThreads>(pkeys, p.n_slots, n_copy, p.victims, *ts, [](int i) { return i; });
+  // 4. the victims: the n_copy largest keys (ties: lower slot), in slot
+  //    order.  Ages are small integers with many ties, so the threshold is
+  //    found from a histogram of ages below the oldest (256 of them); wider
+  //    spreads take the generic CTA top-k.
+  __shared__ int thr_bin, thr_above;
+  __shared__ float amax_s;
+  uint32_t thr = kFree;
+  int eq_take = n_copy;  // keys equal to thr to take, first ones in slot order
+  bool generic = false;
+  if (n_copy > 0) {
+    int nfree = 0;
+    {
+      int f = 0;
+      for (int s = tid; s < p.n_slots; s += kPlanThreads) f += pkeys[s] == kFree;
+      plan_block_scan(f, warp_sums, &nfree);
+    }
+    const int need_used = n_copy - nfree;
+    if (need_used > 0) {
+      float am = 0.0f;
+      for (int s = tid; s < p.n_slots; s += kPlanThreads) {
+        const uint32_t k = pkeys[s];
+        if (k != kFree && k != kKept) am = fmaxf(am, key_float(k));
+      }
+      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 16));
+      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 8));
+      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 4));
+      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
+      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+      for (int i = tid; i < 256; i += kPlanThreads) ts->hist[i] = 0;
+      if (tid == 0) amax_s = 0.0f;
+      __syncthreads();
+      if ((tid & 31) == 0) atomicMax(reinterpret_cast<int*>(&amax_s), __float_as_int(am));  // ages are >= 0
+      __syncthreads();
+      const float amax = amax_s;
+      for (int s = tid; s < p.n_slots; s += kPlanThreads) {
+        const uint32_t k = pkeys[s];
+        if (k == kFree || k == kKept) continue;
+        const float d = amax - key_float(k);
+        if (d < 256.0f) atomicAdd(&ts->hist[(int)d], 1);
+      }
+      __syncthreads();
+      if (tid < 32) {
+        // the bin (age below the oldest) where the count from the oldest reaches need_used
+        int run = 0, bin = -1, above = 0;
+        for (int c = 0; c < 256 && bin < 0; c += 32) {
+          int v = ts->hist[c + tid];
+          int x = v;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (tid >= o) x += y;
+          }
+          const unsigned hit = __ballot_sync(0xffffffffu, run + x >= need_used);
+          if (hit != 0u) {
+            const int l = __ffs(hit) - 1;
+            bin = c + l;
+            above = run + __shfl_sync(0xffffffffu, x - v, l);
+          }
+          run += __shfl_sync(0xffffffffu, x, 31);
+        }
+        if (tid == 0) {
+          thr_bin = bin;
+          thr_above = above;
+        }
+      }
+      __syncthreads();
+      if (thr_bin < 0) {
+        generic = true;
+      } else {
+        thr = float_key(amax - (float)thr_bin);
+        eq_take = need_used - thr_above;
+      }
+    }
+  }
+  if (generic) {
+    cta_topk_ascending<kPlanThreads>(pkeys, p.n_slots, n_copy, p.victims, *ts, [](int i) { return i; });
+  } else if (n_copy > 0) {
+    // victims: keys above thr, and the first eq_take keys equal to thr; then
+    // compacted in slot order (contiguous ranges of slots per thread)
+    const int sp = (p.n_slots + kPlanThreads - 1) / kPlanThreads;
+    const int s0 = min(p.n_slots, tid * sp), s1 = min(p.n_slots, s0 + sp);
+    int eq = 0;
+    for (int s = s0; s < s1; ++s) eq += pkeys[s] == thr;
+    int n_eq = 0;
+    int eq_before = plan_block_scan(eq, warp_sums, &n_eq);
+    int vic = 0;
+    for (int s = s0, e = eq_before; s < s1; ++s) {
+      const uint32_t k = pkeys[s];
+      if (k == thr) vic += e++ < eq_take;
+      else vic += k > thr && k != kKept;
+    }
+    int n_vic = 0;
+    int pos = plan_block_scan(vic, warp_sums, &n_vic);
+    for (int s = s0, e = eq_before; s < s1; ++s) {
+      const uint32_t k = pkeys[s];
+      bool v;
+      if (k == thr) v = e++ < eq_take;
+      else v = k > thr && k != kKept;
+      if (v && pos < n_copy) p.victims[pos++] = s;
+    }
+  }
   __syncthreads();
+  // the pull kernel may become resident from here (it waits for this grid)
+  grid_launch_dependents();
   // 5. copy i takes victim i: the evicted block loses its entry, the copied
   //    one gets the slot (no entry is touched twice: copied blocks are not
   //    resident, evicted ones are)
@@ -552,13 +662,14 @@ tls_status prefetch_device_impl(tls_block_cache* c, const int32_t* new_dev, cons
   const int64_t kblk = (int64_t)c->shape.block_size * c->hk_stride * 2;
   const int64_t vblk = (int64_t)c->shape.block_size * c->hv_stride * 2;
   const bool with_v = c->host_v != nullptr && c->slot_v != nullptr;
-  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)c->rows * K_b, 4 * (int64_t)kNumSMs));
-  if (e == cudaSuccess) {
-    block_pull_jobs_kernel<<<grid, kPullThreads, 0, cs>>>(c->dev_host_k, with_v ? c->dev_host_v : nullptr, c->slot_k,
-                                                          with_v ? c->slot_v : nullptr, kblk, vblk, c->hk_stride * 2,
-                                                          c->hv_stride * 2, c->jobs_dev, c->n_jobs_dev);
-    e = cudaGetLastError();
-  }
+  // one CTA an SM at most: the grid becomes resident while the plan kernel
+  // still runs (programmatic launch), beside the step's other kernels
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)c->rows * K_b, (int64_t)kNumSMs));
+  if (e == cudaSuccess)
+    e = launch_ex(block_pull_jobs_kernel, dim3(grid), dim3(kPullThreads), 0, cs, /*pdl=*/true, 0u,
+                  (const uint8_t*)c->dev_host_k, (const uint8_t*)(with_v ? c->dev_host_v : nullptr), c->slot_k,
+                  (uint8_t*)(with_v ? c->slot_v : nullptr), kblk, vblk, c->hk_stride * 2, c->hv_stride * 2,
+                  (const int4*)c->jobs_dev, (const int32_t*)c->n_jobs_dev);
   if (e != cudaSuccess) {
     c->failed = TLS_ERR_COPY;
     return fail(TLS_ERR_COPY, "prefetch_diff_device: launch failed: %s", cudaGetErrorString(e));
