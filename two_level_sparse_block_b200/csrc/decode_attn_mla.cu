@@ -13,8 +13,8 @@
 //               a partial S; the four partials are summed in a fixed order
 //               through shared memory, so every warp holds the same S
 //   softmax     online, base 2, fp32, identical in the four warps
-//   O += P.V    each warp its own 128 of the 512 value dims; P split into
-//               bf16 hi + lo parts (two MMAs)
+//   O += P.V    each warp its own 128 of the 512 value dims, in fp16 (P
+//               rounded to fp16, V converted exactly)
 // The split merge needs no workspace: each CTA leaves (m, l, O) in its
 // drained ring, and after a cluster barrier CTA r merges output dims
 // [64r, 64r + 64) of the 16 heads by log-sum-exp over the 8 CTAs, reading
@@ -57,13 +57,6 @@ constexpr int kMlaSmem = kMlaOffRid;
 constexpr int kMlaOStride = kMlaV + 8;
 static_assert(kMlaHeads * kMlaOStride * 4 <= kMlaStages * kMlaStageBytes, "partial O must fit the ring");
 
-__device__ __forceinline__ uint32_t mla_pack_bf16(float a, float b) {
-  uint32_t r;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
-  return r;
-}
-__device__ __forceinline__ float mla_lo_f(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float mla_hi_f(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 __device__ __forceinline__ float mla_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -72,6 +65,25 @@ __device__ __forceinline__ float mla_exp2(float x) {
 __device__ __forceinline__ void mla_mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// O += P.V in fp16: P (in [0, 1]) rounds to fp16 with 11 significant bits
+// (relative error <= 2^-11), and a pair of bf16 values of V converts to fp16
+// exactly within fp16's range (bf16 carries 8 significant bits), so one MMA
+// replaces the bf16 hi + lo pair at well under the output tolerance
+__device__ __forceinline__ uint32_t mla_pack_f16(float a, float b) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+  return r;
+}
+__device__ __forceinline__ uint32_t mla_bf16x2_to_f16x2(uint32_t w) {
+  return mla_pack_f16(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+__device__ __forceinline__ void mla_mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
@@ -270,25 +282,20 @@ __global__ void __launch_bounds__(kMlaWarps * 32, 2) sparse_attn_mla_kernel(Attn
       for (int e = 0; e < 4; ++e) pr[nt][e] = mla_exp2(s[nt][e] - (e < 2 ? z0 : z1));
     l0 += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
     l1 += (pr[0][2] + pr[0][3]) + (pr[1][2] + pr[1][3]);
-    uint32_t ph[4], pl[4];
+    uint32_t pf[4];
     {
       const float a[4][2] = {{pr[0][0], pr[0][1]}, {pr[0][2], pr[0][3]}, {pr[1][0], pr[1][1]}, {pr[1][2], pr[1][3]}};
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        ph[r] = mla_pack_bf16(a[r][0], a[r][1]);
-        pl[r] = mla_pack_bf16(a[r][0] - mla_lo_f(ph[r]), a[r][1] - mla_hi_f(ph[r]));
-      }
+      for (int r = 0; r < 4; ++r) pf[r] = mla_pack_f16(a[r][0], a[r][1]);
     }
-    // O += P . V over this warp's 128 value dims (units 16 w .. 16 w + 15)
+    // O += P . V over this warp's 128 value dims (units 16 w .. 16 w + 15), fp16
 #pragma unroll
     for (int j = 0; j < 16; j += 2) {
       const int mtx = lane >> 3;
       uint32_t b0, b1, b2, b3;
       mla_ldsm4_t(st + mla_off((mtx & 1) * 8 + (lane & 7), 16 * warp + j + (mtx >> 1)), b0, b1, b2, b3);
-      mla_mma(o[j], ph, b0, b1);
-      mla_mma(o[j], pl, b0, b1);
-      mla_mma(o[j + 1], ph, b2, b3);
-      mla_mma(o[j + 1], pl, b2, b3);
+      mla_mma_f16(o[j], pf, mla_bf16x2_to_f16x2(b0), mla_bf16x2_to_f16x2(b1));
+      mla_mma_f16(o[j + 1], pf, mla_bf16x2_to_f16x2(b2), mla_bf16x2_to_f16x2(b3));
     }
   }
   cp_async_wait<0>();
