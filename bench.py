@@ -121,8 +121,8 @@ def load_peaks():
 # Sources compiled into each attention kernel: a recorded ncu traffic figure
 # holds only while all of them are unchanged.
 ATTN_SOURCES = {
-    "sparse_attn_mma_kernel": ("decode_attn_mma.cu", "attn_common.cuh", "device_common.cuh"),
-    "sparse_attn_mma_cluster_kernel": ("decode_attn_mma.cu", "attn_common.cuh", "device_common.cuh"),
+    "sparse_attn_mma_kernel": ("decode_attn_mma.cu", "mma_attn.cuh", "attn_common.cuh", "device_common.cuh"),
+    "sparse_attn_mma_cluster_kernel": ("decode_attn_mma.cu", "mma_attn.cuh", "attn_common.cuh", "device_common.cuh"),
     "sparse_attn_mla_kernel": ("decode_attn_mla.cu", "attn_common.cuh", "device_common.cuh"),
     "sparse_attn_kernel": ("decode_attn.cu", "attn_common.cuh", "device_common.cuh"),
 }

@@ -42,6 +42,21 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ uint32_t pack_f16(float a, float b) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+  return r;
+}
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) { return pack_f16(bf16_lo_f(w), bf16_hi_f(w)); }
+
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
@@ -217,15 +232,14 @@ __device__ __forceinline__ void mma_chunk(const AttnParams& p, const uint32_t (&
     for (int e = 0; e < 4; ++e) pr[nt][e] = fast_exp2(s[nt][e] - (e < 2 ? z0 : z1));
   l0 += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
   l1 += (pr[0][2] + pr[0][3]) + (pr[1][2] + pr[1][3]);
-  // P as the A operand (k = the 16 tokens), hi and lo parts
-  uint32_t ph[4], pl[4];
+  // P as the A operand (k = the 16 tokens) in fp16: P in [0, 1] rounds with
+  // relative error <= 2^-11, and V's bf16 pairs convert to fp16 exactly
+  // within fp16's range, so one MMA per n-tile replaces a bf16 hi + lo pair
+  uint32_t pf[4];
   {
     const float a[4][2] = {{pr[0][0], pr[0][1]}, {pr[0][2], pr[0][3]}, {pr[1][0], pr[1][1]}, {pr[1][2], pr[1][3]}};
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      ph[r] = pack_bf16(a[r][0], a[r][1]);
-      pl[r] = pack_bf16(a[r][0] - bf16_lo_f(ph[r]), a[r][1] - bf16_hi_f(ph[r]));
-    }
+    for (int r = 0; r < 4; ++r) pf[r] = pack_f16(a[r][0], a[r][1]);
   }
   // O += P . V over 16 n-tiles of 8 value columns
 #pragma unroll
@@ -235,10 +249,8 @@ __device__ __forceinline__ void mma_chunk(const AttnParams& p, const uint32_t (&
     const uint32_t addr = vb + tile_off((mtx & 1) * 8 + (lane & 7), j + (mtx >> 1));
     uint32_t b0, b1, b2, b3;
     ldsm_x4_t(addr, b0, b1, b2, b3);
-    mma_bf16_16816(o[j], ph, b0, b1);
-    mma_bf16_16816(o[j], pl, b0, b1);
-    mma_bf16_16816(o[j + 1], ph, b2, b3);
-    mma_bf16_16816(o[j + 1], pl, b2, b3);
+    mma_f16_16816(o[j], pf, bf16x2_to_f16x2(b0), bf16x2_to_f16x2(b1));
+    mma_f16_16816(o[j + 1], pf, bf16x2_to_f16x2(b2), bf16x2_to_f16x2(b3));
   }
 }
 
