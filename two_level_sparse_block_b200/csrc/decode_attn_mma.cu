@@ -11,9 +11,9 @@
 //   S  = Q . K^T   A = q of the group's heads (rows >= G are zero), B = K rows
 //                  via ldmatrix from a 128B-swizzled stage
 //   softmax        online per head in fp32 registers, base 2
-//   O += P . V     A = P from the S accumulators, split into bf16 hi + lo
-//                  parts (two MMAs: P keeps ~16 significant bits), B = V rows
-//                  via ldmatrix.trans
+//   O += P . V     in fp16: A = P from the S accumulators rounded to fp16
+//                  (relative error <= 2^-11), B = V rows via ldmatrix.trans,
+//                  their bf16 pairs converted to fp16 exactly
 // At the end of each (row) segment of its range the CTA folds its warps in
 // shared memory and writes (m, l, O) to the split workspace; the last CTA to
 // finish a row merges the splits by log-sum-exp (attn_common.cuh).

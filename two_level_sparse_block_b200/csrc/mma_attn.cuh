@@ -17,12 +17,7 @@ constexpr int kChunk = 16;           // tokens per chunk
 constexpr int kChunkBytes = 8192;    // K (4 KB) + V (4 KB) of 16 tokens
 constexpr int kMmaDv = 128;          // K and V row width of these kernels
 
-// two floats -> bf16x2 (round to nearest even); `a` goes to the low half
-__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-  uint32_t r;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
-  return r;
-}
+// the two bf16 halves of a 32-bit word as floats
 __device__ __forceinline__ float bf16_lo_f(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi_f(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
@@ -163,8 +158,8 @@ __device__ __forceinline__ void mma_issue_rows(const AttnParams& p, int row, int
 // One chunk of 16 list entries for the fragment rows gq (m0, l0) and gq + 8
 // (m1, l1): S = Q.K^T scaled to base 2 and masked where the entry is no token
 // (bit e of vm clear: past the list end, or padding), the online softmax
-// update, and O += P.V with P split into bf16 hi + lo parts.  K and V tiles
-// of the chunk at shared address kb / kb + 4096.
+// update, and O += P.V in fp16.  K and V tiles of the chunk at shared
+// address kb / kb + 4096.
 __device__ __forceinline__ void mma_chunk(const AttnParams& p, const uint32_t (&qa)[8][4], float (&o)[16][4],
                                           float& m0, float& m1, float& l0, float& l1, uint32_t kb, uint32_t vm,
                                           int lane) {
