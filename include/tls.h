@@ -437,7 +437,9 @@ TLS_API tls_status tls_prefetch_diff(tls_block_cache* cache, const int32_t* new_
  * plan changes nothing, and the cache then returns that status from every
  * later transfer, plan or engine step.  done_event as in tls_prefetch_diff.
  * Needs a cache whose K/V are mapped pinned host memory (the pull path),
- * n_slots <= 32768 and B*Hkv*K_b <= 65536 (else TLS_ERR_UNSUPPORTED).  From
+ * n_slots <= 32768, B*Hkv*K_b <= 65536, and the plan's shared memory within
+ * 227 KB: 4 bytes per slot, per list entry and per possible victim
+ * (min(n_slots, B*Hkv*K_b)), plus about 4 KB (else TLS_ERR_UNSUPPORTED).  From
  * the first call on, the device holds the cache state: the host calls
  * (tls_block_cache_plan, tls_prefetch_diff, tls_block_cache_table) first
  * wait for the device to finish (cudaDeviceSynchronize) and read it back.

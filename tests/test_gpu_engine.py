@@ -132,6 +132,48 @@ def test_engine_follows_the_staggered_oracle(cfg, planner, monkeypatch):
         layer.close()
 
 
+@pytest.mark.parametrize("pool", ["2K_b", "3K_b+5"])
+@pytest.mark.parametrize("cfg", ENGINE, ids=lambda c: c.name)
+def test_engine_planners_leave_the_same_tables(cfg, pool, monkeypatch):
+    # the device planner keeps the slots its previous plan used (those of
+    # M_{t-1}) without reading the list M_{t-1}; the host planner keeps the
+    # slots of the list: step by step both engines copy as many blocks and
+    # leave the same slot table (12 steps of the drifting trajectory; the
+    # larger pool leaves older blocks resident, so the least-recently-used
+    # order picks the victims)
+    runtime, tls = _rt()
+    n_slots = None if pool == "2K_b" else (3 * cfg.K_b + 5) * cfg.rows
+    qs = synth.gen_query_trajectory(cfg, 12)
+    K, V, _ = synth.gen_kv(cfg, qs[0])
+    lab = synth.gen_label_channels(cfg)
+    layers = []
+    try:
+        for planner in ("host", "device"):
+            monkeypatch.setenv("TLS_ENGINE_PLANNER", planner)
+            layers.append(runtime.offloaded_layer_for_config(cfg, K, V, lab, n_slots=n_slots))
+        kernels = [tls.tls_engine_step_kernels(layer.engine) for layer in layers]
+        assert kernels[1] == kernels[0] + 1  # plan + pull against the host planner's pull alone
+        moved = 0
+        for t, q in enumerate(qs):
+            tabs = []
+            for layer in layers:
+                layer.step(_dev_q(q))
+                torch.cuda.synchronize()
+                assert layer.check_device_error() == 0
+                tab = np.empty(tuple(layer.slot_table.shape), dtype=np.int32)
+                tls.tls_block_cache_table(layer.cache, tab)
+                tabs.append(tab)
+            assert np.array_equal(tabs[0], tabs[1]), f"{cfg.name} step {t}: slot tables differ"
+            if t > 0:
+                n = [layer.stats(t - 1).n_copied for layer in layers]
+                assert n[0] == n[1], f"{cfg.name} step {t - 1}: copied {n[1]} (device) vs {n[0]} (host)"
+                moved += n[0]
+        assert moved > 0  # the trajectory drifts: blocks were evicted and copied
+    finally:
+        for layer in layers:
+            layer.close()
+
+
 def test_engine_copy_failure_is_reported_and_sticks(monkeypatch):
     # host-side fault injection: the transfer of step 2 fails before anything
     # is issued; that step and every later one return TLS_ERR_COPY, and the

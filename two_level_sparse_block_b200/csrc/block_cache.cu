@@ -55,9 +55,9 @@ struct tls_block_cache {
   int64_t* owner_dev = nullptr;
   int64_t* last_use_dev = nullptr;
   int4* jobs_dev = nullptr;      // [rows * K_b max] {tok0 lo, tok0 hi, slot, list entry}
-  int32_t* victims_dev = nullptr;
   int32_t* n_jobs_dev = nullptr;
   int32_t* dev_failed = nullptr;  // pinned, mapped: set by a plan that found too few evictable slots
+  int32_t* dev_failed_dptr = nullptr;  // its device address
   int max_entries = 0;            // rows * K_b the device arrays were sized for
 };
 
@@ -293,94 +293,171 @@ struct PlanParams {
   const int32_t* new_idx;  // M_t [rows, K_b]
   const int32_t* in_use;   // M_{t-1} [rows, K_b] or NULL
   int rows, nb, K_b, n_slots, bs;
+  int keep_prev;           // 1: the slots the previous plan used are kept (its list was M_{t-1})
   int64_t ctx_len, step;   // step: the plan's number (last use of M_t's slots)
   int4* jobs;
-  int32_t* victims;
   int32_t* n_jobs;
   int32_t* n_out;    // optional: n_copy, or -1 when the plan failed
   int32_t* failed;   // mapped pinned flag, sticky
 };
 
-// Exclusive prefix of v over the CTA; *total receives the sum.  All threads call it.
-__device__ __forceinline__ int plan_block_scan(int v, int* warp_sums, int* total) {
+// Dynamic shared memory of the plan kernel (byte offsets): the slots' keys,
+// the kept bits, the victims in slot order, the state of every list entry
+// and the top-k scratch.
+struct PlanSmem {
+  size_t keys, kept, vic, ent, ts, total;
+};
+__host__ __device__ inline PlanSmem plan_smem(int n_slots, int n_entries) {
+  auto a16 = [](size_t x) { return (x + 15) & ~(size_t)15; };
+  PlanSmem m;
+  const int nv = n_entries < n_slots ? n_entries : n_slots;
+  m.keys = 0;
+  m.kept = m.keys + a16((size_t)n_slots * 4);
+  m.vic = m.kept + a16((size_t)((n_slots + 31) / 32) * 4);
+  m.ent = m.vic + a16((size_t)nv * 4);
+  m.ts = m.ent + a16((size_t)n_entries * 4);
+  m.total = m.ts + a16(sizeof(TopkScratch));
+  return m;
+}
+
+// Exclusive prefix of v over the CTA, with the total and the CTA's largest
+// x.  All threads call it; three barriers.
+__device__ __forceinline__ unsigned long long plan_scan_max(unsigned long long v, uint32_t x,
+                                                            unsigned long long* wsum, uint32_t* wmax,
+                                                            unsigned long long* total, uint32_t* xmax) {
+  constexpr int NW = kPlanThreads / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int x = v;
+  unsigned long long s = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
+    const unsigned long long y = __shfl_up_sync(0xffffffffu, s, o);
+    if (lane >= o) s += y;
   }
-  if (lane == 31) warp_sums[warp] = x;
+  x = __reduce_max_sync(0xffffffffu, x);
+  if (lane == 31) wsum[warp] = s;
+  if (lane == 0) wmax[warp] = x;
   __syncthreads();
   if (warp == 0) {
-    int w = lane < kPlanThreads / 32 ? warp_sums[lane] : 0;
+    unsigned long long w = lane < NW ? wsum[lane] : 0ull;
+    uint32_t m = lane < NW ? wmax[lane] : 0u;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      const unsigned long long y = __shfl_up_sync(0xffffffffu, w, o);
       if (lane >= o) w += y;
     }
-    warp_sums[lane] = w;  // inclusive
+    m = __reduce_max_sync(0xffffffffu, m);
+    if (lane < NW) wsum[lane] = w;  // inclusive
+    if (lane == 0) wmax[NW] = m;
   }
   __syncthreads();
-  const int before = (warp > 0 ? warp_sums[warp - 1] : 0) + x - v;
-  *total = warp_sums[kPlanThreads / 32 - 1];
-  __syncthreads();  // warp_sums may be reused
+  const unsigned long long before = (warp > 0 ? wsum[warp - 1] : 0ull) + s - v;
+  *total = wsum[NW - 1];
+  *xmax = wmax[NW];
+  __syncthreads();  // wsum / wmax may be reused
   return before;
 }
 
+// One CTA plans T_t and applies it.  The memory round trips on the path are
+// few on purpose (the kernel runs beside the attention, which keeps DRAM busy
+// and each round trip long): the first slot's state, the first list entries
+// and the sticky flag are loaded together; then the table entries of M_t
+// (and M_{t-1}); everything else is shared memory until the evicted slots'
+// owners are read.  A list entry's state: its slot when resident, -1 when not
+// a block (padding), -2 - block when it must be copied.
 __global__ void __launch_bounds__(kPlanThreads, 1) block_plan_kernel(PlanParams p) {
-  extern __shared__ __align__(16) uint32_t pkeys[];  // [n_slots], then need flags [rows * K_b]
-  uint8_t* needf = reinterpret_cast<uint8_t*>(pkeys + ((p.n_slots + 3) & ~3));
-  const int E = p.rows * p.K_b;
-  TopkScratch* ts = reinterpret_cast<TopkScratch*>(needf + ((E + 15) & ~15));
-  __shared__ int warp_sums[32];
-  __shared__ int bad;
+  extern __shared__ __align__(16) uint8_t psm[];
+  constexpr int NT = kPlanThreads;
+  const int E = p.rows * p.K_b, nsl = p.n_slots;
+  const PlanSmem L = plan_smem(nsl, E);
+  uint32_t* pkeys = reinterpret_cast<uint32_t*>(psm + L.keys);
+  uint32_t* kept = reinterpret_cast<uint32_t*>(psm + L.kept);
+  int* vic = reinterpret_cast<int*>(psm + L.vic);
+  int* ent = reinterpret_cast<int*>(psm + L.ent);
+  TopkScratch* ts = reinterpret_cast<TopkScratch*>(psm + L.ts);
+  __shared__ unsigned long long wsum[NT / 32];
+  __shared__ uint32_t wmax[NT / 32 + 1];
+  __shared__ int bad, failed_s, thr_bin, thr_above;
   const int tid = threadIdx.x;
   const int32_t* __restrict__ new_idx = p.new_idx;
   const int32_t* __restrict__ in_use = p.in_use;
-  if (*reinterpret_cast<volatile int32_t*>(p.failed) != 0) {
+  const uint32_t kFree = float_key(33554432.0f), kKept = float_key(0.0f);
+
+  // 1. loads that depend on nothing: this thread's first slot and first list entry, the flag
+  int64_t own0 = -1, lu0 = 0;
+  if (tid < nsl) {
+    own0 = p.owner[tid];
+    lu0 = p.last_use[tid];
+  }
+  int blk0 = -1, prv0 = -1, ub0 = -1;
+  if (tid < E) {
+    blk0 = new_idx[tid];
+    prv0 = tid % p.K_b > 0 ? new_idx[tid - 1] : -1;
+    ub0 = in_use != nullptr ? in_use[tid] : -1;
+  }
+  const int32_t failed0 = tid == 0 ? *reinterpret_cast<volatile int32_t*>(p.failed) : 0;
+  for (int w = tid; w < (nsl + 31) / 32; w += NT) kept[w] = 0u;
+  if (tid < 256) ts->hist[tid] = 0;
+  if (tid == 0) bad = 0;
+  __syncthreads();
+  // 2. the slots of M_t and M_{t-1} are kept; M_t must list distinct blocks
+  //    in [0, NB) in ascending order (as level 1 writes it)
+  for (int j = tid; j < E; j += NT) {
+    int blk = blk0, prv = prv0, ub = ub0;
+    if (j != tid) {
+      blk = new_idx[j];
+      prv = j % p.K_b > 0 ? new_idx[j - 1] : -1;
+      ub = in_use != nullptr ? in_use[j] : -1;
+    }
+    const int64_t r = j / p.K_b;
+    const bool ok = blk >= 0 && blk < p.nb;
+    if (blk >= p.nb || (blk >= 0 && j % p.K_b > 0 && (prv >= blk || prv < 0))) bad = 1;
+    const int s = ok ? p.table[r * p.nb + blk] : -1;
+    const int su = (ub >= 0 && ub < p.nb) ? p.table[r * p.nb + ub] : -1;
+    if (s >= 0 && s < nsl) atomicOr(&kept[s >> 5], 1u << (s & 31));
+    if (su >= 0 && su < nsl) atomicOr(&kept[su >> 5], 1u << (su & 31));
+    ent[j] = !ok ? -1 : s < 0 ? -2 - blk : s < nsl ? s : -1;
+  }
+  //    and the keys: free slots highest, then by the age of their last use
+  for (int s = tid; s < nsl; s += NT) {
+    int64_t own = own0, lu = lu0;
+    if (s != tid) {
+      own = p.owner[s];
+      lu = p.last_use[s];
+    }
+    const int64_t age = p.step - lu;
+    pkeys[s] = own < 0 ? kFree
+                       : (p.keep_prev && age == 1) ? kKept
+                                                   : float_key((float)(age < 1 ? 1 : (age > 16777215 ? 16777215 : age)));
+  }
+  if (tid == 0) failed_s = failed0;
+  __syncthreads();
+  if (failed_s != 0) {
     if (tid == 0) {
       *p.n_jobs = 0;
       if (p.n_out != nullptr) *p.n_out = -1;
     }
     return;
   }
-  if (tid == 0) bad = 0;
-  // 1. keys: free slots highest, then by the age of their last use
-  const uint32_t kFree = float_key(33554432.0f), kKept = float_key(0.0f);
-#pragma unroll 4
-  for (int s = tid; s < p.n_slots; s += kPlanThreads) {
-    const int64_t age = p.step - p.last_use[s];
-    pkeys[s] = p.owner[s] < 0 ? kFree : float_key((float)(age < 1 ? 1 : (age > 16777215 ? 16777215 : age)));
-  }
-  __syncthreads();
-  // 2. slots holding a block of M_t or M_{t-1} are kept, and the blocks of
-  //    M_t that are not resident flagged; M_t must list distinct blocks in
-  //    [0, NB) in ascending order (as level 1 writes it)
-#pragma unroll 4
-  for (int j = tid; j < E; j += kPlanThreads) {
-    const int64_t r = j / p.K_b;
-    const int blk = new_idx[j];
-    const int prv = j % p.K_b > 0 ? new_idx[j - 1] : -1;
-    const int ub = in_use != nullptr ? in_use[j] : -1;
-    const bool ok = blk >= 0 && blk < p.nb;
-    if (blk >= p.nb || (blk >= 0 && j % p.K_b > 0 && (prv >= blk || prv < 0))) bad = 1;
-    const int s = ok ? p.table[r * p.nb + blk] : -1;
-    const int su = (ub >= 0 && ub < p.nb) ? p.table[r * p.nb + ub] : -1;
-    if (s >= 0 && s < p.n_slots) pkeys[s] = kKept;
-    if (su >= 0 && su < p.n_slots) pkeys[su] = kKept;
-    needf[j] = ok && s < 0;
-  }
-  __syncthreads();
-  // 3. T_t in row, then list order: each thread a contiguous range of entries
-  const int per = (E + kPlanThreads - 1) / kPlanThreads;
+  // 3. counts: blocks to copy (this thread's contiguous range of entries),
+  //    evictable and free slots, and the oldest age
+  const int per = (E + NT - 1) / NT;
   const int j0 = min(E, tid * per), j1 = min(E, j0 + per);
-  int cnt = 0, avail = 0;
-  for (int j = j0; j < j1; ++j) cnt += needf[j];
-  for (int s = tid; s < p.n_slots; s += kPlanThreads) avail += pkeys[s] != kKept;
-  int n_copy = 0, n_avail = 0;
-  const int base = plan_block_scan(cnt, warp_sums, &n_copy);
-  plan_block_scan(avail, warp_sums, &n_avail);
+  int cnt = 0, avail = 0, nfree = 0;
+  uint32_t kmax = 0u;
+  for (int j = j0; j < j1; ++j) cnt += ent[j] <= -2;
+  for (int s = tid; s < nsl; s += NT) {
+    uint32_t k = pkeys[s];
+    if ((kept[s >> 5] >> (s & 31)) & 1u) pkeys[s] = k = kKept;
+    avail += k != kKept;
+    nfree += k == kFree;
+    if (k != kFree && k != kKept) kmax = max(kmax, k);
+  }
+  unsigned long long tot = 0ull;
+  uint32_t amax_key = 0u;
+  const unsigned long long before =
+      plan_scan_max(((unsigned long long)cnt << 40) | ((unsigned long long)avail << 20) | (unsigned long long)nfree,
+                    kmax, wsum, wmax, &tot, &amax_key);
+  const int n_copy = (int)(tot >> 40), n_avail = (int)((tot >> 20) & 0xFFFFFu), n_free = (int)(tot & 0xFFFFFu);
   if (bad != 0 || n_copy > n_avail) {
     // nothing changes; the cache refuses later plans
     if (tid == 0) {
@@ -390,140 +467,110 @@ __global__ void __launch_bounds__(kPlanThreads, 1) block_plan_kernel(PlanParams 
     }
     return;
   }
-  int pos = base;
-  for (int j = j0; j < j1; ++j) {
-    if (!needf[j]) continue;
-    const int64_t tok0 = (int64_t)(j / p.K_b) * p.ctx_len + (int64_t)new_idx[j] * p.bs;
-    p.jobs[pos++] = make_int4((int)(uint32_t)(tok0 & 0xFFFFFFFF), (int)(tok0 >> 32), 0, j);
+  if (tid == 0) {
+    *p.n_jobs = n_copy;
+    if (p.n_out != nullptr) *p.n_out = n_copy;
   }
   // 4. the victims: the n_copy largest keys (ties: lower slot), in slot
-  //    order.  Ages are small integers with many ties, so the threshold is
-  //    found from a histogram of ages below the oldest (256 of them); wider
-  //    spreads take the generic CTA top-k.
-  __shared__ int thr_bin, thr_above;
-  __shared__ float amax_s;
+  //    order.  Free slots first; ages are small integers with many ties, so
+  //    the threshold among used slots is found from a histogram of ages below
+  //    the oldest (256 of them); wider spreads take the generic CTA top-k.
   uint32_t thr = kFree;
-  int eq_take = n_copy;  // keys equal to thr to take, first ones in slot order
+  int eq_take = n_copy;  // keys equal to thr to take, the first ones in slot order
   bool generic = false;
-  if (n_copy > 0) {
-    int nfree = 0;
-    {
-      int f = 0;
-      for (int s = tid; s < p.n_slots; s += kPlanThreads) f += pkeys[s] == kFree;
-      plan_block_scan(f, warp_sums, &nfree);
+  const int need_used = n_copy - n_free;
+  if (n_copy > 0 && need_used > 0) {
+    const float amax = key_float(amax_key);
+    for (int s = tid; s < nsl; s += NT) {
+      const uint32_t k = pkeys[s];
+      if (k == kFree || k == kKept) continue;
+      const float d = amax - key_float(k);
+      if (d < 256.0f) atomicAdd(&ts->hist[(int)d], 1);
     }
-    const int need_used = n_copy - nfree;
-    if (need_used > 0) {
-      float am = 0.0f;
-      for (int s = tid; s < p.n_slots; s += kPlanThreads) {
-        const uint32_t k = pkeys[s];
-        if (k != kFree && k != kKept) am = fmaxf(am, key_float(k));
-      }
-      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 16));
-      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 8));
-      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 4));
-      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
-      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
-      for (int i = tid; i < 256; i += kPlanThreads) ts->hist[i] = 0;
-      if (tid == 0) amax_s = 0.0f;
-      __syncthreads();
-      if ((tid & 31) == 0) atomicMax(reinterpret_cast<int*>(&amax_s), __float_as_int(am));  // ages are >= 0
-      __syncthreads();
-      const float amax = amax_s;
-      for (int s = tid; s < p.n_slots; s += kPlanThreads) {
-        const uint32_t k = pkeys[s];
-        if (k == kFree || k == kKept) continue;
-        const float d = amax - key_float(k);
-        if (d < 256.0f) atomicAdd(&ts->hist[(int)d], 1);
-      }
-      __syncthreads();
-      if (tid < 32) {
-        // the bin (age below the oldest) where the count from the oldest reaches need_used
-        int run = 0, bin = -1, above = 0;
-        for (int c = 0; c < 256 && bin < 0; c += 32) {
-          int v = ts->hist[c + tid];
-          int x = v;
+    __syncthreads();
+    if (tid < 32) {
+      // the bin (age below the oldest) where the count from the oldest reaches need_used
+      int run = 0, bin = -1, above = 0;
+      for (int c = 0; c < 256 && bin < 0; c += 32) {
+        const int v = ts->hist[c + tid];
+        int x = v;
 #pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, x, o);
-            if (tid >= o) x += y;
-          }
-          const unsigned hit = __ballot_sync(0xffffffffu, run + x >= need_used);
-          if (hit != 0u) {
-            const int l = __ffs(hit) - 1;
-            bin = c + l;
-            above = run + __shfl_sync(0xffffffffu, x - v, l);
-          }
-          run += __shfl_sync(0xffffffffu, x, 31);
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, x, o);
+          if (tid >= o) x += y;
         }
-        if (tid == 0) {
-          thr_bin = bin;
-          thr_above = above;
+        const unsigned hit = __ballot_sync(0xffffffffu, run + x >= need_used);
+        if (hit != 0u) {
+          const int l = __ffs(hit) - 1;
+          bin = c + l;
+          above = run + __shfl_sync(0xffffffffu, x - v, l);
         }
+        run += __shfl_sync(0xffffffffu, x, 31);
       }
-      __syncthreads();
-      if (thr_bin < 0) {
-        generic = true;
-      } else {
-        thr = float_key(amax - (float)thr_bin);
-        eq_take = need_used - thr_above;
+      if (tid == 0) {
+        thr_bin = bin;
+        thr_above = above;
       }
+    }
+    __syncthreads();
+    if (thr_bin < 0) {
+      generic = true;
+    } else {
+      thr = float_key(amax - (float)thr_bin);
+      eq_take = need_used - thr_above;
     }
   }
   if (generic) {
-    cta_topk_ascending<kPlanThreads>(pkeys, p.n_slots, n_copy, p.victims, *ts, [](int i) { return i; });
+    cta_topk_ascending<NT>(pkeys, nsl, n_copy, vic, *ts, [](int i) { return i; });
   } else if (n_copy > 0) {
-    // victims: keys above thr, and the first eq_take keys equal to thr; then
-    // compacted in slot order (contiguous ranges of slots per thread)
-    const int sp = (p.n_slots + kPlanThreads - 1) / kPlanThreads;
-    const int s0 = min(p.n_slots, tid * sp), s1 = min(p.n_slots, s0 + sp);
-    int eq = 0;
-    for (int s = s0; s < s1; ++s) eq += pkeys[s] == thr;
-    int n_eq = 0;
-    int eq_before = plan_block_scan(eq, warp_sums, &n_eq);
-    int vic = 0;
-    for (int s = s0, e = eq_before; s < s1; ++s) {
+    // keys above thr and the first eq_take keys equal to it, compacted in
+    // slot order (a contiguous range of slots per thread)
+    const int sp = (nsl + NT - 1) / NT;
+    const int s0 = min(nsl, tid * sp), s1 = min(nsl, s0 + sp);
+    int above = 0, eq = 0;
+    for (int s = s0; s < s1; ++s) {
       const uint32_t k = pkeys[s];
-      if (k == thr) vic += e++ < eq_take;
-      else vic += k > thr && k != kKept;
+      above += k > thr && k != kKept;
+      eq += k == thr;
     }
-    int n_vic = 0;
-    int pos = plan_block_scan(vic, warp_sums, &n_vic);
-    for (int s = s0, e = eq_before; s < s1; ++s) {
+    unsigned long long t2 = 0ull;
+    uint32_t unused = 0u;
+    const unsigned long long b2 =
+        plan_scan_max(((unsigned long long)above << 32) | (unsigned long long)eq, 0u, wsum, wmax, &t2, &unused);
+    int e = (int)(b2 & 0xFFFFFFFFu);
+    int pos = (int)(b2 >> 32) + min(eq_take, e);
+    for (int s = s0; s < s1; ++s) {
       const uint32_t k = pkeys[s];
-      bool v;
-      if (k == thr) v = e++ < eq_take;
-      else v = k > thr && k != kKept;
-      if (v && pos < n_copy) p.victims[pos++] = s;
+      const bool v = k == thr ? e++ < eq_take : (k > thr && k != kKept);
+      if (v && pos < n_copy) vic[pos++] = s;
     }
   }
   __syncthreads();
   // the pull kernel may become resident from here (it waits for this grid)
   grid_launch_dependents();
-  // 5. copy i takes victim i: the evicted block loses its entry, the copied
-  //    one gets the slot (no entry is touched twice: copied blocks are not
-  //    resident, evicted ones are)
-  for (int i = tid; i < n_copy; i += kPlanThreads) {
-    const int slot = p.victims[i];
-    const int j = p.jobs[i].w;
-    const int64_t key = (int64_t)(j / p.K_b) * p.nb + new_idx[j];
-    const int64_t old = p.owner[slot];
-    if (old >= 0) p.table[old] = -1;
-    p.table[key] = slot;
-    p.owner[slot] = key;
-    p.jobs[i].z = slot;
-  }
-  __syncthreads();
-  // 6. every block of M_t is resident now: its slot was used at this step
-#pragma unroll 4
-  for (int j = tid; j < E; j += kPlanThreads) {
-    const int blk = new_idx[j];
-    const int s = (blk >= 0 && blk < p.nb) ? p.table[(int64_t)(j / p.K_b) * p.nb + blk] : -1;
-    if (s >= 0 && s < p.n_slots) p.last_use[s] = p.step;
-  }
-  if (tid == 0) {
-    *p.n_jobs = n_copy;
-    if (p.n_out != nullptr) *p.n_out = n_copy;
+  // 5. copy i (row, then list order) takes victim i: the evicted block loses
+  //    its entry, the copied one gets the slot (no entry is touched twice:
+  //    copied blocks are not resident, evicted ones are); every slot of M_t
+  //    was used at this step
+  int pos = (int)(before >> 40);
+  for (int j = j0; j < j1; ++j) {
+    int s = ent[j];
+    if (s == -1) continue;
+    const int64_t r = j / p.K_b;
+    if (s <= -2) {
+      const int blk = -2 - s;
+      const int i = pos++;
+      s = vic[i];
+      if (s < 0 || s >= nsl) continue;  // unreachable: n_copy victims were chosen
+      const int64_t key = r * p.nb + blk;
+      const int64_t old = p.owner[s];
+      if (old >= 0) p.table[old] = -1;
+      p.table[key] = s;
+      p.owner[s] = key;
+      const int64_t tok0 = r * p.ctx_len + (int64_t)blk * p.bs;
+      p.jobs[i] = make_int4((int)(uint32_t)(tok0 & 0xFFFFFFFF), (int)(tok0 >> 32), s, j);
+    }
+    p.last_use[s] = p.step;
   }
 }
 
@@ -573,6 +620,10 @@ tls_status block_cache_device_ready(tls_block_cache* c, int K_b) {
   if (c->n_slots > kPlanMaxSlots || entries > kPlanMaxEntries)
     return fail(TLS_ERR_UNSUPPORTED, "device planning takes at most %d slots and %d list entries", kPlanMaxSlots,
                 kPlanMaxEntries);
+  const size_t smem = plan_smem(c->n_slots, (int)entries).total;
+  if (smem > kMaxDynSmem)
+    return fail(TLS_ERR_UNSUPPORTED, "device planning of %d slots and %lld list entries needs %zu bytes of shared "
+                "memory (at most %zu)", c->n_slots, (long long)entries, smem, kMaxDynSmem);
   cudaError_t e = cudaSuccess;
   if (c->owner_dev == nullptr) {
     e = cudaMalloc((void**)&c->owner_dev, (size_t)c->n_slots * sizeof(int64_t));
@@ -581,14 +632,12 @@ tls_status block_cache_device_ready(tls_block_cache* c, int K_b) {
     if (e == cudaSuccess)
       e = cudaHostAlloc((void**)&c->dev_failed, sizeof(int32_t), cudaHostAllocMapped | cudaHostAllocPortable);
     if (e == cudaSuccess) *c->dev_failed = 0;
+    if (e == cudaSuccess) e = cudaHostGetDevicePointer((void**)&c->dev_failed_dptr, c->dev_failed, 0);
   }
   if (e == cudaSuccess && entries > c->max_entries) {
     if (c->jobs_dev != nullptr) cudaFree(c->jobs_dev);
-    if (c->victims_dev != nullptr) cudaFree(c->victims_dev);
     c->jobs_dev = nullptr;
-    c->victims_dev = nullptr;
     e = cudaMalloc((void**)&c->jobs_dev, (size_t)entries * sizeof(int4));
-    if (e == cudaSuccess) e = cudaMalloc((void**)&c->victims_dev, (size_t)entries * sizeof(int32_t));
     if (e == cudaSuccess) c->max_entries = (int)entries;
   }
   if (e == cudaSuccess && !c->device_owned) {
@@ -620,12 +669,15 @@ int64_t block_cache_block_bytes(const tls_block_cache* c) {
 }
 
 // The incremental prefetch planned on the device: one plan kernel (one CTA)
-// reads M_t and M_{t-1} from device memory and updates the slot table, the
-// owners and the last uses; a pull kernel copies its jobs.  n_out (device or
-// mapped memory, may be NULL) receives the number of copied blocks, or -1
+// reads M_t (and M_{t-1}) from device memory and updates the slot table, the
+// owners and the last uses; a pull kernel copies its jobs.  keep_prev: the
+// slots the previous plan used are kept instead of those of in_use_dev (the
+// engine, whose previous plan was for M_{t-1}: the plan then no longer reads
+// M_{t-1}, and level 1 may overwrite it while the plan runs).  n_out (device
+// or mapped memory, may be NULL) receives the number of copied blocks, or -1
 // when the plan failed (the cache is failed from then on).
 tls_status prefetch_device_impl(tls_block_cache* c, const int32_t* new_dev, const int32_t* in_use_dev, int K_b,
-                                cudaStream_t cs, int32_t* n_out, cudaEvent_t planned) {
+                                cudaStream_t cs, int32_t* n_out, bool keep_prev) {
   tls_status st = device_plan_status(*c);
   if (st != TLS_OK) return st;
   if (fault_injected_copy()) return fail(TLS_ERR_COPY, "prefetch_diff: copy failure injected (TLS_FAULT_INJECT=copy)");
@@ -637,7 +689,8 @@ tls_status prefetch_device_impl(tls_block_cache* c, const int32_t* new_dev, cons
   p.owner = c->owner_dev;
   p.last_use = c->last_use_dev;
   p.new_idx = new_dev;
-  p.in_use = in_use_dev;
+  p.in_use = keep_prev ? nullptr : in_use_dev;
+  p.keep_prev = keep_prev ? 1 : 0;
   p.rows = c->rows;
   p.nb = c->nb;
   p.K_b = K_b;
@@ -646,19 +699,14 @@ tls_status prefetch_device_impl(tls_block_cache* c, const int32_t* new_dev, cons
   p.ctx_len = c->shape.ctx_len;
   p.step = c->step;
   p.jobs = c->jobs_dev;
-  p.victims = c->victims_dev;
   p.n_jobs = c->n_jobs_dev;
   p.n_out = n_out;
-  int32_t* dflag = nullptr;
-  cudaError_t e = cudaHostGetDevicePointer((void**)&dflag, c->dev_failed, 0);
-  p.failed = dflag;
-  const size_t smem = (size_t)((c->n_slots + 3) & ~3) * 4 + (size_t)((c->rows * K_b + 15) & ~15) +
-                      sizeof(TopkScratch) + 16;
-  if (e == cudaSuccess) e = kernel_attrs((const void*)block_plan_kernel, smem);
+  p.failed = c->dev_failed_dptr;
+  const size_t smem = plan_smem(c->n_slots, c->rows * K_b).total;
+  cudaError_t e = kernel_attrs((const void*)block_plan_kernel, smem);
   if (e != cudaSuccess) return cuda_check(e, "prefetch_diff_device: plan kernel setup");
   block_plan_kernel<<<1, kPlanThreads, smem, cs>>>(p);
   e = cudaGetLastError();
-  if (e == cudaSuccess && planned != nullptr) e = cudaEventRecord(planned, cs);  // the lists have been read
   const int64_t kblk = (int64_t)c->shape.block_size * c->hk_stride * 2;
   const int64_t vblk = (int64_t)c->shape.block_size * c->hv_stride * 2;
   const bool with_v = c->host_v != nullptr && c->slot_v != nullptr;
@@ -875,7 +923,6 @@ extern "C" void tls_block_cache_destroy(tls_block_cache* c) {
     cudaFreeHost(c->dev_failed);
   }
   if (c->jobs_dev != nullptr) cudaFree(c->jobs_dev);
-  if (c->victims_dev != nullptr) cudaFree(c->victims_dev);
   delete c;
 }
 
@@ -946,7 +993,7 @@ extern "C" tls_status tls_prefetch_diff_device(tls_block_cache* c, const int32_t
   if (c == nullptr || new_block_idx_dev == nullptr) return fail(TLS_ERR_INVALID_ARG, "prefetch_diff_device: NULL argument");
   if (K_b < 1 || K_b > c->nb) return fail(TLS_ERR_INVALID_ARG, "prefetch_diff_device: K_b out of range");
   tls_status st = prefetch_device_impl(c, new_block_idx_dev, in_use_block_idx_dev, K_b, (cudaStream_t)copy_stream,
-                                       n_copied_dev, nullptr);
+                                       n_copied_dev, /*keep_prev=*/false);
   if (st != TLS_OK || done_event == nullptr) return st;
   cudaError_t e = cudaEventRecord((cudaEvent_t)done_event, (cudaStream_t)copy_stream);
   return e == cudaSuccess ? TLS_OK : cuda_check(e, "prefetch_diff_device: done event");

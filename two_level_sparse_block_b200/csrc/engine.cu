@@ -37,7 +37,7 @@ tls_status prefetch_diff_impl(tls_block_cache* c, const int32_t* new_idx, const 
 tls_status block_cache_view(const tls_block_cache* c, tls_kv_view* kv);
 tls_status block_cache_device_ready(tls_block_cache* c, int K_b);
 tls_status prefetch_device_impl(tls_block_cache* c, const int32_t* new_dev, const int32_t* in_use_dev, int K_b,
-                                cudaStream_t cs, int32_t* n_out, cudaEvent_t planned);
+                                cudaStream_t cs, int32_t* n_out, bool keep_prev);
 int64_t block_cache_block_bytes(const tls_block_cache* c);
 tls_status block_cache_check(tls_block_cache* c);
 }  // namespace tls
@@ -69,7 +69,6 @@ struct tls_engine {
   bool device_plan = false;
   int32_t* n_copied_map = nullptr;  // pinned, mapped [kRing]
   int32_t* n_copied_dev = nullptr;  // its device address
-  cudaEvent_t ev_planned = nullptr;  // after the plan kernel, before the pull
   int64_t t = 0;
   tls_status failed = TLS_OK;
   double wait_ms = 10000.0;  // deadline of the host waits (TLS_HOST_WAIT_MS)
@@ -82,7 +81,7 @@ namespace {
 void release(tls_engine* e) {
   if (e->sel != nullptr) cudaStreamSynchronize(e->sel);
   if (e->copy != nullptr) cudaStreamSynchronize(e->copy);
-  for (cudaEvent_t* ev : {&e->ev_q, &e->ev_sel, &e->ev_attn[0], &e->ev_attn[1], &e->ev_planned})
+  for (cudaEvent_t* ev : {&e->ev_q, &e->ev_sel, &e->ev_attn[0], &e->ev_attn[1]})
     if (*ev != nullptr) cudaEventDestroy(*ev);
   if (e->n_copied_map != nullptr) cudaFreeHost(e->n_copied_map);
   for (int i = 0; i < kRing; ++i)
@@ -170,7 +169,6 @@ tls_status engine_create(const tls_shape* shape, int32_t K_b, int32_t k, const v
     if (st == TLS_OK) {
       ce = cudaHostAlloc((void**)&e->n_copied_map, kRing * sizeof(int32_t), cudaHostAllocMapped | cudaHostAllocPortable);
       if (ce == cudaSuccess) ce = cudaHostGetDevicePointer((void**)&e->n_copied_dev, e->n_copied_map, 0);
-      if (ce == cudaSuccess) ce = cudaEventCreateWithFlags(&e->ev_planned, cudaEventDisableTiming);
       if (ce != cudaSuccess) {
         release(e);
         return cuda_check(ce, "engine_create: device planning buffers");
@@ -257,10 +255,11 @@ tls_status resident_step(tls_engine* e, const void* q, int32_t out_dtype, void* 
 }
 
 // The offloaded step with the transfer planned on the device: no host wait.
-// Beside the host-planned order, two device-side waits take the place of the
-// host's: level 2 waits for the level 1 of the step before (it reads M_{t-1}),
-// and level 1 waits for the plan kernel of the step before (which read the
-// list level 1 now overwrites).
+// Beside the host-planned order, one device-side wait takes the place of the
+// host's: level 2 waits for the level 1 of the step before (it reads M_{t-1}).
+// The plan of step t keeps the slots the plan of step t-1 used (M_{t-1}'s)
+// without reading M_{t-1}, so level 1 of step t+1 may overwrite that list
+// while the plan runs.
 tls_status device_step(tls_engine* e, const void* q, int32_t out_dtype, void* out, float* lse, cudaStream_t A) {
   const tls_shape& s = e->shape;
   const int cur = (int)(e->t & 1), prev = cur ^ 1;
@@ -277,7 +276,8 @@ tls_status device_step(tls_engine* e, const void* q, int32_t out_dtype, void* ou
     if (ce == cudaSuccess) ce = cudaEventRecord(e->copy_start[rp], e->copy);
     if (ce != cudaSuccess) return cuda_check(ce, "engine_step: prologue");
     e->n_copied_map[rp] = 0;
-    st = prefetch_device_impl(e->cache, e->bidx[prev], nullptr, e->K_b, e->copy, e->n_copied_dev + rp, e->ev_planned);
+    st = prefetch_device_impl(e->cache, e->bidx[prev], nullptr, e->K_b, e->copy, e->n_copied_dev + rp,
+                              /*keep_prev=*/false);
     if (st != TLS_OK) return st;
     ce = cudaEventRecord(e->copy_end[rp], e->copy);
     if (ce != cudaSuccess) return cuda_check(ce, "engine_step: prologue");
@@ -285,34 +285,35 @@ tls_status device_step(tls_engine* e, const void* q, int32_t out_dtype, void* ou
   // M_{t-1} (written by level 1 of the step before) is complete before level 2
   ce = cudaStreamWaitEvent(A, e->ev_sel, 0);
   if (ce == cudaSuccess) ce = cudaEventRecord(e->ev_q, A);
-  // level 1 for q_t on the select stream: M_t, once the plan of the step
-  // before has read the list it overwrites
-  if (ce == cudaSuccess) ce = cudaStreamWaitEvent(e->sel, e->ev_q, 0);
-  if (ce == cudaSuccess) ce = cudaStreamWaitEvent(e->sel, e->ev_planned, 0);
+  if (ce != cudaSuccess) return cuda_check(ce, "engine_step: q event");
+  // level 2 within M_{t-1} first, on A, on at most half the SMs (as in the
+  // resident step: launched first, its CTAs are placed first, and level 1
+  // keeps the other half)
+  st = select_tokens_impl(s, q, e->label_ch, e->codes, e->scales, e->bidx[prev], e->K_b, e->k, e->token_idx, nullptr,
+                          e->ws, e->L, A, /*pdl=*/false, /*lean=*/true);
+  if (st != TLS_OK) return st;
+  // level 1 for q_t on the select stream: M_t
+  ce = cudaStreamWaitEvent(e->sel, e->ev_q, 0);
   if (ce != cudaSuccess) return cuda_check(ce, "engine_step: select stream");
   st = select_blocks_impl(s, q, e->meta, e->K_b, e->bidx[cur], nullptr, e->ws, e->L, e->sel);
   if (st != TLS_OK) return st;
   ce = cudaEventRecord(e->ev_sel, e->sel);
   if (ce != cudaSuccess) return cuda_check(ce, "engine_step: select stream");
-  // level 2 within M_{t-1} and the attention over the slot pool, on A
-  st = select_tokens_impl(s, q, e->label_ch, e->codes, e->scales, e->bidx[prev], e->K_b, e->k, e->token_idx, nullptr,
-                          e->ws, e->L, A, /*pdl=*/false);
-  if (st != TLS_OK) return st;
+  // the attention over the slot pool, on A, once T_{t-1} has landed
   ce = cudaEventRecord(e->ready[ri], A);
   if (ce == cudaSuccess) ce = cudaStreamWaitEvent(A, e->copy_end[rp], 0);  // T_{t-1} has landed
   if (ce != cudaSuccess) return cuda_check(ce, "engine_step: wait for the transfer");
   st = sparse_attn_impl(s, q, e->kv, e->token_idx, e->k, out_dtype, out, lse, e->ws, e->L, A, /*pdl=*/false);
   if (st != TLS_OK) return st;
-  ce = cudaEventRecord(e->ev_attn[cur], A);
-  // T_t on the copy stream, once M_t is chosen and the attention of step t-1
-  // (whose slots may be evicted now) is done; alongside the attention of step t
-  if (ce == cudaSuccess) ce = cudaStreamWaitEvent(e->copy, e->ev_sel, 0);
-  if (ce == cudaSuccess) ce = cudaStreamWaitEvent(e->copy, e->ev_attn[prev], 0);
+  // T_t on the copy stream once M_t is chosen, alongside the attention of
+  // step t.  The attention of step t-1 (whose slots may be evicted now) is
+  // done by then: level 1 started after q_t, which A records after it.
+  ce = cudaStreamWaitEvent(e->copy, e->ev_sel, 0);
   if (ce == cudaSuccess) ce = cudaEventRecord(e->copy_start[ri], e->copy);
   if (ce != cudaSuccess) return cuda_check(ce, "engine_step: copy stream");
   e->n_copied_map[ri] = 0;
-  st = prefetch_device_impl(e->cache, e->bidx[cur], e->bidx[prev], e->K_b, e->copy, e->n_copied_dev + ri,
-                            e->ev_planned);
+  st = prefetch_device_impl(e->cache, e->bidx[cur], nullptr, e->K_b, e->copy, e->n_copied_dev + ri,
+                            /*keep_prev=*/true);
   if (st != TLS_OK) return st;
   ce = cudaEventRecord(e->copy_end[ri], e->copy);
   if (ce != cudaSuccess) return cuda_check(ce, "engine_step: copy stream");
