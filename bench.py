@@ -827,46 +827,67 @@ def main():
     value = job_tokens_per_s(world, c.batch, ms_per_step)
 
     # end to end through the public API: pinned host q in, host out back, every
-    # step.  As a serving loop runs it: the host -> device copy of q, the
-    # engine step and the device -> host copy of the output captured together
-    # into graphs (one per block-list parity) and replayed; and, for
-    # reference, the same three calls issued eagerly every step.
+    # step.  As a serving loop runs it: q brought in from pinned host memory by
+    # tls_copy_from_host (one kernel whose loads cross PCIe) and the engine
+    # step, whose attention writes the output straight into pinned host memory
+    # (its stores cross PCIe), captured together into graphs (one per
+    # block-list parity) and replayed; for reference, the same calls issued
+    # eagerly every step, and the graphs with copy-engine transfers instead (q
+    # by a host -> device copy, the output by a device -> host copy).
     q_host = torch.empty(st.q.shape, dtype=torch.bfloat16).pin_memory()
     q_host.copy_(st.q.cpu())
     out_host = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
     q_dev = torch.empty_like(st.q)
-    g_e2e = [torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()]
+
+    def e2e_step(s, copy_back):
+        if copy_back:
+            q_dev.copy_(q_host, non_blocking=True)
+            eng.step(q=q_dev, stream=s)
+            out_host.copy_(eng.out, non_blocking=True)
+        else:
+            tls.tls_copy_from_host(q_dev, q_host, None, s)
+            eng.step(q=q_dev, stream=s, out=out_host)
+
+    e2e_step(stream, False)  # checks the pinned source once, outside the captures
+    torch.cuda.synchronize(dev)
+    graphs = {}
     cap.wait_stream(stream)
     with torch.cuda.stream(cap):
-        for g in g_e2e:
-            with torch.cuda.graph(g, stream=cap):
-                q_dev.copy_(q_host, non_blocking=True)
-                eng.step(q=q_dev, stream=cap)
-                out_host.copy_(eng.out, non_blocking=True)
+        for copy_back in (False, True):
+            graphs[copy_back] = [torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()]
+            for g in graphs[copy_back]:
+                with torch.cuda.graph(g, stream=cap):
+                    e2e_step(cap, copy_back)
     stream.wait_stream(cap)
     torch.cuda.synchronize(dev)
 
-    def e2e_times(n, eager):
+    def e2e_times(n, eager, copy_back=False):
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
         for i in range(n):
             flush_l2(i)
             evs[i][0].record(stream)
             if eager:
-                q_dev.copy_(q_host, non_blocking=True)
-                eng.step(q=q_dev, stream=stream)
-                out_host.copy_(eng.out, non_blocking=True)
+                e2e_step(stream, copy_back)
             else:
-                g_e2e[i & 1].replay()
+                graphs[copy_back][i & 1].replay()
             evs[i][1].record(stream)
         torch.cuda.synchronize(dev)
         return sum(e[0].elapsed_time(e[1]) for e in evs) / n
 
     e2e_ms = e2e_times(args.e2e_steps, eager=False)
     e2e_eager_ms = e2e_times(args.e2e_steps, eager=True)
+    e2e_copy_ms = e2e_times(args.e2e_steps, eager=False, copy_back=True)
     if eng.check_device_error() != 0:
         raise RuntimeError("device error in the end-to-end steps")
-    e2e_ms, e2e_eager_ms = max_over_ranks([e2e_ms, e2e_eager_ms], world, dev)
-    del g_e2e
+    # the kernels' transfers give the copy engine's output bit for bit (the
+    # same q every step, so every steady step has the same output)
+    e2e_times(1, eager=True, copy_back=False)
+    zero_copy_out = out_host.clone()
+    e2e_times(1, eager=True, copy_back=True)
+    if not torch.equal(zero_copy_out, out_host):
+        raise RuntimeError("the end-to-end output differs from the copy-engine path's")
+    e2e_ms, e2e_eager_ms, e2e_copy_ms = max_over_ranks([e2e_ms, e2e_eager_ms, e2e_copy_ms], world, dev)
+    del graphs
 
     ab = algorithmic_bytes(c)
     attn_kernel = tls.tls_attn_kernel(st.shape)
@@ -903,11 +924,15 @@ def main():
         "gpu_launches": launches_per_step(c) * args.steps,
         "e2e": {"value": job_tokens_per_s(world, c.batch, e2e_ms), "unit": "decode tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": int(st.q.numel() * 2), "d2h_bytes_per_step": int(st.out.numel() * st.out.element_size()),
-                "path": "tls_engine_step (resident engine) via the Python binding, q copied in from pinned host "
-                        "and the output copied back to pinned host every step, the three captured together in "
-                        "graphs (one per block-list parity) and replayed",
+                "path": "tls_copy_from_host (q from pinned host memory, one kernel whose loads cross PCIe) and "
+                        "tls_engine_step (resident engine) via the Python binding every step, the attention "
+                        "writing the output straight into pinned host memory (its stores cross PCIe); the two "
+                        "captured together in graphs (one per block-list parity) and replayed",
                 "eager_ms_per_step": e2e_eager_ms,
-                "eager_path": "the same three calls issued from Python every step, no graph"},
+                "eager_path": "the same calls issued from Python every step, no graph",
+                "copy_back_ms_per_step": e2e_copy_ms,
+                "copy_back_path": "the same graphs with copy-engine transfers: q by a host -> device copy, the "
+                                  "output written to device memory and copied back by a device -> host copy"},
         "clocks": clocks,
         "wall_s_timed": wall,
     }

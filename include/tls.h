@@ -110,6 +110,20 @@ TLS_API const char* tls_last_error(void);
 TLS_API int32_t tls_version(void);
 
 /*
+ * Copies `bytes` from pinned host memory that the device can address
+ * (cudaHostAlloc, cudaHostRegister'd or pinned torch buffers) into device
+ * memory with one kernel on `stream`, whose 16-byte loads cross PCIe: for a
+ * decode step's small inputs (q), it starts sooner than a copy-engine
+ * transfer, most of all inside a captured step.  src (host), dst (device) and
+ * bytes must be multiples of 16 bytes; bytes = 0 does nothing.  The source
+ * range is checked once per (address, size) (cudaPointerGetAttributes at
+ * both ends; the result is remembered, so a captured call does not repeat
+ * it): memory that is not pinned and mapped returns TLS_ERR_INVALID_ARG and
+ * launches nothing.  The source must stay allocated while the copy runs.
+ */
+TLS_API tls_status tls_copy_from_host(void* dst_device, const void* src_host, size_t bytes, void* stream);
+
+/*
  * Name of the attention kernel tls_sparse_decode_attn launches for this
  * shape: "sparse_attn_mma_cluster_kernel" or "sparse_attn_mma_kernel" for
  * 128-wide K and V rows (one cluster of CTAs per row and head group of <= 16
@@ -124,8 +138,9 @@ TLS_API const char* tls_attn_kernel(const tls_shape* shape);
 
 /*
  * Name of the level-2 kernel tls_select_tokens (staggered = 0: as in
- * tls_select and tls_decode_step) or a resident engine's step (staggered !=
- * 0, which keeps level 2 to half the SMs) takes for this shape, K_b and k,
+ * tls_select and tls_decode_step) or an engine's step (staggered != 0: the
+ * resident step and the device-planned offloaded step, which keep level 2 to
+ * half the SMs) takes for this shape, K_b and k,
  * for 16-byte aligned codes and scales: "token_select_row_kernel",
  * "token_select_cluster_kernel" or "token_select_kernel".  cluster_ctas and
  * cta_threads (nullable, host) receive its CTAs per row (a thread-block
@@ -505,7 +520,10 @@ TLS_API tls_status tls_engine_create_resident(const tls_shape* shape, int32_t K_
 
 /*
  * One decode step t with query q (device bf16 [B, Hq, Dqk], ready on
- * `stream`).  Output as tls_sparse_decode_attn, written on `stream`.  Level 2
+ * `stream`).  Output as tls_sparse_decode_attn, written on `stream`; `out` may
+ * also be pinned host memory that the device can address (the attention's
+ * stores then cross PCIe, and the result is in host memory once the step's
+ * work on `stream` is complete, with no separate copy).  Level 2
  * and the attention use the blocks chosen at step t-1 (M_{t-1}, resident in
  * the cache) with q; level 1 chooses M_t from q on the engine's second stream,
  * and the blocks of M_t not yet resident are copied from host memory on the

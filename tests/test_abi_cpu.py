@@ -45,6 +45,20 @@ def test_version_and_error_string(tls):
     assert isinstance(tls.tls_last_error(), str)
 
 
+def test_copy_from_host_checks_its_arguments_before_anything(tls):
+    # NULL pointers and sizes or addresses that are not multiples of 16 bytes
+    # are rejected on the host (no CUDA call is reached)
+    lib = tls.lib()
+    buf = np.zeros(64, dtype=np.uint8)
+    p = buf.ctypes.data + (-buf.ctypes.data) % 16
+    assert lib.tls_copy_from_host(None, p, 16, None) == tls.TLS_ERR_INVALID_ARG
+    assert lib.tls_copy_from_host(p, None, 16, None) == tls.TLS_ERR_INVALID_ARG
+    assert lib.tls_copy_from_host(p, p, 24, None) == tls.TLS_ERR_INVALID_ARG
+    assert lib.tls_copy_from_host(p + 8, p, 16, None) == tls.TLS_ERR_INVALID_ARG
+    assert "16 bytes" in tls.tls_last_error()
+    assert lib.tls_copy_from_host(p, p, 0, None) == tls.TLS_OK
+
+
 def c2_shape(tls, **kw):
     f = dict(batch=8, n_q_heads=32, n_kv_heads=8, qk_dim=128, v_dim=128, v_offset=-1, block_size=64, n_label=16,
              ctx_len=32768, softmax_scale=128 ** -0.5)

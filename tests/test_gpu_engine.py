@@ -629,3 +629,28 @@ def test_device_planner_failures_stick():
         finally:
             for c in caches:
                 tls.tls_block_cache_destroy(c[0])
+
+
+def test_copy_from_host_moves_pinned_bytes():
+    # the per-step input path of a serving loop: pinned host bytes into device
+    # memory by one kernel (sizes from one 16-byte word to several grid
+    # strides, an interior source address); memory that is not pinned is
+    # refused before anything runs
+    runtime, tls = _rt()
+    rng = np.random.default_rng(5)
+    for n in (16, 4096 + 48, 65536, (4 << 20) + 16):
+        src = torch.from_numpy(rng.integers(0, 256, n + 32, dtype=np.uint8)).pin_memory()
+        dst = torch.zeros(n, dtype=torch.uint8, device="cuda")
+        tls.tls_copy_from_host(dst, src[16:16 + n].data_ptr(), n)
+        torch.cuda.synchronize()
+        assert torch.equal(dst.cpu(), src[16:16 + n]), f"{n} bytes"
+    # the same buffer again: the remembered check, the same result
+    tls.tls_copy_from_host(dst, src[16:16 + n].data_ptr(), n)
+    torch.cuda.synchronize()
+    assert torch.equal(dst.cpu(), src[16:16 + n])
+    plain = np.zeros(4096, dtype=np.uint8)
+    off = (-plain.ctypes.data) % 16
+    with pytest.raises(tls.TlsError) as e:
+        tls.tls_copy_from_host(dst, plain.ctypes.data + off, 1024)
+    assert e.value.status == tls.TLS_ERR_INVALID_ARG
+    torch.cuda.synchronize()

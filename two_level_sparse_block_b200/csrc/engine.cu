@@ -299,14 +299,15 @@ tls_status device_step(tls_engine* e, const void* q, int32_t out_dtype, void* ou
   if (st != TLS_OK) return st;
   ce = cudaEventRecord(e->ev_sel, e->sel);
   if (ce != cudaSuccess) return cuda_check(ce, "engine_step: select stream");
-  // the attention over the slot pool, on A, once T_{t-1} has landed: a
-  // programmatic launch, as in the resident step (the event wait still
-  // holds it back until the transfer is complete; only the dependence on
-  // level 2 is relaxed, and the attention waits for level 2's lists itself)
+  // the attention over the slot pool, on A, once T_{t-1} has landed (a
+  // plain launch: as a programmatic one, its CTAs would wait on SMs the pull
+  // of T_t needs; measured once, the transfer-bound 36-layer workload's layer
+  // ran about 10 % slower that way, for about 1 us gained on the MQA offload
+  // workload)
   ce = cudaEventRecord(e->ready[ri], A);
   if (ce == cudaSuccess) ce = cudaStreamWaitEvent(A, e->copy_end[rp], 0);  // T_{t-1} has landed
   if (ce != cudaSuccess) return cuda_check(ce, "engine_step: wait for the transfer");
-  st = sparse_attn_impl(s, q, e->kv, e->token_idx, e->k, out_dtype, out, lse, e->ws, e->L, A, /*pdl=*/true);
+  st = sparse_attn_impl(s, q, e->kv, e->token_idx, e->k, out_dtype, out, lse, e->ws, e->L, A, /*pdl=*/false);
   if (st != TLS_OK) return st;
   // T_t on the copy stream once M_t is chosen, alongside the attention of
   // step t.  The attention of step t-1 (whose slots may be evicted now) is

@@ -178,9 +178,12 @@ class ResidentEngine:
         self.engine = tls.tls_engine_create_resident(s, self.K_b, self.k, st.meta, st.label_ch, st.codes, st.scales,
                                                      st.kv, self.block_idx, self.token_idx, self.ws, self.ws_bytes)
 
-    def step(self, q=None, stream=None):
-        """One staggered step with q (default: the state's q); writes self.out / self.lse."""
-        tls.tls_engine_step(self.engine, self.st.q if q is None else q, self.out_dtype, self.out, self.lse, stream)
+    def step(self, q=None, stream=None, out=None):
+        """One staggered step with q (default: the state's q); writes self.out (or `out`: any memory the
+        device can address, e.g. pinned host memory, which the attention then writes over PCIe) and
+        self.lse."""
+        tls.tls_engine_step(self.engine, self.st.q if q is None else q, self.out_dtype,
+                            self.out if out is None else out, self.lse, stream)
 
     def steps_taken(self) -> int:
         return tls.tls_engine_steps(self.engine)

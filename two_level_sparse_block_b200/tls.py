@@ -76,6 +76,7 @@ _SZ = ctypes.c_size_t
 _SIG = {
     "tls_last_error": (ctypes.c_char_p, []),
     "tls_version": (_I32, []),
+    "tls_copy_from_host": (_I32, [_P, _P, _SZ, _P]),
     "tls_attn_kernel": (ctypes.c_char_p, [_P]),
     "tls_token_kernel": (ctypes.c_char_p, [_P, _I32, _I32, _I32, _P, _P]),
     "tls_workspace_bytes": (_SZ, [_P, _I32, _I32]),
@@ -176,6 +177,13 @@ def tls_last_error() -> str:
 
 def tls_version() -> int:
     return lib().tls_version()
+
+
+def tls_copy_from_host(dst, src, nbytes=None, stream=None):
+    """dst (device) <- src (pinned host), nbytes (default: src's size) by one kernel on `stream`."""
+    if nbytes is None:
+        nbytes = src.numel() * src.element_size() if isinstance(src, torch.Tensor) else src.nbytes
+    _check(lib().tls_copy_from_host(_ptr(dst), _ptr(src), nbytes, _stream(stream)), "tls_copy_from_host")
 
 
 def tls_token_kernel(shape: Shape, K_b: int, k: int, staggered: bool = False):
