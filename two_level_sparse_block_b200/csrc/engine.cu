@@ -17,6 +17,15 @@
 // The table update changes only entries of copied and evicted blocks, none of
 // which step t's attention reads, so C may run alongside it.
 //
+// Planned on the device (where the cache allows it) the step has no host wait:
+//   A: wait sel_{t-1}; event q_t; level 2 over M_{t-1} (half the SMs);
+//      event ready_t; wait copy_end_{t-1}; attention over the slot pool
+//   B: wait q_t; level 1 -> M_t; event sel_t
+//   C: wait sel_t (level 1 started after q_t, so the attention of step t-1
+//      is done too); event copy_start_t; plan kernel (T_t, its victims, the
+//      table; the slots the previous plan used are kept); pull kernel;
+//      event copy_end_t
+//
 // A resident engine (K/V in HBM, no cache) keeps only the stagger, with no
 // host wait: A: event q_t, level 2 over M_{t-1}; B: wait q_t, level 1 -> M_t,
 // event sel_t; A: attention, wait sel_t.  Level 1 of step t overwrites the list
