@@ -48,6 +48,7 @@ const void* mapped_source(const void* p, size_t bytes) {
       (const uint8_t*)b.devicePointer - (const uint8_t*)a.devicePointer != (ptrdiff_t)(bytes - 1))
     return nullptr;
   std::lock_guard<std::mutex> lock(mu);
+  if (seen.size() >= 4096) seen.clear();  // a loop reuses a few buffers; bound the memory all the same
   seen[key] = a.devicePointer;
   return a.devicePointer;
 }
