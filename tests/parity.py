@@ -1,13 +1,13 @@
 """Comparison helpers for the CUDA path against the oracle.
 
-Rules (each is a reading of the tolerances the workload statement gives):
+Rules (the tolerances of the comparison):
   * Index sets: bit-exact, except that an element may differ when the
     oracle's float64 score of every differing element lies within
     1e-6 * max|score| of the oracle's k-th score (a tie at the boundary within
     float32 rounding).  The number of accepted swaps is returned.
   * When the GPU's level-1 set differs inside that band, the oracle's later
     stages are re-run on the GPU's set (conditional oracle), so each stage is
-    judged on the same inputs.
+    checked on the same inputs.
   * Attention outputs: per (batch, head) row, max|out - ref| / max|ref| <= 2e-3.
 """
 
