@@ -57,6 +57,10 @@ def test_copy_from_host_checks_its_arguments_before_anything(tls):
     assert lib.tls_copy_from_host(p + 8, p, 16, None) == tls.TLS_ERR_INVALID_ARG
     assert "16 bytes" in tls.tls_last_error()
     assert lib.tls_copy_from_host(p, p, 0, None) == tls.TLS_OK
+    # memory that is not pinned (here: no device at all, or plain malloc'd
+    # memory on a GPU machine) is refused before anything is launched
+    assert lib.tls_copy_from_host(p, p, 16, None) == tls.TLS_ERR_INVALID_ARG
+    assert "pinned" in tls.tls_last_error()
 
 
 def c2_shape(tls, **kw):
