@@ -1,10 +1,10 @@
 // Per-step inputs straight from pinned host memory.  A decode step's query
-// is tens of kilobytes; a copy-engine transfer of it starts several
-// microseconds later than a kernel whose loads cross PCIe, and in a captured
-// step the hand-off between the copy engine and the SMs costs more again.
-// tls_copy_from_host moves such a buffer with one kernel: every thread one
-// 16-byte load from the host (all in flight at once: one PCIe round trip for
-// up to 16 KB per CTA) and one store to device memory.
+// is tens of kilobytes; brought in by a copy-engine transfer inside a captured
+// step, it lands about 2 us later than with a kernel whose loads cross PCIe
+// (the copy engine's start and its hand-off to the SMs).  tls_copy_from_host
+// moves such a buffer with one kernel: every thread one 16-byte load from the
+// host and one store to device memory, 4 KB per CTA, all CTAs' loads in
+// flight at once (one PCIe round trip for up to 2.4 MB).
 
 #include <cuda_runtime.h>
 
